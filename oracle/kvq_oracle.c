@@ -1,0 +1,404 @@
+/*
+ * CPU oracle for pattern-aligned residual KV quantization and decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only tests/, the package smoke check and the benchmark's CPU
+ * baseline use it.  It shares no code, header, table or constant with the CUDA
+ * library; it restates the method from the pages, plainly and slowly.
+ *
+ * Sources (page title, section / equation):
+ *   [PKV]   "PatternKV: Flattening KV Representation Expands Quantization Headroom"
+ *   [KVarN] "KVarN: Variance-Normalized KV-Cache Quantization Mitigates Error
+ *            Accumulation in Reasoning Tasks" (abstract)
+ *
+ * Precision contract: everything is float64 except the quantization step, which
+ * is written as single IEEE fp32 operations in a fixed order (pre-transform
+ * apply, residual, min-max distance, group min/max, scale and zero, the
+ * (R - z) / s division, round-half-even, clamp), so that a GPU can reproduce
+ * indices and codes bit for bit.  Build with -ffp-contract=off (no fused
+ * multiply-add) and without fast-math.
+ *
+ * Head dimension is fixed at D = 128 everywhere in this file.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define D 128
+
+/* ------------------------------------------------------------------------- */
+/* Pattern mining: Lloyd k-means under the Euclidean metric.                 */
+/* [PKV] Section 3.1 "Pattern Mining", Eq. 4: minimise the within-pattern    */
+/* sum of squared distances; centroids are the patterns.                     */
+/*                                                                           */
+/* Readings where the page is silent: deterministic strided initialisation   */
+/* M_j = x[floor(j*n/P)]; squared distances in float64 summed over channels  */
+/* 0..127 in order; ties go to the lowest index; centroid = fp32 rounding of */
+/* the float64 mean (sum in token order); an empty cluster keeps its pattern.*/
+/* ------------------------------------------------------------------------- */
+
+/* Squared Euclidean distance, float64, channels in ascending order, no FMA. */
+double kvqo_sqdist(const float* x, const float* m) {
+  double acc = 0.0;
+  for (int d = 0; d < D; ++d) {
+    double t = (double)x[d] - (double)m[d];
+    double sq = t * t;
+    acc = acc + sq;
+  }
+  return acc;
+}
+
+/* Index of the nearest pattern under kvqo_sqdist; the lowest index wins ties. */
+int32_t kvqo_nearest_euclid(const float* x, const float* M, int32_t P) {
+  int32_t best = 0;
+  double bd = kvqo_sqdist(x, M);
+  for (int32_t j = 1; j < P; ++j) {
+    double dj = kvqo_sqdist(x, M + (size_t)j * D);
+    if (dj < bd) { bd = dj; best = j; }
+  }
+  return best;
+}
+
+/*
+ * x: n rows of 128 floats.  M (out): P x 128 patterns.  assign (out, may be
+ * NULL): the assignment of the last iteration (made against the patterns
+ * that iteration started from).  Returns 0, or -1 if n < P or P < 1.
+ */
+int kvqo_mine(const float* x, int64_t n, int32_t P, int32_t iters, float* M, int32_t* assign) {
+  if (P < 1 || n < P || iters < 0) return -1;
+  for (int32_t j = 0; j < P; ++j) {
+    int64_t src = (int64_t)((j * n) / P);
+    memcpy(M + (size_t)j * D, x + (size_t)src * D, D * sizeof(float));
+  }
+  int32_t* a = (int32_t*)malloc((size_t)n * sizeof(int32_t));
+  double* sum = (double*)malloc((size_t)P * D * sizeof(double));
+  int64_t* cnt = (int64_t*)malloc((size_t)P * sizeof(int64_t));
+  if (!a || !sum || !cnt) { free(a); free(sum); free(cnt); return -2; }
+  for (int32_t it = 0; it < iters; ++it) {
+    /* assignment step */
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) a[i] = kvqo_nearest_euclid(x + (size_t)i * D, M, P);
+    /* update step: float64 sums in token order, then the mean rounded to fp32 */
+    memset(sum, 0, (size_t)P * D * sizeof(double));
+    memset(cnt, 0, (size_t)P * sizeof(int64_t));
+    for (int64_t i = 0; i < n; ++i) {
+      double* s = sum + (size_t)a[i] * D;
+      const float* xi = x + (size_t)i * D;
+      for (int d = 0; d < D; ++d) s[d] = s[d] + (double)xi[d];
+      cnt[a[i]] += 1;
+    }
+    for (int32_t j = 0; j < P; ++j) {
+      if (cnt[j] == 0) continue;
+      for (int d = 0; d < D; ++d) M[(size_t)j * D + d] = (float)(sum[(size_t)j * D + d] / (double)cnt[j]);
+    }
+  }
+  if (assign) memcpy(assign, a, (size_t)n * sizeof(int32_t));
+  free(a); free(sum); free(cnt);
+  return 0;
+}
+
+/* Within-pattern objective of Eq. 4 for given patterns and assignment (float64). */
+double kvqo_objective(const float* x, int64_t n, const float* M, const int32_t* a) {
+  double tot = 0.0;
+  for (int64_t i = 0; i < n; ++i) tot += kvqo_sqdist(x + (size_t)i * D, M + (size_t)a[i] * D);
+  return tot;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Pre-transform: Hadamard rotation + dual-axis variance normalisation.      */
+/* [KVarN] abstract: a Hadamard rotation followed by a dual-scaling variance */
+/* normalisation over both axes (tokens and channels) of K and of V.         */
+/*                                                                           */
+/* Readings: Sylvester-ordered Walsh-Hadamard transform of size 128, as the  */
+/* in-place butterfly with strides 1, 2, 4, ..., 64, each step (a+b, a-b) in */
+/* fp32; left unnormalised (a global factor cancels in the per-token         */
+/* normalisation below and is undone exactly by 1/128 on the way back).      */
+/* Column factors c are fitted once on the prefill block in float64 by 3     */
+/* alternating passes (divide every row by its population std, then every    */
+/* column by its population std; c = product of the column divisors, rounded */
+/* to fp32).  Every token then gets its own row factor r = population std of */
+/* u = x'/c over the 128 channels, computed in fp32 with halving sums; the   */
+/* quantized vector is y = u / r.  A zero std counts as 1.                   */
+/* ------------------------------------------------------------------------- */
+
+/* In-place fp32 butterfly: for h = 1, 2, ..., 64 pair i and i+h inside each block of 2h. */
+void kvqo_fwht(float* v) {
+  for (int h = 1; h < D; h *= 2)
+    for (int i0 = 0; i0 < D; i0 += 2 * h)
+      for (int i = i0; i < i0 + h; ++i) {
+        float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+}
+
+/* Same butterfly in float64. */
+void kvqo_fwht64(double* v) {
+  for (int h = 1; h < D; h *= 2)
+    for (int i0 = 0; i0 < D; i0 += 2 * h)
+      for (int i = i0; i < i0 + h; ++i) {
+        double a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+}
+
+/* fp32 sum of 128 values by halving: add the upper half onto the lower half until one is left. */
+float kvqo_halving_sum(const float* v) {
+  float w[D];
+  memcpy(w, v, sizeof(w));
+  for (int h = D / 2; h >= 1; h /= 2)
+    for (int i = 0; i < h; ++i) w[i] = w[i] + w[i + h];
+  return w[0];
+}
+
+/* Population std of the n values v[0], v[stride], ... in float64 (two passes). */
+static double std64(const double* v, int64_t n, int64_t stride) {
+  double mean = 0.0, var = 0.0;
+  for (int64_t i = 0; i < n; ++i) mean += v[i * stride];
+  mean /= (double)n;
+  for (int64_t i = 0; i < n; ++i) {
+    double t = v[i * stride] - mean;
+    var += t * t;
+  }
+  return sqrt(var / (double)n);
+}
+
+/* xp: n rows already passed through kvqo_fwht.  c (out): 128 column factors. */
+int kvqo_fit_colscale(const float* xp, int64_t n, int32_t passes, float* c) {
+  if (n < 1) return -1;
+  double* v = (double*)malloc((size_t)n * D * sizeof(double));
+  if (!v) return -2;
+  double C[D];
+  for (int d = 0; d < D; ++d) C[d] = 1.0;
+  for (int64_t i = 0; i < n * D; ++i) v[i] = (double)xp[i];
+  for (int p = 0; p < passes; ++p) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n; ++t) {
+      double r = std64(v + (size_t)t * D, D, 1);
+      if (r == 0.0) r = 1.0;
+      for (int d = 0; d < D; ++d) v[(size_t)t * D + d] /= r;
+    }
+    for (int d = 0; d < D; ++d) {
+      double s = std64(v + d, n, D);
+      if (s == 0.0) s = 1.0;
+      for (int64_t t = 0; t < n; ++t) v[(size_t)t * D + d] /= s;
+      C[d] *= s;
+    }
+  }
+  for (int d = 0; d < D; ++d) c[d] = (float)C[d];
+  free(v);
+  return 0;
+}
+
+/* One token: x (raw row) -> y (normalised, fp32) and its row factor r. */
+void kvqo_apply_row(const float* x, const float* c, float* y, float* r_out) {
+  float u[D], dev2[D];
+  memcpy(u, x, sizeof(u));
+  kvqo_fwht(u);
+  for (int d = 0; d < D; ++d) u[d] = u[d] / c[d];
+  float mean = kvqo_halving_sum(u) / 128.0f;
+  for (int d = 0; d < D; ++d) {
+    float t = u[d] - mean;
+    dev2[d] = t * t;
+  }
+  float var = kvqo_halving_sum(dev2) / 128.0f;
+  float r = sqrtf(var);
+  if (r == 0.0f) r = 1.0f;
+  for (int d = 0; d < D; ++d) y[d] = u[d] / r;
+  *r_out = r;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Pattern alignment: [PKV] Section 3.2, min-max distance and Eq. 6.         */
+/*   d_mm(x, m) = max_i (x_i - m_i) - min_j (x_j - m_j)                      */
+/*   M* = argmin over the pattern set of d_mm(X, M),  R = X - M*             */
+/* Evaluated in fp32: r_d = fl32(x_d - m_d), d = fl32(max r - min r); the    */
+/* lowest index wins ties.                                                   */
+/* ------------------------------------------------------------------------- */
+
+float kvqo_dmm(const float* x, const float* m) {
+  float mx = x[0] - m[0], mn = mx;
+  for (int d = 1; d < D; ++d) {
+    float r = x[d] - m[d];
+    if (r > mx) mx = r;
+    if (r < mn) mn = r;
+  }
+  return mx - mn;
+}
+
+int32_t kvqo_assign(const float* x, const float* M, int32_t P) {
+  int32_t best = 0;
+  float bd = kvqo_dmm(x, M);
+  for (int32_t j = 1; j < P; ++j) {
+    float dj = kvqo_dmm(x, M + (size_t)j * D);
+    if (dj < bd) { bd = dj; best = j; }
+  }
+  return best;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Asymmetric n-bit group quantizer: [PKV] Section 2.1, Eq. 1.               */
+/*   Q = round((X - z) / s),  s = (max X - min X) / (2^n - 1),  z = min X    */
+/* fp32, in this order: mn, mx exact; s = fl32(fl32(mx - mn) / (2^n - 1));   */
+/* z = mn; q = s == 0 ? 0 : clamp(rne(fl32(fl32(R - z) / s)), 0, 2^n - 1).   */
+/* ------------------------------------------------------------------------- */
+
+void kvqo_quant_group(const float* R, int64_t n, int64_t stride, int32_t bits, float* s_out, float* z_out,
+                      int32_t* q, int64_t qstride) {
+  float mn = R[0], mx = R[0];
+  for (int64_t i = 1; i < n; ++i) {
+    float v = R[i * stride];
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  const float levels = (float)((1 << bits) - 1);
+  float span = mx - mn;
+  float s = span / levels;
+  float z = mn;
+  for (int64_t i = 0; i < n; ++i) {
+    int32_t code = 0;
+    if (s != 0.0f) {
+      float t = R[i * stride] - z;
+      float u = t / s;
+      float rq = rintf(u); /* round-half-even under the default rounding mode */
+      code = (int32_t)rq;
+      if (code < 0) code = 0;
+      if (code > (1 << bits) - 1) code = (1 << bits) - 1;
+    }
+    q[i * qstride] = code;
+  }
+  *s_out = s;
+  *z_out = z;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Encoding of one (sequence, KV head) token stream of N tokens.             */
+/* Granularity ([PKV] Section 4.1, matching KIVI): K per channel, V per      */
+/* token, group 32.  V is quantized per token over 4 groups of 32 channels.  */
+/* K is quantized per channel over each complete group of 32 tokens; the    */
+/* N % 32 most recent K tokens are not quantized (they stay full precision). */
+/* Patterns are aligned after RoPE, i.e. on the inputs as given ([PKV] 4.1). */
+/*                                                                           */
+/* Outputs (natural order, one byte per code):                               */
+/*   kcode[G][32][128], ks/kz[G][128], kidx[G][32], krow[G][32]              */
+/*   vcode[N][128], vs/vz[N][4], vidx[N], vrow[N]                            */
+/* with G = N / 32.  cK/cV NULL means no pre-transform (rows are then 1).    */
+/* ------------------------------------------------------------------------- */
+
+static void prep_row(const float* x, const float* c, float* y, float* r) {
+  if (c) {
+    kvqo_apply_row(x, c, y, r);
+  } else {
+    memcpy(y, x, D * sizeof(float));
+    *r = 1.0f;
+  }
+}
+
+int kvqo_encode(const float* K, const float* V, int64_t N, int32_t bits, int32_t P, const float* MK,
+                const float* MV, const float* cK, const float* cV, uint8_t* kcode, float* ks, float* kz,
+                uint8_t* kidx, float* krow, uint8_t* vcode, float* vs, float* vz, uint8_t* vidx, float* vrow) {
+  if (bits != 2 && bits != 4) return -1;
+  if (P < 1 || P > 255) return -1;
+  /* V: every token */
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < N; ++t) {
+    float y[D], R[D];
+    prep_row(V + (size_t)t * D, cV, y, &vrow[t]);
+    int32_t j = kvqo_assign(y, MV, P);
+    vidx[t] = (uint8_t)j;
+    for (int d = 0; d < D; ++d) R[d] = y[d] - MV[(size_t)j * D + d];
+    int32_t q[D];
+    for (int g = 0; g < 4; ++g) kvqo_quant_group(R + 32 * g, 32, 1, bits, &vs[t * 4 + g], &vz[t * 4 + g], q + 32 * g, 1);
+    for (int d = 0; d < D; ++d) vcode[(size_t)t * D + d] = (uint8_t)q[d];
+  }
+  /* K: complete groups of 32 tokens */
+  int64_t G = N / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t g = 0; g < G; ++g) {
+    float R[32][D];
+    for (int t = 0; t < 32; ++t) {
+      float y[D];
+      int64_t tok = g * 32 + t;
+      prep_row(K + (size_t)tok * D, cK, y, &krow[g * 32 + t]);
+      int32_t j = kvqo_assign(y, MK, P);
+      kidx[g * 32 + t] = (uint8_t)j;
+      for (int d = 0; d < D; ++d) R[t][d] = y[d] - MK[(size_t)j * D + d];
+    }
+    int32_t q[32][D];
+    for (int d = 0; d < D; ++d) kvqo_quant_group(&R[0][d], 32, D, bits, &ks[g * D + d], &kz[g * D + d], &q[0][d], D);
+    for (int t = 0; t < 32; ++t)
+      for (int d = 0; d < D; ++d) kcode[((size_t)g * 32 + t) * D + d] = (uint8_t)q[t][d];
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dequantization / reconstruction ([PKV] Section 3.2: fetch the pattern by  */
+/* its stored index and undo the residualisation; Eq. 1: s*Q + z), float64.  */
+/* With the pre-transform the result is mapped back: x = r * (y (.) c) H / 128.*/
+/* ------------------------------------------------------------------------- */
+
+static void unrotate(double* v, const float* c, float r) {
+  for (int d = 0; d < D; ++d) v[d] = (double)r * (v[d] * (double)c[d]);
+  kvqo_fwht64(v);
+  for (int d = 0; d < D; ++d) v[d] /= 128.0;
+}
+
+/* Khat[G*32][128] from the K groups, Vhat[N][128] from the V tokens (original space). */
+void kvqo_dequant(int64_t N, const float* MK, const float* MV, const float* cK, const float* cV,
+                  const uint8_t* kcode, const float* ks, const float* kz, const uint8_t* kidx, const float* krow,
+                  const uint8_t* vcode, const float* vs, const float* vz, const uint8_t* vidx, const float* vrow,
+                  double* Khat, double* Vhat) {
+  int64_t G = N / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < G * 32; ++t) {
+    int64_t g = t / 32;
+    double* o = Khat + (size_t)t * D;
+    const float* m = MK + (size_t)kidx[t] * D;
+    for (int d = 0; d < D; ++d)
+      o[d] = (double)ks[g * D + d] * (double)kcode[(size_t)t * D + d] + (double)kz[g * D + d] + (double)m[d];
+    if (cK) unrotate(o, cK, krow[t]);
+  }
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < N; ++t) {
+    double* o = Vhat + (size_t)t * D;
+    const float* m = MV + (size_t)vidx[t] * D;
+    for (int d = 0; d < D; ++d)
+      o[d] = (double)vs[t * 4 + d / 32] * (double)vcode[(size_t)t * D + d] + (double)vz[t * 4 + d / 32] + (double)m[d];
+    if (cV) unrotate(o, cV, vrow[t]);
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Decode attention for the query heads sharing one KV head (GQA), float64:  */
+/*   o_h = softmax(scale * q_h . Khat^T) Vhat, max-subtracted softmax.       */
+/* Khat / Vhat hold N rows (quantized tokens reconstructed, the K tail exact).*/
+/* ------------------------------------------------------------------------- */
+
+void kvqo_attention(const double* q, int32_t Gq, const double* Khat, const double* Vhat, int64_t N, double scale,
+                    double* out) {
+  double* sc = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+  for (int32_t h = 0; h < Gq; ++h) {
+    const double* qh = q + (size_t)h * D;
+    double mx = -INFINITY;
+    for (int64_t t = 0; t < N; ++t) {
+      double s = 0.0;
+      for (int d = 0; d < D; ++d) s += qh[d] * Khat[(size_t)t * D + d];
+      sc[t] = scale * s;
+      if (sc[t] > mx) mx = sc[t];
+    }
+    double l = 0.0;
+    for (int64_t t = 0; t < N; ++t) {
+      sc[t] = exp(sc[t] - mx);
+      l += sc[t];
+    }
+    double* o = out + (size_t)h * D;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t t = 0; t < N; ++t)
+      for (int d = 0; d < D; ++d) o[d] += sc[t] * Vhat[(size_t)t * D + d];
+    for (int d = 0; d < D; ++d) o[d] = (N > 0) ? o[d] / l : 0.0;
+  }
+  free(sc);
+}
