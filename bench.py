@@ -1,0 +1,339 @@
+"""Benchmark of the hot path on B200: pattern mining + quantize-append + decode attention.
+
+One step = one pass of the whole path over one batch of synthetic input (Llama-3-8B-shaped
+layer by default: 8 sequences x 32768 tokens, 8 KV heads, 32 query heads, head_dim 128,
+bf16, P=64, 2-bit):
+  mine K patterns, mine V patterns      (kvq_mine_patterns x2)
+  quantize-append the whole context     (kvq_quantize_append, into a freshly reset cache)
+  one decode step of attention          (kvq_decode_attention)
+All work runs in libkvq's CUDA kernels through the C ABI.  Inputs (1 GiB of K/V) exceed the
+126 MB L2, so every step streams from HBM.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME] [--bits 2|4]
+
+Multi-GPU (torchrun): every rank runs its own batch (different seed); there is no data-path
+collective, the step time is the max over ranks, and value counts all ranks' tokens (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2-bit quantized-KV decode attn KV-tokens/s & HBM GB/s vs ~8 TB/s; quant-append GB/s"
+DEFAULT_WORKLOAD = "llama3_8b_32k"
+D = 128
+
+
+def bytes_per_token_head(bits: int, transform: int) -> int:
+    """Algorithmic cache bytes per (token, KV head): K+V codes, fp32 scale/zero, indices (+ row factors)."""
+    codes = 2 * D * bits // 8
+    return codes + 64 + 2 + (8 if transform else 0)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample of the workload.
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, sample_tokens: int = 4096):
+    import numpy as np
+
+    import oracle
+    import synth
+
+    sw = w.with_(B=1, S=sample_tokens)
+    k, v = synth.gen_kv(sw, 0, 1, 0, sample_tokens)
+    Kf, Vf = synth.to_float(k, w.dtype)[0, :, 0], synth.to_float(v, w.dtype)[0, :, 0]
+    q = synth.to_float(synth.gen_q(sw, b0=0, b1=1), w.dtype)[0, : w.Hq // w.Hkv]
+    t0 = time.perf_counter()
+    MK, cK, _ = oracle.mine_set(Kf, w.P, w.iters, w.transform)
+    MV, cV, _ = oracle.mine_set(Vf, w.P, w.iters, w.transform)
+    e = oracle.encode(Kf, Vf, w.bits, MK, MV, cK, cV)
+    oracle.attention_unit(q, Kf, e, MK, MV, cK, cV)
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    # one KV head of sample_tokens tokens; a KV-token covers all Hkv heads
+    value = sample_tokens / (dt * w.Hkv)
+    sample = (f"oracle mine(K,V) + encode + decode attention of 1 sequence x {sample_tokens} tokens x 1 KV head "
+              f"({w.Hq // w.Hkv} query heads), scaled to KV-tokens/s over {w.Hkv} KV heads; {dt:.2f} s")
+    return {"value": value, "unit": "KV-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}, dt
+
+
+def run_reference(args):
+    import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    synth.build()
+    import oracle
+    oracle.build()
+    vals, times = [], []
+    for i in range(args.warmup + args.steps):
+        cb, dt = cpu_baseline(w, sample_tokens=args.ref_tokens)
+        if i >= args.warmup:
+            vals.append(cb["value"])
+            times.append(dt)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "KV-tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args),
+            "cpu_baseline": dict(cb, value=value),
+            "e2e": {"value": value, "unit": "KV-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "batch": w.B, "context": w.S, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": D,
+            "patterns": w.P, "lloyd_iters": w.iters, "bits": w.bits, "group": 32,
+            "transform": "hadamard+varnorm" if w.transform else "none",
+            "input_dtype": "bf16" if w.dtype == 1 else "fp16", "parallelism": f"replica x{args.gpus} (batch-sharded)",
+            "l2": "inputs larger than L2 (1 GiB K/V per step, 126 MB L2)"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--ref-tokens", type=int, default=65536)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bit_kv_cache_26_b200 as kvq
+    import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    w = base.with_(seed=base.seed + 1000 * rank)  # each rank its own batch
+    k, v = synth.gen_kv(w)
+    q = synth.gen_q(w)
+    tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
+
+    def pinned(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(tdt)
+        return t.pin_memory()
+
+    kh, vh, qh = pinned(k), pinned(v), pinned(q)
+    del k, v
+    kd, vd, qd = kh.to(dev), vh.to(dev), qh.to(dev)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, w.S, w.bits, w.P, dtype=w.dtype, transform=w.transform, device=dev)
+    n = w.B * w.S
+    ws_m = kvq._alloc_aligned(kvq.kvq_mine_workspace_bytes(n, 1, w.Hkv, w.P, w.transform), dev)
+    ws_d = cache.decode_workspace(w.Hq)
+    out = torch.empty(w.B, w.Hq, D, device=dev)
+    out_h = torch.empty(w.B, w.Hq, D).pin_memory()
+    tok_stride, set_stride = w.Hkv * D, n * w.Hkv * D
+    stream = torch.cuda.current_stream()
+
+    def step(kx, vx, qx, ev=None):
+        if ev: ev[0].record()
+        kvq.kvq_mine_patterns(kx, w.dtype, n, 1, w.Hkv, tok_stride, D, set_stride, w.P, w.iters, w.transform,
+                              cache.k_patterns, cache.k_colscale, None, ws_m)
+        kvq.kvq_mine_patterns(vx, w.dtype, n, 1, w.Hkv, tok_stride, D, set_stride, w.P, w.iters, w.transform,
+                              cache.v_patterns, cache.v_colscale, None, ws_m)
+        if ev: ev[1].record()
+        cache.seq_len.zero_()
+        kvq.kvq_quantize_append(cache.c, kx, vx, w.S)
+        if ev: ev[2].record()
+        kvq.kvq_decode_attention(cache.c, qx, w.Hq, D ** -0.5, out, ws_d)
+        if ev: ev[3].record()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(kd, vd, qd)
+    torch.cuda.synchronize()
+    assert cache.read_status() == 0, "device status bits set"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        step(kd, vd, qd, evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    mine_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    # end to end through host buffers: H2D of K, V, q from pinned memory, the step, D2H of the output
+    for _ in range(2):
+        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        step(kd, vd, qd)
+        out_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        step(kd, vd, qd)
+        out_h.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    barrier()
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = t.tolist()
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens = n * world
+    value = tokens / (ms_per_step * 1e-3)
+    e2e_value = tokens / (e2e_ms / args.steps * 1e-3)
+    pk = peaks()
+    bpt = bytes_per_token_head(w.bits, w.transform)
+    token_heads = n * w.Hkv
+    dec_bytes = token_heads * bpt
+    app_bytes = token_heads * (bpt + 2 * 2 * D)
+    mine_flops = 2 * 2 * n * w.P * D * w.iters * w.Hkv  # 2 flops per MAC, K and V
+    rooflines = {
+        "decode_attention": {"bound": "hbm", "achieved": dec_bytes / (decode_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "ms": decode_ms, "algorithmic_bytes": dec_bytes},
+        "quantize_append": {"bound": "hbm", "achieved": app_bytes / (append_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                            "unit": "GB/s", "ms": append_ms, "algorithmic_bytes": app_bytes},
+        "mine_patterns": {"bound": "tensor", "achieved": mine_flops / (mine_ms * 1e-3) / 1e12,
+                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "ms": mine_ms, "algorithmic_flops": mine_flops},
+    }
+    for r in rooflines.values():
+        r["frac"] = r["achieved"] / r["peak"]
+    dominant = max(rooflines, key=lambda k: rooflines[k]["ms"])
+    dom = rooflines[dominant]
+    roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
+                "frac": dom["frac"], "traffic": None, "kernel": dominant, "peak_source": pk["source"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "KV-tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (fp32 quantization, f64 mining distances, bf16 inputs)",
+            "data": "synthetic (seeded Gaussian-mixture K/V with outlier channels and RoPE)",
+            "config": workload_config(w, args),
+            "phases_ms": {"mine_patterns_KV": mine_ms, "quantize_append": append_ms, "decode_attention": decode_ms},
+            "decode_kv_tokens_per_s": n * world / (decode_ms * 1e-3),
+            "decode_hbm_gbs": rooflines["decode_attention"]["achieved"],
+            "quant_append_gbs": rooflines["quantize_append"]["achieved"],
+            "roofline": roofline, "rooflines": rooflines,
+            "e2e": {"value": e2e_value, "unit": "KV-tokens/s",
+                    "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
+                    "d2h_bytes_per_step": int(out_h.numel() * 4)},
+            "gpu_launches": args.steps * (2 * (1 + 3 * w.iters + (13 if w.transform else 0)) + 2 + 2),
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"], _ = cpu_baseline(w, sample_tokens=131072)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

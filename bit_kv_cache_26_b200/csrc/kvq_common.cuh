@@ -1,0 +1,256 @@
+// Shared device-side definitions of libkvq: cache geometry, the page layout,
+// exact fp32 building blocks and warp utilities.
+//
+// Every bit-exact step (pre-transform, residual, min-max distance, group
+// quantization) is written with explicit round-to-nearest intrinsics so the
+// compiler cannot fuse a multiply into an add.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kD = 128;       // head_dim
+constexpr int kG = 32;        // tokens per page / K group; channels per V group
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Geometry of one cache, copied by value into every kernel.
+// ---------------------------------------------------------------------------
+struct Geom {
+  int32_t B, H, bits, P, S, maxp, npages, dtype, tx;
+  int64_t sub_bytes, page_bytes;
+  int32_t cb;          // code bytes per K or V block
+  int32_t off_ks, off_kz, off_vc, off_vs, off_vz, off_kidx, off_vidx, off_krow, off_vrow;
+  uint8_t* pool;
+  const int32_t* page_table;
+  int32_t* seq_len;
+  uint16_t* k_tail;
+  const float* kpat;
+  const float* vpat;
+  const int32_t* seq_to_set;
+  const float* kcol;
+  const float* vcol;
+  int32_t* status;
+};
+
+__host__ __device__ inline int64_t subblock_bytes_of(int bits, int tx) {
+  return 2 * (kG * kD * bits / 8) + 2112 + (tx ? 256 : 0);
+}
+
+inline Geom make_geom(const kvq_cache& c) {
+  Geom g;
+  g.B = c.num_seqs; g.H = c.num_kv_heads; g.bits = c.bits; g.P = c.num_patterns; g.S = c.num_sets;
+  g.maxp = c.max_pages_per_seq; g.npages = c.num_pages; g.dtype = c.dtype; g.tx = c.transform;
+  g.cb = kG * kD * c.bits / 8;
+  g.sub_bytes = subblock_bytes_of(c.bits, c.transform);
+  g.page_bytes = g.sub_bytes * c.num_kv_heads;
+  g.off_ks = g.cb;
+  g.off_kz = g.cb + 512;
+  g.off_vc = g.cb + 1024;
+  g.off_vs = 2 * g.cb + 1024;
+  g.off_vz = 2 * g.cb + 1536;
+  g.off_kidx = 2 * g.cb + 2048;
+  g.off_vidx = 2 * g.cb + 2080;
+  g.off_krow = 2 * g.cb + 2112;
+  g.off_vrow = 2 * g.cb + 2240;
+  g.pool = (uint8_t*)c.page_pool;
+  g.page_table = c.page_table;
+  g.seq_len = c.seq_len;
+  g.k_tail = (uint16_t*)c.k_tail;
+  g.kpat = c.k_patterns;
+  g.vpat = c.v_patterns;
+  g.seq_to_set = c.seq_to_set;
+  g.kcol = c.k_colscale;
+  g.vcol = c.v_colscale;
+  g.status = c.status;
+  return g;
+}
+
+// ---------------------------------------------------------------------------
+// Page layout (see include/kvq.h): fragment order of the code matrices and the
+// orders of the per-channel / per-token fields.
+// ---------------------------------------------------------------------------
+
+// Position of element (row, col) of a (16*MT)x(16*KS) code matrix: 32-bit word and bit offset.
+__device__ __forceinline__ void frag_pos(int bits, int KS, int row, int col, int& word, int& bit) {
+  int rr = row & 15, cc = col & 15;
+  int lane = (rr & 7) * 4 + ((cc & 7) >> 1);
+  int reg = ((row >> 4) * KS + (col >> 4)) * 4 + (rr >> 3) + 2 * (cc >> 3);
+  int odd = col & 1;
+  if (bits == 2) { word = lane * 8 + (reg >> 3); bit = 2 * (reg & 7) + 16 * odd; }
+  else           { word = lane * 16 + (reg >> 2); bit = 4 * (reg & 3) + 16 * odd; }
+}
+
+// Inverse: the element held in word `word` at slot `slot` (0..codes_per_half-1) of half `odd`.
+__device__ __forceinline__ void frag_elem(int bits, int KS, int word, int slot, int odd, int& row, int& col) {
+  int lane, reg;
+  if (bits == 2) { lane = word >> 3; reg = (word & 7) * 8 + slot; }
+  else           { lane = word >> 4; reg = (word & 15) * 4 + slot; }
+  int g = lane >> 2, tig = lane & 3;
+  int r = reg & 3, tile = reg >> 2;
+  row = 16 * (tile / KS) + 8 * (r & 1) + g;
+  col = 16 * (tile % KS) + 8 * (r >> 1) + 2 * tig + odd;
+}
+
+// KSC: field position -> channel, and channel -> position.
+__host__ __device__ __forceinline__ int ksc_channel(int i) {
+  int tig = i >> 5, ks = (i >> 2) & 7, e = i & 3;
+  return 16 * ks + 2 * tig + (e & 1) + 8 * (e >> 1);
+}
+__host__ __device__ __forceinline__ int ksc_pos(int ch) {
+  int ks = ch >> 4, c = ch & 15;
+  int hi = c >> 3, rem = c & 7;  // rem = 2*tig + (e&1)
+  int tig = rem >> 1, e = (rem & 1) + 2 * hi;
+  return tig * 32 + ks * 4 + e;
+}
+// VSC: position of (token, group).
+__host__ __device__ __forceinline__ int vsc_pos(int tok, int grp) {
+  int ks = tok >> 4, c = tok & 15;
+  int hi = c >> 3, rem = c & 7;
+  int tig = rem >> 1, e = (rem & 1) + 2 * hi;
+  return ((tig * 2 + ks) * 4 + e) * 4 + grp;
+}
+// VZC: position of (token, group).
+__host__ __device__ __forceinline__ int vzc_pos(int tok, int grp) { return ((tok & 7) * 4 + (tok >> 3)) * 4 + grp; }
+// TOK: position of a token.
+__host__ __device__ __forceinline__ int tok_pos(int tok) { return (tok & 7) * 4 + (tok >> 3); }
+
+// ---------------------------------------------------------------------------
+// Element access
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float load_elem(const uint16_t* p, int dtype) {
+  uint16_t u = __ldg(p);
+  if (dtype == KVQ_BF16) return __uint_as_float(((uint32_t)u) << 16);
+  return __half2float(__ushort_as_half(u));
+}
+
+__device__ __forceinline__ float bits_to_float(uint16_t u, int dtype) {
+  if (dtype == KVQ_BF16) return __uint_as_float(((uint32_t)u) << 16);
+  return __half2float(__ushort_as_half(u));
+}
+
+__device__ __forceinline__ void set_status(int32_t* st, int bit) {
+  if (st) atomicOr(st, bit);
+}
+
+// ---------------------------------------------------------------------------
+// Warp helpers.  A 128-vector is held by a warp as v[k] = element lane + 32*k.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fminf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// Walsh-Hadamard butterfly, strides 1, 2, ..., 64 in that order, (a+b, a-b) with a the lower
+// index; unnormalised.  Matches the reference definition operation for operation.
+__device__ __forceinline__ void fwht_warp(float v[4], int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float p = __shfl_xor_sync(kFull, v[k], h);
+      v[k] = (lane & h) ? __fsub_rn(p, v[k]) : __fadd_rn(v[k], p);
+    }
+  }
+  // stride 32: pairs (k=0,k=1), (k=2,k=3)
+  float a0 = v[0], b0 = v[1], a1 = v[2], b1 = v[3];
+  v[0] = __fadd_rn(a0, b0); v[1] = __fsub_rn(a0, b0);
+  v[2] = __fadd_rn(a1, b1); v[3] = __fsub_rn(a1, b1);
+  // stride 64: pairs (k=0,k=2), (k=1,k=3)
+  a0 = v[0]; b0 = v[2]; a1 = v[1]; b1 = v[3];
+  v[0] = __fadd_rn(a0, b0); v[2] = __fsub_rn(a0, b0);
+  v[1] = __fadd_rn(a1, b1); v[3] = __fsub_rn(a1, b1);
+}
+
+// fp32 sum of 128 values by halving (upper half added onto the lower half, stride 64 first).
+// Every lane returns the total.
+__device__ __forceinline__ float halving_sum_warp(const float v[4]) {
+  float s0 = __fadd_rn(v[0], v[2]);  // i and i+64 for i = lane
+  float s1 = __fadd_rn(v[1], v[3]);  // i = lane + 32
+  float s = __fadd_rn(s0, s1);       // stride 32
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(kFull, s, o));
+  return s;
+}
+
+// Pre-transform of one token held by a warp: x -> y = fl32(fl32(x'/c) / r), r = population std.
+__device__ __forceinline__ void transform_row_warp(float v[4], const float* c, float& r_out, int lane) {
+  fwht_warp(v, lane);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __fdiv_rn(v[k], __ldg(c + lane + 32 * k));
+  float mean = __fmul_rn(halving_sum_warp(v), 0.0078125f);  // exact: divide by 128
+  float dev[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float t = __fsub_rn(v[k], mean);
+    dev[k] = __fmul_rn(t, t);
+  }
+  float var = __fmul_rn(halving_sum_warp(dev), 0.0078125f);
+  float r = __fsqrt_rn(var);
+  if (r == 0.0f) r = 1.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __fdiv_rn(v[k], r);
+  r_out = r;
+}
+
+// Nearest pattern under the min-max distance, warp-cooperative, lowest index on ties.
+// y: this lane's 4 channels (lane + 32k).  M: P x 128 fp32 patterns (global or shared).
+__device__ __forceinline__ int assign_warp(const float y[4], const float* M, int P, int lane) {
+  float best = 0.0f;
+  int bj = 0;
+  for (int j = 0; j < P; ++j) {
+    const float* m = M + (size_t)j * kD;
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float r = __fsub_rn(y[k], m[lane + 32 * k]);
+      mx = fmaxf(mx, r);
+      mn = fminf(mn, r);
+    }
+    mx = warp_max(mx);
+    mn = warp_min(mn);
+    float d = __fsub_rn(mx, mn);
+    if (j == 0 || d < best) { best = d; bj = j; }
+  }
+  return bj;
+}
+
+// Group quantizer on the 32 lanes of a warp (one value per lane): s, z and this lane's code.
+__device__ __forceinline__ int quant_warp(float R, int bits, float& s_out, float& z_out) {
+  float mn = warp_min(R), mx = warp_max(R);
+  float levels = (float)((1 << bits) - 1);
+  float s = __fdiv_rn(__fsub_rn(mx, mn), levels);
+  int code = 0;
+  if (s != 0.0f) {
+    float u = __fdiv_rn(__fsub_rn(R, mn), s);
+    code = __float2int_rn(u);
+    code = min(max(code, 0), (1 << bits) - 1);
+  }
+  s_out = s;
+  z_out = mn;
+  return code;
+}
+
+}  // namespace kvq

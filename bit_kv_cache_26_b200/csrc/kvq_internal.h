@@ -1,0 +1,41 @@
+// Internal host-side interfaces between the C-ABI layer (kvq_api.cu) and the
+// kernel translation units.  Not installed, not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvq {
+
+struct Geom;
+
+// quantize-append (kvq_append.cu)
+cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, int n_new, cudaStream_t st);
+
+// decode attention (kvq_decode.cu)
+int decode_num_splits(const Geom& g, int num_sms);
+size_t decode_workspace(const Geom& g, int Hq, int nsplit);
+cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, float* out, void* ws, int nsplit,
+                          cudaStream_t st);
+
+// dequantize (kvq_dequant.cu)
+cudaError_t launch_dequant(const Geom& g, int seq, int start, int count, float* k_out, float* v_out,
+                           cudaStream_t st);
+
+// pattern mining (kvq_mine.cu)
+struct MineArgs {
+  const void* x;
+  int dtype;
+  int64_t n;
+  int sets, heads;
+  int64_t tok_stride, head_stride, set_stride;
+  int P, iters, transform;
+  float* patterns;
+  float* colscale;
+  int32_t* assign;
+};
+size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform);
+cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace kvq

@@ -92,6 +92,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -146,8 +152,8 @@ typedef struct kvq_cache {
 } kvq_cache;
 
 /* Bytes of one page (all KV heads) and of one KV head's sub-block.  Host only; 0 if unsupported. */
-size_t kvq_page_bytes(const kvq_cache* cache);
-size_t kvq_subblock_bytes(int32_t bits, int32_t transform);
+KVQ_API size_t kvq_page_bytes(const kvq_cache* cache);
+KVQ_API size_t kvq_subblock_bytes(int32_t bits, int32_t transform);
 
 /*
  * kvq_mine_patterns -- prefill pattern mining ([PKV] Section 3.1, Eq. 4; Section 3.4
@@ -166,9 +172,9 @@ size_t kvq_subblock_bytes(int32_t bits, int32_t transform);
  *                 iteration started from)
  * Requires n >= P.  Workspace: kvq_mine_workspace_bytes().
  */
-size_t kvq_mine_workspace_bytes(int64_t n, int32_t num_sets, int32_t num_kv_heads, int32_t P,
+KVQ_API size_t kvq_mine_workspace_bytes(int64_t n, int32_t num_sets, int32_t num_kv_heads, int32_t P,
                                 int32_t transform);
-kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t num_sets, int32_t num_kv_heads,
+KVQ_API kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t num_sets, int32_t num_kv_heads,
                              int64_t tok_stride, int64_t head_stride, int64_t set_stride, int32_t P,
                              int32_t iters, int32_t transform, float* patterns_out, float* colscale_out,
                              int32_t* assign_out, void* ws, size_t ws_bytes, kvq_stream_t stream);
@@ -184,8 +190,8 @@ kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t nu
  * unchanged and flags KVQ_DEV_OVERFLOW).  n_new = 0 is a no-op.
  * Workspace: kvq_append_workspace_bytes() (currently 0; pass NULL, 0).
  */
-size_t kvq_append_workspace_bytes(const kvq_cache* cache, int32_t n_new);
-kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
+KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache* cache, int32_t n_new);
+KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
                                void* ws, size_t ws_bytes, kvq_stream_t stream);
 
 /*
@@ -200,8 +206,8 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
  * Split-K over the token axis; partial results go to the workspace
  * (kvq_decode_workspace_bytes()).
  */
-size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads);
-kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t num_q_heads, float sm_scale,
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads);
+KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t num_q_heads, float sm_scale,
                                 float* out, void* ws, size_t ws_bytes, kvq_stream_t stream);
 
 /*
@@ -213,18 +219,18 @@ kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t n
  * 0 <= start, start + count <= the sequence's length, which the caller asserts
  * through `seq_len_host` (the host-side copy of seq_len[seq]).
  */
-kvq_status kvq_dequantize(const kvq_cache* cache, int32_t seq, int32_t seq_len_host, int32_t start, int32_t count,
+KVQ_API kvq_status kvq_dequantize(const kvq_cache* cache, int32_t seq, int32_t seq_len_host, int32_t start, int32_t count,
                           float* k_out, float* v_out, kvq_stream_t stream);
 
 /* Synchronise `stream`, copy cache->status to *bits_out (host), optionally clear it.
  * Returns KVQ_ERR_DEVICE if any bit is set, else KVQ_OK. */
-kvq_status kvq_read_status(const kvq_cache* cache, int32_t* bits_out, int32_t clear, kvq_stream_t stream);
+KVQ_API kvq_status kvq_read_status(const kvq_cache* cache, int32_t* bits_out, int32_t clear, kvq_stream_t stream);
 
 /* Message of the last failed call on this thread ("" if none). */
-const char* kvq_last_error(void);
+KVQ_API const char* kvq_last_error(void);
 
 /* Library version string. */
-const char* kvq_version(void);
+KVQ_API const char* kvq_version(void);
 
 #ifdef __cplusplus
 }

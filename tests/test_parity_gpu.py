@@ -1,0 +1,139 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle on identical
+seeded inputs.  Pattern indices, codes, scales and the K tail are compared bit for bit;
+dequantized values to max-abs 1e-3; attention outputs to 2e-3 relative per output vector."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from kvq_testlib import (D, DEQ_ATOL, attention_ok, check_pages, check_tail, encode_unit, make_cache,
+                         oracle_patterns, to_torch)
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+CASES = {
+    # the tiny reference workload, exactly: 1 x 4096 tokens, 1 KV head, fp16, P=16, 2-bit
+    "tiny_ref": (W["tiny_ref_4k"], [4096]),
+    # Llama-shaped heads at small size: GQA 4, P=64, ragged length, appended in uneven chunks
+    "gqa4_2bit_ragged": (W["llama3_8b_32k"].with_(B=2, S=1000, Hkv=2, Hq=8), [37, 1, 462, 500]),
+    "gqa4_4bit_ragged": (W["llama3_8b_32k"].with_(B=2, S=1000, Hkv=2, Hq=8, bits=4), [1000]),
+    # Qwen-shaped heads, GQA 7, with the Hadamard + dual-axis pre-transform
+    "gqa7_transform": (W["qwen25_7b_128k"].with_(B=2, S=777, Hkv=2, Hq=14, P=16, transform=1), [700, 77]),
+    # tail only (fewer than 32 tokens), one pattern
+    "tail_only_p1": (W["llama3_8b_32k"].with_(B=1, S=20, Hkv=1, Hq=1, P=1), [20]),
+    # exact multiple of the group: no tail; one-token appends across a page boundary
+    "no_tail_token_steps": (W["llama3_8b_32k"].with_(B=3, S=64, Hkv=1, Hq=2, P=8), [30, 1, 1, 32]),
+    # many sequences, per-sample perturbed centers
+    "breadth_small": (W["breadth_256x16k"].with_(B=16, S=100, Hkv=2, Hq=8, P=32), [100]),
+}
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def case(request):
+    w, chunks = CASES[request.param]
+    assert sum(chunks) == w.S
+    k, v = synth.gen_kv(w)
+    Kf, Vf = synth.to_float(k, w.dtype), synth.to_float(v, w.dtype)
+    MK, MV, cK, cV = oracle_patterns(w, Kf, Vf) if w.B * w.S >= w.P else (None,) * 4
+    cache = make_cache(w, MK, MV, cK, cV)
+    kt, vt = to_torch(k, w.dtype), to_torch(v, w.dtype)
+    s0 = 0
+    for n in chunks:
+        cache.append(kt[:, s0:s0 + n].contiguous(), vt[:, s0:s0 + n].contiguous())
+        s0 += n
+    torch.cuda.synchronize()
+    assert cache.read_status() == 0
+    return dict(name=request.param, w=w, k=k, v=v, Kf=Kf, Vf=Vf, MK=MK, MV=MV, cK=cK, cV=cV, cache=cache)
+
+
+def test_seq_len(case):
+    assert (case["cache"].seq_len.cpu().numpy() == case["w"].S).all()
+
+
+def test_pages_and_tail_bit_exact(case):
+    w = case["w"]
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            e = encode_unit(w, case["Kf"], case["Vf"], b, h, case["MK"], case["MV"], case["cK"], case["cV"])
+            check_pages(case["cache"], w, e, b, h)
+            check_tail(case["cache"], w, case["k"], b, h, w.S)
+
+
+def test_dequantize(case):
+    import bit_kv_cache_26_b200 as kvq
+    w, cache = case["w"], case["cache"]
+    for b in range(min(w.B, 3)):
+        ko = torch.empty(w.S, w.Hkv, D, device="cuda")
+        vo = torch.empty(w.S, w.Hkv, D, device="cuda")
+        kvq.kvq_dequantize(cache.c, b, w.S, 0, w.S, ko, vo)
+        ko, vo = ko.cpu().numpy(), vo.cpu().numpy()
+        for h in range(w.Hkv):
+            e = encode_unit(w, case["Kf"], case["Vf"], b, h, case["MK"], case["MV"], case["cK"], case["cV"])
+            Kh, Vh = oracle.dequant(e, case["MK"][h], case["MV"][h], None if case["cK"] is None else case["cK"][h],
+                                    None if case["cV"] is None else case["cV"][h])
+            G = (w.S // 32) * 32
+            Kfull = np.concatenate([Kh, case["Kf"][b, G:w.S, h]])
+            assert np.abs(ko[:, h] - Kfull).max() <= DEQ_ATOL
+            assert np.abs(vo[:, h] - Vh).max() <= DEQ_ATOL
+
+
+def test_decode_attention(case):
+    w, cache = case["w"], case["cache"]
+    q = synth.gen_q(w)
+    qt = to_torch(q, w.dtype)
+    out = torch.empty(w.B, w.Hq, D, device="cuda")
+    ws = cache.decode_workspace(w.Hq)
+    cache.decode(qt, out, ws)
+    got = out.cpu().numpy()
+    qf = synth.to_float(q, w.dtype)
+    Gq = w.Hq // w.Hkv
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            e = encode_unit(w, case["Kf"], case["Vf"], b, h, case["MK"], case["MV"], case["cK"], case["cV"])
+            want = oracle.attention_unit(qf[b, h * Gq:(h + 1) * Gq], case["Kf"][b, :, h], e, case["MK"][h],
+                                         case["MV"][h], None if case["cK"] is None else case["cK"][h],
+                                         None if case["cV"] is None else case["cV"][h])
+            ok, rel = attention_ok(got[b, h * Gq:(h + 1) * Gq], want)
+            assert ok.all(), f"seq {b} kv head {h}: relative errors {rel}"
+
+
+def test_mining_matches_oracle(case):
+    import bit_kv_cache_26_b200 as kvq
+    w = case["w"]
+    if w.B * w.S < w.P:
+        pytest.skip("fewer tokens than patterns")
+    x = to_torch(case["k"], w.dtype).reshape(1, w.B * w.S, w.Hkv, D).contiguous()
+    pats, col, _ = kvq.mine(x, w.P, w.iters, w.transform)
+    pats = pats.cpu().numpy()[0]
+    if w.transform:
+        col = col.cpu().numpy()[0]
+        assert np.allclose(col, case["cK"], rtol=1e-6, atol=0)
+        assert np.abs(pats - case["MK"]).max() <= 1e-3
+    else:
+        assert np.array_equal(pats, case["MK"]), f"max diff {np.abs(pats - case['MK']).max()}"
+
+
+def test_empty_sequence_decodes_to_zero():
+    import bit_kv_cache_26_b200 as kvq
+    w = W["llama3_8b_32k"].with_(B=2, S=64, Hkv=1, Hq=4, P=4)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, 64, 2, 4)
+    out = torch.full((w.B, w.Hq, D), 7.0, device="cuda")
+    q = to_torch(synth.gen_q(w), w.dtype)
+    cache.decode(q, out, cache.decode_workspace(w.Hq))
+    assert (out == 0).all()
+
+
+def test_overflow_flags_device_status():
+    import bit_kv_cache_26_b200 as kvq
+    w = W["llama3_8b_32k"].with_(B=1, S=40, Hkv=1, Hq=1, P=2)
+    cache = kvq.PagedKVCache(1, 1, 32, 2, 2)
+    k, v = synth.gen_kv(w)
+    cache.append(to_torch(k, w.dtype)[:, :30].contiguous(), to_torch(v, w.dtype)[:, :30].contiguous())
+    cache.append(to_torch(k, w.dtype)[:, 30:40].contiguous(), to_torch(v, w.dtype)[:, 30:40].contiguous())
+    torch.cuda.synchronize()
+    assert cache.read_status(clear=True) == kvq.KVQ_DEV_OVERFLOW
+    assert int(cache.seq_len[0]) == 30
+    assert cache.read_status() == 0
