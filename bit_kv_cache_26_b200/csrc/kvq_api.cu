@@ -144,7 +144,7 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
 size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads) {
   if (!cache || num_q_heads < 1 || cache->num_kv_heads < 1) return 0;
   kvq::Geom g = kvq::make_geom(*cache);
-  return kvq::decode_workspace(g, num_q_heads, kvq::decode_num_splits(g, num_sms()));
+  return kvq::decode_workspace(g, num_q_heads, kvq::decode_num_splits(g, num_q_heads, num_sms()));
 }
 
 kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t num_q_heads, float sm_scale,
@@ -162,7 +162,7 @@ kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t n
   if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
   if (!(sm_scale > 0.0f)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale must be positive");
   kvq::Geom g = kvq::make_geom(*cache);
-  int nsplit = kvq::decode_num_splits(g, num_sms());
+  int nsplit = kvq::decode_num_splits(g, num_q_heads, num_sms());
   size_t need = kvq::decode_workspace(g, num_q_heads, nsplit);
   if (ws_bytes < need || !ws) return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned(ws, 256)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");

@@ -93,11 +93,15 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, co
   const int b = blockIdx.z, h = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
 
-  __shared__ uint8_t vq[kD][kG];          // V codes, [channel][token]
-  __shared__ uint8_t kq[kG][kD];          // K codes, [token][channel]
-  __shared__ float kres[kG][kD];          // K residuals
+  // vectors of this page: the new V tokens (slots lo..hi-1), then all 32 K tokens if the group seals
+  constexpr int kLd = kD + 4;                       // padded row (floats)
+  __shared__ __align__(16) float vec[2 * kG][kLd];  // pre-transformed rows y
+  __shared__ uint8_t vq[kD][kG];                    // V codes, [channel][token]
+  __shared__ uint8_t kq[kG][kD];                    // K codes, [token][channel]
   __shared__ float vs_s[kG][4], vz_s[kG][4], vrow_s[kG], krow_s[kG];
   __shared__ uint8_t vidx_s[kG], kidx_s[kG];
+  const int lo = c.a - c.pg * kG, hi = c.e - c.pg * kG;  // new slots [lo, hi)
+  const int nv = hi - lo, nk = c.seal ? kG : 0, nvec = nv + nk;
 
   for (int i = threadIdx.x; i < kD * kG; i += blockDim.x) (&vq[0][0])[i] = 0;
   if (threadIdx.x < kG) {
@@ -105,60 +109,96 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, co
     vrow_s[threadIdx.x] = 0.f;
     vidx_s[threadIdx.x] = 0;
   }
-  __syncthreads();
 
-  // ---- V: every new token of the page
-  for (int t = c.a + warp; t < c.e; t += nwarps) {
-    const int slot = t - c.pg * kG;
-    const uint16_t* src = v_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
+  // ---- load (and pre-transform) every vector: warp per vector
+  for (int v = warp; v < nvec; v += nwarps) {
+    const uint16_t* src;
+    const float* col;
+    if (v < nv) {
+      const int t = c.a + v;
+      src = v_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
+      col = c.cV;
+    } else {
+      const int slot = v - nv, t = c.pg * kG + slot;
+      src = (t < c.L) ? g.k_tail + (((size_t)b * g.H + h) * kG + slot) * kD
+                      : k_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
+      col = c.cK;
+    }
     float y[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) y[k] = load_elem(src + lane + 32 * k, g.dtype);
     float r = 1.0f;
-    if (g.tx) transform_row_warp(y, c.cV, r, lane);
-    int j = assign_warp(y, c.MV, g.P, lane);
+    if (g.tx) transform_row_warp(y, col, r, lane);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float R = __fsub_rn(y[k], c.MV[(size_t)j * kD + lane + 32 * k]);
-      float s, z;
-      int code = quant_warp(R, g.bits, s, z);
-      vq[lane + 32 * k][slot] = (uint8_t)code;
-      if (lane == 0) { vs_s[slot][k] = s; vz_s[slot][k] = z; }
-    }
-    if (lane == 0) { vidx_s[slot] = (uint8_t)j; vrow_s[slot] = r; }
-  }
-
-  // ---- K: seal the group when its last token arrives
-  if (c.seal) {
-    for (int slot = warp; slot < kG; slot += nwarps) {
-      const int t = c.pg * kG + slot;
-      const uint16_t* src = (t < c.L) ? g.k_tail + (((size_t)b * g.H + h) * kG + slot) * kD
-                                      : k_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
-      float y[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) y[k] = load_elem(src + lane + 32 * k, g.dtype);
-      float r = 1.0f;
-      if (g.tx) transform_row_warp(y, c.cK, r, lane);
-      int j = assign_warp(y, c.MK, g.P, lane);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) kres[slot][lane + 32 * k] = __fsub_rn(y[k], c.MK[(size_t)j * kD + lane + 32 * k]);
-      if (lane == 0) { kidx_s[slot] = (uint8_t)j; krow_s[slot] = r; }
+    for (int k = 0; k < 4; ++k) vec[v][lane + 32 * k] = y[k];
+    if (lane == 0) {
+      if (v < nv) vrow_s[lo + v] = r;
+      else krow_s[v - nv] = r;
     }
   }
   __syncthreads();
 
+  // ---- nearest pattern: two threads per vector, each over half of the patterns
+  {
+    const int v = threadIdx.x >> 1, half = threadIdx.x & 1;
+    float best = INFINITY;
+    int bj = 0x7fffffff;
+    if (v < nvec) {
+      float y[kD];
+#pragma unroll
+      for (int d4 = 0; d4 < kD / 4; ++d4) {
+        const float4 t = *reinterpret_cast<const float4*>(&vec[v][4 * d4]);
+        y[4 * d4] = t.x; y[4 * d4 + 1] = t.y; y[4 * d4 + 2] = t.z; y[4 * d4 + 3] = t.w;
+      }
+      const float* M = (v < nv) ? c.MV : c.MK;
+      for (int j = half; j < g.P; j += 2) {
+        const float d = dmm_reg(y, M + (size_t)j * kD);
+        if (d < best) { best = d; bj = j; }
+      }
+    }
+    const float ob = __shfl_xor_sync(kFull, best, 1);
+    const int oj = __shfl_xor_sync(kFull, bj, 1);
+    if (ob < best || (ob == best && oj < bj)) { best = ob; bj = oj; }
+    if (v < nvec && half == 0) {
+      if (v < nv) vidx_s[lo + v] = (uint8_t)bj;
+      else kidx_s[v - nv] = (uint8_t)bj;
+    }
+  }
+  __syncthreads();
+
+  // ---- V: residual and per-token group quantization, warp per token
+  for (int v = warp; v < nv; v += nwarps) {
+    const int slot = lo + v;
+    const int j = vidx_s[slot];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float R = __fsub_rn(vec[v][lane + 32 * k], c.MV[(size_t)j * kD + lane + 32 * k]);
+      float s, z;
+      const int code = quant_warp(R, g.bits, s, z);
+      vq[lane + 32 * k][slot] = (uint8_t)code;
+      if (lane == 0) { vs_s[slot][k] = s; vz_s[slot][k] = z; }
+    }
+  }
+
+  // ---- K: per-channel quantization over the 32 tokens of the sealed group
   float* ks_g = reinterpret_cast<float*>(c.sub + g.off_ks);
   float* kz_g = reinterpret_cast<float*>(c.sub + g.off_kz);
   if (c.seal) {
-    // per channel over the 32 tokens
     for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-      float mn = kres[0][d], mx = mn;
-      for (int t = 1; t < kG; ++t) { mn = fminf(mn, kres[t][d]); mx = fmaxf(mx, kres[t][d]); }
-      float s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << g.bits) - 1));
+      float R[kG];
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < kG; ++t) {
+        R[t] = __fsub_rn(vec[nv + t][d], c.MK[(size_t)kidx_s[t] * kD + d]);
+        mn = fminf(mn, R[t]);
+        mx = fmaxf(mx, R[t]);
+      }
+      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << g.bits) - 1));
+#pragma unroll
       for (int t = 0; t < kG; ++t) {
         int code = 0;
         if (s != 0.0f) {
-          code = __float2int_rn(__fdiv_rn(__fsub_rn(kres[t][d], mn), s));
+          code = __float2int_rn(__fdiv_rn(__fsub_rn(R[t], mn), s));
           code = min(max(code, 0), (1 << g.bits) - 1);
         }
         kq[t][d] = (uint8_t)code;
@@ -170,7 +210,6 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, co
   __syncthreads();
 
   // ---- stores
-  const int lo = c.a - c.pg * kG, hi = c.e - c.pg * kG;  // new slots [lo, hi)
   write_code_block(reinterpret_cast<uint32_t*>(c.sub + g.off_vc), &vq[0][0], kG, g.bits, 2, !c.fresh,
                    [&](int row, int col) { return col < lo; });
   float* vs_g = reinterpret_cast<float*>(c.sub + g.off_vs);
@@ -178,7 +217,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, co
   uint8_t* vidx_g = c.sub + g.off_vidx;
   float* vrow_g = reinterpret_cast<float*>(c.sub + g.off_vrow);
   for (int i = threadIdx.x; i < kG * 4; i += blockDim.x) {
-    int slot = i >> 2, q = i & 3;
+    const int slot = i >> 2, q = i & 3;
     if (c.fresh || (slot >= lo && slot < hi)) {
       vs_g[vsc_pos(slot, q)] = vs_s[slot][q];
       vz_g[vzc_pos(slot, q)] = vz_s[slot][q];

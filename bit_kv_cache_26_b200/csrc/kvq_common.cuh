@@ -77,48 +77,43 @@ inline Geom make_geom(const kvq_cache& c) {
 // orders of the per-channel / per-token fields.
 // ---------------------------------------------------------------------------
 
-// Position of element (row, col) of a (16*MT)x(16*KS) code matrix: 32-bit word and bit offset.
-__device__ __forceinline__ void frag_pos(int bits, int KS, int row, int col, int& word, int& bit) {
-  int rr = row & 15, cc = col & 15;
-  int lane = (rr & 7) * 4 + ((cc & 7) >> 1);
-  int reg = ((row >> 4) * KS + (col >> 4)) * 4 + (rr >> 3) + 2 * (cc >> 3);
-  int odd = col & 1;
-  if (bits == 2) { word = lane * 8 + (reg >> 3); bit = 2 * (reg & 7) + 16 * odd; }
-  else           { word = lane * 16 + (reg >> 2); bit = 4 * (reg & 3) + 16 * odd; }
+// Position of element (row, col) of a (16*MT)x(16*KS) code matrix: 32-bit word of the block and bit.
+// The lane's word w sits at block word (w/4)*128 + lane*4 + w%4 (lane-interleaved 16-byte chunks).
+__host__ __device__ __forceinline__ void frag_pos(int bits, int KS, int row, int col, int& word, int& bit) {
+  const int rr = row & 15, cc = col & 15;
+  const int lane = (rr & 7) * 4 + ((cc & 7) >> 1);
+  const int reg = ((row >> 4) * KS + (col >> 4)) * 4 + (rr >> 3) + 2 * (cc >> 3);
+  const int odd = col & 1;
+  int w;
+  if (bits == 2) { w = reg >> 3; bit = 2 * (reg & 7) + 16 * odd; }
+  else           { w = reg >> 2; bit = 4 * (reg & 3) + 16 * odd; }
+  word = (w >> 2) * 128 + lane * 4 + (w & 3);
 }
 
-// Inverse: the element held in word `word` at slot `slot` (0..codes_per_half-1) of half `odd`.
-__device__ __forceinline__ void frag_elem(int bits, int KS, int word, int slot, int odd, int& row, int& col) {
-  int lane, reg;
-  if (bits == 2) { lane = word >> 3; reg = (word & 7) * 8 + slot; }
-  else           { lane = word >> 4; reg = (word & 15) * 4 + slot; }
-  int g = lane >> 2, tig = lane & 3;
-  int r = reg & 3, tile = reg >> 2;
+// Inverse: the element held by block word `word` at slot `slot` of half `odd`.
+__host__ __device__ __forceinline__ void frag_elem(int bits, int KS, int word, int slot, int odd, int& row, int& col) {
+  const int lane = (word & 127) >> 2;
+  const int w = (word >> 7) * 4 + (word & 3);
+  const int reg = bits == 2 ? w * 8 + slot : w * 4 + slot;
+  const int g = lane >> 2, tig = lane & 3;
+  const int r = reg & 3, tile = reg >> 2;
   row = 16 * (tile / KS) + 8 * (r & 1) + g;
   col = 16 * (tile % KS) + 8 * (r >> 1) + 2 * tig + odd;
 }
 
-// KSC: field position -> channel, and channel -> position.
-__host__ __device__ __forceinline__ int ksc_channel(int i) {
-  int tig = i >> 5, ks = (i >> 2) & 7, e = i & 3;
-  return 16 * ks + 2 * tig + (e & 1) + 8 * (e >> 1);
-}
+// Field orders (include/kvq.h): position of a channel (KSC), of (token, group) (VSC, VZC),
+// of a token (TOK).  A channel / token inside its 16-block is 2*tig + (e&1) + 8*(e>>1).
 __host__ __device__ __forceinline__ int ksc_pos(int ch) {
-  int ks = ch >> 4, c = ch & 15;
-  int hi = c >> 3, rem = c & 7;  // rem = 2*tig + (e&1)
-  int tig = rem >> 1, e = (rem & 1) + 2 * hi;
-  return tig * 32 + ks * 4 + e;
+  const int ks = ch >> 4, c = ch & 15;
+  const int tig = (c & 7) >> 1, e = (c & 1) + 2 * (c >> 3);
+  return ks * 16 + tig * 4 + e;
 }
-// VSC: position of (token, group).
 __host__ __device__ __forceinline__ int vsc_pos(int tok, int grp) {
-  int ks = tok >> 4, c = tok & 15;
-  int hi = c >> 3, rem = c & 7;
-  int tig = rem >> 1, e = (rem & 1) + 2 * hi;
-  return ((tig * 2 + ks) * 4 + e) * 4 + grp;
+  const int ks = tok >> 4, c = tok & 15;
+  const int tig = (c & 7) >> 1, e = (c & 1) + 2 * (c >> 3);
+  return ((ks * 4 + e) * 4 + tig) * 4 + grp;
 }
-// VZC: position of (token, group).
-__host__ __device__ __forceinline__ int vzc_pos(int tok, int grp) { return ((tok & 7) * 4 + (tok >> 3)) * 4 + grp; }
-// TOK: position of a token.
+__host__ __device__ __forceinline__ int vzc_pos(int tok, int grp) { return ((tok >> 3) * 8 + (tok & 7)) * 4 + grp; }
 __host__ __device__ __forceinline__ int tok_pos(int tok) { return (tok & 7) * 4 + (tok >> 3); }
 
 // ---------------------------------------------------------------------------
@@ -235,6 +230,43 @@ __device__ __forceinline__ int assign_warp(const float y[4], const float* M, int
     if (j == 0 || d < best) { best = d; bj = j; }
   }
   return bj;
+}
+
+// fp32 range of x - m over 128 channels, exact (no rounding beyond the per-element
+// subtraction): packed f32x2 subtractions and three-input max / min.
+__device__ __forceinline__ void sub2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  unsigned long long a, b, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// d_mm(y, m) for a vector held in registers (natural channel order) and a pattern in memory.
+__device__ __forceinline__ float dmm_reg(const float (&y)[kD], const float* __restrict__ m) {
+  const float4* m4 = reinterpret_cast<const float4*>(m);
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int c = 0; c < kD / 4; ++c) {
+    const float4 v = __ldg(m4 + c);
+    float r0, r1, r2, r3;
+    sub2(y[4 * c], y[4 * c + 1], v.x, v.y, r0, r1);
+    sub2(y[4 * c + 2], y[4 * c + 3], v.z, v.w, r2, r3);
+    mx = max3(mx, r0, r1);
+    mn = min3(mn, r0, r1);
+    mx = max3(mx, r2, r3);
+    mn = min3(mn, r2, r3);
+  }
+  return __fsub_rn(mx, mn);
 }
 
 // Group quantizer on the 32 lanes of a warp (one value per lane): s, z and this lane's code.

@@ -1,0 +1,707 @@
+// Split-K decode attention over the quantized paged cache on tensor cores
+// ("PatternKV", Section 3.4: pattern-index restoration, dequantization and the
+// QK^T / P.V products fused into the attention kernel).
+//
+// Design (per CTA: one (sequence, KV head, split); 4 warps, each streaming its own
+// pages through a ring of shared-memory stages filled by cp.async.bulk):
+//
+//   K side, per 32-token page with per-channel scale s_d, zero z_d:
+//     q.k_t = sum_d (q_d s_d) code_td + sum_d q_d z_d + T[idx_t],  T_j = q . M_K[j]
+//   The codes are turned into exact bf16 integers and used as the A operand of
+//   m16n8k16 MMAs (rows = tokens); B = q (.) s split into bf16 hi + lo parts by
+//   truncation (columns = query head x {hi, lo}), so each product keeps 16 bits
+//   (relative error below 2^-15) with no conversion instructions at all.
+//
+//   V side, per token with per-group scale s_tg and zero z_tg:
+//     sum_t p_t v_t = sum_t (p_t s_tg) code_td + sum_t p_t z_tg + sum_j W_j M_V[j]
+//   A = codes (rows = channels), B = p (.) s split into bf16 hi + lo parts (columns =
+//   query head x {hi, lo}; a single 8- or 11-bit part loses too much once the
+//   cancellation between residual and zero-point terms amplifies it),
+//   W_j = sum of p over tokens with V pattern j (shared-memory atomics), the z term
+//   in registers.
+//
+// The page layout (include/kvq.h) stores every lane's MMA operands contiguously.
+// Online softmax runs in base 2 in the MMA accumulator layout; the newest
+// incomplete group (exact keys in the K tail) is folded in on CUDA cores by the
+// last split.  Partials (m, l, o, W) go to the combine kernel.
+#include <cstdlib>
+
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kStages = 3;
+constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr float kRangeLimit = 30000.0f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// Bounded wait on an mbarrier phase: false if the phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
+  const uint32_t addr = smem_u32(bar);
+  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(phase)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Packed fp32 pairs (sm_100a f32x2 instructions).
+__device__ __forceinline__ unsigned long long pk(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// bf16 pair (lo half = first value) of the hi parts (fp32 truncated to bf16) or, on lanes with
+// lo_sel = 1, of the truncated remainders v - hi.  hi + lo keeps 16 significant bits.
+__device__ __forceinline__ uint32_t split_bf16(unsigned long long v, unsigned long long neg_sel) {
+  float v0, v1;
+  upk(v, v0, v1);
+  const float t0 = __uint_as_float(__float_as_uint(v0) & 0xFFFF0000u);
+  const float t1 = __uint_as_float(__float_as_uint(v1) & 0xFFFF0000u);
+  float r0, r1;
+  upk(fma2(neg_sel, pk(t0, t1), v), r0, r1);  // v - sel * trunc(v), exact
+  return __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+}
+
+// Two codes at bit `S` of each 16-bit half of `src` -> bf16 pair of the exact integers:
+// (src & mask) | 0x4300 puts 128 + code * 2^S in each half; one bf16 FMA removes the
+// bias and the 2^S factor exactly.  Needs code * 2^S < 128.
+template <int BITS, int S>
+__device__ __forceinline__ uint32_t code_pair(uint32_t src) {
+  static_assert((((1 << BITS) - 1) << S) < 128, "code does not fit the bf16 mantissa");
+  constexpr uint32_t mask = ((1u << BITS) - 1u) * 0x00010001u << S;
+  uint32_t v;
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(v) : "r"(src), "r"(mask), "r"(0x43004300u));  // (a & b) | c
+  constexpr uint32_t kScale = S == 0 ? 0x3F803F80u : (S == 2 ? 0x3E803E80u : 0x3D803D80u);
+  constexpr uint32_t kBias = S == 0 ? 0xC300C300u : (S == 2 ? 0xC200C200u : 0xC100C100u);
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(kScale), "r"(kBias));
+  return r;
+}
+
+// A operand registers {a0a1, a2a3, a4a5, a6a7} for the 4 consecutive code slots starting at
+// SLOT0 of lane word w (slot k holds bits [BITS*k, BITS*k + BITS) of each half).
+template <int BITS, int SLOT0>
+__device__ __forceinline__ void frag_a(uint32_t w, uint32_t (&a)[4]) {
+  if constexpr (BITS == 2) {
+    const uint32_t w6 = w >> 6, w12 = w >> 12;
+    if constexpr (SLOT0 == 0) {
+      a[0] = code_pair<2, 0>(w); a[1] = code_pair<2, 2>(w); a[2] = code_pair<2, 4>(w); a[3] = code_pair<2, 0>(w6);
+    } else {
+      a[0] = code_pair<2, 2>(w6); a[1] = code_pair<2, 4>(w6); a[2] = code_pair<2, 0>(w12); a[3] = code_pair<2, 2>(w12);
+    }
+  } else {
+    a[0] = code_pair<4, 0>(w); a[1] = code_pair<4, 0>(w >> 4); a[2] = code_pair<4, 0>(w >> 8);
+    a[3] = code_pair<4, 0>(w >> 12);
+  }
+}
+
+template <int BITS>
+struct Cfg {
+  static constexpr int kWordsPerLane = BITS * 4;  // 32-bit code words per lane per K/V block
+};
+
+// Shared memory carve-up (bytes) for one CTA.
+struct Smem {
+  int ring, bars, qk, qraw, T, W, pex;
+  int total;
+};
+constexpr int kPexLd = 36;  // padded row of the p exchange (floats): conflict-free 16-byte reads
+
+__host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int P) {
+  Smem s;
+  int o = 0;
+  s.ring = o; o += kWarps * stages * sub_bytes;
+  o = (o + 15) & ~15;
+  s.bars = o; o += kWarps * stages * 8;
+  s.qk = o; o += NT * 4 * kD * 4;          // query in the quantized space, per padded head, KSC order
+  s.qraw = o; o += NT * 4 * kD * 4;        // raw query (exact tail keys), natural order
+  s.T = o; o += NT * 4 * P * 4;            // T[h][j] = q . M_K[j]
+  s.W = o; o += kWarps * NT * 4 * P * 4;   // per-warp pattern weights
+  s.pex = o; o += kWarps * NT * 4 * kPexLd * 4;  // per-warp p exchange
+  s.total = o;
+  return s;
+}
+
+template <int BITS, int NT, int STAGES>
+__global__ void __launch_bounds__(kWarps * 32, (STAGES <= 2 ? 4 : 3))
+    decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
+                      float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w) {
+  constexpr int NH = NT * 4;  // padded heads
+  constexpr int WPL = Cfg<BITS>::kWordsPerLane;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int split = blockIdx.x, h_kv = blockIdx.y, b = blockIdx.z;
+  const int Gq = Hq / g.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gq = lane >> 2, tig = lane & 3;
+  const float lo_sel = (gq & 1) ? 1.0f : 0.0f;
+  const unsigned long long nsel = pk(-lo_sel, -lo_sel);
+  const int P = g.P;
+  const uint32_t sub_bytes = (uint32_t)g.sub_bytes;
+  const Smem sp = smem_plan((int)sub_bytes, STAGES, NT, P);
+
+  uint8_t* ring = smem + sp.ring + warp * STAGES * sub_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * STAGES;
+  float* qk = reinterpret_cast<float*>(smem + sp.qk);     // [NH][128] KSC order
+  float* qraw = reinterpret_cast<float*>(smem + sp.qraw); // [NH][128]
+  float* T = reinterpret_cast<float*>(smem + sp.T);       // [NH][P]
+  float* Wall = reinterpret_cast<float*>(smem + sp.W);
+  float* Ww = Wall + warp * NH * P;                       // this warp's [NH][P]
+  float* pex = reinterpret_cast<float*>(smem + sp.pex) + warp * NH * kPexLd;
+
+  int L = g.seq_len[b];
+  if (L < 0 || L > g.maxp * kG) {
+    if (threadIdx.x == 0 && split == 0) set_status(g.status, KVQ_DEV_OVERFLOW);
+    L = 0;
+  }
+  int set = g.seq_to_set ? g.seq_to_set[b] : 0;
+  if (set < 0 || set >= g.S) {
+    if (threadIdx.x == 0 && split == 0) set_status(g.status, KVQ_DEV_BAD_SET);
+    set = 0;
+    L = 0;
+  }
+  const int nfull = L / kG, ntail = L % kG;
+  const int per = (nfull + nsplit - 1) / nsplit;
+  const int p0 = min(nfull, split * per), p1 = min(nfull, p0 + per);
+  const size_t sh = (size_t)set * g.H + h_kv;
+  const float* MK = g.kpat + sh * P * kD;
+  const float* cK = g.tx ? g.kcol + sh * kD : nullptr;
+
+  // ---- setup: queries, T table, zeroed W, barriers
+  for (int hh = warp; hh < NH; hh += kWarps) {
+    float v[4];
+    const bool real = hh < Gq;
+    const uint16_t* src = q + ((size_t)b * Hq + h_kv * Gq + min(hh, Gq - 1)) * kD;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[k] = real ? load_elem(src + lane + 32 * k, g.dtype) : 0.f;
+      qraw[hh * kD + lane + 32 * k] = v[k];
+    }
+    if (g.tx) {
+      fwht_warp(v, lane);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = v[k] * __ldg(cK + lane + 32 * k) * 0.0078125f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qk[hh * kD + ksc_pos(lane + 32 * k)] = v[k];
+  }
+  for (int i = threadIdx.x; i < kWarps * NH * P; i += blockDim.x) Wall[i] = 0.f;
+  if (lane < STAGES) mbar_init(&bars[lane], 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncthreads();
+  for (int i = threadIdx.x; i < NH * P; i += blockDim.x) {
+    const int hh = i / P, j = i % P;
+    float t = 0.f;
+    if (hh < Gq) {
+      const float* m = MK + (size_t)j * kD;
+      for (int d = 0; d < kD; ++d) t = fmaf(qk[hh * kD + ksc_pos(d)], __ldg(m + d), t);
+    }
+    T[i] = t;
+  }
+  __syncthreads();
+
+  // query of this lane's B column (head 4j + gq/2), its 32 channels, as fp32 pairs
+  unsigned long long qreg[NT == 1 ? 8 : 1][4];
+  if constexpr (NT == 1) {
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const float4 q4 = reinterpret_cast<const float4*>(qk + (gq >> 1) * kD)[ks * 4 + tig];
+      qreg[ks][0] = pk(q4.x, q4.y);
+      qreg[ks][1] = pk(q4.z, q4.w);
+    }
+  }
+
+  // ---- per-thread state (head of n-tile j: 4j + tig)
+  float accv[NT][8][4];
+  float zacc[NT][4];
+  float mrun[NT], lrun[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    mrun[j] = -INFINITY;
+    lrun[j] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) zacc[j][u] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) accv[j][mt][u] = 0.f;
+  }
+
+  // pages of this warp: p0 + warp + kWarps*i
+  const int my_n = (p1 - p0 - warp + kWarps - 1) / kWarps;
+  auto page_src = [&](int i, bool& ok) -> const uint8_t* {
+    const int pg = p0 + warp + kWarps * i;
+    const int phys = g.page_table[(size_t)b * g.maxp + pg];
+    ok = phys >= 0 && phys < g.npages;
+    return g.pool + (size_t)(ok ? phys : 0) * g.page_bytes + (size_t)h_kv * g.sub_bytes;
+  };
+  uint32_t bad_mask = 0;  // lane 0: stages whose page id was invalid
+  if (lane == 0) {
+    for (int i = 0; i < min(STAGES, my_n); ++i) {
+      bool ok;
+      const uint8_t* src = page_src(i, ok);
+      if (ok) {
+        mbar_expect_tx(&bars[i], sub_bytes);
+        bulk_g2s(ring + i * sub_bytes, src, sub_bytes, &bars[i]);
+      } else {
+        set_status(g.status, KVQ_DEV_BAD_PAGE);
+        bad_mask |= 1u << i;
+        mbar_arrive(&bars[i]);
+      }
+    }
+  }
+  __syncwarp();
+
+  int stuck_at = -1;
+  for (int i = 0; i < my_n; ++i) {
+    const int st = i % STAGES;
+    const uint32_t phase = (i / STAGES) & 1;
+    const bool ok = mbar_wait(&bars[st], phase);
+    if (!__all_sync(kFull, ok)) { stuck_at = i; break; }
+    const bool skip = __shfl_sync(kFull, (bad_mask >> st) & 1, 0);
+    const uint8_t* pgp = ring + st * sub_bytes;
+    if (!skip) {
+      // ---------------- K side: scores of 32 tokens for the query heads
+      uint32_t kw[WPL];
+#pragma unroll
+      for (int c = 0; c < WPL / 4; ++c) {
+        const uint4 t = reinterpret_cast<const uint4*>(pgp + c * 512)[lane];
+        kw[4 * c] = t.x; kw[4 * c + 1] = t.y; kw[4 * c + 2] = t.z; kw[4 * c + 3] = t.w;
+      }
+      const float4* ks4 = reinterpret_cast<const float4*>(pgp + g.off_ks) + tig;
+      const float4* kz4 = reinterpret_cast<const float4*>(pgp + g.off_kz) + tig;
+      float sc[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        float accs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        unsigned long long zk2 = 0ull;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const float4 s4 = ks4[ks * 4];
+          const float4 z4 = kz4[ks * 4];
+          unsigned long long qa, qb;
+          if constexpr (NT == 1) {
+            qa = qreg[ks][0]; qb = qreg[ks][1];
+          } else {
+            const float4 q4 = reinterpret_cast<const float4*>(qk + (4 * j + (gq >> 1)) * kD)[ks * 4 + tig];
+            qa = pk(q4.x, q4.y); qb = pk(q4.z, q4.w);
+          }
+          zk2 = fma2(qa, pk(z4.x, z4.y), zk2);
+          zk2 = fma2(qb, pk(z4.z, z4.w), zk2);
+          const uint32_t b0 = split_bf16(mul2(qa, pk(s4.x, s4.y)), nsel);
+          const uint32_t b1 = split_bf16(mul2(qb, pk(s4.z, s4.w)), nsel);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            uint32_t a[4];
+            if constexpr (BITS == 2) {
+              const uint32_t w = kw[mt * 4 + ks / 2];
+              if (ks & 1) frag_a<2, 4>(w, a); else frag_a<2, 0>(w, a);
+            } else {
+              frag_a<4, 0>(kw[mt * 8 + ks], a);
+            }
+            mma16816(accs[mt], a, b0, b1);
+          }
+        }
+        // K zero term of head 4j + gq/2: reduce over the 4 tig lanes, then fetch for head 4j + tig
+        float za, zb;
+        upk(zk2, za, zb);
+        float zk = za + zb;
+        zk += __shfl_xor_sync(kFull, zk, 1);
+        zk += __shfl_xor_sync(kFull, zk, 2);
+        zk = __shfl_sync(kFull, zk, 8 * tig);
+        sc[j][0] = accs[0][0] + accs[0][1] + zk;
+        sc[j][1] = accs[0][2] + accs[0][3] + zk;
+        sc[j][2] = accs[1][0] + accs[1][1] + zk;
+        sc[j][3] = accs[1][2] + accs[1][3] + zk;
+      }
+      const uint32_t kidx4 = *reinterpret_cast<const uint32_t*>(pgp + g.off_kidx + gq * 4);
+      const uint32_t vidx4 = *reinterpret_cast<const uint32_t*>(pgp + g.off_vidx + gq * 4);
+      float krow[4] = {1.f, 1.f, 1.f, 1.f}, vrow[4] = {1.f, 1.f, 1.f, 1.f};
+      if (g.tx) {
+        const float4 kr = *reinterpret_cast<const float4*>(pgp + g.off_krow + gq * 16);
+        const float4 vr = *reinterpret_cast<const float4*>(pgp + g.off_vrow + gq * 16);
+        krow[0] = kr.x; krow[1] = kr.y; krow[2] = kr.z; krow[3] = kr.w;
+        vrow[0] = vr.x; vrow[1] = vr.y; vrow[2] = vr.z; vrow[3] = vr.w;
+      }
+      const float4* vz4 = reinterpret_cast<const float4*>(pgp + g.off_vz) + gq;
+      const float4 vz[4] = {vz4[0], vz4[8], vz4[16], vz4[24]};
+
+      // ---------------- online softmax (base 2), per head 4j + tig over the 32 tokens
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int hh = 4 * j + tig;
+        const bool real = hh < Gq;
+        float pm = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = min((int)((kidx4 >> (8 * u)) & 0xff), P - 1);
+          sc[j][u] = (sc[j][u] + T[hh * P + idx]) * krow[u] * scale_log2;
+          pm = fmaxf(pm, sc[j][u]);
+        }
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 4));
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 8));
+        pm = fmaxf(pm, __shfl_xor_sync(kFull, pm, 16));
+        const float mnew = fmaxf(mrun[j], pm);
+        const float alpha = ex2(mrun[j] - mnew);
+        if (__any_sync(kFull, alpha != 1.0f)) {
+          lrun[j] *= alpha;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) zacc[j][u] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
+          for (int jj = gq; jj < P; jj += 8) Ww[hh * P + jj] *= alpha;
+          __syncwarp();
+        }
+        mrun[j] = mnew;
+        float pv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = real ? ex2(sc[j][u] - mnew) : 0.f;
+          lrun[j] += p;
+          pv[u] = p * vrow[u];
+          if (real) atomicAdd(&Ww[hh * P + min((int)((vidx4 >> (8 * u)) & 0xff), P - 1)], pv[u]);
+          zacc[j][0] = fmaf(pv[u], vz[u].x, zacc[j][0]);
+          zacc[j][1] = fmaf(pv[u], vz[u].y, zacc[j][1]);
+          zacc[j][2] = fmaf(pv[u], vz[u].z, zacc[j][2]);
+          zacc[j][3] = fmaf(pv[u], vz[u].w, zacc[j][3]);
+        }
+        *reinterpret_cast<float4*>(pex + hh * kPexLd + gq * 4) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      }
+      __syncwarp();
+
+      // ---------------- V side: p-weighted residual codes for the query heads
+      uint32_t vw[WPL];
+#pragma unroll
+      for (int c = 0; c < WPL / 4; ++c) {
+        const uint4 t = reinterpret_cast<const uint4*>(pgp + g.off_vc + c * 512)[lane];
+        vw[4 * c] = t.x; vw[4 * c + 1] = t.y; vw[4 * c + 2] = t.z; vw[4 * c + 3] = t.w;
+      }
+      const float4* vs4 = reinterpret_cast<const float4*>(pgp + g.off_vs) + tig;
+      float4 vsv[8];  // [(ks*4 + e)] -> the 4 channel groups
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vsv[u] = vs4[u * 4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const float* prow = pex + (4 * j + (gq >> 1)) * kPexLd;
+        const float4 pa = *reinterpret_cast<const float4*>(prow + (2 * tig) * 4);
+        const float4 pb = *reinterpret_cast<const float4*>(prow + (2 * tig + 1) * 4);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const unsigned long long p01 = ks ? pk(pa.z, pb.z) : pk(pa.x, pb.x);  // tokens e=0, e=1
+          const unsigned long long p23 = ks ? pk(pa.w, pb.w) : pk(pa.y, pb.y);  // tokens e=2, e=3
+          const float4 s0 = vsv[ks * 4 + 0], s1 = vsv[ks * 4 + 1], s2 = vsv[ks * 4 + 2], s3 = vsv[ks * 4 + 3];
+#pragma unroll
+          for (int grp = 0; grp < 4; ++grp) {
+            const uint32_t b0 = split_bf16(mul2(p01, pk((&s0.x)[grp], (&s1.x)[grp])), nsel);
+            const uint32_t b1 = split_bf16(mul2(p23, pk((&s2.x)[grp], (&s3.x)[grp])), nsel);
+#pragma unroll
+            for (int mh = 0; mh < 2; ++mh) {
+              const int mt = grp * 2 + mh;
+              uint32_t a[4];
+              if constexpr (BITS == 2) {
+                if (ks) frag_a<2, 4>(vw[mt], a); else frag_a<2, 0>(vw[mt], a);
+              } else {
+                frag_a<4, 0>(vw[mt * 2 + ks], a);
+              }
+              mma16816(accv[j][mt], a, b0, b1);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // refill this stage with the page STAGES ahead
+    if (lane == 0 && i + STAGES < my_n) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      bool okp;
+      const uint8_t* src = page_src(i + STAGES, okp);
+      bad_mask &= ~(1u << st);
+      if (okp) {
+        mbar_expect_tx(&bars[st], sub_bytes);
+        bulk_g2s(ring + st * sub_bytes, src, sub_bytes, &bars[st]);
+      } else {
+        set_status(g.status, KVQ_DEV_BAD_PAGE);
+        bad_mask |= 1u << st;
+        mbar_arrive(&bars[st]);
+      }
+    }
+    __syncwarp();
+  }
+  if (stuck_at >= 0) {
+    if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
+    // give the copies already issued (pages stuck_at .. stuck_at + STAGES - 1) a bounded
+    // chance to land before the CTA's shared memory is reused or released
+    for (int i = stuck_at; i < my_n && i < stuck_at + STAGES; ++i)
+      (void)mbar_wait(&bars[i % STAGES], (i / STAGES) & 1);
+  }
+
+  // ---- newest incomplete group: exact keys from the K tail, values from the partial page
+  if (split == nsplit - 1 && warp == 0 && ntail > 0) {
+    const int phys = g.page_table[(size_t)b * g.maxp + nfull];
+    if (phys >= 0 && phys < g.npages) {
+      const uint8_t* sub = g.pool + (size_t)phys * g.page_bytes + (size_t)h_kv * g.sub_bytes;
+      const uint32_t* vwords = reinterpret_cast<const uint32_t*>(sub + g.off_vc);
+      const float* vs = reinterpret_cast<const float*>(sub + g.off_vs);
+      const float* vz = reinterpret_cast<const float*>(sub + g.off_vz);
+      const float* vr = reinterpret_cast<const float*>(sub + g.off_vrow);
+      for (int t = 0; t < ntail; ++t) {
+        const uint16_t* kt = g.k_tail + (((size_t)b * g.H + h_kv) * kG + t) * kD;
+        float kv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) kv[k] = load_elem(kt + lane + 32 * k, g.dtype);
+        const int vidx = min((int)sub[g.off_vidx + tok_pos(t)], P - 1);
+        const float vrow = g.tx ? vr[tok_pos(t)] : 1.0f;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          // score of head 4j + tig (every lane computes the tile's 4 heads, keeps its own)
+          float myscore = 0.f;
+#pragma unroll
+          for (int hl = 0; hl < 4; ++hl) {
+            const int hh = 4 * j + hl;
+            float part = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) part = fmaf(qraw[hh * kD + lane + 32 * k], kv[k], part);
+            part = warp_sum(part) * scale_log2;
+            if (hl == tig) myscore = part;
+          }
+          const int hh = 4 * j + tig;
+          const bool real = hh < Gq;
+          const float mnew = fmaxf(mrun[j], myscore);
+          const float alpha = ex2(mrun[j] - mnew);
+          if (__any_sync(kFull, alpha != 1.0f)) {
+            lrun[j] *= alpha;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) zacc[j][u] *= alpha;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+              for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
+            for (int jj = gq; jj < P; jj += 8) Ww[hh * P + jj] *= alpha;
+          }
+          mrun[j] = mnew;
+          __syncwarp();
+          const float p = real ? ex2(myscore - mnew) : 0.f;
+          const float pv = p * vrow;
+          if (gq == 0) {
+            lrun[j] += p;
+            if (real) Ww[hh * P + vidx] += pv;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) zacc[j][u] = fmaf(pv, vz[vzc_pos(t, u)], zacc[j][u]);
+          }
+          // residual codes of this thread's 16 channels
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int rh = 0; rh < 2; ++rh) {
+              const int d = 16 * mt + 8 * rh + gq;
+              int w, bt;
+              frag_pos(BITS, 2, d, t, w, bt);
+              const int code = (vwords[w] >> bt) & ((1 << BITS) - 1);
+              accv[j][mt][2 * rh] = fmaf(pv * vs[vsc_pos(t, mt >> 1)], (float)code, accv[j][mt][2 * rh]);
+            }
+          __syncwarp();
+        }
+      }
+    } else if (lane == 0) {
+      set_status(g.status, KVQ_DEV_BAD_PAGE);
+    }
+  }
+
+  // ---- merge the warps and write the partials
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    float l = lrun[j];
+    l += __shfl_xor_sync(kFull, l, 4);
+    l += __shfl_xor_sync(kFull, l, 8);
+    l += __shfl_xor_sync(kFull, l, 16);
+    lrun[j] = l;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float z = zacc[j][u];
+      z += __shfl_xor_sync(kFull, z, 4);
+      z += __shfl_xor_sync(kFull, z, 8);
+      z += __shfl_xor_sync(kFull, z, 16);
+      zacc[j][u] = z;
+    }
+  }
+  __syncthreads();  // every warp is done with its ring: reuse it for the merge
+  float* mo = reinterpret_cast<float*>(smem + sp.ring);   // [kWarps][NH][128]
+  float* mm = mo + kWarps * NH * kD;                      // [kWarps][NH] max
+  float* ml = mm + kWarps * NH;                           // [kWarps][NH] sum
+  float* mz = ml + kWarps * NH;                           // [kWarps][NH][4]
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int hh = 4 * j + tig;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      mo[(warp * NH + hh) * kD + 16 * mt + gq] = accv[j][mt][0] + accv[j][mt][1];
+      mo[(warp * NH + hh) * kD + 16 * mt + gq + 8] = accv[j][mt][2] + accv[j][mt][3];
+    }
+    if (gq == 0) {
+      mm[warp * NH + hh] = mrun[j];
+      ml[warp * NH + hh] = lrun[j];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) mz[(warp * NH + hh) * 4 + u] = zacc[j][u];
+    }
+  }
+  __syncthreads();
+  for (int hh = warp; hh < Gq; hh += kWarps) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * NH + hh]);
+    float f[kWarps], Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = mm[w * NH + hh];
+      f[w] = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+      Ls += f[w] * ml[w * NH + hh];
+    }
+    const size_t base = ((size_t)b * Hq + h_kv * Gq + hh) * nsplit + split;
+    if (lane == 0) { part_ml[2 * base] = M; part_ml[2 * base + 1] = Ls; }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        o += f[w] * (mo[(w * NH + hh) * kD + lane + 32 * k] + mz[(w * NH + hh) * 4 + k]);
+      part_o[base * kD + lane + 32 * k] = o;
+    }
+    for (int jj = lane; jj < P; jj += 32) {
+      float Wv = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) Wv += f[w] * Wall[(w * NH + hh) * P + jj];
+      part_w[base * P + jj] = Wv;
+    }
+  }
+}
+
+template <int BITS, int NT, int STAGES>
+struct Launcher {
+  static auto kernel() { return decode_mma_kernel<BITS, NT, STAGES>; }
+  static int smem(const Geom& g) { return smem_plan((int)g.sub_bytes, STAGES, NT, g.P).total; }
+  static int occupancy(const Geom& g) {
+    int n = 0;
+    if (cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, smem(g)) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel(), kWarps * 32, smem(g)) != cudaSuccess) return 1;
+    return n > 0 ? n : 1;
+  }
+  static cudaError_t launch(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml, float* o,
+                            float* w, cudaStream_t st) {
+    const int total = smem(g);
+    cudaError_t e = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit, g.H, g.B);
+    kernel()<<<grid, kWarps * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w);
+    return cudaGetLastError();
+  }
+};
+
+// Dispatch on (bits, n-tiles, stages) with a functor receiving the Launcher type.
+template <typename F>
+auto dispatch(const Geom& g, int Hq, int stages, F&& f) {
+  const int NT = (Hq / g.H + 3) / 4;
+#define KVQ_NT(B, S)                                         \
+  switch (NT) {                                              \
+    case 1: return f(Launcher<B, 1, S>{});                   \
+    case 2: return f(Launcher<B, 2, S>{});                   \
+    case 3: return f(Launcher<B, 3, S>{});                   \
+    default: return f(Launcher<B, 4, S>{});                  \
+  }
+  if (g.bits == 2) {
+    if (stages <= 2) { KVQ_NT(2, 2) } else { KVQ_NT(2, 3) }
+  } else {
+    if (stages <= 2) { KVQ_NT(4, 2) } else { KVQ_NT(4, 3) }
+  }
+#undef KVQ_NT
+}
+
+int decode_stages() {
+  const char* s = getenv("KVQ_DECODE_STAGES");
+  return (s && atoi(s) == 2) ? 2 : 3;
+}
+
+}  // namespace
+
+// Number of splits of the token axis: the CTAs of all (sequence, KV head, split) units run in
+// as few and as full waves as possible, with a small charge per extra split (setup, combine).
+int decode_mma_splits(const Geom& g, int Hq, int num_sms) {
+  const int occ = dispatch(g, Hq, decode_stages(), [&](auto L) { return decltype(L)::occupancy(g); });
+  const int slots = occ * num_sms;
+  const int units = g.B * g.H > 0 ? g.B * g.H : 1;
+  const int maxns = g.maxp > 1 ? (g.maxp < 256 ? g.maxp : 256) : 1;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int ns = 1; ns <= maxns; ++ns) {
+    const double waves = (double)((units * ns + slots - 1) / slots);
+    const double cost = waves / ns * (1.0 + 0.01 * ns);
+    if (cost < best_cost - 1e-12) { best_cost = cost; best = ns; }
+  }
+  return best;
+}
+
+size_t decode_mma_smem(const Geom& g, int Hq) {
+  return (size_t)dispatch(g, Hq, decode_stages(), [&](auto L) { return decltype(L)::smem(g); });
+}
+
+cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
+                              float* o, float* w, cudaStream_t st) {
+  return dispatch(g, Hq, decode_stages(), [&](auto L) {
+    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, w, st);
+  });
+}
+
+}  // namespace kvq

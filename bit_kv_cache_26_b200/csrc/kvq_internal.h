@@ -14,10 +14,14 @@ struct Geom;
 cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, int n_new, cudaStream_t st);
 
 // decode attention (kvq_decode.cu)
-int decode_num_splits(const Geom& g, int num_sms);
+int decode_num_splits(const Geom& g, int Hq, int num_sms);
 size_t decode_workspace(const Geom& g, int Hq, int nsplit);
 cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, float* out, void* ws, int nsplit,
                           cudaStream_t st);
+cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
+                              float* o, float* w, cudaStream_t st);
+size_t decode_mma_smem(const Geom& g, int Hq);
+int decode_mma_splits(const Geom& g, int Hq, int num_sms);
 
 // dequantize (kvq_dequant.cu)
 cudaError_t launch_dequant(const Geom& g, int seq, int start, int count, float* k_out, float* v_out,

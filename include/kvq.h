@@ -51,15 +51,17 @@
  *   V: X[channel][token]): element (row, col) belongs to
  *       lane = ((row % 16) % 8) * 4 + ((col % 16) % 8) / 2,   odd = col % 2,
  *       reg  = ((row / 16) * KS + col / 16) * 4 + (row % 16) / 8 + 2 * ((col % 16) / 8)
- *   and sits in the little-endian 32-bit word  lane*8 + reg/8  at bit 2*(reg%8) + 16*odd
- *   (2-bit), or in word lane*16 + reg/4 at bit 4*(reg%4) + 16*odd (4-bit).  (This is
- *   the register order of the A operand of a 16x8x16 tensor-core MMA, so a decode
- *   warp lane reads its operands as one contiguous run.)
+ *   and to the lane's word w = reg/8 at bit 2*(reg%8) + 16*odd (2-bit), or w = reg/4 at
+ *   bit 4*(reg%4) + 16*odd (4-bit).  A lane's words are stored in 16-byte chunks that
+ *   interleave the lanes: word w of lane l is the little-endian 32-bit word number
+ *       (w / 4) * 128 + l * 4 + (w % 4)
+ *   of the code block.  (The register order of the A operand of a 16x8x16 tensor-core
+ *   MMA: each lane reads its operands with conflict-free 16-byte loads.)
  *   Orders of the per-channel / per-token fields (i = position in the field):
- *       KSC: i = tig*32 + ks*4 + e            -> channel 16*ks + 2*tig + (e&1) + 8*(e>>1)
- *       VSC: i = ((tig*2 + ks)*4 + e)*4 + grp -> token 16*ks + 2*tig + (e&1) + 8*(e>>1),
+ *       KSC: i = ks*16 + tig*4 + e            -> channel 16*ks + 2*tig + (e&1) + 8*(e>>1)
+ *       VSC: i = ((ks*4 + e)*4 + tig)*4 + grp -> token 16*ks + 2*tig + (e&1) + 8*(e>>1),
  *                                                channel group grp (channels 32*grp..32*grp+31)
- *       VZC: i = (g*4 + j)*4 + grp            -> token g + 8*j, channel group grp
+ *       VZC: i = (j*8 + g)*4 + grp            -> token g + 8*j, channel group grp
  *       TOK: i = g*4 + j                      -> token g + 8*j
  *   Entries of tokens not yet appended are zero.  The K part of a page (codes,
  *   scales, indices, row factors) is written when its 32nd token arrives; until
@@ -118,6 +120,8 @@ typedef enum {
 #define KVQ_DEV_BAD_PAGE 0x1   /* page_table entry outside [0, num_pages) */
 #define KVQ_DEV_OVERFLOW 0x2   /* seq_len + n_new > max_pages_per_seq * 32 */
 #define KVQ_DEV_BAD_SET 0x4    /* seq_to_set entry outside [0, num_sets) */
+#define KVQ_DEV_TIMEOUT 0x8    /* a bounded wait for a page copy expired; that step's output is invalid */
+#define KVQ_DEV_RANGE 0x10     /* decode: |q_d * s_d| or a V scale exceeded the fp16 operand range (~3e4) */
 
 typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 typedef enum { KVQ_TX_NONE = 0, KVQ_TX_HADAMARD_VARNORM = 1 } kvq_transform;

@@ -291,12 +291,13 @@ def attention_unit(q: np.ndarray, K: np.ndarray, e: Encoded, MK, MV, cK=None, cV
 # MT=2, KS=8; V: X[channel][token], MT=8, KS=2): element (row, col) has
 #   lane = (row%16 % 8)*4 + (col%16 % 8)//2,  odd = col % 2,
 #   reg  = ((row//16)*KS + col//16)*4 + (row%16)//8 + 2*((col%16)//8)
-# and sits in little-endian 32-bit word  lane*8 + reg//8  at bit 2*(reg%8) + 16*odd
-# (2-bit), or word lane*16 + reg//4 at bit 4*(reg%4) + 16*odd (4-bit).
-# Orders:  KSC[i], i = tig*32 + ks*4 + e     -> channel 16ks + 2tig + (e&1) + 8(e>>1)
-#          VSC[i], i = ((tig*2+ks)*4+e)*4+grp -> (token 16ks + 2tig + (e&1) + 8(e>>1), group grp)
-#          VZC[i], i = (g*4 + j)*4 + grp     -> (token g + 8j, group grp)
-#          TOK[i], i = g*4 + j               -> token g + 8j
+# and belongs to the lane's word w = reg//8 at bit 2*(reg%8) + 16*odd (2-bit), or
+# w = reg//4 at bit 4*(reg%4) + 16*odd (4-bit); word w of lane l is the little-endian
+# 32-bit word (w//4)*128 + l*4 + w%4 of the block (lane-interleaved 16-byte chunks).
+# Orders:  KSC[i], i = ks*16 + tig*4 + e      -> channel 16ks + 2tig + (e&1) + 8(e>>1)
+#          VSC[i], i = ((ks*4+e)*4+tig)*4+grp -> (token 16ks + 2tig + (e&1) + 8(e>>1), group grp)
+#          VZC[i], i = (j*8 + g)*4 + grp      -> (token g + 8j, group grp)
+#          TOK[i], i = g*4 + j                -> token g + 8j
 # Entries of tokens not yet appended are zero; the K part of a page is
 # undefined until its 32nd token arrives.
 # ---------------------------------------------------------------------------
@@ -316,9 +317,10 @@ def _frag_words(MT: int, KS: int, bits: int):
     reg = ((rows // 16) * KS + cols // 16) * 4 + rr // 8 + 2 * (cc // 8)
     odd = cols % 2
     if bits == 2:
-        word, bit = lane * 8 + reg // 8, 2 * (reg % 8) + 16 * odd
+        w, bit = reg // 8, 2 * (reg % 8) + 16 * odd
     else:
-        word, bit = lane * 16 + reg // 4, 4 * (reg % 4) + 16 * odd
+        w, bit = reg // 4, 4 * (reg % 4) + 16 * odd
+    word = (w // 4) * 128 + lane * 4 + w % 4
     return word, bit
 
 
@@ -337,15 +339,15 @@ def unpack_codes(buf: np.ndarray, MT: int, KS: int, bits: int) -> np.ndarray:
 
 def _orders():
     i = np.arange(128)
-    tig, ks, e = i // 32, (i // 4) % 8, i % 4
+    ks, tig, e = i // 16, (i // 4) % 4, i % 4
     ksc = 16 * ks + 2 * tig + (e & 1) + 8 * (e >> 1)
     grp = i % 4
-    e2 = (i // 4) % 4
-    ks2 = (i // 16) % 2
-    tig2 = i // 32
+    tig2 = (i // 4) % 4
+    e2 = (i // 16) % 4
+    ks2 = i // 64
     vsc_tok = 16 * ks2 + 2 * tig2 + (e2 & 1) + 8 * (e2 >> 1)
-    j = (i // 4) % 4
-    g = i // 16
+    g = (i // 4) % 8
+    j = i // 32
     vzc_tok = g + 8 * j
     t = np.arange(32)
     tok = (t // 4) + 8 * (t % 4)
