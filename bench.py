@@ -152,6 +152,23 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def rank_workload(base, rank: int):
+    """The batch rank `rank` processes: same shape, its own seed (batch-sharded replicas, weak scaling)."""
+    return base.with_(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity on a single process)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def workload_config(w, args):
     return {"workload": w.name, "batch": w.B, "context": w.S, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": D,
             "patterns": w.P, "lloyd_iters": w.iters, "bits": w.bits, "group": 32,
@@ -198,7 +215,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
-    w = base.with_(seed=base.seed + 1000 * rank)  # each rank its own batch
+    w = rank_workload(base, rank)
     k, v = synth.gen_kv(w)
     q = synth.gen_q(w)
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
@@ -214,6 +231,7 @@ def main():
     n = w.B * w.S
     ws_m = kvq._alloc_aligned(kvq.kvq_mine_workspace_bytes(n, 1, w.Hkv, w.P, w.transform), dev)
     ws_d = cache.decode_workspace(w.Hq)
+    ws_a = cache.append_workspace()
     out = torch.empty(w.B, w.Hq, D, device=dev)
     out_h = torch.empty(w.B, w.Hq, D).pin_memory()
     tok_stride, set_stride = w.Hkv * D, n * w.Hkv * D
@@ -227,7 +245,7 @@ def main():
                               cache.v_patterns, cache.v_colscale, None, ws_m)
         if ev: ev[1].record()
         cache.seq_len.zero_()
-        kvq.kvq_quantize_append(cache.c, kx, vx, w.S)
+        kvq.kvq_quantize_append(cache.c, kx, vx, w.S, ws_a)
         if ev: ev[2].record()
         kvq.kvq_decode_attention(cache.c, qx, w.Hq, D ** -0.5, out, ws_d)
         if ev: ev[3].record()
@@ -280,10 +298,7 @@ def main():
     e2e_ms = e0.elapsed_time(e1)
     barrier()
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = t.tolist()
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], device=dev)
 
     ms_per_step = elapsed_ms / args.steps
     tokens = n * world
@@ -325,7 +340,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
                     "d2h_bytes_per_step": int(out_h.numel() * 4)},
-            "gpu_launches": args.steps * (2 * (1 + 3 * w.iters + (13 if w.transform else 0)) + 2 + 2),
+            "gpu_launches": args.steps * (2 * (1 + 5 * w.iters + (15 if w.transform else 0)) + 3 + 2),
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

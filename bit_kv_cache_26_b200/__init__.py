@@ -24,7 +24,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA, KVQ_ERR_DEVICE = range(7)
-KVQ_DEV_BAD_PAGE, KVQ_DEV_OVERFLOW, KVQ_DEV_BAD_SET = 0x1, 0x2, 0x4
+KVQ_DEV_BAD_PAGE, KVQ_DEV_OVERFLOW, KVQ_DEV_BAD_SET, KVQ_DEV_TIMEOUT, KVQ_DEV_RANGE = 0x1, 0x2, 0x4, 0x8, 0x10
 KVQ_F16, KVQ_BF16 = 0, 1
 KVQ_TX_NONE, KVQ_TX_HADAMARD_VARNORM = 0, 1
 HEAD_DIM, GROUP = 128, 32
@@ -223,8 +223,13 @@ class PagedKVCache:
         o = phys * self.page_bytes + head * self.subblock_bytes
         return self.pool[o:o + self.subblock_bytes]
 
+    def append_workspace(self) -> torch.Tensor:
+        if getattr(self, "_append_ws", None) is None:
+            self._append_ws = _alloc_aligned(max(256, kvq_append_workspace_bytes(self.c, 1)), self.device)
+        return self._append_ws
+
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
-        kvq_quantize_append(self.c, k_new, v_new, int(k_new.shape[1]), None, stream)
+        kvq_quantize_append(self.c, k_new, v_new, int(k_new.shape[1]), self.append_workspace(), stream)
 
     def decode_workspace(self, num_q_heads: int) -> torch.Tensor:
         return _alloc_aligned(kvq_decode_workspace_bytes(self.c, num_q_heads), self.device)

@@ -102,7 +102,8 @@ kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t nu
   if (transform && !colscale_out) return fail(KVQ_ERR_INVALID_ARG, "transform needs colscale_out");
   if (tok_stride < 0 || head_stride < 0 || set_stride < 0)
     return fail(KVQ_ERR_INVALID_ARG, "negative stride");
-  if (!aligned(x, 2)) return fail(KVQ_ERR_INVALID_ARG, "x must be 2-byte aligned");
+  if (!aligned(x, 16) || tok_stride % 8 || head_stride % 8 || set_stride % 8)
+    return fail(KVQ_ERR_INVALID_ARG, "x must be 16-byte aligned and its strides multiples of 8 elements");
   size_t need = kvq::mine_workspace(n, num_sets, num_kv_heads, P, transform);
   if (ws_bytes < need || (!ws && need))
     return fail(KVQ_ERR_WORKSPACE, "mine workspace %zu < %zu bytes", ws_bytes, need);
@@ -116,16 +117,14 @@ kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t nu
 }
 
 size_t kvq_append_workspace_bytes(const kvq_cache* cache, int32_t n_new) {
-  (void)cache;
   (void)n_new;
-  return 0;
+  if (!cache || cache->num_kv_heads < 1 || cache->num_sets < 1 || cache->num_patterns < 1) return 0;
+  return kvq::append_workspace(kvq::make_geom(*cache));
 }
 
 kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
                                void* ws, size_t ws_bytes, kvq_stream_t stream) {
   g_err[0] = 0;
-  (void)ws;
-  (void)ws_bytes;
   kvq_status s = check_cache(cache);
   if (s != KVQ_OK) return s;
   if (n_new < 0) return fail(KVQ_ERR_INVALID_ARG, "n_new %d < 0", n_new);
@@ -136,7 +135,10 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
   if (!k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "k_new / v_new is NULL");
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return fail(KVQ_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
   kvq::Geom g = kvq::make_geom(*cache);
-  cudaError_t e = kvq::launch_append(g, k_new, v_new, n_new, (cudaStream_t)stream);
+  const size_t need = kvq::append_workspace(g);
+  if (ws_bytes < need || !ws) return fail(KVQ_ERR_WORKSPACE, "append workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned(ws, 256)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaError_t e = kvq::launch_append(g, k_new, v_new, n_new, ws, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kvq_quantize_append");
   return KVQ_OK;
 }

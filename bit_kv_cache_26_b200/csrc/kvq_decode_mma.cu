@@ -33,7 +33,6 @@ namespace kvq {
 
 namespace {
 
-constexpr int kWarps = 4;
 constexpr int kStages = 3;
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr float kRangeLimit = 30000.0f;
@@ -160,10 +159,13 @@ struct Smem {
 };
 constexpr int kPexLd = 36;  // padded row of the p exchange (floats): conflict-free 16-byte reads
 
-__host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int P) {
+__host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int P, int kWarps) {
   Smem s;
   int o = 0;
-  s.ring = o; o += kWarps * stages * sub_bytes;
+  // the ring; the merge at the end reuses this region, so it is at least as large as the merge
+  const int merge = (kWarps * NT * 4 * kD + 2 * kWarps * NT * 4 + kWarps * NT * 4 * 4) * 4;
+  const int ring = kWarps * stages * sub_bytes;
+  s.ring = o; o += ring > merge ? ring : merge;
   o = (o + 15) & ~15;
   s.bars = o; o += kWarps * stages * 8;
   s.qk = o; o += NT * 4 * kD * 4;          // query in the quantized space, per padded head, KSC order
@@ -175,8 +177,8 @@ __host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int
   return s;
 }
 
-template <int BITS, int NT, int STAGES>
-__global__ void __launch_bounds__(kWarps * 32, (STAGES <= 2 ? 4 : 3))
+template <int BITS, int NT, int STAGES, int kWarps>
+__global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 : 3) : 2))
     decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
                       float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w) {
   constexpr int NH = NT * 4;  // padded heads
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kWarps * 32, (STAGES <= 2 ? 4 : 3))
   const unsigned long long nsel = pk(-lo_sel, -lo_sel);
   const int P = g.P;
   const uint32_t sub_bytes = (uint32_t)g.sub_bytes;
-  const Smem sp = smem_plan((int)sub_bytes, STAGES, NT, P);
+  const Smem sp = smem_plan((int)sub_bytes, STAGES, NT, P, kWarps);
 
   uint8_t* ring = smem + sp.ring + warp * STAGES * sub_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * STAGES;
@@ -629,14 +631,14 @@ __global__ void __launch_bounds__(kWarps * 32, (STAGES <= 2 ? 4 : 3))
   }
 }
 
-template <int BITS, int NT, int STAGES>
+template <int BITS, int NT, int STAGES, int NW>
 struct Launcher {
-  static auto kernel() { return decode_mma_kernel<BITS, NT, STAGES>; }
-  static int smem(const Geom& g) { return smem_plan((int)g.sub_bytes, STAGES, NT, g.P).total; }
+  static auto kernel() { return decode_mma_kernel<BITS, NT, STAGES, NW>; }
+  static int smem(const Geom& g) { return smem_plan((int)g.sub_bytes, STAGES, NT, g.P, NW).total; }
   static int occupancy(const Geom& g) {
     int n = 0;
     if (cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, smem(g)) != cudaSuccess) return 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel(), kWarps * 32, smem(g)) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel(), NW * 32, smem(g)) != cudaSuccess) return 1;
     return n > 0 ? n : 1;
   }
   static cudaError_t launch(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml, float* o,
@@ -645,33 +647,46 @@ struct Launcher {
     cudaError_t e = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, g.H, g.B);
-    kernel()<<<grid, kWarps * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w);
+    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w);
     return cudaGetLastError();
   }
 };
 
-// Dispatch on (bits, n-tiles, stages) with a functor receiving the Launcher type.
+// Dispatch on (bits, n-tiles, pipeline configuration) with a functor receiving the Launcher
+// type.  Configurations (stages per warp, warps per CTA): 0 = (3, 4), 1 = (2, 4), 2 = (2, 8),
+// 3 = (3, 8); the query-head tiles beyond the first use configuration 0 or 1.
 template <typename F>
-auto dispatch(const Geom& g, int Hq, int stages, F&& f) {
+auto dispatch(const Geom& g, int Hq, int cfg, F&& f) {
   const int NT = (Hq / g.H + 3) / 4;
-#define KVQ_NT(B, S)                                         \
-  switch (NT) {                                              \
-    case 1: return f(Launcher<B, 1, S>{});                   \
-    case 2: return f(Launcher<B, 2, S>{});                   \
-    case 3: return f(Launcher<B, 3, S>{});                   \
-    default: return f(Launcher<B, 4, S>{});                  \
+#define KVQ_CFG(B)                                                   \
+  if (NT == 1) {                                                     \
+    switch (cfg) {                                                   \
+      case 1: return f(Launcher<B, 1, 2, 4>{});                      \
+      case 2: return f(Launcher<B, 1, 2, 8>{});                      \
+      case 3: return f(Launcher<B, 1, 3, 8>{});                      \
+      default: return f(Launcher<B, 1, 3, 4>{});                     \
+    }                                                                \
+  }                                                                  \
+  if (cfg == 1) {                                                    \
+    switch (NT) {                                                    \
+      case 2: return f(Launcher<B, 2, 2, 4>{});                      \
+      case 3: return f(Launcher<B, 3, 2, 4>{});                      \
+      default: return f(Launcher<B, 4, 2, 4>{});                     \
+    }                                                                \
+  }                                                                  \
+  switch (NT) {                                                      \
+    case 2: return f(Launcher<B, 2, 3, 4>{});                        \
+    case 3: return f(Launcher<B, 3, 3, 4>{});                        \
+    default: return f(Launcher<B, 4, 3, 4>{});                       \
   }
-  if (g.bits == 2) {
-    if (stages <= 2) { KVQ_NT(2, 2) } else { KVQ_NT(2, 3) }
-  } else {
-    if (stages <= 2) { KVQ_NT(4, 2) } else { KVQ_NT(4, 3) }
-  }
-#undef KVQ_NT
+  if (g.bits == 2) { KVQ_CFG(2) } else { KVQ_CFG(4) }
+#undef KVQ_CFG
 }
 
 int decode_stages() {
-  const char* s = getenv("KVQ_DECODE_STAGES");
-  return (s && atoi(s) == 2) ? 2 : 3;
+  const char* s = getenv("KVQ_DECODE_CFG");
+  const int v = s ? atoi(s) : 1;
+  return (v >= 0 && v <= 3) ? v : 1;
 }
 
 }  // namespace

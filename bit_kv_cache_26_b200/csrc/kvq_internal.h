@@ -11,7 +11,8 @@ namespace kvq {
 struct Geom;
 
 // quantize-append (kvq_append.cu)
-cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, int n_new, cudaStream_t st);
+size_t append_workspace(const Geom& g);
+cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, int n_new, void* ws, cudaStream_t st);
 
 // decode attention (kvq_decode.cu)
 int decode_num_splits(const Geom& g, int Hq, int num_sms);

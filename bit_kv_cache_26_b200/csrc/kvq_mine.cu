@@ -22,6 +22,8 @@ constexpr int kReduceChunk = 4096;
 struct MineWs {
   double* sums;     // [NP][P][128]
   uint32_t* cnt;    // [NP][P]
+  uint32_t* cursor; // [NP][P]  slots handed out per cluster by the counting sort
+  int32_t* order;   // [NP][n]  token indices grouped by cluster
   int32_t* assign;  // [NP][n]
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
@@ -38,6 +40,8 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   MineWs w{};
   w.sums = (double*)p; p += align256((size_t)NP * P * kD * sizeof(double));
   w.cnt = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
+  w.cursor = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
+  w.order = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t));
   if (assign_out) w.assign = assign_out;
   else { w.assign = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t)); }
   if (transform) {
@@ -190,42 +194,80 @@ __global__ void __launch_bounds__(128) mine_assign_kernel(Src s, int P, const fl
 //
 // Scores e_j = |m_j|^2 - 2 x.m_j come from bf16 m16n8k16 MMAs: every pattern is split
 // exactly into three bf16 terms (8+8+8 bits), inputs are exact in bf16 (bf16 input) or
-// split into two bf16 terms (fp16 input exactly; fp32 pre-transformed rows to 2^-17).
+// split into two bf16 terms (fp16 input exactly; fp32 pre-transformed rows to 2^-16).
 // With E_j a bound on |e_hat_j - e_j| and U = min_j (e_hat_j + E_j), the float64
-// argmin can only be a pattern with e_hat_j - E_j <= U + delta.  One such pattern is
-// the answer; several are decided by recomputing their float64 distances exactly as
-// the sequential reference does.  E_j = 2^-10 |x| |m_j| + 2^-20 (|x|^2 + |m_j|^2)
-// covers fp32 accumulation in the tensor cores with a wide margin (the exact bound
-// for 400 fp32 additions of exact products is below 2^-13.6 |x| |m_j|).
+// argmin can only be a pattern with e_hat_j - E_j <= U + delta.  A token whose best two
+// scores are more than 2 max_j E_j + delta apart is decided at once; the others (1-2 %)
+// are decided by recomputing float64 distances of the candidates exactly as the
+// sequential reference does.  E_j = 2^-12 |x| |m_j| + 2^-20 (|x|^2 + |m_j|^2) covers fp32
+// accumulation in the tensor cores with margin: 24 chained MMAs of exact bf16 products
+// stay below 2^-18 |x| |m_j| with one correctly rounded fp32 sum per MMA, and below
+// 2^-13.4 |x| |m_j| even if each MMA truncated its 16-term sum to 22 bits.
+//
+// The MMA k index runs over channels in the order pi(kp, tig, e) = 8 (4 kp + tig) + e for
+// k-step 2 kp + (e >> 2) ... so that every lane's A operands of a pair of k-steps are 8
+// consecutive channels (one 16-byte load) and its B operands 8 consecutive bf16 values of
+// a pattern row (one 16-byte shared load).  A dot product does not depend on the order of k.
 constexpr int kMmaMaxP = 128;
 constexpr int kMmaWarps = 4;
-constexpr int kBLd = kD + 8;  // padded bf16 row of a pattern split in shared memory
+constexpr int kBLd = kD + 32;  // bf16 row of a pattern split: 320 B = 64 mod 128, conflict-free 16-byte loads
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+// bf16 hi / lo parts of two fp32 values by truncation (hi + lo keeps 16 significant bits).
+__device__ __forceinline__ void split_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+  hi = __byte_perm(u0, u1, 0x7632);
+  const float r0 = x0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = x1 - __uint_as_float(u1 & 0xFFFF0000u);
+  lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
 }
 
-// hi and lo bf16 parts of two fp32 values (hi = rn(x), lo = rn(x - hi)).
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  float2 hf = __bfloat1622float2(h);
-  hi = *reinterpret_cast<uint32_t*>(&h);
-  lo = pack_bf16(x0 - hf.x, x1 - hf.y);
+struct Top2 {
+  float m1, m2;
+  int j1;
+};
+__device__ __forceinline__ void top2_add(Top2& t, float e, int j) {
+  if (e < t.m1 || (e == t.m1 && j < t.j1)) { t.m2 = t.m1; t.m1 = e; t.j1 = j; }
+  else if (e < t.m2) t.m2 = e;
+}
+__device__ __forceinline__ void top2_merge_xor(Top2& t, int mask) {
+  const float om1 = __shfl_xor_sync(kFull, t.m1, mask), om2 = __shfl_xor_sync(kFull, t.m2, mask);
+  const int oj = __shfl_xor_sync(kFull, t.j1, mask);
+  const float lo2 = fminf(t.m2, om2);
+  if (om1 < t.m1 || (om1 == t.m1 && oj < t.j1)) { t.m2 = fminf(t.m1, lo2); t.m1 = om1; t.j1 = oj; }
+  else t.m2 = fminf(om1, lo2);
+}
+
+// 8 consecutive input values of row i starting at channel c (bf16 input: one 16-byte load).
+template <int NA>
+__device__ __forceinline__ void load8(const Src& s, int prob, int64_t i, int c, float (&v)[8]) {
+  if (s.y) {
+    const float4* p = reinterpret_cast<const float4*>(s.y + ((size_t)prob * s.n + i) * kD + c);
+    const float4 a = p[0], b = p[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const int set = prob / s.heads, h = prob % s.heads;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(s.x + set * s.ss + i * s.ts + h * s.hs + c));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = bits_to_float((uint16_t)(w[k] & 0xffff), s.dtype);
+      v[2 * k + 1] = bits_to_float((uint16_t)(w[k] >> 16), s.dtype);
+    }
+  }
 }
 
 // NA = number of bf16 terms of the input (1: exact bf16 input; 2: fp16 or fp32 input).
 template <int NA>
-__global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, int P, const float* __restrict__ M,
-                                                                          int32_t* __restrict__ assign) {
-  constexpr int kMt = NA == 1 ? 2 : 1;  // 16-token m-tiles per warp
+__global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src s, int P, const float* __restrict__ M,
+                                                                             int32_t* __restrict__ assign) {
+  constexpr int kMt = NA == 1 ? 2 : 1;  // 16-token m-tiles per warp tile
   constexpr int kTok = 16 * kMt;        // tokens per warp tile
   extern __shared__ __align__(16) uint8_t smraw[];
   uint8_t* sm = smraw;
@@ -236,11 +278,13 @@ __global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, 
   __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(sm);                       // [3][Pp][kBLd]
   float* mnorm = reinterpret_cast<float*>(sm + (size_t)3 * Pp * kBLd * 2);           // [Pp] |m_j|
   float* msq = mnorm + Pp;                                                            // [Pp] |m_j|^2
-  float* escr = msq + Pp;                                                             // [warps][kTok][Pp+1]
-  float* xn = escr + kMmaWarps * kTok * (Pp + 1);                                     // [warps][kTok] |x|^2
+  const int eld = Pp + 2;                                                             // even: aligned float2 rows
+  float* escr = msq + Pp;                                                             // [warps][kTok][eld]
+  float* xn = escr + kMmaWarps * kTok * eld;                                          // [warps][kTok] |x|^2
+  float* gmax = xn + kMmaWarps * kTok;                                                // [2] max |m|, max |m|^2
   const float* Mp = M + (size_t)prob * P * kD;
 
-  // pattern splits and norms
+  // pattern splits (natural channel order) and norms
   for (int i = threadIdx.x; i < Pp * kD; i += blockDim.x) {
     const int j = i / kD, d = i % kD;
     const float m = j < P ? Mp[(size_t)j * kD + d] : 0.f;
@@ -252,46 +296,55 @@ __global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, 
     Bs[(1 * Pp + j) * kBLd + d] = mid;
     Bs[(2 * Pp + j) * kBLd + d] = lo;
   }
+  if (threadIdx.x == 0) { gmax[0] = 0.f; gmax[1] = 0.f; }
+  __syncthreads();
   for (int j = threadIdx.x; j < Pp; j += blockDim.x) {
     double acc = 0.0;
     if (j < P)
       for (int d = 0; d < kD; ++d) { const double m = Mp[(size_t)j * kD + d]; acc += m * m; }
     msq[j] = (float)acc;
     mnorm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
+    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int(mnorm[j]));
+    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq[j] * (1.0f + 1e-6f)));
   }
   __syncthreads();
+  const float nm_max = gmax[0], msq_max = gmax[1];
 
-  float* esc = escr + warp * kTok * (Pp + 1);
+  float* esc = escr + warp * kTok * eld;
   float* xnw = xn + warp * kTok;
   const int64_t ntiles = (s.n + kTok - 1) / kTok;
   for (int64_t tile = (int64_t)blockIdx.x * kMmaWarps + warp; tile < ntiles; tile += (int64_t)gridDim.x * kMmaWarps) {
     const int64_t t0 = tile * kTok;
-    // A fragments (NA bf16 terms) and the squared norms of the rows
-    uint32_t A[NA][kMt][8][4];
+    // A operands: rows gq (+8) of each m-tile, channels 8(4kp + tig) .. +7 for k-step pair kp
+    uint32_t A[NA][kMt][2][4][4];  // [term][mt][row half][kp][reg]: reg 0,1 = k-step 2kp (b0 half, b1 half)...
     float nrm[kMt][2];
 #pragma unroll
-    for (int mt = 0; mt < kMt; ++mt) {
-      nrm[mt][0] = nrm[mt][1] = 0.f;
+    for (int mt = 0; mt < kMt; ++mt)
 #pragma unroll
       for (int rh = 0; rh < 2; ++rh) {
         const int64_t i = t0 + 16 * mt + 8 * rh + gq;
         const bool ok = i < s.n;
+        nrm[mt][rh] = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
+        for (int kp = 0; kp < 4; ++kp) {
+          float v[8];
+          if (ok) load8<NA>(s, prob, i, 8 * (4 * kp + tig), v);
+          else {
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const int d = 16 * ks + 8 * ch + 2 * tig;
-            const float x0 = ok ? s.at(prob, i, d) : 0.f, x1 = ok ? s.at(prob, i, d + 1) : 0.f;
-            nrm[mt][rh] = fmaf(x0, x0, fmaf(x1, x1, nrm[mt][rh]));
-            const int r = rh + 2 * ch;
+            for (int u = 0; u < 8; ++u) v[u] = 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) nrm[mt][rh] = fmaf(v[u], v[u], nrm[mt][rh]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
             if constexpr (NA == 1) {
-              A[0][mt][ks][r] = pack_bf16(x0, x1);
+              A[0][mt][rh][kp][q] = __byte_perm(__float_as_uint(v[2 * q]), __float_as_uint(v[2 * q + 1]), 0x7632);
             } else {
-              split2(x0, x1, A[0][mt][ks][r], A[NA - 1][mt][ks][r]);
+              split_trunc(v[2 * q], v[2 * q + 1], A[0][mt][rh][kp][q], A[NA - 1][mt][rh][kp][q]);
             }
           }
+        }
       }
-    }
 #pragma unroll
     for (int mt = 0; mt < kMt; ++mt)
 #pragma unroll
@@ -299,8 +352,14 @@ __global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, 
         float v = nrm[mt][rh];
         v += __shfl_xor_sync(kFull, v, 1);
         v += __shfl_xor_sync(kFull, v, 2);
+        nrm[mt][rh] = v;
         if (tig == 0) xnw[16 * mt + 8 * rh + gq] = v * (1.0f + 1e-6f);
       }
+    Top2 top[kMt][2];
+#pragma unroll
+    for (int mt = 0; mt < kMt; ++mt)
+#pragma unroll
+      for (int rh = 0; rh < 2; ++rh) top[mt][rh] = Top2{INFINITY, INFINITY, 0x7fffffff};
     // scores, one n-tile (8 patterns) at a time
     for (int nt = 0; nt < Pp / 8; ++nt) {
       float acc[kMt][4];
@@ -308,65 +367,95 @@ __global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, 
       for (int mt = 0; mt < kMt; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 #pragma unroll
       for (int sp = 0; sp < 3; ++sp) {
-        const __nv_bfloat16* brow = Bs + ((size_t)sp * Pp + 8 * nt + gq) * kBLd + 2 * tig;
+        const __nv_bfloat16* brow = Bs + ((size_t)sp * Pp + 8 * nt + gq) * kBLd + 8 * tig;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(brow + 16 * ks);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(brow + 16 * ks + 8);
+        for (int kp = 0; kp < 4; ++kp) {
+          const uint4 bv = *reinterpret_cast<const uint4*>(brow + 32 * kp);  // channels 8(4kp+tig)..+7
 #pragma unroll
           for (int a = 0; a < NA; ++a)
 #pragma unroll
-            for (int mt = 0; mt < kMt; ++mt) mma_bf16(acc[mt], A[a][mt][ks], b0, b1);
+            for (int mt = 0; mt < kMt; ++mt) {
+              // k-step 2kp: channels +0..+3 -> (a0a1, a4a5) / (b0, b1); rows gq and gq+8 -> a0a1 / a2a3
+              mma_bf16(acc[mt], A[a][mt][0][kp][0], A[a][mt][1][kp][0], A[a][mt][0][kp][1], A[a][mt][1][kp][1], bv.x,
+                       bv.y);
+              mma_bf16(acc[mt], A[a][mt][0][kp][2], A[a][mt][1][kp][2], A[a][mt][0][kp][3], A[a][mt][1][kp][3], bv.z,
+                       bv.w);
+            }
         }
       }
 #pragma unroll
       for (int mt = 0; mt < kMt; ++mt) {
         const int j0 = 8 * nt + 2 * tig;
-        esc[(16 * mt + gq) * (Pp + 1) + j0] = msq[j0] - 2.0f * acc[mt][0];
-        esc[(16 * mt + gq) * (Pp + 1) + j0 + 1] = msq[j0 + 1] - 2.0f * acc[mt][1];
-        esc[(16 * mt + gq + 8) * (Pp + 1) + j0] = msq[j0] - 2.0f * acc[mt][2];
-        esc[(16 * mt + gq + 8) * (Pp + 1) + j0 + 1] = msq[j0 + 1] - 2.0f * acc[mt][3];
+        const float e0 = msq[j0] - 2.0f * acc[mt][0], e1 = msq[j0 + 1] - 2.0f * acc[mt][1];
+        const float e2 = msq[j0] - 2.0f * acc[mt][2], e3 = msq[j0 + 1] - 2.0f * acc[mt][3];
+        *reinterpret_cast<float2*>(&esc[(16 * mt + gq) * eld + j0]) = make_float2(e0, e1);
+        *reinterpret_cast<float2*>(&esc[(16 * mt + gq + 8) * eld + j0]) = make_float2(e2, e3);
+        if (j0 < P) { top2_add(top[mt][0], e0, j0); top2_add(top[mt][1], e2, j0); }
+        if (j0 + 1 < P) { top2_add(top[mt][0], e1, j0 + 1); top2_add(top[mt][1], e3, j0 + 1); }
       }
     }
-    __syncwarp();
-    // certify per token (lane = token of the tile)
-    if (lane < kTok) {
-      const int64_t i = t0 + lane;
-      if (i < s.n) {
-        const float* e = esc + lane * (Pp + 1);
-        const float xsq = xnw[lane];
-        const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
-        float U = INFINITY, best = INFINITY;
-        int bj = 0;
-        for (int j = 0; j < P; ++j) {
-          const float E = 0x1p-10f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
-          U = fminf(U, e[j] + E);
-          if (e[j] < best) { best = e[j]; bj = j; }
-        }
-        int cnt = 0;
-        float emax = 0.f;
-        for (int j = 0; j < P; ++j) {
-          const float E = 0x1p-10f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
-          emax = fmaxf(emax, msq[j]);
-          if (e[j] - E <= U + 1e-9f * (xsq + msq[j])) ++cnt;
-        }
-        if (cnt > 1) {
-          // exact float64 distances of the candidates, channel order, lowest index on ties
+    // gap test per row, then the exact path for the rows that fail it
+    uint32_t need = 0;
+#pragma unroll
+    for (int mt = 0; mt < kMt; ++mt)
+#pragma unroll
+      for (int rh = 0; rh < 2; ++rh) {
+        top2_merge_xor(top[mt][rh], 1);
+        top2_merge_xor(top[mt][rh], 2);
+        const float xsq = nrm[mt][rh] * (1.0f + 1e-6f), nx = sqrtf(xsq) * (1.0f + 1e-6f);
+        const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xsq + msq_max);
+        const int64_t i = t0 + 16 * mt + 8 * rh + gq;
+        const bool unique = top[mt][rh].m2 - top[mt][rh].m1 > 2.0f * Eb + 1e-9f * (xsq + msq_max);
+        if (unique && tig == 0 && i < s.n) assign[(size_t)prob * s.n + i] = top[mt][rh].j1;
+        if (!unique) need |= 1u << (16 * mt + 8 * rh + gq);
+      }
+    need = __reduce_or_sync(kFull, need);
+    if (need) {
+      __syncwarp();
+      if (lane < kTok && ((need >> lane) & 1)) {
+        const int64_t i = t0 + lane;
+        if (i < s.n) {
+          const float* e = esc + lane * eld;
+          const float xsq = xnw[lane];
+          const uint16_t* xrow = s.x ? s.x + (prob / s.heads) * s.ss + i * s.ts + (prob % s.heads) * s.hs : nullptr;
+          const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
+          float U = INFINITY;
+          for (int j = 0; j < P; ++j) U = fminf(U, e[j] + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
           double bd = 0.0;
+          int bj = 0;
           bool have = false;
           for (int j = 0; j < P; ++j) {
-            const float E = 0x1p-10f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
+            const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
             if (!(e[j] - E <= U + 1e-9f * (xsq + msq[j]))) continue;
+            // exact float64 distance, channels in order, as the sequential reference computes it;
+            // the loads do not depend on the running sum, so they are issued well ahead of it
             const float* m = Mp + (size_t)j * kD;
             double acc = 0.0;
-            for (int d = 0; d < kD; ++d) {
-              const double t = __dsub_rn((double)s.at(prob, i, d), (double)__ldg(m + d));
-              acc = __dadd_rn(acc, __dmul_rn(t, t));
+#pragma unroll 8
+            for (int d = 0; d < kD; d += 4) {
+              float xv[4];
+              if (s.y) {
+                const float4 t4 = *reinterpret_cast<const float4*>(s.y + ((size_t)prob * s.n + i) * kD + d);
+                xv[0] = t4.x; xv[1] = t4.y; xv[2] = t4.z; xv[3] = t4.w;
+              } else {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
+                xv[0] = bits_to_float((uint16_t)(u.x & 0xffff), s.dtype);
+                xv[1] = bits_to_float((uint16_t)(u.x >> 16), s.dtype);
+                xv[2] = bits_to_float((uint16_t)(u.y & 0xffff), s.dtype);
+                xv[3] = bits_to_float((uint16_t)(u.y >> 16), s.dtype);
+              }
+              const float4 m4 = __ldg(reinterpret_cast<const float4*>(m + d));
+              const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const double t = __dsub_rn((double)xv[q], (double)mv[q]);
+                acc = __dadd_rn(acc, __dmul_rn(t, t));
+              }
             }
             if (!have || acc < bd) { bd = acc; bj = j; have = true; }
           }
+          assign[(size_t)prob * s.n + i] = bj;
         }
-        assign[(size_t)prob * s.n + i] = bj;
       }
     }
     __syncwarp();
@@ -375,67 +464,162 @@ __global__ void __launch_bounds__(kMmaWarps * 32) mine_assign_mma_kernel(Src s, 
 
 size_t mine_mma_smem(int P, int NA) {
   const int Pp = (P + 7) & ~7, kTok = NA == 1 ? 32 : 16;
-  return (size_t)3 * Pp * kBLd * 2 + 2 * Pp * 4 + (size_t)kMmaWarps * kTok * (Pp + 1) * 4 + kMmaWarps * kTok * 4;
+  return (size_t)3 * Pp * kBLd * 2 + 2 * Pp * 4 + (size_t)kMmaWarps * kTok * (Pp + 2) * 4 + kMmaWarps * kTok * 4 + 16;
 }
 
-// Per-cluster float64 sums over a chunk of tokens for one quarter of the channels;
-// one warp per CTA, lane = channel; flushed with global atomics.
-__global__ void __launch_bounds__(32) mine_reduce_kernel(Src s, int P, const int32_t* __restrict__ assign,
-                                                         double* __restrict__ sums, uint32_t* __restrict__ cnt) {
-  extern __shared__ __align__(16) uint8_t smraw[];
-  double* sm = reinterpret_cast<double*>(smraw);  // [P][32] sums, then [P] counts (as uint32 in the tail)
-  uint32_t* scnt = reinterpret_cast<uint32_t*>(sm + (size_t)P * 32);
-  const int prob = blockIdx.z, quarter = blockIdx.y, lane = threadIdx.x;
-  const int d = quarter * 32 + lane;
-  for (int j = 0; j < P; ++j) sm[j * 32 + lane] = 0.0;
-  for (int j = lane; j < P; j += 32) scnt[j] = 0;
-  __syncwarp();
-  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk, i1 = min(s.n, i0 + kReduceChunk);
-  const int32_t* a = assign + (size_t)prob * s.n;
-  int64_t i = i0;
-  for (; i + 8 <= i1; i += 8) {  // 8 independent loads in flight, then the dependent adds
-    int j[8];
-    float x[8];
+// Per-cluster float64 sums by counting sort: (1) cluster sizes, (2) every token's index
+// written into its cluster's bucket (slots handed out by an atomic cursor, so the order
+// inside a bucket varies), (3) each warp sums a run of consecutive bucket entries in
+// registers and adds the run's partial sums to the cluster total once per cluster it
+// crosses.  float64 sums of fp16 / bf16 values are exact, so the order of the additions
+// does not change them.
+__global__ void __launch_bounds__(256) mine_count_kernel(int64_t n, int P, const int32_t* __restrict__ assign,
+                                                         uint32_t* __restrict__ cnt) {
+  extern __shared__ uint32_t hist[];
+  const int prob = blockIdx.y;
+  for (int j = threadIdx.x; j < P; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk, i1 = min(n, i0 + kReduceChunk);
+  const int32_t* a = assign + (size_t)prob * n;
+  for (int64_t i = i0 + threadIdx.x; i < i1; i += blockDim.x) atomicAdd(&hist[a[i]], 1u);
+  __syncthreads();
+  for (int j = threadIdx.x; j < P; j += blockDim.x)
+    if (hist[j]) atomicAdd(cnt + (size_t)prob * P + j, hist[j]);
+}
+
+// exclusive prefix of the cluster sizes into base[0..P] (base[P] = n), one thread
+__device__ __forceinline__ void cluster_base(const uint32_t* c, int P, uint32_t* base) {
+  uint32_t s = 0;
+  for (int j = 0; j < P; ++j) { base[j] = s; s += c[j]; }
+  base[P] = s;
+}
+
+constexpr int kScatterPer = kReduceChunk / 256;
+
+__global__ void __launch_bounds__(256) mine_scatter_kernel(int64_t n, int P, const int32_t* __restrict__ assign,
+                                                           const uint32_t* __restrict__ cnt,
+                                                           uint32_t* __restrict__ cursor, int32_t* __restrict__ order) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* base = sm;         // [P + 1]
+  uint32_t* lc = sm + P + 1;   // [P] this CTA's tokens per cluster, then its first slot
+  const int prob = blockIdx.y;
+  if (threadIdx.x == 0) cluster_base(cnt + (size_t)prob * P, P, base);
+  for (int j = threadIdx.x; j < P; j += blockDim.x) lc[j] = 0;
+  __syncthreads();
+  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk;
+  const int32_t* a = assign + (size_t)prob * n;
+  int jj[kScatterPer];
+  uint32_t rk[kScatterPer];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) { j[u] = a[i + u]; x[u] = s.at(prob, i + u, d); }
+  for (int u = 0; u < kScatterPer; ++u) {
+    const int64_t i = i0 + u * 256 + threadIdx.x;
+    jj[u] = i < n ? a[i] : -1;
+    if (jj[u] >= 0) rk[u] = atomicAdd(&lc[jj[u]], 1u);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < P; j += blockDim.x)
+    if (lc[j]) lc[j] = base[j] + atomicAdd(cursor + (size_t)prob * P + j, lc[j]);
+  __syncthreads();
+  int32_t* o = order + (size_t)prob * n;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      sm[j[u] * 32 + lane] += (double)x[u];
-      if (quarter == 0 && lane == 0) scnt[j[u]] += 1;
+  for (int u = 0; u < kScatterPer; ++u)
+    if (jj[u] >= 0) o[lc[jj[u]] + rk[u]] = (int32_t)(i0 + u * 256 + threadIdx.x);
+}
+
+constexpr int kSegRun = 256;  // bucket entries per warp
+constexpr int kSegUnroll = 8;
+
+__device__ __forceinline__ void flush4(double* dst, double a0, double a1, double a2, double a3) {
+  if (a0 != 0.0) atomicAdd(dst + 0, a0);
+  if (a1 != 0.0) atomicAdd(dst + 1, a1);
+  if (a2 != 0.0) atomicAdd(dst + 2, a2);
+  if (a3 != 0.0) atomicAdd(dst + 3, a3);
+}
+
+// lane l holds channels 4l..4l+3 of the token rows it sums
+__global__ void __launch_bounds__(256, 3) mine_segsum_kernel(Src s, int P, const int32_t* __restrict__ order,
+                                                          const uint32_t* __restrict__ cnt,
+                                                          double* __restrict__ sums) {
+  extern __shared__ uint32_t base[];  // [P + 1]
+  const int prob = blockIdx.y;
+  if (threadIdx.x == 0) cluster_base(cnt + (size_t)prob * P, P, base);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kSegRun;
+  if (r0 >= s.n) return;
+  const int64_t r1 = min(s.n, r0 + kSegRun);
+  const int32_t* o = order + (size_t)prob * s.n;
+  const int set = prob / s.heads, h = prob % s.heads;
+  const uint16_t* xb = s.x + set * s.ss + h * s.hs + 4 * lane;
+  const float* yb = s.y ? s.y + (size_t)prob * s.n * kD + 4 * lane : nullptr;
+  double* gs = sums + (size_t)prob * P * kD + 4 * lane;
+  // cluster of entry r0: the last j with base[j] <= r0 (skipping empty clusters)
+  int j = 0;
+  {
+    int lo = 0, hi = P - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (base[mid] <= (uint32_t)r0) lo = mid; else hi = mid - 1;
+    }
+    j = lo;
+  }
+  uint32_t jend = base[j + 1];
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int64_t r = r0; r < r1; r += 32) {
+    const int tok_l = r + lane < r1 ? o[r + lane] : 0;
+    const int m = (int)(r1 - r < 32 ? r1 - r : 32);
+    for (int u0 = 0; u0 < m; u0 += kSegUnroll) {
+      float v[kSegUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kSegUnroll; ++u) {
+        const int t = __shfl_sync(0xffffffffu, tok_l, (u0 + u) & 31);
+        if (u0 + u < m) {
+          if (yb) {
+            const float4 f = *reinterpret_cast<const float4*>(yb + (size_t)t * kD);
+            v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+          } else {
+            const uint2 b = __ldg(reinterpret_cast<const uint2*>(xb + (size_t)t * s.ts));
+            v[u][0] = bits_to_float((uint16_t)(b.x & 0xffffu), s.dtype);
+            v[u][1] = bits_to_float((uint16_t)(b.x >> 16), s.dtype);
+            v[u][2] = bits_to_float((uint16_t)(b.y & 0xffffu), s.dtype);
+            v[u][3] = bits_to_float((uint16_t)(b.y >> 16), s.dtype);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSegUnroll; ++u) {
+        if (u0 + u >= m) break;
+        const uint32_t rr = (uint32_t)(r + u0 + u);
+        if (rr >= jend) {  // crossed into a later cluster (warp-uniform)
+          flush4(gs + (size_t)j * kD, acc[0], acc[1], acc[2], acc[3]);
+          acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
+          do { ++j; } while (base[j + 1] <= rr);
+          jend = base[j + 1];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] += (double)v[u][e];
+      }
     }
   }
-  for (; i < i1; ++i) {
-    const int j = a[i];
-    sm[j * 32 + lane] += (double)s.at(prob, i, d);
-    if (quarter == 0 && lane == 0) scnt[j] += 1;
-  }
-  __syncwarp();
-  double* gs = sums + (size_t)prob * P * kD;
-  for (int j = 0; j < P; ++j) {
-    double v = sm[j * 32 + lane];
-    if (v != 0.0) atomicAdd(gs + j * kD + d, v);
-  }
-  if (quarter == 0)
-    for (int j = lane; j < P; j += 32)
-      if (scnt[j]) atomicAdd(cnt + (size_t)prob * P + j, scnt[j]);
+  flush4(gs + (size_t)j * kD, acc[0], acc[1], acc[2], acc[3]);
 }
 
-__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt) {
+__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt, uint32_t* cursor) {
   const int prob = blockIdx.y, j = blockIdx.x, d = threadIdx.x;
   const size_t pj = (size_t)prob * P + j;
   uint32_t c = cnt[pj];
   if (c > 0) M[pj * kD + d] = (float)(sums[pj * kD + d] / (double)c);
   sums[pj * kD + d] = 0.0;
   __syncthreads();
-  if (d == 0) cnt[pj] = 0;
+  if (d == 0) { cnt[pj] = 0; cursor[pj] = 0; }
 }
 
 }  // namespace
 
 size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
   size_t NP = (size_t)sets * heads;
-  size_t b = align256(NP * P * kD * sizeof(double)) + align256(NP * P * sizeof(uint32_t)) +
-             align256(NP * (size_t)n * sizeof(int32_t));
+  size_t b = align256(NP * P * kD * sizeof(double)) + 2 * align256(NP * P * sizeof(uint32_t)) +
+             2 * align256(NP * (size_t)n * sizeof(int32_t));
   if (transform)
     b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
          4 * align256(NP * kD * sizeof(double));
@@ -470,13 +654,10 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   mine_init_kernel<<<dim3(a.P, NP), kD, 0, st>>>(s, a.P, a.patterns);
   cudaMemsetAsync(w.sums, 0, (size_t)NP * a.P * kD * sizeof(double), st);
   cudaMemsetAsync(w.cnt, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
+  cudaMemsetAsync(w.cursor, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
   size_t smem_assign = (size_t)a.P * kD * sizeof(float);
-  size_t smem_reduce = (size_t)a.P * 32 * sizeof(double) + (size_t)a.P * sizeof(uint32_t);
   if ((e = cudaFuncSetAttribute(mine_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_assign)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(mine_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_reduce)) != cudaSuccess)
     return e;
   const int NA = (a.transform || a.dtype == KVQ_F16) ? 2 : 1;
   const bool use_mma = a.P <= kMmaMaxP;
@@ -492,6 +673,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   const int tok_per_cta = kMmaWarps * (NA == 1 ? 32 : 16);
   const unsigned mma_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + tok_per_cta - 1) / tok_per_cta, (int64_t)(2 * sms + NP - 1) / NP));
+  const unsigned seg_ctas = (unsigned)((a.n + 8 * kSegRun - 1) / (8 * kSegRun));
   for (int it = 0; it < a.iters; ++it) {
     if (use_mma && NA == 1)
       mine_assign_mma_kernel<1><<<dim3(mma_ctas, NP), kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
@@ -500,8 +682,12 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     else
       mine_assign_kernel<<<dim3((unsigned)((a.n + 127) / 128), NP), 128, smem_assign, st>>>(s, a.P, a.patterns,
                                                                                            w.assign);
-    mine_reduce_kernel<<<dim3(chunks, 4, NP), 32, smem_reduce, st>>>(s, a.P, w.assign, w.sums, w.cnt);
-    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
+    mine_count_kernel<<<dim3(chunks, NP), 256, a.P * sizeof(uint32_t), st>>>(a.n, a.P, w.assign, w.cnt);
+    mine_scatter_kernel<<<dim3(chunks, NP), 256, (2 * a.P + 1) * sizeof(uint32_t), st>>>(a.n, a.P, w.assign, w.cnt,
+                                                                                         w.cursor, w.order);
+    mine_segsum_kernel<<<dim3(seg_ctas, NP), 256, (a.P + 1) * sizeof(uint32_t), st>>>(s, a.P, w.order, w.cnt,
+                                                                                       w.sums);
+    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt, w.cursor);
   }
   return cudaGetLastError();
 }

@@ -165,7 +165,8 @@ KVQ_API size_t kvq_subblock_bytes(int32_t bits, int32_t transform);
  *
  * For every set s < num_sets and KV head h < num_kv_heads independently, the n
  * vectors x(s, i, h) at  x + s*set_stride + i*tok_stride + h*head_stride  (element
- * strides; 128 contiguous elements each, dtype fp16/bf16) are clustered into P
+ * strides, multiples of 8; x 16-byte aligned; 128 contiguous elements each, dtype
+ * fp16/bf16) are clustered into P
  * patterns with `iters` Lloyd iterations.  With transform = KVQ_TX_HADAMARD_VARNORM
  * the column factors are fitted first and written to colscale_out, and the
  * clustering runs on the normalised vectors y.
@@ -192,7 +193,9 @@ KVQ_API kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, in
  * reaches 32 tokens is quantized per channel and written to its page.  seq_len is
  * advanced by n_new (a sequence that would overflow its page table is left
  * unchanged and flags KVQ_DEV_OVERFLOW).  n_new = 0 is a no-op.
- * Workspace: kvq_append_workspace_bytes() (currently 0; pass NULL, 0).
+ * Workspace: kvq_append_workspace_bytes() (per-call pattern tables: bf16 copies and
+ * the pattern-to-pattern min-max distances used to prune the exact assignment; about
+ * 20 KB + 4 P^2 B per (set, KV head) and K / V); 256-byte aligned.
  */
 KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache* cache, int32_t n_new);
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new, int32_t n_new,

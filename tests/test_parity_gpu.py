@@ -137,3 +137,19 @@ def test_overflow_flags_device_status():
     assert cache.read_status(clear=True) == kvq.KVQ_DEV_OVERFLOW
     assert int(cache.seq_len[0]) == 30
     assert cache.read_status() == 0
+
+
+def test_identical_patterns_resolve_ties_to_lowest_index():
+    # Every pattern equal: the min-max distances all tie, the pruning bound excludes nothing
+    # (the kernel falls back to evaluating every pattern) and index 0 must win everywhere.
+    w = W["llama3_8b_32k"].with_(B=1, S=96, Hkv=1, Hq=2, P=64)
+    k, v = synth.gen_kv(w)
+    Kf, Vf = synth.to_float(k, w.dtype), synth.to_float(v, w.dtype)
+    MK = np.repeat(Kf[0, :1, 0], 64, axis=0)[None]
+    MV = np.repeat(Vf[0, :1, 0], 64, axis=0)[None]
+    cache = make_cache(w, MK, MV, None, None)
+    cache.append(to_torch(k, w.dtype), to_torch(v, w.dtype))
+    torch.cuda.synchronize()
+    e = encode_unit(w, Kf, Vf, 0, 0, MK, MV, None, None)
+    assert (e.kidx == 0).all() and (e.vidx == 0).all()
+    check_pages(cache, w, e, 0, 0)
