@@ -2,29 +2,32 @@
 // min-max distance, quantize the residual per group and store it in the paged
 // cache ("PatternKV", Section 3.2 and Eq. 6; Eq. 1; granularity of Section 4.1).
 //
-// Launch 0 (prep, per call): for every (set, KV head) and K / V pattern set, bf16
-//   copies of the patterns and their squared norms (for a tensor-core Euclidean
-//   guess), and the table T[j][k] = d_mm(m_j, m_k) of min-max distances between
-//   patterns.
+// Launch 0 (prep, per call): for every (set, KV head) and K / V pattern set, the 16
+//   probe channels (those whose values differ most across the patterns) and every
+//   pattern's values there.
 // Launch 1 (page tasks): one CTA per (touched page, KV head, sequence).
 //   * the new V vectors of the page and, when the page's 32nd token arrives, its 32
 //     K vectors (older ones from the K tail) are staged in shared memory (after the
 //     pre-transform, if enabled);
-//   * a seed pattern per vector from bf16 MMAs (Euclidean nearest, approximate);
-//   * the exact fp32 d_mm of the seed, then exact pruning: d_mm is a seminorm, so
-//     d_mm(x, m_j) >= T[j][s] - d_mm(x, m_s); every j with T[j][s] > 2 d_mm(x, m_s) plus
-//     a rounding margin is strictly farther than the seed and skipped;
-//   * a second exact bound for the survivors: the residual range over 16 channels (those
-//     whose values differ most across the patterns) never exceeds the full range, so a
-//     pattern whose partial range already exceeds the seed's distance is farther too;
-//   * the remaining (vector, pattern) pairs go through a shared work queue; their
-//     exact d_mm values meet in a 64-bit (distance, index) atomic minimum, so the
-//     lowest index wins ties exactly as in the definition;
-//   * residuals, group quantization (fp32; the correctly rounded division decides
-//     wherever it could change a code), packing and stores.
+//   * an exact lower bound of d_mm(y, m_j) for every pattern: max and min only grow
+//     with the channel set, so the residual range over the probe channels never
+//     exceeds the range over all channels (same fp32 subtractions, no rounding of its
+//     own); one lane per vector, every pattern;
+//   * the pattern with the smallest bound is the seed; its exact d_mm is an upper bound
+//     of the minimum, and every pattern whose bound already exceeds it (or equals it
+//     with a higher index) is excluded exactly;
+//   * the few remaining (vector, pattern) pairs go through a shared work queue and are
+//     evaluated exactly, channel block by channel block, stopping as soon as the partial
+//     range rules the pattern out; the exact distances meet in a 64-bit (distance,
+//     index) atomic minimum, so the lowest index wins ties as in the definition;
+//   * residuals, fp32 scale / zero per group, then every 32-bit code word of the page
+//     computed by one thread straight from the residuals (the correctly rounded
+//     division decides wherever the fast quotient could change a code), and stores.
 // Launch 2 (tail + commit): one CTA per sequence writes the keys of the newest,
 //   incomplete group into the K tail and advances seq_len.  Splitting launches 1 and
 //   2 keeps every tail read ahead of every tail write.
+#include <algorithm>
+
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -33,101 +36,52 @@ namespace kvq {
 namespace {
 
 constexpr int kAppendThreads = 128;
-constexpr int kPLd = kD + 32;  // bf16 pattern row in the prep workspace (16-byte aligned rows)
-constexpr int kQueueCap = 1024;
-
+constexpr int kQueueCap = 512;
 constexpr int kProbe = 16;  // channels of the partial-range bound
+constexpr int kLd = kD + 4;  // staged row stride (floats): 16-byte aligned, conflict-free columns
 
 struct AppendWs {
-  __nv_bfloat16* pb;  // [S][H][2][Pp][kPLd] bf16 patterns (0 = K, 1 = V)
-  float* msq;         // [S][H][2][Pp] squared norms
-  float* tab;         // [S][H][2][P][P] d_mm between patterns
-  float* minf;        // [S][H][2] max |m|_inf
-  int32_t* probe;     // [S][H][2][kProbe] channels with the widest spread across patterns
+  int32_t* probe;  // [S][H][2][kProbe] probe channels (0 = K, 1 = V)
+  float* pv;       // [S][H][2][P][kProbe] pattern values at the probe channels
 };
 
 __host__ __device__ inline size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 inline AppendWs carve_append(void* ws, int S, int H, int P) {
-  const int Pp = (P + 7) & ~7;
   uint8_t* p = (uint8_t*)ws;
   AppendWs w;
-  w.pb = (__nv_bfloat16*)p; p += al256((size_t)S * H * 2 * Pp * kPLd * 2);
-  w.msq = (float*)p; p += al256((size_t)S * H * 2 * Pp * 4);
-  w.tab = (float*)p; p += al256((size_t)S * H * 2 * P * P * 4);
-  w.minf = (float*)p; p += al256((size_t)S * H * 2 * 4);
-  w.probe = (int32_t*)p;
+  w.probe = (int32_t*)p; p += al256((size_t)S * H * 2 * kProbe * 4);
+  w.pv = (float*)p;
   return w;
 }
 
-// ---- launch 0: per (set, head, K|V) pattern tables --------------------------------------
-__global__ void append_prep_kernel(Geom g, AppendWs w) {
+// ---- launch 0: probe channels and pattern values there, per (set, head, K|V) ----------
+__global__ void __launch_bounds__(kD) append_prep_kernel(Geom g, AppendWs w) {
   const int sh = blockIdx.x, kv = blockIdx.y;  // sh = set * H + head
-  const int P = g.P, Pp = (P + 7) & ~7;
+  const int P = g.P;
   const float* M = (kv ? g.vpat : g.kpat) + (size_t)sh * P * kD;
   const size_t o = (size_t)sh * 2 + kv;
-  __nv_bfloat16* pb = w.pb + o * Pp * kPLd;
-  for (int i = threadIdx.x; i < Pp * kD; i += blockDim.x) {
-    const int j = i / kD, d = i % kD;
-    pb[j * kPLd + d] = __float2bfloat16_rn(j < P ? M[(size_t)j * kD + d] : 0.f);
-  }
-  float mx = 0.f;
-  for (int j = threadIdx.x; j < Pp; j += blockDim.x) {
-    float acc = 0.f;
-    if (j < P)
-      for (int d = 0; d < kD; ++d) {
-        const float m = M[(size_t)j * kD + d];
-        acc = fmaf(m, m, acc);
-        mx = fmaxf(mx, fabsf(m));
-      }
-    w.msq[o * Pp + j] = acc;
-  }
-  mx = warp_max(mx);
-  __shared__ float wm[32];
-  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = 0.f;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m = fmaxf(m, wm[i]);
-    w.minf[o] = m;
-  }
-  // d_mm(m_j, m_k) for all pairs, from a shared copy of the patterns
-  extern __shared__ __align__(16) float Ms[];  // [P][kD + 4]
-  constexpr int ld = kD + 4;
-  for (int i = threadIdx.x; i < P * kD; i += blockDim.x) Ms[(i / kD) * ld + i % kD] = M[i];
-  __syncthreads();
-  float* tab = w.tab + o * P * P;
-  for (int i = threadIdx.x; i < P * P; i += blockDim.x) {
-    const int j = i / P, k = i % P;
-    const float4* a4 = reinterpret_cast<const float4*>(Ms + j * ld);
-    const float4* b4 = reinterpret_cast<const float4*>(Ms + k * ld);
-    float hi = -INFINITY, lo = INFINITY;
-#pragma unroll 8
-    for (int d = 0; d < kD / 4; ++d) {
-      const float4 x = a4[d], y = b4[d];
-      float r0, r1, r2, r3;
-      sub2(x.x, x.y, y.x, y.y, r0, r1);
-      sub2(x.z, x.w, y.z, y.w, r2, r3);
-      hi = max3(hi, r0, r1);
-      lo = min3(lo, r0, r1);
-      hi = max3(hi, r2, r3);
-      lo = min3(lo, r2, r3);
-    }
-    tab[i] = __fsub_rn(hi, lo);
-  }
-  // probe channels: the kProbe widest spreads (max_j m_jd - min_j m_jd), by rank selection
   __shared__ float spread[kD];
-  for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-    float hi = -INFINITY, lo = INFINITY;
-    for (int j = 0; j < P; ++j) { hi = fmaxf(hi, Ms[j * ld + d]); lo = fminf(lo, Ms[j * ld + d]); }
-    spread[d] = hi - lo;
+  __shared__ int pcs[kProbe];
+  const int d = threadIdx.x;
+  float hi = -INFINITY, lo = INFINITY;
+  for (int j = 0; j < P; ++j) {
+    const float m = M[(size_t)j * kD + d];
+    hi = fmaxf(hi, m);
+    lo = fminf(lo, m);
+  }
+  spread[d] = hi - lo;
+  __syncthreads();
+  // rank of channel d by decreasing spread (ties: lower channel first)
+  int rank = 0;
+  for (int e = 0; e < kD; ++e) rank += (spread[e] > spread[d]) || (spread[e] == spread[d] && e < d);
+  if (rank < kProbe) {
+    w.probe[o * kProbe + rank] = d;
+    pcs[rank] = d;
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-    int rank = 0;
-    for (int e = 0; e < kD; ++e) rank += (spread[e] > spread[d]) || (spread[e] == spread[d] && e < d);
-    if (rank < kProbe) w.probe[o * kProbe + rank] = d;
-  }
+  float* pv = w.pv + o * P * kProbe;
+  for (int i = threadIdx.x; i < P * kProbe; i += blockDim.x) pv[i] = M[(size_t)(i / kProbe) * kD + pcs[i % kProbe]];
 }
 
 struct PageCtx {
@@ -174,23 +128,13 @@ __device__ bool page_context(const Geom& g, int n_new, PageCtx& c) {
   return true;
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Exact partial max / min of y - m over channels [c0, c0 + 64) (y staged, m global).
-__device__ __forceinline__ void dmm_half(const float* __restrict__ y, const float* __restrict__ m, int c0, float& mx,
-                                         float& mn) {
+// Exact partial max / min of y - m over channels [c0, c0 + 32) (y staged, m global).
+__device__ __forceinline__ void range32(const float* __restrict__ y, const float* __restrict__ m, int c0, float& mx,
+                                        float& mn) {
   const float4* y4 = reinterpret_cast<const float4*>(y + c0);
   const float4* m4 = reinterpret_cast<const float4*>(m + c0);
-  mx = -INFINITY;
-  mn = INFINITY;
-#pragma unroll 4
-  for (int c = 0; c < 16; ++c) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
     const float4 a = y4[c], bq = __ldg(m4 + c);
     float r0, r1, r2, r3;
     sub2(a.x, a.y, bq.x, bq.y, r0, r1);
@@ -202,215 +146,245 @@ __device__ __forceinline__ void dmm_half(const float* __restrict__ y, const floa
   }
 }
 
-__device__ __forceinline__ float dmm_full(const float* __restrict__ y, const float* __restrict__ m) {
-  float mx0, mn0, mx1, mn1;
-  dmm_half(y, m, 0, mx0, mn0);
-  dmm_half(y, m, 64, mx1, mn1);
-  return __fsub_rn(fmaxf(mx0, mx1), fminf(mn0, mn1));
+__device__ __forceinline__ unsigned long long dkey(float d, int j) {
+  return ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j;
 }
 
-// Code of one value: q = rne(fl32((R - z) / s)) clamped to [0, maxc].  The quotient comes
-// from a multiply by the correctly rounded reciprocal (error < 3e-6 for quotients below 16)
-// unless it lies within 1e-5 of a rounding boundary, where the correctly rounded division
-// decides.
-__device__ __forceinline__ int quant_code(float R, float z, float s, float rinv, int maxc) {
-  if (s == 0.0f) return 0;
-  const float t = __fsub_rn(R, z);
-  const float u = __fmul_rn(t, rinv);
-  const float f = __fsub_rn(u, floorf(u));
-  float q = rintf(u);
-  if (fabsf(f - 0.5f) < 1e-5f) q = rintf(__fdiv_rn(t, s));
-  return min(max((int)q, 0), maxc);
+// Two codes q = rne(fl32((R - z) / s)) clamped to [0, maxc].  The quotients come from a
+// multiply by the correctly rounded reciprocal (error below 2^-19 for quotients below 16),
+// rounded to an integer by the 1.5 * 2^23 shift; a quotient within 1e-5 of a rounding
+// boundary is recomputed with the correctly rounded division.  s == 0 gives rinv == 0 and
+// code 0.
+__device__ __forceinline__ void code_pair(float R0, float R1, float z0, float z1, float ri0, float ri1,
+                                          const float* s2, int maxc, uint32_t& c0, uint32_t& c1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  float t0, t1, u0, u1, v0, v1, b0, b1, e0, e1;
+  sub2(R0, R1, z0, z1, t0, t1);
+  mul2f(t0, t1, ri0, ri1, u0, u1);
+  add2f(u0, u1, kShift, kShift, v0, v1);
+  sub2(v0, v1, kShift, kShift, b0, b1);
+  sub2(u0, u1, b0, b1, e0, e1);  // u - rne(u), exact
+  int q0 = (int)(__float_as_uint(v0) - 0x4B400000u), q1 = (int)(__float_as_uint(v1) - 0x4B400000u);
+  if (fabsf(e0) > 0.5f - 1e-5f) q0 = (int)rintf(__fdiv_rn(t0, s2[0]));
+  if (fabsf(e1) > 0.5f - 1e-5f) q1 = (int)rintf(__fdiv_rn(t1, s2[1]));
+  c0 = (uint32_t)min(max(q0, 0), maxc);
+  c1 = (uint32_t)min(max(q1, 0), maxc);
 }
 
-// Write the 32-bit code words of one block from a shared code matrix X (row-major, ld = cols).
-// Elements whose token index is below keep_lo keep their old bits.
-__device__ void write_code_block(uint32_t* dst, const uint8_t* X, int ld, int bits, int KS, int keep_lo,
-                                 bool cols_are_tokens) {
-  const int nwords = kG * kD * bits / 32;
-  const int slots = 16 / bits;
-  const uint32_t cmask = (1u << bits) - 1u;
-  for (int wd = threadIdx.x; wd < nwords; wd += blockDim.x) {
-    uint32_t word = 0, keep = 0;
-    for (int odd = 0; odd < 2; ++odd)
-      for (int sl = 0; sl < slots; ++sl) {
-        int row, col;
-        frag_elem(bits, KS, wd, sl, odd, row, col);
-        const int bit = bits * sl + 16 * odd;
-        const int tok = cols_are_tokens ? col : row;
-        if (tok < keep_lo) keep |= cmask << bit;
-        else word |= ((uint32_t)X[row * ld + col] & cmask) << bit;
-      }
-    if (keep) word |= dst[wd] & keep;
-    dst[wd] = word;
+// One 32-bit code word of the V block (rows = channels, 2 column tiles of 16 tokens) from
+// the staged residuals Rv[token][channel] and per-(group, token) s / z / 1/s.  Tokens below
+// keep_lo keep their bits from `old`; tokens at or above tok_hi get code 0.
+template <int BITS>
+__device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const float* vs, const float* vz,
+                                           const float* vr, int keep_lo, int tok_hi, uint32_t old) {
+  constexpr int SPW = 16 / BITS, maxc = (1 << BITS) - 1;
+  const int ln = (wd & 127) >> 2, gq = ln >> 2, tig = ln & 3;
+  const int w = (wd >> 7) * 4 + (wd & 3);
+  uint32_t word = 0;
+#pragma unroll
+  for (int slot = 0; slot < SPW; ++slot) {
+    const int tile = (SPW * w + slot) >> 2, r = slot & 3;
+    const int ch = 16 * (tile >> 1) + 8 * (r & 1) + gq;
+    const int tok = 16 * (tile & 1) + 8 * (r >> 1) + 2 * tig;
+    const int gi = (ch >> 5) * kG + tok;
+    const float2 z = *reinterpret_cast<const float2*>(vz + gi);
+    const float2 ri = *reinterpret_cast<const float2*>(vr + gi);
+    uint32_t c0, c1;
+    code_pair(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi, maxc, c0, c1);
+    const int b0 = BITS * slot, b1 = b0 + 16;
+    word |= (tok < keep_lo ? (old >> b0) & maxc : tok < tok_hi ? c0 : 0u) << b0;
+    word |= (tok + 1 < keep_lo ? (old >> b1) & maxc : tok + 1 < tok_hi ? c1 : 0u) << b1;
   }
+  return word;
 }
 
-__global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, AppendWs wsp,
-                                                                      const uint16_t* __restrict__ k_new,
-                                                                      const uint16_t* __restrict__ v_new,
-                                                                      int n_new) {
+// One 32-bit code word of the K block (rows = tokens, 8 column tiles of 16 channels) from
+// the staged residuals Rk[token][channel] and per-channel s / z / 1/s.
+template <int BITS>
+__device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const float* ks, const float* kz,
+                                           const float* kr) {
+  constexpr int SPW = 16 / BITS, maxc = (1 << BITS) - 1;
+  const int ln = (wd & 127) >> 2, gq = ln >> 2, tig = ln & 3;
+  const int w = (wd >> 7) * 4 + (wd & 3);
+  uint32_t word = 0;
+#pragma unroll
+  for (int slot = 0; slot < SPW; ++slot) {
+    const int tile = (SPW * w + slot) >> 2, r = slot & 3;
+    const int tok = 16 * (tile >> 3) + 8 * (r & 1) + gq;
+    const int ch = 16 * (tile & 7) + 8 * (r >> 1) + 2 * tig;
+    const float2 R = *reinterpret_cast<const float2*>(&Rk[tok][ch]);
+    const float2 z = *reinterpret_cast<const float2*>(kz + ch);
+    const float2 ri = *reinterpret_cast<const float2*>(kr + ch);
+    uint32_t c0, c1;
+    code_pair(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch, maxc, c0, c1);
+    word |= c0 << (BITS * slot);
+    word |= c1 << (BITS * slot + 16);
+  }
+  return word;
+}
+
+// fp32 scale / zero / reciprocal of a group from its min and max
+__device__ __forceinline__ void group_sz(float mn, float mx, int bits, float& s, float& z, float& rinv) {
+  s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << bits) - 1));
+  z = mn;
+  rinv = s != 0.0f ? __frcp_rn(s) : 0.0f;
+}
+
+__global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g, AppendWs wsp,
+                                                                         const uint16_t* __restrict__ k_new,
+                                                                         const uint16_t* __restrict__ v_new,
+                                                                         int n_new) {
   PageCtx c;
   if (!page_context(g, n_new, c)) return;
   const int b = blockIdx.z, h = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int gq = lane >> 2, tig = lane & 3;
-  const int P = g.P, Pp = (P + 7) & ~7;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int P = g.P;
 
   // staged vectors: rows 0..31 = V page slots, rows 32..63 = K page slots
-  constexpr int kLd = kD + 4;
   __shared__ __align__(16) float vec[2 * kG][kLd];
-  __shared__ uint8_t vq[kD][kG];  // V codes, [channel][token]
-  __shared__ uint8_t kq[kG][kD];  // K codes, [token][channel]
-  __shared__ float vs_s[kG][4], vz_s[kG][4], vrow_s[kG], krow_s[kG];
+  __shared__ float vrow_s[kG], krow_s[kG];
   __shared__ unsigned long long best[2 * kG];  // (d_mm bits << 32) | pattern, per row
-  __shared__ float dseed[2 * kG], xinf[2 * kG];
-  __shared__ int seed[2 * kG];
+  __shared__ float dseed[2 * kG], hlb[2][2 * kG];
+  __shared__ int seed[2 * kG], hj[2][2 * kG];
   __shared__ uint32_t queue[kQueueCap];
   __shared__ int qn;
+  // dynamic: lower bounds lb[j][row] during the assignment, then s / z / 1/s tables
+  extern __shared__ __align__(16) float dsm[];
+  float* lbuf = dsm;
+  float* vsz = dsm;            // [3][4][kG]: s, z, 1/s per (group, V slot)
+  float* ksz = dsm + 12 * kG;  // [3][kD]:   s, z, 1/s per K channel
+
   const int lo = c.a - c.pg * kG, hi = c.e - c.pg * kG;  // new slots [lo, hi)
   const size_t shk = ((size_t)c.set * g.H + h) * 2;       // tables: K at shk, V at shk + 1
   auto row_on = [&](int r) { return r < kG ? (r >= lo && r < hi) : c.seal; };
-
-  for (int i = threadIdx.x; i < kD * kG; i += blockDim.x) (&vq[0][0])[i] = 0;
-  if (threadIdx.x < kG) {
-    for (int q = 0; q < 4; ++q) { vs_s[threadIdx.x][q] = 0.f; vz_s[threadIdx.x][q] = 0.f; }
-    vrow_s[threadIdx.x] = 0.f;
-  }
-  if (threadIdx.x == 0) qn = 0;
-
-  // ---- stage (and pre-transform) every vector: warp per row
-  for (int r = warp; r < 2 * kG; r += nwarps) {
-    if (!row_on(r)) continue;
-    const bool isv = r < kG;
-    const int slot = isv ? r : r - kG;
+  auto row_src = [&](int r) -> const uint16_t* {
+    const int slot = r < kG ? r : r - kG;
     const int t = c.pg * kG + slot;
-    const uint16_t* src;
-    if (isv) src = v_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
-    else src = (t < c.L) ? g.k_tail + (((size_t)b * g.H + h) * kG + slot) * kD
-                         : k_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
-    float y[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) y[k] = load_elem(src + lane + 32 * k, g.dtype);
-    float rr = 1.0f;
-    if (g.tx) transform_row_warp(y, isv ? c.cV : c.cK, rr, lane);
-    float am = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      vec[r][lane + 32 * k] = y[k];
-      am = fmaxf(am, fabsf(y[k]));
-    }
-    am = warp_max(am);
-    if (lane == 0) {
-      xinf[r] = am;
-      if (isv) vrow_s[slot] = rr;
-      else krow_s[slot] = rr;
-    }
-  }
-  __syncthreads();
+    if (r < kG) return v_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
+    return (t < c.L) ? g.k_tail + (((size_t)b * g.H + h) * kG + slot) * kD
+                     : k_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
+  };
+  if (tid == 0) qn = 0;
 
-  // ---- seed: Euclidean nearest pattern from bf16 MMAs; warp w owns rows 16w .. 16w+15.
-  // The MMA k index runs over channels 8(4kp + tig) + e so every lane's operands of a
-  // pair of k-steps are 8 consecutive channels (a dot product does not depend on k order).
-  {
-    const int r0 = 16 * warp;
-    bool active = false;
-    for (int r = r0; r < r0 + 16; ++r) active |= row_on(r);
-    if (active) {
-      const size_t o = shk + (r0 < kG ? 1 : 0);
-      const __nv_bfloat16* pb = wsp.pb + o * Pp * kPLd;
-      const float* msq = wsp.msq + o * Pp;
-      uint32_t A[2][4][4];
+  // ---- stage (and pre-transform) every vector
+  if (!g.tx) {
+    // 16 threads per row, 8 channels (one 16-byte load) each; all loads issued first
+    uint4 raw[8];
 #pragma unroll
-      for (int rh = 0; rh < 2; ++rh)
+    for (int u = 0; u < 8; ++u) {
+      const int r = (tid >> 4) + 8 * u;
+      if (row_on(r)) raw[u] = __ldg(reinterpret_cast<const uint4*>(row_src(r) + 8 * (tid & 15)));
+    }
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          const float4* p = reinterpret_cast<const float4*>(&vec[r0 + 8 * rh + gq][8 * (4 * kp + tig)]);
-          const float4 u = p[0], v = p[1];
-          A[rh][kp][0] = __byte_perm(__float_as_uint(u.x), __float_as_uint(u.y), 0x7632);
-          A[rh][kp][1] = __byte_perm(__float_as_uint(u.z), __float_as_uint(u.w), 0x7632);
-          A[rh][kp][2] = __byte_perm(__float_as_uint(v.x), __float_as_uint(v.y), 0x7632);
-          A[rh][kp][3] = __byte_perm(__float_as_uint(v.z), __float_as_uint(v.w), 0x7632);
-        }
-      float bmin[2] = {INFINITY, INFINITY};
-      int bj[2] = {0, 0};
-      for (int nt = 0; nt < Pp / 8; ++nt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const __nv_bfloat16* brow = pb + (size_t)(8 * nt + gq) * kPLd + 8 * tig;
+    for (int u = 0; u < 8; ++u) {
+      const int r = (tid >> 4) + 8 * u;
+      if (!row_on(r)) continue;
+      const uint32_t wv[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      float f[8];
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          const uint4 bv = __ldg(reinterpret_cast<const uint4*>(brow + 32 * kp));
-          mma_bf16(acc, A[0][kp][0], A[1][kp][0], A[0][kp][1], A[1][kp][1], bv.x, bv.y);
-          mma_bf16(acc, A[0][kp][2], A[1][kp][2], A[0][kp][3], A[1][kp][3], bv.z, bv.w);
-        }
-        const int j0 = 8 * nt + 2 * tig;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int j = j0 + (q & 1), rh = q >> 1;
-          const float e = msq[j] - 2.0f * acc[q];
-          if (j < P && e < bmin[rh]) { bmin[rh] = e; bj[rh] = j; }
-        }
+      for (int k = 0; k < 4; ++k) {
+        f[2 * k] = bits_to_float((uint16_t)(wv[k] & 0xffffu), g.dtype);
+        f[2 * k + 1] = bits_to_float((uint16_t)(wv[k] >> 16), g.dtype);
       }
+      float4* dst = reinterpret_cast<float4*>(&vec[r][8 * (tid & 15)]);
+      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  } else {
+    // warp per row: Hadamard rotation and the fitted column / row normalisation
+    for (int r = warp; r < 2 * kG; r += nwarps) {
+      if (!row_on(r)) continue;
+      const bool isv = r < kG;
+      const uint16_t* src = row_src(r);
+      float y[4];
 #pragma unroll
-      for (int rh = 0; rh < 2; ++rh) {
+      for (int k = 0; k < 4; ++k) y[k] = load_elem(src + lane + 32 * k, g.dtype);
+      float rr = 1.0f;
+      transform_row_warp(y, isv ? c.cV : c.cK, rr, lane);
 #pragma unroll
-        for (int m = 1; m <= 2; m <<= 1) {
-          const float ob = __shfl_xor_sync(kFull, bmin[rh], m);
-          const int oj = __shfl_xor_sync(kFull, bj[rh], m);
-          if (ob < bmin[rh] || (ob == bmin[rh] && oj < bj[rh])) { bmin[rh] = ob; bj[rh] = oj; }
-        }
-        if (tig == 0) seed[r0 + 8 * rh + gq] = bj[rh];
+      for (int k = 0; k < 4; ++k) vec[r][lane + 32 * k] = y[k];
+      if (lane == 0) {
+        if (isv) vrow_s[r] = rr;
+        else krow_s[r - kG] = rr;
       }
     }
   }
   __syncthreads();
 
-  // ---- exact d_mm of the seed: two threads per row (channel halves)
+  // ---- probe-channel lower bounds: warp (kind = warp & 1: 0 V, 1 K; half = warp >> 1),
+  // lane = row; patterns split in two halves.  Running argmin per half (ties: lowest j).
+  const int P0 = (P + 1) >> 1;
   {
-    const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const bool on = row_on(r);
-    float mx = -INFINITY, mn = INFINITY;
-    if (on) dmm_half(vec[r], (r < kG ? c.MV : c.MK) + (size_t)seed[r] * kD, 64 * half, mx, mn);
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-    mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
-    if (on && half == 0) {
-      const float d = __fsub_rn(mx, mn);
-      dseed[r] = d;
-      best[r] = ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)seed[r];
-    }
-  }
-  __syncthreads();
-
-  // ---- exact pruning: queue every pattern neither bound can exclude
-  {
-    const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
-    if (row_on(r)) {
-      const size_t o = shk + (r < kG ? 1 : 0);
-      const int s = seed[r];
-      const float ds = dseed[r];
-      const float* trow = wsp.tab + o * P * P + (size_t)s * P;
-      const float thr = 2.0f * ds + 0x1p-19f * (xinf[r] + wsp.minf[o]);
-      const float* M = r < kG ? c.MV : c.MK;
-      int pc[kProbe];
+    const int kind = warp & 1, half = warp >> 1;
+    const int r = kind * kG + lane;
+    if (kind == 0 || c.seal) {
+      const size_t o = shk + (kind ? 0 : 1);
+      const int32_t* pc = wsp.probe + o * kProbe;
+      const float* pvt = wsp.pv + o * P * kProbe;
       float py[kProbe];
 #pragma unroll
-      for (int u = 0; u < kProbe; ++u) {
-        pc[u] = __ldg(wsp.probe + o * kProbe + u);
-        py[u] = vec[r][pc[u]];
-      }
-      for (int j = half; j < P; j += 2) {
-        if (j == s || __ldg(trow + j) > thr) continue;
-        // residual range over the probe channels: a lower bound of d_mm(x, m_j), exactly
-        const float* m = M + (size_t)j * kD;
-        float hi = -INFINITY, lo = INFINITY;
+      for (int u = 0; u < kProbe; ++u) py[u] = vec[r][__ldg(pc + u)];
+      float blb = INFINITY;
+      int bj = half ? P0 : 0;
+      const int j1 = half ? P : P0;
+      for (int j = half ? P0 : 0; j < j1; ++j) {
+        const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * kProbe);
+        float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int u = 0; u < kProbe; ++u) {
-          const float rr = __fsub_rn(py[u], __ldg(m + pc[u]));
-          hi = fmaxf(hi, rr);
-          lo = fminf(lo, rr);
+        for (int q = 0; q < kProbe / 4; ++q) {
+          const float4 m = __ldg(m4 + q);
+          float r0, r1, r2, r3;
+          sub2(py[4 * q], py[4 * q + 1], m.x, m.y, r0, r1);
+          sub2(py[4 * q + 2], py[4 * q + 3], m.z, m.w, r2, r3);
+          mx = max3(mx, r0, r1);
+          mn = min3(mn, r0, r1);
+          mx = max3(mx, r2, r3);
+          mn = min3(mn, r2, r3);
         }
-        const float lb = __fsub_rn(hi, lo);
-        if (lb > ds || (lb == ds && j > s)) continue;
+        const float lb = __fsub_rn(mx, mn);
+        lbuf[j * (2 * kG) + r] = lb;
+        if (lb < blb) { blb = lb; bj = j; }
+      }
+      hlb[half][r] = blb;
+      hj[half][r] = bj;
+    }
+  }
+  __syncthreads();
+
+  // ---- seed = smallest bound; its exact d_mm, two threads per row (channel halves)
+  {
+    const int r = tid >> 1, hh = tid & 1;
+    const bool on = row_on(r);
+    int s = 0;
+    float mx = -INFINITY, mn = INFINITY;
+    if (on) {
+      s = hlb[1][r] < hlb[0][r] ? hj[1][r] : hj[0][r];
+      s = min(max(s, 0), P - 1);
+      const float* m = (r < kG ? c.MV : c.MK) + (size_t)s * kD;
+      range32(vec[r], m, 64 * hh, mx, mn);
+      range32(vec[r], m, 64 * hh + 32, mx, mn);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+    if (on && hh == 0) {
+      const float d = __fsub_rn(mx, mn);
+      dseed[r] = d;
+      seed[r] = s;
+      best[r] = dkey(d, s);
+    }
+  }
+  __syncthreads();
+
+  // ---- survivors: patterns whose bound does not exclude them
+  {
+    const int r = tid & (2 * kG - 1), hh = tid >> 6;
+    if (row_on(r)) {
+      const int s = seed[r];
+      const float ds = dseed[r];
+      const int j1 = hh ? P : P0;
+      for (int j = hh ? P0 : 0; j < j1; ++j) {
+        const float lb = lbuf[j * (2 * kG) + r];
+        if (j == s || lb > ds || (lb == ds && j > s)) continue;
         const int pos = atomicAdd(&qn, 1);
         if (pos < kQueueCap) queue[pos] = ((uint32_t)r << 16) | (uint32_t)j;
       }
@@ -418,22 +392,34 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, Ap
   }
   __syncthreads();
 
-  // ---- exact d_mm of the candidates; (distance, index) minimum per row
+  // ---- exact d_mm of the survivors, 32-channel blocks, stopping once a block's partial
+  // range excludes the pattern; (distance, index) minimum per row
   if (qn <= kQueueCap) {
-    for (int i = threadIdx.x; i < qn; i += blockDim.x) {
+    for (int i = tid; i < qn; i += blockDim.x) {
       const uint32_t e = queue[i];
       const int r = e >> 16, j = e & 0xffff;
-      const float d = dmm_full(vec[r], (r < kG ? c.MV : c.MK) + (size_t)j * kD);
-      atomicMin(&best[r], ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j);
+      const float* m = (r < kG ? c.MV : c.MK) + (size_t)j * kD;
+      const float ds = dseed[r];
+      const int s = seed[r];
+      float mx = -INFINITY, mn = INFINITY, d = 0.f;
+      bool out = false;
+#pragma unroll 1
+      for (int cb = 0; cb < kD; cb += 32) {
+        range32(vec[r], m, cb, mx, mn);
+        d = __fsub_rn(mx, mn);
+        if (d > ds || (d == ds && j > s)) { out = true; break; }
+      }
+      if (!out) atomicMin(&best[r], dkey(d, j));
     }
   } else {
     // the bound excluded too little: every pattern for every row, two threads per row
-    const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int r = tid >> 1, hh = tid & 1;
     if (row_on(r)) {
       const float* M = r < kG ? c.MV : c.MK;
-      for (int j = half; j < P; j += 2) {
-        const float d = dmm_full(vec[r], M + (size_t)j * kD);
-        atomicMin(&best[r], ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j);
+      for (int j = hh; j < P; j += 2) {
+        float mx = -INFINITY, mn = INFINITY;
+        for (int cb = 0; cb < kD; cb += 32) range32(vec[r], M + (size_t)j * kD, cb, mx, mn);
+        atomicMin(&best[r], dkey(__fsub_rn(mx, mn), j));
       }
     }
   }
@@ -443,75 +429,100 @@ __global__ void __launch_bounds__(kAppendThreads) append_pages_kernel(Geom g, Ap
   for (int r = warp; r < 2 * kG; r += nwarps) {
     if (!row_on(r)) continue;
     const float* m = (r < kG ? c.MV : c.MK) + (size_t)(best[r] & 0xffffffffu) * kD;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) vec[r][lane + 32 * k] = __fsub_rn(vec[r][lane + 32 * k], __ldg(m + lane + 32 * k));
+    float4* y4 = reinterpret_cast<float4*>(&vec[r][4 * lane]);
+    const float4 a = *y4, mv = __ldg(reinterpret_cast<const float4*>(m) + lane);
+    float4 o;
+    sub2(a.x, a.y, mv.x, mv.y, o.x, o.y);
+    sub2(a.z, a.w, mv.z, mv.w, o.z, o.w);
+    *y4 = o;
   }
   __syncthreads();
 
-  // ---- V: per-token group quantization, warp per token
-  for (int slot = lo + warp; slot < hi; slot += nwarps) {
+  // ---- scale / zero: V per (token, group of 32 channels), K per channel over the page
+  {
+    const int q = tid >> 5, slot = tid & 31;  // V: group q, token slot (conflict-free rows)
+    float s = 0.f, z = 0.f, ri = 0.f;
+    if (slot >= lo && slot < hi) {
+      const float4* p = reinterpret_cast<const float4*>(&vec[slot][32 * q]);
+      float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float R = vec[slot][lane + 32 * k];
-      const float mn = warp_min(R), mx = warp_max(R);
-      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << g.bits) - 1));
-      const float rinv = s != 0.0f ? __frcp_rn(s) : 0.0f;
-      vq[lane + 32 * k][slot] = (uint8_t)quant_code(R, mn, s, rinv, (1 << g.bits) - 1);
-      if (lane == 0) { vs_s[slot][k] = s; vz_s[slot][k] = mn; }
+      for (int k = 0; k < 8; ++k) {
+        const float4 v = p[k];
+        mx = max3(mx, v.x, v.y);
+        mn = min3(mn, v.x, v.y);
+        mx = max3(mx, v.z, v.w);
+        mn = min3(mn, v.z, v.w);
+      }
+      group_sz(mn, mx, g.bits, s, z, ri);
     }
+    vsz[(0 * 4 + q) * kG + slot] = s;
+    vsz[(1 * 4 + q) * kG + slot] = z;
+    vsz[(2 * 4 + q) * kG + slot] = ri;
   }
-
-  // ---- K: per-channel quantization over the 32 tokens of the sealed group
   float* ks_g = reinterpret_cast<float*>(c.sub + g.off_ks);
   float* kz_g = reinterpret_cast<float*>(c.sub + g.off_kz);
   if (c.seal) {
-    for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-      float R[kG];
-      float mn = INFINITY, mx = -INFINITY;
+    for (int d = tid; d < kD; d += blockDim.x) {
+      float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-      for (int t = 0; t < kG; ++t) {
-        R[t] = vec[kG + t][d];
-        mn = fminf(mn, R[t]);
-        mx = fmaxf(mx, R[t]);
+      for (int t = 0; t < kG; t += 2) {
+        mx = max3(mx, vec[kG + t][d], vec[kG + t + 1][d]);
+        mn = min3(mn, vec[kG + t][d], vec[kG + t + 1][d]);
       }
-      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << g.bits) - 1));
-      const float rinv = s != 0.0f ? __frcp_rn(s) : 0.0f;
-#pragma unroll
-      for (int t = 0; t < kG; ++t) kq[t][d] = (uint8_t)quant_code(R[t], mn, s, rinv, (1 << g.bits) - 1);
+      float s, z, ri;
+      group_sz(mn, mx, g.bits, s, z, ri);
+      ksz[0 * kD + d] = s;
+      ksz[1 * kD + d] = z;
+      ksz[2 * kD + d] = ri;
       ks_g[ksc_pos(d)] = s;
-      kz_g[ksc_pos(d)] = mn;
+      kz_g[ksc_pos(d)] = z;
     }
   }
   __syncthreads();
 
-  // ---- stores
-  write_code_block(reinterpret_cast<uint32_t*>(c.sub + g.off_vc), &vq[0][0], kG, g.bits, 2, c.fresh ? 0 : lo, true);
+  // ---- code words, one thread per 32-bit word; scales, zeros, indices
+  {
+    uint32_t* vdst = reinterpret_cast<uint32_t*>(c.sub + g.off_vc);
+    const int nwords = kG * kD * g.bits / 32;
+    const int keep_lo = c.fresh ? 0 : lo;
+    const float(*Rv)[kLd] = vec;
+    const float(*Rk)[kLd] = vec + kG;
+    for (int wd = tid; wd < nwords; wd += blockDim.x) {
+      const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;
+      vdst[wd] = g.bits == 2 ? v_word<2>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old)
+                             : v_word<4>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old);
+    }
+    if (c.seal) {
+      uint32_t* kdst = reinterpret_cast<uint32_t*>(c.sub);
+      for (int wd = tid; wd < nwords; wd += blockDim.x)
+        kdst[wd] = g.bits == 2 ? k_word<2>(wd, Rk, ksz, ksz + kD, ksz + 2 * kD)
+                               : k_word<4>(wd, Rk, ksz, ksz + kD, ksz + 2 * kD);
+    }
+  }
   float* vs_g = reinterpret_cast<float*>(c.sub + g.off_vs);
   float* vz_g = reinterpret_cast<float*>(c.sub + g.off_vz);
   uint8_t* vidx_g = c.sub + g.off_vidx;
   float* vrow_g = reinterpret_cast<float*>(c.sub + g.off_vrow);
-  for (int i = threadIdx.x; i < kG * 4; i += blockDim.x) {
-    const int slot = i >> 2, q = i & 3;
+  {
+    const int slot = tid >> 2, q = tid & 3;
     if (c.fresh || (slot >= lo && slot < hi)) {
-      vs_g[vsc_pos(slot, q)] = vs_s[slot][q];
-      vz_g[vzc_pos(slot, q)] = vz_s[slot][q];
+      vs_g[vsc_pos(slot, q)] = vsz[(0 * 4 + q) * kG + slot];
+      vz_g[vzc_pos(slot, q)] = vsz[(1 * 4 + q) * kG + slot];
     }
   }
-  for (int slot = threadIdx.x; slot < kG; slot += blockDim.x) {
+  if (tid < kG) {
+    const int slot = tid;
     const bool present = slot >= lo && slot < hi;
     if (c.fresh || present) {
       vidx_g[tok_pos(slot)] = present ? (uint8_t)(best[slot] & 0xff) : (uint8_t)0;
-      if (g.tx) vrow_g[tok_pos(slot)] = vrow_s[slot];
+      if (g.tx) vrow_g[tok_pos(slot)] = present ? vrow_s[slot] : 0.f;
     }
   }
-  if (c.seal) {
-    write_code_block(reinterpret_cast<uint32_t*>(c.sub), &kq[0][0], kD, g.bits, 8, 0, false);
+  if (c.seal && tid < kG) {
     uint8_t* kidx_g = c.sub + g.off_kidx;
     float* krow_g = reinterpret_cast<float*>(c.sub + g.off_krow);
-    for (int slot = threadIdx.x; slot < kG; slot += blockDim.x) {
-      kidx_g[tok_pos(slot)] = (uint8_t)(best[kG + slot] & 0xff);
-      if (g.tx) krow_g[tok_pos(slot)] = krow_s[slot];
-    }
+    kidx_g[tok_pos(tid)] = (uint8_t)(best[kG + tid] & 0xff);
+    if (g.tx) krow_g[tok_pos(tid)] = krow_s[tid];
   }
 }
 
@@ -535,23 +546,22 @@ __global__ void append_tail_kernel(Geom g, const uint16_t* __restrict__ k_new, i
 }  // namespace
 
 size_t append_workspace(const Geom& g) {
-  const int Pp = (g.P + 7) & ~7;
-  return al256((size_t)g.S * g.H * 2 * Pp * kPLd * 2) + al256((size_t)g.S * g.H * 2 * Pp * 4) +
-         al256((size_t)g.S * g.H * 2 * g.P * g.P * 4) + al256((size_t)g.S * g.H * 2 * 4) +
-         al256((size_t)g.S * g.H * 2 * kProbe * 4) + 256;
+  return al256((size_t)g.S * g.H * 2 * kProbe * 4) + al256((size_t)g.S * g.H * 2 * g.P * kProbe * 4) + 256;
 }
 
 cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, int n_new, void* ws, cudaStream_t st) {
   if (n_new <= 0 || g.B == 0) return cudaSuccess;
   AppendWs w = carve_append(ws, g.S, g.H, g.P);
-  const size_t prep_smem = (size_t)g.P * (kD + 4) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(append_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem);
+  append_prep_kernel<<<dim3(g.S * g.H, 2), kD, 0, st>>>(g, w);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  append_prep_kernel<<<dim3(g.S * g.H, 2), 256, prep_smem, st>>>(g, w);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // lower bounds [P][64 rows], later reused for the s / z tables (12 kG + 3 kD floats)
+  const size_t dyn = std::max<size_t>((size_t)g.P * 2 * kG, 12 * kG + 3 * kD) * sizeof(float);
+  if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
+      cudaSuccess)
+    return e;
   dim3 grid(n_new / kG + 2, g.H, g.B);
-  append_pages_kernel<<<grid, kAppendThreads, 0, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new, n_new);
+  append_pages_kernel<<<grid, kAppendThreads, dyn, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new, n_new);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_tail_kernel<<<g.B, 256, 0, st>>>(g, (const uint16_t*)k_new, n_new);

@@ -22,8 +22,6 @@ constexpr int kReduceChunk = 4096;
 struct MineWs {
   double* sums;     // [NP][P][128]
   uint32_t* cnt;    // [NP][P]
-  uint32_t* cursor; // [NP][P]  slots handed out per cluster by the counting sort
-  int32_t* order;   // [NP][n]  token indices grouped by cluster
   int32_t* assign;  // [NP][n]
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
@@ -40,8 +38,6 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   MineWs w{};
   w.sums = (double*)p; p += align256((size_t)NP * P * kD * sizeof(double));
   w.cnt = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
-  w.cursor = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
-  w.order = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t));
   if (assign_out) w.assign = assign_out;
   else { w.assign = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t)); }
   if (transform) {
@@ -192,17 +188,22 @@ __global__ void __launch_bounds__(128) mine_assign_kernel(Src s, int P, const fl
 
 // ---- tensor-core assignment with exact certification ------------------------------
 //
-// Scores e_j = |m_j|^2 - 2 x.m_j come from bf16 m16n8k16 MMAs: every pattern is split
-// exactly into three bf16 terms (8+8+8 bits), inputs are exact in bf16 (bf16 input) or
-// split into two bf16 terms (fp16 input exactly; fp32 pre-transformed rows to 2^-16).
-// With E_j a bound on |e_hat_j - e_j| and U = min_j (e_hat_j + E_j), the float64
-// argmin can only be a pattern with e_hat_j - E_j <= U + delta.  A token whose best two
-// scores are more than 2 max_j E_j + delta apart is decided at once; the others (1-2 %)
-// are decided by recomputing float64 distances of the candidates exactly as the
-// sequential reference does.  E_j = 2^-12 |x| |m_j| + 2^-20 (|x|^2 + |m_j|^2) covers fp32
-// accumulation in the tensor cores with margin: 24 chained MMAs of exact bf16 products
-// stay below 2^-18 |x| |m_j| with one correctly rounded fp32 sum per MMA, and below
-// 2^-13.4 |x| |m_j| even if each MMA truncated its 16-term sum to 22 bits.
+// Scores e_j = |m_j|^2 - 2 x.m_j come from bf16 m16n8k16 MMAs.  Every pattern value is
+// split into bf16 terms hi + mid (the remainder below them is at most 2^-16 |m|); inputs
+// are exact in one bf16 term (bf16 input) or split into hi + lo (fp16 input exactly,
+// fp32 pre-transformed rows to 2^-16).  Each product of terms (x_a, m_b) runs in its own
+// fp32 accumulator chain of 8 MMAs (x_lo . m_mid, below 2^-16 |x| |m|, is left out), and
+// the chains are added at the end.  If a tensor core truncated each MMA's sum to 22 bits
+// of its largest term, a chain would be off by at most 8 * 17 * 2^-22 |x_a| |m_b|; with
+// the terms left out and the final adds, |e_hat_j - e_j| stays below 2^-12.6 |x| |m_j|
+// plus the fp32 rounding of |m_j|^2 and of the final combination, which
+// E_j = 2^-12 |x| |m_j| + 2^-20 (|x|^2 + |m_j|^2) covers.
+//
+// With U = min_j (e_hat_j + E_j), the float64 argmin can only be a pattern with
+// e_hat_j - E_j <= U + delta.  A token whose best two scores are more than 2 max_j E_j +
+// delta apart is decided at once; the others (well under 1 %) are decided by
+// recomputing float64 distances of the candidates exactly as the sequential reference
+// does.
 //
 // The MMA k index runs over channels in the order pi(kp, tig, e) = 8 (4 kp + tig) + e for
 // k-step 2 kp + (e >> 2) ... so that every lane's A operands of a pair of k-steps are 8
@@ -228,13 +229,17 @@ __device__ __forceinline__ void split_trunc(float x0, float x1, uint32_t& hi, ui
   lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
 }
 
+// Smallest score, its pattern and the second smallest score.  A thread sees its patterns
+// in increasing order, so a strict comparison keeps the lowest index among equal scores.
 struct Top2 {
   float m1, m2;
   int j1;
 };
 __device__ __forceinline__ void top2_add(Top2& t, float e, int j) {
-  if (e < t.m1 || (e == t.m1 && j < t.j1)) { t.m2 = t.m1; t.m1 = e; t.j1 = j; }
-  else if (e < t.m2) t.m2 = e;
+  const bool lt = e < t.m1;
+  t.m2 = lt ? t.m1 : fminf(t.m2, e);
+  t.j1 = lt ? j : t.j1;
+  t.m1 = lt ? e : t.m1;
 }
 __device__ __forceinline__ void top2_merge_xor(Top2& t, int mask) {
   const float om1 = __shfl_xor_sync(kFull, t.m1, mask), om2 = __shfl_xor_sync(kFull, t.m2, mask);
@@ -244,39 +249,93 @@ __device__ __forceinline__ void top2_merge_xor(Top2& t, int mask) {
   else t.m2 = fminf(om1, lo2);
 }
 
-// 8 consecutive input values of row i starting at channel c (bf16 input: one 16-byte load).
-template <int NA>
-__device__ __forceinline__ void load8(const Src& s, int prob, int64_t i, int c, float (&v)[8]) {
-  if (s.y) {
-    const float4* p = reinterpret_cast<const float4*>(s.y + ((size_t)prob * s.n + i) * kD + c);
-    const float4 a = p[0], b = p[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  } else {
-    const int set = prob / s.heads, h = prob % s.heads;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(s.x + set * s.ss + i * s.ts + h * s.hs + c));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Input kinds: 0 = bf16 rows (one exact bf16 term), 1 = fp16 rows, 2 = fp32 pre-transformed rows.
+// A warp tile's raw row data (8 consecutive channels per load) is fetched one tile ahead.
+template <int KIND>
+struct RawRows {
+  static constexpr int kMt = KIND == 0 ? 2 : 1;
+  static constexpr int kW = KIND == 2 ? 2 : 1;  // 16-byte words per 8 channels
+  uint4 u[kMt][2][4][kW];
+};
+
+template <int KIND>
+__device__ __forceinline__ void load_raw(const Src& s, int prob, int64_t t0, int gq, int tig, RawRows<KIND>& R) {
+  constexpr int kMt = RawRows<KIND>::kMt;
+  const int set = prob / s.heads, h = prob % s.heads;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[2 * k] = bits_to_float((uint16_t)(w[k] & 0xffff), s.dtype);
-      v[2 * k + 1] = bits_to_float((uint16_t)(w[k] >> 16), s.dtype);
+  for (int mt = 0; mt < kMt; ++mt)
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+      const int64_t i = t0 + 16 * mt + 8 * rh + gq;
+#pragma unroll
+      for (int kp = 0; kp < 4; ++kp) {
+        const int c = 8 * (4 * kp + tig);
+        if (i < s.n) {
+          if constexpr (KIND == 2) {
+            const uint4* p = reinterpret_cast<const uint4*>(s.y + ((size_t)prob * s.n + i) * kD + c);
+            R.u[mt][rh][kp][0] = p[0];
+            R.u[mt][rh][kp][1] = p[1];
+          } else {
+            R.u[mt][rh][kp][0] = __ldg(reinterpret_cast<const uint4*>(s.x + set * s.ss + i * s.ts + h * s.hs + c));
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < RawRows<KIND>::kW; ++k) R.u[mt][rh][kp][k] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+}
+
+// MMA operand words (bf16 pairs, lower channel in the low half) of 8 raw values, and the
+// sum of their squares.
+template <int KIND>
+__device__ __forceinline__ void to_operands(const uint4 (&raw)[RawRows<KIND>::kW], uint32_t (&hi)[4],
+                                            uint32_t (&lo)[4], float& nrm) {
+  if constexpr (KIND == 2) {
+    const float v[8] = {__uint_as_float(raw[0].x), __uint_as_float(raw[0].y), __uint_as_float(raw[0].z),
+                        __uint_as_float(raw[0].w), __uint_as_float(raw[1].x), __uint_as_float(raw[1].y),
+                        __uint_as_float(raw[1].z), __uint_as_float(raw[1].w)};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      split_trunc(v[2 * q], v[2 * q + 1], hi[q], lo[q]);
+      nrm = fmaf(v[2 * q], v[2 * q], nrm);
+      nrm = fmaf(v[2 * q + 1], v[2 * q + 1], nrm);
+    }
+  } else {
+    const uint32_t w[4] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float v0, v1;
+      if constexpr (KIND == 0) {
+        hi[q] = w[q];
+        v0 = __uint_as_float(w[q] << 16);
+        v1 = __uint_as_float(w[q] & 0xFFFF0000u);
+      } else {
+        v0 = __half2float(__ushort_as_half((uint16_t)(w[q] & 0xffff)));
+        v1 = __half2float(__ushort_as_half((uint16_t)(w[q] >> 16)));
+        split_trunc(v0, v1, hi[q], lo[q]);
+      }
+      nrm = fmaf(v0, v0, nrm);
+      nrm = fmaf(v1, v1, nrm);
     }
   }
 }
 
-// NA = number of bf16 terms of the input (1: exact bf16 input; 2: fp16 or fp32 input).
-template <int NA>
+template <int KIND>
 __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src s, int P, const float* __restrict__ M,
                                                                              int32_t* __restrict__ assign) {
-  constexpr int kMt = NA == 1 ? 2 : 1;  // 16-token m-tiles per warp tile
-  constexpr int kTok = 16 * kMt;        // tokens per warp tile
+  constexpr int NA = KIND == 0 ? 1 : 2;  // bf16 terms of an input value
+  constexpr int NC = NA + 1;             // accumulator chains: (hi,hi), (hi,mid), (lo,hi)
+  constexpr int kMt = NA == 1 ? 2 : 1;   // 16-token m-tiles per warp tile
+  constexpr int kTok = 16 * kMt;         // tokens per warp tile
   extern __shared__ __align__(16) uint8_t smraw[];
   uint8_t* sm = smraw;
   const int prob = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, tig = lane & 3;
   const int Pp = (P + 7) & ~7;  // padded to whole n-tiles
-  __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(sm);                       // [3][Pp][kBLd]
-  float* mnorm = reinterpret_cast<float*>(sm + (size_t)3 * Pp * kBLd * 2);           // [Pp] |m_j|
+  __nv_bfloat16* Bs = reinterpret_cast<__nv_bfloat16*>(sm);                       // [2][Pp][kBLd]
+  float* mnorm = reinterpret_cast<float*>(sm + (size_t)2 * Pp * kBLd * 2);           // [Pp] |m_j|
   float* msq = mnorm + Pp;                                                            // [Pp] |m_j|^2
   const int eld = Pp + 2;                                                             // even: aligned float2 rows
   float* escr = msq + Pp;                                                             // [warps][kTok][eld]
@@ -289,12 +348,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src 
     const int j = i / kD, d = i % kD;
     const float m = j < P ? Mp[(size_t)j * kD + d] : 0.f;
     const __nv_bfloat16 h = __float2bfloat16_rn(m);
-    const float r1 = m - __bfloat162float(h);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
     Bs[(0 * Pp + j) * kBLd + d] = h;
-    Bs[(1 * Pp + j) * kBLd + d] = mid;
-    Bs[(2 * Pp + j) * kBLd + d] = lo;
+    Bs[(1 * Pp + j) * kBLd + d] = __float2bfloat16_rn(m - __bfloat162float(h));
   }
   if (threadIdx.x == 0) { gmax[0] = 0.f; gmax[1] = 0.f; }
   __syncthreads();
@@ -313,38 +368,26 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src 
   float* esc = escr + warp * kTok * eld;
   float* xnw = xn + warp * kTok;
   const int64_t ntiles = (s.n + kTok - 1) / kTok;
-  for (int64_t tile = (int64_t)blockIdx.x * kMmaWarps + warp; tile < ntiles; tile += (int64_t)gridDim.x * kMmaWarps) {
+  const int64_t tstep = (int64_t)gridDim.x * kMmaWarps;
+  int64_t tile = (int64_t)blockIdx.x * kMmaWarps + warp;
+  RawRows<KIND> raw;
+  if (tile < ntiles) load_raw<KIND>(s, prob, tile * kTok, gq, tig, raw);
+  for (; tile < ntiles; tile += tstep) {
     const int64_t t0 = tile * kTok;
     // A operands: rows gq (+8) of each m-tile, channels 8(4kp + tig) .. +7 for k-step pair kp
-    uint32_t A[NA][kMt][2][4][4];  // [term][mt][row half][kp][reg]: reg 0,1 = k-step 2kp (b0 half, b1 half)...
+    uint32_t A[NA][kMt][2][4][4];  // [term][mt][row half][kp][reg]
     float nrm[kMt][2];
 #pragma unroll
     for (int mt = 0; mt < kMt; ++mt)
 #pragma unroll
       for (int rh = 0; rh < 2; ++rh) {
-        const int64_t i = t0 + 16 * mt + 8 * rh + gq;
-        const bool ok = i < s.n;
         nrm[mt][rh] = 0.f;
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          float v[8];
-          if (ok) load8<NA>(s, prob, i, 8 * (4 * kp + tig), v);
-          else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = 0.f;
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) nrm[mt][rh] = fmaf(v[u], v[u], nrm[mt][rh]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if constexpr (NA == 1) {
-              A[0][mt][rh][kp][q] = __byte_perm(__float_as_uint(v[2 * q]), __float_as_uint(v[2 * q + 1]), 0x7632);
-            } else {
-              split_trunc(v[2 * q], v[2 * q + 1], A[0][mt][rh][kp][q], A[NA - 1][mt][rh][kp][q]);
-            }
-          }
-        }
+        for (int kp = 0; kp < 4; ++kp)
+          to_operands<KIND>(raw.u[mt][rh][kp], A[0][mt][rh][kp], A[NA - 1][mt][rh][kp], nrm[mt][rh]);
       }
+    // the next tile's rows are in flight while this one is scored
+    if (tile + tstep < ntiles) load_raw<KIND>(s, prob, (tile + tstep) * kTok, gq, tig, raw);
 #pragma unroll
     for (int mt = 0; mt < kMt; ++mt)
 #pragma unroll
@@ -359,35 +402,47 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src 
 #pragma unroll
     for (int mt = 0; mt < kMt; ++mt)
 #pragma unroll
-      for (int rh = 0; rh < 2; ++rh) top[mt][rh] = Top2{INFINITY, INFINITY, 0x7fffffff};
+      for (int rh = 0; rh < 2; ++rh) top[mt][rh] = Top2{INFINITY, INFINITY, 0};
     // scores, one n-tile (8 patterns) at a time
     for (int nt = 0; nt < Pp / 8; ++nt) {
-      float acc[kMt][4];
+      float acc[NC][kMt][4];
 #pragma unroll
-      for (int mt = 0; mt < kMt; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      for (int ch = 0; ch < NC; ++ch)
 #pragma unroll
-      for (int sp = 0; sp < 3; ++sp) {
+        for (int mt = 0; mt < kMt; ++mt) acc[ch][mt][0] = acc[ch][mt][1] = acc[ch][mt][2] = acc[ch][mt][3] = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < 2; ++sp) {
         const __nv_bfloat16* brow = Bs + ((size_t)sp * Pp + 8 * nt + gq) * kBLd + 8 * tig;
 #pragma unroll
         for (int kp = 0; kp < 4; ++kp) {
           const uint4 bv = *reinterpret_cast<const uint4*>(brow + 32 * kp);  // channels 8(4kp+tig)..+7
 #pragma unroll
-          for (int a = 0; a < NA; ++a)
+          for (int a = 0; a < NA; ++a) {
+            if (a == 1 && sp == 1) continue;  // x_lo . m_mid: left out
+            const int ch = a == 0 ? sp : 2;
 #pragma unroll
             for (int mt = 0; mt < kMt; ++mt) {
               // k-step 2kp: channels +0..+3 -> (a0a1, a4a5) / (b0, b1); rows gq and gq+8 -> a0a1 / a2a3
-              mma_bf16(acc[mt], A[a][mt][0][kp][0], A[a][mt][1][kp][0], A[a][mt][0][kp][1], A[a][mt][1][kp][1], bv.x,
-                       bv.y);
-              mma_bf16(acc[mt], A[a][mt][0][kp][2], A[a][mt][1][kp][2], A[a][mt][0][kp][3], A[a][mt][1][kp][3], bv.z,
-                       bv.w);
+              mma_bf16(acc[ch][mt], A[a][mt][0][kp][0], A[a][mt][1][kp][0], A[a][mt][0][kp][1], A[a][mt][1][kp][1],
+                       bv.x, bv.y);
+              mma_bf16(acc[ch][mt], A[a][mt][0][kp][2], A[a][mt][1][kp][2], A[a][mt][0][kp][3], A[a][mt][1][kp][3],
+                       bv.z, bv.w);
             }
+          }
         }
       }
 #pragma unroll
       for (int mt = 0; mt < kMt; ++mt) {
+        float dot[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float v = acc[0][mt][q] + acc[1][mt][q];
+          if constexpr (NC == 3) v += acc[2][mt][q];
+          dot[q] = v;
+        }
         const int j0 = 8 * nt + 2 * tig;
-        const float e0 = msq[j0] - 2.0f * acc[mt][0], e1 = msq[j0 + 1] - 2.0f * acc[mt][1];
-        const float e2 = msq[j0] - 2.0f * acc[mt][2], e3 = msq[j0 + 1] - 2.0f * acc[mt][3];
+        const float e0 = msq[j0] - 2.0f * dot[0], e1 = msq[j0 + 1] - 2.0f * dot[1];
+        const float e2 = msq[j0] - 2.0f * dot[2], e3 = msq[j0 + 1] - 2.0f * dot[3];
         *reinterpret_cast<float2*>(&esc[(16 * mt + gq) * eld + j0]) = make_float2(e0, e1);
         *reinterpret_cast<float2*>(&esc[(16 * mt + gq + 8) * eld + j0]) = make_float2(e2, e3);
         if (j0 < P) { top2_add(top[mt][0], e0, j0); top2_add(top[mt][1], e2, j0); }
@@ -434,7 +489,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src 
 #pragma unroll 8
             for (int d = 0; d < kD; d += 4) {
               float xv[4];
-              if (s.y) {
+              if constexpr (KIND == 2) {
                 const float4 t4 = *reinterpret_cast<const float4*>(s.y + ((size_t)prob * s.n + i) * kD + d);
                 xv[0] = t4.x; xv[1] = t4.y; xv[2] = t4.z; xv[3] = t4.w;
               } else {
@@ -462,164 +517,199 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 2) mine_assign_mma_kernel(Src 
   }
 }
 
-size_t mine_mma_smem(int P, int NA) {
-  const int Pp = (P + 7) & ~7, kTok = NA == 1 ? 32 : 16;
-  return (size_t)3 * Pp * kBLd * 2 + 2 * Pp * 4 + (size_t)kMmaWarps * kTok * (Pp + 2) * 4 + kMmaWarps * kTok * 4 + 16;
+size_t mine_mma_smem(int P, int KIND) {
+  const int Pp = (P + 7) & ~7, kTok = KIND == 0 ? 32 : 16;
+  return (size_t)2 * Pp * kBLd * 2 + 2 * Pp * 4 + (size_t)kMmaWarps * kTok * (Pp + 2) * 4 + kMmaWarps * kTok * 4 + 16;
 }
 
-// Per-cluster float64 sums by counting sort: (1) cluster sizes, (2) every token's index
-// written into its cluster's bucket (slots handed out by an atomic cursor, so the order
-// inside a bucket varies), (3) each warp sums a run of consecutive bucket entries in
-// registers and adds the run's partial sums to the cluster total once per cluster it
-// crosses.  float64 sums of fp16 / bf16 values are exact, so the order of the additions
-// does not change them.
-__global__ void __launch_bounds__(256) mine_count_kernel(int64_t n, int P, const int32_t* __restrict__ assign,
-                                                         uint32_t* __restrict__ cnt) {
-  extern __shared__ uint32_t hist[];
-  const int prob = blockIdx.y;
-  for (int j = threadIdx.x; j < P; j += blockDim.x) hist[j] = 0;
-  __syncthreads();
-  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk, i1 = min(n, i0 + kReduceChunk);
-  const int32_t* a = assign + (size_t)prob * n;
-  for (int64_t i = i0 + threadIdx.x; i < i1; i += blockDim.x) atomicAdd(&hist[a[i]], 1u);
-  __syncthreads();
-  for (int j = threadIdx.x; j < P; j += blockDim.x)
-    if (hist[j]) atomicAdd(cnt + (size_t)prob * P + j, hist[j]);
+// Per-cluster float64 sums and sizes in one streaming pass.  A CTA walks a contiguous run
+// of 128-token tiles of one problem (and one channel slice), staged into shared memory by a
+// cp.async ring.  Warp w owns clusters w, w + 16, w + 32, ...; for each tile it finds the
+// members of each of its clusters with ballots over the tile's assignments and adds their
+// rows into float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1 of
+// the slice).  Each CTA adds its totals to global memory once at the end.  float64 sums of
+// fp16 / bf16 values are exact, so the order of the additions does not change them.
+constexpr int kAccWarps = 16;
+constexpr int kAccT = 128;  // tokens per tile
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
 }
-
-// exclusive prefix of the cluster sizes into base[0..P] (base[P] = n), one thread
-__device__ __forceinline__ void cluster_base(const uint32_t* c, int P, uint32_t* base) {
-  uint32_t s = 0;
-  for (int j = 0; j < P; ++j) { base[j] = s; s += c[j]; }
-  base[P] = s;
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-constexpr int kScatterPer = kReduceChunk / 256;
-
-__global__ void __launch_bounds__(256) mine_scatter_kernel(int64_t n, int P, const int32_t* __restrict__ assign,
-                                                           const uint32_t* __restrict__ cnt,
-                                                           uint32_t* __restrict__ cursor, int32_t* __restrict__ order) {
-  extern __shared__ uint32_t sm[];
-  uint32_t* base = sm;         // [P + 1]
-  uint32_t* lc = sm + P + 1;   // [P] this CTA's tokens per cluster, then its first slot
-  const int prob = blockIdx.y;
-  if (threadIdx.x == 0) cluster_base(cnt + (size_t)prob * P, P, base);
-  for (int j = threadIdx.x; j < P; j += blockDim.x) lc[j] = 0;
-  __syncthreads();
-  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk;
-  const int32_t* a = assign + (size_t)prob * n;
-  int jj[kScatterPer];
-  uint32_t rk[kScatterPer];
-#pragma unroll
-  for (int u = 0; u < kScatterPer; ++u) {
-    const int64_t i = i0 + u * 256 + threadIdx.x;
-    jj[u] = i < n ? a[i] : -1;
-    if (jj[u] >= 0) rk[u] = atomicAdd(&lc[jj[u]], 1u);
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < P; j += blockDim.x)
-    if (lc[j]) lc[j] = base[j] + atomicAdd(cursor + (size_t)prob * P + j, lc[j]);
-  __syncthreads();
-  int32_t* o = order + (size_t)prob * n;
-#pragma unroll
-  for (int u = 0; u < kScatterPer; ++u)
-    if (jj[u] >= 0) o[lc[jj[u]] + rk[u]] = (int32_t)(i0 + u * 256 + threadIdx.x);
-}
-
-constexpr int kSegRun = 256;  // bucket entries per warp
-constexpr int kSegUnroll = 8;
-
-__device__ __forceinline__ void flush4(double* dst, double a0, double a1, double a2, double a3) {
-  if (a0 != 0.0) atomicAdd(dst + 0, a0);
-  if (a1 != 0.0) atomicAdd(dst + 1, a1);
-  if (a2 != 0.0) atomicAdd(dst + 2, a2);
-  if (a3 != 0.0) atomicAdd(dst + 3, a3);
-}
-
-// lane l holds channels 4l..4l+3 of the token rows it sums
-__global__ void __launch_bounds__(256, 3) mine_segsum_kernel(Src s, int P, const int32_t* __restrict__ order,
-                                                          const uint32_t* __restrict__ cnt,
-                                                          double* __restrict__ sums) {
-  extern __shared__ uint32_t base[];  // [P + 1]
-  const int prob = blockIdx.y;
-  if (threadIdx.x == 0) cluster_base(cnt + (size_t)prob * P, P, base);
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t r0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kSegRun;
-  if (r0 >= s.n) return;
-  const int64_t r1 = min(s.n, r0 + kSegRun);
-  const int32_t* o = order + (size_t)prob * s.n;
+// CPW clusters per warp, E channels per lane (slice = 32 E channels), ES bytes per element
+// (2: the fp16 / bf16 input, 4: the fp32 pre-transformed rows)
+template <int CPW, int E, int ES>
+__global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, int P, const int32_t* __restrict__ assign,
+                                                                      double* __restrict__ sums,
+                                                                      uint32_t* __restrict__ cnt) {
+  constexpr int CW = 32 * E, RB = CW * ES;          // channels and bytes of a staged row
+  constexpr int kStages = ES == 2 ? 4 : 3;
+  constexpr int kStageBytes = kAccT * RB + kAccT * 4;
+  extern __shared__ __align__(16) uint8_t smraw[];
+  const int slice = blockIdx.y, prob = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
+  const int64_t per = (ntiles + gridDim.x - 1) / gridDim.x;
+  const int64_t k0 = (int64_t)blockIdx.x * per, k1 = min(ntiles, k0 + per);
+  if (k0 >= k1) return;
+  const int nt = (int)(k1 - k0);
   const int set = prob / s.heads, h = prob % s.heads;
-  const uint16_t* xb = s.x + set * s.ss + h * s.hs + 4 * lane;
-  const float* yb = s.y ? s.y + (size_t)prob * s.n * kD + 4 * lane : nullptr;
-  double* gs = sums + (size_t)prob * P * kD + 4 * lane;
-  // cluster of entry r0: the last j with base[j] <= r0 (skipping empty clusters)
-  int j = 0;
-  {
-    int lo = 0, hi = P - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (base[mid] <= (uint32_t)r0) lo = mid; else hi = mid - 1;
+  const int32_t* a = assign + (size_t)prob * s.n;
+
+  auto issue = [&](int k) {  // tile k0 + k into its stage
+    if (k < nt) {
+      uint8_t* st = smraw + (size_t)(k % kStages) * kStageBytes;
+      int32_t* sa = reinterpret_cast<int32_t*>(st + kAccT * RB);
+      const int64_t tb = (k0 + k) * kAccT;
+      constexpr int kChunks = RB / 16;
+      for (int i = threadIdx.x; i < kAccT * kChunks; i += blockDim.x) {
+        const int t = i / kChunks, cix = i % kChunks;
+        if (tb + t < s.n) {
+          const uint8_t* src =
+              ES == 2 ? reinterpret_cast<const uint8_t*>(s.x + set * s.ss + h * s.hs + (tb + t) * s.ts + slice * CW)
+                      : reinterpret_cast<const uint8_t*>(s.y + ((size_t)prob * s.n + tb + t) * kD + slice * CW);
+          cp_async16(st + t * RB + cix * 16, src + cix * 16);
+        }
+      }
+      for (int t = threadIdx.x; t < kAccT; t += blockDim.x) {
+        if (tb + t < s.n) cp_async4(sa + t, a + tb + t);
+        else sa[t] = -1;
+      }
     }
-    j = lo;
-  }
-  uint32_t jend = base[j + 1];
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int64_t r = r0; r < r1; r += 32) {
-    const int tok_l = r + lane < r1 ? o[r + lane] : 0;
-    const int m = (int)(r1 - r < 32 ? r1 - r : 32);
-    for (int u0 = 0; u0 < m; u0 += kSegUnroll) {
-      float v[kSegUnroll][4];
+    cp_async_commit();
+  };
+
+  double acc[CPW][E];
+  uint32_t members[CPW];
 #pragma unroll
-      for (int u = 0; u < kSegUnroll; ++u) {
-        const int t = __shfl_sync(0xffffffffu, tok_l, (u0 + u) & 31);
-        if (u0 + u < m) {
-          if (yb) {
-            const float4 f = *reinterpret_cast<const float4*>(yb + (size_t)t * kD);
-            v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+  for (int c = 0; c < CPW; ++c) {
+    members[c] = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[c][e] = 0.0;
+  }
+
+#pragma unroll
+  for (int k = 0; k < kStages - 1; ++k) issue(k);
+  for (int k = 0; k < nt; ++k) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();  // tile k visible to all; every warp is done with tile k - 1
+    issue(k + kStages - 1);
+    const uint8_t* st = smraw + (size_t)(k % kStages) * kStageBytes;
+    const int32_t* sa = reinterpret_cast<const int32_t*>(st + kAccT * RB);
+    int aj[kAccT / 32];
+#pragma unroll
+    for (int q = 0; q < kAccT / 32; ++q) aj[q] = sa[32 * q + lane];
+#pragma unroll
+    for (int c = 0; c < CPW; ++c) {
+      const int j = warp + kAccWarps * c;
+      if (j >= P) break;
+#pragma unroll
+      for (int q = 0; q < kAccT / 32; ++q) {
+        uint32_t m = __ballot_sync(0xffffffffu, aj[q] == j);
+        members[c] += __popc(m);
+        while (m) {
+          const int t = 32 * q + __ffs(m) - 1;
+          m &= m - 1;
+          const uint8_t* row = st + t * RB + lane * (E * ES);
+          float v[E];
+          if constexpr (ES == 4) {
+            if constexpr (E == 4) { const float4 f = *reinterpret_cast<const float4*>(row); v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w; }
+            else if constexpr (E == 2) { const float2 f = *reinterpret_cast<const float2*>(row); v[0] = f.x; v[1] = f.y; }
+            else v[0] = *reinterpret_cast<const float*>(row);
           } else {
-            const uint2 b = __ldg(reinterpret_cast<const uint2*>(xb + (size_t)t * s.ts));
-            v[u][0] = bits_to_float((uint16_t)(b.x & 0xffffu), s.dtype);
-            v[u][1] = bits_to_float((uint16_t)(b.x >> 16), s.dtype);
-            v[u][2] = bits_to_float((uint16_t)(b.y & 0xffffu), s.dtype);
-            v[u][3] = bits_to_float((uint16_t)(b.y >> 16), s.dtype);
+            if constexpr (E == 4) {
+              const uint2 b = *reinterpret_cast<const uint2*>(row);
+              v[0] = bits_to_float((uint16_t)(b.x & 0xffffu), s.dtype);
+              v[1] = bits_to_float((uint16_t)(b.x >> 16), s.dtype);
+              v[2] = bits_to_float((uint16_t)(b.y & 0xffffu), s.dtype);
+              v[3] = bits_to_float((uint16_t)(b.y >> 16), s.dtype);
+            } else if constexpr (E == 2) {
+              const uint32_t b = *reinterpret_cast<const uint32_t*>(row);
+              v[0] = bits_to_float((uint16_t)(b & 0xffffu), s.dtype);
+              v[1] = bits_to_float((uint16_t)(b >> 16), s.dtype);
+            } else {
+              v[0] = bits_to_float(*reinterpret_cast<const uint16_t*>(row), s.dtype);
+            }
           }
-        }
-      }
 #pragma unroll
-      for (int u = 0; u < kSegUnroll; ++u) {
-        if (u0 + u >= m) break;
-        const uint32_t rr = (uint32_t)(r + u0 + u);
-        if (rr >= jend) {  // crossed into a later cluster (warp-uniform)
-          flush4(gs + (size_t)j * kD, acc[0], acc[1], acc[2], acc[3]);
-          acc[0] = acc[1] = acc[2] = acc[3] = 0.0;
-          do { ++j; } while (base[j + 1] <= rr);
-          jend = base[j + 1];
+          for (int e = 0; e < E; ++e) acc[c][e] += (double)v[e];
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] += (double)v[u][e];
       }
     }
   }
-  flush4(gs + (size_t)j * kD, acc[0], acc[1], acc[2], acc[3]);
+  cp_async_wait<0>();
+
+  double* gs = sums + (size_t)prob * P * kD + slice * CW + lane * E;
+#pragma unroll
+  for (int c = 0; c < CPW; ++c) {
+    const int j = warp + kAccWarps * c;
+    if (j >= P) break;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (acc[c][e] != 0.0) atomicAdd(gs + (size_t)j * kD + e, acc[c][e]);
+    if (slice == 0 && lane == 0 && members[c]) atomicAdd(cnt + (size_t)prob * P + j, members[c]);
+  }
 }
 
-__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt, uint32_t* cursor) {
+template <int CPW, int E, int ES>
+constexpr size_t accum_smem() {
+  return (size_t)(ES == 2 ? 4 : 3) * (kAccT * 32 * E * ES + kAccT * 4);
+}
+
+template <int CPW, int E, int ES>
+cudaError_t launch_accum_t(const Src& s, int P, int NP, int sms, const int32_t* assign, double* sums, uint32_t* cnt,
+                           cudaStream_t st) {
+  constexpr size_t smem = accum_smem<CPW, E, ES>();
+  cudaError_t e = cudaFuncSetAttribute(mine_accum_kernel<CPW, E, ES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int slices = 4 / E;
+  const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
+  const int64_t want = std::max<int64_t>(1, sms / std::max(1, slices * NP));
+  const unsigned chunks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, want));
+  mine_accum_kernel<CPW, E, ES><<<dim3(chunks, slices, NP), kAccWarps * 32, smem, st>>>(s, P, assign, sums, cnt);
+  return cudaGetLastError();
+}
+
+// P <= 64: one 128-channel slice, 4 clusters per warp; P <= 128: two 64-channel slices, 8
+// clusters per warp; P <= 256: four 32-channel slices, 16 clusters per warp
+cudaError_t launch_accum(const Src& s, int P, int NP, int sms, const int32_t* assign, double* sums, uint32_t* cnt,
+                         cudaStream_t st) {
+  const bool f32 = s.y != nullptr;
+  if (P <= 4 * kAccWarps)
+    return f32 ? launch_accum_t<4, 4, 4>(s, P, NP, sms, assign, sums, cnt, st)
+               : launch_accum_t<4, 4, 2>(s, P, NP, sms, assign, sums, cnt, st);
+  if (P <= 8 * kAccWarps)
+    return f32 ? launch_accum_t<8, 2, 4>(s, P, NP, sms, assign, sums, cnt, st)
+               : launch_accum_t<8, 2, 2>(s, P, NP, sms, assign, sums, cnt, st);
+  return f32 ? launch_accum_t<16, 1, 4>(s, P, NP, sms, assign, sums, cnt, st)
+             : launch_accum_t<16, 1, 2>(s, P, NP, sms, assign, sums, cnt, st);
+}
+
+__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt) {
   const int prob = blockIdx.y, j = blockIdx.x, d = threadIdx.x;
   const size_t pj = (size_t)prob * P + j;
   uint32_t c = cnt[pj];
   if (c > 0) M[pj * kD + d] = (float)(sums[pj * kD + d] / (double)c);
   sums[pj * kD + d] = 0.0;
   __syncthreads();
-  if (d == 0) { cnt[pj] = 0; cursor[pj] = 0; }
+  if (d == 0) cnt[pj] = 0;
 }
 
 }  // namespace
 
 size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
   size_t NP = (size_t)sets * heads;
-  size_t b = align256(NP * P * kD * sizeof(double)) + 2 * align256(NP * P * sizeof(uint32_t)) +
-             2 * align256(NP * (size_t)n * sizeof(int32_t));
+  size_t b = align256(NP * P * kD * sizeof(double)) + align256(NP * P * sizeof(uint32_t)) +
+             align256(NP * (size_t)n * sizeof(int32_t));
   if (transform)
     b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
          4 * align256(NP * kD * sizeof(double));
@@ -654,40 +744,38 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   mine_init_kernel<<<dim3(a.P, NP), kD, 0, st>>>(s, a.P, a.patterns);
   cudaMemsetAsync(w.sums, 0, (size_t)NP * a.P * kD * sizeof(double), st);
   cudaMemsetAsync(w.cnt, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
-  cudaMemsetAsync(w.cursor, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
   size_t smem_assign = (size_t)a.P * kD * sizeof(float);
   if ((e = cudaFuncSetAttribute(mine_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_assign)) != cudaSuccess)
     return e;
-  const int NA = (a.transform || a.dtype == KVQ_F16) ? 2 : 1;
+  const int KIND = a.transform ? 2 : (a.dtype == KVQ_F16 ? 1 : 0);
   const bool use_mma = a.P <= kMmaMaxP;
-  const size_t smem_mma = mine_mma_smem(a.P, NA);
+  const size_t smem_mma = mine_mma_smem(a.P, KIND);
   if (use_mma) {
-    if (NA == 1) e = cudaFuncSetAttribute(mine_assign_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_mma);
+    if (KIND == 0) e = cudaFuncSetAttribute(mine_assign_mma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_mma);
+    else if (KIND == 1) e = cudaFuncSetAttribute(mine_assign_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_mma);
     else e = cudaFuncSetAttribute(mine_assign_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_mma);
     if (e != cudaSuccess) return e;
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tok_per_cta = kMmaWarps * (NA == 1 ? 32 : 16);
+  const int tok_per_cta = kMmaWarps * (KIND == 0 ? 32 : 16);
   const unsigned mma_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + tok_per_cta - 1) / tok_per_cta, (int64_t)(2 * sms + NP - 1) / NP));
-  const unsigned seg_ctas = (unsigned)((a.n + 8 * kSegRun - 1) / (8 * kSegRun));
   for (int it = 0; it < a.iters; ++it) {
-    if (use_mma && NA == 1)
-      mine_assign_mma_kernel<1><<<dim3(mma_ctas, NP), kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
+    const dim3 ag(mma_ctas, NP);
+    if (use_mma && KIND == 0)
+      mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
+    else if (use_mma && KIND == 1)
+      mine_assign_mma_kernel<1><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else if (use_mma)
-      mine_assign_mma_kernel<2><<<dim3(mma_ctas, NP), kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
+      mine_assign_mma_kernel<2><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else
       mine_assign_kernel<<<dim3((unsigned)((a.n + 127) / 128), NP), 128, smem_assign, st>>>(s, a.P, a.patterns,
                                                                                            w.assign);
-    mine_count_kernel<<<dim3(chunks, NP), 256, a.P * sizeof(uint32_t), st>>>(a.n, a.P, w.assign, w.cnt);
-    mine_scatter_kernel<<<dim3(chunks, NP), 256, (2 * a.P + 1) * sizeof(uint32_t), st>>>(a.n, a.P, w.assign, w.cnt,
-                                                                                         w.cursor, w.order);
-    mine_segsum_kernel<<<dim3(seg_ctas, NP), 256, (a.P + 1) * sizeof(uint32_t), st>>>(s, a.P, w.order, w.cnt,
-                                                                                       w.sums);
-    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt, w.cursor);
+    if ((e = launch_accum(s, a.P, NP, sms, w.assign, w.sums, w.cnt, st)) != cudaSuccess) return e;
+    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
   }
   return cudaGetLastError();
 }
