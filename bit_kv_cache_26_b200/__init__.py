@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libkvq.so not found at {LIB_PATH}; build it with `python -m bit_kv_cache_26_b200.build`")
+    raise ImportError(f"libkvq.so not found at {LIB_PATH}; build it with `python bit_kv_cache_26_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA, KVQ_ERR_DEVICE = range(7)

@@ -1,6 +1,6 @@
 """Build libkvq.so in-tree: every .cu under csrc/ compiled for sm_100a and linked into one shared library.
 
-    python -m bit_kv_cache_26_b200.build [--force] [--verbose]
+    python bit_kv_cache_26_b200/build.py [--force] [--verbose]
 """
 from __future__ import annotations
 

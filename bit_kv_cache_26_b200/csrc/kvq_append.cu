@@ -150,13 +150,14 @@ __device__ __forceinline__ unsigned long long dkey(float d, int j) {
   return ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j;
 }
 
-// Two codes q = rne(fl32((R - z) / s)) clamped to [0, maxc].  The quotients come from a
-// multiply by the correctly rounded reciprocal (error below 2^-19 for quotients below 16),
-// rounded to an integer by the 1.5 * 2^23 shift; a quotient within 1e-5 of a rounding
-// boundary is recomputed with the correctly rounded division.  s == 0 gives rinv == 0 and
-// code 0.
-__device__ __forceinline__ void code_pair(float R0, float R1, float z0, float z1, float ri0, float ri1,
-                                          const float* s2, int maxc, uint32_t& c0, uint32_t& c1) {
+// Two codes q = rne(fl32((R - z) / s)), returned as (q0 | q1 << 16).  The quotients come
+// from a multiply by the correctly rounded reciprocal (error below 2^-19 for quotients below
+// 16), rounded to an integer by adding 1.5 * 2^23 (the integer is then the low mantissa
+// bits); a quotient within 1e-5 of a rounding boundary is recomputed with the correctly
+// rounded division.  R >= z and the quotient stays below maxc + 2^-19, so no clamp is
+// needed; s == 0 gives rinv == 0 and code 0.
+__device__ __forceinline__ uint32_t code_pair(float R0, float R1, float z0, float z1, float ri0, float ri1,
+                                              const float* s2) {
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   float t0, t1, u0, u1, v0, v1, b0, b1, e0, e1;
   sub2(R0, R1, z0, z1, t0, t1);
@@ -164,11 +165,11 @@ __device__ __forceinline__ void code_pair(float R0, float R1, float z0, float z1
   add2f(u0, u1, kShift, kShift, v0, v1);
   sub2(v0, v1, kShift, kShift, b0, b1);
   sub2(u0, u1, b0, b1, e0, e1);  // u - rne(u), exact
-  int q0 = (int)(__float_as_uint(v0) - 0x4B400000u), q1 = (int)(__float_as_uint(v1) - 0x4B400000u);
-  if (fabsf(e0) > 0.5f - 1e-5f) q0 = (int)rintf(__fdiv_rn(t0, s2[0]));
-  if (fabsf(e1) > 0.5f - 1e-5f) q1 = (int)rintf(__fdiv_rn(t1, s2[1]));
-  c0 = (uint32_t)min(max(q0, 0), maxc);
-  c1 = (uint32_t)min(max(q1, 0), maxc);
+  if (fmaxf(fabsf(e0), fabsf(e1)) > 0.5f - 1e-5f) {
+    if (fabsf(e0) > 0.5f - 1e-5f) v0 = __fadd_rn(rintf(__fdiv_rn(t0, s2[0])), kShift);
+    if (fabsf(e1) > 0.5f - 1e-5f) v1 = __fadd_rn(rintf(__fdiv_rn(t1, s2[1])), kShift);
+  }
+  return __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410) & 0x00FF00FFu;
 }
 
 // One 32-bit code word of the V block (rows = channels, 2 column tiles of 16 tokens) from
@@ -189,9 +190,9 @@ __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const
     const int gi = (ch >> 5) * kG + tok;
     const float2 z = *reinterpret_cast<const float2*>(vz + gi);
     const float2 ri = *reinterpret_cast<const float2*>(vr + gi);
-    uint32_t c0, c1;
-    code_pair(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi, maxc, c0, c1);
+    const uint32_t c01 = code_pair(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi);
     const int b0 = BITS * slot, b1 = b0 + 16;
+    const uint32_t c0 = c01 & 0xffu, c1 = c01 >> 16;
     word |= (tok < keep_lo ? (old >> b0) & maxc : tok < tok_hi ? c0 : 0u) << b0;
     word |= (tok + 1 < keep_lo ? (old >> b1) & maxc : tok + 1 < tok_hi ? c1 : 0u) << b1;
   }
@@ -203,7 +204,7 @@ __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const
 template <int BITS>
 __device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const float* ks, const float* kz,
                                            const float* kr) {
-  constexpr int SPW = 16 / BITS, maxc = (1 << BITS) - 1;
+  constexpr int SPW = 16 / BITS;
   const int ln = (wd & 127) >> 2, gq = ln >> 2, tig = ln & 3;
   const int w = (wd >> 7) * 4 + (wd & 3);
   uint32_t word = 0;
@@ -215,10 +216,7 @@ __device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const
     const float2 R = *reinterpret_cast<const float2*>(&Rk[tok][ch]);
     const float2 z = *reinterpret_cast<const float2*>(kz + ch);
     const float2 ri = *reinterpret_cast<const float2*>(kr + ch);
-    uint32_t c0, c1;
-    code_pair(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch, maxc, c0, c1);
-    word |= c0 << (BITS * slot);
-    word |= c1 << (BITS * slot + 16);
+    word |= code_pair(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch) << (BITS * slot);
   }
   return word;
 }
@@ -403,11 +401,15 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       const int s = seed[r];
       float mx = -INFINITY, mn = INFINITY, d = 0.f;
       bool out = false;
-#pragma unroll 1
-      for (int cb = 0; cb < kD; cb += 32) {
-        range32(vec[r], m, cb, mx, mn);
+      range32(vec[r], m, 0, mx, mn);  // both 32-channel blocks' loads in flight together
+      range32(vec[r], m, 32, mx, mn);
+      d = __fsub_rn(mx, mn);
+      out = d > ds || (d == ds && j > s);
+      if (!out) {
+        range32(vec[r], m, 64, mx, mn);
+        range32(vec[r], m, 96, mx, mn);
         d = __fsub_rn(mx, mn);
-        if (d > ds || (d == ds && j > s)) { out = true; break; }
+        out = d > ds || (d == ds && j > s);
       }
       if (!out) atomicMin(&best[r], dkey(d, j));
     }
@@ -425,16 +427,31 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   }
   __syncthreads();
 
-  // ---- residuals in place: R = y - M[k*], warp per row
-  for (int r = warp; r < 2 * kG; r += nwarps) {
-    if (!row_on(r)) continue;
-    const float* m = (r < kG ? c.MV : c.MK) + (size_t)(best[r] & 0xffffffffu) * kD;
-    float4* y4 = reinterpret_cast<float4*>(&vec[r][4 * lane]);
-    const float4 a = *y4, mv = __ldg(reinterpret_cast<const float4*>(m) + lane);
-    float4 o;
-    sub2(a.x, a.y, mv.x, mv.y, o.x, o.y);
-    sub2(a.z, a.w, mv.z, mv.w, o.z, o.w);
-    *y4 = o;
+  // ---- residuals in place: R = y - M[k*], warp per row, pattern loads issued 8 rows at a time
+  {
+    constexpr int kRows = 2 * kG / (kAppendThreads / 32), kBatch = 8;
+#pragma unroll
+    for (int u0 = 0; u0 < kRows; u0 += kBatch) {
+      float4 mv[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int r = warp + (u0 + u) * nwarps;
+        if (row_on(r))
+          mv[u] = __ldg(reinterpret_cast<const float4*>((r < kG ? c.MV : c.MK) + (size_t)(best[r] & 0xffffffffu) * kD) +
+                        lane);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int r = warp + (u0 + u) * nwarps;
+        if (!row_on(r)) continue;
+        float4* y4 = reinterpret_cast<float4*>(&vec[r][4 * lane]);
+        const float4 a = *y4;
+        float4 o;
+        sub2(a.x, a.y, mv[u].x, mv[u].y, o.x, o.y);
+        sub2(a.z, a.w, mv[u].z, mv[u].w, o.z, o.w);
+        *y4 = o;
+      }
+    }
   }
   __syncthreads();
 
@@ -488,7 +505,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const float(*Rv)[kLd] = vec;
     const float(*Rk)[kLd] = vec + kG;
     for (int wd = tid; wd < nwords; wd += blockDim.x) {
-      const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;
+      const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;  // tokens already in the page keep their codes
       vdst[wd] = g.bits == 2 ? v_word<2>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old)
                              : v_word<4>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old);
     }
