@@ -24,6 +24,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA, KVQ_ERR_DEVICE = range(7)
+KVQ_DECODE_STATIC_SCRATCH_BYTES = 16 << 20  # size of the fixed scratch of kvq_decode_attention_static
 KVQ_DEV_BAD_PAGE, KVQ_DEV_OVERFLOW, KVQ_DEV_BAD_SET, KVQ_DEV_TIMEOUT, KVQ_DEV_RANGE = 0x1, 0x2, 0x4, 0x8, 0x10
 KVQ_F16, KVQ_BF16 = 0, 1
 KVQ_TX_NONE, KVQ_TX_HADAMARD_VARNORM = 0, 1
@@ -61,6 +62,7 @@ _SIGS = {
     "kvq_quantize_append": (ctypes.c_int, [_P, _vp, _vp, _i32, _vp, _sz, _vp]),
     "kvq_decode_workspace_bytes": (_sz, [_P, _i32]),
     "kvq_decode_attention": (ctypes.c_int, [_P, _vp, _i32, _f32, _vp, _vp, _sz, _vp]),
+    "kvq_decode_attention_static": (ctypes.c_int, [_P, _vp, _i32, _f32, _vp, _vp]),
     "kvq_dequantize": (ctypes.c_int, [_P, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "kvq_read_status": (ctypes.c_int, [_P, ctypes.POINTER(_i32), _i32, _vp]),
     "kvq_last_error": (ctypes.c_char_p, []),
@@ -138,6 +140,13 @@ def kvq_decode_attention(cache: kvq_cache, q: torch.Tensor, num_q_heads: int, sm
                          ws: torch.Tensor, stream=None) -> None:
     _check(_lib.kvq_decode_attention(ctypes.byref(cache), _ptr(q), num_q_heads, sm_scale, _ptr(out), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvq_decode_attention_static(cache: kvq_cache, q: torch.Tensor, num_q_heads: int, sm_scale: float,
+                                out: torch.Tensor, stream=None) -> None:
+    """kvq_decode_attention with its partials in the library's fixed device array (no workspace)."""
+    _check(_lib.kvq_decode_attention_static(ctypes.byref(cache), _ptr(q), num_q_heads, sm_scale, _ptr(out),
+                                            _stream(stream)))
 
 
 def kvq_dequantize(cache: kvq_cache, seq: int, seq_len_host: int, start: int, count: int,

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
@@ -206,6 +207,55 @@ kvq_status kvq_read_status(const kvq_cache* cache, int32_t* bits_out, int32_t cl
   }
   *bits_out = v;
   if (v) return fail(KVQ_ERR_DEVICE, "device status bits 0x%x", v);
+  return KVQ_OK;
+}
+
+// ---- allocation-free decode: the split partials in a file-scope device array ----------
+namespace {
+__device__ __align__(256) uint8_t g_decode_scratch[KVQ_DECODE_STATIC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices];  // per device, resolved on first use
+}  // namespace
+
+kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, int32_t num_q_heads, float sm_scale,
+                                       float* out, kvq_stream_t stream) {
+  g_err[0] = 0;
+  kvq_status s = check_cache(cache);
+  if (s != KVQ_OK) return s;
+  if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads)
+    return fail(KVQ_ERR_UNSUPPORTED, "num_q_heads %d is not a multiple of num_kv_heads %d", num_q_heads,
+                cache->num_kv_heads);
+  if (num_q_heads / cache->num_kv_heads > 16)
+    return fail(KVQ_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+  if (cache->num_seqs == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q / out is NULL");
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if (!(sm_scale > 0.0f)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale must be positive");
+  kvq::Geom g = kvq::make_geom(*cache);
+  const int nsplit = kvq::decode_num_splits(g, num_q_heads, num_sms());
+  const size_t need = kvq::decode_workspace(g, num_q_heads, nsplit);
+  if (need > KVQ_DECODE_STATIC_SCRATCH_BYTES)
+    return fail(KVQ_ERR_WORKSPACE, "decode partials need %zu bytes; the static scratch holds %zu", need,
+                (size_t)KVQ_DECODE_STATIC_SCRATCH_BYTES);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "kvq_decode_attention_static (cudaGetDevice)");
+  if (dev < 0 || dev >= kMaxDevices) return fail(KVQ_ERR_UNSUPPORTED, "device %d beyond %d", dev, kMaxDevices);
+  void* ws;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+      e = cudaGetSymbolAddress(&g_scratch_addr[dev], g_decode_scratch);
+      if (e != cudaSuccess) {
+        g_scratch_addr[dev] = nullptr;
+        return cuda_fail(e, "kvq_decode_attention_static (cudaGetSymbolAddress)");
+      }
+    }
+    ws = g_scratch_addr[dev];
+  }
+  e = kvq::launch_decode(g, q, num_q_heads, sm_scale, out, ws, nsplit, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kvq_decode_attention_static");
   return KVQ_OK;
 }
 

@@ -218,6 +218,28 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, i
                                 float* out, void* ws, size_t ws_bytes, kvq_stream_t stream);
 
 /*
+ * kvq_decode_attention_static -- kvq_decode_attention without a caller workspace.
+ * This entry point has no counterpart in the method's description.  It is for callers
+ * that cannot hand the library a scratch buffer: a runtime whose device memory is
+ * partitioned up front with no pool left over for per-call scratch, or code that must
+ * not call back into its framework's allocator at this point.  It allocates nothing.
+ *   Same arguments, layout and result as kvq_decode_attention, minus ws / ws_bytes.
+ *   The split partials live in one file-scope device array of
+ *   KVQ_DECODE_STATIC_SCRATCH_BYTES (16 MiB) per device, shared by every call on that
+ *   device.  Calls whose partials need more (kvq_decode_workspace_bytes() larger than
+ *   the array) return KVQ_ERR_WORKSPACE before launching anything.
+ *   Overlapping calls race: two calls in flight at once on one device (different
+ *   streams, or different host threads) write the same array and corrupt each other's
+ *   results.  Calls issued to one stream run one after another and are safe.
+ *   The first call on each device resolves the array's address (cudaGetSymbolAddress,
+ *   once per device, under a lock); make that first call before any stream capture is
+ *   started on that device.
+ */
+#define KVQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+KVQ_API kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, int32_t num_q_heads,
+                                               float sm_scale, float* out, kvq_stream_t stream);
+
+/*
  * kvq_dequantize -- reconstruct tokens [start, start+count) of sequence `seq`
  * ([PKV] Section 3.2: pattern by index + dequantized residual; Eq. 1 inverted),
  * in the original space (the pre-transform is undone).

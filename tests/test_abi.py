@@ -98,3 +98,9 @@ def test_decode_validation_on_host():
     rc = kvq._lib.kvq_decode_attention(ctypes.byref(c), ctypes.c_void_p(16), 4, 0.1, ctypes.c_void_p(16),
                                        ctypes.c_void_p(256), 8, None)
     assert rc == kvq.KVQ_ERR_WORKSPACE
+
+
+def test_static_scratch_size_matches_header():
+    import bit_kv_cache_26_b200 as kvq
+    m = re.search(r"#define\s+KVQ_DECODE_STATIC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", open(HEADER).read())
+    assert m and int(m.group(1)) << int(m.group(2)) == kvq.KVQ_DECODE_STATIC_SCRATCH_BYTES
