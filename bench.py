@@ -48,6 +48,37 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
+def source_digest() -> str:
+    """Digest of the CUDA sources and the layout header: DRAM traffic taken with ncu is only
+    reported while the kernels it was taken on are unchanged."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "bit_kv_cache_26_b200", "csrc", "*"))) + \
+        [os.path.join(ROOT, "include", "kvq.h")]
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload: str, bits: int, batch: int):
+    """DRAM bytes (read + write) per call of each phase, from profiles/dram_traffic.txt (one ncu
+    capture per source digest); {} if there is none for the current sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    digest = source_digest()
+    with open(path) as f:
+        for line in f:
+            t = line.split()
+            if len(t) == 6 and not line.startswith("#") and t[0] == digest and t[1] == workload and \
+                    int(t[2]) == bits and int(t[3]) == batch:
+                out[t[4]] = float(t[5])
+    return out
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -191,6 +222,8 @@ def main():
     ap.add_argument("--bits", type=int, default=2)
     ap.add_argument("--ref-tokens", type=int, default=65536)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases of the same kernels, for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -215,6 +248,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    if args.batch:
+        base = base.with_(B=args.batch)
     w = rank_workload(base, rank)
     k, v = synth.gen_kv(w)
     q = synth.gen_q(w)
@@ -309,21 +344,25 @@ def main():
     token_heads = n * w.Hkv
     dec_bytes = token_heads * bpt
     app_bytes = token_heads * (bpt + 2 * 2 * D)
-    mine_flops = 2 * 2 * n * w.P * D * w.iters * w.Hkv  # 2 flops per MAC, K and V
+    # mining: every vector read once per Lloyd iteration (K and V calls; the minimum for unfused Lloyd)
+    mine_bytes = 2 * w.iters * n * w.Hkv * D * 2
     rooflines = {
         "decode_attention": {"bound": "hbm", "achieved": dec_bytes / (decode_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                              "unit": "GB/s", "ms": decode_ms, "algorithmic_bytes": dec_bytes},
         "quantize_append": {"bound": "hbm", "achieved": app_bytes / (append_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "ms": append_ms, "algorithmic_bytes": app_bytes},
-        "mine_patterns": {"bound": "tensor", "achieved": mine_flops / (mine_ms * 1e-3) / 1e12,
-                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "ms": mine_ms, "algorithmic_flops": mine_flops},
+        "mine_patterns": {"bound": "hbm", "achieved": mine_bytes / (mine_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                          "unit": "GB/s", "ms": mine_ms, "algorithmic_bytes": mine_bytes},
     }
+    traffic = dram_traffic(w.name, w.bits, w.B)
+    for name, r in rooflines.items():
+        r["traffic"] = traffic.get(name)
     for r in rooflines.values():
         r["frac"] = r["achieved"] / r["peak"]
     dominant = max(rooflines, key=lambda k: rooflines[k]["ms"])
     dom = rooflines[dominant]
     roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
-                "frac": dom["frac"], "traffic": None, "kernel": dominant, "peak_source": pk["source"]}
+                "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dominant, "peak_source": pk["source"]}
 
     if rank == 0:
         line = {
