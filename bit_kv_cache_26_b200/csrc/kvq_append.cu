@@ -175,7 +175,7 @@ __device__ __forceinline__ uint32_t code_pair(float R0, float R1, float z0, floa
 // One 32-bit code word of the V block (rows = channels, 2 column tiles of 16 tokens) from
 // the staged residuals Rv[token][channel] and per-(group, token) s / z / 1/s.  Tokens below
 // keep_lo keep their bits from `old`; tokens at or above tok_hi get code 0.
-template <int BITS>
+template <int BITS, bool MASK>
 __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const float* vs, const float* vz,
                                            const float* vr, int keep_lo, int tok_hi, uint32_t old) {
   constexpr int SPW = 16 / BITS, maxc = (1 << BITS) - 1;
@@ -192,9 +192,13 @@ __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const
     const float2 ri = *reinterpret_cast<const float2*>(vr + gi);
     const uint32_t c01 = code_pair(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi);
     const int b0 = BITS * slot, b1 = b0 + 16;
-    const uint32_t c0 = c01 & 0xffu, c1 = c01 >> 16;
-    word |= (tok < keep_lo ? (old >> b0) & maxc : tok < tok_hi ? c0 : 0u) << b0;
-    word |= (tok + 1 < keep_lo ? (old >> b1) & maxc : tok + 1 < tok_hi ? c1 : 0u) << b1;
+    if constexpr (MASK) {
+      const uint32_t c0 = c01 & 0xffu, c1 = c01 >> 16;
+      word |= (tok < keep_lo ? (old >> b0) & maxc : tok < tok_hi ? c0 : 0u) << b0;
+      word |= (tok + 1 < keep_lo ? (old >> b1) & maxc : tok + 1 < tok_hi ? c1 : 0u) << b1;
+    } else {
+      word |= c01 << b0;
+    }
   }
   return word;
 }
@@ -248,7 +252,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __shared__ int qn;
   // dynamic: lower bounds lb[j][row] during the assignment, then s / z / 1/s tables
   extern __shared__ __align__(16) float dsm[];
-  float* lbuf = dsm;
+  float* lbuf = dsm;           // [P][64 rows] lower bounds
   float* vsz = dsm;            // [3][4][kG]: s, z, 1/s per (group, V slot)
   float* ksz = dsm + 12 * kG;  // [3][kD]:   s, z, 1/s per K channel
 
@@ -349,7 +353,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   }
   __syncthreads();
 
-  // ---- seed = smallest bound; its exact d_mm, two threads per row (channel halves)
+  // ---- seed = smallest bound; its exact d_mm, two threads per row (channel halves); then the
+  // same two threads queue the patterns (one half each) whose bound does not exclude them
   {
     const int r = tid >> 1, hh = tid & 1;
     const bool on = row_on(r);
@@ -364,22 +369,15 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     }
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
     mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+    const float ds = __fsub_rn(mx, mn);
     if (on && hh == 0) {
-      const float d = __fsub_rn(mx, mn);
-      dseed[r] = d;
+      dseed[r] = ds;
       seed[r] = s;
-      best[r] = dkey(d, s);
+      best[r] = dkey(ds, s);
     }
-  }
-  __syncthreads();
-
-  // ---- survivors: patterns whose bound does not exclude them
-  {
-    const int r = tid & (2 * kG - 1), hh = tid >> 6;
-    if (row_on(r)) {
-      const int s = seed[r];
-      const float ds = dseed[r];
+    if (on) {
       const int j1 = hh ? P : P0;
+#pragma unroll 4
       for (int j = hh ? P0 : 0; j < j1; ++j) {
         const float lb = lbuf[j * (2 * kG) + r];
         if (j == s || lb > ds || (lb == ds && j > s)) continue;
@@ -427,55 +425,46 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   }
   __syncthreads();
 
-  // ---- residuals in place: R = y - M[k*], warp per row, pattern loads issued 8 rows at a time
+  // ---- residuals in place, R = y - M[k*], one thread per (row, 32-channel group): rows
+  // lane and lane + 32 (V slot, K slot) of group `warp`; the V groups' scale / zero on the way
   {
-    constexpr int kRows = 2 * kG / (kAppendThreads / 32), kBatch = 8;
+    const int q = warp;
 #pragma unroll
-    for (int u0 = 0; u0 < kRows; u0 += kBatch) {
-      float4 mv[kBatch];
+    for (int u = 0; u < 2; ++u) {
+      const int r = lane + kG * u;
+      float s = 0.f, z = 0.f, ri = 0.f;
+      if (row_on(r)) {
+        const float4* m4 = reinterpret_cast<const float4*>((u ? c.MK : c.MV) + (size_t)(best[r] & 0xffffffffu) * kD +
+                                                           32 * q);
+        float4* y4 = reinterpret_cast<float4*>(&vec[r][32 * q]);
+        float4 mv[8];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int r = warp + (u0 + u) * nwarps;
-        if (row_on(r))
-          mv[u] = __ldg(reinterpret_cast<const float4*>((r < kG ? c.MV : c.MK) + (size_t)(best[r] & 0xffffffffu) * kD) +
-                        lane);
+        for (int k = 0; k < 8; ++k) mv[k] = __ldg(m4 + k);
+        float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 a = y4[k];
+          float4 o;
+          sub2(a.x, a.y, mv[k].x, mv[k].y, o.x, o.y);
+          sub2(a.z, a.w, mv[k].z, mv[k].w, o.z, o.w);
+          y4[k] = o;
+          mx = max3(mx, o.x, o.y);
+          mn = min3(mn, o.x, o.y);
+          mx = max3(mx, o.z, o.w);
+          mn = min3(mn, o.z, o.w);
+        }
+        if (u == 0) group_sz(mn, mx, g.bits, s, z, ri);
       }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int r = warp + (u0 + u) * nwarps;
-        if (!row_on(r)) continue;
-        float4* y4 = reinterpret_cast<float4*>(&vec[r][4 * lane]);
-        const float4 a = *y4;
-        float4 o;
-        sub2(a.x, a.y, mv[u].x, mv[u].y, o.x, o.y);
-        sub2(a.z, a.w, mv[u].z, mv[u].w, o.z, o.w);
-        *y4 = o;
+      if (u == 0) {  // V: every slot, zeros for tokens not in this call
+        vsz[(0 * 4 + q) * kG + lane] = s;
+        vsz[(1 * 4 + q) * kG + lane] = z;
+        vsz[(2 * 4 + q) * kG + lane] = ri;
       }
     }
   }
   __syncthreads();
 
-  // ---- scale / zero: V per (token, group of 32 channels), K per channel over the page
-  {
-    const int q = tid >> 5, slot = tid & 31;  // V: group q, token slot (conflict-free rows)
-    float s = 0.f, z = 0.f, ri = 0.f;
-    if (slot >= lo && slot < hi) {
-      const float4* p = reinterpret_cast<const float4*>(&vec[slot][32 * q]);
-      float mx = -INFINITY, mn = INFINITY;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 v = p[k];
-        mx = max3(mx, v.x, v.y);
-        mn = min3(mn, v.x, v.y);
-        mx = max3(mx, v.z, v.w);
-        mn = min3(mn, v.z, v.w);
-      }
-      group_sz(mn, mx, g.bits, s, z, ri);
-    }
-    vsz[(0 * 4 + q) * kG + slot] = s;
-    vsz[(1 * 4 + q) * kG + slot] = z;
-    vsz[(2 * 4 + q) * kG + slot] = ri;
-  }
+  // ---- K scale / zero per channel over the page
   float* ks_g = reinterpret_cast<float*>(c.sub + g.off_ks);
   float* kz_g = reinterpret_cast<float*>(c.sub + g.off_kz);
   if (c.seal) {
@@ -504,10 +493,16 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const int keep_lo = c.fresh ? 0 : lo;
     const float(*Rv)[kLd] = vec;
     const float(*Rk)[kLd] = vec + kG;
+    const bool whole = keep_lo == 0 && hi == kG;  // every token of the page is new
     for (int wd = tid; wd < nwords; wd += blockDim.x) {
-      const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;  // tokens already in the page keep their codes
-      vdst[wd] = g.bits == 2 ? v_word<2>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old)
-                             : v_word<4>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old);
+      if (whole) {
+        vdst[wd] = g.bits == 2 ? v_word<2, false>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, 0, kG, 0u)
+                               : v_word<4, false>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, 0, kG, 0u);
+      } else {
+        const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;  // tokens already in the page keep their codes
+        vdst[wd] = g.bits == 2 ? v_word<2, true>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old)
+                               : v_word<4, true>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old);
+      }
     }
     if (c.seal) {
       uint32_t* kdst = reinterpret_cast<uint32_t*>(c.sub);

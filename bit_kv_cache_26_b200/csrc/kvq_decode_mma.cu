@@ -33,9 +33,7 @@ namespace kvq {
 
 namespace {
 
-constexpr int kStages = 3;
 constexpr uint32_t kSpinLimit = 1u << 22;
-constexpr float kRangeLimit = 30000.0f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -247,8 +245,23 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
     const int hh = i / P, j = i % P;
     float t = 0.f;
     if (hh < Gq) {
+      // qk holds KSC order: its float4 p covers channels c, c + 1, c + 8, c + 9 with
+      // c = 16 (p >> 2) + 2 (p & 3); four independent partial sums
       const float* m = MK + (size_t)j * kD;
-      for (int d = 0; d < kD; ++d) t = fmaf(qk[hh * kD + ksc_pos(d)], __ldg(m + d), t);
+      const float4* q4 = reinterpret_cast<const float4*>(qk + hh * kD);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+      for (int p = 0; p < kD / 4; ++p) {
+        const float4 qv = q4[p];
+        const int c = 16 * (p >> 2) + 2 * (p & 3);
+        const float2 ma = __ldg(reinterpret_cast<const float2*>(m + c));
+        const float2 mb = __ldg(reinterpret_cast<const float2*>(m + c + 8));
+        a0 = fmaf(qv.x, ma.x, a0);
+        a1 = fmaf(qv.y, ma.y, a1);
+        a2 = fmaf(qv.z, mb.x, a2);
+        a3 = fmaf(qv.w, mb.y, a3);
+      }
+      t = (a0 + a1) + (a2 + a3);
     }
     T[i] = t;
   }
@@ -281,19 +294,27 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
       for (int u = 0; u < 4; ++u) accv[j][mt][u] = 0.f;
   }
 
-  // pages of this warp: p0 + warp + kWarps*i
+  // pages of this warp: p0 + warp + kWarps*i.  Their physical ids are read 32 at a time (lane l
+  // holds page 32w + l of window w), one window ahead, so no page-table load sits between a
+  // page and the copy of the page STAGES ahead.
   const int my_n = (p1 - p0 - warp + kWarps - 1) / kWarps;
-  auto page_src = [&](int i, bool& ok) -> const uint8_t* {
-    const int pg = p0 + warp + kWarps * i;
-    const int phys = g.page_table[(size_t)b * g.maxp + pg];
+  auto load_ids = [&](int base) -> int {
+    const int i = base + lane;
+    return i < my_n ? g.page_table[(size_t)b * g.maxp + p0 + warp + kWarps * i] : -1;
+  };
+  int ids = load_ids(0), ids_next = load_ids(32);
+  auto page_src = [&](int phys, bool& ok) -> const uint8_t* {
     ok = phys >= 0 && phys < g.npages;
     return g.pool + (size_t)(ok ? phys : 0) * g.page_bytes + (size_t)h_kv * g.sub_bytes;
   };
   uint32_t bad_mask = 0;  // lane 0: stages whose page id was invalid
+  int first_ids[STAGES];
+#pragma unroll
+  for (int i = 0; i < STAGES; ++i) first_ids[i] = __shfl_sync(kFull, ids, i);
   if (lane == 0) {
     for (int i = 0; i < min(STAGES, my_n); ++i) {
       bool ok;
-      const uint8_t* src = page_src(i, ok);
+      const uint8_t* src = page_src(first_ids[i], ok);
       if (ok) {
         mbar_expect_tx(&bars[i], sub_bytes);
         bulk_g2s(ring + i * sub_bytes, src, sub_bytes, &bars[i]);
@@ -467,10 +488,16 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
     }
     __syncwarp();
     // refill this stage with the page STAGES ahead
-    if (lane == 0 && i + STAGES < my_n) {
+    const int nxt = i + STAGES;
+    if ((nxt & 31) == 0 && nxt > 0) {  // next window of page ids
+      ids = ids_next;
+      ids_next = load_ids(nxt + 32);
+    }
+    const int nxt_phys = __shfl_sync(kFull, ids, nxt & 31);
+    if (lane == 0 && nxt < my_n) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       bool okp;
-      const uint8_t* src = page_src(i + STAGES, okp);
+      const uint8_t* src = page_src(nxt_phys, okp);
       bad_mask &= ~(1u << st);
       if (okp) {
         mbar_expect_tx(&bars[st], sub_bytes);

@@ -694,6 +694,351 @@ cudaError_t launch_accum(const Src& s, int P, int NP, int sms, const int32_t* as
              : launch_accum_t<16, 1, 2>(s, P, NP, sms, assign, sums, cnt, st);
 }
 
+// ---- tcgen05 assignment (bf16 input, P <= 128) ------------------------------------------
+//
+// The same certified argmin as mine_assign_mma_kernel, with the distance contraction on
+// the 5th-generation tensor cores: per 128-token tile, one thread issues 8 MMAs of
+// M = 128 (tokens) x N = 2 Pn (the bf16 hi parts of the Pn padded patterns, then their mid
+// parts) x K = 16 into a TMEM accumulator, so each product term keeps its own fp32 chain
+// of 8 MMAs (the error model of the certification above).  Tiles reach shared memory
+// through cp.async in the canonical K-major layout without swizzle (8-row x 16-byte core
+// matrices; LBO = 128 B between core matrices along K, SBO = 2048 B between 8-row groups);
+// the accumulators are double-buffered in TMEM, so the MMAs of tile k overlap the epilogue
+// of tile k - 1, in which thread t reads row t (token t) back with tcgen05.ld, adds the
+// two chains, and runs the gap test.  A token that fails it re-reads its scores (the whole
+// warp, tcgen05.ld is warp-collective) and is decided exactly in float64.
+constexpr int kTcM = 128;
+constexpr int kTcStages = 2;
+constexpr int kTcTileBytes = kTcM * kD * 2;
+constexpr uint32_t kTcLBO = 128, kTcSBO = 2048;
+constexpr uint32_t kTcSpinLimit = 1u << 24;
+
+__host__ __device__ constexpr uint32_t kmaj_off(int row, int k) {
+  return (uint32_t)(row >> 3) * kTcSBO + (uint32_t)(k >> 3) * kTcLBO + (uint32_t)(row & 7) * 16u + (uint32_t)(k & 7) * 2u;
+}
+
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// shared-memory matrix descriptor: start, LBO, SBO (all >> 4), descriptor version 1, no swizzle
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((kTcLBO >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((kTcSBO >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, N >> 3, M >> 4
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, int accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tc_mbar_init(uint64_t* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(bar)) : "memory");
+}
+__device__ __forceinline__ bool tc_mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kTcSpinLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(su32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(256, 2) mine_assign_tc_kernel(Src s, int P, const float* __restrict__ M,
+                                                                 int32_t* __restrict__ assign, int32_t* status) {
+  const int prob = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Pn = (P + 7) & ~7, N = 2 * Pn;
+  const uint32_t tcols = N <= 128 ? 256u : 512u;  // two accumulator buffers
+  const uint32_t buf_cols = tcols / 2;
+  extern __shared__ __align__(16) uint8_t smraw[];
+  uint8_t* Bt = smraw;                                                   // [N][128] bf16, canonical K-major
+  uint8_t* At = smraw + (size_t)N * kD * 2;                              // [stages][128][128] bf16
+  float* msq = reinterpret_cast<float*>(At + (size_t)kTcStages * kTcTileBytes);  // [Pn]
+  float* mnorm = msq + Pn;                                               // [Pn]
+  float* gmax = mnorm + Pn;                                              // [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);                // [2] (16-byte aligned: Pn % 8 == 0)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2);
+  float* xch = reinterpret_cast<float*>(tslot + 4);  // [4][128]: warpgroup 1's m1, m2, j1, partial |x|^2
+  const float* Mp = M + (size_t)prob * P * kD;
+  const int set = prob / s.heads, h = prob % s.heads;
+
+  // ---- B: bf16 hi parts (rows 0..Pn-1) and mid parts (rows Pn..2Pn-1) of the patterns
+  for (int i = tid; i < N * 16; i += blockDim.x) {
+    const int n = i >> 4, c = i & 15;
+    const int j = n < Pn ? n : n - Pn;
+    uint32_t wv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint16_t hv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float m = j < P ? Mp[(size_t)j * kD + 8 * c + 2 * q + e] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(m);
+        const __nv_bfloat16 v = n < Pn ? hi : __float2bfloat16_rn(m - __bfloat162float(hi));
+        hv[e] = __bfloat16_as_ushort(v);
+      }
+      wv[q] = (uint32_t)hv[0] | ((uint32_t)hv[1] << 16);
+    }
+    *reinterpret_cast<uint4*>(Bt + kmaj_off(n, 8 * c)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  }
+  if (tid == 0) {
+    gmax[0] = 0.f;
+    gmax[1] = 0.f;
+    tc_mbar_init(&bars[0]);
+    tc_mbar_init(&bars[1]);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tslot)), "r"(tcols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  for (int j = tid; j < Pn; j += blockDim.x) {
+    double acc = 0.0;
+    if (j < P)
+      for (int d = 0; d < kD; ++d) { const double m = Mp[(size_t)j * kD + d]; acc += m * m; }
+    msq[j] = (float)acc;
+    mnorm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
+    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int(mnorm[j]));
+    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq[j] * (1.0f + 1e-6f)));
+  }
+  fence_proxy_async();  // B (generic stores) before the tensor cores read it
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  const float nm_max = gmax[0], msq_max = gmax[1];
+  const uint32_t idesc = umma_idesc(kTcM, N);
+
+  const int64_t ntiles = (s.n + kTcM - 1) / kTcM;
+  const int nt = ntiles > blockIdx.x ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  auto tile_t0 = [&](int k) { return ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * kTcM; };
+  auto load_tile = [&](int k) {
+    if (k < nt) {
+      const int64_t t0 = tile_t0(k);
+      uint8_t* st = At + (size_t)(k % kTcStages) * kTcTileBytes;
+      // a warp writes 8 rows x 4 chunks: four contiguous 128-byte runs, no bank conflicts
+      for (int i = tid; i < kTcM * 16; i += blockDim.x) {
+        const int r = ((i >> 7) << 3) | (i & 7), c = (i >> 3) & 15;
+        const int64_t tok = t0 + r;
+        uint8_t* dst = st + kmaj_off(r, 8 * c);
+        if (tok < s.n) cp_async16(dst, s.x + set * s.ss + tok * s.ts + h * s.hs + 8 * c);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
+  };
+
+  bool ok_all = true;
+  // epilogue of tile k; once its MMAs are complete, the copy of tile k + 2 goes into its stage
+  auto epilogue = [&](int k, float xsq_raw) {
+    const int buf = k & 1;
+    const bool ok = tc_mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1));
+    load_tile(k + 2);
+    // the same verdict for every thread of the CTA (barriers follow)
+    if (!__syncthreads_and(ok)) {  // the accumulator never arrived: flag it and skip the tile
+      ok_all = false;
+      return;
+    }
+    tc_fence_after();
+    const int wg = warp >> 2, q4 = warp & 3;  // warpgroup: which 32-column blocks; q4: TMEM lane quarter
+    const int row = q4 * 32 + lane;
+    const int64_t i = tile_t0(k) + row;
+    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)buf * buf_cols;
+    Top2 top{INFINITY, INFINITY, 0}, top_b{INFINITY, INFINITY, 0};  // even / odd patterns: two chains
+    for (int c0 = 32 * wg; c0 < Pn; c0 += 64) {
+      float hv[32], mv[32];
+      tmem_ld32(taddr + c0, hv);
+      tmem_ld32(taddr + Pn + c0, mv);
+#pragma unroll
+      for (int q = 0; q < 32; q += 2) {
+        const int j = c0 + q;
+        if (j < P) top2_add(top, msq[j] - 2.0f * (hv[q] + mv[q]), j);
+        if (j + 1 < P) top2_add(top_b, msq[j + 1] - 2.0f * (hv[q + 1] + mv[q + 1]), j + 1);
+      }
+    }
+    // merge (lower index wins equal minima)
+    if (top_b.m1 < top.m1 || (top_b.m1 == top.m1 && top_b.j1 < top.j1)) {
+      top.m2 = fminf(top.m1, top_b.m2);
+      top.m1 = top_b.m1;
+      top.j1 = top_b.j1;
+    } else {
+      top.m2 = fminf(top.m2, top_b.m1);
+    }
+    // warpgroup 1 hands its partial results to warpgroup 0, which decides the row
+    if (wg == 1) {
+      xch[0 * kTcM + row] = top.m1;
+      xch[1 * kTcM + row] = top.m2;
+      xch[2 * kTcM + row] = __int_as_float(top.j1);
+      xch[3 * kTcM + row] = xsq_raw;
+    }
+    __syncthreads();
+    if (wg == 1) {
+      tc_fence_before();
+      return;
+    }
+    {
+      const float om1 = xch[0 * kTcM + row], om2 = xch[1 * kTcM + row];
+      const int oj = __float_as_int(xch[2 * kTcM + row]);
+      const float lo2 = fminf(top.m2, om2);
+      if (om1 < top.m1 || (om1 == top.m1 && oj < top.j1)) { top.m2 = fminf(top.m1, lo2); top.m1 = om1; top.j1 = oj; }
+      else top.m2 = fminf(om1, lo2);
+    }
+    float xsq = xsq_raw + xch[3 * kTcM + row];
+    xsq *= (1.0f + 1e-6f);
+    const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
+    const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xsq + msq_max);
+    const bool unique = top.m2 - top.m1 > 2.0f * Eb + 1e-9f * (xsq + msq_max);
+    if (unique && i < s.n) assign[(size_t)prob * s.n + i] = top.j1;
+    const bool need = !unique && i < s.n;
+    if (__any_sync(kFull, need)) {
+      // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
+      float U = INFINITY;
+      for (int c0 = 0; c0 < Pn; c0 += 32) {
+        float hv[32], mv[32];
+        tmem_ld32(taddr + c0, hv);
+        tmem_ld32(taddr + Pn + c0, mv);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int j = c0 + q;
+          if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
+        }
+      }
+      uint32_t cand[4] = {0u, 0u, 0u, 0u};  // candidate bit mask over j < 128
+      for (int c0 = 0; c0 < Pn; c0 += 32) {
+        float hv[32], mv[32];
+        tmem_ld32(taddr + c0, hv);
+        tmem_ld32(taddr + Pn + c0, mv);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int j = c0 + q;
+          const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
+          const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
+          if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cand[c0 >> 5] |= 1u << q;
+        }
+      }
+      if (need) {
+        const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
+        double bd = 0.0;
+        int bj = 0;
+        bool have = false;
+        for (int cw = 0; cw < 4; ++cw)
+          for (uint32_t m = cand[cw]; m; m &= m - 1) {
+            const int j = cw * 32 + __ffs(m) - 1;
+            const float* mrow = Mp + (size_t)j * kD;
+            double acc = 0.0;
+#pragma unroll 8
+            for (int d = 0; d < kD; d += 4) {
+              const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
+              const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                   __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+              const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
+              const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
+                acc = __dadd_rn(acc, __dmul_rn(t, t));
+              }
+            }
+            if (!have || acc < bd) { bd = acc; bj = j; have = true; }
+          }
+        assign[(size_t)prob * s.n + i] = bj;
+      }
+    }
+    tc_fence_before();
+  };
+
+  // |x|^2 of this thread's row of tile k, from its stage (read while the MMAs read it too)
+  auto row_norm = [&](int k) {  // half of the row's channels per warpgroup
+    const uint8_t* st = At + (size_t)(k % kTcStages) * kTcTileBytes;
+    const int row = (warp & 3) * 32 + lane, c0 = 8 * (warp >> 2);
+    float xs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = c0; c < c0 + 8; ++c) {
+      const uint4 u = *reinterpret_cast<const uint4*>(st + kmaj_off(row, 8 * c));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
+        xs[q] = fmaf(v0, v0, xs[q]);
+        xs[q] = fmaf(v1, v1, xs[q]);
+      }
+    }
+    return (xs[0] + xs[1]) + (xs[2] + xs[3]);
+  };
+
+  // stage s holds tile k with k % 2 == s; the copy of tile k + 2 starts once tile k's MMAs are done
+  load_tile(0);
+  load_tile(1);
+  float xsq_prev = 0.f;
+  for (int k = 0; k < nt; ++k) {
+    // this thread's copies of tile k: the newest group, except at k = 0 (tile 1 is newer)
+    if (k == 0) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    fence_proxy_async();
+    __syncthreads();  // all copies of tile k; the epilogue of tile k - 2 (same TMEM buffer) is done
+    tc_fence_after();
+    if (tid == 0 && ok_all) {
+      const uint32_t a0 = su32(At + (size_t)(k % kTcStages) * kTcTileBytes), b0 = su32(Bt);
+      const uint32_t d = tbase + (uint32_t)(k & 1) * buf_cols;
+#pragma unroll
+      for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(d, umma_desc(a0 + ks * 256), umma_desc(b0 + ks * 256), idesc, ks > 0);
+      umma_commit(&bars[k & 1]);
+    }
+    const float xsq_k = row_norm(k);
+    if (k > 0 && ok_all) epilogue(k - 1, xsq_prev);
+    else if (k > 0) load_tile(k + 1);
+    xsq_prev = xsq_k;
+  }
+  if (nt > 0 && ok_all) epilogue(nt - 1, xsq_prev);
+  cp_async_wait<0>();
+  if (!ok_all && lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
+}
+
+size_t mine_tc_smem(int P) {
+  const int Pn = (P + 7) & ~7;
+  return (size_t)2 * Pn * kD * 2 + (size_t)kTcStages * kTcTileBytes + 2 * Pn * 4 + 16 + 16 + 16 + 4 * kTcM * 4 + 1024;
+}
+
 __global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt) {
   const int prob = blockIdx.y, j = blockIdx.x, d = threadIdx.x;
   const size_t pj = (size_t)prob * P + j;
@@ -763,9 +1108,20 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   const int tok_per_cta = kMmaWarps * (KIND == 0 ? 32 : 16);
   const unsigned mma_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + tok_per_cta - 1) / tok_per_cta, (int64_t)(2 * sms + NP - 1) / NP));
+  // bf16 input and P <= 128: the tcgen05 kernel, two CTAs (each with 256 TMEM columns) per SM
+  const bool use_tc = KIND == 0 && a.P <= kMmaMaxP;
+  const size_t smem_tc = mine_tc_smem(a.P);
+  if (use_tc &&
+      (e = cudaFuncSetAttribute(mine_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_tc)) !=
+          cudaSuccess)
+    return e;
+  const unsigned tc_ctas = (unsigned)std::max<int64_t>(
+      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, 2 * sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
-    if (use_mma && KIND == 0)
+    if (use_tc)
+      mine_assign_tc_kernel<<<dim3(tc_ctas, NP), 256, smem_tc, st>>>(s, a.P, a.patterns, w.assign, nullptr);
+    else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else if (use_mma && KIND == 1)
       mine_assign_mma_kernel<1><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
