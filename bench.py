@@ -379,7 +379,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
                     "d2h_bytes_per_step": int(out_h.numel() * 4)},
-            "gpu_launches": args.steps * (2 * (1 + 3 * w.iters + (15 if w.transform else 0)) + 3 + 2),
+            "gpu_launches": args.steps * (2 * (1 + 3 * w.iters + (15 if w.transform else 0)) + 3 + 1),
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -2,17 +2,17 @@
 // min-max distance, quantize the residual per group and store it in the paged
 // cache ("PatternKV", Section 3.2 and Eq. 6; Eq. 1; granularity of Section 4.1).
 //
-// Launch 0 (prep, per call): for every (set, KV head) and K / V pattern set, the 16
-//   probe channels (those whose values differ most across the patterns) and every
-//   pattern's values there.
+// Launch 0 (prep, per call): for every (set, KV head) and K / V pattern set, the 32
+//   probe channels (those whose values differ most across the patterns, in that order) and
+//   every pattern's values there.
 // Launch 1 (page tasks): one CTA per (touched page, KV head, sequence).
 //   * the new V vectors of the page and, when the page's 32nd token arrives, its 32
 //     K vectors (older ones from the K tail) are staged in shared memory (after the
 //     pre-transform, if enabled);
 //   * an exact lower bound of d_mm(y, m_j) for every pattern: max and min only grow
-//     with the channel set, so the residual range over the probe channels never
-//     exceeds the range over all channels (same fp32 subtractions, no rounding of its
-//     own); one lane per vector, every pattern;
+//     with the channel set, so the residual range over the probe channels (the first 16
+//     for K, all 32 for V) never exceeds the range over all channels (same fp32
+//     subtractions, no rounding of its own); one lane per vector, every pattern;
 //   * the pattern with the smallest bound is the seed; its exact d_mm is an upper bound
 //     of the minimum, and every pattern whose bound already exceeds it (or equals it
 //     with a higher index) is excluded exactly;
@@ -37,7 +37,9 @@ namespace {
 
 constexpr int kAppendThreads = 128;
 constexpr int kQueueCap = 512;
-constexpr int kProbe = 16;  // channels of the partial-range bound
+constexpr int kProbe = 32;   // probe channels stored per pattern set (by decreasing spread)
+constexpr int kProbeK = 16;  // used for K rows (outlier channels make 16 enough)
+constexpr int kProbeV = 32;  // used for V rows (a tighter bound picks a better seed)
 constexpr int kLd = kD + 4;  // staged row stride (floats): 16-byte aligned, conflict-free columns
 
 struct AppendWs {
@@ -225,6 +227,38 @@ __device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const
   return word;
 }
 
+// Lower bounds over the first NPROBE probe channels for patterns [j0, j1) of one staged vector
+// y (one lane), written to lbuf[j][row]; running argmin (ties: lowest j) to (blb, bj).
+template <int NPROBE>
+__device__ __forceinline__ void lb_pass(const float* y, const int32_t* __restrict__ pc, const float* __restrict__ pvt,
+                                        int j0, int j1, float* lbuf, int row, float& blb_out, int& bj_out) {
+  float py[NPROBE];
+#pragma unroll
+  for (int u = 0; u < NPROBE; ++u) py[u] = y[__ldg(pc + u)];
+  float blb = INFINITY;
+  int bj = j0;
+  for (int j = j0; j < j1; ++j) {
+    const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * kProbe);
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int q = 0; q < NPROBE / 4; ++q) {
+      const float4 m = __ldg(m4 + q);
+      float r0, r1, r2, r3;
+      sub2(py[4 * q], py[4 * q + 1], m.x, m.y, r0, r1);
+      sub2(py[4 * q + 2], py[4 * q + 3], m.z, m.w, r2, r3);
+      mx = max3(mx, r0, r1);
+      mn = min3(mn, r0, r1);
+      mx = max3(mx, r2, r3);
+      mn = min3(mn, r2, r3);
+    }
+    const float lb = __fsub_rn(mx, mn);
+    lbuf[j * (2 * kG) + row] = lb;
+    if (lb < blb) { blb = lb; bj = j; }
+  }
+  blb_out = blb;
+  bj_out = bj;
+}
+
 // fp32 scale / zero / reciprocal of a group from its min and max
 __device__ __forceinline__ void group_sz(float mn, float mx, int bits, float& s, float& z, float& rinv) {
   s = __fdiv_rn(__fsub_rn(mx, mn), (float)((1 << bits) - 1));
@@ -319,37 +353,10 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   {
     const int kind = warp & 1, half = warp >> 1;
     const int r = kind * kG + lane;
-    if (kind == 0 || c.seal) {
-      const size_t o = shk + (kind ? 0 : 1);
-      const int32_t* pc = wsp.probe + o * kProbe;
-      const float* pvt = wsp.pv + o * P * kProbe;
-      float py[kProbe];
-#pragma unroll
-      for (int u = 0; u < kProbe; ++u) py[u] = vec[r][__ldg(pc + u)];
-      float blb = INFINITY;
-      int bj = half ? P0 : 0;
-      const int j1 = half ? P : P0;
-      for (int j = half ? P0 : 0; j < j1; ++j) {
-        const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * kProbe);
-        float mx = -INFINITY, mn = INFINITY;
-#pragma unroll
-        for (int q = 0; q < kProbe / 4; ++q) {
-          const float4 m = __ldg(m4 + q);
-          float r0, r1, r2, r3;
-          sub2(py[4 * q], py[4 * q + 1], m.x, m.y, r0, r1);
-          sub2(py[4 * q + 2], py[4 * q + 3], m.z, m.w, r2, r3);
-          mx = max3(mx, r0, r1);
-          mn = min3(mn, r0, r1);
-          mx = max3(mx, r2, r3);
-          mn = min3(mn, r2, r3);
-        }
-        const float lb = __fsub_rn(mx, mn);
-        lbuf[j * (2 * kG) + r] = lb;
-        if (lb < blb) { blb = lb; bj = j; }
-      }
-      hlb[half][r] = blb;
-      hj[half][r] = bj;
-    }
+    if (kind == 0) lb_pass<kProbeV>(vec[r], wsp.probe + (shk + 1) * kProbe, wsp.pv + (shk + 1) * P * kProbe,
+                                    half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    else if (c.seal) lb_pass<kProbeK>(vec[r], wsp.probe + shk * kProbe, wsp.pv + shk * P * kProbe,
+                                      half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
   }
   __syncthreads();
 

@@ -175,10 +175,79 @@ __host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int
   return s;
 }
 
+// Combine of one (sequence, KV head) group, run by the CTA that finished the group's last
+// split: log-sum-exp merge of the splits, the pattern term sum_j W_j M_V[j] and the inverse
+// pre-transform.  Warp w takes query heads w, w + warps, ...; lane l holds channels
+// l + 32 k.  The partials come from other CTAs, so they are read through L2 (after the fence
+// that follows the arrival counter).  A non-finite output (an operand outside the fp32 /
+// bf16 range upstream) sets KVQ_DEV_RANGE.
+__device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv, int Gq, int set,
+                              const float* part_ml, const float* part_o, const float* part_w, float* out,
+                              float* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  float* Wsh = scratch + warp * 256;  // this warp's W (P <= 256)
+  const float* MV = g.vpat + ((size_t)set * g.H + h_kv) * g.P * kD;
+  for (int hh = warp; hh < Gq; hh += nwarps) {
+    const int row = b * Hq + h_kv * Gq + hh;
+    const size_t base = (size_t)row * nsplit;
+    float* outp = out + (size_t)row * kD;
+    float M = -INFINITY;
+    for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(part_ml + 2 * (base + s)));
+    M = warp_max(M);
+    if (M == -INFINITY) {  // no tokens
+#pragma unroll
+      for (int k = 0; k < 4; ++k) outp[lane + 32 * k] = 0.f;
+      continue;
+    }
+    float Lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < nsplit; ++s) {
+      const float ms = __ldcg(part_ml + 2 * (base + s));
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      Lsum += f * __ldcg(part_ml + 2 * (base + s) + 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] += f * __ldcg(part_o + (base + s) * kD + lane + 32 * k);
+    }
+    for (int j = lane; j < g.P; j += 32) {
+      float W = 0.f;
+      for (int s = 0; s < nsplit; ++s) {
+        const float ms = __ldcg(part_ml + 2 * (base + s));
+        if (ms == -INFINITY) continue;
+        W += exp2f(ms - M) * __ldcg(part_w + (base + s) * g.P + j);
+      }
+      Wsh[j] = W;
+    }
+    __syncwarp();
+    for (int j = 0; j < g.P; ++j) {
+      const float W = Wsh[j];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] = fmaf(W, __ldg(MV + (size_t)j * kD + lane + 32 * k), o[k]);
+    }
+    __syncwarp();
+    const float inv = 1.0f / Lsum;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] *= inv;
+    if (g.tx) {
+      const float* cV = g.vcol + ((size_t)set * g.H + h_kv) * kD;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] *= cV[lane + 32 * k];
+      fwht_warp(o, lane);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] *= 0.0078125f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (!isfinite(o[k])) set_status(g.status, KVQ_DEV_RANGE);
+      outp[lane + 32 * k] = o[k];
+    }
+  }
+}
+
 template <int BITS, int NT, int STAGES, int kWarps>
 __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 : 3) : 2))
     decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
-                      float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w) {
+                      float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w,
+                      int* __restrict__ arrivals, float* __restrict__ out) {
   constexpr int NH = NT * 4;  // padded heads
   constexpr int WPL = Cfg<BITS>::kWordsPerLane;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -656,6 +725,17 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
       part_w[base * P + jj] = Wv;
     }
   }
+
+  // ---- the CTA that completes a (sequence, KV head) group merges its splits into `out`
+  __shared__ int last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(arrivals + (size_t)b * g.H + h_kv, 1) == nsplit - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  combine_group(g, Hq, nsplit, b, h_kv, Gq, set, part_ml, part_o, part_w, out,
+                reinterpret_cast<float*>(smem + sp.ring));
 }
 
 template <int BITS, int NT, int STAGES, int NW>
@@ -669,12 +749,12 @@ struct Launcher {
     return n > 0 ? n : 1;
   }
   static cudaError_t launch(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml, float* o,
-                            float* w, cudaStream_t st) {
+                            float* w, int* arrivals, float* out, cudaStream_t st) {
     const int total = smem(g);
     cudaError_t e = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, g.H, g.B);
-    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w);
+    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w, arrivals, out);
     return cudaGetLastError();
   }
 };
@@ -740,9 +820,9 @@ size_t decode_mma_smem(const Geom& g, int Hq) {
 }
 
 cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
-                              float* o, float* w, cudaStream_t st) {
+                              float* o, float* w, int* arrivals, float* out, cudaStream_t st) {
   return dispatch(g, Hq, decode_stages(), [&](auto L) {
-    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, w, st);
+    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, w, arrivals, out, st);
   });
 }
 

@@ -9,6 +9,9 @@
 // fp32 rounding of the float64 mean, empty clusters keep their pattern.
 #include <algorithm>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -523,37 +526,77 @@ size_t mine_mma_smem(int P, int KIND) {
 }
 
 // Per-cluster float64 sums and sizes in one streaming pass.  A CTA walks a contiguous run
-// of 128-token tiles of one problem (and one channel slice), staged into shared memory by a
-// cp.async ring.  Warp w owns clusters w, w + 16, w + 32, ...; for each tile it finds the
-// members of each of its clusters with ballots over the tile's assignments and adds their
-// rows into float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1 of
-// the slice).  Each CTA adds its totals to global memory once at the end.  float64 sums of
-// fp16 / bf16 values are exact, so the order of the additions does not change them.
+// of 128-token tiles of one problem (and one channel slice).  One producer warp copies the
+// tiles' rows into a ring of shared-memory stages with cp.async.bulk (one 16-byte-aligned row
+// per copy, completion counted in bytes on the stage's "full" mbarrier); 16 consumer warps
+// each take every tile: warp w owns clusters w, w + 16, w + 32, ..., finds their members with
+// ballots over the tile's assignments (prefetched one tile ahead) and adds their rows into
+// float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1 of the slice),
+// then arrives on the stage's "empty" mbarrier.  A stage is refilled once all 16 warps are
+// done with it, so fast warps run ahead instead of waiting at a block barrier.  Each CTA adds
+// its totals to global memory once at the end.  float64 sums of fp16 / bf16 values are
+// exact, so the order of the additions does not change them.  Every wait is bounded.
 constexpr int kAccWarps = 16;
 constexpr int kAccT = 128;  // tokens per tile
+constexpr uint32_t kAccSpinLimit = 1u << 24;
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
+__device__ __forceinline__ uint32_t sa32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mb_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sa32(bar)), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
-               : "memory");
+__device__ __forceinline__ void mb_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sa32(bar)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void mb_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sa32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mb_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kAccSpinLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(sa32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(sa32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(sa32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(sa32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(sa32(bar))
+      : "memory");
+}
+
+template <int RB>
+constexpr int accum_stages() {
+  return (200 * 1024) / (kAccT * RB) < 4 ? (200 * 1024) / (kAccT * RB) : 4;
+}
 
 // CPW clusters per warp, E channels per lane (slice = 32 E channels), ES bytes per element
 // (2: the fp16 / bf16 input, 4: the fp32 pre-transformed rows)
 template <int CPW, int E, int ES>
-__global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, int P, const int32_t* __restrict__ assign,
-                                                                      double* __restrict__ sums,
-                                                                      uint32_t* __restrict__ cnt) {
-  constexpr int CW = 32 * E, RB = CW * ES;          // channels and bytes of a staged row
-  constexpr int kStages = ES == 2 ? 4 : 3;
-  constexpr int kStageBytes = kAccT * RB + kAccT * 4;
+__global__ void __launch_bounds__((kAccWarps + 1) * 32, 1) mine_accum_kernel(const __grid_constant__ CUtensorMap amap,
+                                                                            Src s, int P,
+                                                                            const int32_t* __restrict__ assign,
+                                                                            double* __restrict__ sums,
+                                                                            uint32_t* __restrict__ cnt) {
+  constexpr int CW = 32 * E, RB = CW * ES;  // channels and bytes of a staged row
+  constexpr int kStages = accum_stages<RB>();
+  constexpr int kStageBytes = kAccT * RB;
   extern __shared__ __align__(16) uint8_t smraw[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
   const int slice = blockIdx.y, prob = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
@@ -563,30 +606,36 @@ __global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, in
   const int nt = (int)(k1 - k0);
   const int set = prob / s.heads, h = prob % s.heads;
   const int32_t* a = assign + (size_t)prob * s.n;
-
-  auto issue = [&](int k) {  // tile k0 + k into its stage
-    if (k < nt) {
-      uint8_t* st = smraw + (size_t)(k % kStages) * kStageBytes;
-      int32_t* sa = reinterpret_cast<int32_t*>(st + kAccT * RB);
-      const int64_t tb = (k0 + k) * kAccT;
-      constexpr int kChunks = RB / 16;
-      for (int i = threadIdx.x; i < kAccT * kChunks; i += blockDim.x) {
-        const int t = i / kChunks, cix = i % kChunks;
-        if (tb + t < s.n) {
-          const uint8_t* src =
-              ES == 2 ? reinterpret_cast<const uint8_t*>(s.x + set * s.ss + h * s.hs + (tb + t) * s.ts + slice * CW)
-                      : reinterpret_cast<const uint8_t*>(s.y + ((size_t)prob * s.n + tb + t) * kD + slice * CW);
-          cp_async16(st + t * RB + cix * 16, src + cix * 16);
-        }
-      }
-      for (int t = threadIdx.x; t < kAccT; t += blockDim.x) {
-        if (tb + t < s.n) cp_async4(sa + t, a + tb + t);
-        else sa[t] = -1;
-      }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mb_init(&full[i], 1);
+      mb_init(&empty[i], kAccWarps);
     }
-    cp_async_commit();
-  };
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
 
+  if (warp == kAccWarps) {
+    // ---- producer: rows of tile k into stage k % kStages once every consumer left it
+    for (int k = 0; k < nt; ++k) {
+      const int st = k % kStages;
+      bool ok = true;
+      if (k >= kStages) ok = mb_wait(&empty[st], (uint32_t)(((k / kStages) - 1) & 1));
+      if (!__all_sync(kFull, ok)) break;  // consumers time out on the full barrier in turn
+      const int tb = (int)((k0 + k) * kAccT);
+      if (lane == 0) {
+        // one box of 128 tokens x CW channels lands row-major; rows past the end read as zeros
+        uint8_t* dst = smraw + (size_t)st * kStageBytes;
+        mb_expect_tx(&full[st], (uint32_t)kStageBytes);
+        if constexpr (ES == 2) tma_load_4d(dst, &amap, slice * CW, h, tb, set, &full[st]);
+        else tma_load_3d(dst, &amap, slice * CW, tb, prob, &full[st]);
+      }
+      __syncwarp();
+    }
+    return;
+  }
+
+  // ---- consumers
   double acc[CPW][E];
   uint32_t members[CPW];
 #pragma unroll
@@ -595,18 +644,22 @@ __global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, in
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[c][e] = 0.0;
   }
-
+  auto load_aj = [&](int k, int (&aj)[kAccT / 32]) {
+    const int64_t tb = (k0 + k) * kAccT;
 #pragma unroll
-  for (int k = 0; k < kStages - 1; ++k) issue(k);
+    for (int q = 0; q < kAccT / 32; ++q) {
+      const int64_t i = tb + 32 * q + lane;
+      aj[q] = i < s.n ? __ldg(a + i) : -1;
+    }
+  };
+  int aj[kAccT / 32], ajn[kAccT / 32];
+  load_aj(0, aj);
   for (int k = 0; k < nt; ++k) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();  // tile k visible to all; every warp is done with tile k - 1
-    issue(k + kStages - 1);
-    const uint8_t* st = smraw + (size_t)(k % kStages) * kStageBytes;
-    const int32_t* sa = reinterpret_cast<const int32_t*>(st + kAccT * RB);
-    int aj[kAccT / 32];
-#pragma unroll
-    for (int q = 0; q < kAccT / 32; ++q) aj[q] = sa[32 * q + lane];
+    const int st = k % kStages;
+    if (k + 1 < nt) load_aj(k + 1, ajn);
+    const bool ok = mb_wait(&full[st], (uint32_t)((k / kStages) & 1));
+    if (!__all_sync(kFull, ok)) break;
+    const uint8_t* stg = smraw + (size_t)st * kStageBytes;
 #pragma unroll
     for (int c = 0; c < CPW; ++c) {
       const int j = warp + kAccWarps * c;
@@ -618,7 +671,7 @@ __global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, in
         while (m) {
           const int t = 32 * q + __ffs(m) - 1;
           m &= m - 1;
-          const uint8_t* row = st + t * RB + lane * (E * ES);
+          const uint8_t* row = stg + t * RB + lane * (E * ES);
           float v[E];
           if constexpr (ES == 4) {
             if constexpr (E == 4) { const float4 f = *reinterpret_cast<const float4*>(row); v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w; }
@@ -644,8 +697,11 @@ __global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, in
         }
       }
     }
+    __syncwarp();
+    if (lane == 0) mb_arrive(&empty[st]);
+#pragma unroll
+    for (int q = 0; q < kAccT / 32; ++q) aj[q] = ajn[q];
   }
-  cp_async_wait<0>();
 
   double* gs = sums + (size_t)prob * P * kD + slice * CW + lane * E;
 #pragma unroll
@@ -661,12 +717,12 @@ __global__ void __launch_bounds__(kAccWarps * 32, 1) mine_accum_kernel(Src s, in
 
 template <int CPW, int E, int ES>
 constexpr size_t accum_smem() {
-  return (size_t)(ES == 2 ? 4 : 3) * (kAccT * 32 * E * ES + kAccT * 4);
+  return (size_t)accum_stages<32 * E * ES>() * (kAccT * 32 * E * ES) + 2 * 4 * sizeof(uint64_t);
 }
 
 template <int CPW, int E, int ES>
-cudaError_t launch_accum_t(const Src& s, int P, int NP, int sms, const int32_t* assign, double* sums, uint32_t* cnt,
-                           cudaStream_t st) {
+cudaError_t launch_accum_t(const CUtensorMap& amap, const Src& s, int P, int NP, int sms, const int32_t* assign,
+                           double* sums, uint32_t* cnt, cudaStream_t st) {
   constexpr size_t smem = accum_smem<CPW, E, ES>();
   cudaError_t e = cudaFuncSetAttribute(mine_accum_kernel<CPW, E, ES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -675,54 +731,67 @@ cudaError_t launch_accum_t(const Src& s, int P, int NP, int sms, const int32_t* 
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
   const int64_t want = std::max<int64_t>(1, sms / std::max(1, slices * NP));
   const unsigned chunks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, want));
-  mine_accum_kernel<CPW, E, ES><<<dim3(chunks, slices, NP), kAccWarps * 32, smem, st>>>(s, P, assign, sums, cnt);
+  mine_accum_kernel<CPW, E, ES><<<dim3(chunks, slices, NP), (kAccWarps + 1) * 32, smem, st>>>(amap, s, P, assign,
+                                                                                              sums, cnt);
   return cudaGetLastError();
 }
 
 // P <= 64: one 128-channel slice, 4 clusters per warp; P <= 128: two 64-channel slices, 8
 // clusters per warp; P <= 256: four 32-channel slices, 16 clusters per warp
-cudaError_t launch_accum(const Src& s, int P, int NP, int sms, const int32_t* assign, double* sums, uint32_t* cnt,
-                         cudaStream_t st) {
+int accum_slice_channels(int P) { return P <= 4 * kAccWarps ? 128 : (P <= 8 * kAccWarps ? 64 : 32); }
+
+cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, int sms, const int32_t* assign,
+                         double* sums, uint32_t* cnt, cudaStream_t st) {
   const bool f32 = s.y != nullptr;
   if (P <= 4 * kAccWarps)
-    return f32 ? launch_accum_t<4, 4, 4>(s, P, NP, sms, assign, sums, cnt, st)
-               : launch_accum_t<4, 4, 2>(s, P, NP, sms, assign, sums, cnt, st);
+    return f32 ? launch_accum_t<4, 4, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
+               : launch_accum_t<4, 4, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
   if (P <= 8 * kAccWarps)
-    return f32 ? launch_accum_t<8, 2, 4>(s, P, NP, sms, assign, sums, cnt, st)
-               : launch_accum_t<8, 2, 2>(s, P, NP, sms, assign, sums, cnt, st);
-  return f32 ? launch_accum_t<16, 1, 4>(s, P, NP, sms, assign, sums, cnt, st)
-             : launch_accum_t<16, 1, 2>(s, P, NP, sms, assign, sums, cnt, st);
+    return f32 ? launch_accum_t<8, 2, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
+               : launch_accum_t<8, 2, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
+  return f32 ? launch_accum_t<16, 1, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
+             : launch_accum_t<16, 1, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
 }
 
 // ---- tcgen05 assignment (bf16 input, P <= 128) ------------------------------------------
 //
 // The same certified argmin as mine_assign_mma_kernel, with the distance contraction on
-// the 5th-generation tensor cores: per 128-token tile, one thread issues 8 MMAs of
-// M = 128 (tokens) x N = 2 Pn (the bf16 hi parts of the Pn padded patterns, then their mid
-// parts) x K = 16 into a TMEM accumulator, so each product term keeps its own fp32 chain
-// of 8 MMAs (the error model of the certification above).  Tiles reach shared memory
-// through cp.async in the canonical K-major layout without swizzle (8-row x 16-byte core
-// matrices; LBO = 128 B between core matrices along K, SBO = 2048 B between 8-row groups);
-// the accumulators are double-buffered in TMEM, so the MMAs of tile k overlap the epilogue
-// of tile k - 1, in which thread t reads row t (token t) back with tcgen05.ld, adds the
-// two chains, and runs the gap test.  A token that fails it re-reads its scores (the whole
-// warp, tcgen05.ld is warp-collective) and is decided exactly in float64.
+// the 5th-generation tensor cores, as a warp-specialised pipeline with no block barrier in
+// its loop (one CTA per SM; roles hand stages and accumulators over through mbarriers):
+//   * producer warp: per 128-token tile, two TMA loads (a box of 64 channels x 128 tokens
+//     each, 4-D tensor map over channels x heads x tokens x sets, 128-byte swizzle; rows past
+//     the end read as zeros) into a ring of shared-memory stages: the canonical K-major
+//     layout with 128-byte swizzle, 8-row x 128-byte atoms (SBO = 1024 B), channels 0-63
+//     and 64-127 in two 16 KB halves;
+//   * MMA warp (one thread): 8 tcgen05.mma of M = 128 (tokens) x N = 2 Pn (the bf16 hi parts
+//     of the Pn padded patterns, then their mid parts) x K = 16, fp32 accumulation in one of
+//     two TMEM buffers, so each product term keeps its own chain of 8 MMAs (the error model
+//     of the certification above); commits to the buffer's "full" and the stage's "free"
+//     barriers;
+//   * 8 epilogue warps, two warpgroups: warpgroup g owns TMEM buffer g and takes every other
+//     tile; token t's scores are TMEM lane t, so each warp handles its 32 tokens alone (top-2
+//     over all patterns, |x|^2 from the staged tile, the gap test and, for a token that fails
+//     it, the float64 recomputation of its candidates), with no barrier between warps.
+// Every mbarrier wait is bounded.
 constexpr int kTcM = 128;
-constexpr int kTcStages = 2;
+constexpr int kTcMaxStages = 6;
 constexpr int kTcTileBytes = kTcM * kD * 2;
-constexpr uint32_t kTcLBO = 128, kTcSBO = 2048;
-constexpr uint32_t kTcSpinLimit = 1u << 24;
-
-__host__ __device__ constexpr uint32_t kmaj_off(int row, int k) {
-  return (uint32_t)(row >> 3) * kTcSBO + (uint32_t)(k >> 3) * kTcLBO + (uint32_t)(row & 7) * 16u + (uint32_t)(k & 7) * 2u;
-}
+constexpr uint32_t kTcSpinLimit = 1u << 22;
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
 
 __device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// shared-memory matrix descriptor: start, LBO, SBO (all >> 4), descriptor version 1, no swizzle
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((kTcLBO >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((kTcSBO >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+// shared-memory matrix descriptor, K-major with 128-byte swizzle: start (bytes >> 4), LBO unused
+// (1), SBO = 1024 B between 8-row atoms, descriptor version 1, layout type 2 (128-byte swizzle).
+// The start may move by 32 B per K = 16 step inside an atom; atoms are 1024-byte aligned.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+// byte offset of (row, 16-byte chunk c of the 128-byte atom row) in a 128-byte-swizzled block
+__host__ __device__ constexpr uint32_t sw128_off(int row, int c) {
+  return (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u + (uint32_t)((c ^ (row & 7)) * 16);
 }
 // instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, N >> 3, M >> 4
 __host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
@@ -760,10 +829,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tc_mbar_init(uint64_t* bar) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(bar)) : "memory");
-}
-__device__ __forceinline__ bool tc_mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t it = 0; it < kTcSpinLimit; ++it) {
     uint32_t ok;
     asm volatile(
@@ -776,22 +842,29 @@ __device__ __forceinline__ bool tc_mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
-__global__ void __launch_bounds__(256, 2) mine_assign_tc_kernel(Src s, int P, const float* __restrict__ M,
-                                                                 int32_t* __restrict__ assign, int32_t* status) {
+
+__global__ void __launch_bounds__(kTcThreads, 1) mine_assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s,
+                                                                      int P, const float* __restrict__ M,
+                                                                      int32_t* __restrict__ assign, int nst) {
   const int prob = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Pn = (P + 7) & ~7, N = 2 * Pn;
   const uint32_t tcols = N <= 128 ? 256u : 512u;  // two accumulator buffers
   const uint32_t buf_cols = tcols / 2;
+  const uint32_t half_b = (uint32_t)N * 128u;      // B: channels 64-127 start N x 128 B in
   extern __shared__ __align__(16) uint8_t smraw[];
-  uint8_t* Bt = smraw;                                                   // [N][128] bf16, canonical K-major
-  uint8_t* At = smraw + (size_t)N * kD * 2;                              // [stages][128][128] bf16
-  float* msq = reinterpret_cast<float*>(At + (size_t)kTcStages * kTcTileBytes);  // [Pn]
-  float* mnorm = msq + Pn;                                               // [Pn]
-  float* gmax = mnorm + Pn;                                              // [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);                // [2] (16-byte aligned: Pn % 8 == 0)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2);
-  float* xch = reinterpret_cast<float*>(tslot + 4);  // [4][128]: warpgroup 1's m1, m2, j1, partial |x|^2
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Bt = base;                                                   // [2 halves][N rows][128 B], swizzled
+  uint8_t* At = base + (size_t)N * kD * 2;                              // [nst][2 halves][128 rows][128 B]
+  float* msq = reinterpret_cast<float*>(At + (size_t)nst * kTcTileBytes);  // [Pn]
+  float* mnorm = msq + Pn;                                              // [Pn]
+  float* gmax = mnorm + Pn;                                             // [4]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);               // full[nst], sfree[nst], tfull[2], tempty[2]
+  uint64_t* full = bars;
+  uint64_t* sfree = bars + nst;
+  uint64_t* tfull = bars + 2 * nst;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
   const float* Mp = M + (size_t)prob * P * kD;
   const int set = prob / s.heads, h = prob % s.heads;
 
@@ -812,16 +885,23 @@ __global__ void __launch_bounds__(256, 2) mine_assign_tc_kernel(Src s, int P, co
       }
       wv[q] = (uint32_t)hv[0] | ((uint32_t)hv[1] << 16);
     }
-    *reinterpret_cast<uint4*>(Bt + kmaj_off(n, 8 * c)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    *reinterpret_cast<uint4*>(Bt + (size_t)(c >> 3) * half_b + sw128_off(n, c & 7)) =
+        make_uint4(wv[0], wv[1], wv[2], wv[3]);
   }
   if (tid == 0) {
     gmax[0] = 0.f;
     gmax[1] = 0.f;
-    tc_mbar_init(&bars[0]);
-    tc_mbar_init(&bars[1]);
+    for (int i = 0; i < nst; ++i) {
+      mb_init(&full[i], 1);
+      mb_init(&sfree[i], 1 + kTcEpiWarps / 2);  // the MMA commit and the 4 warps of the tile's warpgroup
+    }
+    for (int i = 0; i < 2; ++i) {
+      mb_init(&tfull[i], 1);
+      mb_init(&tempty[i], kTcEpiWarps / 2);  // buffer i belongs to warpgroup i
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tslot)), "r"(tcols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -841,202 +921,173 @@ __global__ void __launch_bounds__(256, 2) mine_assign_tc_kernel(Src s, int P, co
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const float nm_max = gmax[0], msq_max = gmax[1];
-  const uint32_t idesc = umma_idesc(kTcM, N);
 
   const int64_t ntiles = (s.n + kTcM - 1) / kTcM;
   const int nt = ntiles > blockIdx.x ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
   auto tile_t0 = [&](int k) { return ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * kTcM; };
-  auto load_tile = [&](int k) {
-    if (k < nt) {
-      const int64_t t0 = tile_t0(k);
-      uint8_t* st = At + (size_t)(k % kTcStages) * kTcTileBytes;
-      // a warp writes 8 rows x 4 chunks: four contiguous 128-byte runs, no bank conflicts
-      for (int i = tid; i < kTcM * 16; i += blockDim.x) {
-        const int r = ((i >> 7) << 3) | (i & 7), c = (i >> 3) & 15;
-        const int64_t tok = t0 + r;
-        uint8_t* dst = st + kmaj_off(r, 8 * c);
-        if (tok < s.n) cp_async16(dst, s.x + set * s.ss + tok * s.ts + h * s.hs + 8 * c);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+
+  if (warp == 0) {
+    // ---- producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      for (int k = 0; k < nt; ++k) {
+        const int st = k % nst;
+        if (k >= nst && !tc_wait(&sfree[st], (uint32_t)(((k / nst) - 1) & 1))) break;
+        uint8_t* dst = At + (size_t)st * kTcTileBytes;
+        mb_expect_tx(&full[st], (uint32_t)kTcTileBytes);
+        const int t0 = (int)tile_t0(k);
+        tma_load_4d(dst, &xmap, 0, h, t0, set, &full[st]);
+        tma_load_4d(dst + kTcTileBytes / 2, &xmap, 64, h, t0, set, &full[st]);
       }
     }
-    cp_async_commit();
-  };
-
-  bool ok_all = true;
-  // epilogue of tile k; once its MMAs are complete, the copy of tile k + 2 goes into its stage
-  auto epilogue = [&](int k, float xsq_raw) {
-    const int buf = k & 1;
-    const bool ok = tc_mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1));
-    load_tile(k + 2);
-    // the same verdict for every thread of the CTA (barriers follow)
-    if (!__syncthreads_and(ok)) {  // the accumulator never arrived: flag it and skip the tile
-      ok_all = false;
-      return;
+  } else if (warp == 1) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc(kTcM, N);
+      const uint32_t b0 = su32(Bt);
+      for (int k = 0; k < nt; ++k) {
+        const int st = k % nst, buf = k & 1;
+        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1))) break;
+        if (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t a0 = su32(At + (size_t)st * kTcTileBytes);
+        const uint32_t d = tbase + (uint32_t)buf * buf_cols;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks)  // K step ks: half ks / 4, 32 B per step inside the atom
+          umma_bf16(d, umma_desc_sw128(a0 + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32),
+                    umma_desc_sw128(b0 + (ks >> 2) * half_b + (ks & 3) * 32), idesc, ks > 0);
+        umma_commit(&tfull[buf]);
+        umma_commit(&sfree[st]);
+      }
     }
-    tc_fence_after();
-    const int wg = warp >> 2, q4 = warp & 3;  // warpgroup: which 32-column blocks; q4: TMEM lane quarter
+  } else {
+    // ---- epilogue warps: warpgroup g takes tiles k with k % 2 == g, i.e. TMEM buffer g, each
+    // warp its 32 rows, with no barrier between warps
+    const int ew = warp - 2, wg = ew >> 2, q4 = warp & 3;  // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;
-    const int64_t i = tile_t0(k) + row;
-    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)buf * buf_cols;
-    Top2 top{INFINITY, INFINITY, 0}, top_b{INFINITY, INFINITY, 0};  // even / odd patterns: two chains
-    for (int c0 = 32 * wg; c0 < Pn; c0 += 64) {
-      float hv[32], mv[32];
-      tmem_ld32(taddr + c0, hv);
-      tmem_ld32(taddr + Pn + c0, mv);
+    const float nm_max = gmax[0], msq_max = gmax[1];
+    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)wg * buf_cols;
+    for (int k = wg; k < nt; k += 2) {
+      const int st = k % nst;
+      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) break;
+      tc_fence_after();
+      // |x|^2 of the row from the staged tile (two swizzled halves of 64 channels)
+      float xs[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* stg = At + (size_t)st * kTcTileBytes;
 #pragma unroll
-      for (int q = 0; q < 32; q += 2) {
-        const int j = c0 + q;
-        if (j < P) top2_add(top, msq[j] - 2.0f * (hv[q] + mv[q]), j);
-        if (j + 1 < P) top2_add(top_b, msq[j + 1] - 2.0f * (hv[q + 1] + mv[q + 1]), j + 1);
+      for (int hc = 0; hc < 16; ++hc) {
+        const uint4 u = *reinterpret_cast<const uint4*>(stg + (hc >> 3) * (kTcTileBytes / 2) + sw128_off(row, hc & 7));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
+          xs[q] = fmaf(v0, v0, xs[q]);
+          xs[q] = fmaf(v1, v1, xs[q]);
+        }
       }
-    }
-    // merge (lower index wins equal minima)
-    if (top_b.m1 < top.m1 || (top_b.m1 == top.m1 && top_b.j1 < top.j1)) {
-      top.m2 = fminf(top.m1, top_b.m2);
-      top.m1 = top_b.m1;
-      top.j1 = top_b.j1;
-    } else {
-      top.m2 = fminf(top.m2, top_b.m1);
-    }
-    // warpgroup 1 hands its partial results to warpgroup 0, which decides the row
-    if (wg == 1) {
-      xch[0 * kTcM + row] = top.m1;
-      xch[1 * kTcM + row] = top.m2;
-      xch[2 * kTcM + row] = __int_as_float(top.j1);
-      xch[3 * kTcM + row] = xsq_raw;
-    }
-    __syncthreads();
-    if (wg == 1) {
-      tc_fence_before();
-      return;
-    }
-    {
-      const float om1 = xch[0 * kTcM + row], om2 = xch[1 * kTcM + row];
-      const int oj = __float_as_int(xch[2 * kTcM + row]);
-      const float lo2 = fminf(top.m2, om2);
-      if (om1 < top.m1 || (om1 == top.m1 && oj < top.j1)) { top.m2 = fminf(top.m1, lo2); top.m1 = om1; top.j1 = oj; }
-      else top.m2 = fminf(om1, lo2);
-    }
-    float xsq = xsq_raw + xch[3 * kTcM + row];
-    xsq *= (1.0f + 1e-6f);
-    const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
-    const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xsq + msq_max);
-    const bool unique = top.m2 - top.m1 > 2.0f * Eb + 1e-9f * (xsq + msq_max);
-    if (unique && i < s.n) assign[(size_t)prob * s.n + i] = top.j1;
-    const bool need = !unique && i < s.n;
-    if (__any_sync(kFull, need)) {
-      // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
-      float U = INFINITY;
+      __syncwarp();
+      if (lane == 0) mb_arrive(&sfree[st]);
+      Top2 top{INFINITY, INFINITY, 0}, top_b{INFINITY, INFINITY, 0};  // even / odd patterns: two chains
       for (int c0 = 0; c0 < Pn; c0 += 32) {
         float hv[32], mv[32];
         tmem_ld32(taddr + c0, hv);
         tmem_ld32(taddr + Pn + c0, mv);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 32; q += 2) {
           const int j = c0 + q;
-          if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
+          if (j < P) top2_add(top, msq[j] - 2.0f * (hv[q] + mv[q]), j);
+          if (j + 1 < P) top2_add(top_b, msq[j + 1] - 2.0f * (hv[q + 1] + mv[q + 1]), j + 1);
         }
       }
-      uint32_t cand[4] = {0u, 0u, 0u, 0u};  // candidate bit mask over j < 128
-      for (int c0 = 0; c0 < Pn; c0 += 32) {
-        float hv[32], mv[32];
-        tmem_ld32(taddr + c0, hv);
-        tmem_ld32(taddr + Pn + c0, mv);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = c0 + q;
-          const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
-          const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
-          if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cand[c0 >> 5] |= 1u << q;
-        }
+      if (top_b.m1 < top.m1 || (top_b.m1 == top.m1 && top_b.j1 < top.j1)) {
+        top.m2 = fminf(top.m1, top_b.m2);
+        top.m1 = top_b.m1;
+        top.j1 = top_b.j1;
+      } else {
+        top.m2 = fminf(top.m2, top_b.m1);
       }
-      if (need) {
-        const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
-        double bd = 0.0;
-        int bj = 0;
-        bool have = false;
-        for (int cw = 0; cw < 4; ++cw)
-          for (uint32_t m = cand[cw]; m; m &= m - 1) {
-            const int j = cw * 32 + __ffs(m) - 1;
-            const float* mrow = Mp + (size_t)j * kD;
-            double acc = 0.0;
-#pragma unroll 8
-            for (int d = 0; d < kD; d += 4) {
-              const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
-              const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                   __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-              const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
-              const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
+      const int64_t i = tile_t0(k) + row;
+      const float xsq = ((xs[0] + xs[1]) + (xs[2] + xs[3])) * (1.0f + 1e-6f);
+      const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
+      const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xsq + msq_max);
+      const bool unique = top.m2 - top.m1 > 2.0f * Eb + 1e-9f * (xsq + msq_max);
+      if (unique && i < s.n) assign[(size_t)prob * s.n + i] = top.j1;
+      const bool need = !unique && i < s.n;
+      if (__any_sync(kFull, need)) {
+        // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
+        float U = INFINITY;
+        for (int c0 = 0; c0 < Pn; c0 += 32) {
+          float hv[32], mv[32];
+          tmem_ld32(taddr + c0, hv);
+          tmem_ld32(taddr + Pn + c0, mv);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
-                acc = __dadd_rn(acc, __dmul_rn(t, t));
-              }
-            }
-            if (!have || acc < bd) { bd = acc; bj = j; have = true; }
+          for (int q = 0; q < 32; ++q) {
+            const int j = c0 + q;
+            if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
           }
-        assign[(size_t)prob * s.n + i] = bj;
+        }
+        uint32_t cand[4] = {0u, 0u, 0u, 0u};  // candidate bit mask over j < 128
+        for (int c0 = 0; c0 < Pn; c0 += 32) {
+          float hv[32], mv[32];
+          tmem_ld32(taddr + c0, hv);
+          tmem_ld32(taddr + Pn + c0, mv);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int j = c0 + q;
+            const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
+            const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
+            if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cand[c0 >> 5] |= 1u << q;
+          }
+        }
+        if (need) {
+          const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
+          double bd = 0.0;
+          int bj = 0;
+          bool have = false;
+          for (int cw = 0; cw < 4; ++cw)
+            for (uint32_t m = cand[cw]; m; m &= m - 1) {
+              const int j = cw * 32 + __ffs(m) - 1;
+              const float* mrow = Mp + (size_t)j * kD;
+              double acc = 0.0;
+#pragma unroll 8
+              for (int d = 0; d < kD; d += 4) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
+                const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+                const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
+                const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
+                  acc = __dadd_rn(acc, __dmul_rn(t, t));
+                }
+              }
+              if (!have || acc < bd) { bd = acc; bj = j; have = true; }
+            }
+          assign[(size_t)prob * s.n + i] = bj;
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mb_arrive(&tempty[wg]);
     }
-    tc_fence_before();
-  };
-
-  // |x|^2 of this thread's row of tile k, from its stage (read while the MMAs read it too)
-  auto row_norm = [&](int k) {  // half of the row's channels per warpgroup
-    const uint8_t* st = At + (size_t)(k % kTcStages) * kTcTileBytes;
-    const int row = (warp & 3) * 32 + lane, c0 = 8 * (warp >> 2);
-    float xs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int c = c0; c < c0 + 8; ++c) {
-      const uint4 u = *reinterpret_cast<const uint4*>(st + kmaj_off(row, 8 * c));
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
-        xs[q] = fmaf(v0, v0, xs[q]);
-        xs[q] = fmaf(v1, v1, xs[q]);
-      }
-    }
-    return (xs[0] + xs[1]) + (xs[2] + xs[3]);
-  };
-
-  // stage s holds tile k with k % 2 == s; the copy of tile k + 2 starts once tile k's MMAs are done
-  load_tile(0);
-  load_tile(1);
-  float xsq_prev = 0.f;
-  for (int k = 0; k < nt; ++k) {
-    // this thread's copies of tile k: the newest group, except at k = 0 (tile 1 is newer)
-    if (k == 0) cp_async_wait<1>();
-    else cp_async_wait<0>();
-    fence_proxy_async();
-    __syncthreads();  // all copies of tile k; the epilogue of tile k - 2 (same TMEM buffer) is done
-    tc_fence_after();
-    if (tid == 0 && ok_all) {
-      const uint32_t a0 = su32(At + (size_t)(k % kTcStages) * kTcTileBytes), b0 = su32(Bt);
-      const uint32_t d = tbase + (uint32_t)(k & 1) * buf_cols;
-#pragma unroll
-      for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(d, umma_desc(a0 + ks * 256), umma_desc(b0 + ks * 256), idesc, ks > 0);
-      umma_commit(&bars[k & 1]);
-    }
-    const float xsq_k = row_norm(k);
-    if (k > 0 && ok_all) epilogue(k - 1, xsq_prev);
-    else if (k > 0) load_tile(k + 1);
-    xsq_prev = xsq_k;
   }
-  if (nt > 0 && ok_all) epilogue(nt - 1, xsq_prev);
-  cp_async_wait<0>();
-  if (!ok_all && lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
+  if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
 }
 
-size_t mine_tc_smem(int P) {
+// ring depth that fits next to the patterns in 227 KB, and the dynamic shared memory it needs
+int mine_tc_stages(int P) {
   const int Pn = (P + 7) & ~7;
-  return (size_t)2 * Pn * kD * 2 + (size_t)kTcStages * kTcTileBytes + 2 * Pn * 4 + 16 + 16 + 16 + 4 * kTcM * 4 + 1024;
+  const int fixed = 2 * Pn * kD * 2 + 2 * Pn * 4 + 16 + (2 * kTcMaxStages + 4) * 8 + 16 + 1024;
+  return std::max(2, std::min(kTcMaxStages, (227 * 1024 - fixed) / kTcTileBytes));
+}
+size_t mine_tc_smem(int P) {
+  const int Pn = (P + 7) & ~7, nst = mine_tc_stages(P);
+  return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + 2 * Pn * 4 + 16 + (2 * nst + 4) * 8 + 16 + 1024;
 }
 
 __global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt) {
@@ -1059,6 +1110,48 @@ size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
     b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
          4 * align256(NP * kD * sizeof(double));
   return b + 256;
+}
+
+// Tiled TMA tensor maps (no swizzle; loads past the end read as zeros).  cuTensorMapEncodeTiled
+// comes from the driver through the runtime's entry-point query.
+static cudaError_t encode_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = encode(map, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The 16-bit input as (128 channels, heads, tokens, sets) with a box of `box_ch` channels x 1
+// head x 128 tokens x 1 set.
+static cudaError_t make_x_map(const MineArgs& a, CUtensorMap* map, int box_ch,
+                              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.heads, (cuuint64_t)a.n, (cuuint64_t)a.sets};
+  const cuuint64_t strides[3] = {(cuuint64_t)a.head_stride * 2, (cuuint64_t)a.tok_stride * 2,
+                                 (cuuint64_t)std::max<int64_t>(a.set_stride, 8) * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)box_ch, 1, 128, 1};
+  return encode_map(map, a.dtype == KVQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                    a.x, dims, strides, box, swz);
+}
+
+// The fp32 pre-transformed rows y [problems][n][128] as (128 channels, tokens, problems) with a
+// box of `box_ch` channels x 128 tokens x 1 problem.
+static cudaError_t make_y_map(const float* y, int64_t n, int NP, CUtensorMap* map, int box_ch) {
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)NP};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 4, (cuuint64_t)n * kD * 4};
+  const cuuint32_t box[3] = {(cuuint32_t)box_ch, 128, 1};
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y, dims, strides, box);
 }
 
 cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -1108,19 +1201,29 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   const int tok_per_cta = kMmaWarps * (KIND == 0 ? 32 : 16);
   const unsigned mma_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + tok_per_cta - 1) / tok_per_cta, (int64_t)(2 * sms + NP - 1) / NP));
-  // bf16 input and P <= 128: the tcgen05 kernel, two CTAs (each with 256 TMEM columns) per SM
+  // the cluster-sum kernel reads tiles of 128 rows through a tensor map (x, or the pre-transformed y)
+  CUtensorMap amap;
+  if ((e = a.transform ? make_y_map(w.y, a.n, NP, &amap, accum_slice_channels(a.P))
+                       : make_x_map(a, &amap, accum_slice_channels(a.P))) != cudaSuccess)
+    return e;
+  // bf16 input and P <= 128: the tcgen05 kernel, one CTA (copy ring, 256 or 512 TMEM columns) per SM,
+  // reading x through a 4-D tensor map (channels, heads, tokens, sets)
   const bool use_tc = KIND == 0 && a.P <= kMmaMaxP;
   const size_t smem_tc = mine_tc_smem(a.P);
-  if (use_tc &&
-      (e = cudaFuncSetAttribute(mine_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_tc)) !=
-          cudaSuccess)
-    return e;
+  CUtensorMap xmap;
+  if (use_tc) {
+    if ((e = cudaFuncSetAttribute(mine_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem_tc)) != cudaSuccess)
+      return e;
+    if ((e = make_x_map(a, &xmap, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+  }
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
-      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, 2 * sms / NP)));
+      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
     if (use_tc)
-      mine_assign_tc_kernel<<<dim3(tc_ctas, NP), 256, smem_tc, st>>>(s, a.P, a.patterns, w.assign, nullptr);
+      mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(xmap, s, a.P, a.patterns, w.assign,
+                                                                             mine_tc_stages(a.P));
     else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else if (use_mma && KIND == 1)
@@ -1130,7 +1233,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     else
       mine_assign_kernel<<<dim3((unsigned)((a.n + 127) / 128), NP), 128, smem_assign, st>>>(s, a.P, a.patterns,
                                                                                            w.assign);
-    if ((e = launch_accum(s, a.P, NP, sms, w.assign, w.sums, w.cnt, st)) != cudaSuccess) return e;
+    if ((e = launch_accum(amap, s, a.P, NP, sms, w.assign, w.sums, w.cnt, st)) != cudaSuccess) return e;
     mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
   }
   return cudaGetLastError();

@@ -193,9 +193,9 @@ KVQ_API kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, in
  * reaches 32 tokens is quantized per channel and written to its page.  seq_len is
  * advanced by n_new (a sequence that would overflow its page table is left
  * unchanged and flags KVQ_DEV_OVERFLOW).  n_new = 0 is a no-op.
- * Workspace: kvq_append_workspace_bytes() (per-call pattern tables: bf16 copies and
- * the pattern-to-pattern min-max distances used to prune the exact assignment; about
- * 20 KB + 4 P^2 B per (set, KV head) and K / V); 256-byte aligned.
+ * Workspace: kvq_append_workspace_bytes() (per-call pattern tables: the 32 channels whose
+ * values differ most across the patterns and every pattern's values there, used to prune
+ * the exact assignment; 128 + 128 P bytes per (set, KV head) and K / V); 256-byte aligned.
  */
 KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache* cache, int32_t n_new);
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new, int32_t n_new,
