@@ -774,7 +774,7 @@ cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, i
 //     it, the float64 recomputation of its candidates), with no barrier between warps.
 // Every mbarrier wait is bounded.
 constexpr int kTcM = 128;
-constexpr int kTcMaxStages = 6;
+constexpr int kTcMaxStages = 2;  // two CTAs per SM share the SM's shared memory and TMEM
 constexpr int kTcTileBytes = kTcM * kD * 2;
 constexpr uint32_t kTcSpinLimit = 1u << 22;
 constexpr int kTcEpiWarps = 8;
@@ -813,21 +813,16 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+// 8 consecutive fp32 columns of this thread's TMEM lane, without waiting (tmem_ld_wait() before use)
+__device__ __forceinline__ void tmem_ld8_issue(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t it = 0; it < kTcSpinLimit; ++it) {
@@ -843,7 +838,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
 }
 
 
-__global__ void __launch_bounds__(kTcThreads, 1) mine_assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s,
+__global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s,
                                                                       int P, const float* __restrict__ M,
                                                                       int32_t* __restrict__ assign, int nst) {
   const int prob = blockIdx.y;
@@ -988,15 +983,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) mine_assign_tc_kernel(const __g
       __syncwarp();
       if (lane == 0) mb_arrive(&sfree[st]);
       Top2 top{INFINITY, INFINITY, 0}, top_b{INFINITY, INFINITY, 0};  // even / odd patterns: two chains
-      for (int c0 = 0; c0 < Pn; c0 += 32) {
-        float hv[32], mv[32];
-        tmem_ld32(taddr + c0, hv);
-        tmem_ld32(taddr + Pn + c0, mv);
+      // 8 columns at a time; the loads of block c0 + 8 are in flight while block c0 is scored
+      float hv[8], mv[8];
+      tmem_ld8_issue(taddr, hv);
+      tmem_ld8_issue(taddr + Pn, mv);
+      tmem_ld_wait();
+      for (int c0 = 0; c0 < Pn; c0 += 8) {
+        float hn[8], mn_[8];
+        const bool more = c0 + 8 < Pn;
+        if (more) {
+          tmem_ld8_issue(taddr + c0 + 8, hn);
+          tmem_ld8_issue(taddr + Pn + c0 + 8, mn_);
+        }
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) {
+        for (int q = 0; q < 8; q += 2) {
           const int j = c0 + q;
           if (j < P) top2_add(top, msq[j] - 2.0f * (hv[q] + mv[q]), j);
           if (j + 1 < P) top2_add(top_b, msq[j + 1] - 2.0f * (hv[q + 1] + mv[q + 1]), j + 1);
+        }
+        if (more) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) { hv[q] = hn[q]; mv[q] = mn_[q]; }
         }
       }
       if (top_b.m1 < top.m1 || (top_b.m1 == top.m1 && top_b.j1 < top.j1)) {
@@ -1016,28 +1024,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) mine_assign_tc_kernel(const __g
       if (__any_sync(kFull, need)) {
         // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
         float U = INFINITY;
-        for (int c0 = 0; c0 < Pn; c0 += 32) {
-          float hv[32], mv[32];
-          tmem_ld32(taddr + c0, hv);
-          tmem_ld32(taddr + Pn + c0, mv);
+        for (int c0 = 0; c0 < Pn; c0 += 8) {
+          float hv[8], mv[8];
+          tmem_ld8_issue(taddr + c0, hv);
+          tmem_ld8_issue(taddr + Pn + c0, mv);
+          tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < 8; ++q) {
             const int j = c0 + q;
             if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
           }
         }
         uint32_t cand[4] = {0u, 0u, 0u, 0u};  // candidate bit mask over j < 128
-        for (int c0 = 0; c0 < Pn; c0 += 32) {
-          float hv[32], mv[32];
-          tmem_ld32(taddr + c0, hv);
-          tmem_ld32(taddr + Pn + c0, mv);
+        for (int c0 = 0; c0 < Pn; c0 += 8) {
+          float hv[8], mv[8];
+          tmem_ld8_issue(taddr + c0, hv);
+          tmem_ld8_issue(taddr + Pn + c0, mv);
+          tmem_ld_wait();
+          uint32_t cm = 0u;
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < 8; ++q) {
             const int j = c0 + q;
             const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
             const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
-            if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cand[c0 >> 5] |= 1u << q;
+            if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cm |= 1u << q;
           }
+          cand[c0 >> 5] |= cm << (c0 & 31);
         }
         if (need) {
           const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
@@ -1218,7 +1230,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     if ((e = make_x_map(a, &xmap, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
-      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, sms / NP)));
+      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, (a.P <= 64 ? 2 : 1) * sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
     if (use_tc)
