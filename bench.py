@@ -133,27 +133,36 @@ class ClockSampler:
 # CPU baseline: the oracle, as it stands, on a bounded sample of the workload.
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(w, sample_tokens: int = 4096):
+def cpu_baseline(w, heads: int = 4, seqs: int | None = None):
+    """The oracle, as it stands, on a bounded sample of the workload: every sequence (or the
+    first `seqs`) of `heads` of the KV heads, the whole path (mining of K and V on the pooled
+    prefill, encoding, decode attention of each sequence's query heads), scaled to KV-tokens/s
+    of the whole job (all KV heads)."""
     import numpy as np
 
     import oracle
     import synth
 
-    sw = w.with_(B=1, S=sample_tokens)
-    k, v = synth.gen_kv(sw, 0, 1, 0, sample_tokens)
-    Kf, Vf = synth.to_float(k, w.dtype)[0, :, 0], synth.to_float(v, w.dtype)[0, :, 0]
-    q = synth.to_float(synth.gen_q(sw, b0=0, b1=1), w.dtype)[0, : w.Hq // w.Hkv]
+    B = w.B if seqs is None else min(seqs, w.B)
+    heads = max(1, min(heads, w.Hkv))
+    sw = w.with_(B=B)
+    k, v = synth.gen_kv(sw)
+    q = synth.gen_q(sw)
+    Gq = w.Hq // w.Hkv
     t0 = time.perf_counter()
-    MK, cK, _ = oracle.mine_set(Kf, w.P, w.iters, w.transform)
-    MV, cV, _ = oracle.mine_set(Vf, w.P, w.iters, w.transform)
-    e = oracle.encode(Kf, Vf, w.bits, MK, MV, cK, cV)
-    oracle.attention_unit(q, Kf, e, MK, MV, cK, cV)
+    for h in range(heads):
+        Kf, Vf = synth.to_float(k[:, :, h], w.dtype), synth.to_float(v[:, :, h], w.dtype)
+        MK, cK, _ = oracle.mine_set(Kf.reshape(-1, D), w.P, w.iters, w.transform)
+        MV, cV, _ = oracle.mine_set(Vf.reshape(-1, D), w.P, w.iters, w.transform)
+        for b in range(B):
+            e = oracle.encode(Kf[b], Vf[b], w.bits, MK, MV, cK, cV)
+            qf = synth.to_float(q[b, h * Gq:(h + 1) * Gq], w.dtype)
+            oracle.attention_unit(qf, Kf[b], e, MK, MV, cK, cV)
     dt = time.perf_counter() - t0
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    # one KV head of sample_tokens tokens; a KV-token covers all Hkv heads
-    value = sample_tokens / (dt * w.Hkv)
-    sample = (f"oracle mine(K,V) + encode + decode attention of 1 sequence x {sample_tokens} tokens x 1 KV head "
-              f"({w.Hq // w.Hkv} query heads), scaled to KV-tokens/s over {w.Hkv} KV heads; {dt:.2f} s")
+    value = B * w.S * heads / (dt * w.Hkv)  # KV-tokens/s of the whole job: all KV heads take heads/Hkv longer
+    sample = (f"oracle mining (K and V, pooled prefill), encoding and decode attention of {B} sequences x {w.S} tokens "
+              f"for {heads} of {w.Hkv} KV heads ({Gq} query heads each), scaled to all KV heads; {dt:.2f} s")
     return {"value": value, "unit": "KV-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}, dt
 
 
@@ -169,7 +178,7 @@ def run_reference(args):
     oracle.build()
     vals, times = [], []
     for i in range(args.warmup + args.steps):
-        cb, dt = cpu_baseline(w, sample_tokens=args.ref_tokens)
+        cb, dt = cpu_baseline(w, heads=args.ref_heads, seqs=args.ref_seqs)
         if i >= args.warmup:
             vals.append(cb["value"])
             times.append(dt)
@@ -220,7 +229,8 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--bits", type=int, default=2)
-    ap.add_argument("--ref-tokens", type=int, default=65536)
+    ap.add_argument("--ref-heads", type=int, default=1, help="reference arm: KV heads per step (bounded sample)")
+    ap.add_argument("--ref-seqs", type=int, default=2, help="reference arm: sequences per step (bounded sample)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases of the same kernels, for ncu captures)")
@@ -383,7 +393,7 @@ def main():
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"], _ = cpu_baseline(w, sample_tokens=131072)
+            line["cpu_baseline"], _ = cpu_baseline(w, heads=4)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -244,7 +244,7 @@ __device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv
 }
 
 template <int BITS, int NT, int STAGES, int kWarps>
-__global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 : 3) : 2))
+__global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT == 1 ? 4 : 3) : 2))
     decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
                       float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w,
                       int* __restrict__ arrivals, float* __restrict__ out) {
@@ -336,16 +336,6 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
   }
   __syncthreads();
 
-  // query of this lane's B column (head 4j + gq/2), its 32 channels, as fp32 pairs
-  unsigned long long qreg[NT == 1 ? 8 : 1][4];
-  if constexpr (NT == 1) {
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const float4 q4 = reinterpret_cast<const float4*>(qk + (gq >> 1) * kD)[ks * 4 + tig];
-      qreg[ks][0] = pk(q4.x, q4.y);
-      qreg[ks][1] = pk(q4.z, q4.w);
-    }
-  }
 
   // ---- per-thread state (head of n-tile j: 4j + tig)
   float accv[NT][8][4];
@@ -423,13 +413,9 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
         for (int ks = 0; ks < 8; ++ks) {
           const float4 s4 = ks4[ks * 4];
           const float4 z4 = kz4[ks * 4];
-          unsigned long long qa, qb;
-          if constexpr (NT == 1) {
-            qa = qreg[ks][0]; qb = qreg[ks][1];
-          } else {
-            const float4 q4 = reinterpret_cast<const float4*>(qk + (4 * j + (gq >> 1)) * kD)[ks * 4 + tig];
-            qa = pk(q4.x, q4.y); qb = pk(q4.z, q4.w);
-          }
+          // query of this lane's B column (head 4j + gq/2), channels of k-step ks, from shared memory
+          const float4 q4 = reinterpret_cast<const float4*>(qk + (4 * j + (gq >> 1)) * kD)[ks * 4 + tig];
+          const unsigned long long qa = pk(q4.x, q4.y), qb = pk(q4.z, q4.w);
           zk2 = fma2(qa, pk(z4.x, z4.y), zk2);
           zk2 = fma2(qb, pk(z4.z, z4.w), zk2);
           const uint32_t b0 = split_bf16(mul2(qa, pk(s4.x, s4.y)), nsel);
@@ -523,9 +509,6 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
         vw[4 * c] = t.x; vw[4 * c + 1] = t.y; vw[4 * c + 2] = t.z; vw[4 * c + 3] = t.w;
       }
       const float4* vs4 = reinterpret_cast<const float4*>(pgp + g.off_vs) + tig;
-      float4 vsv[8];  // [(ks*4 + e)] -> the 4 channel groups
-#pragma unroll
-      for (int u = 0; u < 8; ++u) vsv[u] = vs4[u * 4];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         const float* prow = pex + (4 * j + (gq >> 1)) * kPexLd;
@@ -535,7 +518,9 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 ? 4 :
         for (int ks = 0; ks < 2; ++ks) {
           const unsigned long long p01 = ks ? pk(pa.z, pb.z) : pk(pa.x, pb.x);  // tokens e=0, e=1
           const unsigned long long p23 = ks ? pk(pa.w, pb.w) : pk(pa.y, pb.y);  // tokens e=2, e=3
-          const float4 s0 = vsv[ks * 4 + 0], s1 = vsv[ks * 4 + 1], s2 = vsv[ks * 4 + 2], s3 = vsv[ks * 4 + 3];
+          // V scales of tokens (ks, e = 0..3), the 4 channel groups each
+          const float4 s0 = vs4[(ks * 4 + 0) * 4], s1 = vs4[(ks * 4 + 1) * 4], s2 = vs4[(ks * 4 + 2) * 4],
+                       s3 = vs4[(ks * 4 + 3) * 4];
 #pragma unroll
           for (int grp = 0; grp < 4; ++grp) {
             const uint32_t b0 = split_bf16(mul2(p01, pk((&s0.x)[grp], (&s1.x)[grp])), nsel);
