@@ -6,8 +6,8 @@
 //
 // Partial results per (sequence, query head, split):
 //   m  running max of the base-2 logits, l  sum of 2^(logit - m),
-//   o[128]  sum of p * (s*q + z) [+ pattern] in the quantized space,
-//   W[P]    sum of p over the tokens that use each V pattern.
+//   o[128]  sum of p * (s*code + z) + sum_j W_j M_V[j] in the quantized space, with
+//           W_j the sum of p over the split's tokens that use V pattern j.
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -23,7 +23,7 @@ int decode_num_splits(const Geom& g, int Hq, int num_sms) { return decode_mma_sp
 
 size_t decode_workspace(const Geom& g, int Hq, int nsplit) {
   const size_t rows = (size_t)g.B * Hq * nsplit;
-  return rows * (2 + kD + g.P) * sizeof(float) + (size_t)g.B * g.H * sizeof(int) + 256;
+  return rows * (2 + kD) * sizeof(float) + (size_t)g.B * g.H * sizeof(int) + 256;
 }
 
 // Split partials, then the per-(sequence, KV head) arrival counters (zeroed here, on the stream).
@@ -33,11 +33,10 @@ cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, 
   const size_t rows = (size_t)g.B * Hq * nsplit;
   float* part_ml = reinterpret_cast<float*>(ws);
   float* part_o = part_ml + 2 * rows;
-  float* part_w = part_o + kD * rows;
-  int* arrivals = reinterpret_cast<int*>(part_w + (size_t)g.P * rows);
+  int* arrivals = reinterpret_cast<int*>(part_o + kD * rows);
   cudaError_t e = cudaMemsetAsync(arrivals, 0, (size_t)g.B * g.H * sizeof(int), st);
   if (e != cudaSuccess) return e;
-  return launch_decode_mma(g, q, Hq, sm_scale * kLog2e, nsplit, part_ml, part_o, part_w, arrivals, out, st);
+  return launch_decode_mma(g, q, Hq, sm_scale * kLog2e, nsplit, part_ml, part_o, arrivals, out, st);
 }
 
 }  // namespace kvq

@@ -23,7 +23,8 @@
 // The page layout (include/kvq.h) stores every lane's MMA operands contiguously.
 // Online softmax runs in base 2 in the MMA accumulator layout; the newest
 // incomplete group (exact keys in the K tail) is folded in on CUDA cores by the
-// last split.  Partials (m, l, o, W) go to the combine kernel.
+// last split.  Each CTA folds its pattern term sum_j W_j M_V[j] into its partial o, so the
+// partials are (m, l, o); the CTA that finishes a group's last split merges them.
 #include <cstdlib>
 
 #include "kvq_common.cuh"
@@ -161,7 +162,7 @@ __host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int
   Smem s;
   int o = 0;
   // the ring; the merge at the end reuses this region, so it is at least as large as the merge
-  const int merge = (kWarps * NT * 4 * kD + 2 * kWarps * NT * 4 + kWarps * NT * 4 * 4) * 4;
+  const int merge = (kWarps * NT * 4 * kD + 2 * kWarps * NT * 4 + kWarps * NT * 4 * 4 + P * NT * 4 + NT * 4 * kWarps) * 4;
   const int ring = kWarps * stages * sub_bytes;
   s.ring = o; o += ring > merge ? ring : merge;
   o = (o + 15) & ~15;
@@ -176,17 +177,17 @@ __host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int
 }
 
 // Combine of one (sequence, KV head) group, run by the CTA that finished the group's last
-// split: log-sum-exp merge of the splits, the pattern term sum_j W_j M_V[j] and the inverse
-// pre-transform.  Warp w takes query heads w, w + warps, ...; lane l holds channels
-// l + 32 k.  The partials come from other CTAs, so they are read through L2 (after the fence
-// that follows the arrival counter).  A non-finite output (an operand outside the fp32 /
-// bf16 range upstream) sets KVQ_DEV_RANGE.
+// split: log-sum-exp merge of the splits' (m, l, o) (each o already holds its pattern term)
+// and the inverse pre-transform.  Warp w takes query heads w, w + warps, ...; lane l holds
+// channels l + 32 k.  Lane s computes the weight of split s (32 splits at a time) and the
+// weights are broadcast, so the loads of consecutive splits are independent and overlap.
+// The partials come from other CTAs, so they are read through L2 (after the fence that
+// follows the arrival counter).  A non-finite output (an operand outside the fp32 / bf16
+// range upstream) sets KVQ_DEV_RANGE.
 __device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv, int Gq, int set,
-                              const float* part_ml, const float* part_o, const float* part_w, float* out,
-                              float* scratch) {
+                              const float* part_ml, const float* part_o, float* out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  float* Wsh = scratch + warp * 256;  // this warp's W (P <= 256)
-  const float* MV = g.vpat + ((size_t)set * g.H + h_kv) * g.P * kD;
+  const float2* ml2 = reinterpret_cast<const float2*>(part_ml);
   for (int hh = warp; hh < Gq; hh += nwarps) {
     const int row = b * Hq + h_kv * Gq + hh;
     const size_t base = (size_t)row * nsplit;
@@ -200,30 +201,23 @@ __device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv
       continue;
     }
     float Lsum = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = __ldcg(part_ml + 2 * (base + s));
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      Lsum += f * __ldcg(part_ml + 2 * (base + s) + 1);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) o[k] += f * __ldcg(part_o + (base + s) * kD + lane + 32 * k);
-    }
-    for (int j = lane; j < g.P; j += 32) {
-      float W = 0.f;
-      for (int s = 0; s < nsplit; ++s) {
-        const float ms = __ldcg(part_ml + 2 * (base + s));
-        if (ms == -INFINITY) continue;
-        W += exp2f(ms - M) * __ldcg(part_w + (base + s) * g.P + j);
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      float fs = 0.f;
+      if (s0 + lane < nsplit) {
+        const float2 ml = __ldcg(ml2 + base + s0 + lane);
+        fs = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+        Lsum = fmaf(fs, ml.y, Lsum);
       }
-      Wsh[j] = W;
-    }
-    __syncwarp();
-    for (int j = 0; j < g.P; ++j) {
-      const float W = Wsh[j];
+      const int n = min(32, nsplit - s0);
+      const float* po = part_o + (base + s0) * kD + lane;
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) {
+        const float f = __shfl_sync(kFull, fs, i);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) o[k] = fmaf(W, __ldg(MV + (size_t)j * kD + lane + 32 * k), o[k]);
+        for (int k = 0; k < 4; ++k) o[k] = fmaf(f, __ldcg(po + (size_t)i * kD + 32 * k), o[k]);
+      }
     }
-    __syncwarp();
+    Lsum = warp_sum(Lsum);
     const float inv = 1.0f / Lsum;
 #pragma unroll
     for (int k = 0; k < 4; ++k) o[k] *= inv;
@@ -246,8 +240,8 @@ __device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv
 template <int BITS, int NT, int STAGES, int kWarps>
 __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT == 1 ? 4 : 3) : 2))
     decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
-                      float* __restrict__ part_ml, float* __restrict__ part_o, float* __restrict__ part_w,
-                      int* __restrict__ arrivals, float* __restrict__ out) {
+                      float* __restrict__ part_ml, float* __restrict__ part_o, int* __restrict__ arrivals,
+                      float* __restrict__ out) {
   constexpr int NH = NT * 4;  // padded heads
   constexpr int WPL = Cfg<BITS>::kWordsPerLane;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -288,7 +282,44 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   const float* MK = g.kpat + sh * P * kD;
   const float* cK = g.tx ? g.kcol + sh * kD : nullptr;
 
-  // ---- setup: queries, T table, zeroed W, barriers
+  // ---- the first STAGES page copies of each warp go out before the setup below
+  // pages of this warp: p0 + warp + kWarps*i.  Their physical ids are read 32 at a time (lane l
+  // holds page 32w + l of window w), one window ahead, so no page-table load sits between a
+  // page and the copy of the page STAGES ahead.
+  const int my_n = (p1 - p0 - warp + kWarps - 1) / kWarps;
+  auto load_ids = [&](int base) -> int {
+    const int i = base + lane;
+    return i < my_n ? g.page_table[(size_t)b * g.maxp + p0 + warp + kWarps * i] : -1;
+  };
+  int ids = load_ids(0), ids_next = load_ids(32);
+  auto page_src = [&](int phys, bool& ok) -> const uint8_t* {
+    ok = phys >= 0 && phys < g.npages;
+    return g.pool + (size_t)(ok ? phys : 0) * g.page_bytes + (size_t)h_kv * g.sub_bytes;
+  };
+  uint32_t bad_mask = 0;  // lane 0: stages whose page id was invalid
+  if (lane < STAGES) mbar_init(&bars[lane], 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncwarp();
+  int first_ids[STAGES];
+#pragma unroll
+  for (int i = 0; i < STAGES; ++i) first_ids[i] = __shfl_sync(kFull, ids, i);
+  if (lane == 0) {
+    for (int i = 0; i < min(STAGES, my_n); ++i) {
+      bool ok;
+      const uint8_t* src = page_src(first_ids[i], ok);
+      if (ok) {
+        mbar_expect_tx(&bars[i], sub_bytes);
+        bulk_g2s(ring + i * sub_bytes, src, sub_bytes, &bars[i]);
+      } else {
+        set_status(g.status, KVQ_DEV_BAD_PAGE);
+        bad_mask |= 1u << i;
+        mbar_arrive(&bars[i]);
+      }
+    }
+  }
+  __syncwarp();
+
+  // ---- setup (overlapping the first copies): queries, T table, zeroed W
   for (int hh = warp; hh < NH; hh += kWarps) {
     float v[4];
     const bool real = hh < Gq;
@@ -307,8 +338,6 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
     for (int k = 0; k < 4; ++k) qk[hh * kD + ksc_pos(lane + 32 * k)] = v[k];
   }
   for (int i = threadIdx.x; i < kWarps * NH * P; i += blockDim.x) Wall[i] = 0.f;
-  if (lane < STAGES) mbar_init(&bars[lane], 1);
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
   for (int i = threadIdx.x; i < NH * P; i += blockDim.x) {
     const int hh = i / P, j = i % P;
@@ -352,39 +381,6 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
 #pragma unroll
       for (int u = 0; u < 4; ++u) accv[j][mt][u] = 0.f;
   }
-
-  // pages of this warp: p0 + warp + kWarps*i.  Their physical ids are read 32 at a time (lane l
-  // holds page 32w + l of window w), one window ahead, so no page-table load sits between a
-  // page and the copy of the page STAGES ahead.
-  const int my_n = (p1 - p0 - warp + kWarps - 1) / kWarps;
-  auto load_ids = [&](int base) -> int {
-    const int i = base + lane;
-    return i < my_n ? g.page_table[(size_t)b * g.maxp + p0 + warp + kWarps * i] : -1;
-  };
-  int ids = load_ids(0), ids_next = load_ids(32);
-  auto page_src = [&](int phys, bool& ok) -> const uint8_t* {
-    ok = phys >= 0 && phys < g.npages;
-    return g.pool + (size_t)(ok ? phys : 0) * g.page_bytes + (size_t)h_kv * g.sub_bytes;
-  };
-  uint32_t bad_mask = 0;  // lane 0: stages whose page id was invalid
-  int first_ids[STAGES];
-#pragma unroll
-  for (int i = 0; i < STAGES; ++i) first_ids[i] = __shfl_sync(kFull, ids, i);
-  if (lane == 0) {
-    for (int i = 0; i < min(STAGES, my_n); ++i) {
-      bool ok;
-      const uint8_t* src = page_src(first_ids[i], ok);
-      if (ok) {
-        mbar_expect_tx(&bars[i], sub_bytes);
-        bulk_g2s(ring + i * sub_bytes, src, sub_bytes, &bars[i]);
-      } else {
-        set_status(g.status, KVQ_DEV_BAD_PAGE);
-        bad_mask |= 1u << i;
-        mbar_arrive(&bars[i]);
-      }
-    }
-  }
-  __syncwarp();
 
   int stuck_at = -1;
   for (int i = 0; i < my_n; ++i) {
@@ -681,6 +677,8 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
       for (int u = 0; u < 4; ++u) mz[(warp * NH + hh) * 4 + u] = zacc[j][u];
     }
   }
+  float* wc = mz + kWarps * NH * 4;                       // [P][NH] merged pattern weights
+  float* fsh = wc + P * NH;                               // [NH][kWarps] warp weights
   __syncthreads();
   for (int hh = warp; hh < Gq; hh += kWarps) {
     float M = -INFINITY;
@@ -692,22 +690,43 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
       const float mw = mm[w * NH + hh];
       f[w] = (mw == -INFINITY) ? 0.f : ex2(mw - M);
       Ls += f[w] * ml[w * NH + hh];
+      if (lane == w) fsh[hh * kWarps + w] = f[w];
     }
     const size_t base = ((size_t)b * Hq + h_kv * Gq + hh) * nsplit + split;
     if (lane == 0) { part_ml[2 * base] = M; part_ml[2 * base + 1] = Ls; }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float o = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w)
-        o += f[w] * (mo[(w * NH + hh) * kD + lane + 32 * k] + mz[(w * NH + hh) * 4 + k]);
-      part_o[base * kD + lane + 32 * k] = o;
-    }
     for (int jj = lane; jj < P; jj += 32) {
       float Wv = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) Wv += f[w] * Wall[(w * NH + hh) * P + jj];
-      part_w[base * P + jj] = Wv;
+      wc[jj * NH + hh] = Wv;
+    }
+  }
+  __syncthreads();
+  // o = sum_w f_w (residual + zero terms of warp w) + sum_j W_j M_V[j]: thread = channel c,
+  // query heads hg, hg + HG, ...; each M_V value is read once per CTA
+  {
+    constexpr int HG = kWarps * 32 / kD;
+    constexpr int NA = NH / HG;
+    const int c = threadIdx.x % kD, hg = threadIdx.x / kD;
+    const float* mv = g.vpat + sh * P * kD + c;
+    float acc[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc[i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < P; ++j) {
+      const float m = __ldg(mv + (size_t)j * kD);
+#pragma unroll
+      for (int i = 0; i < NA; ++i) acc[i] = fmaf(wc[j * NH + hg + HG * i], m, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NA; ++i) {
+      const int hh = hg + HG * i;
+      if (hh >= Gq) continue;
+      float o = acc[i];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        o = fmaf(fsh[hh * kWarps + w], mo[(w * NH + hh) * kD + c] + mz[(w * NH + hh) * 4 + (c >> 5)], o);
+      part_o[(((size_t)b * Hq + h_kv * Gq + hh) * nsplit + split) * kD + c] = o;
     }
   }
 
@@ -719,8 +738,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   __syncthreads();
   if (!last) return;
   __threadfence();
-  combine_group(g, Hq, nsplit, b, h_kv, Gq, set, part_ml, part_o, part_w, out,
-                reinterpret_cast<float*>(smem + sp.ring));
+  combine_group(g, Hq, nsplit, b, h_kv, Gq, set, part_ml, part_o, out);
 }
 
 template <int BITS, int NT, int STAGES, int NW>
@@ -734,12 +752,12 @@ struct Launcher {
     return n > 0 ? n : 1;
   }
   static cudaError_t launch(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml, float* o,
-                            float* w, int* arrivals, float* out, cudaStream_t st) {
+                            int* arrivals, float* out, cudaStream_t st) {
     const int total = smem(g);
     cudaError_t e = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, g.H, g.B);
-    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, w, arrivals, out);
+    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, arrivals, out);
     return cudaGetLastError();
   }
 };
@@ -805,9 +823,9 @@ size_t decode_mma_smem(const Geom& g, int Hq) {
 }
 
 cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
-                              float* o, float* w, int* arrivals, float* out, cudaStream_t st) {
+                              float* o, int* arrivals, float* out, cudaStream_t st) {
   return dispatch(g, Hq, decode_stages(), [&](auto L) {
-    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, w, arrivals, out, st);
+    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, arrivals, out, st);
   });
 }
 

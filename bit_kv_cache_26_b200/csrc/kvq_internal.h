@@ -20,7 +20,7 @@ size_t decode_workspace(const Geom& g, int Hq, int nsplit);
 cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, float* out, void* ws, int nsplit,
                           cudaStream_t st);
 cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
-                              float* o, float* w, int* arrivals, float* out, cudaStream_t st);
+                              float* o, int* arrivals, float* out, cudaStream_t st);
 size_t decode_mma_smem(const Geom& g, int Hq);
 int decode_mma_splits(const Geom& g, int Hq, int num_sms);
 
