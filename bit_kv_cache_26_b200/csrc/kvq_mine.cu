@@ -26,6 +26,7 @@ struct MineWs {
   double* sums;     // [NP][P][128]
   uint32_t* cnt;    // [NP][P]
   int32_t* assign;  // [NP][n]
+  float* xsq;       // [NP][n] |x|^2 of every token (the fused Lloyd step's cache)
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
   double* colsum;   // [NP][128]
@@ -43,6 +44,7 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   w.cnt = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
   if (assign_out) w.assign = assign_out;
   else { w.assign = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t)); }
+  w.xsq = (float*)p; p += align256((size_t)NP * n * sizeof(float));
   if (transform) {
     w.y = (float*)p; p += align256((size_t)NP * n * kD * sizeof(float));
     w.v64 = (double*)p; p += align256((size_t)NP * n * kD * sizeof(double));
@@ -1091,6 +1093,389 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
 }
 
+// ---- fused Lloyd step: bf16 input, P <= 64 ------------------------------------------------
+//
+// One pass over x per iteration: the assignment of mine_assign_tc_kernel and the cluster sums
+// of mine_accum_kernel from the same staged tile.  One CTA per SM, warp-specialised, no block
+// barrier in the loop:
+//   * warp 0: TMA loads of 128-token tiles into a ring of stages (as mine_assign_tc_kernel);
+//   * warp 1: the distance contraction of each tile into one of two TMEM buffers (as there);
+//   * warps 2-9, two warpgroups (warpgroup g takes the tiles k with k % 2 == g, TMEM buffer g),
+//     one token per thread: u_j = |m_j|^2 / 2 - x.m_j (so e_j = 2 u_j) with the pattern index
+//     written into the 6 low mantissa bits, which moves u_j by at most 2^-17 |u_j|.  The two
+//     smallest tagged scores give the candidate and the gap; the gap test of
+//     mine_assign_tc_kernel, widened by twice the largest such move, certifies the candidate,
+//     and a token that fails it is decided by the float64 recomputation of its candidates.
+//     |x|^2 comes from the staged tile in the first iteration and from a per-token cache after
+//     that.  The tile's assignment goes to shared memory (and to `assign`);
+//   * warps 10-17: warp a owns the clusters j with j % 8 == a and keeps their float64 sums
+//     (channels 4l .. 4l + 3 in lane l) in registers for the whole kernel; one ballot per 32
+//     tokens of a tile finds its members (the assigners count them in shared memory).  At the
+//     end each warp adds its totals to global memory.  float64 sums of bf16 values are exact, so the order of the additions
+//     does not change them.
+// A stage is refilled once the MMA has read it and every accumulator warp is done with it.
+// Every mbarrier wait is bounded.
+constexpr int kLlAsgWarps = 8;
+constexpr int kLlAccWarps = 8;
+constexpr int kLlThreads = (2 + kLlAsgWarps + kLlAccWarps) * 32;
+constexpr int kLlMaxStages = 6;
+constexpr float kLlPad = 1.0e38f;  // |m_j|^2 / 2 of the padding patterns past P: never the minimum
+
+// dynamic shared memory: B (N rows x 256 B), the stages, their assignments, the pattern
+// tables, the barriers, and the slack for 1024-byte alignment
+size_t ll_smem_bytes(int P, int nst) {
+  const int Pn = (P + 7) & ~7, N = 2 * Pn;
+  return (size_t)N * 256 + (size_t)nst * kTcTileBytes + (size_t)nst * kTcM * 4 + (size_t)4 * Pn * 4 + 16 +
+         (size_t)(3 * nst + 4) * 8 + 16 + 1024;
+}
+int mine_ll_stages(int P) {
+  int nst = kLlMaxStages;
+  while (nst > 2 && ll_smem_bytes(P, nst) > 227 * 1024) --nst;
+  return nst;
+}
+
+// u with its 6 low mantissa bits replaced by j (j < 64)
+__device__ __forceinline__ float tag_score(float u, int j) {
+  return __uint_as_float((__float_as_uint(u) & 0xFFFFFFC0u) | (uint32_t)j);
+}
+// running two smallest values
+__device__ __forceinline__ void low2_add(float& m1, float& m2, float v) {
+  m2 = fminf(m2, fmaxf(m1, v));
+  m1 = fminf(m1, v);
+}
+
+__global__ void __launch_bounds__(kLlThreads, 1)
+    mine_lloyd_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s, int P, const float* __restrict__ M,
+                         int32_t* __restrict__ assign, float* __restrict__ xsq_cache, int first,
+                         double* __restrict__ sums, uint32_t* __restrict__ cnt, int nst) {
+  const int prob = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Pn = (P + 7) & ~7, N = 2 * Pn;
+  uint32_t tcols = 32;
+  while (tcols < 2u * (uint32_t)N) tcols <<= 1;  // two accumulator buffers
+  const uint32_t buf_cols = tcols / 2;
+  const uint32_t half_b = (uint32_t)N * 128u;  // B: channels 64-127 start N x 128 B in
+  extern __shared__ __align__(16) uint8_t smraw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Bt = base;                                                                   // [2][N][128 B]
+  uint8_t* At = base + (size_t)N * 256;                                                 // [nst][2][128][128 B]
+  int32_t* asg = reinterpret_cast<int32_t*>(At + (size_t)nst * kTcTileBytes);           // [nst][128]
+  float* msq = reinterpret_cast<float*>(asg + nst * kTcM);                              // [Pn]
+  float* hm = msq + Pn;                                                                 // [Pn]
+  float* mnorm = hm + Pn;                                                               // [Pn]
+  float* gmax = mnorm + Pn;                                                             // [4]
+  uint32_t* members = reinterpret_cast<uint32_t*>(gmax + 4);                            // [Pn]
+  uint64_t* full = reinterpret_cast<uint64_t*>(members + Pn);
+  uint64_t* sfree = full + nst;
+  uint64_t* asgd = sfree + nst;
+  uint64_t* tfull = asgd + nst;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+  const float* Mp = M + (size_t)prob * P * kD;
+  const int set = prob / s.heads, h = prob % s.heads;
+
+  // ---- B: bf16 hi parts (rows 0..Pn-1) and mid parts (rows Pn..2Pn-1) of the patterns
+  for (int i = tid; i < N * 16; i += blockDim.x) {
+    const int n = i >> 4, c = i & 15;
+    const int j = n < Pn ? n : n - Pn;
+    uint32_t wv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint16_t hv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float m = j < P ? Mp[(size_t)j * kD + 8 * c + 2 * q + e] : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(m);
+        const __nv_bfloat16 v = n < Pn ? hi : __float2bfloat16_rn(m - __bfloat162float(hi));
+        hv[e] = __bfloat16_as_ushort(v);
+      }
+      wv[q] = (uint32_t)hv[0] | ((uint32_t)hv[1] << 16);
+    }
+    *reinterpret_cast<uint4*>(Bt + (size_t)(c >> 3) * half_b + sw128_off(n, c & 7)) =
+        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  }
+  if (tid == 0) {
+    gmax[0] = 0.f;
+    gmax[1] = 0.f;
+    for (int i = 0; i < nst; ++i) {
+      mb_init(&full[i], 1);
+      mb_init(&sfree[i], 1 + kLlAccWarps);    // the MMA commit and every accumulator warp
+      mb_init(&asgd[i], kLlAsgWarps / 2);     // the 4 warps of the tile's warpgroup
+    }
+    for (int i = 0; i < 2; ++i) {
+      mb_init(&tfull[i], 1);
+      mb_init(&tempty[i], kLlAsgWarps / 2);  // buffer i belongs to warpgroup i
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tslot)), "r"(tcols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  __syncthreads();
+  for (int j = tid; j < Pn; j += blockDim.x) {
+    double acc = 0.0;
+    if (j < P)
+      for (int d = 0; d < kD; ++d) { const double m = Mp[(size_t)j * kD + d]; acc += m * m; }
+    msq[j] = (float)acc;
+    hm[j] = j < P ? 0.5f * (float)acc : kLlPad;
+    members[j] = 0u;
+    mnorm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
+    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int(mnorm[j]));
+    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq[j] * (1.0f + 1e-6f)));
+  }
+  fence_proxy_async();  // B (generic stores) before the tensor cores read it
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+
+  const int64_t ntiles = (s.n + kTcM - 1) / kTcM;
+  const int nt = ntiles > blockIdx.x ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  auto tile_t0 = [&](int k) { return ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * kTcM; };
+
+  if (warp == 0) {
+    // ---- producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      int issued = 0;
+      for (int k = 0; k < nt; ++k) {
+        const int st = k % nst;
+        if (k >= nst && !tc_wait(&sfree[st], (uint32_t)(((k / nst) - 1) & 1))) break;
+        uint8_t* dst = At + (size_t)st * kTcTileBytes;
+        mb_expect_tx(&full[st], (uint32_t)kTcTileBytes);
+        const int t0 = (int)tile_t0(k);
+        tma_load_4d(dst, &xmap, 0, h, t0, set, &full[st]);
+        tma_load_4d(dst + kTcTileBytes / 2, &xmap, 64, h, t0, set, &full[st]);
+        issued = k + 1;
+      }
+      // every copy issued has landed before the CTA may leave (bounded, as every wait)
+      for (int k = max(0, issued - nst); k < issued; ++k) (void)tc_wait(&full[k % nst], (uint32_t)((k / nst) & 1));
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc(kTcM, N);
+      const uint32_t b0 = su32(Bt);
+      for (int k = 0; k < nt; ++k) {
+        const int st = k % nst, buf = k & 1;
+        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1))) break;
+        if (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t a0 = su32(At + (size_t)st * kTcTileBytes);
+        const uint32_t d = tbase + (uint32_t)buf * buf_cols;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks)  // K step ks: half ks / 4, 32 B per step inside the atom
+          umma_bf16(d, umma_desc_sw128(a0 + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32),
+                    umma_desc_sw128(b0 + (ks >> 2) * half_b + (ks & 3) * 32), idesc, ks > 0);
+        umma_commit(&tfull[buf]);
+        umma_commit(&sfree[st]);
+      }
+    }
+  } else if (warp < 2 + kLlAsgWarps) {
+    // ---- assigners: warpgroup g, TMEM lane quarter q4, token `row` of the tile
+    const int g = (warp - 2) >> 2, q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const float nm_max = gmax[0], msq_max = gmax[1];
+    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)g * buf_cols;
+    for (int k = g; k < nt; k += 2) {
+      const int st = k % nst;
+      const int64_t i = tile_t0(k) + row;
+      const bool valid = i < s.n;
+      float xsq = 0.f;
+      if (!first && valid) xsq = xsq_cache[(size_t)prob * s.n + i];
+      if (!__all_sync(kFull, tc_wait(&tfull[g], (uint32_t)((k >> 1) & 1)))) break;
+      tc_fence_after();
+      if (first) {
+        // |x|^2 of the row from the staged tile (two swizzled halves of 64 channels)
+        const uint8_t* stg = At + (size_t)st * kTcTileBytes;
+        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+        for (int hc = 0; hc < 16; ++hc) {
+          const uint4 u = *reinterpret_cast<const uint4*>(stg + (hc >> 3) * (kTcTileBytes / 2) + sw128_off(row, hc & 7));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
+            if (q & 1) fma2f(v0, v1, v0, v1, b0, b1, b0, b1);
+            else fma2f(v0, v1, v0, v1, a0, a1, a0, a1);
+          }
+        }
+        xsq = (a0 + a1) + (b0 + b1);
+        if (valid) xsq_cache[(size_t)prob * s.n + i] = xsq;
+      }
+      const float xs = xsq * (1.0f + 1e-6f);
+      const float nx = sqrtf(xs) * (1.0f + 1e-6f);
+      // the two smallest tagged scores, in two chains (even / odd patterns)
+      float m1a = INFINITY, m2a = INFINITY, m1b = INFINITY, m2b = INFINITY;
+      float hv[8], mv[8];
+      tmem_ld8_issue(taddr, hv);
+      tmem_ld8_issue(taddr + Pn, mv);
+      tmem_ld_wait();
+      for (int c0 = 0; c0 < Pn; c0 += 8) {
+        float hn[8], mn_[8];
+        const bool more = c0 + 8 < Pn;
+        if (more) {
+          tmem_ld8_issue(taddr + c0 + 8, hn);
+          tmem_ld8_issue(taddr + Pn + c0 + 8, mn_);
+        }
+        const float4 ha = *reinterpret_cast<const float4*>(hm + c0);
+        const float4 hb = *reinterpret_cast<const float4*>(hm + c0 + 4);
+        const float hq[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+#pragma unroll
+        for (int q = 0; q < 8; q += 2) {
+          float s0, s1, u0, u1;
+          add2f(hv[q], hv[q + 1], mv[q], mv[q + 1], s0, s1);
+          sub2(hq[q], hq[q + 1], s0, s1, u0, u1);
+          low2_add(m1a, m2a, tag_score(u0, c0 + q));
+          low2_add(m1b, m2b, tag_score(u1, c0 + q + 1));
+        }
+        if (more) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) { hv[q] = hn[q]; mv[q] = mn_[q]; }
+        }
+      }
+      const float m1 = fminf(m1a, m1b);
+      const float m2 = fminf(fmaxf(m1a, m1b), fminf(m2a, m2b));
+      int jw = (int)(__float_as_uint(m1) & 63u);
+      // e = 2 u: certified when the gap beats both error bounds and both tags' moves
+      const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xs + msq_max);
+      const float Pe = 0x1p-17f * (msq_max + 2.0f * nx * nm_max);
+      const bool unique = 2.0f * (m2 - m1) > 2.0f * Eb + 2.0f * Pe + 1e-9f * (xs + msq_max);
+      const bool need = !unique && valid;
+      if (__any_sync(kFull, need)) {
+        // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
+        float U = INFINITY;
+        for (int c0 = 0; c0 < Pn; c0 += 8) {
+          tmem_ld8_issue(taddr + c0, hv);
+          tmem_ld8_issue(taddr + Pn + c0, mv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j = c0 + q;
+            if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xs + msq[j]));
+          }
+        }
+        uint32_t cand[2] = {0u, 0u};  // candidate bit mask over j < 64
+        for (int c0 = 0; c0 < Pn; c0 += 8) {
+          tmem_ld8_issue(taddr + c0, hv);
+          tmem_ld8_issue(taddr + Pn + c0, mv);
+          tmem_ld_wait();
+          uint32_t cm = 0u;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j = c0 + q;
+            const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
+            const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xs + msq[j]);
+            if (j < P && e - E <= U + 1e-9f * (xs + msq[j])) cm |= 1u << q;
+          }
+          cand[c0 >> 5] |= cm << (c0 & 31);
+        }
+        if (need) {
+          const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
+          double bd = 0.0;
+          int bj = 0;
+          bool have = false;
+          for (int cw = 0; cw < 2; ++cw)
+            for (uint32_t m = cand[cw]; m; m &= m - 1) {
+              const int j = cw * 32 + __ffs(m) - 1;
+              const float* mrow = Mp + (size_t)j * kD;
+              double acc = 0.0;
+#pragma unroll 8
+              for (int d = 0; d < kD; d += 4) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
+                const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
+                const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
+                const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
+                  acc = __dadd_rn(acc, __dmul_rn(t, t));
+                }
+              }
+              if (!have || acc < bd) { bd = acc; bj = j; have = true; }
+            }
+          jw = bj;
+        }
+      }
+      if (valid) {
+        assign[(size_t)prob * s.n + i] = jw;
+        atomicAdd(&members[jw], 1u);
+      }
+      asg[st * kTcM + row] = valid ? jw : -1;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mb_arrive(&asgd[st]);
+        mb_arrive(&tempty[g]);
+      }
+    }
+  } else {
+    // ---- accumulators: warp aw owns clusters aw + 8 c; lane l holds channels 4l .. 4l + 3
+    const int aw = warp - 2 - kLlAsgWarps;
+    double acc[8][4];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[c][e] = 0.0;
+    }
+    // channels 4l .. 4l + 3: half l >> 4, 16-byte chunk (l >> 1) & 7 of the swizzled row, 8 bytes in when l is odd
+    const uint32_t lane_off = (uint32_t)(lane >> 4) * (kTcTileBytes / 2) + (uint32_t)(lane & 1) * 8u;
+    const int cidx = (lane >> 1) & 7;
+    for (int k = 0; k < nt; ++k) {
+      const int st = k % nst;
+      if (!__all_sync(kFull, tc_wait(&asgd[st], (uint32_t)((k / nst) & 1)))) break;
+      const int32_t* as = asg + st * kTcM;
+      int aj[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) aj[q] = as[32 * q + lane];
+      const uint8_t* stg = At + (size_t)st * kTcTileBytes + lane_off;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t m = __ballot_sync(kFull, aj[q] >= 0 && (aj[q] & 7) == aw);
+        while (m) {
+          const int t = 32 * q + __ffs(m) - 1;
+          m &= m - 1;
+          const int c = __shfl_sync(kFull, aj[q], t & 31) >> 3;
+          const uint2 u = *reinterpret_cast<const uint2*>(stg + (t >> 3) * 1024 + (t & 7) * 128 + ((cidx ^ (t & 7)) << 4));
+          const double v0 = (double)__uint_as_float(u.x << 16), v1 = (double)__uint_as_float(u.x & 0xFFFF0000u);
+          const double v2 = (double)__uint_as_float(u.y << 16), v3 = (double)__uint_as_float(u.y & 0xFFFF0000u);
+          switch (c) {
+#define KVQ_LL_ACC(C)                                                                     \
+  case C:                                                                                 \
+    acc[C][0] += v0; acc[C][1] += v1; acc[C][2] += v2; acc[C][3] += v3; break;
+            KVQ_LL_ACC(0) KVQ_LL_ACC(1) KVQ_LL_ACC(2) KVQ_LL_ACC(3)
+            KVQ_LL_ACC(4) KVQ_LL_ACC(5) KVQ_LL_ACC(6) KVQ_LL_ACC(7)
+#undef KVQ_LL_ACC
+            default: break;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mb_arrive(&sfree[st]);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = aw + 8 * c;
+      if (j >= P) break;
+      double* gs = sums + ((size_t)prob * P + j) * kD + 4 * lane;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (acc[c][e] != 0.0) atomicAdd(gs + e, acc[c][e]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  for (int j = tid; j < P; j += blockDim.x)
+    if (members[j]) atomicAdd(cnt + (size_t)prob * P + j, members[j]);
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
+}
+
 // ring depth that fits next to the patterns in 227 KB, and the dynamic shared memory it needs
 int mine_tc_stages(int P) {
   const int Pn = (P + 7) & ~7;
@@ -1117,7 +1502,7 @@ __global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt)
 size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
   size_t NP = (size_t)sets * heads;
   size_t b = align256(NP * P * kD * sizeof(double)) + align256(NP * P * sizeof(uint32_t)) +
-             align256(NP * (size_t)n * sizeof(int32_t));
+             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * (size_t)n * sizeof(float));
   if (transform)
     b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
          4 * align256(NP * kD * sizeof(double));
@@ -1231,8 +1616,23 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   }
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, (a.P <= 64 ? 2 : 1) * sms / NP)));
+  // bf16 input and P <= 64: assignment and cluster sums in one pass (one CTA per SM)
+  const bool use_ll = KIND == 0 && a.P <= 8 * kLlAccWarps;
+  const int ll_nst = mine_ll_stages(a.P);
+  const size_t smem_ll = ll_smem_bytes(a.P, ll_nst);
+  if (use_ll && (e = cudaFuncSetAttribute(mine_lloyd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)smem_ll)) != cudaSuccess)
+    return e;
+  const unsigned ll_ctas = (unsigned)std::max<int64_t>(
+      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
+    if (use_ll) {
+      mine_lloyd_tc_kernel<<<dim3(ll_ctas, NP), kLlThreads, smem_ll, st>>>(xmap, s, a.P, a.patterns, w.assign, w.xsq,
+                                                                           it == 0, w.sums, w.cnt, ll_nst);
+      mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
+      continue;
+    }
     if (use_tc)
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(xmap, s, a.P, a.patterns, w.assign,
                                                                              mine_tc_stages(a.P));
