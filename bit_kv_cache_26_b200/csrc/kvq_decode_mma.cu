@@ -339,29 +339,38 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   }
   for (int i = threadIdx.x; i < kWarps * NH * P; i += blockDim.x) Wall[i] = 0.f;
   __syncthreads();
-  for (int i = threadIdx.x; i < NH * P; i += blockDim.x) {
-    const int hh = i / P, j = i % P;
-    float t = 0.f;
-    if (hh < Gq) {
-      // qk holds KSC order: its float4 p covers channels c, c + 1, c + 8, c + 9 with
-      // c = 16 (p >> 2) + 2 (p & 3); four independent partial sums
-      const float* m = MK + (size_t)j * kD;
-      const float4* q4 = reinterpret_cast<const float4*>(qk + hh * kD);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-      for (int p = 0; p < kD / 4; ++p) {
-        const float4 qv = q4[p];
-        const int c = 16 * (p >> 2) + 2 * (p & 3);
-        const float2 ma = __ldg(reinterpret_cast<const float2*>(m + c));
-        const float2 mb = __ldg(reinterpret_cast<const float2*>(m + c + 8));
-        a0 = fmaf(qv.x, ma.x, a0);
-        a1 = fmaf(qv.y, ma.y, a1);
-        a2 = fmaf(qv.z, mb.x, a2);
-        a3 = fmaf(qv.w, mb.y, a3);
+  // T[hh][j] = q_hh . M_K[j] (transformed space): warp w takes patterns w, w + warps, ...;
+  // lane l holds channels 4l .. 4l + 3 of four query heads and reads the pattern row with one
+  // coalesced 16-byte load; the four head sums are reduced across the warp
+#pragma unroll 1
+  for (int hg = 0; hg < NT; ++hg) {
+    float qv[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qv[a][e] = qk[(4 * hg + a) * kD + ksc_pos(4 * lane + e)];
+    // eight pattern rows' loads in flight at a time
+    for (int j0 = warp; j0 < P; j0 += 8 * kWarps) {
+      float4 m4[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kWarps;
+        m4[u] = j < P ? __ldg(reinterpret_cast<const float4*>(MK + (size_t)j * kD) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      t = (a0 + a1) + (a2 + a3);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kWarps;
+        float t[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          t[a] = fmaf(qv[a][3], m4[u].w, fmaf(qv[a][2], m4[u].z, fmaf(qv[a][1], m4[u].y, qv[a][0] * m4[u].x)));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+          for (int a = 0; a < 4; ++a) t[a] += __shfl_xor_sync(kFull, t[a], off);
+        if (lane < 4 && j < P) T[(4 * hg + lane) * P + j] = lane == 0 ? t[0] : lane == 1 ? t[1] : lane == 2 ? t[2] : t[3];
+      }
     }
-    T[i] = t;
   }
   __syncthreads();
 

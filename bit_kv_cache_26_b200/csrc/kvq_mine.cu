@@ -26,7 +26,9 @@ struct MineWs {
   double* sums;     // [NP][P][128]
   uint32_t* cnt;    // [NP][P]
   int32_t* assign;  // [NP][n]
-  float* xsq;       // [NP][n] |x|^2 of every token (the fused Lloyd step's cache)
+  float* xsq;       // [NP][n] |x|^2 of every token (the tcgen05 assignment's cache)
+  int32_t* amb;     // [NP][n] tokens the tcgen05 assignment left undecided
+  int32_t* amb_cnt; // [NP]
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
   double* colsum;   // [NP][128]
@@ -45,6 +47,8 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   if (assign_out) w.assign = assign_out;
   else { w.assign = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t)); }
   w.xsq = (float*)p; p += align256((size_t)NP * n * sizeof(float));
+  w.amb = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t));
+  w.amb_cnt = (int32_t*)p; p += align256((size_t)NP * sizeof(int32_t));
   if (transform) {
     w.y = (float*)p; p += align256((size_t)NP * n * kD * sizeof(float));
     w.v64 = (double*)p; p += align256((size_t)NP * n * kD * sizeof(double));
@@ -580,21 +584,50 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-template <int RB>
+// x * 2^-896 as a float64 built from the bits of the bf16 value x in the low / high half of
+// w: the bf16 sign, exponent and mantissa fields become the float64 sign, the low 8 bits of
+// its exponent and the top of its mantissa, so every finite bf16 value (subnormals included,
+// as float64 subnormals) maps exactly; float64 sums of these stay exact and the factor is
+// undone once at the end.  Integer operations instead of a float conversion, whose unit runs
+// at a fraction of the integer pipe's rate.  The fp16 forms give x * 2^-1008 (5-bit exponent
+// field), the fp32 form x * 2^-896 (both words of the float64).
+__device__ __forceinline__ double bf16lo_scaled(uint32_t w) {
+  return __hiloint2double((int)(((w << 16) & 0x80000000u) | ((w << 13) & 0x0FFFE000u)), 0);
+}
+__device__ __forceinline__ double bf16hi_scaled(uint32_t w) {
+  return __hiloint2double((int)((w & 0x80000000u) | ((w >> 3) & 0x0FFFE000u)), 0);
+}
+__device__ __forceinline__ double f16lo_scaled(uint32_t w) {
+  return __hiloint2double((int)(((w << 16) & 0x80000000u) | ((w << 10) & 0x01FFFC00u)), 0);
+}
+__device__ __forceinline__ double f16hi_scaled(uint32_t w) {
+  return __hiloint2double((int)((w & 0x80000000u) | ((w >> 6) & 0x01FFFC00u)), 0);
+}
+__device__ __forceinline__ double f32_scaled(uint32_t f) {
+  return __hiloint2double((int)((f & 0x80000000u) | ((f & 0x7FFFFFFFu) >> 3)), (int)(f << 29));
+}
+
+// 16-bit rows and up to 4 clusters per warp: two CTAs per SM, each with a ring in half the
+// shared memory (and registers for two); otherwise one
+template <int CPW, int ES>
+constexpr int accum_ctas_per_sm() { return ES == 2 && CPW <= 4 ? 2 : 1; }
+template <int CPW, int RB, int ES>
 constexpr int accum_stages() {
-  return (200 * 1024) / (kAccT * RB) < 4 ? (200 * 1024) / (kAccT * RB) : 4;
+  return (200 * 1024 / accum_ctas_per_sm<CPW, ES>()) / (kAccT * RB) < 4
+             ? (200 * 1024 / accum_ctas_per_sm<CPW, ES>()) / (kAccT * RB)
+             : 4;
 }
 
 // CPW clusters per warp, E channels per lane (slice = 32 E channels), ES bytes per element
 // (2: the fp16 / bf16 input, 4: the fp32 pre-transformed rows)
 template <int CPW, int E, int ES>
-__global__ void __launch_bounds__((kAccWarps + 1) * 32, 1) mine_accum_kernel(const __grid_constant__ CUtensorMap amap,
+__global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, ES>()) mine_accum_kernel(const __grid_constant__ CUtensorMap amap,
                                                                             Src s, int P,
                                                                             const int32_t* __restrict__ assign,
                                                                             double* __restrict__ sums,
                                                                             uint32_t* __restrict__ cnt) {
   constexpr int CW = 32 * E, RB = CW * ES;  // channels and bytes of a staged row
-  constexpr int kStages = accum_stages<RB>();
+  constexpr int kStages = accum_stages<CPW, RB, ES>();
   constexpr int kStageBytes = kAccT * RB;
   extern __shared__ __align__(16) uint8_t smraw[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStages * kStageBytes);
@@ -637,7 +670,8 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, 1) mine_accum_kernel(con
     return;
   }
 
-  // ---- consumers
+  // ---- consumers: float64 sums of the rows scaled by 2^-896 (bf16, fp32) or 2^-1008 (fp16)
+  const bool f16 = ES == 2 && s.dtype == KVQ_F16;
   double acc[CPW][E];
   uint32_t members[CPW];
 #pragma unroll
@@ -674,28 +708,29 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, 1) mine_accum_kernel(con
           const int t = 32 * q + __ffs(m) - 1;
           m &= m - 1;
           const uint8_t* row = stg + t * RB + lane * (E * ES);
-          float v[E];
+          double v[E];
           if constexpr (ES == 4) {
-            if constexpr (E == 4) { const float4 f = *reinterpret_cast<const float4*>(row); v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w; }
-            else if constexpr (E == 2) { const float2 f = *reinterpret_cast<const float2*>(row); v[0] = f.x; v[1] = f.y; }
-            else v[0] = *reinterpret_cast<const float*>(row);
-          } else {
             if constexpr (E == 4) {
-              const uint2 b = *reinterpret_cast<const uint2*>(row);
-              v[0] = bits_to_float((uint16_t)(b.x & 0xffffu), s.dtype);
-              v[1] = bits_to_float((uint16_t)(b.x >> 16), s.dtype);
-              v[2] = bits_to_float((uint16_t)(b.y & 0xffffu), s.dtype);
-              v[3] = bits_to_float((uint16_t)(b.y >> 16), s.dtype);
+              const uint4 f = *reinterpret_cast<const uint4*>(row);
+              v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y); v[2] = f32_scaled(f.z); v[3] = f32_scaled(f.w);
             } else if constexpr (E == 2) {
-              const uint32_t b = *reinterpret_cast<const uint32_t*>(row);
-              v[0] = bits_to_float((uint16_t)(b & 0xffffu), s.dtype);
-              v[1] = bits_to_float((uint16_t)(b >> 16), s.dtype);
+              const uint2 f = *reinterpret_cast<const uint2*>(row);
+              v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y);
             } else {
-              v[0] = bits_to_float(*reinterpret_cast<const uint16_t*>(row), s.dtype);
+              v[0] = f32_scaled(*reinterpret_cast<const uint32_t*>(row));
             }
+          } else {
+            uint32_t b[(E + 1) / 2];
+            if constexpr (E == 4) { const uint2 u = *reinterpret_cast<const uint2*>(row); b[0] = u.x; b[1] = u.y; }
+            else if constexpr (E == 2) b[0] = *reinterpret_cast<const uint32_t*>(row);
+            else b[0] = *reinterpret_cast<const uint16_t*>(row);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+              v[e] = f16 ? ((e & 1) ? f16hi_scaled(b[e >> 1]) : f16lo_scaled(b[e >> 1]))
+                         : ((e & 1) ? bf16hi_scaled(b[e >> 1]) : bf16lo_scaled(b[e >> 1]));
           }
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[c][e] += (double)v[e];
+          for (int e = 0; e < E; ++e) acc[c][e] += v[e];
         }
       }
     }
@@ -706,20 +741,21 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, 1) mine_accum_kernel(con
   }
 
   double* gs = sums + (size_t)prob * P * kD + slice * CW + lane * E;
+  const double unscale = f16 ? 0x1p1008 : 0x1p896;
 #pragma unroll
   for (int c = 0; c < CPW; ++c) {
     const int j = warp + kAccWarps * c;
     if (j >= P) break;
 #pragma unroll
     for (int e = 0; e < E; ++e)
-      if (acc[c][e] != 0.0) atomicAdd(gs + (size_t)j * kD + e, acc[c][e]);
+      if (acc[c][e] != 0.0) atomicAdd(gs + (size_t)j * kD + e, acc[c][e] * unscale);
     if (slice == 0 && lane == 0 && members[c]) atomicAdd(cnt + (size_t)prob * P + j, members[c]);
   }
 }
 
 template <int CPW, int E, int ES>
 constexpr size_t accum_smem() {
-  return (size_t)accum_stages<32 * E * ES>() * (kAccT * 32 * E * ES) + 2 * 4 * sizeof(uint64_t);
+  return (size_t)accum_stages<CPW, 32 * E * ES, ES>() * (kAccT * 32 * E * ES) + 2 * 4 * sizeof(uint64_t);
 }
 
 template <int CPW, int E, int ES>
@@ -731,7 +767,7 @@ cudaError_t launch_accum_t(const CUtensorMap& amap, const Src& s, int P, int NP,
   if (e != cudaSuccess) return e;
   const int slices = 4 / E;
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
-  const int64_t want = std::max<int64_t>(1, sms / std::max(1, slices * NP));
+  const int64_t want = std::max<int64_t>(1, accum_ctas_per_sm<CPW, ES>() * sms / std::max(1, slices * NP));
   const unsigned chunks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, want));
   mine_accum_kernel<CPW, E, ES><<<dim3(chunks, slices, NP), (kAccWarps + 1) * 32, smem, st>>>(amap, s, P, assign,
                                                                                               sums, cnt);
@@ -771,9 +807,14 @@ cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, i
 //     of the certification above); commits to the buffer's "full" and the stage's "free"
 //     barriers;
 //   * 8 epilogue warps, two warpgroups: warpgroup g owns TMEM buffer g and takes every other
-//     tile; token t's scores are TMEM lane t, so each warp handles its 32 tokens alone (top-2
-//     over all patterns, |x|^2 from the staged tile, the gap test and, for a token that fails
-//     it, the float64 recomputation of its candidates), with no barrier between warps.
+//     tile; token t's scores are TMEM lane t, so each warp handles its 32 tokens alone, with
+//     no barrier between warps: u_j = |m_j|^2 / 2 - x.m_j (e_j = 2 u_j) with the pattern index
+//     written into the 7 low mantissa bits (a move of at most 2^-16 |u_j|), one running pair
+//     of smallest tagged values per chain, so one min chain yields the candidate, its index
+//     and the gap; the gap test widened by twice the largest move.  A token that fails it
+//     (well under 1 %) is listed for mine_fixup_kernel, which decides it with float64
+//     distances before the cluster sums.  |x|^2 comes from the staged tile in the first
+//     iteration and from a per-token cache after that.
 // Every mbarrier wait is bounded.
 constexpr int kTcM = 128;
 constexpr int kTcMaxStages = 2;  // two CTAs per SM share the SM's shared memory and TMEM
@@ -840,12 +881,26 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
 }
 
 
+constexpr float kTcPad = 1.0e38f;  // |m_j|^2 / 2 of the padding patterns past P: never the minimum
+
+// u with its 7 low mantissa bits replaced by j (j < 128)
+__device__ __forceinline__ float tag_score(float u, int j) {
+  return __uint_as_float((__float_as_uint(u) & 0xFFFFFF80u) | (uint32_t)j);
+}
+// running two smallest values
+__device__ __forceinline__ void low2_add(float& m1, float& m2, float v) {
+  m2 = fminf(m2, fmaxf(m1, v));
+  m1 = fminf(m1, v);
+}
 __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s,
                                                                       int P, const float* __restrict__ M,
-                                                                      int32_t* __restrict__ assign, int nst) {
+                                                                      int32_t* __restrict__ assign,
+                                                                      float* __restrict__ xsq_cache, int first,
+                                                                      int32_t* __restrict__ amb,
+                                                                      int32_t* __restrict__ amb_cnt, int nst) {
   const int prob = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Pn = (P + 7) & ~7, N = 2 * Pn;
+  const int Pn = (P + 15) & ~15, N = 2 * Pn;
   const uint32_t tcols = N <= 128 ? 256u : 512u;  // two accumulator buffers
   const uint32_t buf_cols = tcols / 2;
   const uint32_t half_b = (uint32_t)N * 128u;      // B: channels 64-127 start N x 128 B in
@@ -853,9 +908,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   uint8_t* Bt = base;                                                   // [2 halves][N rows][128 B], swizzled
   uint8_t* At = base + (size_t)N * kD * 2;                              // [nst][2 halves][128 rows][128 B]
-  float* msq = reinterpret_cast<float*>(At + (size_t)nst * kTcTileBytes);  // [Pn]
-  float* mnorm = msq + Pn;                                              // [Pn]
-  float* gmax = mnorm + Pn;                                             // [4]
+  float* hm = reinterpret_cast<float*>(At + (size_t)nst * kTcTileBytes);   // [Pn] |m_j|^2 / 2, padding past P
+  float* gmax = hm + Pn;                                                // [4]
   uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);               // full[nst], sfree[nst], tfull[2], tempty[2]
   uint64_t* full = bars;
   uint64_t* sfree = bars + nst;
@@ -908,10 +962,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     double acc = 0.0;
     if (j < P)
       for (int d = 0; d < kD; ++d) { const double m = Mp[(size_t)j * kD + d]; acc += m * m; }
-    msq[j] = (float)acc;
-    mnorm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
-    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int(mnorm[j]));
-    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq[j] * (1.0f + 1e-6f)));
+    const float msq = (float)acc;
+    hm[j] = j < P ? 0.5f * msq : kTcPad;
+    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int((float)(sqrt(acc) * (1.0 + 1e-6))));
+    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq * (1.0f + 1e-6f)));
   }
   fence_proxy_async();  // B (generic stores) before the tensor cores read it
   tc_fence_before();
@@ -966,332 +1020,20 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)wg * buf_cols;
     for (int k = wg; k < nt; k += 2) {
       const int st = k % nst;
-      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) break;
-      tc_fence_after();
-      // |x|^2 of the row from the staged tile (two swizzled halves of 64 channels)
-      float xs[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint8_t* stg = At + (size_t)st * kTcTileBytes;
-#pragma unroll
-      for (int hc = 0; hc < 16; ++hc) {
-        const uint4 u = *reinterpret_cast<const uint4*>(stg + (hc >> 3) * (kTcTileBytes / 2) + sw128_off(row, hc & 7));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float v0 = __uint_as_float(w[q] << 16), v1 = __uint_as_float(w[q] & 0xFFFF0000u);
-          xs[q] = fmaf(v0, v0, xs[q]);
-          xs[q] = fmaf(v1, v1, xs[q]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mb_arrive(&sfree[st]);
-      Top2 top{INFINITY, INFINITY, 0}, top_b{INFINITY, INFINITY, 0};  // even / odd patterns: two chains
-      // 8 columns at a time; the loads of block c0 + 8 are in flight while block c0 is scored
-      float hv[8], mv[8];
-      tmem_ld8_issue(taddr, hv);
-      tmem_ld8_issue(taddr + Pn, mv);
-      tmem_ld_wait();
-      for (int c0 = 0; c0 < Pn; c0 += 8) {
-        float hn[8], mn_[8];
-        const bool more = c0 + 8 < Pn;
-        if (more) {
-          tmem_ld8_issue(taddr + c0 + 8, hn);
-          tmem_ld8_issue(taddr + Pn + c0 + 8, mn_);
-        }
-#pragma unroll
-        for (int q = 0; q < 8; q += 2) {
-          const int j = c0 + q;
-          if (j < P) top2_add(top, msq[j] - 2.0f * (hv[q] + mv[q]), j);
-          if (j + 1 < P) top2_add(top_b, msq[j + 1] - 2.0f * (hv[q + 1] + mv[q + 1]), j + 1);
-        }
-        if (more) {
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) { hv[q] = hn[q]; mv[q] = mn_[q]; }
-        }
-      }
-      if (top_b.m1 < top.m1 || (top_b.m1 == top.m1 && top_b.j1 < top.j1)) {
-        top.m2 = fminf(top.m1, top_b.m2);
-        top.m1 = top_b.m1;
-        top.j1 = top_b.j1;
-      } else {
-        top.m2 = fminf(top.m2, top_b.m1);
-      }
-      const int64_t i = tile_t0(k) + row;
-      const float xsq = ((xs[0] + xs[1]) + (xs[2] + xs[3])) * (1.0f + 1e-6f);
-      const float nx = sqrtf(xsq) * (1.0f + 1e-6f);
-      const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xsq + msq_max);
-      const bool unique = top.m2 - top.m1 > 2.0f * Eb + 1e-9f * (xsq + msq_max);
-      if (unique && i < s.n) assign[(size_t)prob * s.n + i] = top.j1;
-      const bool need = !unique && i < s.n;
-      if (__any_sync(kFull, need)) {
-        // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
-        float U = INFINITY;
-        for (int c0 = 0; c0 < Pn; c0 += 8) {
-          float hv[8], mv[8];
-          tmem_ld8_issue(taddr + c0, hv);
-          tmem_ld8_issue(taddr + Pn + c0, mv);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = c0 + q;
-            if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]));
-          }
-        }
-        uint32_t cand[4] = {0u, 0u, 0u, 0u};  // candidate bit mask over j < 128
-        for (int c0 = 0; c0 < Pn; c0 += 8) {
-          float hv[8], mv[8];
-          tmem_ld8_issue(taddr + c0, hv);
-          tmem_ld8_issue(taddr + Pn + c0, mv);
-          tmem_ld_wait();
-          uint32_t cm = 0u;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = c0 + q;
-            const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
-            const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xsq + msq[j]);
-            if (j < P && e - E <= U + 1e-9f * (xsq + msq[j])) cm |= 1u << q;
-          }
-          cand[c0 >> 5] |= cm << (c0 & 31);
-        }
-        if (need) {
-          const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
-          double bd = 0.0;
-          int bj = 0;
-          bool have = false;
-          for (int cw = 0; cw < 4; ++cw)
-            for (uint32_t m = cand[cw]; m; m &= m - 1) {
-              const int j = cw * 32 + __ffs(m) - 1;
-              const float* mrow = Mp + (size_t)j * kD;
-              double acc = 0.0;
-#pragma unroll 8
-              for (int d = 0; d < kD; d += 4) {
-                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
-                const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-                const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
-                const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
-                  acc = __dadd_rn(acc, __dmul_rn(t, t));
-                }
-              }
-              if (!have || acc < bd) { bd = acc; bj = j; have = true; }
-            }
-          assign[(size_t)prob * s.n + i] = bj;
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mb_arrive(&tempty[wg]);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
-}
-
-// ---- fused Lloyd step: bf16 input, P <= 64 ------------------------------------------------
-//
-// One pass over x per iteration: the assignment of mine_assign_tc_kernel and the cluster sums
-// of mine_accum_kernel from the same staged tile.  One CTA per SM, warp-specialised, no block
-// barrier in the loop:
-//   * warp 0: TMA loads of 128-token tiles into a ring of stages (as mine_assign_tc_kernel);
-//   * warp 1: the distance contraction of each tile into one of two TMEM buffers (as there);
-//   * warps 2-9, two warpgroups (warpgroup g takes the tiles k with k % 2 == g, TMEM buffer g),
-//     one token per thread: u_j = |m_j|^2 / 2 - x.m_j (so e_j = 2 u_j) with the pattern index
-//     written into the 6 low mantissa bits, which moves u_j by at most 2^-17 |u_j|.  The two
-//     smallest tagged scores give the candidate and the gap; the gap test of
-//     mine_assign_tc_kernel, widened by twice the largest such move, certifies the candidate,
-//     and a token that fails it is decided by the float64 recomputation of its candidates.
-//     |x|^2 comes from the staged tile in the first iteration and from a per-token cache after
-//     that.  The tile's assignment goes to shared memory (and to `assign`);
-//   * warps 10-17: warp a owns the clusters j with j % 8 == a and keeps their float64 sums
-//     (channels 4l .. 4l + 3 in lane l) in registers for the whole kernel; one ballot per 32
-//     tokens of a tile finds its members (the assigners count them in shared memory).  At the
-//     end each warp adds its totals to global memory.  float64 sums of bf16 values are exact, so the order of the additions
-//     does not change them.
-// A stage is refilled once the MMA has read it and every accumulator warp is done with it.
-// Every mbarrier wait is bounded.
-constexpr int kLlAsgWarps = 8;
-constexpr int kLlAccWarps = 8;
-constexpr int kLlThreads = (2 + kLlAsgWarps + kLlAccWarps) * 32;
-constexpr int kLlMaxStages = 6;
-constexpr float kLlPad = 1.0e38f;  // |m_j|^2 / 2 of the padding patterns past P: never the minimum
-
-// dynamic shared memory: B (N rows x 256 B), the stages, their assignments, the pattern
-// tables, the barriers, and the slack for 1024-byte alignment
-size_t ll_smem_bytes(int P, int nst) {
-  const int Pn = (P + 7) & ~7, N = 2 * Pn;
-  return (size_t)N * 256 + (size_t)nst * kTcTileBytes + (size_t)nst * kTcM * 4 + (size_t)4 * Pn * 4 + 16 +
-         (size_t)(3 * nst + 4) * 8 + 16 + 1024;
-}
-int mine_ll_stages(int P) {
-  int nst = kLlMaxStages;
-  while (nst > 2 && ll_smem_bytes(P, nst) > 227 * 1024) --nst;
-  return nst;
-}
-
-// u with its 6 low mantissa bits replaced by j (j < 64)
-__device__ __forceinline__ float tag_score(float u, int j) {
-  return __uint_as_float((__float_as_uint(u) & 0xFFFFFFC0u) | (uint32_t)j);
-}
-// running two smallest values
-__device__ __forceinline__ void low2_add(float& m1, float& m2, float v) {
-  m2 = fminf(m2, fmaxf(m1, v));
-  m1 = fminf(m1, v);
-}
-
-__global__ void __launch_bounds__(kLlThreads, 1)
-    mine_lloyd_tc_kernel(const __grid_constant__ CUtensorMap xmap, Src s, int P, const float* __restrict__ M,
-                         int32_t* __restrict__ assign, float* __restrict__ xsq_cache, int first,
-                         double* __restrict__ sums, uint32_t* __restrict__ cnt, int nst) {
-  const int prob = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Pn = (P + 7) & ~7, N = 2 * Pn;
-  uint32_t tcols = 32;
-  while (tcols < 2u * (uint32_t)N) tcols <<= 1;  // two accumulator buffers
-  const uint32_t buf_cols = tcols / 2;
-  const uint32_t half_b = (uint32_t)N * 128u;  // B: channels 64-127 start N x 128 B in
-  extern __shared__ __align__(16) uint8_t smraw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  uint8_t* Bt = base;                                                                   // [2][N][128 B]
-  uint8_t* At = base + (size_t)N * 256;                                                 // [nst][2][128][128 B]
-  int32_t* asg = reinterpret_cast<int32_t*>(At + (size_t)nst * kTcTileBytes);           // [nst][128]
-  float* msq = reinterpret_cast<float*>(asg + nst * kTcM);                              // [Pn]
-  float* hm = msq + Pn;                                                                 // [Pn]
-  float* mnorm = hm + Pn;                                                               // [Pn]
-  float* gmax = mnorm + Pn;                                                             // [4]
-  uint32_t* members = reinterpret_cast<uint32_t*>(gmax + 4);                            // [Pn]
-  uint64_t* full = reinterpret_cast<uint64_t*>(members + Pn);
-  uint64_t* sfree = full + nst;
-  uint64_t* asgd = sfree + nst;
-  uint64_t* tfull = asgd + nst;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
-  const float* Mp = M + (size_t)prob * P * kD;
-  const int set = prob / s.heads, h = prob % s.heads;
-
-  // ---- B: bf16 hi parts (rows 0..Pn-1) and mid parts (rows Pn..2Pn-1) of the patterns
-  for (int i = tid; i < N * 16; i += blockDim.x) {
-    const int n = i >> 4, c = i & 15;
-    const int j = n < Pn ? n : n - Pn;
-    uint32_t wv[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint16_t hv[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float m = j < P ? Mp[(size_t)j * kD + 8 * c + 2 * q + e] : 0.f;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(m);
-        const __nv_bfloat16 v = n < Pn ? hi : __float2bfloat16_rn(m - __bfloat162float(hi));
-        hv[e] = __bfloat16_as_ushort(v);
-      }
-      wv[q] = (uint32_t)hv[0] | ((uint32_t)hv[1] << 16);
-    }
-    *reinterpret_cast<uint4*>(Bt + (size_t)(c >> 3) * half_b + sw128_off(n, c & 7)) =
-        make_uint4(wv[0], wv[1], wv[2], wv[3]);
-  }
-  if (tid == 0) {
-    gmax[0] = 0.f;
-    gmax[1] = 0.f;
-    for (int i = 0; i < nst; ++i) {
-      mb_init(&full[i], 1);
-      mb_init(&sfree[i], 1 + kLlAccWarps);    // the MMA commit and every accumulator warp
-      mb_init(&asgd[i], kLlAsgWarps / 2);     // the 4 warps of the tile's warpgroup
-    }
-    for (int i = 0; i < 2; ++i) {
-      mb_init(&tfull[i], 1);
-      mb_init(&tempty[i], kLlAsgWarps / 2);  // buffer i belongs to warpgroup i
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tslot)), "r"(tcols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  __syncthreads();
-  for (int j = tid; j < Pn; j += blockDim.x) {
-    double acc = 0.0;
-    if (j < P)
-      for (int d = 0; d < kD; ++d) { const double m = Mp[(size_t)j * kD + d]; acc += m * m; }
-    msq[j] = (float)acc;
-    hm[j] = j < P ? 0.5f * (float)acc : kLlPad;
-    members[j] = 0u;
-    mnorm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
-    atomicMax(reinterpret_cast<int*>(&gmax[0]), __float_as_int(mnorm[j]));
-    atomicMax(reinterpret_cast<int*>(&gmax[1]), __float_as_int(msq[j] * (1.0f + 1e-6f)));
-  }
-  fence_proxy_async();  // B (generic stores) before the tensor cores read it
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = *tslot;
-
-  const int64_t ntiles = (s.n + kTcM - 1) / kTcM;
-  const int nt = ntiles > blockIdx.x ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
-  auto tile_t0 = [&](int k) { return ((int64_t)blockIdx.x + (int64_t)k * gridDim.x) * kTcM; };
-
-  if (warp == 0) {
-    // ---- producer
-    if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
-      int issued = 0;
-      for (int k = 0; k < nt; ++k) {
-        const int st = k % nst;
-        if (k >= nst && !tc_wait(&sfree[st], (uint32_t)(((k / nst) - 1) & 1))) break;
-        uint8_t* dst = At + (size_t)st * kTcTileBytes;
-        mb_expect_tx(&full[st], (uint32_t)kTcTileBytes);
-        const int t0 = (int)tile_t0(k);
-        tma_load_4d(dst, &xmap, 0, h, t0, set, &full[st]);
-        tma_load_4d(dst + kTcTileBytes / 2, &xmap, 64, h, t0, set, &full[st]);
-        issued = k + 1;
-      }
-      // every copy issued has landed before the CTA may leave (bounded, as every wait)
-      for (int k = max(0, issued - nst); k < issued; ++k) (void)tc_wait(&full[k % nst], (uint32_t)((k / nst) & 1));
-    }
-  } else if (warp == 1) {
-    // ---- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc(kTcM, N);
-      const uint32_t b0 = su32(Bt);
-      for (int k = 0; k < nt; ++k) {
-        const int st = k % nst, buf = k & 1;
-        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1))) break;
-        if (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1))) break;
-        tc_fence_after();
-        const uint32_t a0 = su32(At + (size_t)st * kTcTileBytes);
-        const uint32_t d = tbase + (uint32_t)buf * buf_cols;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks)  // K step ks: half ks / 4, 32 B per step inside the atom
-          umma_bf16(d, umma_desc_sw128(a0 + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32),
-                    umma_desc_sw128(b0 + (ks >> 2) * half_b + (ks & 3) * 32), idesc, ks > 0);
-        umma_commit(&tfull[buf]);
-        umma_commit(&sfree[st]);
-      }
-    }
-  } else if (warp < 2 + kLlAsgWarps) {
-    // ---- assigners: warpgroup g, TMEM lane quarter q4, token `row` of the tile
-    const int g = (warp - 2) >> 2, q4 = warp & 3;
-    const int row = q4 * 32 + lane;
-    const float nm_max = gmax[0], msq_max = gmax[1];
-    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)g * buf_cols;
-    for (int k = g; k < nt; k += 2) {
-      const int st = k % nst;
       const int64_t i = tile_t0(k) + row;
       const bool valid = i < s.n;
       float xsq = 0.f;
       if (!first && valid) xsq = xsq_cache[(size_t)prob * s.n + i];
-      if (!__all_sync(kFull, tc_wait(&tfull[g], (uint32_t)((k >> 1) & 1)))) break;
+      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) break;
       tc_fence_after();
+      float hv[8], mv[8], hn[8], mn_[8];
+      tmem_ld8_issue(taddr, hv);
+      tmem_ld8_issue(taddr + Pn, mv);
       if (first) {
         // |x|^2 of the row from the staged tile (two swizzled halves of 64 channels)
         const uint8_t* stg = At + (size_t)st * kTcTileBytes;
         float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
+#pragma unroll 2
         for (int hc = 0; hc < 16; ++hc) {
           const uint4 u = *reinterpret_cast<const uint4*>(stg + (hc >> 3) * (kTcTileBytes / 2) + sw128_off(row, hc & 7));
           const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -1305,31 +1047,30 @@ __global__ void __launch_bounds__(kLlThreads, 1)
         xsq = (a0 + a1) + (b0 + b1);
         if (valid) xsq_cache[(size_t)prob * s.n + i] = xsq;
       }
-      const float xs = xsq * (1.0f + 1e-6f);
-      const float nx = sqrtf(xs) * (1.0f + 1e-6f);
-      // the two smallest tagged scores, in two chains (even / odd patterns)
-      float m1a = INFINITY, m2a = INFINITY, m1b = INFINITY, m2b = INFINITY;
-      float hv[8], mv[8];
-      tmem_ld8_issue(taddr, hv);
-      tmem_ld8_issue(taddr + Pn, mv);
+      __syncwarp();
+      if (lane == 0) mb_arrive(&sfree[st]);
       tmem_ld_wait();
+      // the two smallest tagged scores in two chains (even / odd patterns); blocks of 8
+      // columns, the next block's loads in flight while one is scored
+      float m1a = INFINITY, m2a = INFINITY, m1b = INFINITY, m2b = INFINITY;
       for (int c0 = 0; c0 < Pn; c0 += 8) {
-        float hn[8], mn_[8];
         const bool more = c0 + 8 < Pn;
         if (more) {
           tmem_ld8_issue(taddr + c0 + 8, hn);
           tmem_ld8_issue(taddr + Pn + c0 + 8, mn_);
         }
-        const float4 ha = *reinterpret_cast<const float4*>(hm + c0);
-        const float4 hb = *reinterpret_cast<const float4*>(hm + c0 + 4);
-        const float hq[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
 #pragma unroll
-        for (int q = 0; q < 8; q += 2) {
-          float s0, s1, u0, u1;
+        for (int q = 0; q < 8; q += 4) {
+          const float4 hq = *reinterpret_cast<const float4*>(hm + c0 + q);
+          float s0, s1, s2, s3, u0, u1, u2, u3;
           add2f(hv[q], hv[q + 1], mv[q], mv[q + 1], s0, s1);
-          sub2(hq[q], hq[q + 1], s0, s1, u0, u1);
+          add2f(hv[q + 2], hv[q + 3], mv[q + 2], mv[q + 3], s2, s3);
+          sub2(hq.x, hq.y, s0, s1, u0, u1);
+          sub2(hq.z, hq.w, s2, s3, u2, u3);
           low2_add(m1a, m2a, tag_score(u0, c0 + q));
           low2_add(m1b, m2b, tag_score(u1, c0 + q + 1));
+          low2_add(m1a, m2a, tag_score(u2, c0 + q + 2));
+          low2_add(m1b, m2b, tag_score(u3, c0 + q + 3));
         }
         if (more) {
           tmem_ld_wait();
@@ -1339,156 +1080,92 @@ __global__ void __launch_bounds__(kLlThreads, 1)
       }
       const float m1 = fminf(m1a, m1b);
       const float m2 = fminf(fmaxf(m1a, m1b), fminf(m2a, m2b));
-      int jw = (int)(__float_as_uint(m1) & 63u);
-      // e = 2 u: certified when the gap beats both error bounds and both tags' moves
+      const float xs = xsq * (1.0f + 1e-6f);
+      const float nx = sqrtf(xs) * (1.0f + 1e-6f);
       const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xs + msq_max);
-      const float Pe = 0x1p-17f * (msq_max + 2.0f * nx * nm_max);
-      const bool unique = 2.0f * (m2 - m1) > 2.0f * Eb + 2.0f * Pe + 1e-9f * (xs + msq_max);
-      const bool need = !unique && valid;
-      if (__any_sync(kFull, need)) {
-        // candidate window from the same scores (whole warp re-reads, only `need` lanes use them)
-        float U = INFINITY;
-        for (int c0 = 0; c0 < Pn; c0 += 8) {
-          tmem_ld8_issue(taddr + c0, hv);
-          tmem_ld8_issue(taddr + Pn + c0, mv);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = c0 + q;
-            if (j < P) U = fminf(U, msq[j] - 2.0f * (hv[q] + mv[q]) + 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xs + msq[j]));
-          }
-        }
-        uint32_t cand[2] = {0u, 0u};  // candidate bit mask over j < 64
-        for (int c0 = 0; c0 < Pn; c0 += 8) {
-          tmem_ld8_issue(taddr + c0, hv);
-          tmem_ld8_issue(taddr + Pn + c0, mv);
-          tmem_ld_wait();
-          uint32_t cm = 0u;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = c0 + q;
-            const float e = msq[j] - 2.0f * (hv[q] + mv[q]);
-            const float E = 0x1p-12f * nx * mnorm[j] + 0x1p-20f * (xs + msq[j]);
-            if (j < P && e - E <= U + 1e-9f * (xs + msq[j])) cm |= 1u << q;
-          }
-          cand[c0 >> 5] |= cm << (c0 & 31);
-        }
-        if (need) {
-          const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
-          double bd = 0.0;
-          int bj = 0;
-          bool have = false;
-          for (int cw = 0; cw < 2; ++cw)
-            for (uint32_t m = cand[cw]; m; m &= m - 1) {
-              const int j = cw * 32 + __ffs(m) - 1;
-              const float* mrow = Mp + (size_t)j * kD;
-              double acc = 0.0;
-#pragma unroll 8
-              for (int d = 0; d < kD; d += 4) {
-                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xrow + d));
-                const float xv[4] = {__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u)};
-                const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + d));
-                const float mv4[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const double t = __dsub_rn((double)xv[q], (double)mv4[q]);
-                  acc = __dadd_rn(acc, __dmul_rn(t, t));
-                }
-              }
-              if (!have || acc < bd) { bd = acc; bj = j; have = true; }
-            }
-          jw = bj;
-        }
-      }
+      const float Pe = 0x1p-16f * (msq_max + 2.0f * nx * nm_max);  // largest tag move of e = 2 u
       if (valid) {
-        assign[(size_t)prob * s.n + i] = jw;
-        atomicAdd(&members[jw], 1u);
+        if (2.0f * (m2 - m1) > 2.0f * Eb + 2.0f * Pe + 1e-9f * (xs + msq_max))
+          assign[(size_t)prob * s.n + i] = (int32_t)(__float_as_uint(m1) & 127u);
+        else
+          amb[(size_t)prob * s.n + atomicAdd(amb_cnt + prob, 1)] = (int32_t)i;
       }
-      asg[st * kTcM + row] = valid ? jw : -1;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mb_arrive(&asgd[st]);
-        mb_arrive(&tempty[g]);
-      }
-    }
-  } else {
-    // ---- accumulators: warp aw owns clusters aw + 8 c; lane l holds channels 4l .. 4l + 3
-    const int aw = warp - 2 - kLlAsgWarps;
-    double acc[8][4];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[c][e] = 0.0;
-    }
-    // channels 4l .. 4l + 3: half l >> 4, 16-byte chunk (l >> 1) & 7 of the swizzled row, 8 bytes in when l is odd
-    const uint32_t lane_off = (uint32_t)(lane >> 4) * (kTcTileBytes / 2) + (uint32_t)(lane & 1) * 8u;
-    const int cidx = (lane >> 1) & 7;
-    for (int k = 0; k < nt; ++k) {
-      const int st = k % nst;
-      if (!__all_sync(kFull, tc_wait(&asgd[st], (uint32_t)((k / nst) & 1)))) break;
-      const int32_t* as = asg + st * kTcM;
-      int aj[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) aj[q] = as[32 * q + lane];
-      const uint8_t* stg = At + (size_t)st * kTcTileBytes + lane_off;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t m = __ballot_sync(kFull, aj[q] >= 0 && (aj[q] & 7) == aw);
-        while (m) {
-          const int t = 32 * q + __ffs(m) - 1;
-          m &= m - 1;
-          const int c = __shfl_sync(kFull, aj[q], t & 31) >> 3;
-          const uint2 u = *reinterpret_cast<const uint2*>(stg + (t >> 3) * 1024 + (t & 7) * 128 + ((cidx ^ (t & 7)) << 4));
-          const double v0 = (double)__uint_as_float(u.x << 16), v1 = (double)__uint_as_float(u.x & 0xFFFF0000u);
-          const double v2 = (double)__uint_as_float(u.y << 16), v3 = (double)__uint_as_float(u.y & 0xFFFF0000u);
-          switch (c) {
-#define KVQ_LL_ACC(C)                                                                     \
-  case C:                                                                                 \
-    acc[C][0] += v0; acc[C][1] += v1; acc[C][2] += v2; acc[C][3] += v3; break;
-            KVQ_LL_ACC(0) KVQ_LL_ACC(1) KVQ_LL_ACC(2) KVQ_LL_ACC(3)
-            KVQ_LL_ACC(4) KVQ_LL_ACC(5) KVQ_LL_ACC(6) KVQ_LL_ACC(7)
-#undef KVQ_LL_ACC
-            default: break;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mb_arrive(&sfree[st]);
-    }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int j = aw + 8 * c;
-      if (j >= P) break;
-      double* gs = sums + ((size_t)prob * P + j) * kD + 4 * lane;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (acc[c][e] != 0.0) atomicAdd(gs + e, acc[c][e]);
+      if (lane == 0) mb_arrive(&tempty[wg]);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  for (int j = tid; j < P; j += blockDim.x)
-    if (members[j]) atomicAdd(cnt + (size_t)prob * P + j, members[j]);
   if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
 }
 
+// Tokens the tcgen05 assignment listed as undecided: float64 squared distances to every
+// pattern (channels in order, as the sequential definition), the lowest index among equal
+// distances.  A 128-thread block takes one token at a time, one thread per pattern (P <= 128).
+__global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
+                                                         const int32_t* __restrict__ amb,
+                                                         const int32_t* __restrict__ amb_cnt,
+                                                         int32_t* __restrict__ assign) {
+  const int prob = blockIdx.y, j = threadIdx.x;
+  __shared__ float xr[kD];
+  __shared__ double dist[128];
+  const int count = amb_cnt[prob];
+  const float* Mp = M + (size_t)prob * P * kD;
+  for (int r = blockIdx.x; r < count; r += gridDim.x) {
+    const int64_t i = amb[(size_t)prob * s.n + r];
+    xr[j] = s.at(prob, i, j);
+    __syncthreads();
+    double d = 0.0;
+    if (j < P) {
+      // the pattern row arrives 32 channels (eight 16-byte loads) at a time; the sum runs over
+      // the channels in order
+      const float4* m4 = reinterpret_cast<const float4*>(Mp + (size_t)j * kD);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float4 mv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mv[u] = __ldg(m4 + c0 / 4 + u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float m[4] = {mv[u].x, mv[u].y, mv[u].z, mv[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const double t = __dsub_rn((double)xr[c0 + 4 * u + e], (double)m[e]);
+            d = __dadd_rn(d, __dmul_rn(t, t));
+          }
+        }
+      }
+    }
+    dist[j] = d;
+    __syncthreads();
+    if (j == 0) {
+      double bd = dist[0];
+      int bj = 0;
+      for (int q = 1; q < P; ++q)
+        if (dist[q] < bd) { bd = dist[q]; bj = q; }
+      assign[(size_t)prob * s.n + i] = bj;
+    }
+    __syncthreads();
+  }
+}
+
 // ring depth that fits next to the patterns in 227 KB, and the dynamic shared memory it needs
 int mine_tc_stages(int P) {
-  const int Pn = (P + 7) & ~7;
-  const int fixed = 2 * Pn * kD * 2 + 2 * Pn * 4 + 16 + (2 * kTcMaxStages + 4) * 8 + 16 + 1024;
+  const int Pn = (P + 15) & ~15;
+  const int fixed = 2 * Pn * kD * 2 + Pn * 4 + 16 + (2 * kTcMaxStages + 4) * 8 + 16 + 1024;
   return std::max(2, std::min(kTcMaxStages, (227 * 1024 - fixed) / kTcTileBytes));
 }
 size_t mine_tc_smem(int P) {
-  const int Pn = (P + 7) & ~7, nst = mine_tc_stages(P);
-  return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + 2 * Pn * 4 + 16 + (2 * nst + 4) * 8 + 16 + 1024;
+  const int Pn = (P + 15) & ~15, nst = mine_tc_stages(P);
+  return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + Pn * 4 + 16 + (2 * nst + 4) * 8 + 16 + 1024;
 }
 
-__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt) {
+__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt, int32_t* amb_cnt) {
   const int prob = blockIdx.y, j = blockIdx.x, d = threadIdx.x;
+  if (amb_cnt && j == 0 && d == 0) amb_cnt[prob] = 0;  // the next iteration's list starts empty
   const size_t pj = (size_t)prob * P + j;
   uint32_t c = cnt[pj];
   if (c > 0) M[pj * kD + d] = (float)(sums[pj * kD + d] / (double)c);
@@ -1502,7 +1179,8 @@ __global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt)
 size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
   size_t NP = (size_t)sets * heads;
   size_t b = align256(NP * P * kD * sizeof(double)) + align256(NP * P * sizeof(uint32_t)) +
-             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * (size_t)n * sizeof(float));
+             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * (size_t)n * sizeof(float)) +
+             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * sizeof(int32_t));
   if (transform)
     b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
          4 * align256(NP * kD * sizeof(double));
@@ -1577,6 +1255,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   }
 
   mine_init_kernel<<<dim3(a.P, NP), kD, 0, st>>>(s, a.P, a.patterns);
+  cudaMemsetAsync(w.amb_cnt, 0, (size_t)NP * sizeof(int32_t), st);
   cudaMemsetAsync(w.sums, 0, (size_t)NP * a.P * kD * sizeof(double), st);
   cudaMemsetAsync(w.cnt, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
   size_t smem_assign = (size_t)a.P * kD * sizeof(float);
@@ -1616,27 +1295,14 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   }
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, (a.P <= 64 ? 2 : 1) * sms / NP)));
-  // bf16 input and P <= 64: assignment and cluster sums in one pass (one CTA per SM)
-  const bool use_ll = KIND == 0 && a.P <= 8 * kLlAccWarps;
-  const int ll_nst = mine_ll_stages(a.P);
-  const size_t smem_ll = ll_smem_bytes(a.P, ll_nst);
-  if (use_ll && (e = cudaFuncSetAttribute(mine_lloyd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem_ll)) != cudaSuccess)
-    return e;
-  const unsigned ll_ctas = (unsigned)std::max<int64_t>(
-      1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
-    if (use_ll) {
-      mine_lloyd_tc_kernel<<<dim3(ll_ctas, NP), kLlThreads, smem_ll, st>>>(xmap, s, a.P, a.patterns, w.assign, w.xsq,
-                                                                           it == 0, w.sums, w.cnt, ll_nst);
-      mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
-      continue;
-    }
-    if (use_tc)
-      mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(xmap, s, a.P, a.patterns, w.assign,
-                                                                             mine_tc_stages(a.P));
-    else if (use_mma && KIND == 0)
+    if (use_tc) {
+      mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
+          xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P));
+      mine_fixup_kernel<<<dim3((unsigned)std::max(1, std::min(256, sms * 16 / NP)), NP), 128, 0, st>>>(
+          s, a.P, a.patterns, w.amb, w.amb_cnt, w.assign);
+    } else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else if (use_mma && KIND == 1)
       mine_assign_mma_kernel<1><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
@@ -1646,7 +1312,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
       mine_assign_kernel<<<dim3((unsigned)((a.n + 127) / 128), NP), 128, smem_assign, st>>>(s, a.P, a.patterns,
                                                                                            w.assign);
     if ((e = launch_accum(amap, s, a.P, NP, sms, w.assign, w.sums, w.cnt, st)) != cudaSuccess) return e;
-    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt);
+    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt, use_tc ? w.amb_cnt : nullptr);
   }
   return cudaGetLastError();
 }
