@@ -28,6 +28,8 @@
 //   2 keeps every tail read ahead of every tail write.
 #include <algorithm>
 
+#include <cuda_fp16.h>
+
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -227,22 +229,24 @@ __device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const
   return word;
 }
 
-// Lower bounds over the first NPROBE probe channels for patterns [j0, j1) of one staged vector
-// y (one lane), written to lbuf[j][row]; running argmin (ties: lowest j) to (blb, bj).
+// Lower bounds over the NPROBE probe channels pc (shared memory) for patterns [j0, j1) of one
+// staged vector y (one lane), from the patterns' values there (shared memory, [P][NPROBE]);
+// written to lbuf[j][row] rounded toward zero to fp16 (still a lower bound); running argmin
+// of the fp32 bounds (ties: lowest j) to (blb, bj).
 template <int NPROBE>
-__device__ __forceinline__ void lb_pass(const float* y, const int32_t* __restrict__ pc, const float* __restrict__ pvt,
-                                        int j0, int j1, float* lbuf, int row, float& blb_out, int& bj_out) {
+__device__ __forceinline__ void lb_pass(const float* y, const int32_t* pc, const float* pvt, int j0, int j1,
+                                        __half* lbuf, int row, float& blb_out, int& bj_out) {
   float py[NPROBE];
 #pragma unroll
-  for (int u = 0; u < NPROBE; ++u) py[u] = y[__ldg(pc + u)];
+  for (int u = 0; u < NPROBE; ++u) py[u] = y[pc[u]];
   float blb = INFINITY;
   int bj = j0;
   for (int j = j0; j < j1; ++j) {
-    const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * kProbe);
+    const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * NPROBE);
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
     for (int q = 0; q < NPROBE / 4; ++q) {
-      const float4 m = __ldg(m4 + q);
+      const float4 m = m4[q];
       float r0, r1, r2, r3;
       sub2(py[4 * q], py[4 * q + 1], m.x, m.y, r0, r1);
       sub2(py[4 * q + 2], py[4 * q + 3], m.z, m.w, r2, r3);
@@ -252,7 +256,7 @@ __device__ __forceinline__ void lb_pass(const float* y, const int32_t* __restric
       mn = min3(mn, r2, r3);
     }
     const float lb = __fsub_rn(mx, mn);
-    lbuf[j * (2 * kG) + row] = lb;
+    lbuf[j * (2 * kG) + row] = __float2half_rz(lb);
     if (lb < blb) { blb = lb; bj = j; }
   }
   blb_out = blb;
@@ -282,11 +286,17 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __shared__ unsigned long long best[2 * kG];  // (d_mm bits << 32) | pattern, per row
   __shared__ float dseed[2 * kG], hlb[2][2 * kG];
   __shared__ int seed[2 * kG], hj[2][2 * kG];
-  __shared__ uint32_t queue[kQueueCap];
   __shared__ int qn;
-  // dynamic: lower bounds lb[j][row] during the assignment, then s / z / 1/s tables
+  // dynamic: fp16 lower bounds lb[j][row], then the probe tables (V: [P][32], K: [P][16]) and
+  // probe channels (32 + 16), whose region holds the work queue once the bounds are done;
+  // after the assignment the s / z / 1/s tables reuse the start of the whole region
   extern __shared__ __align__(16) float dsm[];
-  float* lbuf = dsm;           // [P][64 rows] lower bounds
+  __half* lbuf = reinterpret_cast<__half*>(dsm);  // [P][64 rows]
+  float* tabV = dsm + 32 * P;
+  float* tabK = tabV + kProbeV * P;
+  int32_t* pcV = reinterpret_cast<int32_t*>(tabK + kProbeK * P);
+  int32_t* pcK = pcV + kProbeV;
+  uint32_t* queue = reinterpret_cast<uint32_t*>(tabV);  // [kQueueCap]
   float* vsz = dsm;            // [3][4][kG]: s, z, 1/s per (group, V slot)
   float* ksz = dsm + 12 * kG;  // [3][kD]:   s, z, 1/s per K channel
 
@@ -301,6 +311,19 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
                      : k_new + (((size_t)b * n_new + (t - c.L)) * g.H + h) * kD;
   };
   if (tid == 0) qn = 0;
+  {
+    // probe tables of this (set, head): V's 32 probe channels, K's first 16
+    const float4* gV = reinterpret_cast<const float4*>(wsp.pv + (shk + 1) * P * kProbe);
+    const float* gK = wsp.pv + shk * P * kProbe;
+#pragma unroll 4
+    for (int i = tid; i < P * (kProbeV / 4); i += kAppendThreads) reinterpret_cast<float4*>(tabV)[i] = __ldg(gV + i);
+#pragma unroll 2
+    for (int i = tid; i < P * (kProbeK / 4); i += kAppendThreads)
+      reinterpret_cast<float4*>(tabK)[i] =
+          __ldg(reinterpret_cast<const float4*>(gK + (size_t)(i / (kProbeK / 4)) * kProbe) + i % (kProbeK / 4));
+    if (tid < kProbeV) pcV[tid] = __ldg(wsp.probe + (shk + 1) * kProbe + tid);
+    if (tid < kProbeK) pcK[tid] = __ldg(wsp.probe + shk * kProbe + tid);
+  }
 
   // ---- stage (and pre-transform) every vector
   if (!g.tx) {
@@ -353,10 +376,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   {
     const int kind = warp & 1, half = warp >> 1;
     const int r = kind * kG + lane;
-    if (kind == 0) lb_pass<kProbeV>(vec[r], wsp.probe + (shk + 1) * kProbe, wsp.pv + (shk + 1) * P * kProbe,
-                                    half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
-    else if (c.seal) lb_pass<kProbeK>(vec[r], wsp.probe + shk * kProbe, wsp.pv + shk * P * kProbe,
-                                      half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    if (kind == 0) lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    else if (c.seal) lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
   }
   __syncthreads();
 
@@ -386,7 +407,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       const int j1 = hh ? P : P0;
 #pragma unroll 4
       for (int j = hh ? P0 : 0; j < j1; ++j) {
-        const float lb = lbuf[j * (2 * kG) + r];
+        const float lb = __half2float(lbuf[j * (2 * kG) + r]);
         if (j == s || lb > ds || (lb == ds && j > s)) continue;
         const int pos = atomicAdd(&qn, 1);
         if (pos < kQueueCap) queue[pos] = ((uint32_t)r << 16) | (uint32_t)j;
@@ -574,8 +595,10 @@ cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, i
   append_prep_kernel<<<dim3(g.S * g.H, 2), kD, 0, st>>>(g, w);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // lower bounds [P][64 rows], later reused for the s / z tables (12 kG + 3 kD floats)
-  const size_t dyn = std::max<size_t>((size_t)g.P * 2 * kG, 12 * kG + 3 * kD) * sizeof(float);
+  // fp16 lower bounds [P][64 rows], probe tables and channels (later the work queue); later the
+  // s / z tables (12 kG + 3 kD floats) from the start
+  const size_t tabs = std::max<size_t>((size_t)(kProbeV + kProbeK) * g.P + kProbeV + kProbeK, kQueueCap);
+  const size_t dyn = std::max<size_t>((size_t)32 * g.P + tabs, 12 * kG + 3 * kD) * sizeof(float);
   if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
       cudaSuccess)
     return e;

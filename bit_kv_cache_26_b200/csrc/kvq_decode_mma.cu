@@ -338,7 +338,9 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
     for (int k = 0; k < 4; ++k) qk[hh * kD + ksc_pos(lane + 32 * k)] = v[k];
   }
   for (int i = threadIdx.x; i < kWarps * NH * P; i += blockDim.x) Wall[i] = 0.f;
-  __syncthreads();
+  // the transformed query comes from shared memory (after this barrier); the plain one straight
+  // from global memory, so that its loads and the pattern rows' below share one round trip
+  if (g.tx) __syncthreads();
   // T[hh][j] = q_hh . M_K[j] (transformed space): warp w takes patterns w, w + warps, ...;
   // lane l holds channels 4l .. 4l + 3 of four query heads and reads the pattern row with one
   // coalesced 16-byte load; the four head sums are reduced across the warp
@@ -346,19 +348,27 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   for (int hg = 0; hg < NT; ++hg) {
     float qv[4][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 4; ++a) {
+      const int hh = 4 * hg + a;
+      if (g.tx) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) qv[a][e] = qk[(4 * hg + a) * kD + ksc_pos(4 * lane + e)];
-    // eight pattern rows' loads in flight at a time
-    for (int j0 = warp; j0 < P; j0 += 8 * kWarps) {
-      float4 m4[8];
+        for (int e = 0; e < 4; ++e) qv[a][e] = qk[hh * kD + ksc_pos(4 * lane + e)];
+      } else {
+        const uint16_t* src = q + ((size_t)b * Hq + h_kv * Gq + min(hh, Gq - 1)) * kD + 4 * lane;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+        for (int e = 0; e < 4; ++e) qv[a][e] = hh < Gq ? load_elem(src + e, g.dtype) : 0.f;
+      }
+    }
+    // sixteen pattern rows' loads in flight at a time
+    for (int j0 = warp; j0 < P; j0 += 16 * kWarps) {
+      float4 m4[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
         const int j = j0 + u * kWarps;
         m4[u] = j < P ? __ldg(reinterpret_cast<const float4*>(MK + (size_t)j * kD) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const int j = j0 + u * kWarps;
         float t[4];
 #pragma unroll

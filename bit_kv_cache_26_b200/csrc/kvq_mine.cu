@@ -1104,39 +1104,36 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
 
 // Tokens the tcgen05 assignment listed as undecided: float64 squared distances to every
 // pattern (channels in order, as the sequential definition), the lowest index among equal
-// distances.  A 128-thread block takes one token at a time, one thread per pattern (P <= 128).
+// distances.  Each block stages the problem's patterns once in shared memory (rows padded to
+// 129 floats: thread j reads row j without bank conflicts) and takes tokens r = blockIdx.x,
+// r + gridDim.x, ... one at a time, one thread per pattern (P <= 128).  Pattern values become
+// float64 through the integer construction of f32_scaled and one exact multiply, so the float
+// conversion unit stays out of the inner loop.
+constexpr int kFixLd = kD + 1;
 __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
                                                          const int32_t* __restrict__ amb,
                                                          const int32_t* __restrict__ amb_cnt,
                                                          int32_t* __restrict__ assign) {
-  const int prob = blockIdx.y, j = threadIdx.x;
-  __shared__ float xr[kD];
+  extern __shared__ float Ms[];  // [P][kFixLd]
+  __shared__ double xr[kD];
   __shared__ double dist[128];
+  const int prob = blockIdx.y, j = threadIdx.x;
   const int count = amb_cnt[prob];
+  if ((int)blockIdx.x >= count) return;  // uniform across the block
   const float* Mp = M + (size_t)prob * P * kD;
+  for (int i = threadIdx.x; i < P * kD; i += blockDim.x) Ms[(i / kD) * kFixLd + i % kD] = __ldg(Mp + i);
+  const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + (size_t)(j < P ? j : 0) * kFixLd);
   for (int r = blockIdx.x; r < count; r += gridDim.x) {
     const int64_t i = amb[(size_t)prob * s.n + r];
-    xr[j] = s.at(prob, i, j);
+    xr[j] = (double)s.at(prob, i, j);
     __syncthreads();
     double d = 0.0;
     if (j < P) {
-      // the pattern row arrives 32 channels (eight 16-byte loads) at a time; the sum runs over
-      // the channels in order
-      const float4* m4 = reinterpret_cast<const float4*>(Mp + (size_t)j * kD);
-#pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
-        float4 mv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mv[u] = __ldg(m4 + c0 / 4 + u);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float m[4] = {mv[u].x, mv[u].y, mv[u].z, mv[u].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const double t = __dsub_rn((double)xr[c0 + 4 * u + e], (double)m[e]);
-            d = __dadd_rn(d, __dmul_rn(t, t));
-          }
-        }
+#pragma unroll 8
+      for (int c = 0; c < kD; ++c) {
+        const double m = __dmul_rn(f32_scaled(mrow[c]), 0x1p896);
+        const double t = __dsub_rn(xr[c], m);
+        d = __dadd_rn(d, __dmul_rn(t, t));
       }
     }
     dist[j] = d;
@@ -1293,6 +1290,10 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
       return e;
     if ((e = make_x_map(a, &xmap, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
+  const size_t fix_smem = (size_t)a.P * kFixLd * sizeof(float);
+  if (use_tc && (e = cudaFuncSetAttribute(mine_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)fix_smem)) != cudaSuccess)
+    return e;
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, (a.P <= 64 ? 2 : 1) * sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
@@ -1300,7 +1301,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     if (use_tc) {
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
           xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P));
-      mine_fixup_kernel<<<dim3((unsigned)std::max(1, std::min(256, sms * 16 / NP)), NP), 128, 0, st>>>(
+      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 8 * sms / NP), NP), 128, fix_smem, st>>>(
           s, a.P, a.patterns, w.amb, w.amb_cnt, w.assign);
     } else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
