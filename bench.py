@@ -282,6 +282,8 @@ def main():
     tok_stride, set_stride = w.Hkv * D, n * w.Hkv * D
     stream = torch.cuda.current_stream()
 
+    tc_path = w.dtype == kvq.KVQ_BF16 and not w.transform and w.P <= 128
+
     def step(kx, vx, qx, ev=None):
         if ev: ev[0].record()
         kvq.kvq_mine_patterns(kx, w.dtype, n, 1, w.Hkv, tok_stride, D, set_stride, w.P, w.iters, w.transform,
@@ -389,7 +391,10 @@ def main():
             "e2e": {"value": e2e_value, "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
                     "d2h_bytes_per_step": int(out_h.numel() * 4)},
-            "gpu_launches": args.steps * (2 * (1 + 3 * w.iters + (15 if w.transform else 0)) + 3 + 1),
+            # per mining call: init, then per iteration assignment (+ the float64 fix-up after the
+            # tcgen05 assignment: bf16 input, P <= 128), cluster sums and update; the pre-transform
+            # fit adds 15; append: prep, pages, tail; decode: one kernel
+            "gpu_launches": args.steps * (2 * (1 + (4 if tc_path else 3) * w.iters + (15 if w.transform else 0)) + 3 + 1),
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -1121,7 +1121,24 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
   const int count = amb_cnt[prob];
   if ((int)blockIdx.x >= count) return;  // uniform across the block
   const float* Mp = M + (size_t)prob * P * kD;
-  for (int i = threadIdx.x; i < P * kD; i += blockDim.x) Ms[(i / kD) * kFixLd + i % kD] = __ldg(Mp + i);
+  // 16-byte loads, eight in flight per thread, stored into the padded rows
+  const float4* M4 = reinterpret_cast<const float4*>(Mp);
+  for (int i0 = threadIdx.x; i0 < P * (kD / 4); i0 += 8 * blockDim.x) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = i < P * (kD / 4) ? __ldg(M4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < P * (kD / 4)) {
+        float* dst = Ms + (i / (kD / 4)) * kFixLd + 4 * (i % (kD / 4));
+        dst[0] = v[u].x; dst[1] = v[u].y; dst[2] = v[u].z; dst[3] = v[u].w;
+      }
+    }
+  }
   const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + (size_t)(j < P ? j : 0) * kFixLd);
   for (int r = blockIdx.x; r < count; r += gridDim.x) {
     const int64_t i = amb[(size_t)prob * s.n + r];
