@@ -241,6 +241,7 @@ __device__ __forceinline__ void lb_pass(const float* y, const int32_t* pc, const
   for (int u = 0; u < NPROBE; ++u) py[u] = y[pc[u]];
   float blb = INFINITY;
   int bj = j0;
+#pragma unroll 2
   for (int j = j0; j < j1; ++j) {
     const float4* m4 = reinterpret_cast<const float4*>(pvt + (size_t)j * NPROBE);
     float mx = -INFINITY, mn = INFINITY;

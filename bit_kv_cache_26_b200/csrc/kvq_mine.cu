@@ -1106,7 +1106,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
 // pattern (channels in order, as the sequential definition), the lowest index among equal
 // distances.  Each block stages the problem's patterns once in shared memory (rows padded to
 // 129 floats: thread j reads row j without bank conflicts) and takes tokens r = blockIdx.x,
-// r + gridDim.x, ... one at a time, one thread per pattern (P <= 128).  Pattern values become
+// r + gridDim.x, ... one at a time, one thread per pattern (P <= 128); padding threads carry
+// an infinite distance into the (distance, index) minimum.  Pattern values become
 // float64 through the integer construction of f32_scaled and one exact multiply, so the float
 // conversion unit stays out of the inner loop.
 constexpr int kFixLd = kD + 1;
@@ -1116,7 +1117,6 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
                                                          int32_t* __restrict__ assign) {
   extern __shared__ float Ms[];  // [P][kFixLd]
   __shared__ double xr[kD];
-  __shared__ double dist[128];
   const int prob = blockIdx.y, j = threadIdx.x;
   const int count = amb_cnt[prob];
   if ((int)blockIdx.x >= count) return;  // uniform across the block
@@ -1140,12 +1140,21 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
     }
   }
   const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + (size_t)(j < P ? j : 0) * kFixLd);
-  for (int r = blockIdx.x; r < count; r += gridDim.x) {
-    const int64_t i = amb[(size_t)prob * s.n + r];
-    xr[j] = (double)s.at(prob, i, j);
+  __shared__ double wbest[4];
+  __shared__ int wbj[4];
+  // the next token's index and row are fetched while the current one is scored
+  int r = blockIdx.x;
+  int64_t i = amb[(size_t)prob * s.n + r];
+  float xv = s.at(prob, i, j);
+  while (r < count) {
+    const int rn = r + gridDim.x;
+    const int64_t in = rn < count ? amb[(size_t)prob * s.n + rn] : 0;
+    xr[j] = (double)xv;
     __syncthreads();
-    double d = 0.0;
+    const float xn = rn < count ? s.at(prob, in, j) : 0.f;
+    double d = INFINITY;
     if (j < P) {
+      d = 0.0;
 #pragma unroll 8
       for (int c = 0; c < kD; ++c) {
         const double m = __dmul_rn(f32_scaled(mrow[c]), 0x1p896);
@@ -1153,16 +1162,27 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
         d = __dadd_rn(d, __dmul_rn(t, t));
       }
     }
-    dist[j] = d;
+    // (distance, index) minimum: within each warp by shuffles, then across the 4 warps
+    int bj = j;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const double od = __shfl_xor_sync(kFull, d, off);
+      const int oj = __shfl_xor_sync(kFull, bj, off);
+      if (od < d || (od == d && oj < bj)) { d = od; bj = oj; }
+    }
+    if ((threadIdx.x & 31) == 0) { wbest[threadIdx.x >> 5] = d; wbj[threadIdx.x >> 5] = bj; }
     __syncthreads();
-    if (j == 0) {
-      double bd = dist[0];
-      int bj = 0;
-      for (int q = 1; q < P; ++q)
-        if (dist[q] < bd) { bd = dist[q]; bj = q; }
-      assign[(size_t)prob * s.n + i] = bj;
+    if (threadIdx.x == 0) {
+      double bd = wbest[0];
+      int bw = wbj[0];
+      for (int w = 1; w < 4; ++w)
+        if (wbest[w] < bd || (wbest[w] == bd && wbj[w] < bw)) { bd = wbest[w]; bw = wbj[w]; }
+      assign[(size_t)prob * s.n + i] = bw;
     }
     __syncthreads();
+    r = rn;
+    i = in;
+    xv = xn;
   }
 }
 
