@@ -1105,10 +1105,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
 // Tokens the tcgen05 assignment listed as undecided: float64 squared distances to every
 // pattern (channels in order, as the sequential definition), the lowest index among equal
 // distances.  Each block stages the problem's patterns once in shared memory (rows padded to
-// 129 floats: thread j reads row j without bank conflicts) and takes tokens r = blockIdx.x,
-// r + gridDim.x, ... one at a time, one thread per pattern (P <= 128); padding threads carry
-// an infinite distance into the (distance, index) minimum.  Pattern values become
-// float64 through the integer construction of f32_scaled and one exact multiply, so the float
+// 129 floats: thread j reads row j without bank conflicts).  With P <= 64 the block scores two
+// tokens at a time (threads 64 h .. 64 h + 63 take token slot h), otherwise one, one thread
+// per pattern; the tokens of slot h are r = 2 blockIdx.x + h, r + 2 gridDim.x, ... and the
+// next one's index and row are fetched while one is scored.  Padding threads carry an
+// infinite distance into the (distance, index) minimum.  Pattern values become float64
+// through the integer construction of f32_scaled and one exact multiply, so the float
 // conversion unit stays out of the inner loop.
 constexpr int kFixLd = kD + 1;
 __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
@@ -1116,10 +1118,15 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
                                                          const int32_t* __restrict__ amb_cnt,
                                                          int32_t* __restrict__ assign) {
   extern __shared__ float Ms[];  // [P][kFixLd]
-  __shared__ double xr[kD];
-  const int prob = blockIdx.y, j = threadIdx.x;
+  __shared__ double xr[2][kD];
+  __shared__ double wbest[4];
+  __shared__ int wbj[4];
+  const int prob = blockIdx.y;
+  const int slots = P <= 64 ? 2 : 1, tpr = 128 / slots;  // token slots, threads per token
+  const int h = threadIdx.x / tpr, j = threadIdx.x % tpr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int count = amb_cnt[prob];
-  if ((int)blockIdx.x >= count) return;  // uniform across the block
+  if ((int)blockIdx.x * slots >= count) return;  // uniform across the block
   const float* Mp = M + (size_t)prob * P * kD;
   // 16-byte loads, eight in flight per thread, stored into the padded rows
   const float4* M4 = reinterpret_cast<const float4*>(Mp);
@@ -1140,29 +1147,37 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
     }
   }
   const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + (size_t)(j < P ? j : 0) * kFixLd);
-  __shared__ double wbest[4];
-  __shared__ int wbj[4];
-  // the next token's index and row are fetched while the current one is scored
-  int r = blockIdx.x;
-  int64_t i = amb[(size_t)prob * s.n + r];
-  float xv = s.at(prob, i, j);
-  while (r < count) {
-    const int rn = r + gridDim.x;
-    const int64_t in = rn < count ? amb[(size_t)prob * s.n + rn] : 0;
-    xr[j] = (double)xv;
+  const int stride = slots * gridDim.x;
+  // the x row of a token: its tpr threads load kD / tpr channels each
+  auto load_row = [&](int r, float (&xv)[2]) {
+    const int64_t i = r < count ? amb[(size_t)prob * s.n + r] : 0;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) xv[u] = (r < count && u * tpr + j < kD) ? s.at(prob, i, u * tpr + j) : 0.f;
+    return i;
+  };
+  int r = blockIdx.x * slots + h;
+  float xv[2];
+  int64_t i = load_row(r, xv);
+  for (int rb = blockIdx.x * slots; rb < count; rb += stride) {
+    const int rn = r + stride;
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (u * tpr + j < kD) xr[h][u * tpr + j] = (double)xv[u];
     __syncthreads();
-    const float xn = rn < count ? s.at(prob, in, j) : 0.f;
+    float xn[2];
+    const int64_t in = load_row(rn, xn);
     double d = INFINITY;
-    if (j < P) {
+    if (j < P && r < count) {
       d = 0.0;
 #pragma unroll 8
       for (int c = 0; c < kD; ++c) {
         const double m = __dmul_rn(f32_scaled(mrow[c]), 0x1p896);
-        const double t = __dsub_rn(xr[c], m);
+        const double t = __dsub_rn(xr[h][c], m);
         d = __dadd_rn(d, __dmul_rn(t, t));
       }
     }
-    // (distance, index) minimum: within each warp by shuffles, then across the 4 warps
+    // (distance, index) minimum per token: within each warp by shuffles, then across the
+    // token's warps
     int bj = j;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -1170,19 +1185,21 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
       const int oj = __shfl_xor_sync(kFull, bj, off);
       if (od < d || (od == d && oj < bj)) { d = od; bj = oj; }
     }
-    if ((threadIdx.x & 31) == 0) { wbest[threadIdx.x >> 5] = d; wbj[threadIdx.x >> 5] = bj; }
+    if (lane == 0) { wbest[warp] = d; wbj[warp] = bj; }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      double bd = wbest[0];
-      int bw = wbj[0];
-      for (int w = 1; w < 4; ++w)
+    if (j == 0 && r < count) {
+      const int w0 = h * (tpr / 32);
+      double bd = wbest[w0];
+      int bw = wbj[w0];
+      for (int w = w0 + 1; w < w0 + tpr / 32; ++w)
         if (wbest[w] < bd || (wbest[w] == bd && wbj[w] < bw)) { bd = wbest[w]; bw = wbj[w]; }
       assign[(size_t)prob * s.n + i] = bw;
     }
     __syncthreads();
     r = rn;
     i = in;
-    xv = xn;
+    xv[0] = xn[0];
+    xv[1] = xn[1];
   }
 }
 
