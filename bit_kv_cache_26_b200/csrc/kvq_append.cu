@@ -150,6 +150,27 @@ __device__ __forceinline__ void range32(const float* __restrict__ y, const float
   }
 }
 
+// Exact partial max / min of y - m over the 64 channels [c0, c0 + 64), its 16-byte chunks
+// taken from chunk `rot` on (wrapping), so that two threads reading the two halves of one
+// staged row (rot 0 and 1) hit different shared-memory banks.
+__device__ __forceinline__ void range64(const float* __restrict__ y, const float* __restrict__ m, int c0, int rot,
+                                        float& mx, float& mn) {
+  const float4* y4 = reinterpret_cast<const float4*>(y + c0);
+  const float4* m4 = reinterpret_cast<const float4*>(m + c0);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int c = (k + rot) & 15;
+    const float4 a = y4[c], bq = __ldg(m4 + c);
+    float r0, r1, r2, r3;
+    sub2(a.x, a.y, bq.x, bq.y, r0, r1);
+    sub2(a.z, a.w, bq.z, bq.w, r2, r3);
+    mx = max3(mx, r0, r1);
+    mn = min3(mn, r0, r1);
+    mx = max3(mx, r2, r3);
+    mn = min3(mn, r2, r3);
+  }
+}
+
 __device__ __forceinline__ unsigned long long dkey(float d, int j) {
   return ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j;
 }
@@ -379,6 +400,12 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const int r = kind * kG + lane;
     if (kind == 0) lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
     else if (c.seal) lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    if (kind == 0 || c.seal) {
+      // the half's best pattern is the likely seed: its row into L1 ahead of the exact range
+      const float* mrow = (kind ? c.MK : c.MV) + (size_t)min(max(hj[half][r], 0), P - 1) * kD;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) asm volatile("prefetch.global.L1 [%0];" ::"l"(mrow + 32 * u));
+    }
   }
   __syncthreads();
 
@@ -393,8 +420,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       s = hlb[1][r] < hlb[0][r] ? hj[1][r] : hj[0][r];
       s = min(max(s, 0), P - 1);
       const float* m = (r < kG ? c.MV : c.MK) + (size_t)s * kD;
-      range32(vec[r], m, 64 * hh, mx, mn);
-      range32(vec[r], m, 64 * hh + 32, mx, mn);
+      range64(vec[r], m, 64 * hh, hh, mx, mn);
     }
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
     mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
