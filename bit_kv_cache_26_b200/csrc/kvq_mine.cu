@@ -629,9 +629,13 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
   constexpr int CW = 32 * E, RB = CW * ES;  // channels and bytes of a staged row
   constexpr int kStages = accum_stages<CPW, RB, ES>();
   constexpr int kStageBytes = kAccT * RB;
+  constexpr int kOff = kAccWarps * CPW + 1;  // cluster offsets of a stage's member list
   extern __shared__ __align__(16) uint8_t smraw[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smraw + (size_t)kStages * kStageBytes);
   uint64_t* empty = full + kStages;
+  int32_t* offs = reinterpret_cast<int32_t*>(empty + kStages);  // [kStages][kOff]
+  int32_t* lists = offs + kStages * kOff;                        // [kStages][kAccT] rows by cluster
+  int32_t* counts = lists + kStages * kAccT;                     // [kOff] producer scratch
   const int slice = blockIdx.y, prob = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
@@ -658,6 +662,40 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
       if (k >= kStages) ok = mb_wait(&empty[st], (uint32_t)(((k / kStages) - 1) & 1));
       if (!__all_sync(kFull, ok)) break;  // consumers time out on the full barrier in turn
       const int tb = (int)((k0 + k) * kAccT);
+      // the tile's rows grouped by cluster (counting sort): offs[st][j] .. offs[st][j + 1] of
+      // lists[st] are the rows of cluster j
+      int aj[kAccT / 32], pos[kAccT / 32];
+#pragma unroll
+      for (int q = 0; q < kAccT / 32; ++q) {
+        const int64_t i = (int64_t)tb + 32 * q + lane;
+        aj[q] = i < s.n ? __ldg(a + i) : -1;
+      }
+      for (int i = lane; i < P; i += 32) counts[i] = 0;
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < kAccT / 32; ++q) pos[q] = aj[q] >= 0 ? atomicAdd(&counts[aj[q]], 1) : -1;
+      __syncwarp();
+      {
+        // exclusive scan: lane l owns clusters [l * per, (l + 1) * per)
+        const int per = (P + 31) / 32, c0 = lane * per;
+        int run = 0;
+        for (int c = c0; c < min(P, c0 + per); ++c) run += counts[c];
+        int incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(kFull, incl, off);
+          if (lane >= off) incl += v;
+        }
+        int base = incl - run;
+        int32_t* o = offs + st * kOff;
+        for (int c = c0; c < min(P, c0 + per); ++c) { o[c] = base; base += counts[c]; }
+        if (lane == 31) o[P] = incl;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < kAccT / 32; ++q)
+        if (aj[q] >= 0) lists[st * kAccT + offs[st * kOff + aj[q]] + pos[q]] = 32 * q + lane;
+      __syncwarp();
       if (lane == 0) {
         // one box of 128 tokens x CW channels lands row-major; rows past the end read as zeros
         uint8_t* dst = smraw + (size_t)st * kStageBytes;
@@ -680,64 +718,49 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[c][e] = 0.0;
   }
-  auto load_aj = [&](int k, int (&aj)[kAccT / 32]) {
-    const int64_t tb = (k0 + k) * kAccT;
-#pragma unroll
-    for (int q = 0; q < kAccT / 32; ++q) {
-      const int64_t i = tb + 32 * q + lane;
-      aj[q] = i < s.n ? __ldg(a + i) : -1;
-    }
-  };
-  int aj[kAccT / 32], ajn[kAccT / 32];
-  load_aj(0, aj);
   for (int k = 0; k < nt; ++k) {
     const int st = k % kStages;
-    if (k + 1 < nt) load_aj(k + 1, ajn);
     const bool ok = mb_wait(&full[st], (uint32_t)((k / kStages) & 1));
     if (!__all_sync(kFull, ok)) break;
     const uint8_t* stg = smraw + (size_t)st * kStageBytes;
+    const int32_t* o = offs + st * kOff;
+    const int32_t* lst = lists + st * kAccT;
 #pragma unroll
     for (int c = 0; c < CPW; ++c) {
       const int j = warp + kAccWarps * c;
       if (j >= P) break;
-#pragma unroll
-      for (int q = 0; q < kAccT / 32; ++q) {
-        uint32_t m = __ballot_sync(0xffffffffu, aj[q] == j);
-        members[c] += __popc(m);
-        while (m) {
-          const int t = 32 * q + __ffs(m) - 1;
-          m &= m - 1;
-          const uint8_t* row = stg + t * RB + lane * (E * ES);
-          double v[E];
-          if constexpr (ES == 4) {
-            if constexpr (E == 4) {
-              const uint4 f = *reinterpret_cast<const uint4*>(row);
-              v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y); v[2] = f32_scaled(f.z); v[3] = f32_scaled(f.w);
-            } else if constexpr (E == 2) {
-              const uint2 f = *reinterpret_cast<const uint2*>(row);
-              v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y);
-            } else {
-              v[0] = f32_scaled(*reinterpret_cast<const uint32_t*>(row));
-            }
+      const int x0 = o[j], x1 = o[j + 1];
+      members[c] += (uint32_t)(x1 - x0);
+      for (int x = x0; x < x1; ++x) {
+        const int t = lst[x];
+        const uint8_t* row = stg + t * RB + lane * (E * ES);
+        double v[E];
+        if constexpr (ES == 4) {
+          if constexpr (E == 4) {
+            const uint4 f = *reinterpret_cast<const uint4*>(row);
+            v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y); v[2] = f32_scaled(f.z); v[3] = f32_scaled(f.w);
+          } else if constexpr (E == 2) {
+            const uint2 f = *reinterpret_cast<const uint2*>(row);
+            v[0] = f32_scaled(f.x); v[1] = f32_scaled(f.y);
           } else {
-            uint32_t b[(E + 1) / 2];
-            if constexpr (E == 4) { const uint2 u = *reinterpret_cast<const uint2*>(row); b[0] = u.x; b[1] = u.y; }
-            else if constexpr (E == 2) b[0] = *reinterpret_cast<const uint32_t*>(row);
-            else b[0] = *reinterpret_cast<const uint16_t*>(row);
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-              v[e] = f16 ? ((e & 1) ? f16hi_scaled(b[e >> 1]) : f16lo_scaled(b[e >> 1]))
-                         : ((e & 1) ? bf16hi_scaled(b[e >> 1]) : bf16lo_scaled(b[e >> 1]));
+            v[0] = f32_scaled(*reinterpret_cast<const uint32_t*>(row));
           }
+        } else {
+          uint32_t b[(E + 1) / 2];
+          if constexpr (E == 4) { const uint2 u = *reinterpret_cast<const uint2*>(row); b[0] = u.x; b[1] = u.y; }
+          else if constexpr (E == 2) b[0] = *reinterpret_cast<const uint32_t*>(row);
+          else b[0] = *reinterpret_cast<const uint16_t*>(row);
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[c][e] += v[e];
+          for (int e = 0; e < E; ++e)
+            v[e] = f16 ? ((e & 1) ? f16hi_scaled(b[e >> 1]) : f16lo_scaled(b[e >> 1]))
+                       : ((e & 1) ? bf16hi_scaled(b[e >> 1]) : bf16lo_scaled(b[e >> 1]));
         }
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[c][e] += v[e];
       }
     }
     __syncwarp();
     if (lane == 0) mb_arrive(&empty[st]);
-#pragma unroll
-    for (int q = 0; q < kAccT / 32; ++q) aj[q] = ajn[q];
   }
 
   double* gs = sums + (size_t)prob * P * kD + slice * CW + lane * E;
@@ -755,7 +778,9 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
 
 template <int CPW, int E, int ES>
 constexpr size_t accum_smem() {
-  return (size_t)accum_stages<CPW, 32 * E * ES, ES>() * (kAccT * 32 * E * ES) + 2 * 4 * sizeof(uint64_t);
+  constexpr int st = accum_stages<CPW, 32 * E * ES, ES>();
+  return (size_t)st * (kAccT * 32 * E * ES) + 2 * st * sizeof(uint64_t) +
+         ((size_t)st * (kAccWarps * CPW + 1) + (size_t)st * kAccT + kAccWarps * CPW + 1) * sizeof(int32_t);
 }
 
 template <int CPW, int E, int ES>
