@@ -532,16 +532,18 @@ size_t mine_mma_smem(int P, int KIND) {
 }
 
 // Per-cluster float64 sums and sizes in one streaming pass.  A CTA walks a contiguous run
-// of 128-token tiles of one problem (and one channel slice).  One producer warp copies the
-// tiles' rows into a ring of shared-memory stages with cp.async.bulk (one 16-byte-aligned row
-// per copy, completion counted in bytes on the stage's "full" mbarrier); 16 consumer warps
-// each take every tile: warp w owns clusters w, w + 16, w + 32, ..., finds their members with
-// ballots over the tile's assignments (prefetched one tile ahead) and adds their rows into
-// float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1 of the slice),
-// then arrives on the stage's "empty" mbarrier.  A stage is refilled once all 16 warps are
-// done with it, so fast warps run ahead instead of waiting at a block barrier.  Each CTA adds
-// its totals to global memory once at the end.  float64 sums of fp16 / bf16 values are
-// exact, so the order of the additions does not change them.  Every wait is bounded.
+// of 128-token tiles of one problem (and one channel slice).  One producer warp copies each
+// tile with one TMA box (128 tokens x the slice's channels, row-major; completion counted in
+// bytes on the stage's "full" mbarrier) into a ring of shared-memory stages, and before that
+// groups the tile's rows by cluster (a counting sort through shared-memory counters and a
+// warp scan: per stage an offset per cluster and the list of rows).  16 consumer warps each
+// take every tile: warp w owns clusters w, w + 16, w + 32, ..., walks exactly their rows and
+// adds them into float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1
+// of the slice), then arrives on the stage's "empty" mbarrier.  A stage is refilled once all
+// 16 warps are done with it, so fast warps run ahead instead of waiting at a block barrier.
+// Each CTA adds its totals to global memory once at the end.  float64 sums of fp16 / bf16
+// values are exact, so the order of the additions does not change them (fp32 rows: up to
+// rounding).  Every wait is bounded.
 constexpr int kAccWarps = 16;
 constexpr int kAccT = 128;  // tokens per tile
 constexpr uint32_t kAccSpinLimit = 1u << 24;
@@ -820,7 +822,8 @@ cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, i
 //
 // The same certified argmin as mine_assign_mma_kernel, with the distance contraction on
 // the 5th-generation tensor cores, as a warp-specialised pipeline with no block barrier in
-// its loop (one CTA per SM; roles hand stages and accumulators over through mbarriers):
+// its loop (two CTAs per SM for P <= 64, one above; roles hand stages and accumulators over
+// through mbarriers):
 //   * producer warp: per 128-token tile, two TMA loads (a box of 64 channels x 128 tokens
 //     each, 4-D tensor map over channels x heads x tokens x sets, 128-byte swizzle; rows past
 //     the end read as zeros) into a ring of shared-memory stages: the canonical K-major
