@@ -28,6 +28,11 @@ CASES = {
     "no_tail_token_steps": (W["llama3_8b_32k"].with_(B=3, S=64, Hkv=1, Hq=2, P=8), [30, 1, 1, 32]),
     # many sequences, per-sample perturbed centers
     "breadth_small": (W["breadth_256x16k"].with_(B=16, S=100, Hkv=2, Hq=8, P=32), [100]),
+    # more than 64 patterns: the tcgen05 assignment with 7-bit tags, 224 score columns and one
+    # CTA per SM, the cluster sums with 8 clusters per warp, the fix-up with 128 threads a token
+    "gqa4_p100": (W["llama3_8b_32k"].with_(B=2, S=1000, Hkv=2, Hq=8, P=100), [1000]),
+    # the largest pattern count the u8 indices allow: float64 assignment, 16 clusters per warp
+    "p255": (W["llama3_8b_32k"].with_(B=1, S=600, Hkv=1, Hq=4, P=255), [300, 300]),
 }
 
 
