@@ -1130,31 +1130,31 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
 }
 
-// Tokens the tcgen05 assignment listed as undecided: float64 squared distances to every
-// pattern (channels in order, as the sequential definition), the lowest index among equal
-// distances.  Each block stages the problem's patterns once in shared memory (rows padded to
-// 129 floats: thread j reads row j without bank conflicts).  With P <= 64 the block scores two
-// tokens at a time (threads 64 h .. 64 h + 63 take token slot h), otherwise one, one thread
-// per pattern; the tokens of slot h are r = 2 blockIdx.x + h, r + 2 gridDim.x, ... and the
-// next one's index and row are fetched while one is scored.  Padding threads carry an
-// infinite distance into the (distance, index) minimum.  Pattern values become float64
-// through the integer construction of f32_scaled and one exact multiply, so the float
-// conversion unit stays out of the inner loop.
+// Tokens the tcgen05 assignment listed as undecided (P <= 128).  A warp takes one token at a
+// time (tokens r = its global warp index, r + all warps, ...), with no block barrier in the
+// loop.  fp32 scores e_j = |m_j|^2 - 2 x.m_j for every pattern (lane l: patterns l + 32 q,
+// an in-order fp32 FMA chain over the channels) are within E_j = 2^-15 |x| |m_j| +
+// 2^-22 (|x|^2 + |m_j|^2) of the exact values (a 128-term fp32 dot product is off by at most
+// 128 2^-24 |x| |m_j|, plus the roundings of |m_j|^2 and of e), so the float64 argmin can
+// only be a pattern with e_j - E_j <= min_k (e_k + E_k) + delta (delta: the float64
+// rounding allowance), and only those candidates (about two) get the float64 squared distance
+// in channel order, as the sequential definition; the lowest index wins among equal
+// distances.  The patterns are staged once per block in shared memory (rows padded to 129
+// floats: lane l reads row l without bank conflicts); their float64 values come from the
+// integer construction of f32_scaled and one exact multiply.
 constexpr int kFixLd = kD + 1;
-__global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
-                                                         const int32_t* __restrict__ amb,
-                                                         const int32_t* __restrict__ amb_cnt,
-                                                         int32_t* __restrict__ assign) {
+constexpr int kFixWarps = 8;
+__global__ void __launch_bounds__(kFixWarps * 32) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
+                                                                    const int32_t* __restrict__ amb,
+                                                                    const int32_t* __restrict__ amb_cnt,
+                                                                    int32_t* __restrict__ assign) {
   extern __shared__ float Ms[];  // [P][kFixLd]
-  __shared__ double xr[2][kD];
-  __shared__ double wbest[4];
-  __shared__ int wbj[4];
-  const int prob = blockIdx.y;
-  const int slots = P <= 64 ? 2 : 1, tpr = 128 / slots;  // token slots, threads per token
-  const int h = threadIdx.x / tpr, j = threadIdx.x % tpr;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float mn2[128], mnrm[128];
+  __shared__ float xs[kFixWarps][kD];
+  __shared__ double xd[kFixWarps][kD];
+  const int prob = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int count = amb_cnt[prob];
-  if ((int)blockIdx.x * slots >= count) return;  // uniform across the block
+  if ((int)blockIdx.x * kFixWarps >= count) return;  // uniform across the block
   const float* Mp = M + (size_t)prob * P * kD;
   // 16-byte loads, eight in flight per thread, stored into the padded rows
   const float4* M4 = reinterpret_cast<const float4*>(Mp);
@@ -1174,60 +1174,71 @@ __global__ void __launch_bounds__(128) mine_fixup_kernel(Src s, int P, const flo
       }
     }
   }
-  const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + (size_t)(j < P ? j : 0) * kFixLd);
-  const int stride = slots * gridDim.x;
-  // the x row of a token: its tpr threads load kD / tpr channels each
-  auto load_row = [&](int r, float (&xv)[2]) {
-    const int64_t i = r < count ? amb[(size_t)prob * s.n + r] : 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < P; j += blockDim.x) {
+    double acc = 0.0;
+    for (int c = 0; c < kD; ++c) {
+      const double m = Ms[j * kFixLd + c];
+      acc = fma(m, m, acc);
+    }
+    mn2[j] = (float)acc;
+    mnrm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
+  }
+  __syncthreads();
+  for (int r = blockIdx.x * kFixWarps + warp; r < count; r += gridDim.x * kFixWarps) {
+    const int64_t i = amb[(size_t)prob * s.n + r];
+    float xx = 0.f;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) xv[u] = (r < count && u * tpr + j < kD) ? s.at(prob, i, u * tpr + j) : 0.f;
-    return i;
-  };
-  int r = blockIdx.x * slots + h;
-  float xv[2];
-  int64_t i = load_row(r, xv);
-  for (int rb = blockIdx.x * slots; rb < count; rb += stride) {
-    const int rn = r + stride;
+    for (int k = 0; k < 4; ++k) {
+      const float v = s.at(prob, i, lane + 32 * k);
+      xs[warp][lane + 32 * k] = v;
+      xd[warp][lane + 32 * k] = (double)v;
+      xx = fmaf(v, v, xx);
+    }
+    xx = warp_sum(xx) * (1.0f + 1e-5f);
+    const float nx = sqrtf(xx) * (1.0f + 1e-5f);
+    __syncwarp();
+    float e[4], E[4];
+    float U = INFINITY;
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (u * tpr + j < kD) xr[h][u * tpr + j] = (double)xv[u];
-    __syncthreads();
-    float xn[2];
-    const int64_t in = load_row(rn, xn);
-    double d = INFINITY;
-    if (j < P && r < count) {
-      d = 0.0;
+    for (int q = 0; q < 4; ++q) {
+      const int j = lane + 32 * q;
+      e[q] = INFINITY;
+      E[q] = 0.f;
+      if (j < P) {
+        const float* mr = Ms + j * kFixLd;
+        float dot = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < kD; ++c) {
-        const double m = __dmul_rn(f32_scaled(mrow[c]), 0x1p896);
-        const double t = __dsub_rn(xr[h][c], m);
-        d = __dadd_rn(d, __dmul_rn(t, t));
+        for (int c = 0; c < kD; ++c) dot = fmaf(xs[warp][c], mr[c], dot);
+        e[q] = mn2[j] - 2.0f * dot;
+        E[q] = 0x1p-15f * nx * mnrm[j] + 0x1p-22f * (xx + mn2[j]);
+        U = fminf(U, e[q] + E[q]);
       }
     }
-    // (distance, index) minimum per token: within each warp by shuffles, then across the
-    // token's warps
-    int bj = j;
+    U = warp_min(U);
+    double bd = INFINITY;
+    int bj = 1 << 30;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = lane + 32 * q;
+      if (j < P && e[q] - E[q] <= U + 1e-9f * (xx + mn2[j])) {
+        const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + j * kFixLd);
+        double d = 0.0;
+        for (int c = 0; c < kD; ++c) {
+          const double t = __dsub_rn(xd[warp][c], __dmul_rn(f32_scaled(mrow[c]), 0x1p896));
+          d = __dadd_rn(d, __dmul_rn(t, t));
+        }
+        if (d < bd) { bd = d; bj = j; }  // q ascending: the lowest index of this lane wins ties
+      }
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      const double od = __shfl_xor_sync(kFull, d, off);
+      const double od = __shfl_xor_sync(kFull, bd, off);
       const int oj = __shfl_xor_sync(kFull, bj, off);
-      if (od < d || (od == d && oj < bj)) { d = od; bj = oj; }
+      if (od < bd || (od == bd && oj < bj)) { bd = od; bj = oj; }
     }
-    if (lane == 0) { wbest[warp] = d; wbj[warp] = bj; }
-    __syncthreads();
-    if (j == 0 && r < count) {
-      const int w0 = h * (tpr / 32);
-      double bd = wbest[w0];
-      int bw = wbj[w0];
-      for (int w = w0 + 1; w < w0 + tpr / 32; ++w)
-        if (wbest[w] < bd || (wbest[w] == bd && wbj[w] < bw)) { bd = wbest[w]; bw = wbj[w]; }
-      assign[(size_t)prob * s.n + i] = bw;
-    }
-    __syncthreads();
-    r = rn;
-    i = in;
-    xv[0] = xn[0];
-    xv[1] = xn[1];
+    if (lane == 0) assign[(size_t)prob * s.n + i] = bj;
+    __syncwarp();
   }
 }
 
@@ -1383,7 +1394,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     if (use_tc) {
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
           xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P));
-      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 8 * sms / NP), NP), 128, fix_smem, st>>>(
+      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 4 * sms / NP), NP), kFixWarps * 32, fix_smem, st>>>(
           s, a.P, a.patterns, w.amb, w.amb_cnt, w.assign);
     } else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
