@@ -64,7 +64,10 @@ def _load():
             "kvqo_dmm": (ctypes.c_float, [_vp, _vp]),
             "kvqo_assign": (i32, [_vp, _vp, i32]),
             "kvqo_quant_group": (None, [_vp, i64, i64, i32, _vp, _vp, _vp, i64]),
-            "kvqo_encode": (ctypes.c_int, [_vp, _vp, i64, i32, i32, _vp, _vp, _vp, _vp] + [_vp] * 10),
+            "kvqo_encode": (ctypes.c_int, [_vp, _vp, i64, i32, i32, _vp, _vp, _vp, _vp, ctypes.c_float] + [_vp] * 10),
+            "kvqo_normal_upper_quantile": (f64, [f64]),
+            "kvqo_rho_star": (f64, [i32, f64]),
+            "kvqo_range": (ctypes.c_float, [_vp]),
             "kvqo_dequant": (None, [i64, _vp, _vp, _vp, _vp] + [_vp] * 10 + [_vp, _vp]),
             "kvqo_attention": (None, [_vp, i32, _vp, _vp, i64, f64, _vp]),
         }
@@ -95,6 +98,12 @@ def _f64(a):
 def sqdist(x, m) -> float:
     x, m = _f32(x), _f32(m)
     return _load().kvqo_sqdist(_p(x), _p(m))
+
+
+def nearest_euclid(x, M) -> int:
+    """Index of the nearest pattern under the float64 squared distance (lowest index on ties)."""
+    x, M = _f32(x), _f32(M)
+    return int(_load().kvqo_nearest_euclid(_p(x), _p(M), M.shape[0]))
 
 
 def mine(x: np.ndarray, P: int, iters: int = 4):
@@ -218,8 +227,31 @@ class Encoded:
     vrow: np.ndarray   # [N] fp32
 
 
-def encode(K: np.ndarray, V: np.ndarray, bits: int, MK, MV, cK=None, cV=None) -> Encoded:
-    """Encode N tokens of one (sequence, KV head): K, V are [N,128] fp32 (exact input values)."""
+def normal_upper_quantile(a: float) -> float:
+    """z with P(Z > z) = a for a standard normal Z (bisection)."""
+    return float(_load().kvqo_normal_upper_quantile(a))
+
+
+def rho_star(d: int, alpha: float) -> float:
+    """rho*(d, alpha) of PatternKV Eq. 10 (float64, bisection)."""
+    return float(_load().kvqo_rho_star(d, alpha))
+
+
+def v_rho(alpha: float, d: int = D) -> float:
+    """The fp32 threshold the encoder compares with (0 = adaptive threshold off)."""
+    return 0.0 if alpha <= 0 else float(np.float32(rho_star(d, alpha)))
+
+
+def vrange(x) -> float:
+    x = _f32(x)
+    return float(_load().kvqo_range(_p(x)))
+
+
+def encode(K: np.ndarray, V: np.ndarray, bits: int, MK, MV, cK=None, cV=None, v_rho: float = 0.0) -> Encoded:
+    """Encode N tokens of one (sequence, KV head): K, V are [N,128] fp32 (exact input values).
+
+    v_rho > 0 enables the V adaptive threshold (PatternKV Section 3.3): a V vector whose
+    residual range exceeds fl32(v_rho * its own range) is quantized raw, with index 255."""
     K, V, MK, MV = _f32(K), _f32(V), _f32(MK), _f32(MV)
     cK = None if cK is None else _f32(cK)
     cV = None if cV is None else _f32(cV)
@@ -229,7 +261,7 @@ def encode(K: np.ndarray, V: np.ndarray, bits: int, MK, MV, cK=None, cV=None) ->
                 np.zeros((G, D), np.float32), np.zeros(G * GROUP, np.uint8), np.zeros(G * GROUP, np.float32),
                 np.zeros((N, D), np.uint8), np.zeros((N, 4), np.float32), np.zeros((N, 4), np.float32),
                 np.zeros(N, np.uint8), np.zeros(N, np.float32))
-    rc = _load().kvqo_encode(_p(K), _p(V), N, bits, MK.shape[0], _p(MK), _p(MV), _p(cK), _p(cV),
+    rc = _load().kvqo_encode(_p(K), _p(V), N, bits, MK.shape[0], _p(MK), _p(MV), _p(cK), _p(cV), float(v_rho),
                              _p(e.kcode), _p(e.ks), _p(e.kz), _p(e.kidx), _p(e.krow),
                              _p(e.vcode), _p(e.vs), _p(e.vz), _p(e.vidx), _p(e.vrow))
     if rc != 0:

@@ -239,6 +239,52 @@ int32_t kvqo_assign(const float* x, const float* M, int32_t P) {
 }
 
 /* ------------------------------------------------------------------------- */
+/* Flattening-sensitive adaptive threshold for V: [PKV] Section 3.3, Eq. 7-10.*/
+/* A one-sided z-test at level alpha accepts flattening (use of the pattern) */
+/* only when the contraction ratio rho = R_flat / R_raw satisfies            */
+/*   1 - rho^2 >= 2 z_{1-alpha} / sqrt(5 d) * sqrt(1 + rho^4),               */
+/* i.e. rho <= rho*(d, alpha), the root of the equality (Eq. 10).            */
+/* Readings: R_raw = max v - min v of the V vector, R_flat = d_mm(v, M*)     */
+/* (the range of its residual); the test is made in fp32 as                  */
+/*   use the pattern  iff  R_flat <= fl32(rho*_fp32 * R_raw);                */
+/* a rejected vector stores index 255 and is quantized raw (pattern 0).      */
+/* ------------------------------------------------------------------------- */
+
+/* Standard normal upper quantile z with P(Z > z) = a, by bisection on erfc. */
+double kvqo_normal_upper_quantile(double a) {
+  double lo = -40.0, hi = 40.0;
+  for (int it = 0; it < 200; ++it) {
+    double mid = 0.5 * (lo + hi);
+    double tail = 0.5 * erfc(mid / sqrt(2.0)); /* P(Z > mid), decreasing in mid */
+    if (tail > a) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+/* rho*(d, alpha): the root in (0, 1) of (1 - rho^2) - 2 z / sqrt(5 d) sqrt(1 + rho^4), by bisection. */
+double kvqo_rho_star(int32_t d, double alpha) {
+  const double z = kvqo_normal_upper_quantile(alpha);
+  const double k = 2.0 * z / sqrt(5.0 * (double)d);
+  double lo = 0.0, hi = 1.0; /* f(0) = 1 - k > 0 for the d, alpha of interest; f(1) < 0 */
+  for (int it = 0; it < 200; ++it) {
+    double mid = 0.5 * (lo + hi);
+    double f = (1.0 - mid * mid) - k * sqrt(1.0 + mid * mid * mid * mid);
+    if (f > 0.0) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+/* fp32 range max - min of a 128-vector. */
+float kvqo_range(const float* x) {
+  float mx = x[0], mn = x[0];
+  for (int d = 1; d < D; ++d) {
+    if (x[d] > mx) mx = x[d];
+    if (x[d] < mn) mn = x[d];
+  }
+  return mx - mn;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Asymmetric n-bit group quantizer: [PKV] Section 2.1, Eq. 1.               */
 /*   Q = round((X - z) / s),  s = (max X - min X) / (2^n - 1),  z = min X    */
 /* fp32, in this order: mn, mx exact; s = fl32(fl32(mx - mn) / (2^n - 1));   */
@@ -285,6 +331,8 @@ void kvqo_quant_group(const float* R, int64_t n, int64_t stride, int32_t bits, f
 /*   kcode[G][32][128], ks/kz[G][128], kidx[G][32], krow[G][32]              */
 /*   vcode[N][128], vs/vz[N][4], vidx[N], vrow[N]                            */
 /* with G = N / 32.  cK/cV NULL means no pre-transform (rows are then 1).    */
+/* v_rho > 0 enables the V adaptive threshold (Section 3.3) with that fp32   */
+/* rho*; v_rho <= 0 always uses the nearest pattern.                         */
 /* ------------------------------------------------------------------------- */
 
 static void prep_row(const float* x, const float* c, float* y, float* r) {
@@ -297,8 +345,9 @@ static void prep_row(const float* x, const float* c, float* y, float* r) {
 }
 
 int kvqo_encode(const float* K, const float* V, int64_t N, int32_t bits, int32_t P, const float* MK,
-                const float* MV, const float* cK, const float* cV, uint8_t* kcode, float* ks, float* kz,
-                uint8_t* kidx, float* krow, uint8_t* vcode, float* vs, float* vz, uint8_t* vidx, float* vrow) {
+                const float* MV, const float* cK, const float* cV, float v_rho, uint8_t* kcode, float* ks,
+                float* kz, uint8_t* kidx, float* krow, uint8_t* vcode, float* vs, float* vz, uint8_t* vidx,
+                float* vrow) {
   if (bits != 2 && bits != 4) return -1;
   if (P < 1 || P > 255) return -1;
   /* V: every token */
@@ -307,8 +356,15 @@ int kvqo_encode(const float* K, const float* V, int64_t N, int32_t bits, int32_t
     float y[D], R[D];
     prep_row(V + (size_t)t * D, cV, y, &vrow[t]);
     int32_t j = kvqo_assign(y, MV, P);
-    vidx[t] = (uint8_t)j;
-    for (int d = 0; d < D; ++d) R[d] = y[d] - MV[(size_t)j * D + d];
+    int use = 1;
+    if (v_rho > 0.0f) {
+      float r_flat = kvqo_dmm(y, MV + (size_t)j * D);
+      float r_raw = kvqo_range(y);
+      float limit = v_rho * r_raw;
+      use = r_flat <= limit;
+    }
+    vidx[t] = use ? (uint8_t)j : (uint8_t)255;
+    for (int d = 0; d < D; ++d) R[d] = use ? y[d] - MV[(size_t)j * D + d] : y[d];
     int32_t q[D];
     for (int g = 0; g < 4; ++g) kvqo_quant_group(R + 32 * g, 32, 1, bits, &vs[t * 4 + g], &vz[t * 4 + g], q + 32 * g, 1);
     for (int d = 0; d < D; ++d) vcode[(size_t)t * D + d] = (uint8_t)q[d];
@@ -364,9 +420,10 @@ void kvqo_dequant(int64_t N, const float* MK, const float* MV, const float* cK, 
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < N; ++t) {
     double* o = Vhat + (size_t)t * D;
-    const float* m = MV + (size_t)vidx[t] * D;
+    const float* m = vidx[t] == 255 ? NULL : MV + (size_t)vidx[t] * D; /* 255: quantized raw */
     for (int d = 0; d < D; ++d)
-      o[d] = (double)vs[t * 4 + d / 32] * (double)vcode[(size_t)t * D + d] + (double)vz[t * 4 + d / 32] + (double)m[d];
+      o[d] = (double)vs[t * 4 + d / 32] * (double)vcode[(size_t)t * D + d] + (double)vz[t * 4 + d / 32] +
+             (m ? (double)m[d] : 0.0);
     if (cV) unrotate(o, cV, vrow[t]);
   }
 }

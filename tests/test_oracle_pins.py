@@ -472,3 +472,87 @@ def test_pack_round_trip(bits, transform):
     back = oracle.parse_subblock(buf, bits, transform)
     assert np.array_equal(back["vcode"][:11], e.vcode[64:75]) and not back["vcode"][11:].any()
     assert not defined[:oracle.code_bytes(bits)].any()
+
+
+# ---------------------------------------------------------------- V adaptive threshold (Eq. 7-10)
+
+def test_rho_star_worked_values_and_closed_form(golden):
+    import scipy.stats
+    for case in golden("rho_star_eq10.json")["cases"]:
+        r = oracle.rho_star(case["d"], case["alpha"])
+        assert abs(r - case["rho_star"]) < 6e-6, case
+    for d in (64, 96, 128, 256):
+        for a in (0.1, 0.05, 0.01):
+            z = scipy.stats.norm.isf(a)                       # library quantile
+            assert abs(oracle.normal_upper_quantile(a) - z) < 1e-12
+            k = 2 * z / np.sqrt(5 * d)                        # closed-form root of the quadratic in rho^2
+            A = 1 - k * k
+            u = (1 - np.sqrt(1 - A * A)) / A
+            r = oracle.rho_star(d, a)
+            assert abs(r - np.sqrt(u)) < 1e-12
+            assert abs((1 - r * r) - k * np.sqrt(1 + r ** 4)) < 1e-12   # Eq. 10 holds with equality
+            assert r > oracle.rho_star(d, a / 2)              # a smaller alpha asks for more contraction
+
+
+def _vec_with_ranges(raw, flat):
+    """A V vector with range `raw` (channels 0 and 1) and a pattern whose residual range is `flat`
+    (the residual is 0 except channel 2 = flat); small dyadic values, so every fp32 step is exact."""
+    v = np.zeros(D, np.float32)
+    v[0], v[1] = raw / 2, -raw / 2
+    m = v.copy()
+    m[2] -= flat
+    return v, m
+
+
+def test_v_threshold_decision_and_raw_fallback():
+    rho = oracle.v_rho(0.05)
+    assert rho == np.float32(0.91155338)
+    raw = np.float32(8.0)
+    limit = float(np.float32(rho) * raw)                      # fl32(rho* x R_raw)
+    on_edge = np.float32(limit)
+    above = np.nextafter(on_edge, np.float32(np.inf))
+    K = np.zeros((32, D), np.float32)
+    MK = np.zeros((1, D), np.float32)
+    for flat, want_use in ((np.float32(1.0), True), (on_edge, True), (above, False), (np.float32(7.99), False)):
+        v, m = _vec_with_ranges(raw, flat)
+        assert oracle.dmm(v, m) == flat and oracle.vrange(v) == raw
+        V = np.tile(v, (32, 1))
+        e = oracle.encode(K, V, 2, MK, m[None], v_rho=rho)
+        assert (e.vidx == (0 if want_use else 255)).all(), (flat, want_use)
+        # with the threshold off the pattern is always used
+        assert (oracle.encode(K, V, 2, MK, m[None]).vidx == 0).all()
+        if not want_use:
+            # quantized raw: the codes and scales of plain Eq. 1 on v itself, and dequant adds no pattern
+            for g in range(4):
+                s, z, q = oracle.quant_group(v[32 * g:32 * g + 32], 2)
+                assert e.vs[0, g] == s and e.vz[0, g] == z and np.array_equal(e.vcode[0, 32 * g:32 * g + 32], q)
+            _, Vh = oracle.dequant(e, MK, m[None])
+            assert np.abs(Vh[0] - v).max() <= e.vs[0].max() / 2 * (1 + 2 ** -20)
+
+
+def test_v_threshold_matches_eq10_on_clustered_data():
+    # Every accepted V vector has rho = R_flat / R_raw <= rho* (up to the fp32 product), every
+    # rejected one has rho > rho*; on data with a planted fraction of unclustered vectors the
+    # rejections are about that fraction.
+    w = synth.WORKLOADS["llama3_8b_32k"].with_(B=1, S=512, Hkv=1, Hq=4, P=16, ncv=4)
+    k, v = synth.gen_kv(w)
+    K = synth.to_float(k, w.dtype)[0, :, 0]
+    V = synth.to_float(v, w.dtype)[0, :, 0]
+    MV, _, _ = oracle.mine_set(V, 16)
+    MK, _, _ = oracle.mine_set(K, 16)
+    V2 = V.copy()
+    V2[::4] = (rng.standard_normal((128, D)) * 3).astype(np.float32)  # a quarter far from every pattern
+    rho = oracle.v_rho(0.05)
+    e = oracle.encode(K, V2, 2, MK, MV, v_rho=rho)
+    rs = oracle.rho_star(128, 0.05)
+    for t in range(len(V2)):
+        j = oracle.assign(V2[t], MV)
+        ratio = oracle.dmm(V2[t], MV[j]) / oracle.vrange(V2[t])
+        if e.vidx[t] == 255:
+            assert ratio > rs * (1 - 1e-6)
+        else:
+            assert e.vidx[t] == j and ratio <= rs * (1 + 1e-6)
+    planted = np.zeros(len(V2), bool)
+    planted[::4] = True
+    assert (e.vidx[planted] == 255).mean() > 0.9       # far from every pattern: flattening rejected
+    assert (e.vidx[~planted] == 255).mean() < 0.1      # near their pattern: flattening kept
