@@ -1,13 +1,15 @@
 """Benchmark of the hot path on B200: pattern mining + quantize-append + decode attention.
 
-One step = one pass of the whole path over one batch of synthetic input (Llama-3-8B-shaped
-layer by default: 8 sequences x 32768 tokens, 8 KV heads, 32 query heads, head_dim 128,
-bf16, P=64, 2-bit):
-  mine K patterns, mine V patterns      (kvq_mine_patterns x2)
+One step = one pass of the whole path over one batch of synthetic input (by default the
+breadth workload: 256 independent samples x 16384 tokens, 8 KV heads, 32 query heads,
+head_dim 128, bf16, P=64, 2-bit, per-sample perturbed centers):
+  mine K patterns, mine V patterns      (kvq_mine_patterns x2, pooled prefill of every sample)
   quantize-append the whole context     (kvq_quantize_append, into a freshly reset cache)
   one decode step of attention          (kvq_decode_attention)
-All work runs in libkvq's CUDA kernels through the C ABI.  Inputs (1 GiB of K/V) exceed the
-126 MB L2, so every step streams from HBM.
+All work runs in libkvq's CUDA kernels through the C ABI.  Inputs (16 GiB of K/V) exceed the
+126 MB L2, so every step streams from HBM.  After the headline the same step is measured on the
+Llama-shaped layer (2- and 4-bit) and the Qwen-shaped 128K layer (with and without the
+pre-transform), and the long chain-of-thought loop is timed per decode step (`per_config`).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME] [--bits 2|4]
 
@@ -29,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "2-bit quantized-KV decode attn KV-tokens/s & HBM GB/s vs ~8 TB/s; quant-append GB/s"
-DEFAULT_WORKLOAD = "llama3_8b_32k"
+DEFAULT_WORKLOAD = "breadth_256x16k"
 D = 128
 
 
@@ -155,7 +157,7 @@ def cpu_baseline(w, heads: int = 4, seqs: int | None = None):
         MK, cK, _ = oracle.mine_set(Kf.reshape(-1, D), w.P, w.iters, w.transform)
         MV, cV, _ = oracle.mine_set(Vf.reshape(-1, D), w.P, w.iters, w.transform)
         for b in range(B):
-            e = oracle.encode(Kf[b], Vf[b], w.bits, MK, MV, cK, cV)
+            e = oracle.encode(Kf[b], Vf[b], w.bits, MK, MV, cK, cV, v_rho=oracle.v_rho(w.v_alpha))
             qf = synth.to_float(q[b, h * Gq:(h + 1) * Gq], w.dtype)
             oracle.attention_unit(qf, Kf[b], e, MK, MV, cK, cV)
     dt = time.perf_counter() - t0
@@ -214,65 +216,51 @@ def workload_config(w, args):
             "patterns": w.P, "lloyd_iters": w.iters, "bits": w.bits, "group": 32,
             "transform": "hadamard+varnorm" if w.transform else "none",
             "input_dtype": "bf16" if w.dtype == 1 else "fp16", "parallelism": f"replica x{args.gpus} (batch-sharded)",
-            "l2": "inputs larger than L2 (1 GiB K/V per step, 126 MB L2)"}
+            "l2": f"inputs larger than L2 ({w.B * w.S * w.Hkv * D * 4 / 2**30:.1f} GiB of K/V per step, 126 MB L2)",
+            "v_threshold_alpha": w.v_alpha}
 
 
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--bits", type=int, default=2)
-    ap.add_argument("--ref-heads", type=int, default=1, help="reference arm: KV heads per step (bounded sample)")
-    ap.add_argument("--ref-seqs", type=int, default=2, help="reference arm: sequences per step (bounded sample)")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=0,
-                    help="override the workload's batch (smaller cases of the same kernels, for ncu captures)")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
-    if args.impl == "reference":
-        run_reference(args)
-        return
+# Sub-records measured after the headline (each its own workload and roofline): the Llama-shaped
+# layer at 2 and 4 bits, the Qwen-shaped 128K layer without and with the pre-transform.
+PER_CONFIG = [("llama3_8b_32k", {"bits": 2}), ("llama3_8b_32k", {"bits": 4}),
+              ("qwen25_7b_128k", {}), ("qwen25_7b_128k", {"transform": 1})]
 
+
+def launches_per_step(w, full_pages: bool) -> int:
+    """Kernels this library launches per step: per mining call init + per Lloyd iteration
+    assignment (+ the float64 fix-up after the tcgen05 assignment), cluster sums and update (+16
+    for the pre-transform fit and apply); append: prep, full pages, partial pages, tail; decode: 1."""
+    tc = w.dtype == 1 and not w.transform and w.P <= 128
+    mine = 1 + (4 if tc else 3) * w.iters + (16 if w.transform else 0)
+    return 2 * mine + (4 if full_pages else 3) + 1
+
+
+def measure_path(w, args, dev, world: int, rank: int, headline: bool):
+    """Time `args.steps` steps of the whole path on workload w (mine K and V patterns on the
+    pooled prefill, quantize-append the whole context into a reset cache, one decode step).
+    Returns the record (and, for the headline, the end-to-end measurement through host buffers)."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     import bit_kv_cache_26_b200 as kvq
     import synth
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-
-    base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
-    if args.batch:
-        base = base.with_(B=args.batch)
-    w = rank_workload(base, rank)
     k, v = synth.gen_kv(w)
     q = synth.gen_q(w)
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
 
     def pinned(a):
-        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(tdt)
-        return t.pin_memory()
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(tdt).pin_memory()
 
     kh, vh, qh = pinned(k), pinned(v), pinned(q)
     del k, v
     kd, vd, qd = kh.to(dev), vh.to(dev), qh.to(dev)
-    cache = kvq.PagedKVCache(w.B, w.Hkv, w.S, w.bits, w.P, dtype=w.dtype, transform=w.transform, device=dev)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, w.S, w.bits, w.P, dtype=w.dtype, transform=w.transform, device=dev,
+                             v_rho=kvq.kvq_v_rho_star(D, w.v_alpha))
     n = w.B * w.S
     ws_m = kvq._alloc_aligned(kvq.kvq_mine_workspace_bytes(n, 1, w.Hkv, w.P, w.transform), dev)
     ws_d = cache.decode_workspace(w.Hq)
@@ -280,9 +268,6 @@ def main():
     out = torch.empty(w.B, w.Hq, D, device=dev)
     out_h = torch.empty(w.B, w.Hq, D).pin_memory()
     tok_stride, set_stride = w.Hkv * D, n * w.Hkv * D
-    stream = torch.cuda.current_stream()
-
-    tc_path = w.dtype == kvq.KVQ_BF16 and not w.transform and w.P <= 128
 
     def step(kx, vx, qx, ev=None):
         if ev: ev[0].record()
@@ -299,19 +284,22 @@ def main():
 
     def barrier():
         if world > 1:
+            import torch.distributed as dist
             dist.barrier()
 
     for _ in range(args.warmup):
         step(kd, vd, qd)
     torch.cuda.synchronize()
     assert cache.read_status() == 0, "device status bits set"
+    assert kvq.kvq_mine_read_status(ws_m) == 0, "mining status bits set"
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0) if headline else None
     barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
@@ -319,38 +307,44 @@ def main():
         step(kd, vd, qd, evs[i])
     t_end.record()
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     mine_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     append_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    # V adaptive threshold: share of V vectors stored with their pattern (index != 255)
+    sub = cache.subblock_bytes
+    cb = 32 * D * w.bits // 8
+    pool = cache.pool.view(-1, sub)
+    vidx = pool[:, 2 * cb + 2080:2 * cb + 2112]
+    utilisation = float((vidx != 255).float().mean()) if w.v_alpha > 0 else 1.0
 
-    # end to end through host buffers: H2D of K, V, q from pinned memory, the step, D2H of the output
-    for _ in range(2):
-        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
-        step(kd, vd, qd)
-        out_h.copy_(out, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
-        step(kd, vd, qd)
-        out_h.copy_(out, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    barrier()
-
-    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], device=dev)
+    e2e = None
+    if headline:
+        # end to end through host buffers: H2D of K, V, q from pinned memory, the step, D2H of the output
+        for _ in range(2):
+            kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+            step(kd, vd, qd)
+            out_h.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+            step(kd, vd, qd)
+            out_h.copy_(out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        barrier()
+        elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], device=dev)
+        e2e = {"ms": e2e_ms, "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
+               "d2h_bytes_per_step": int(out_h.numel() * 4)}
 
     ms_per_step = elapsed_ms / args.steps
-    tokens = n * world
-    value = tokens / (ms_per_step * 1e-3)
-    e2e_value = tokens / (e2e_ms / args.steps * 1e-3)
     pk = peaks()
     bpt = bytes_per_token_head(w.bits, w.transform)
     token_heads = n * w.Hkv
@@ -369,36 +363,163 @@ def main():
     traffic = dram_traffic(w.name, w.bits, w.B)
     for name, r in rooflines.items():
         r["traffic"] = traffic.get(name)
-    for r in rooflines.values():
         r["frac"] = r["achieved"] / r["peak"]
-    dominant = max(rooflines, key=lambda k: rooflines[k]["ms"])
+    dominant = max(rooflines, key=lambda kk: rooflines[kk]["ms"])
     dom = rooflines[dominant]
     roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
                 "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dominant, "peak_source": pk["source"]}
+    tokens = n * world
+    rec = {"workload": w.name, "bits": w.bits, "transform": bool(w.transform), "value": tokens / (ms_per_step * 1e-3),
+           "unit": "KV-tokens/s", "ms_per_step": ms_per_step,
+           "phases_ms": {"mine_patterns_KV": mine_ms, "quantize_append": append_ms, "decode_attention": decode_ms},
+           "decode_kv_tokens_per_s": tokens / (decode_ms * 1e-3), "decode_hbm_gbs": rooflines["decode_attention"]["achieved"],
+           "quant_append_gbs": rooflines["quantize_append"]["achieved"], "v_pattern_utilisation": utilisation,
+           "roofline": roofline, "rooflines": rooflines,
+           "gpu_launches": args.steps * launches_per_step(w, kvq_full_pages(w))}
+    del kd, vd, qd, kh, vh, qh, cache, ws_m, ws_d, ws_a
+    torch.cuda.empty_cache()
+    return rec, e2e, clk
+
+
+def kvq_full_pages(w) -> bool:
+    """Whether the full-page append kernel serves this workload (16-bit input, no pre-transform, P <= 128)."""
+    return not w.transform and w.P <= 128
+
+
+def measure_decode_loop(w, args, dev, nsteps: int = 512):
+    """Long chain-of-thought decode: mine patterns on the 8192-token prefill (frozen after it),
+    append the prefill, then steps of a one-token quantize-append per sequence followed by decode
+    attention with a new query; each step timed with CUDA events (median over `nsteps` steps after
+    32 warm-up steps)."""
+    import numpy as np
+    import torch
+
+    import bit_kv_cache_26_b200 as kvq
+    import synth
+
+    total = w.S + nsteps + 32
+    k, v = synth.gen_kv(w.with_(S=total))
+    tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
+    kd = torch.from_numpy(np.ascontiguousarray(k).view(np.int16)).view(tdt).to(dev)
+    vd = torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(tdt).to(dev)
+    del k, v
+    qs = torch.stack([torch.from_numpy(np.ascontiguousarray(synth.gen_q(w, step=t)).view(np.int16)).view(tdt)
+                      for t in range(nsteps + 32)]).to(dev)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, total, w.bits, w.P, dtype=w.dtype, transform=w.transform, device=dev,
+                             v_rho=kvq.kvq_v_rho_star(D, w.v_alpha))
+    n = w.B * w.S
+    pre_k, pre_v = kd[:, :w.S].contiguous(), vd[:, :w.S].contiguous()
+    ws_m = kvq._alloc_aligned(kvq.kvq_mine_workspace_bytes(n, 1, w.Hkv, w.P, w.transform), dev)
+    for x, pat, col in ((pre_k, cache.k_patterns, cache.k_colscale), (pre_v, cache.v_patterns, cache.v_colscale)):
+        kvq.kvq_mine_patterns(x, w.dtype, n, 1, w.Hkv, w.Hkv * D, D, n * w.Hkv * D, w.P, w.iters, w.transform,
+                              pat, col, None, ws_m)
+    del pre_k, pre_v
+    cache.append(kd[:, :w.S].contiguous(), vd[:, :w.S].contiguous())
+    steps_k = [kd[:, w.S + t:w.S + t + 1].contiguous() for t in range(nsteps + 32)]
+    steps_v = [vd[:, w.S + t:w.S + t + 1].contiguous() for t in range(nsteps + 32)]
+    ws_d = cache.decode_workspace(w.Hq)
+    out = torch.empty(w.B, w.Hq, D, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+    for t in range(nsteps + 32):
+        e = ev[t - 32] if t >= 32 else None
+        if e: e[0].record()
+        cache.append(steps_k[t], steps_v[t])
+        cache.decode(qs[t], out, ws_d)
+        if e: e[1].record()
+    torch.cuda.synchronize()
+    assert cache.read_status() == 0, "device status bits set"
+    us = sorted(1e3 * a.elapsed_time(b) for a, b in ev)
+    med = us[len(us) // 2]
+    ctx = w.S + 32 + nsteps // 2
+    pk = peaks()
+    step_bytes = w.B * ctx * w.Hkv * bytes_per_token_head(w.bits, w.transform)
+    rec = {"workload": w.name, "bits": w.bits, "metric": "us per decode step (1-token quantize-append + decode)",
+           "us_per_step_median": med, "us_per_step_p10": us[len(us) // 10], "us_per_step_p90": us[9 * len(us) // 10],
+           "steps_timed": nsteps, "context_tokens_mid": ctx, "launches_per_step": 4,
+           "value": w.B * ctx / (med * 1e-6), "unit": "KV-tokens/s (decode, at the median step)",
+           "roofline": {"bound": "hbm", "achieved": step_bytes / (med * 1e-6) / 1e9, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": step_bytes / (med * 1e-6) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                        "kernel": "decode step (append + decode)", "peak_source": pk["source"]}}
+    del kd, vd, qs, cache, ws_m, ws_d, steps_k, steps_v
+    torch.cuda.empty_cache()
+    return rec
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--ref-heads", type=int, default=1, help="reference arm: KV heads per step (bounded sample)")
+    ap.add_argument("--ref-seqs", type=int, default=2, help="reference arm: sequences per step (bounded sample)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="headline workload only")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases of the same kernels, for ncu captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    if args.batch:
+        base = base.with_(B=args.batch)
+    w = rank_workload(base, rank)
+    rec, e2e, clk = measure_path(w, args, dev, world, rank, headline=True)
+
+    per_config = []
+    if world == 1 and not args.no_per_config and not args.batch:
+        for name, kw in PER_CONFIG:
+            wc = synth.WORKLOADS[name].with_(**kw)
+            r, _, _ = measure_path(wc, args, dev, 1, 0, headline=False)
+            if not args.no_cpu_baseline:
+                r["cpu_baseline"], _ = cpu_baseline(wc, heads=1, seqs=1)
+            per_config.append(r)
+        wl = synth.WORKLOADS["long_cot_8k"]
+        r = measure_decode_loop(wl, args, dev)
+        if not args.no_cpu_baseline:
+            r["cpu_baseline"], _ = cpu_baseline(wl.with_(S=wl.S + 256), heads=1, seqs=1)
+        per_config.append(r)
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "KV-tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": rec["value"], "unit": "KV-tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32 (fp32 quantization, f64 mining distances, bf16 inputs)",
             "data": "synthetic (seeded Gaussian-mixture K/V with outlier channels and RoPE)",
             "config": workload_config(w, args),
-            "phases_ms": {"mine_patterns_KV": mine_ms, "quantize_append": append_ms, "decode_attention": decode_ms},
-            "decode_kv_tokens_per_s": n * world / (decode_ms * 1e-3),
-            "decode_hbm_gbs": rooflines["decode_attention"]["achieved"],
-            "quant_append_gbs": rooflines["quantize_append"]["achieved"],
-            "roofline": roofline, "rooflines": rooflines,
-            "e2e": {"value": e2e_value, "unit": "KV-tokens/s",
-                    "h2d_bytes_per_step": int(kh.numel() * 2 + vh.numel() * 2 + qh.numel() * 2),
-                    "d2h_bytes_per_step": int(out_h.numel() * 4)},
-            # per mining call: init, then per iteration assignment (+ the float64 fix-up after the
-            # tcgen05 assignment: bf16 input, P <= 128), cluster sums and update; the pre-transform
-            # fit adds 15; append: prep, pages, tail; decode: one kernel
-            "gpu_launches": args.steps * (2 * (1 + (4 if tc_path else 3) * w.iters + (15 if w.transform else 0)) + 3 + 1),
+            "phases_ms": rec["phases_ms"], "decode_kv_tokens_per_s": rec["decode_kv_tokens_per_s"],
+            "decode_hbm_gbs": rec["decode_hbm_gbs"], "quant_append_gbs": rec["quant_append_gbs"],
+            "v_pattern_utilisation": rec["v_pattern_utilisation"],
+            "roofline": rec["roofline"], "rooflines": rec["rooflines"],
+            "e2e": {"value": w.B * w.S * world / (e2e["ms"] / args.steps * 1e-3), "unit": "KV-tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]},
+            "gpu_launches": rec["gpu_launches"],
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"], _ = cpu_baseline(w, heads=4)
+            line["cpu_baseline"], _ = cpu_baseline(w, heads=1, seqs=2)
+        if per_config:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

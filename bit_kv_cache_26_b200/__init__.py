@@ -42,7 +42,7 @@ class kvq_cache(ctypes.Structure):
         ("num_seqs", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("group", ctypes.c_int32), ("bits", ctypes.c_int32), ("num_patterns", ctypes.c_int32),
         ("num_sets", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
-        ("dtype", ctypes.c_int32), ("transform", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("transform", ctypes.c_int32), ("v_rho", ctypes.c_float),
         ("page_pool", ctypes.c_void_p), ("page_table", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
         ("k_tail", ctypes.c_void_p), ("k_patterns", ctypes.c_void_p), ("v_patterns", ctypes.c_void_p),
         ("seq_to_set", ctypes.c_void_p), ("k_colscale", ctypes.c_void_p), ("v_colscale", ctypes.c_void_p),
@@ -55,6 +55,7 @@ _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ct
 _SIGS = {
     "kvq_page_bytes": (_sz, [_P]),
     "kvq_subblock_bytes": (_sz, [_i32, _i32]),
+    "kvq_v_rho_star": (_f32, [_i32, ctypes.c_double]),
     "kvq_mine_workspace_bytes": (_sz, [_i64, _i32, _i32, _i32, _i32]),
     "kvq_mine_patterns": (ctypes.c_int, [_vp, _i32, _i64, _i32, _i32, _i64, _i64, _i64, _i32, _i32, _i32,
                                          _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -65,6 +66,7 @@ _SIGS = {
     "kvq_decode_attention_static": (ctypes.c_int, [_P, _vp, _i32, _f32, _vp, _vp]),
     "kvq_dequantize": (ctypes.c_int, [_P, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "kvq_read_status": (ctypes.c_int, [_P, ctypes.POINTER(_i32), _i32, _vp]),
+    "kvq_mine_read_status": (ctypes.c_int, [_vp, ctypes.POINTER(_i32), _vp]),
     "kvq_last_error": (ctypes.c_char_p, []),
     "kvq_version": (ctypes.c_char_p, []),
 }
@@ -103,6 +105,11 @@ def kvq_subblock_bytes(bits: int, transform: int) -> int:
     return int(_lib.kvq_subblock_bytes(bits, transform))
 
 
+def kvq_v_rho_star(head_dim: int, alpha: float) -> float:
+    """rho*(d, alpha) of PatternKV Eq. 10 as the fp32 value the kernels compare with (0 = off)."""
+    return float(_lib.kvq_v_rho_star(head_dim, alpha))
+
+
 def kvq_page_bytes(cache: kvq_cache) -> int:
     return int(_lib.kvq_page_bytes(ctypes.byref(cache)))
 
@@ -119,6 +126,15 @@ def kvq_mine_patterns(x: torch.Tensor, dtype: int, n: int, num_sets: int, num_kv
     _check(_lib.kvq_mine_patterns(_ptr(x), dtype, n, num_sets, num_kv_heads, tok_stride, head_stride, set_stride, P,
                                   iters, transform, _ptr(patterns_out), _ptr(colscale_out), _ptr(assign_out),
                                   _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def kvq_mine_read_status(ws: torch.Tensor, stream=None) -> int:
+    """Status bits of the mining call that used workspace `ws` (synchronises the stream)."""
+    bits = ctypes.c_int32(0)
+    rc = _lib.kvq_mine_read_status(_ptr(ws), ctypes.byref(bits), _stream(stream))
+    if rc not in (KVQ_OK, KVQ_ERR_DEVICE):
+        _check(rc)
+    return int(bits.value)
 
 
 def kvq_append_workspace_bytes(cache: kvq_cache, n_new: int) -> int:
@@ -178,11 +194,14 @@ class PagedKVCache:
 
     page_order: optional permutation of the physical pages (default: sequence-major,
     page i of sequence b at b * max_pages_per_seq + i).
+    v_rho: V adaptive threshold (PatternKV Section 3.3); kvq_v_rho_star(128, alpha) for a
+    significance level alpha, 0 = off.
     """
 
     def __init__(self, num_seqs: int, num_kv_heads: int, max_tokens: int, bits: int, num_patterns: int,
                  dtype: int = KVQ_BF16, transform: int = KVQ_TX_NONE, num_sets: int = 1, device="cuda",
-                 page_order: torch.Tensor | None = None, seq_to_set: torch.Tensor | None = None):
+                 page_order: torch.Tensor | None = None, seq_to_set: torch.Tensor | None = None,
+                 v_rho: float = 0.0):
         self.device = torch.device(device)
         self.B, self.H, self.bits, self.P, self.S = num_seqs, num_kv_heads, bits, num_patterns, num_sets
         self.dtype, self.transform = dtype, transform
@@ -191,7 +210,8 @@ class PagedKVCache:
         c = kvq_cache()
         c.num_seqs, c.num_kv_heads, c.head_dim, c.group = num_seqs, num_kv_heads, HEAD_DIM, GROUP
         c.bits, c.num_patterns, c.num_sets = bits, num_patterns, num_sets
-        c.max_pages_per_seq, c.num_pages, c.dtype, c.transform, c.reserved = self.maxp, self.num_pages, dtype, transform, 0
+        c.max_pages_per_seq, c.num_pages, c.dtype, c.transform = self.maxp, self.num_pages, dtype, transform
+        c.v_rho = v_rho
         self.page_bytes = kvq_page_bytes(c)
         if self.page_bytes == 0:
             raise KvqError(KVQ_ERR_UNSUPPORTED, f"unsupported cache shape (bits={bits})")
@@ -253,10 +273,12 @@ class PagedKVCache:
 
 
 def mine(x: torch.Tensor, P: int, iters: int = 4, transform: int = KVQ_TX_NONE, num_sets: int = 1,
-         want_assign: bool = False, stream=None):
+         want_assign: bool = False, stream=None, check: bool = True):
     """Mine patterns from x shaped [num_sets, n, H, 128] (fp16/bf16, contiguous).
 
     Returns (patterns [sets,H,P,128] fp32, colscale [sets,H,128] or None, assign [sets,H,n] or None).
+    With `check`, the call's device status word is read back (a stream synchronisation) and a
+    set bit raises KvqError.
     """
     assert x.dim() == 4 and x.shape[-1] == HEAD_DIM and x.is_contiguous()
     S, n, H, _ = x.shape
@@ -267,4 +289,8 @@ def mine(x: torch.Tensor, P: int, iters: int = 4, transform: int = KVQ_TX_NONE, 
     ws = _alloc_aligned(kvq_mine_workspace_bytes(n, S, H, P, transform), x.device)
     kvq_mine_patterns(x, dt, n, S, H, H * HEAD_DIM, HEAD_DIM, n * H * HEAD_DIM, P, iters, transform, pats, col, asg,
                       ws, stream)
+    if check:
+        bits = kvq_mine_read_status(ws, stream)
+        if bits:
+            raise KvqError(KVQ_ERR_DEVICE, f"mining status bits 0x{bits:x}")
     return pats, col, asg

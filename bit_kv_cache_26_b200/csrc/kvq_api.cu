@@ -1,6 +1,7 @@
 // C-ABI entry points of libkvq (declared in include/kvq.h): host-side argument
 // validation, workspace sizing and kernel launches.  No exception crosses the
 // ABI; nothing here allocates device memory.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -43,10 +44,15 @@ kvq_status check_cache(const kvq_cache* c) {
   if (c->dtype != KVQ_F16 && c->dtype != KVQ_BF16) return fail(KVQ_ERR_UNSUPPORTED, "dtype %d", c->dtype);
   if (c->transform != KVQ_TX_NONE && c->transform != KVQ_TX_HADAMARD_VARNORM)
     return fail(KVQ_ERR_UNSUPPORTED, "transform %d", c->transform);
-  if (c->reserved != 0) return fail(KVQ_ERR_INVALID_ARG, "reserved field must be 0");
+  if (!(c->v_rho >= 0.0f) || !(c->v_rho < INFINITY))
+    return fail(KVQ_ERR_INVALID_ARG, "v_rho must be finite and >= 0 (0 = adaptive threshold off)");
   if (c->num_seqs < 0 || c->num_kv_heads < 1 || c->num_sets < 1 || c->max_pages_per_seq < 0 || c->num_pages < 0)
     return fail(KVQ_ERR_INVALID_ARG, "negative or zero size in cache (seqs %d heads %d sets %d pages %d/%d)",
                 c->num_seqs, c->num_kv_heads, c->num_sets, c->max_pages_per_seq, c->num_pages);
+  // sequences and KV heads index the z and y dimensions of the launch grids
+  if (c->num_seqs > 65535 || c->num_kv_heads > 65535)
+    return fail(KVQ_ERR_CAPACITY, "%d sequences / %d KV heads exceed the 65535 the launch grids allow", c->num_seqs,
+                c->num_kv_heads);
   if (c->num_seqs > 0) {
     if (!c->page_pool || !c->page_table || !c->seq_len || !c->k_tail || !c->k_patterns || !c->v_patterns ||
         !c->status)
@@ -67,6 +73,22 @@ extern "C" {
 const char* kvq_last_error(void) { return g_err; }
 
 const char* kvq_version(void) { return "kvq 0.1 (sm_100a)"; }
+
+float kvq_v_rho_star(int32_t head_dim, double alpha) {
+  if (!(alpha > 0.0) || !(alpha < 0.5) || head_dim < 1) return 0.0f;
+  // z = Phi^-1(1 - alpha) by bisection on the upper tail 0.5 erfc(z / sqrt 2)
+  double lo = 0.0, hi = 40.0;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    (0.5 * erfc(mid / sqrt(2.0)) > alpha ? lo : hi) = mid;
+  }
+  const double z = 0.5 * (lo + hi);
+  // Eq. 10 with equality, u = rho^2, k = 2 z / sqrt(5 d): (1 - k^2) u^2 - 2 u + (1 - k^2) = 0
+  const double k = 2.0 * z / sqrt(5.0 * head_dim), a = 1.0 - k * k;
+  if (!(a > 0.0)) return 0.0f;
+  const double u = (1.0 - sqrt(1.0 - a * a)) / a;
+  return (float)sqrt(u);
+}
 
 size_t kvq_subblock_bytes(int32_t bits, int32_t transform) {
   if (bits != 2 && bits != 4) return 0;
@@ -99,6 +121,10 @@ kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, int32_t nu
   if (num_sets == 0 || num_kv_heads == 0) return KVQ_OK;
   if (n < P) return fail(KVQ_ERR_INVALID_ARG, "n = %lld tokens is fewer than P = %d patterns", (long long)n, P);
   if (n > (int64_t)1 << 31) return fail(KVQ_ERR_CAPACITY, "n = %lld exceeds 2^31", (long long)n);
+  // (set, KV head) problems index the y / z dimension of the mining grids
+  if ((int64_t)num_sets * num_kv_heads > 65535)
+    return fail(KVQ_ERR_CAPACITY, "%d sets x %d KV heads exceed the 65535 problems the launch grids allow", num_sets,
+                num_kv_heads);
   if (!x || !patterns_out) return fail(KVQ_ERR_INVALID_ARG, "x / patterns_out is NULL");
   if (transform && !colscale_out) return fail(KVQ_ERR_INVALID_ARG, "transform needs colscale_out");
   if (tok_stride < 0 || head_stride < 0 || set_stride < 0)
@@ -189,6 +215,19 @@ kvq_status kvq_dequantize(const kvq_cache* cache, int32_t seq, int32_t seq_len_h
   kvq::Geom g = kvq::make_geom(*cache);
   cudaError_t e = kvq::launch_dequant(g, seq, start, count, k_out, v_out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kvq_dequantize");
+  return KVQ_OK;
+}
+
+kvq_status kvq_mine_read_status(const void* ws, int32_t* bits_out, kvq_stream_t stream) {
+  g_err[0] = 0;
+  if (!ws || !bits_out) return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "kvq_mine_read_status");
+  *bits_out = v;
+  if (v) return fail(KVQ_ERR_DEVICE, "mining status bits 0x%x", v);
   return KVQ_OK;
 }
 

@@ -98,8 +98,10 @@ struct PageCtx {
   const float* cV;
 };
 
-// Returns false if the CTA has nothing to do (or an error was flagged).
-__device__ bool page_context(const Geom& g, int n_new, PageCtx& c) {
+// Returns false if the CTA has nothing to do (or an error was flagged).  With `partial_only`
+// (the full-page kernel takes every page the call fills completely) CTA x = 0 takes the first
+// page the call touches and x = 1 the last, each only if the call does not fill it completely.
+__device__ bool page_context(const Geom& g, int n_new, bool partial_only, PageCtx& c) {
   const int b = blockIdx.z, h = blockIdx.y;
   c.L = g.seq_len[b];
   c.n = n_new;
@@ -107,10 +109,17 @@ __device__ bool page_context(const Geom& g, int n_new, PageCtx& c) {
     if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(g.status, KVQ_DEV_OVERFLOW);
     return false;
   }
-  c.pg = c.L / kG + blockIdx.x;
+  if (partial_only) {
+    const int first = c.L / kG, last = (c.L + n_new - 1) / kG;
+    if (blockIdx.x == 1 && last == first) return false;
+    c.pg = blockIdx.x == 0 ? first : last;
+  } else {
+    c.pg = c.L / kG + blockIdx.x;
+  }
   c.a = max(c.L, c.pg * kG);
   c.e = min(c.L + n_new, c.pg * kG + kG);
   if (c.a >= c.e) return false;
+  if (partial_only && c.a == c.pg * kG && c.e == c.pg * kG + kG) return false;  // a full page
   const int phys = g.page_table[(size_t)b * g.maxp + c.pg];
   if (phys < 0 || phys >= g.npages) {
     if (threadIdx.x == 0) set_status(g.status, KVQ_DEV_BAD_PAGE);
@@ -295,9 +304,9 @@ __device__ __forceinline__ void group_sz(float mn, float mx, int bits, float& s,
 __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g, AppendWs wsp,
                                                                          const uint16_t* __restrict__ k_new,
                                                                          const uint16_t* __restrict__ v_new,
-                                                                         int n_new) {
+                                                                         int n_new, bool partial_only) {
   PageCtx c;
-  if (!page_context(g, n_new, c)) return;
+  if (!page_context(g, n_new, partial_only, c)) return;
   const int b = blockIdx.z, h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int P = g.P;
@@ -307,6 +316,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __shared__ float vrow_s[kG], krow_s[kG];
   __shared__ unsigned long long best[2 * kG];  // (d_mm bits << 32) | pattern, per row
   __shared__ float dseed[2 * kG], hlb[2][2 * kG];
+  __shared__ float rraw[kG];      // V rows: range max - min of the vector (adaptive threshold)
+  __shared__ bool vkeep[kG];      // V rows: the pattern is kept (else quantized raw, index 255)
   __shared__ int seed[2 * kG], hj[2][2 * kG];
   __shared__ int qn;
   // dynamic: fp16 lower bounds lb[j][row], then the probe tables (V: [P][32], K: [P][16]) and
@@ -415,15 +426,29 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const int r = tid >> 1, hh = tid & 1;
     const bool on = row_on(r);
     int s = 0;
-    float mx = -INFINITY, mn = INFINITY;
+    float mx = -INFINITY, mn = INFINITY, ymx = -INFINITY, ymn = INFINITY;
     if (on) {
       s = hlb[1][r] < hlb[0][r] ? hj[1][r] : hj[0][r];
       s = min(max(s, 0), P - 1);
       const float* m = (r < kG ? c.MV : c.MK) + (size_t)s * kD;
       range64(vec[r], m, 64 * hh, hh, mx, mn);
+      if (r < kG && g.vrho > 0.0f) {  // the V vector's own range, for the adaptive threshold
+        const float4* y4 = reinterpret_cast<const float4*>(vec[r] + 64 * hh);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float4 a = y4[k];
+          ymx = max3(ymx, a.x, a.y);
+          ymn = min3(ymn, a.x, a.y);
+          ymx = max3(ymx, a.z, a.w);
+          ymn = min3(ymn, a.z, a.w);
+        }
+      }
     }
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
     mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+    ymx = fmaxf(ymx, __shfl_xor_sync(kFull, ymx, 1));
+    ymn = fminf(ymn, __shfl_xor_sync(kFull, ymn, 1));
+    if (on && hh == 0 && r < kG) rraw[r] = __fsub_rn(ymx, ymn);
     const float ds = __fsub_rn(mx, mn);
     if (on && hh == 0) {
       dseed[r] = ds;
@@ -489,12 +514,15 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       const int r = lane + kG * u;
       float s = 0.f, z = 0.f, ri = 0.f;
       if (row_on(r)) {
+        // V: the adaptive threshold may drop the pattern (residual = the vector itself)
+        const bool keep = u || v_keep_pattern(g.vrho, __uint_as_float((uint32_t)(best[r] >> 32)), rraw[r]);
+        if (u == 0 && q == 0) vkeep[r] = keep;
         const float4* m4 = reinterpret_cast<const float4*>((u ? c.MK : c.MV) + (size_t)(best[r] & 0xffffffffu) * kD +
                                                            32 * q);
         float4* y4 = reinterpret_cast<float4*>(&vec[r][32 * q]);
         float4 mv[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mv[k] = __ldg(m4 + k);
+        for (int k = 0; k < 8; ++k) mv[k] = keep ? __ldg(m4 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
         float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -581,7 +609,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const int slot = tid;
     const bool present = slot >= lo && slot < hi;
     if (c.fresh || present) {
-      vidx_g[tok_pos(slot)] = present ? (uint8_t)(best[slot] & 0xff) : (uint8_t)0;
+      vidx_g[tok_pos(slot)] = !present ? (uint8_t)0 : vkeep[slot] ? (uint8_t)(best[slot] & 0xff) : (uint8_t)kRawIndex;
       if (g.tx) vrow_g[tok_pos(slot)] = present ? vrow_s[slot] : 0.f;
     }
   }
@@ -629,8 +657,13 @@ cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, i
   if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
       cudaSuccess)
     return e;
-  dim3 grid(n_new / kG + 2, g.H, g.B);
-  append_pages_kernel<<<grid, kAppendThreads, dyn, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new, n_new);
+  // pages the call fills completely: the full-page kernel; the rest (at most the first and the
+  // last touched page of each sequence): the general kernel
+  const bool full = append_full_eligible(g, n_new);
+  if (full && (e = launch_append_full(g, k_new, v_new, n_new, w.probe, w.pv, st)) != cudaSuccess) return e;
+  dim3 grid(full ? 2 : n_new / kG + 2, g.H, g.B);
+  append_pages_kernel<<<grid, kAppendThreads, dyn, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new, n_new,
+                                                         full);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_tail_kernel<<<g.B, 256, 0, st>>>(g, (const uint16_t*)k_new, n_new);

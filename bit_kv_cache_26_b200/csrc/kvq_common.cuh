@@ -37,6 +37,8 @@ struct Geom {
   const float* kcol;
   const float* vcol;
   int32_t* status;
+  uint32_t wait_limit;  // iterations of a bounded page-copy wait (decode)
+  float vrho;           // V adaptive threshold rho* (0 = off)
 };
 
 __host__ __device__ inline int64_t subblock_bytes_of(int bits, int tx) {
@@ -69,6 +71,8 @@ inline Geom make_geom(const kvq_cache& c) {
   g.kcol = c.k_colscale;
   g.vcol = c.v_colscale;
   g.status = c.status;
+  g.wait_limit = 1u << 22;
+  g.vrho = c.v_rho;
   return g;
 }
 
@@ -291,6 +295,12 @@ __device__ __forceinline__ float dmm_reg(const float (&y)[kD], const float* __re
   }
   return __fsub_rn(mx, mn);
 }
+
+// V adaptive threshold: keep the pattern iff R_flat <= fl32(rho* x R_raw) (rho* > 0), else quantize raw.
+__device__ __forceinline__ bool v_keep_pattern(float vrho, float r_flat, float r_raw) {
+  return !(vrho > 0.0f) || r_flat <= __fmul_rn(vrho, r_raw);
+}
+constexpr int kRawIndex = 255;  // stored V index of a vector quantized without its pattern
 
 // Group quantizer on the 32 lanes of a warp (one value per lane): s, z and this lane's code.
 __device__ __forceinline__ int quant_warp(float R, int bits, float& s_out, float& z_out) {

@@ -8,6 +8,9 @@
 //   m  running max of the base-2 logits, l  sum of 2^(logit - m),
 //   o[128]  sum of p * (s*code + z) + sum_j W_j M_V[j] in the quantized space, with
 //           W_j the sum of p over the split's tokens that use V pattern j.
+#include <algorithm>
+#include <cstdlib>
+
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -26,10 +29,22 @@ size_t decode_workspace(const Geom& g, int Hq, int nsplit) {
   return rows * (2 + kD) * sizeof(float) + (size_t)g.B * g.H * sizeof(int) + 256;
 }
 
+// Iteration limit of the page-copy waits: the default, or KVQ_TEST_WAIT_LIMIT (read once) for
+// tests that make the waits expire on purpose.
+uint32_t page_wait_limit(uint32_t dflt) {
+  static const long long v = [] {
+    const char* e = getenv("KVQ_TEST_WAIT_LIMIT");
+    return e ? atoll(e) : -1LL;
+  }();
+  return v >= 0 ? (uint32_t)std::min<long long>(v, 0xffffffffLL) : dflt;
+}
+
 // Split partials, then the per-(sequence, KV head) arrival counters (zeroed here, on the stream).
-cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, float* out, void* ws, int nsplit,
+cudaError_t launch_decode(const Geom& g0, const void* q, int Hq, float sm_scale, float* out, void* ws, int nsplit,
                           cudaStream_t st) {
-  if (g.B == 0) return cudaSuccess;
+  if (g0.B == 0) return cudaSuccess;
+  Geom g = g0;
+  g.wait_limit = page_wait_limit(g0.wait_limit);
   const size_t rows = (size_t)g.B * Hq * nsplit;
   float* part_ml = reinterpret_cast<float*>(ws);
   float* part_o = part_ml + 2 * rows;

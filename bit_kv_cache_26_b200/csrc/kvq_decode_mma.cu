@@ -53,10 +53,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-// Bounded wait on an mbarrier phase: false if the phase did not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
+// Bounded wait on an mbarrier phase: false if the phase did not complete within `limit` tries.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = kSpinLimit) {
   const uint32_t addr = smem_u32(bar);
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+  for (uint32_t it = 0; it < limit; ++it) {
     uint32_t ok;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
@@ -170,7 +170,7 @@ __host__ __device__ inline Smem smem_plan(int sub_bytes, int stages, int NT, int
   s.qk = o; o += NT * 4 * kD * 4;          // query in the quantized space, per padded head, KSC order
   s.qraw = o; o += NT * 4 * kD * 4;        // raw query (exact tail keys), natural order
   s.T = o; o += NT * 4 * P * 4;            // T[h][j] = q . M_K[j]
-  s.W = o; o += kWarps * NT * 4 * P * 4;   // per-warp pattern weights
+  s.W = o; o += kWarps * NT * 4 * (P + 1) * 4;  // per-warp pattern weights (+1: tokens stored raw)
   s.pex = o; o += kWarps * NT * 4 * kPexLd * 4;  // per-warp p exchange
   s.total = o;
   return s;
@@ -261,7 +261,8 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   float* qraw = reinterpret_cast<float*>(smem + sp.qraw); // [NH][128]
   float* T = reinterpret_cast<float*>(smem + sp.T);       // [NH][P]
   float* Wall = reinterpret_cast<float*>(smem + sp.W);
-  float* Ww = Wall + warp * NH * P;                       // this warp's [NH][P]
+  const int P1 = P + 1;                                   // W slot P: V tokens stored raw (index 255)
+  float* Ww = Wall + warp * NH * P1;                      // this warp's [NH][P + 1]
   float* pex = reinterpret_cast<float*>(smem + sp.pex) + warp * NH * kPexLd;
 
   int L = g.seq_len[b];
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
 #pragma unroll
     for (int k = 0; k < 4; ++k) qk[hh * kD + ksc_pos(lane + 32 * k)] = v[k];
   }
-  for (int i = threadIdx.x; i < kWarps * NH * P; i += blockDim.x) Wall[i] = 0.f;
+  for (int i = threadIdx.x; i < kWarps * NH * P1; i += blockDim.x) Wall[i] = 0.f;
   // the transformed query comes from shared memory (after this barrier); the plain one straight
   // from global memory, so that its loads and the pattern rows' below share one round trip
   if (g.tx) __syncthreads();
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   for (int i = 0; i < my_n; ++i) {
     const int st = i % STAGES;
     const uint32_t phase = (i / STAGES) & 1;
-    const bool ok = mbar_wait(&bars[st], phase);
+    const bool ok = mbar_wait(&bars[st], phase, g.wait_limit);
     if (!__all_sync(kFull, ok)) { stuck_at = i; break; }
     const bool skip = __shfl_sync(kFull, (bad_mask >> st) & 1, 0);
     const uint8_t* pgp = ring + st * sub_bytes;
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
           for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
-          for (int jj = gq; jj < P; jj += 8) Ww[hh * P + jj] *= alpha;
+          for (int jj = gq; jj < P; jj += 8) Ww[hh * P1 + jj] *= alpha;
           __syncwarp();
         }
         mrun[j] = mnew;
@@ -506,7 +507,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
           const float p = real ? ex2(sc[j][u] - mnew) : 0.f;
           lrun[j] += p;
           pv[u] = p * vrow[u];
-          if (real) atomicAdd(&Ww[hh * P + min((int)((vidx4 >> (8 * u)) & 0xff), P - 1)], pv[u]);
+          if (real) atomicAdd(&Ww[hh * P1 + min((int)((vidx4 >> (8 * u)) & 0xff), P)], pv[u]);
           zacc[j][0] = fmaf(pv[u], vz[u].x, zacc[j][0]);
           zacc[j][1] = fmaf(pv[u], vz[u].y, zacc[j][1]);
           zacc[j][2] = fmaf(pv[u], vz[u].z, zacc[j][2]);
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
         float kv[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) kv[k] = load_elem(kt + lane + 32 * k, g.dtype);
-        const int vidx = min((int)sub[g.off_vidx + tok_pos(t)], P - 1);
+        const int vidx = min((int)sub[g.off_vidx + tok_pos(t)], P);  // P: stored raw
         const float vrow = g.tx ? vr[tok_pos(t)] : 1.0f;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
             for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
               for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
-            for (int jj = gq; jj < P; jj += 8) Ww[hh * P + jj] *= alpha;
+            for (int jj = gq; jj < P; jj += 8) Ww[hh * P1 + jj] *= alpha;
           }
           mrun[j] = mnew;
           __syncwarp();
@@ -636,7 +637,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
           const float pv = p * vrow;
           if (gq == 0) {
             lrun[j] += p;
-            if (real) Ww[hh * P + vidx] += pv;
+            if (real) Ww[hh * P1 + vidx] += pv;
 #pragma unroll
             for (int u = 0; u < 4; ++u) zacc[j][u] = fmaf(pv, vz[vzc_pos(t, u)], zacc[j][u]);
           }
@@ -716,7 +717,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
     for (int jj = lane; jj < P; jj += 32) {
       float Wv = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) Wv += f[w] * Wall[(w * NH + hh) * P + jj];
+      for (int w = 0; w < kWarps; ++w) Wv += f[w] * Wall[(w * NH + hh) * P1 + jj];
       wc[jj * NH + hh] = Wv;
     }
   }

@@ -64,15 +64,15 @@ __global__ void dequant_kernel(Geom g, int b, int start, int count, float* __res
     const uint32_t* words = reinterpret_cast<const uint32_t*>(sub + g.off_vc);
     const float* vs = reinterpret_cast<const float*>(sub + g.off_vs);
     const float* vz = reinterpret_cast<const float*>(sub + g.off_vz);
-    const int idx = min((int)sub[g.off_vidx + tok_pos(slot)], g.P - 1);
-    const float* M = g.vpat + (sh * g.P + idx) * kD;
+    const int vi = sub[g.off_vidx + tok_pos(slot)];
+    const float* M = vi == kRawIndex ? nullptr : g.vpat + (sh * g.P + min(vi, g.P - 1)) * kD;  // 255: stored raw
     float v[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       int d = lane + 32 * k, w, bt;
       frag_pos(g.bits, 2, d, slot, w, bt);
       int code = (words[w] >> bt) & mask;
-      v[k] = vs[vsc_pos(slot, k)] * (float)code + vz[vzc_pos(slot, k)] + M[d];
+      v[k] = vs[vsc_pos(slot, k)] * (float)code + vz[vzc_pos(slot, k)] + (M ? M[d] : 0.0f);
     }
     if (g.tx) {
       float r = reinterpret_cast<const float*>(sub + g.off_vrow)[tok_pos(slot)];

@@ -23,6 +23,7 @@ constexpr int kFitPasses = 3;
 constexpr int kReduceChunk = 4096;
 
 struct MineWs {
+  int32_t* status;  // device status word (KVQ_DEV_* bits), at offset 0 of the workspace
   double* sums;     // [NP][P][128]
   uint32_t* cnt;    // [NP][P]
   int32_t* assign;  // [NP][n]
@@ -31,17 +32,32 @@ struct MineWs {
   int32_t* amb_cnt; // [NP]
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
+  double* colpart;  // [NP][fit chunks][128] per-chunk column partials (transform only)
   double* colsum;   // [NP][128]
   double* colsq;    // [NP][128]
   double* colscale; // [NP][128]  running product of column divisors
   double* coldiv;   // [NP][128]  this pass's divisor
+  double* accpart;  // [NP][sum chunks][P][128] per-CTA cluster sums of the fp32 rows (transform only)
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Cluster-sum CTAs per problem for the fp32 (pre-transformed) rows, whose float64 sums depend on
+// the order of the additions: each CTA writes its own partials, which the update adds in CTA
+// order, so the result is the same on every run.  A fixed CTA budget (two per SM of a 148-SM
+// part) keeps the workspace independent of the device.
+constexpr int kAccF32Ctas = 296;
+inline int64_t fit_chunks(int64_t n) { return (n + kReduceChunk - 1) / kReduceChunk; }
+inline int accum_f32_chunks(int64_t n, int NP, int P) {
+  const int slices = P <= 64 ? 1 : (P <= 128 ? 2 : 4);
+  const int64_t ntiles = (n + 127) / 128;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(ntiles, std::max(1, kAccF32Ctas / (slices * NP))));
+}
+
 inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* assign_out) {
   uint8_t* p = (uint8_t*)ws;
   MineWs w{};
+  w.status = (int32_t*)p; p += 256;
   w.sums = (double*)p; p += align256((size_t)NP * P * kD * sizeof(double));
   w.cnt = (uint32_t*)p; p += align256((size_t)NP * P * sizeof(uint32_t));
   if (assign_out) w.assign = assign_out;
@@ -52,10 +68,12 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   if (transform) {
     w.y = (float*)p; p += align256((size_t)NP * n * kD * sizeof(float));
     w.v64 = (double*)p; p += align256((size_t)NP * n * kD * sizeof(double));
+    w.colpart = (double*)p; p += align256((size_t)NP * fit_chunks(n) * kD * sizeof(double));
     w.colsum = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
     w.colsq = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
     w.colscale = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
     w.coldiv = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
+    w.accpart = (double*)p; p += align256((size_t)NP * accum_f32_chunks(n, NP, P) * P * kD * sizeof(double));
   }
   return w;
 }
@@ -113,30 +131,37 @@ __global__ void fit_row_kernel(int64_t n, double* v64, const double* coldiv) {
   for (int k = 0; k < 4; ++k) row[lane + 32 * k] = v[k] / r;
 }
 
-// Column statistics: pass 0 sums, pass 1 squared deviations from the mean; 128 threads = channels.
-__global__ void fit_col_kernel(int64_t n, const double* v64, double* colsum, double* colsq, int which) {
+// Column statistics, per chunk of kReduceChunk tokens: pass 0 sums, pass 1 squared deviations
+// from the mean; 128 threads = channels.  Each chunk writes its own partial, and
+// fit_colreduce_kernel adds the partials in chunk order, so the statistics (and the column
+// factors) are the same on every run.
+__global__ void fit_col_kernel(int64_t n, const double* v64, const double* colsum, double* colpart, int which) {
   const int prob = blockIdx.y, d = threadIdx.x;
   const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk, i1 = min(n, i0 + kReduceChunk);
   const double* base = v64 + (size_t)prob * n * kD;
   double acc = 0.0;
   if (which == 0) {
     for (int64_t i = i0; i < i1; ++i) acc += base[i * kD + d];
-    atomicAdd(colsum + prob * kD + d, acc);
   } else {
-    double mean = colsum[prob * kD + d] / (double)n;
-    for (int64_t i = i0; i < i1; ++i) { double t = base[i * kD + d] - mean; acc += t * t; }
-    atomicAdd(colsq + prob * kD + d, acc);
+    const double mean = colsum[prob * kD + d] / (double)n;
+    for (int64_t i = i0; i < i1; ++i) { const double t = base[i * kD + d] - mean; acc += t * t; }
   }
+  colpart[((size_t)prob * gridDim.x + blockIdx.x) * kD + d] = acc;
 }
 
-__global__ void fit_colfinish_kernel(int64_t n, double* colsum, double* colsq, double* colscale, double* coldiv) {
+__global__ void fit_colreduce_kernel(int chunks, const double* colpart, double* out) {
+  const int prob = blockIdx.x, d = threadIdx.x;
+  double acc = 0.0;
+  for (int c = 0; c < chunks; ++c) acc += colpart[((size_t)prob * chunks + c) * kD + d];
+  out[prob * kD + d] = acc;
+}
+
+__global__ void fit_colfinish_kernel(int64_t n, const double* colsq, double* colscale, double* coldiv) {
   const int prob = blockIdx.x, d = threadIdx.x;
   double s = sqrt(colsq[prob * kD + d] / (double)n);
   if (s == 0.0) s = 1.0;
   colscale[prob * kD + d] *= s;
   coldiv[prob * kD + d] = s;
-  colsum[prob * kD + d] = 0.0;
-  colsq[prob * kD + d] = 0.0;
 }
 
 __global__ void fit_output_kernel(const double* colscale, float* colscale_out) {
@@ -541,9 +566,13 @@ size_t mine_mma_smem(int P, int KIND) {
 // adds them into float64 accumulators held in registers (lane l: channels E*l .. E*l + E - 1
 // of the slice), then arrives on the stage's "empty" mbarrier.  A stage is refilled once all
 // 16 warps are done with it, so fast warps run ahead instead of waiting at a block barrier.
-// Each CTA adds its totals to global memory once at the end.  float64 sums of fp16 / bf16
-// values are exact, so the order of the additions does not change them (fp32 rows: up to
-// rounding).  Every wait is bounded.
+// float64 sums of fp16 / bf16 values are exact, so the order of the additions does not change
+// them and each CTA adds its totals to global memory with atomics.  float64 sums of fp32 rows
+// (the pre-transformed input) round, so for them every step has a fixed order: the rows of a
+// cluster are listed in token order (ranks from __match_any_sync, not from atomics), and each
+// CTA writes its totals to its own slot of `part`, which the update adds in CTA order.  Every
+// wait is bounded; on expiry KVQ_DEV_TIMEOUT goes to `status`, and the producer waits
+// (bounded) for the copies it issued before the CTA exits.
 constexpr int kAccWarps = 16;
 constexpr int kAccT = 128;  // tokens per tile
 constexpr uint32_t kAccSpinLimit = 1u << 24;
@@ -627,7 +656,9 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
                                                                             Src s, int P,
                                                                             const int32_t* __restrict__ assign,
                                                                             double* __restrict__ sums,
-                                                                            uint32_t* __restrict__ cnt) {
+                                                                            uint32_t* __restrict__ cnt,
+                                                                            double* __restrict__ part,
+                                                                            int32_t* __restrict__ status) {
   constexpr int CW = 32 * E, RB = CW * ES;  // channels and bytes of a staged row
   constexpr int kStages = accum_stages<CPW, RB, ES>();
   constexpr int kStageBytes = kAccT * RB;
@@ -643,7 +674,13 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
   const int64_t per = (ntiles + gridDim.x - 1) / gridDim.x;
   const int64_t k0 = (int64_t)blockIdx.x * per, k1 = min(ntiles, k0 + per);
-  if (k0 >= k1) return;
+  if (k0 >= k1) {
+    if constexpr (ES == 4) {  // no tiles: this CTA's partial slot is zero
+      double* gp = part + ((size_t)prob * gridDim.x + blockIdx.x) * P * kD;
+      for (int i = threadIdx.x; i < P * CW; i += blockDim.x) gp[(size_t)(i / CW) * kD + slice * CW + i % CW] = 0.0;
+    }
+    return;
+  }
   const int nt = (int)(k1 - k0);
   const int set = prob / s.heads, h = prob % s.heads;
   const int32_t* a = assign + (size_t)prob * s.n;
@@ -658,11 +695,15 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
 
   if (warp == kAccWarps) {
     // ---- producer: rows of tile k into stage k % kStages once every consumer left it
+    int last = -1;  // newest tile whose copy was issued
     for (int k = 0; k < nt; ++k) {
       const int st = k % kStages;
       bool ok = true;
       if (k >= kStages) ok = mb_wait(&empty[st], (uint32_t)(((k / kStages) - 1) & 1));
-      if (!__all_sync(kFull, ok)) break;  // consumers time out on the full barrier in turn
+      if (!__all_sync(kFull, ok)) {  // consumers time out on the full barrier in turn
+        if (lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
+        break;
+      }
       const int tb = (int)((k0 + k) * kAccT);
       // the tile's rows grouped by cluster (counting sort): offs[st][j] .. offs[st][j + 1] of
       // lists[st] are the rows of cluster j
@@ -674,8 +715,21 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
       }
       for (int i = lane; i < P; i += 32) counts[i] = 0;
       __syncwarp();
+      if constexpr (ES == 4) {
+        // fixed order: a cluster's rows in token order (rank among equal lanes, then later q)
 #pragma unroll
-      for (int q = 0; q < kAccT / 32; ++q) pos[q] = aj[q] >= 0 ? atomicAdd(&counts[aj[q]], 1) : -1;
+        for (int q = 0; q < kAccT / 32; ++q) {
+          const unsigned peers = __match_any_sync(kFull, aj[q]);
+          const int leader = __ffs(peers) - 1;
+          int base = 0;
+          if (aj[q] >= 0 && lane == leader) base = atomicAdd(&counts[aj[q]], __popc(peers));
+          base = __shfl_sync(kFull, base, leader);
+          pos[q] = aj[q] >= 0 ? base + __popc(peers & ((1u << lane) - 1u)) : -1;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < kAccT / 32; ++q) pos[q] = aj[q] >= 0 ? atomicAdd(&counts[aj[q]], 1) : -1;
+      }
       __syncwarp();
       {
         // exclusive scan: lane l owns clusters [l * per, (l + 1) * per)
@@ -705,7 +759,16 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
         if constexpr (ES == 2) tma_load_4d(dst, &amap, slice * CW, h, tb, set, &full[st]);
         else tma_load_3d(dst, &amap, slice * CW, tb, prob, &full[st]);
       }
+      last = k;
       __syncwarp();
+    }
+    // drain: a stage is refilled only after every consumer left it, so at most the newest copy of
+    // each stage can still be in flight; wait (bounded) for those before the CTA may exit
+    if (lane == 0) {
+      for (int st = 0; st < kStages && st <= last; ++st) {
+        const int k = st + ((last - st) / kStages) * kStages;
+        if (!mb_wait(&full[st], (uint32_t)((k / kStages) & 1))) set_status(status, KVQ_DEV_TIMEOUT);
+      }
     }
     return;
   }
@@ -723,7 +786,10 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
   for (int k = 0; k < nt; ++k) {
     const int st = k % kStages;
     const bool ok = mb_wait(&full[st], (uint32_t)((k / kStages) & 1));
-    if (!__all_sync(kFull, ok)) break;
+    if (!__all_sync(kFull, ok)) {
+      if (lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
+      break;
+    }
     const uint8_t* stg = smraw + (size_t)st * kStageBytes;
     const int32_t* o = offs + st * kOff;
     const int32_t* lst = lists + st * kAccT;
@@ -765,15 +831,18 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
     if (lane == 0) mb_arrive(&empty[st]);
   }
 
-  double* gs = sums + (size_t)prob * P * kD + slice * CW + lane * E;
   const double unscale = f16 ? 0x1p1008 : 0x1p896;
+  double* gs = (ES == 4 ? part + ((size_t)prob * gridDim.x + blockIdx.x) * P * kD : sums + (size_t)prob * P * kD) +
+               slice * CW + lane * E;
 #pragma unroll
   for (int c = 0; c < CPW; ++c) {
     const int j = warp + kAccWarps * c;
     if (j >= P) break;
 #pragma unroll
-    for (int e = 0; e < E; ++e)
-      if (acc[c][e] != 0.0) atomicAdd(gs + (size_t)j * kD + e, acc[c][e] * unscale);
+    for (int e = 0; e < E; ++e) {
+      if constexpr (ES == 4) gs[(size_t)j * kD + e] = acc[c][e] * unscale;  // this CTA's slot, zeros included
+      else if (acc[c][e] != 0.0) atomicAdd(gs + (size_t)j * kD + e, acc[c][e] * unscale);
+    }
     if (slice == 0 && lane == 0 && members[c]) atomicAdd(cnt + (size_t)prob * P + j, members[c]);
   }
 }
@@ -787,7 +856,7 @@ constexpr size_t accum_smem() {
 
 template <int CPW, int E, int ES>
 cudaError_t launch_accum_t(const CUtensorMap& amap, const Src& s, int P, int NP, int sms, const int32_t* assign,
-                           double* sums, uint32_t* cnt, cudaStream_t st) {
+                           double* sums, uint32_t* cnt, double* part, int32_t* status, cudaStream_t st) {
   constexpr size_t smem = accum_smem<CPW, E, ES>();
   cudaError_t e = cudaFuncSetAttribute(mine_accum_kernel<CPW, E, ES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -795,9 +864,11 @@ cudaError_t launch_accum_t(const CUtensorMap& amap, const Src& s, int P, int NP,
   const int slices = 4 / E;
   const int64_t ntiles = (s.n + kAccT - 1) / kAccT;
   const int64_t want = std::max<int64_t>(1, accum_ctas_per_sm<CPW, ES>() * sms / std::max(1, slices * NP));
-  const unsigned chunks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, want));
+  // fp32 rows: the CTA count fixes the partial slots of the workspace
+  const unsigned chunks = ES == 4 ? (unsigned)accum_f32_chunks(s.n, NP, P)
+                                  : (unsigned)std::max<int64_t>(1, std::min<int64_t>(ntiles, want));
   mine_accum_kernel<CPW, E, ES><<<dim3(chunks, slices, NP), (kAccWarps + 1) * 32, smem, st>>>(amap, s, P, assign,
-                                                                                              sums, cnt);
+                                                                                              sums, cnt, part, status);
   return cudaGetLastError();
 }
 
@@ -806,16 +877,16 @@ cudaError_t launch_accum_t(const CUtensorMap& amap, const Src& s, int P, int NP,
 int accum_slice_channels(int P) { return P <= 4 * kAccWarps ? 128 : (P <= 8 * kAccWarps ? 64 : 32); }
 
 cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, int sms, const int32_t* assign,
-                         double* sums, uint32_t* cnt, cudaStream_t st) {
+                         double* sums, uint32_t* cnt, double* part, int32_t* status, cudaStream_t st) {
   const bool f32 = s.y != nullptr;
   if (P <= 4 * kAccWarps)
-    return f32 ? launch_accum_t<4, 4, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
-               : launch_accum_t<4, 4, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
+    return f32 ? launch_accum_t<4, 4, 4>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st)
+               : launch_accum_t<4, 4, 2>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st);
   if (P <= 8 * kAccWarps)
-    return f32 ? launch_accum_t<8, 2, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
-               : launch_accum_t<8, 2, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
-  return f32 ? launch_accum_t<16, 1, 4>(amap, s, P, NP, sms, assign, sums, cnt, st)
-             : launch_accum_t<16, 1, 2>(amap, s, P, NP, sms, assign, sums, cnt, st);
+    return f32 ? launch_accum_t<8, 2, 4>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st)
+               : launch_accum_t<8, 2, 2>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st);
+  return f32 ? launch_accum_t<16, 1, 4>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st)
+             : launch_accum_t<16, 1, 2>(amap, s, P, NP, sms, assign, sums, cnt, part, status, st);
 }
 
 // ---- tcgen05 assignment (bf16 input, P <= 128) ------------------------------------------
@@ -925,7 +996,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
                                                                       int32_t* __restrict__ assign,
                                                                       float* __restrict__ xsq_cache, int first,
                                                                       int32_t* __restrict__ amb,
-                                                                      int32_t* __restrict__ amb_cnt, int nst) {
+                                                                      int32_t* __restrict__ amb_cnt, int nst,
+                                                                      int32_t* __restrict__ status) {
   const int prob = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Pn = (P + 15) & ~15, N = 2 * Pn;
@@ -1009,14 +1081,25 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     // ---- producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      int last = -1;  // newest tile whose copies were issued
       for (int k = 0; k < nt; ++k) {
         const int st = k % nst;
-        if (k >= nst && !tc_wait(&sfree[st], (uint32_t)(((k / nst) - 1) & 1))) break;
+        if (k >= nst && !tc_wait(&sfree[st], (uint32_t)(((k / nst) - 1) & 1))) {
+          set_status(status, KVQ_DEV_TIMEOUT);
+          break;
+        }
         uint8_t* dst = At + (size_t)st * kTcTileBytes;
         mb_expect_tx(&full[st], (uint32_t)kTcTileBytes);
         const int t0 = (int)tile_t0(k);
         tma_load_4d(dst, &xmap, 0, h, t0, set, &full[st]);
         tma_load_4d(dst + kTcTileBytes / 2, &xmap, 64, h, t0, set, &full[st]);
+        last = k;
+      }
+      // drain: a stage is reloaded only after the MMAs of its previous tile committed, so at most
+      // the newest copy of each stage can still be in flight; wait (bounded) for those
+      for (int st = 0; st < nst && st <= last; ++st) {
+        const int k = st + ((last - st) / nst) * nst;
+        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1))) set_status(status, KVQ_DEV_TIMEOUT);
       }
     }
   } else if (warp == 1) {
@@ -1024,10 +1107,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     if (lane == 0) {
       const uint32_t idesc = umma_idesc(kTcM, N);
       const uint32_t b0 = su32(Bt);
+      int last = -1;  // newest tile whose MMAs were committed
       for (int k = 0; k < nt; ++k) {
         const int st = k % nst, buf = k & 1;
-        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1))) break;
-        if (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1))) break;
+        if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1)) ||
+            (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1)))) {
+          set_status(status, KVQ_DEV_TIMEOUT);
+          break;
+        }
         tc_fence_after();
         const uint32_t a0 = su32(At + (size_t)st * kTcTileBytes);
         const uint32_t d = tbase + (uint32_t)buf * buf_cols;
@@ -1037,7 +1124,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
                     umma_desc_sw128(b0 + (ks >> 2) * half_b + (ks & 3) * 32), idesc, ks > 0);
         umma_commit(&tfull[buf]);
         umma_commit(&sfree[st]);
+        last = k;
       }
+      // drain: a commit tracks every tcgen05 operation this thread issued before it, so the
+      // newest tile's commit landing means no MMA still writes TMEM or reads shared memory
+      if (last >= 0 && !tc_wait(&tfull[last & 1], (uint32_t)((last >> 1) & 1))) set_status(status, KVQ_DEV_TIMEOUT);
     }
   } else {
     // ---- epilogue warps: warpgroup g takes tiles k with k % 2 == g, i.e. TMEM buffer g, each
@@ -1052,7 +1143,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
       const bool valid = i < s.n;
       float xsq = 0.f;
       if (!first && valid) xsq = xsq_cache[(size_t)prob * s.n + i];
-      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) break;
+      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) {
+        if (lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
+        break;
+      }
       tc_fence_after();
       float hv[8], mv[8], hn[8], mn_[8];
       tmem_ld8_issue(taddr, hv);
@@ -1253,12 +1347,22 @@ size_t mine_tc_smem(int P) {
   return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + Pn * 4 + 16 + (2 * nst + 4) * 8 + 16 + 1024;
 }
 
-__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt, int32_t* amb_cnt) {
+// Centroid = fl32(float64 sum / count); an empty cluster keeps its pattern.  With `part` (fp32
+// rows) the sum is the CTAs' partials added in CTA order.
+__global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt, int32_t* amb_cnt,
+                                   const double* part, int chunks) {
   const int prob = blockIdx.y, j = blockIdx.x, d = threadIdx.x;
   if (amb_cnt && j == 0 && d == 0) amb_cnt[prob] = 0;  // the next iteration's list starts empty
   const size_t pj = (size_t)prob * P + j;
   uint32_t c = cnt[pj];
-  if (c > 0) M[pj * kD + d] = (float)(sums[pj * kD + d] / (double)c);
+  double sum;
+  if (part) {
+    sum = 0.0;
+    for (int q = 0; q < chunks; ++q) sum += part[(((size_t)prob * chunks + q) * P + j) * kD + d];
+  } else {
+    sum = sums[pj * kD + d];
+  }
+  if (c > 0) M[pj * kD + d] = (float)(sum / (double)c);
   sums[pj * kD + d] = 0.0;
   __syncthreads();
   if (d == 0) cnt[pj] = 0;
@@ -1267,21 +1371,22 @@ __global__ void mine_update_kernel(int P, float* M, double* sums, uint32_t* cnt,
 }  // namespace
 
 size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
-  size_t NP = (size_t)sets * heads;
-  size_t b = align256(NP * P * kD * sizeof(double)) + align256(NP * P * sizeof(uint32_t)) +
-             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * (size_t)n * sizeof(float)) +
-             align256(NP * (size_t)n * sizeof(int32_t)) + align256(NP * sizeof(int32_t));
+  const int NP = sets * heads;
+  size_t b = 256 + align256((size_t)NP * P * kD * sizeof(double)) + align256((size_t)NP * P * sizeof(uint32_t)) +
+             align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * (size_t)n * sizeof(float)) +
+             align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * sizeof(int32_t));
   if (transform)
-    b += align256(NP * n * kD * sizeof(float)) + align256(NP * n * kD * sizeof(double)) +
-         4 * align256(NP * kD * sizeof(double));
+    b += align256((size_t)NP * n * kD * sizeof(float)) + align256((size_t)NP * n * kD * sizeof(double)) +
+         align256((size_t)NP * fit_chunks(n) * kD * sizeof(double)) + 4 * align256((size_t)NP * kD * sizeof(double)) +
+         align256((size_t)NP * accum_f32_chunks(n, NP, P) * P * kD * sizeof(double));
   return b + 256;
 }
 
 // Tiled TMA tensor maps (no swizzle; loads past the end read as zeros).  cuTensorMapEncodeTiled
 // comes from the driver through the runtime's entry-point query.
-static cudaError_t encode_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
-                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
-                              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+cudaError_t encode_tiled_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                             const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                             CUtensorMapSwizzle swz) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -1306,7 +1411,7 @@ static cudaError_t make_x_map(const MineArgs& a, CUtensorMap* map, int box_ch,
   const cuuint64_t strides[3] = {(cuuint64_t)a.head_stride * 2, (cuuint64_t)a.tok_stride * 2,
                                  (cuuint64_t)std::max<int64_t>(a.set_stride, 8) * 2};
   const cuuint32_t box[4] = {(cuuint32_t)box_ch, 1, 128, 1};
-  return encode_map(map, a.dtype == KVQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+  return encode_tiled_map(map, a.dtype == KVQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                     a.x, dims, strides, box, swz);
 }
 
@@ -1316,7 +1421,7 @@ static cudaError_t make_y_map(const float* y, int64_t n, int NP, CUtensorMap* ma
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)NP};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 4, (cuuint64_t)n * kD * 4};
   const cuuint32_t box[3] = {(cuuint32_t)box_ch, 128, 1};
-  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y, dims, strides, box);
+  return encode_tiled_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -1326,17 +1431,18 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   Src s{(const uint16_t*)a.x, a.dtype, a.n, a.tok_stride, a.head_stride, a.set_stride, a.heads, nullptr};
   cudaError_t e;
   const dim3 rows_grid((unsigned)((a.n + 7) / 8), NP);
-  const unsigned chunks = (unsigned)((a.n + kReduceChunk - 1) / kReduceChunk);
+  const unsigned chunks = (unsigned)fit_chunks(a.n);
+  if ((e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
 
   if (a.transform) {
     fit_prep_kernel<<<rows_grid, 256, 0, st>>>(s, w.v64, w.colscale);
-    cudaMemsetAsync(w.colsum, 0, (size_t)NP * kD * sizeof(double), st);
-    cudaMemsetAsync(w.colsq, 0, (size_t)NP * kD * sizeof(double), st);
     for (int p = 0; p < kFitPasses; ++p) {
       fit_row_kernel<<<rows_grid, 256, 0, st>>>(a.n, w.v64, p == 0 ? nullptr : w.coldiv);
-      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colsq, 0);
-      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colsq, 1);
-      fit_colfinish_kernel<<<NP, kD, 0, st>>>(a.n, w.colsum, w.colsq, w.colscale, w.coldiv);
+      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colpart, 0);
+      fit_colreduce_kernel<<<NP, kD, 0, st>>>((int)chunks, w.colpart, w.colsum);
+      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colpart, 1);
+      fit_colreduce_kernel<<<NP, kD, 0, st>>>((int)chunks, w.colpart, w.colsq);
+      fit_colfinish_kernel<<<NP, kD, 0, st>>>(a.n, w.colsq, w.colscale, w.coldiv);
     }
     fit_output_kernel<<<NP, kD, 0, st>>>(w.colscale, a.colscale);
     apply_kernel<<<rows_grid, 256, 0, st>>>(s, a.colscale, w.y);
@@ -1345,9 +1451,10 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   }
 
   mine_init_kernel<<<dim3(a.P, NP), kD, 0, st>>>(s, a.P, a.patterns);
-  cudaMemsetAsync(w.amb_cnt, 0, (size_t)NP * sizeof(int32_t), st);
-  cudaMemsetAsync(w.sums, 0, (size_t)NP * a.P * kD * sizeof(double), st);
-  cudaMemsetAsync(w.cnt, 0, (size_t)NP * a.P * sizeof(uint32_t), st);
+  if ((e = cudaMemsetAsync(w.amb_cnt, 0, (size_t)NP * sizeof(int32_t), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(w.sums, 0, (size_t)NP * a.P * kD * sizeof(double), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(w.cnt, 0, (size_t)NP * a.P * sizeof(uint32_t), st)) != cudaSuccess)
+    return e;
   size_t smem_assign = (size_t)a.P * kD * sizeof(float);
   if ((e = cudaFuncSetAttribute(mine_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_assign)) != cudaSuccess)
@@ -1393,7 +1500,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     const dim3 ag(mma_ctas, NP);
     if (use_tc) {
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
-          xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P));
+          xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P), w.status);
       mine_fixup_kernel<<<dim3((unsigned)std::max(1, 4 * sms / NP), NP), kFixWarps * 32, fix_smem, st>>>(
           s, a.P, a.patterns, w.amb, w.amb_cnt, w.assign);
     } else if (use_mma && KIND == 0)
@@ -1405,8 +1512,11 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
     else
       mine_assign_kernel<<<dim3((unsigned)((a.n + 127) / 128), NP), 128, smem_assign, st>>>(s, a.P, a.patterns,
                                                                                            w.assign);
-    if ((e = launch_accum(amap, s, a.P, NP, sms, w.assign, w.sums, w.cnt, st)) != cudaSuccess) return e;
-    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt, use_tc ? w.amb_cnt : nullptr);
+    if ((e = launch_accum(amap, s, a.P, NP, sms, w.assign, w.sums, w.cnt, w.accpart, w.status, st)) != cudaSuccess)
+      return e;
+    mine_update_kernel<<<dim3(a.P, NP), kD, 0, st>>>(a.P, a.patterns, w.sums, w.cnt, use_tc ? w.amb_cnt : nullptr,
+                                                     a.transform ? w.accpart : nullptr,
+                                                     a.transform ? accum_f32_chunks(a.n, NP, a.P) : 0);
   }
   return cudaGetLastError();
 }

@@ -28,7 +28,13 @@
  *     the offending sequence is left unchanged.  kvq_read_status() fetches it.
  *   - Supported: head_dim 128, group 32 (tokens per page = 32), bits 2 or 4,
  *     1 <= num_patterns <= 255, fp16 or bf16 inputs, query heads a multiple of the
- *     KV heads.  Other values return KVQ_ERR_UNSUPPORTED.
+ *     KV heads.  Other values return KVQ_ERR_UNSUPPORTED.  At most 65535 sequences and
+ *     65535 KV heads per cache (launch-grid limits; more returns KVQ_ERR_CAPACITY).
+ *   - Every device-side wait is bounded (a counted mbarrier.try_wait loop).  For tests of
+ *     this failure path only, the environment variable KVQ_TEST_WAIT_LIMIT (read once per
+ *     process) replaces the iteration limit of decode attention's page-copy waits; 0 makes
+ *     every such wait expire at once.  The kernel then flags KVQ_DEV_TIMEOUT and still waits,
+ *     under the normal limit, for the copies it issued before it exits.
  *
  * Cache layout in HBM
  *   A page holds 32 consecutive tokens of one sequence for every KV head.  Page p
@@ -87,6 +93,9 @@
  *   - Mining: Lloyd k-means, strided initialisation M_j = x[floor(j*n/P)], float64
  *     squared distances (lowest index on ties), centroid = fl32(float64 mean),
  *     empty clusters keep their pattern.
+ *   - V adaptive threshold (cache->v_rho > 0): with v the (pre-transformed) V vector and
+ *     M* its nearest pattern, R_flat = d_mm(v, M*), R_raw = fl32(max v - min v); the
+ *     pattern is used iff R_flat <= fl32(v_rho * R_raw), else index 255 and R = v.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -142,7 +151,10 @@ typedef struct kvq_cache {
   int32_t num_pages;          /* pages in page_pool */
   int32_t dtype;              /* kvq_dtype of K/V/q inputs and of k_tail */
   int32_t transform;          /* kvq_transform */
-  int32_t reserved;           /* must be 0 */
+  float v_rho;                /* V adaptive threshold rho* ([PKV] Section 3.3, Eq. 7-10): a V vector
+                                 keeps its pattern iff d_mm(v, M*) <= fl32(v_rho * (max v - min v)),
+                                 else it is quantized raw and stores index 255.  0 = off (always use
+                                 the pattern).  kvq_v_rho_star() gives the value for (d, alpha). */
   void* page_pool;            /* num_pages * kvq_page_bytes() bytes, 256-byte aligned */
   const int32_t* page_table;  /* [num_seqs][max_pages_per_seq] physical page ids */
   int32_t* seq_len;           /* [num_seqs] tokens held per sequence (updated by append) */
@@ -154,6 +166,12 @@ typedef struct kvq_cache {
   const float* v_colscale;    /* [num_sets][num_kv_heads][128] fp32; transform only, else NULL */
   int32_t* status;            /* one int32, device-side error bits (KVQ_DEV_*); caller zeroes it */
 } kvq_cache;
+
+/* rho*(d, alpha) of [PKV] Eq. 10 rounded to fp32: the root in (0, 1) of
+ * 1 - rho^2 = 2 z_{1-alpha} / sqrt(5 d) * sqrt(1 + rho^4) (closed form of the quadratic in
+ * rho^2), z the standard normal quantile.  Host only; 0 for alpha <= 0 (threshold off) or
+ * arguments without a root (d < 1, alpha >= 0.5). */
+KVQ_API float kvq_v_rho_star(int32_t head_dim, double alpha);
 
 /* Bytes of one page (all KV heads) and of one KV head's sub-block.  Host only; 0 if unsupported. */
 KVQ_API size_t kvq_page_bytes(const kvq_cache* cache);
@@ -175,7 +193,11 @@ KVQ_API size_t kvq_subblock_bytes(int32_t bits, int32_t transform);
  *   assign_out    [num_sets][num_kv_heads][n] int32, optional (NULL): the Euclidean
  *                 assignment of the last iteration (made against the patterns that
  *                 iteration started from)
- * Requires n >= P.  Workspace: kvq_mine_workspace_bytes().
+ * Requires n >= P and num_sets * num_kv_heads <= 65535 (else KVQ_ERR_CAPACITY).
+ * Workspace: kvq_mine_workspace_bytes(), 256-byte aligned.  Its first 4 bytes are the call's
+ * device status word: the call zeroes it when it starts, and a mining kernel whose bounded
+ * wait expired ORs KVQ_DEV_TIMEOUT into it (that call's patterns are then unreliable);
+ * kvq_mine_read_status() fetches it.
  */
 KVQ_API size_t kvq_mine_workspace_bytes(int64_t n, int32_t num_sets, int32_t num_kv_heads, int32_t P,
                                 int32_t transform);
@@ -183,6 +205,10 @@ KVQ_API kvq_status kvq_mine_patterns(const void* x, int32_t dtype, int64_t n, in
                              int64_t tok_stride, int64_t head_stride, int64_t set_stride, int32_t P,
                              int32_t iters, int32_t transform, float* patterns_out, float* colscale_out,
                              int32_t* assign_out, void* ws, size_t ws_bytes, kvq_stream_t stream);
+
+/* Synchronise `stream` and copy the status word of the mining call that used workspace `ws`
+ * (device pointer) to *bits_out (host).  Returns KVQ_ERR_DEVICE if any bit is set, else KVQ_OK. */
+KVQ_API kvq_status kvq_mine_read_status(const void* ws, int32_t* bits_out, kvq_stream_t stream);
 
 /*
  * kvq_quantize_append -- append n_new tokens to every sequence ([PKV] Section 3.2:

@@ -107,6 +107,7 @@ class Workload:
     bits: int = 2
     transform: int = 0  # 0 = pattern residual only, 1 = Hadamard + dual-axis variance normalisation
     steps: int = 0      # decode steps after the prefill (long chain-of-thought workload)
+    v_alpha: float = 0.05  # significance level of the V adaptive threshold (0 = threshold off)
 
     def params(self) -> _Params:
         return _Params(self.seed, self.B, self.S, self.Hkv, self.D, self.nck, self.ncv, self.sigma_k,

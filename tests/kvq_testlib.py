@@ -33,10 +33,16 @@ def oracle_patterns(w: synth.Workload, Kf: np.ndarray, Vf: np.ndarray):
     return MK, MV, None, None
 
 
+def gpu_v_rho(w: synth.Workload) -> float:
+    """The library's fp32 rho* for the workload's V threshold (0 = off)."""
+    import bit_kv_cache_26_b200 as kvq
+    return kvq.kvq_v_rho_star(D, w.v_alpha)
+
+
 def make_cache(w: synth.Workload, MK, MV, cK, cV, max_tokens=None, page_order=None):
     import bit_kv_cache_26_b200 as kvq
     cache = kvq.PagedKVCache(w.B, w.Hkv, max_tokens or max(w.S, 1), w.bits, w.P, dtype=w.dtype,
-                             transform=w.transform, page_order=page_order)
+                             transform=w.transform, page_order=page_order, v_rho=gpu_v_rho(w))
     cache.k_patterns.copy_(torch.from_numpy(MK[None]))
     cache.v_patterns.copy_(torch.from_numpy(MV[None]))
     if w.transform:
@@ -48,7 +54,7 @@ def make_cache(w: synth.Workload, MK, MV, cK, cV, max_tokens=None, page_order=No
 def encode_unit(w, Kf, Vf, b, h, MK, MV, cK, cV, N=None):
     N = w.S if N is None else N
     return oracle.encode(Kf[b, :N, h], Vf[b, :N, h], w.bits, MK[h], MV[h],
-                         None if cK is None else cK[h], None if cV is None else cV[h])
+                         None if cK is None else cK[h], None if cV is None else cV[h], v_rho=oracle.v_rho(w.v_alpha))
 
 
 def check_pages(cache, w, e: oracle.Encoded, b: int, h: int):

@@ -53,7 +53,8 @@ def _cache(**kw):
 
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 64, 2), ("group", 16, 2), ("bits", 3, 2), ("num_patterns", 0, 2), ("num_patterns", 256, 2),
-    ("dtype", 7, 2), ("transform", 5, 2), ("reserved", 1, 1),
+    ("dtype", 7, 2), ("transform", 5, 2), ("v_rho", -1.0, 1), ("v_rho", float("nan"), 1),
+    ("v_rho", float("inf"), 1),
 ])
 def test_append_rejects_bad_cache_on_host(field, value, status):
     import bit_kv_cache_26_b200 as kvq
@@ -104,3 +105,16 @@ def test_static_scratch_size_matches_header():
     import bit_kv_cache_26_b200 as kvq
     m = re.search(r"#define\s+KVQ_DECODE_STATIC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", open(HEADER).read())
     assert m and int(m.group(1)) << int(m.group(2)) == kvq.KVQ_DECODE_STATIC_SCRATCH_BYTES
+
+
+def test_library_rho_star_equals_the_oracles():
+    # The library's closed form and the oracle's bisection of Eq. 10 give the same fp32 threshold
+    # (the two sides must take the keep-the-pattern decision in the same precision).
+    import numpy as np
+
+    import bit_kv_cache_26_b200 as kvq
+    import oracle
+    for d in (64, 96, 128, 256):
+        for a in (0.2, 0.1, 0.05, 0.01, 0.001):
+            assert kvq.kvq_v_rho_star(d, a) == np.float32(oracle.rho_star(d, a)), (d, a)
+    assert kvq.kvq_v_rho_star(128, 0.0) == 0.0 and oracle.v_rho(0.0) == 0.0

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from kvq_testlib import D, attention_ok, check_pages, check_tail, to_torch
+from kvq_testlib import D, attention_ok, check_pages, check_tail, gpu_v_rho, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -53,7 +53,8 @@ def _check_mining_head(w, k, v, h, MK, MV, cK, cV):
 def _check_unit(cache, w, k, v, b, h, N, MK, MV, cK, cV, q=None, out=None):
     Kf = synth.to_float(k[b, :N, h], w.dtype)
     Vf = synth.to_float(v[b, :N, h], w.dtype)
-    e = oracle.encode(Kf, Vf, w.bits, MK[h], MV[h], None if cK is None else cK[h], None if cV is None else cV[h])
+    e = oracle.encode(Kf, Vf, w.bits, MK[h], MV[h], None if cK is None else cK[h], None if cV is None else cV[h],
+                      v_rho=oracle.v_rho(w.v_alpha))
     check_pages(cache, w, e, b, h)
     check_tail(cache, w, k, b, h, N)
     if q is not None:
@@ -80,7 +81,7 @@ def test_full_size_prefill_and_decode(name):
     w = FULL[name]
     k, v = synth.gen_kv(w)
     kt, vt = to_torch(k, w.dtype), to_torch(v, w.dtype)
-    cache = kvq.PagedKVCache(w.B, w.Hkv, w.S, w.bits, w.P, dtype=w.dtype, transform=w.transform)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, w.S, w.bits, w.P, dtype=w.dtype, transform=w.transform, v_rho=gpu_v_rho(w))
     _gpu_mine(cache, w, kt, vt)
     cache.append(kt, vt)
     q = synth.gen_q(w)
@@ -103,7 +104,7 @@ def test_long_cot_decode_loop():
     total = w.S + w.steps
     k, v = synth.gen_kv(w.with_(S=total))
     kt, vt = to_torch(k, w.dtype), to_torch(v, w.dtype)
-    cache = kvq.PagedKVCache(w.B, w.Hkv, total, w.bits, w.P, dtype=w.dtype, transform=w.transform)
+    cache = kvq.PagedKVCache(w.B, w.Hkv, total, w.bits, w.P, dtype=w.dtype, transform=w.transform, v_rho=gpu_v_rho(w))
     _gpu_mine(cache, w, kt[:, :w.S].contiguous(), vt[:, :w.S].contiguous())
     cache.append(kt[:, :w.S].contiguous(), vt[:, :w.S].contiguous())
     MK, MV, cK, cV = _patterns(cache, w)

@@ -33,7 +33,25 @@ CASES = {
     "gqa4_p100": (W["llama3_8b_32k"].with_(B=2, S=1000, Hkv=2, Hq=8, P=100), [1000]),
     # the largest pattern count the u8 indices allow: float64 assignment, 16 clusters per warp
     "p255": (W["llama3_8b_32k"].with_(B=1, S=600, Hkv=1, Hq=4, P=255), [300, 300]),
+    # V adaptive threshold: every fourth V vector replaced by one far from every pattern (planted
+    # rejections, index 255, quantized raw), with and without the pre-transform, at 2 and 4 bits
+    "v_threshold_planted": (W["llama3_8b_32k"].with_(B=2, S=700, Hkv=2, Hq=8, P=32), [350, 350]),
+    "v_threshold_planted_4bit_tx": (W["qwen25_7b_128k"].with_(B=1, S=500, Hkv=2, Hq=14, P=16, bits=4, transform=1),
+                                    [500]),
+    # the threshold off: every V vector keeps its nearest pattern
+    "v_threshold_off": (W["llama3_8b_32k"].with_(B=2, S=300, Hkv=2, Hq=8, P=16, v_alpha=0.0), [300]),
 }
+PLANT_V = {"v_threshold_planted", "v_threshold_planted_4bit_tx"}
+
+
+def plant_far_v(v: np.ndarray, dtype: int, seed: int) -> np.ndarray:
+    """Every fourth token's V vectors replaced by N(0, 3^2) values (bit patterns of the dtype)."""
+    rng = np.random.default_rng(seed)
+    v = v.copy()
+    x = (rng.standard_normal(v[:, ::4].shape) * 3).astype(np.float32)
+    v[:, ::4] = (x.view(np.uint32) >> 16).astype(np.uint16) if dtype == synth.BF16 else \
+        x.astype(np.float16).view(np.uint16)
+    return v
 
 
 @pytest.fixture(scope="module", params=list(CASES))
@@ -41,6 +59,8 @@ def case(request):
     w, chunks = CASES[request.param]
     assert sum(chunks) == w.S
     k, v = synth.gen_kv(w)
+    if request.param in PLANT_V:
+        v = plant_far_v(v, w.dtype, seed=w.seed)
     Kf, Vf = synth.to_float(k, w.dtype), synth.to_float(v, w.dtype)
     MK, MV, cK, cV = oracle_patterns(w, Kf, Vf) if w.B * w.S >= w.P else (None,) * 4
     cache = make_cache(w, MK, MV, cK, cV)
@@ -65,6 +85,22 @@ def test_pages_and_tail_bit_exact(case):
             e = encode_unit(w, case["Kf"], case["Vf"], b, h, case["MK"], case["MV"], case["cK"], case["cV"])
             check_pages(case["cache"], w, e, b, h)
             check_tail(case["cache"], w, case["k"], b, h, w.S)
+
+
+def test_v_threshold_rejections(case):
+    # the oracle's encoding (which the page bytes match bit for bit) rejects the planted vectors
+    w = case["w"]
+    if w.B * w.S < w.P:
+        pytest.skip("no patterns")
+    raw = np.concatenate([encode_unit(w, case["Kf"], case["Vf"], b, h, case["MK"], case["MV"], case["cK"],
+                                      case["cV"]).vidx == 255 for b in range(w.B) for h in range(w.Hkv)])
+    if case["name"] in PLANT_V:
+        planted = np.zeros(w.S, bool)
+        planted[::4] = True
+        planted = np.tile(planted, w.B * w.Hkv)
+        assert raw[planted].mean() > 0.9 and raw[~planted].mean() < 0.25, (raw[planted].mean(), raw[~planted].mean())
+    elif w.v_alpha == 0:
+        assert not raw.any()
 
 
 def test_dequantize(case):
