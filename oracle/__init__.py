@@ -68,6 +68,9 @@ def _load():
             "kvqo_normal_upper_quantile": (f64, [f64]),
             "kvqo_rho_star": (f64, [i32, f64]),
             "kvqo_range": (ctypes.c_float, [_vp]),
+            "kvqo_chebyshev_center": (None, [_vp, i64, _vp]),
+            "kvqo_encode_stream": (ctypes.c_int, [_vp, _vp, i64, i64, i32, i32, i32, i32, _vp, _vp, _vp, _vp,
+                                                  ctypes.c_float, _vp] + [_vp] * 10),
             "kvqo_dequant": (None, [i64, _vp, _vp, _vp, _vp] + [_vp] * 10 + [_vp, _vp]),
             "kvqo_attention": (None, [_vp, i32, _vp, _vp, i64, f64, _vp]),
         }
@@ -267,6 +270,44 @@ def encode(K: np.ndarray, V: np.ndarray, bits: int, MK, MV, cK=None, cV=None, v_
     if rc != 0:
         raise ValueError(f"kvqo_encode rc={rc}")
     return e
+
+
+def chebyshev_center(X) -> np.ndarray:
+    """Per channel the mean of the minimum and maximum of the rows of X (PatternKV Eq. 5), fp32."""
+    X = _f32(X).reshape(-1, D)
+    M = np.zeros(D, np.float32)
+    _load().kvqo_chebyshev_center(_p(X), X.shape[0], _p(M))
+    return M
+
+
+def encode_stream(K: np.ndarray, V: np.ndarray, L0: int, bits: int, MK0, MV0, Pmax: int, G: int = 0,
+                  cK=None, cV=None, v_rho: float = 0.0):
+    """Streaming encoding with decode-time pattern insertion (PatternKV Section 3.1, Eq. 5).
+
+    Tokens [0, L0) are the prefill (the initial P0 patterns); tokens from L0 on arrive one at a
+    time, and with G > 0 every window of G tokens (aligned to multiples of G) adds the Chebyshev
+    centers of its K and V vectors to the pattern sets (up to Pmax patterns), used from the next
+    token on.  Returns (Encoded, MK [P, 128], MV [P, 128]) with the final pattern count P."""
+    K, V = _f32(K), _f32(V)
+    MK0, MV0 = _f32(MK0), _f32(MV0)
+    cK = None if cK is None else _f32(cK)
+    cV = None if cV is None else _f32(cV)
+    N, P0 = K.shape[0], MK0.shape[0]
+    MK = np.zeros((Pmax, D), np.float32)
+    MV = np.zeros((Pmax, D), np.float32)
+    MK[:P0], MV[:P0] = MK0, MV0
+    G32 = N // GROUP
+    e = Encoded(N, bits, np.zeros((G32, GROUP, D), np.uint8), np.zeros((G32, D), np.float32),
+                np.zeros((G32, D), np.float32), np.zeros(G32 * GROUP, np.uint8), np.zeros(G32 * GROUP, np.float32),
+                np.zeros((N, D), np.uint8), np.zeros((N, 4), np.float32), np.zeros((N, 4), np.float32),
+                np.zeros(N, np.uint8), np.zeros(N, np.float32))
+    P = ctypes.c_int32(0)
+    rc = _load().kvqo_encode_stream(_p(K), _p(V), N, L0, G, bits, P0, Pmax, _p(MK), _p(MV), _p(cK), _p(cV),
+                                    float(v_rho), ctypes.byref(P), _p(e.kcode), _p(e.ks), _p(e.kz), _p(e.kidx),
+                                    _p(e.krow), _p(e.vcode), _p(e.vs), _p(e.vz), _p(e.vidx), _p(e.vrow))
+    if rc != 0:
+        raise ValueError(f"kvqo_encode_stream rc={rc}")
+    return e, MK[:P.value].copy(), MV[:P.value].copy()
 
 
 def dequant(e: Encoded, MK, MV, cK=None, cV=None):

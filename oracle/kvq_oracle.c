@@ -391,6 +391,124 @@ int kvqo_encode(const float* K, const float* V, int64_t N, int32_t bits, int32_t
 }
 
 /* ------------------------------------------------------------------------- */
+/* Decode-time pattern insertion: [PKV] Section 3.1 "Decoding Stage", Eq. 5. */
+/* The Chebyshev center of a window of KV vectors, per dimension the mean of */
+/* its minimum and maximum, becomes a new pattern:                           */
+/*   M_new_d = fl32(fl32(min_i X_id + max_i X_id) * 0.5).                    */
+/* Readings: windows of G_pattern tokens aligned to multiples of G_pattern   */
+/* (the prefill length is one); the vectors are the (pre-transformed) K and  */
+/* V vectors appended after the prefill; the new K and V patterns join their */
+/* sets as index P (the sets grow together, up to a capacity, then stop) and */
+/* are used from the next token on.                                          */
+/* ------------------------------------------------------------------------- */
+
+void kvqo_chebyshev_center(const float* X, int64_t n, float* M) {
+  for (int d = 0; d < D; ++d) {
+    float mn = X[d], mx = X[d];
+    for (int64_t i = 1; i < n; ++i) {
+      float v = X[(size_t)i * D + d];
+      if (v < mn) mn = v;
+      if (v > mx) mx = v;
+    }
+    float s = mn + mx;
+    M[d] = s * 0.5f;
+  }
+}
+
+/* One V token: assign (d_mm), optional adaptive threshold, residual, 4 groups of Eq. 1. */
+static void encode_v_token(const float* x, const float* cV, const float* MV, int32_t P, int32_t bits, float v_rho,
+                           uint8_t* vcode, float* vs, float* vz, uint8_t* vidx, float* vrow, float* y_out) {
+  float y[D], R[D];
+  prep_row(x, cV, y, vrow);
+  int32_t j = kvqo_assign(y, MV, P);
+  int use = 1;
+  if (v_rho > 0.0f) {
+    float r_flat = kvqo_dmm(y, MV + (size_t)j * D);
+    float limit = v_rho * kvqo_range(y);
+    use = r_flat <= limit;
+  }
+  *vidx = use ? (uint8_t)j : (uint8_t)255;
+  for (int d = 0; d < D; ++d) R[d] = use ? y[d] - MV[(size_t)j * D + d] : y[d];
+  int32_t q[D];
+  for (int g = 0; g < 4; ++g) kvqo_quant_group(R + 32 * g, 32, 1, bits, &vs[g], &vz[g], q + 32 * g, 1);
+  for (int d = 0; d < D; ++d) vcode[d] = (uint8_t)q[d];
+  if (y_out) memcpy(y_out, y, sizeof(y));
+}
+
+/* One complete K group of 32 tokens: assign each vector, quantize per channel. */
+static void encode_k_group(const float* K32, const float* cK, const float* MK, int32_t P, int32_t bits,
+                           uint8_t* kcode, float* ks, float* kz, uint8_t* kidx, float* krow) {
+  float R[32][D];
+  for (int t = 0; t < 32; ++t) {
+    float y[D];
+    prep_row(K32 + (size_t)t * D, cK, y, &krow[t]);
+    int32_t j = kvqo_assign(y, MK, P);
+    kidx[t] = (uint8_t)j;
+    for (int d = 0; d < D; ++d) R[t][d] = y[d] - MK[(size_t)j * D + d];
+  }
+  int32_t q[32][D];
+  for (int d = 0; d < D; ++d) kvqo_quant_group(&R[0][d], 32, D, bits, &ks[d], &kz[d], &q[0][d], D);
+  for (int t = 0; t < 32; ++t)
+    for (int d = 0; d < D; ++d) kcode[(size_t)t * D + d] = (uint8_t)q[t][d];
+}
+
+/*
+ * Streaming encoding of one (sequence, KV head): tokens [0, L0) are the prefill (encoded with
+ * the first P0 patterns, as kvqo_encode does); tokens L0 .. N-1 arrive one at a time.  Token p:
+ * its V vector is encoded with the patterns present; if it completes a K group, that group's 32
+ * keys are encoded with the patterns present; then, with G > 0, it joins the window of positions
+ * [G floor(p / G), G floor(p / G) + G), and when p + 1 is a multiple of G the Chebyshev centers
+ * of the window's K and V vectors become patterns P and P + 0 of the K and V sets (if P < Pmax).
+ * MK, MV: [Pmax][128], first P0 rows given, grown in place; *P_out: patterns at the end.
+ * L0 must be a multiple of G when G > 0.  Outputs as kvqo_encode.
+ */
+int kvqo_encode_stream(const float* K, const float* V, int64_t N, int64_t L0, int32_t G, int32_t bits, int32_t P0,
+                       int32_t Pmax, float* MK, float* MV, const float* cK, const float* cV, float v_rho,
+                       int32_t* P_out, uint8_t* kcode, float* ks, float* kz, uint8_t* kidx, float* krow,
+                       uint8_t* vcode, float* vs, float* vz, uint8_t* vidx, float* vrow) {
+  if (bits != 2 && bits != 4) return -1;
+  if (P0 < 1 || Pmax < P0 || Pmax > 255 || L0 < 0 || L0 > N) return -1;
+  if (G < 0 || (G > 0 && L0 % G != 0)) return -1;
+  int32_t P = P0;
+  /* prefill: V tokens and complete K groups with the initial patterns */
+  if (kvqo_encode(K, V, L0, bits, P0, MK, MV, cK, cV, v_rho, kcode, ks, kz, kidx, krow, vcode, vs, vz, vidx,
+                  vrow) != 0)
+    return -1;
+  float* wk = (float*)malloc((size_t)(G > 0 ? G : 1) * D * sizeof(float));
+  float* wv = (float*)malloc((size_t)(G > 0 ? G : 1) * D * sizeof(float));
+  if (!wk || !wv) { free(wk); free(wv); return -2; }
+  int32_t nw = 0; /* vectors in the current window */
+  for (int64_t p = L0; p < N; ++p) {
+    float yv[D];
+    encode_v_token(V + (size_t)p * D, cV, MV, P, bits, v_rho, vcode + (size_t)p * D, vs + p * 4, vz + p * 4,
+                   vidx + p, vrow + p, yv);
+    if ((p + 1) % 32 == 0) {
+      int64_t g = p / 32;
+      encode_k_group(K + (size_t)g * 32 * D, cK, MK, P, bits, kcode + (size_t)g * 32 * D, ks + g * D, kz + g * D,
+                     kidx + g * 32, krow + g * 32);
+    }
+    if (G > 0) {
+      float r;
+      prep_row(K + (size_t)p * D, cK, wk + (size_t)nw * D, &r);
+      memcpy(wv + (size_t)nw * D, yv, sizeof(yv));
+      nw += 1;
+      if ((p + 1) % G == 0) {
+        if (P < Pmax) {
+          kvqo_chebyshev_center(wk, nw, MK + (size_t)P * D);
+          kvqo_chebyshev_center(wv, nw, MV + (size_t)P * D);
+          P += 1;
+        }
+        nw = 0;
+      }
+    }
+  }
+  free(wk);
+  free(wv);
+  *P_out = P;
+  return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Dequantization / reconstruction ([PKV] Section 3.2: fetch the pattern by  */
 /* its stored index and undo the residualisation; Eq. 1: s*Q + z), float64.  */
 /* With the pre-transform the result is mapped back: x = r * (y (.) c) H / 128.*/

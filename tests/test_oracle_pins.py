@@ -556,3 +556,65 @@ def test_v_threshold_matches_eq10_on_clustered_data():
     planted[::4] = True
     assert (e.vidx[planted] == 255).mean() > 0.9       # far from every pattern: flattening rejected
     assert (e.vidx[~planted] == 255).mean() < 0.1      # near their pattern: flattening kept
+
+
+# ---------------------------------------------------------------- decode-time pattern insertion (Eq. 5)
+
+def test_chebyshev_center_worked_example(golden):
+    g = golden("chebyshev_eq5.json")
+    X = np.stack([sparse_vec(v) for v in g["X"]])
+    assert np.array_equal(oracle.chebyshev_center(X), sparse_vec(g["center"]))
+
+
+def test_chebyshev_center_is_the_minimax_point():
+    # Per channel the midrange minimises the largest deviation of the window's values (the l-inf
+    # Chebyshev center, PatternKV Appendix C): no other point has a smaller maximum |X - M|.
+    for _ in range(50):
+        X = (rng.standard_normal((int(rng.integers(1, 40)), D)) * rng.uniform(0.1, 10)).astype(np.float32)
+        M = oracle.chebyshev_center(X).astype(np.float64)
+        X64 = X.astype(np.float64)
+        radius = np.abs(X64 - M).max(axis=0)
+        assert np.allclose(radius, (X64.max(0) - X64.min(0)) / 2, rtol=1e-6, atol=1e-6)
+        for _ in range(5):
+            Mp = M + rng.standard_normal(D) * 0.01
+            assert (np.abs(X64 - Mp).max(axis=0) >= radius - 1e-6).all()
+
+
+def test_stream_without_insertion_equals_batch_encoding():
+    # Appending one token at a time with fixed patterns gives the same encoding as one bulk call.
+    w = synth.WORKLOADS["tiny_ref_4k"]
+    K, V = _unit(w, 320 + 5)
+    MK, _, _ = oracle.mine_set(K[:256], 8)
+    MV, _, _ = oracle.mine_set(V[:256], 8)
+    rho = oracle.v_rho(0.05)
+    for L0 in (0, 100, 256):
+        e0 = oracle.encode(K, V, 2, MK, MV, v_rho=rho)
+        e1, MK1, MV1 = oracle.encode_stream(K, V, L0, 2, MK, MV, Pmax=20, G=0, v_rho=rho)
+        assert MK1.shape[0] == 8 and np.array_equal(MK1, MK)
+        for f in ("kcode", "ks", "kz", "kidx", "vcode", "vs", "vz", "vidx"):
+            assert np.array_equal(getattr(e0, f), getattr(e1, f)), (L0, f)
+
+
+def test_stream_insertion_adds_window_centers():
+    w = synth.WORKLOADS["tiny_ref_4k"]
+    K, V = _unit(w, 128 * 5 + 17)
+    L0, G = 128, 128
+    MK, _, _ = oracle.mine_set(K[:L0], 4)
+    MV, _, _ = oracle.mine_set(V[:L0], 4)
+    e, MKf, MVf = oracle.encode_stream(K, V, L0, 2, MK, MV, Pmax=6, G=G)
+    # windows [128, 256), [256, 384), ... complete at 256, 384, 512, 640: capacity 6 keeps the first two
+    assert MKf.shape[0] == 6
+    for i, w0 in enumerate((128, 256)):
+        assert np.array_equal(MKf[4 + i], ((K[w0:w0 + G].min(0) + K[w0:w0 + G].max(0)) * np.float32(0.5)))
+        assert np.array_equal(MVf[4 + i], ((V[w0:w0 + G].min(0) + V[w0:w0 + G].max(0)) * np.float32(0.5)))
+    # every token is assigned among the patterns present when it (V) or its group (K) arrived
+    for t in range(L0, e.N):
+        P_t = 4 + min(2, (t - L0) // G)
+        assert e.vidx[t] == oracle.assign(V[t], MVf[:P_t]), t
+    for grp in range(L0 // 32, e.N // 32):
+        last = 32 * grp + 31
+        P_t = 4 + min(2, max(0, last - L0) // G) if last >= L0 else 4
+        for t in range(32 * grp, 32 * grp + 32):
+            assert e.kidx[t] == oracle.assign(K[t], MKf[:P_t]), (grp, t)
+    # the inserted patterns are used
+    assert (e.vidx[L0 + G:] >= 4).any()
