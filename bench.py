@@ -386,25 +386,27 @@ def kvq_full_pages(w) -> bool:
     return not w.transform and w.P <= 128
 
 
-def measure_decode_loop(w, args, dev, nsteps: int = 512):
+def measure_decode_loop(w, args, dev, nsteps: int = 512, chunk: int = 64):
     """Long chain-of-thought decode: mine patterns on the 8192-token prefill (frozen after it),
-    append the prefill, then steps of a one-token quantize-append per sequence followed by decode
-    attention with a new query; each step timed with CUDA events (median over `nsteps` steps after
-    32 warm-up steps)."""
+    append the prefill, then decode steps -- kvq_decode_step, one launch that quantize-appends one
+    token per sequence and runs decode attention with a new query.  Steps are captured `chunk` at a
+    time in CUDA graphs and replayed (each replay appends `chunk` new tokens); the time per step is
+    the median replay time / chunk.  Falls back to event-timed batches if capture is refused."""
     import numpy as np
     import torch
 
     import bit_kv_cache_26_b200 as kvq
     import synth
 
-    total = w.S + nsteps + 32
+    warm = 2 * chunk
+    total = w.S + nsteps + warm
     k, v = synth.gen_kv(w.with_(S=total))
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
     kd = torch.from_numpy(np.ascontiguousarray(k).view(np.int16)).view(tdt).to(dev)
     vd = torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(tdt).to(dev)
     del k, v
     qs = torch.stack([torch.from_numpy(np.ascontiguousarray(synth.gen_q(w, step=t)).view(np.int16)).view(tdt)
-                      for t in range(nsteps + 32)]).to(dev)
+                      for t in range(nsteps + warm)]).to(dev)
     cache = kvq.PagedKVCache(w.B, w.Hkv, total, w.bits, w.P, dtype=w.dtype, transform=w.transform, device=dev,
                              v_rho=kvq.kvq_v_rho_star(D, w.v_alpha))
     n = w.B * w.S
@@ -413,36 +415,99 @@ def measure_decode_loop(w, args, dev, nsteps: int = 512):
     for x, pat, col in ((pre_k, cache.k_patterns, cache.k_colscale), (pre_v, cache.v_patterns, cache.v_colscale)):
         kvq.kvq_mine_patterns(x, w.dtype, n, 1, w.Hkv, w.Hkv * D, D, n * w.Hkv * D, w.P, w.iters, w.transform,
                               pat, col, None, ws_m)
+    cache.append(pre_k, pre_v)
     del pre_k, pre_v
-    cache.append(kd[:, :w.S].contiguous(), vd[:, :w.S].contiguous())
-    steps_k = [kd[:, w.S + t:w.S + t + 1].contiguous() for t in range(nsteps + 32)]
-    steps_v = [vd[:, w.S + t:w.S + t + 1].contiguous() for t in range(nsteps + 32)]
-    ws_d = cache.decode_workspace(w.Hq)
+    steps_k = [kd[:, w.S + t].contiguous() for t in range(nsteps + warm)]
+    steps_v = [vd[:, w.S + t].contiguous() for t in range(nsteps + warm)]
+    ws_s = cache.step_workspace(w.Hq)
     out = torch.empty(w.B, w.Hq, D, device=dev)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
-    for t in range(nsteps + 32):
-        e = ev[t - 32] if t >= 32 else None
-        if e: e[0].record()
-        cache.append(steps_k[t], steps_v[t])
-        cache.decode(qs[t], out, ws_d)
-        if e: e[1].record()
+
+    def run(t0, t1):
+        for t in range(t0, t1):
+            cache.step(steps_k[t], steps_v[t], qs[t], out, ws_s)
+
+    run(0, chunk)  # warm-up outside any capture
+    torch.cuda.synchronize()
+    method = "cuda graph replay"
+    us = []
+    try:
+        graphs = []
+        for c0 in range(chunk, warm + nsteps, chunk):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                run(c0, c0 + chunk)
+            graphs.append(gph)
+        # capture only records: seq_len has not moved; replay the chunks in order
+        torch.cuda.synchronize()
+        for i, gph in enumerate(graphs):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 1:
+                us.append(1e3 * e0.elapsed_time(e1) / chunk)
+        del graphs
+    except Exception as exc:  # capture refused: time batches of eagerly launched steps instead
+        method = f"event-timed batches ({type(exc).__name__} in capture)"
+        torch.cuda.synchronize()
+        cache.seq_len.fill_(w.S + chunk)
+        us = []
+        for c0 in range(chunk, warm + nsteps, chunk):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run(c0, c0 + chunk)
+            e1.record()
+            torch.cuda.synchronize()
+            if c0 >= warm:
+                us.append(1e3 * e0.elapsed_time(e1) / chunk)
     torch.cuda.synchronize()
     assert cache.read_status() == 0, "device status bits set"
-    us = sorted(1e3 * a.elapsed_time(b) for a, b in ev)
+    assert int(cache.seq_len.min()) == total, "every step appended its token"
+    us.sort()
     med = us[len(us) // 2]
-    ctx = w.S + 32 + nsteps // 2
+    ctx = w.S + warm + nsteps // 2
     pk = peaks()
     step_bytes = w.B * ctx * w.Hkv * bytes_per_token_head(w.bits, w.transform)
-    rec = {"workload": w.name, "bits": w.bits, "metric": "us per decode step (1-token quantize-append + decode)",
-           "us_per_step_median": med, "us_per_step_p10": us[len(us) // 10], "us_per_step_p90": us[9 * len(us) // 10],
-           "steps_timed": nsteps, "context_tokens_mid": ctx, "launches_per_step": 4,
+    rec = {"workload": w.name, "bits": w.bits, "metric": "us per decode step (1-token quantize-append + decode, one launch)",
+           "us_per_step_median": med, "us_per_step_min": us[0], "us_per_step_max": us[-1],
+           "steps_timed": len(us) * chunk, "timing": method, "context_tokens_mid": ctx, "launches_per_step": 1,
            "value": w.B * ctx / (med * 1e-6), "unit": "KV-tokens/s (decode, at the median step)",
            "roofline": {"bound": "hbm", "achieved": step_bytes / (med * 1e-6) / 1e9, "peak": pk["hbm_gbs"],
                         "unit": "GB/s", "frac": step_bytes / (med * 1e-6) / 1e9 / pk["hbm_gbs"], "traffic": None,
-                        "kernel": "decode step (append + decode)", "peak_source": pk["source"]}}
-    del kd, vd, qs, cache, ws_m, ws_d, steps_k, steps_v
+                        "kernel": "decode_mma_kernel (decode step)", "peak_source": pk["source"]}}
+    del kd, vd, qs, cache, ws_m, ws_s, steps_k, steps_v
     torch.cuda.empty_cache()
     return rec
+
+
+def cpu_baseline_step(w, ctx: int):
+    """The oracle on one decode step of one (sequence, KV head) unit of the long-CoT workload:
+    encode the new token against the frozen patterns and run decode attention over `ctx` tokens;
+    scaled to every unit of the batch (us per step)."""
+    import oracle
+    import synth
+
+    sw = w.with_(B=1, S=ctx)
+    k, v = synth.gen_kv(sw, p1=ctx)
+    Kf = synth.to_float(k[0, :, 0], w.dtype)
+    Vf = synth.to_float(v[0, :, 0], w.dtype)
+    MK, cK, _ = oracle.mine_set(Kf[:2048], w.P, w.iters, w.transform)
+    MV, cV, _ = oracle.mine_set(Vf[:2048], w.P, w.iters, w.transform)
+    e = oracle.encode(Kf, Vf, w.bits, MK, MV, cK, cV, v_rho=oracle.v_rho(w.v_alpha))
+    Gq = w.Hq // w.Hkv
+    qf = synth.to_float(synth.gen_q(sw)[0, :Gq], w.dtype)
+    t0 = time.perf_counter()
+    reps = 3
+    for _ in range(reps):
+        oracle.encode(Kf[-1:], Vf[-1:], w.bits, MK, MV, cK, cV, v_rho=oracle.v_rho(w.v_alpha))
+        oracle.attention_unit(qf, Kf, e, MK, MV, cK, cV)
+    dt = (time.perf_counter() - t0) / reps
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    us = dt * 1e6 * w.B * w.Hkv
+    return {"value": us, "unit": "us per decode step", "cores": cores, "kind": "oracle",
+            "sample": f"one (sequence, KV head) unit at {ctx} tokens ({dt * 1e3:.1f} ms: encode the new token, "
+                      f"attention of {Gq} query heads), times the {w.B * w.Hkv} units of a step"}
 
 
 def main():
@@ -497,7 +562,7 @@ def main():
         wl = synth.WORKLOADS["long_cot_8k"]
         r = measure_decode_loop(wl, args, dev)
         if not args.no_cpu_baseline:
-            r["cpu_baseline"], _ = cpu_baseline(wl.with_(S=wl.S + 256), heads=1, seqs=1)
+            r["cpu_baseline"] = cpu_baseline_step(wl, r["context_tokens_mid"])
         per_config.append(r)
 
     if rank == 0:

@@ -47,6 +47,8 @@ class kvq_cache(ctypes.Structure):
         ("k_tail", ctypes.c_void_p), ("k_patterns", ctypes.c_void_p), ("v_patterns", ctypes.c_void_p),
         ("seq_to_set", ctypes.c_void_p), ("k_colscale", ctypes.c_void_p), ("v_colscale", ctypes.c_void_p),
         ("status", ctypes.c_void_p),
+        ("pattern_counts", ctypes.c_void_p), ("pattern_window", ctypes.c_void_p),
+        ("pattern_window_len", ctypes.c_int32), ("reserved", ctypes.c_int32),
     ]
 
 
@@ -64,6 +66,8 @@ _SIGS = {
     "kvq_decode_workspace_bytes": (_sz, [_P, _i32]),
     "kvq_decode_attention": (ctypes.c_int, [_P, _vp, _i32, _f32, _vp, _vp, _sz, _vp]),
     "kvq_decode_attention_static": (ctypes.c_int, [_P, _vp, _i32, _f32, _vp, _vp]),
+    "kvq_step_workspace_bytes": (_sz, [_P, _i32]),
+    "kvq_decode_step": (ctypes.c_int, [_P, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _sz, _vp]),
     "kvq_dequantize": (ctypes.c_int, [_P, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "kvq_read_status": (ctypes.c_int, [_P, ctypes.POINTER(_i32), _i32, _vp]),
     "kvq_mine_read_status": (ctypes.c_int, [_vp, ctypes.POINTER(_i32), _vp]),
@@ -165,6 +169,17 @@ def kvq_decode_attention_static(cache: kvq_cache, q: torch.Tensor, num_q_heads: 
                                             _stream(stream)))
 
 
+def kvq_step_workspace_bytes(cache: kvq_cache, num_q_heads: int) -> int:
+    return int(_lib.kvq_step_workspace_bytes(ctypes.byref(cache), num_q_heads))
+
+
+def kvq_decode_step(cache: kvq_cache, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, num_q_heads: int,
+                    sm_scale: float, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    """One-token quantize-append + decode attention in one launch (workspace zero-filled before first use)."""
+    _check(_lib.kvq_decode_step(ctypes.byref(cache), _ptr(k_new), _ptr(v_new), _ptr(q), num_q_heads, sm_scale,
+                                _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def kvq_dequantize(cache: kvq_cache, seq: int, seq_len_host: int, start: int, count: int,
                    k_out: torch.Tensor | None, v_out: torch.Tensor | None, stream=None) -> None:
     _check(_lib.kvq_dequantize(ctypes.byref(cache), seq, seq_len_host, start, count, _ptr(k_out), _ptr(v_out),
@@ -183,8 +198,8 @@ def kvq_read_status(cache: kvq_cache, clear: bool = False, stream=None) -> int:
 # Device-memory plumbing: a paged cache whose buffers are torch tensors.
 # ---------------------------------------------------------------------------
 
-def _alloc_aligned(nbytes: int, device, align: int = 256) -> torch.Tensor:
-    buf = torch.empty(nbytes + align, dtype=torch.uint8, device=device)
+def _alloc_aligned(nbytes: int, device, align: int = 256, zero: bool = False) -> torch.Tensor:
+    buf = (torch.zeros if zero else torch.empty)(nbytes + align, dtype=torch.uint8, device=device)
     off = (-buf.data_ptr()) % align
     return buf[off:off + nbytes]
 
@@ -196,12 +211,16 @@ class PagedKVCache:
     page i of sequence b at b * max_pages_per_seq + i).
     v_rho: V adaptive threshold (PatternKV Section 3.3); kvq_v_rho_star(128, alpha) for a
     significance level alpha, 0 = off.
+    patterns_in_use / insertion_window: decode-time pattern insertion (PatternKV Section 3.1,
+    Eq. 5): every set starts with `patterns_in_use` of its `num_patterns` rows in use, and each
+    kvq_decode_step that brings a sequence to a multiple of `insertion_window` tokens adds the
+    window's Chebyshev centers as the next pattern (sequences need sets of their own).
     """
 
     def __init__(self, num_seqs: int, num_kv_heads: int, max_tokens: int, bits: int, num_patterns: int,
                  dtype: int = KVQ_BF16, transform: int = KVQ_TX_NONE, num_sets: int = 1, device="cuda",
                  page_order: torch.Tensor | None = None, seq_to_set: torch.Tensor | None = None,
-                 v_rho: float = 0.0):
+                 v_rho: float = 0.0, patterns_in_use: int | None = None, insertion_window: int = 0):
         self.device = torch.device(device)
         self.B, self.H, self.bits, self.P, self.S = num_seqs, num_kv_heads, bits, num_patterns, num_sets
         self.dtype, self.transform = dtype, transform
@@ -230,6 +249,16 @@ class PagedKVCache:
             self.k_colscale = torch.ones(num_sets, self.H, HEAD_DIM, dtype=torch.float32, device=self.device)
             self.v_colscale = torch.ones_like(self.k_colscale)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.pattern_counts = None
+        self.pattern_window = None
+        if patterns_in_use is not None or insertion_window:
+            self.pattern_counts = torch.full((num_sets, self.H), num_patterns if patterns_in_use is None else patterns_in_use,
+                                             dtype=torch.int32, device=self.device)
+        if insertion_window:
+            w = torch.empty(self.B, self.H, 4, HEAD_DIM, dtype=torch.float32, device=self.device)
+            w[:, :, 0::2] = float("inf")
+            w[:, :, 1::2] = float("-inf")
+            self.pattern_window = w
         c.page_pool = self.pool.data_ptr()
         c.page_table = self.page_table.data_ptr() if self.B else None
         c.seq_len = self.seq_len.data_ptr()
@@ -240,6 +269,10 @@ class PagedKVCache:
         c.k_colscale = None if self.k_colscale is None else self.k_colscale.data_ptr()
         c.v_colscale = None if self.v_colscale is None else self.v_colscale.data_ptr()
         c.status = self.status.data_ptr()
+        c.pattern_counts = None if self.pattern_counts is None else self.pattern_counts.data_ptr()
+        c.pattern_window = None if self.pattern_window is None else self.pattern_window.data_ptr()
+        c.pattern_window_len = int(insertion_window)
+        c.reserved = 0
         self.c = c
 
     @property
@@ -267,6 +300,16 @@ class PagedKVCache:
                stream=None) -> None:
         scale = HEAD_DIM ** -0.5 if sm_scale is None else sm_scale
         kvq_decode_attention(self.c, q, int(q.shape[1]), scale, out, ws, stream)
+
+    def step_workspace(self, num_q_heads: int) -> torch.Tensor:
+        """Zero-filled workspace of kvq_decode_step (the kernel keeps its counters at zero)."""
+        return _alloc_aligned(kvq_step_workspace_bytes(self.c, num_q_heads), self.device, zero=True)
+
+    def step(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+             sm_scale: float | None = None, stream=None) -> None:
+        """kvq_decode_step: k_new / v_new [num_seqs][num_kv_heads][128], q [num_seqs][num_q_heads][128]."""
+        scale = HEAD_DIM ** -0.5 if sm_scale is None else sm_scale
+        kvq_decode_step(self.c, k_new, v_new, q, int(q.shape[1]), scale, out, ws, stream)
 
     def read_status(self, clear: bool = False) -> int:
         return kvq_read_status(self.c, clear)

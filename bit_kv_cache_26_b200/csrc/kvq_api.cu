@@ -46,6 +46,10 @@ kvq_status check_cache(const kvq_cache* c) {
     return fail(KVQ_ERR_UNSUPPORTED, "transform %d", c->transform);
   if (!(c->v_rho >= 0.0f) || !(c->v_rho < INFINITY))
     return fail(KVQ_ERR_INVALID_ARG, "v_rho must be finite and >= 0 (0 = adaptive threshold off)");
+  if (c->reserved != 0) return fail(KVQ_ERR_INVALID_ARG, "reserved field must be 0");
+  if (c->pattern_window_len < 0) return fail(KVQ_ERR_INVALID_ARG, "pattern_window_len %d < 0", c->pattern_window_len);
+  if (c->pattern_window_len > 0 && (!c->pattern_counts || !c->pattern_window))
+    return fail(KVQ_ERR_INVALID_ARG, "pattern insertion needs pattern_counts and pattern_window");
   if (c->num_seqs < 0 || c->num_kv_heads < 1 || c->num_sets < 1 || c->max_pages_per_seq < 0 || c->num_pages < 0)
     return fail(KVQ_ERR_INVALID_ARG, "negative or zero size in cache (seqs %d heads %d sets %d pages %d/%d)",
                 c->num_seqs, c->num_kv_heads, c->num_sets, c->max_pages_per_seq, c->num_pages);
@@ -197,6 +201,39 @@ kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t n
   if (!aligned(ws, 256)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   cudaError_t e = kvq::launch_decode(g, q, num_q_heads, sm_scale, out, ws, nsplit, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kvq_decode_attention");
+  return KVQ_OK;
+}
+
+size_t kvq_step_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads) {
+  if (!cache || num_q_heads < 1 || cache->num_kv_heads < 1) return 0;
+  kvq::Geom g = kvq::make_geom(*cache);
+  return kvq::step_workspace(g, num_q_heads, kvq::decode_num_splits(g, num_q_heads, num_sms()));
+}
+
+kvq_status kvq_decode_step(const kvq_cache* cache, const void* k_new, const void* v_new, const void* q,
+                           int32_t num_q_heads, float sm_scale, float* out, void* ws, size_t ws_bytes,
+                           kvq_stream_t stream) {
+  g_err[0] = 0;
+  kvq_status s = check_cache(cache);
+  if (s != KVQ_OK) return s;
+  if (num_q_heads < 1 || num_q_heads % cache->num_kv_heads)
+    return fail(KVQ_ERR_UNSUPPORTED, "num_q_heads %d is not a multiple of num_kv_heads %d", num_q_heads,
+                cache->num_kv_heads);
+  if (num_q_heads / cache->num_kv_heads > 16)
+    return fail(KVQ_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+  if (cache->num_seqs == 0) return KVQ_OK;
+  if (!q || !out || !k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "q / out / k_new / v_new is NULL");
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(KVQ_ERR_INVALID_ARG, "q / out / k_new / v_new must be 16-byte aligned");
+  if (!(sm_scale > 0.0f)) return fail(KVQ_ERR_INVALID_ARG, "sm_scale must be positive");
+  if (cache->max_pages_per_seq < 1) return fail(KVQ_ERR_CAPACITY, "the page table has no column");
+  kvq::Geom g = kvq::make_geom(*cache);
+  const int nsplit = kvq::decode_num_splits(g, num_q_heads, num_sms());
+  const size_t need = kvq::step_workspace(g, num_q_heads, nsplit);
+  if (ws_bytes < need || !ws) return fail(KVQ_ERR_WORKSPACE, "step workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned(ws, 256)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaError_t e = kvq::launch_decode_step(g, k_new, v_new, q, num_q_heads, sm_scale, out, ws, nsplit, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kvq_decode_step");
   return KVQ_OK;
 }
 

@@ -62,14 +62,14 @@ inline AppendWs carve_append(void* ws, int S, int H, int P) {
 // ---- launch 0: probe channels and pattern values there, per (set, head, K|V) ----------
 __global__ void __launch_bounds__(kD) append_prep_kernel(Geom g, AppendWs w) {
   const int sh = blockIdx.x, kv = blockIdx.y;  // sh = set * H + head
-  const int P = g.P;
+  const int P = g.P, Pe = p_eff(g, sh);  // table strides use the capacity P, contents the Pe patterns in use
   const float* M = (kv ? g.vpat : g.kpat) + (size_t)sh * P * kD;
   const size_t o = (size_t)sh * 2 + kv;
   __shared__ float spread[kD];
   __shared__ int pcs[kProbe];
   const int d = threadIdx.x;
   float hi = -INFINITY, lo = INFINITY;
-  for (int j = 0; j < P; ++j) {
+  for (int j = 0; j < Pe; ++j) {
     const float m = M[(size_t)j * kD + d];
     hi = fmaxf(hi, m);
     lo = fminf(lo, m);
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kD) append_prep_kernel(Geom g, AppendWs w) {
   }
   __syncthreads();
   float* pv = w.pv + o * P * kProbe;
-  for (int i = threadIdx.x; i < P * kProbe; i += blockDim.x) pv[i] = M[(size_t)(i / kProbe) * kD + pcs[i % kProbe]];
+  for (int i = threadIdx.x; i < Pe * kProbe; i += blockDim.x) pv[i] = M[(size_t)(i / kProbe) * kD + pcs[i % kProbe]];
 }
 
 struct PageCtx {
@@ -309,7 +309,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   if (!page_context(g, n_new, partial_only, c)) return;
   const int b = blockIdx.z, h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-  const int P = g.P;
+  const int P = g.P;                          // capacity: the layout of the tables
+  const int Pe = p_eff(g, c.set * g.H + h);   // patterns in use
 
   // staged vectors: rows 0..31 = V page slots, rows 32..63 = K page slots
   __shared__ __align__(16) float vec[2 * kG][kLd];
@@ -349,9 +350,9 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const float4* gV = reinterpret_cast<const float4*>(wsp.pv + (shk + 1) * P * kProbe);
     const float* gK = wsp.pv + shk * P * kProbe;
 #pragma unroll 4
-    for (int i = tid; i < P * (kProbeV / 4); i += kAppendThreads) reinterpret_cast<float4*>(tabV)[i] = __ldg(gV + i);
+    for (int i = tid; i < Pe * (kProbeV / 4); i += kAppendThreads) reinterpret_cast<float4*>(tabV)[i] = __ldg(gV + i);
 #pragma unroll 2
-    for (int i = tid; i < P * (kProbeK / 4); i += kAppendThreads)
+    for (int i = tid; i < Pe * (kProbeK / 4); i += kAppendThreads)
       reinterpret_cast<float4*>(tabK)[i] =
           __ldg(reinterpret_cast<const float4*>(gK + (size_t)(i / (kProbeK / 4)) * kProbe) + i % (kProbeK / 4));
     if (tid < kProbeV) pcV[tid] = __ldg(wsp.probe + (shk + 1) * kProbe + tid);
@@ -405,15 +406,15 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
 
   // ---- probe-channel lower bounds: warp (kind = warp & 1: 0 V, 1 K; half = warp >> 1),
   // lane = row; patterns split in two halves.  Running argmin per half (ties: lowest j).
-  const int P0 = (P + 1) >> 1;
+  const int P0 = (Pe + 1) >> 1;
   {
     const int kind = warp & 1, half = warp >> 1;
     const int r = kind * kG + lane;
-    if (kind == 0) lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
-    else if (c.seal) lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? P : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    if (kind == 0) lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? Pe : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    else if (c.seal) lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, r, hlb[half][r], hj[half][r]);
     if (kind == 0 || c.seal) {
       // the half's best pattern is the likely seed: its row into L1 ahead of the exact range
-      const float* mrow = (kind ? c.MK : c.MV) + (size_t)min(max(hj[half][r], 0), P - 1) * kD;
+      const float* mrow = (kind ? c.MK : c.MV) + (size_t)min(max(hj[half][r], 0), Pe - 1) * kD;
 #pragma unroll
       for (int u = 0; u < 4; ++u) asm volatile("prefetch.global.L1 [%0];" ::"l"(mrow + 32 * u));
     }
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     float mx = -INFINITY, mn = INFINITY, ymx = -INFINITY, ymn = INFINITY;
     if (on) {
       s = hlb[1][r] < hlb[0][r] ? hj[1][r] : hj[0][r];
-      s = min(max(s, 0), P - 1);
+      s = min(max(s, 0), Pe - 1);
       const float* m = (r < kG ? c.MV : c.MK) + (size_t)s * kD;
       range64(vec[r], m, 64 * hh, hh, mx, mn);
       if (r < kG && g.vrho > 0.0f) {  // the V vector's own range, for the adaptive threshold
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       best[r] = dkey(ds, s);
     }
     if (on) {
-      const int j1 = hh ? P : P0;
+      const int j1 = hh ? Pe : P0;
 #pragma unroll 4
       for (int j = hh ? P0 : 0; j < j1; ++j) {
         const float lb = __half2float(lbuf[j * (2 * kG) + r]);
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const int r = tid >> 1, hh = tid & 1;
     if (row_on(r)) {
       const float* M = r < kG ? c.MV : c.MK;
-      for (int j = hh; j < P; j += 2) {
+      for (int j = hh; j < Pe; j += 2) {
         float mx = -INFINITY, mn = INFINITY;
         for (int cb = 0; cb < kD; cb += 32) range32(vec[r], M + (size_t)j * kD, cb, mx, mn);
         atomicMin(&best[r], dkey(__fsub_rn(mx, mn), j));

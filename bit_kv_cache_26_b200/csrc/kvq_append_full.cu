@@ -270,8 +270,6 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
   const int r = lane & 15, hh = lane >> 4;
   const int row = 16 * (warp & 1) + r;
   const int LdP = (P + 7) & ~7;  // row stride of the K bound table (halves)
-  const int P2 = (P + 1) >> 1;
-  const int jb = hh * P2, je = min(P, jb + P2);  // this lane's pattern half
   const int maxc = (1 << g.bits) - 1;
 
   const int64_t T = (int64_t)g.H * g.B * F;
@@ -321,6 +319,9 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
     const int sh = k.set * g.H + k.h;
     const float* MK = g.kpat + (size_t)sh * P * kD;
     const float* MV = g.vpat + (size_t)sh * P * kD;
+    const int Pe = p_eff(g, sh), Pep = (Pe + 7) & ~7;  // patterns in use (P is the capacity)
+    const int P2 = (Pe + 1) >> 1;
+    const int jb = hh * P2, je = min(Pe, jb + P2);  // this lane's pattern half
     uint8_t* sub = g.pool + (size_t)g.page_table[(size_t)k.b * g.maxp + k.pg] * g.page_bytes + (size_t)k.h * g.sub_bytes;
 
     // ---- pattern tables of this (set, head), staged when they change
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       cached_sh = sh;
       for (int i4 = tid; i4 < Pp * (kD / 4); i4 += kFThreads) {
         const int n = i4 / (kD / 4), c4 = i4 % (kD / 4);
-        float4 m = n < P ? __ldg(reinterpret_cast<const float4*>(MV + (size_t)n * kD) + c4) : make_float4(0, 0, 0, 0);
+        float4 m = n < Pe ? __ldg(reinterpret_cast<const float4*>(MV + (size_t)n * kD) + c4) : make_float4(0, 0, 0, 0);
         uint16_t h4[4];
         const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
@@ -341,13 +342,13 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       }
       for (int n = tid; n < Pp; n += kFThreads) {
         float acc = 0.f;
-        if (n < P)
+        if (n < Pe)
           for (int c = 0; c < kD; ++c) { const float m = __ldg(MV + (size_t)n * kD + c); acc = fmaf(m, m, acc); }
-        hnorm[n] = n < P ? 0.5f * acc : 1e30f;
+        hnorm[n] = n < Pe ? 0.5f * acc : 1e30f;
       }
       const size_t o = (size_t)sh * 2;
-      for (int q = tid; q < P * kProbeAll; q += kFThreads) tabv[q] = __ldg(pvals + (o + 1) * P * kProbeAll + q);
-      for (int q = tid; q < P * kK1; q += kFThreads)
+      for (int q = tid; q < Pe * kProbeAll; q += kFThreads) tabv[q] = __ldg(pvals + (o + 1) * P * kProbeAll + q);
+      for (int q = tid; q < Pe * kK1; q += kFThreads)
         tabk[q] = __ldg(pvals + o * P * kProbeAll + (size_t)(q / kK1) * kProbeAll + q % kK1);
       if (tid < kProbeAll) pcv[tid] = __ldg(probe + (o + 1) * kProbeAll + tid);
       if (tid < kK1) pck[tid] = __ldg(probe + o * kProbeAll + tid);
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       }
       const int tig = lane & 3;
       float b0 = INFINITY, b8 = INFINITY;  // tagged scores of rows gq and gq + 8
-      for (int nt = 0; nt < Pp / 8; ++nt) {
+      for (int nt = 0; nt < Pep / 8; ++nt) {
         float acc[4];
         acc[0] = acc[2] = hnorm[8 * nt + 2 * tig];
         acc[1] = acc[3] = hnorm[8 * nt + 2 * tig + 1];
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       b8 = fminf(b8, __shfl_xor_sync(kFull, b8, 2));
       const float s_lo = __shfl_sync(kFull, b0, 4 * (r & 7)), s_hi = __shfl_sync(kFull, b8, 4 * (r & 7));
       int seed = (int)(__float_as_uint(r < 8 ? s_lo : s_hi) & 127u);
-      seed = min(seed, P - 1);
+      seed = min(seed, Pe - 1);
 
       // ---- U = exact d_mm of the seed; the vector's own range (adaptive threshold)
       float mx, mn;
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       const float olb = __shfl_xor_sync(kFull, lbest, 16);
       const int oj = __shfl_xor_sync(kFull, lj, 16);
       if (olb < lbest || (olb == lbest && oj < lj)) { lbest = olb; lj = oj; }
-      const int seed = min(max(lj, 0), P - 1);
+      const int seed = min(max(lj, 0), Pe - 1);
       float mx, mn;
       half_range(x, MK + (size_t)seed * kD + 64 * hh, mx, mn);
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));

@@ -39,7 +39,15 @@ struct Geom {
   int32_t* status;
   uint32_t wait_limit;  // iterations of a bounded page-copy wait (decode)
   float vrho;           // V adaptive threshold rho* (0 = off)
+  int32_t* counts;      // [S][H] patterns in use, or null (all P)
+  float* window;        // [B][H][4][128] running min / max of the insertion window, or null
+  int32_t gwin;         // insertion window length (0 = off)
 };
+
+// Patterns in use by (set, KV head): the set's count (clamped to 1..P) or P.
+__device__ __forceinline__ int p_eff(const Geom& g, int sh) {
+  return g.counts ? min(max(g.counts[sh], 1), g.P) : g.P;
+}
 
 __host__ __device__ inline int64_t subblock_bytes_of(int bits, int tx) {
   return 2 * (kG * kD * bits / 8) + 2112 + (tx ? 256 : 0);
@@ -73,6 +81,9 @@ inline Geom make_geom(const kvq_cache& c) {
   g.status = c.status;
   g.wait_limit = 1u << 22;
   g.vrho = c.v_rho;
+  g.counts = c.pattern_counts;
+  g.window = c.pattern_window;
+  g.gwin = c.pattern_window_len;
   return g;
 }
 

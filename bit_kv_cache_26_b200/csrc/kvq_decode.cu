@@ -54,4 +54,25 @@ cudaError_t launch_decode(const Geom& g0, const void* q, int Hq, float sm_scale,
   return launch_decode_mma(g, q, Hq, sm_scale * kLog2e, nsplit, part_ml, part_o, arrivals, out, st);
 }
 
+// Decode step: partials, the per-(sequence, KV head) arrival counters, then one counter per
+// sequence.  No memset: the kernel leaves every counter at zero (the caller zeroes the workspace
+// once, before its first use).
+size_t step_workspace(const Geom& g, int Hq, int nsplit) {
+  return decode_workspace(g, Hq, nsplit) + (size_t)g.B * sizeof(int) + 256;
+}
+
+cudaError_t launch_decode_step(const Geom& g0, const void* k_new, const void* v_new, const void* q, int Hq,
+                               float sm_scale, float* out, void* ws, int nsplit, cudaStream_t st) {
+  if (g0.B == 0) return cudaSuccess;
+  Geom g = g0;
+  g.wait_limit = page_wait_limit(g0.wait_limit);
+  const size_t rows = (size_t)g.B * Hq * nsplit;
+  float* part_ml = reinterpret_cast<float*>(ws);
+  float* part_o = part_ml + 2 * rows;
+  int* arrivals = reinterpret_cast<int*>(part_o + kD * rows);
+  int* seqcnt = arrivals + (size_t)g.B * g.H;
+  return launch_decode_step_mma(g, k_new, v_new, q, Hq, sm_scale * kLog2e, nsplit, part_ml, part_o, arrivals, seqcnt,
+                                out, st);
+}
+
 }  // namespace kvq

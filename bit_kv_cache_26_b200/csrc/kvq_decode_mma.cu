@@ -237,11 +237,260 @@ __device__ void combine_group(const Geom& g, int Hq, int nsplit, int b, int h_kv
   }
 }
 
-template <int BITS, int NT, int STAGES, int kWarps>
+// ---- one-token append of a decode step (the last split's CTA, before its page copies) ----------
+//
+// The same definitions as the bulk append ("PatternKV", Section 3.2, Eq. 6 and Eq. 1; Section
+// 3.3 for V; Section 3.1, Eq. 5 for the window), for one new token of sequence b and KV head h at
+// position L: the exact min-max argmin over the Pe patterns in use (two threads per pattern, a
+// channel half each, lowest index on ties), the V codes merged into the page's words (atomicOr:
+// two channels of a token share a word), the raw key into the K tail; when the token completes
+// its page, the page's 32 keys are assigned (four threads per key) and quantized per channel.
+// With decode-time insertion, the window's running min / max take the token and, when L + 1 is a
+// multiple of the window length, the Chebyshev centers become pattern Pe of the sequence's set.
+// Scratch: the first bytes of the CTA's page ring (unused until the page copies start).
+constexpr int kYLd = kD + 4;
+
+__device__ __forceinline__ unsigned long long min_key(unsigned long long a, unsigned long long b2) {
+  return a < b2 ? a : b2;
+}
+__device__ __forceinline__ unsigned long long dkey_s(float d, int j) {
+  return ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j;
+}
+
+// nearest pattern of the vector y (shared, 128 channels) among M[0..Pe): exact fp32 d_mm, key
+// (d bits << 32 | j) of the minimum; all 128 threads of the CTA take part, every thread gets it
+__device__ unsigned long long nearest_dmm_cta(const float* y, const float* __restrict__ M, int Pe,
+                                              unsigned long long* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, half = tid & 1;
+  unsigned long long best = ~0ull;
+  for (int j0 = 0; j0 < Pe; j0 += 64) {
+    const int j = j0 + (tid >> 1);
+    float mx = -INFINITY, mn = INFINITY;
+    if (j < Pe) {
+      const float4* m4 = reinterpret_cast<const float4*>(M + (size_t)j * kD + 64 * half);
+      const float4* y4 = reinterpret_cast<const float4*>(y + 64 * half);
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        const float4 m = __ldg(m4 + c), a = y4[c];
+        float r0, r1, r2, r3;
+        sub2(a.x, a.y, m.x, m.y, r0, r1);
+        sub2(a.z, a.w, m.z, m.w, r2, r3);
+        mx = max3(mx, r0, r1);
+        mn = min3(mn, r0, r1);
+        mx = max3(mx, r2, r3);
+        mn = min3(mn, r2, r3);
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+    if (j < Pe) best = min_key(best, dkey_s(__fsub_rn(mx, mn), j));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) best = min_key(best, __shfl_xor_sync(kFull, best, o));
+  if (lane == 0) red[warp] = best;
+  __syncthreads();
+  best = min_key(min_key(red[0], red[1]), min_key(red[2], red[3]));
+  __syncthreads();
+  return best;
+}
+
+template <int BITS>
+__device__ void step_append(const Geom& g, int b, int h, int L, int set, int Pe, const uint16_t* __restrict__ k_new,
+                            const uint16_t* __restrict__ v_new, uint8_t* scratch) {
+  constexpr int maxc = (1 << BITS) - 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int slot = L % kG, pg = L / kG;
+  const size_t sh = (size_t)set * g.H + h;
+  const float* MK = g.kpat + sh * g.P * kD;
+  const float* MV = g.vpat + sh * g.P * kD;
+  uint8_t* sub = g.pool + (size_t)g.page_table[(size_t)b * g.maxp + pg] * g.page_bytes + (size_t)h * g.sub_bytes;
+  float* yv = reinterpret_cast<float*>(scratch);             // [128]
+  float* yk = yv + kD;                                       // [32][kYLd] keys of the page (sealing) or [1]
+  float* rowf = yk + kG * kYLd;                              // [33] row factors: keys 0..31, then V
+  unsigned long long* red = reinterpret_cast<unsigned long long*>(rowf + 40);  // [4]
+  float* vstat = reinterpret_cast<float*>(red + 4);          // [2] range of y_v
+  int* kbest = reinterpret_cast<int*>(vstat + 4);            // [32]
+  float* kz = reinterpret_cast<float*>(kbest + kG);          // [128] K zero, then [128] K scale
+  const uint16_t* kin = k_new + ((size_t)b * g.H + h) * kD;
+  const uint16_t* vin = v_new + ((size_t)b * g.H + h) * kD;
+  const bool seal = slot == kG - 1;
+
+  // ---- the new vectors (and, when the page seals, its other 31 keys from the K tail), pre-transformed
+  uint16_t* tail = g.k_tail + ((size_t)b * g.H + h) * kG * kD;
+  for (int r = warp; r < 2 + (seal ? kG - 1 : 0); r += 4) {
+    // r = 0: V; r = 1: the new key (page slot `slot`); r >= 2: key of slot r - 2 from the tail
+    const uint16_t* src = r == 0 ? vin : r == 1 ? kin : tail + (size_t)(r - 2) * kD;
+    float y[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) y[k] = bits_to_float(src[lane + 32 * k], g.dtype);  // plain loads: the tail is written here
+    float rr = 1.0f;
+    if (g.tx) transform_row_warp(y, r == 0 ? g.vcol + sh * kD : g.kcol + sh * kD, rr, lane);
+    float* dst = r == 0 ? yv : yk + (size_t)(r == 1 ? (seal ? slot : 0) : r - 2) * kYLd;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dst[lane + 32 * k] = y[k];
+    if (lane == 0) rowf[r == 0 ? kG : (r == 1 ? (seal ? slot : 0) : r - 2)] = rr;
+    if (r == 0) {
+      float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) { mx = fmaxf(mx, y[k]); mn = fminf(mn, y[k]); }
+      mx = warp_max(mx);
+      mn = warp_min(mn);
+      if (lane == 0) vstat[0] = __fsub_rn(mx, mn);
+    }
+  }
+  // the raw key joins the K tail
+  if (tid < kD) tail[(size_t)slot * kD + tid] = kin[tid];
+  if (slot == 0) {
+    // a fresh page: the V part of the page starts from zeros (tokens not yet appended are zero)
+    uint32_t* w = reinterpret_cast<uint32_t*>(sub + g.off_vc);
+    for (int i = tid; i < g.cb / 4; i += blockDim.x) w[i] = 0u;
+    float* vs = reinterpret_cast<float*>(sub + g.off_vs);
+    for (int i = tid; i < 2 * 128; i += blockDim.x) vs[i] = 0.f;  // V scales then V zeros (512 B each)
+    if (tid < kG / 4) reinterpret_cast<uint32_t*>(sub + g.off_vidx)[tid] = 0u;
+    if (g.tx && tid < kG) reinterpret_cast<float*>(sub + g.off_vrow)[tid] = 0.f;
+  }
+  __syncthreads();
+
+  // ---- decode-time insertion: the window's running min / max take the new vectors; at the
+  // window's end the centers are written as pattern Pe (its count is raised at the very end,
+  // after this token's own assignments, which use the Pe patterns present)
+  const bool emit = g.gwin > 0 && g.window && (L + 1) % g.gwin == 0 && Pe < g.P;
+  if (g.gwin > 0 && g.window) {
+    float* wnd = g.window + ((size_t)b * g.H + h) * 4 * kD;
+    const int c = tid;
+    const float kk = yk[(size_t)(seal ? slot : 0) * kYLd + c], v = yv[c];
+    const float kmn = fminf(wnd[c], kk), kmx = fmaxf(wnd[kD + c], kk);
+    const float vmn = fminf(wnd[2 * kD + c], v), vmx = fmaxf(wnd[3 * kD + c], v);
+    if ((L + 1) % g.gwin == 0) {
+      if (emit) {
+        // (the pattern buffers are the caller's; with insertion on, steps write their rows Pe .. P - 1)
+        const_cast<float*>(g.kpat)[(sh * g.P + Pe) * kD + c] = __fmul_rn(__fadd_rn(kmn, kmx), 0.5f);
+        const_cast<float*>(g.vpat)[(sh * g.P + Pe) * kD + c] = __fmul_rn(__fadd_rn(vmn, vmx), 0.5f);
+      }
+      wnd[c] = INFINITY;
+      wnd[kD + c] = -INFINITY;
+      wnd[2 * kD + c] = INFINITY;
+      wnd[3 * kD + c] = -INFINITY;
+    } else {
+      wnd[c] = kmn;
+      wnd[kD + c] = kmx;
+      wnd[2 * kD + c] = vmn;
+      wnd[3 * kD + c] = vmx;
+    }
+  }
+
+  // ---- V: nearest pattern, adaptive threshold, residual, 4 groups of 32 channels (warp = group)
+  {
+    const unsigned long long kv = nearest_dmm_cta(yv, MV, Pe, red);
+    const int j = (int)(kv & 0xffffffffu);
+    const bool keep = v_keep_pattern(g.vrho, __uint_as_float((uint32_t)(kv >> 32)), vstat[0]);
+    const int c = 32 * warp + lane;
+    const float R = keep ? __fsub_rn(yv[c], __ldg(MV + (size_t)j * kD + c)) : yv[c];
+    float s, z;
+    int code = quant_warp(R, BITS, s, z);
+    int wd, bt;
+    frag_pos(BITS, 2, c, slot, wd, bt);
+    atomicOr(reinterpret_cast<unsigned int*>(sub + g.off_vc) + wd, (unsigned)code << bt);
+    if (lane == 0) {
+      reinterpret_cast<float*>(sub + g.off_vs)[vsc_pos(slot, warp)] = s;
+      reinterpret_cast<float*>(sub + g.off_vz)[vzc_pos(slot, warp)] = z;
+    }
+    if (tid == 0) {
+      sub[g.off_vidx + tok_pos(slot)] = keep ? (uint8_t)j : (uint8_t)kRawIndex;
+      if (g.tx) reinterpret_cast<float*>(sub + g.off_vrow)[tok_pos(slot)] = rowf[kG];
+    }
+  }
+
+  // ---- K: the page seals: its 32 keys, nearest patterns (4 threads per key), per-channel groups
+  if (seal) {
+    {
+      const int r = tid >> 2, q = tid & 3;  // key r, channels 32 q .. 32 q + 31
+      const float* y = yk + (size_t)r * kYLd + 32 * q;
+      unsigned long long best = ~0ull;
+      for (int j = 0; j < Pe; ++j) {
+        const float4* m4 = reinterpret_cast<const float4*>(MK + (size_t)j * kD + 32 * q);
+        const float4* y4 = reinterpret_cast<const float4*>(y);
+        float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 m = __ldg(m4 + c), a = y4[c];
+          float r0, r1, r2, r3;
+          sub2(a.x, a.y, m.x, m.y, r0, r1);
+          sub2(a.z, a.w, m.z, m.w, r2, r3);
+          mx = max3(mx, r0, r1);
+          mn = min3(mn, r0, r1);
+          mx = max3(mx, r2, r3);
+          mn = min3(mn, r2, r3);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, 2));
+        best = min_key(best, dkey_s(__fsub_rn(mx, mn), j));
+      }
+      if (q == 0) kbest[r] = (int)(best & 0xffffffffu);
+    }
+    __syncthreads();
+    // residuals in place, then scale / zero per channel (thread = channel)
+    for (int i = tid; i < kG * kD; i += blockDim.x) {
+      const int r = i / kD, c = i % kD;
+      yk[(size_t)r * kYLd + c] = __fsub_rn(yk[(size_t)r * kYLd + c], __ldg(MK + (size_t)kbest[r] * kD + c));
+    }
+    __syncthreads();
+    {
+      const int c = tid;
+      float mx = -INFINITY, mn = INFINITY;
+      for (int r = 0; r < kG; ++r) { mx = fmaxf(mx, yk[(size_t)r * kYLd + c]); mn = fminf(mn, yk[(size_t)r * kYLd + c]); }
+      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)maxc);
+      kz[c] = mn;
+      kz[kD + c] = s;
+      reinterpret_cast<float*>(sub + g.off_ks)[ksc_pos(c)] = s;
+      reinterpret_cast<float*>(sub + g.off_kz)[ksc_pos(c)] = mn;
+    }
+    __syncthreads();
+    // every 32-bit word of the K block, codes by the definition
+    for (int wd = tid; wd < g.cb / 4; wd += blockDim.x) {
+      uint32_t word = 0u;
+      constexpr int SPW = 16 / BITS;
+      for (int sl = 0; sl < SPW; ++sl)
+        for (int odd = 0; odd < 2; ++odd) {
+          int r, c;
+          frag_elem(BITS, 8, wd, sl, odd, r, c);
+          const float R = yk[(size_t)r * kYLd + c], sc = kz[kD + c];
+          uint32_t code = 0u;
+          if (sc != 0.0f) code = (uint32_t)min(max(__float2int_rn(__fdiv_rn(__fsub_rn(R, kz[c]), sc)), 0), maxc);
+          word |= code << (BITS * sl + 16 * odd);
+        }
+      reinterpret_cast<uint32_t*>(sub)[wd] = word;
+    }
+    if (tid < kG) {
+      sub[g.off_kidx + tok_pos(tid)] = (uint8_t)kbest[tid];
+      if (g.tx) reinterpret_cast<float*>(sub + g.off_krow)[tok_pos(tid)] = rowf[tid];
+    }
+  }
+
+  // the new pattern rows before the raised count (readers of the count then see the rows)
+  if (emit) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) g.counts[sh] = Pe + 1;
+  }
+  // the page writes above before the tensor / bulk copies of this CTA read the sealed page
+  __threadfence();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncthreads();
+}
+
+// STEP: a decode step -- the last split's CTA of each (sequence, KV head) first appends the
+// sequence's new token (step_append), then decodes over every token including it; the other
+// splits decode the pages complete before the step.  The CTA that starts last among a
+// sequence's CTAs advances its seq_len (all of them have read the old length by then).
+template <int BITS, int NT, int STAGES, int kWarps, bool STEP>
 __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT == 1 ? 4 : 3) : 2))
     decode_mma_kernel(Geom g, const uint16_t* __restrict__ q, int Hq, float scale_log2, int nsplit,
                       float* __restrict__ part_ml, float* __restrict__ part_o, int* __restrict__ arrivals,
-                      float* __restrict__ out) {
+                      float* __restrict__ out, const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
+                      int* __restrict__ seqcnt) {
   constexpr int NH = NT * 4;  // padded heads
   constexpr int WPL = Cfg<BITS>::kWordsPerLane;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -266,21 +515,50 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   float* pex = reinterpret_cast<float*>(smem + sp.pex) + warp * NH * kPexLd;
 
   int L = g.seq_len[b];
+  bool seq_ok = true;  // a sequence with a bad length or set is decoded as empty and left unchanged
   if (L < 0 || L > g.maxp * kG) {
     if (threadIdx.x == 0 && split == 0) set_status(g.status, KVQ_DEV_OVERFLOW);
     L = 0;
+    seq_ok = false;
   }
   int set = g.seq_to_set ? g.seq_to_set[b] : 0;
   if (set < 0 || set >= g.S) {
     if (threadIdx.x == 0 && split == 0) set_status(g.status, KVQ_DEV_BAD_SET);
     set = 0;
     L = 0;
+    seq_ok = false;
   }
-  const int nfull = L / kG, ntail = L % kG;
+  // a decode step appends one token: it needs room in the page table and a valid page
+  bool app = false;
+  if constexpr (STEP) {
+    if (!seq_ok) {
+    } else if (L + 1 > g.maxp * kG) {
+      if (threadIdx.x == 0 && split == 0 && h_kv == 0) set_status(g.status, KVQ_DEV_OVERFLOW);
+    } else {
+      const int phys = g.page_table[(size_t)b * g.maxp + L / kG];
+      app = phys >= 0 && phys < g.npages;
+      if (!app && threadIdx.x == 0 && split == 0 && h_kv == 0) set_status(g.status, KVQ_DEV_BAD_PAGE);
+    }
+    if (threadIdx.x == 0) {
+      // every CTA of sequence b has read its old length once the counter reaches H * nsplit
+      if (atomicAdd(seqcnt + b, 1) == g.H * nsplit - 1) {
+        seqcnt[b] = 0;
+        if (app) g.seq_len[b] = L + 1;
+      }
+    }
+  }
+  const int nfull = L / kG;
   const int per = (nfull + nsplit - 1) / nsplit;
-  const int p0 = min(nfull, split * per), p1 = min(nfull, p0 + per);
+  const int p0 = min(nfull, split * per);
+  // the last split also takes the page the step's token completes (and the tail after it)
+  const int p1 = (STEP && app && split == nsplit - 1) ? (L + 1) / kG : min(nfull, p0 + per);
+  const int ntail = (STEP && app) ? (L + 1) % kG : L % kG;
   const size_t sh = (size_t)set * g.H + h_kv;
   const float* MK = g.kpat + sh * P * kD;
+  const int Pe = p_eff(g, (int)sh);  // patterns in use by this set (rows beyond are capacity)
+  if constexpr (STEP) {
+    if (app && split == nsplit - 1) step_append<BITS>(g, b, h_kv, L, set, Pe, k_new, v_new, ring - warp * STAGES * sub_bytes);
+  }
   const float* cK = g.tx ? g.kcol + sh * kD : nullptr;
 
   // ---- the first STAGES page copies of each warp go out before the setup below
@@ -361,12 +639,12 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
       }
     }
     // sixteen pattern rows' loads in flight at a time
-    for (int j0 = warp; j0 < P; j0 += 16 * kWarps) {
+    for (int j0 = warp; j0 < Pe; j0 += 16 * kWarps) {
       float4 m4[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int j = j0 + u * kWarps;
-        m4[u] = j < P ? __ldg(reinterpret_cast<const float4*>(MK + (size_t)j * kD) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        m4[u] = j < Pe ? __ldg(reinterpret_cast<const float4*>(MK + (size_t)j * kD) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
@@ -379,7 +657,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
         for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
           for (int a = 0; a < 4; ++a) t[a] += __shfl_xor_sync(kFull, t[a], off);
-        if (lane < 4 && j < P) T[(4 * hg + lane) * P + j] = lane == 0 ? t[0] : lane == 1 ? t[1] : lane == 2 ? t[2] : t[3];
+        if (lane < 4 && j < Pe) T[(4 * hg + lane) * P + j] = lane == 0 ? t[0] : lane == 1 ? t[1] : lane == 2 ? t[2] : t[3];
       }
     }
   }
@@ -480,7 +758,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
         float pm = -INFINITY;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int idx = min((int)((kidx4 >> (8 * u)) & 0xff), P - 1);
+          const int idx = min((int)((kidx4 >> (8 * u)) & 0xff), Pe - 1);
           sc[j][u] = (sc[j][u] + T[hh * P + idx]) * krow[u] * scale_log2;
           pm = fmaxf(pm, sc[j][u]);
         }
@@ -497,7 +775,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
           for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
-          for (int jj = gq; jj < P; jj += 8) Ww[hh * P1 + jj] *= alpha;
+          for (int jj = gq; jj < Pe; jj += 8) Ww[hh * P1 + jj] *= alpha;
           __syncwarp();
         }
         mrun[j] = mnew;
@@ -601,7 +879,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
         const uint16_t* kt = g.k_tail + (((size_t)b * g.H + h_kv) * kG + t) * kD;
         float kv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) kv[k] = load_elem(kt + lane + 32 * k, g.dtype);
+        for (int k = 0; k < 4; ++k) kv[k] = bits_to_float(kt[lane + 32 * k], g.dtype);  // plain: a step writes the tail
         const int vidx = min((int)sub[g.off_vidx + tok_pos(t)], P);  // P: stored raw
         const float vrow = g.tx ? vr[tok_pos(t)] : 1.0f;
 #pragma unroll
@@ -629,7 +907,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
             for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
               for (int u = 0; u < 4; ++u) accv[j][mt][u] *= alpha;
-            for (int jj = gq; jj < P; jj += 8) Ww[hh * P1 + jj] *= alpha;
+            for (int jj = gq; jj < Pe; jj += 8) Ww[hh * P1 + jj] *= alpha;
           }
           mrun[j] = mnew;
           __syncwarp();
@@ -714,7 +992,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
     }
     const size_t base = ((size_t)b * Hq + h_kv * Gq + hh) * nsplit + split;
     if (lane == 0) { part_ml[2 * base] = M; part_ml[2 * base + 1] = Ls; }
-    for (int jj = lane; jj < P; jj += 32) {
+    for (int jj = lane; jj < Pe; jj += 32) {
       float Wv = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) Wv += f[w] * Wall[(w * NH + hh) * P1 + jj];
@@ -733,7 +1011,7 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
 #pragma unroll
     for (int i = 0; i < NA; ++i) acc[i] = 0.f;
 #pragma unroll 8
-    for (int j = 0; j < P; ++j) {
+    for (int j = 0; j < Pe; ++j) {
       const float m = __ldg(mv + (size_t)j * kD);
 #pragma unroll
       for (int i = 0; i < NA; ++i) acc[i] = fmaf(wc[j * NH + hg + HG * i], m, acc[i]);
@@ -754,16 +1032,20 @@ __global__ void __launch_bounds__(kWarps * 32, (kWarps == 4 ? (STAGES <= 2 && NT
   __shared__ int last;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(arrivals + (size_t)b * g.H + h_kv, 1) == nsplit - 1;
+  if (threadIdx.x == 0) {
+    last = atomicAdd(arrivals + (size_t)b * g.H + h_kv, 1) == nsplit - 1;
+    if (last) arrivals[(size_t)b * g.H + h_kv] = 0;  // every split has arrived: ready for the next call
+  }
   __syncthreads();
   if (!last) return;
   __threadfence();
   combine_group(g, Hq, nsplit, b, h_kv, Gq, set, part_ml, part_o, out);
 }
 
-template <int BITS, int NT, int STAGES, int NW>
+template <int BITS, int NT, int STAGES, int NW, bool STEP = false>
 struct Launcher {
-  static auto kernel() { return decode_mma_kernel<BITS, NT, STAGES, NW>; }
+  using Step = Launcher<BITS, NT, STAGES, NW, true>;  // the decode-step variant of this configuration
+  static auto kernel() { return decode_mma_kernel<BITS, NT, STAGES, NW, STEP>; }
   static int smem(const Geom& g) { return smem_plan((int)g.sub_bytes, STAGES, NT, g.P, NW).total; }
   static int occupancy(const Geom& g) {
     int n = 0;
@@ -772,12 +1054,14 @@ struct Launcher {
     return n > 0 ? n : 1;
   }
   static cudaError_t launch(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml, float* o,
-                            int* arrivals, float* out, cudaStream_t st) {
+                            int* arrivals, float* out, const void* k_new, const void* v_new, int* seqcnt,
+                            cudaStream_t st) {
     const int total = smem(g);
     cudaError_t e = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, g.H, g.B);
-    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, arrivals, out);
+    kernel()<<<grid, NW * 32, total, st>>>(g, (const uint16_t*)q, Hq, scale_log2, nsplit, ml, o, arrivals, out,
+                                           (const uint16_t*)k_new, (const uint16_t*)v_new, seqcnt);
     return cudaGetLastError();
   }
 };
@@ -845,7 +1129,15 @@ size_t decode_mma_smem(const Geom& g, int Hq) {
 cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
                               float* o, int* arrivals, float* out, cudaStream_t st) {
   return dispatch(g, Hq, decode_stages(), [&](auto L) {
-    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, arrivals, out, st);
+    return decltype(L)::launch(g, q, Hq, scale_log2, nsplit, ml, o, arrivals, out, nullptr, nullptr, nullptr, st);
+  });
+}
+
+cudaError_t launch_decode_step_mma(const Geom& g, const void* k_new, const void* v_new, const void* q, int Hq,
+                                   float scale_log2, int nsplit, float* ml, float* o, int* arrivals, int* seqcnt,
+                                   float* out, cudaStream_t st) {
+  return dispatch(g, Hq, decode_stages(), [&](auto L) {
+    return decltype(L)::Step::launch(g, q, Hq, scale_log2, nsplit, ml, o, arrivals, out, k_new, v_new, seqcnt, st);
   });
 }
 

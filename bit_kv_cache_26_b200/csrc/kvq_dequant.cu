@@ -38,7 +38,7 @@ __global__ void dequant_kernel(Geom g, int b, int start, int count, float* __res
       const uint32_t* words = reinterpret_cast<const uint32_t*>(sub);
       const float* ks = reinterpret_cast<const float*>(sub + g.off_ks);
       const float* kz = reinterpret_cast<const float*>(sub + g.off_kz);
-      const int idx = min((int)sub[g.off_kidx + tok_pos(slot)], g.P - 1);
+      const int idx = min((int)sub[g.off_kidx + tok_pos(slot)], p_eff(g, (int)sh) - 1);
       const float* M = g.kpat + (sh * g.P + idx) * kD;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -65,7 +65,7 @@ __global__ void dequant_kernel(Geom g, int b, int start, int count, float* __res
     const float* vs = reinterpret_cast<const float*>(sub + g.off_vs);
     const float* vz = reinterpret_cast<const float*>(sub + g.off_vz);
     const int vi = sub[g.off_vidx + tok_pos(slot)];
-    const float* M = vi == kRawIndex ? nullptr : g.vpat + (sh * g.P + min(vi, g.P - 1)) * kD;  // 255: stored raw
+    const float* M = vi == kRawIndex ? nullptr : g.vpat + (sh * g.P + min(vi, p_eff(g, (int)sh) - 1)) * kD;  // 255: raw
     float v[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {

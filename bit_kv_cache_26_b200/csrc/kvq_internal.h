@@ -23,6 +23,13 @@ cudaError_t launch_decode(const Geom& g, const void* q, int Hq, float sm_scale, 
 cudaError_t launch_decode_mma(const Geom& g, const void* q, int Hq, float scale_log2, int nsplit, float* ml,
                               float* o, int* arrivals, float* out, cudaStream_t st);
 size_t decode_mma_smem(const Geom& g, int Hq);
+// decode step: one-token append + decode in one launch (the workspace's counters reset themselves)
+size_t step_workspace(const Geom& g, int Hq, int nsplit);
+cudaError_t launch_decode_step(const Geom& g, const void* k_new, const void* v_new, const void* q, int Hq,
+                               float sm_scale, float* out, void* ws, int nsplit, cudaStream_t st);
+cudaError_t launch_decode_step_mma(const Geom& g, const void* k_new, const void* v_new, const void* q, int Hq,
+                                   float scale_log2, int nsplit, float* ml, float* o, int* arrivals, int* seqcnt,
+                                   float* out, cudaStream_t st);
 int decode_mma_splits(const Geom& g, int Hq, int num_sms);
 
 // dequantize (kvq_dequant.cu)

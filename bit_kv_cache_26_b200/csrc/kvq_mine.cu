@@ -29,6 +29,8 @@ struct MineWs {
   int32_t* assign;  // [NP][n]
   float* xsq;       // [NP][n] |x|^2 of every token (the tcgen05 assignment's cache)
   int32_t* amb;     // [NP][n] tokens the tcgen05 assignment left undecided
+  uint32_t* ambc;   // [NP][n][2] their candidate patterns (8 bytes: up to 8 indices)
+  uint8_t* ambn;    // [NP][n] candidates listed (255: more than 8, every pattern is checked)
   int32_t* amb_cnt; // [NP]
   float* y;         // [NP][n][128] (transform only)
   double* v64;      // [NP][n][128] (transform only)
@@ -64,6 +66,8 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   else { w.assign = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t)); }
   w.xsq = (float*)p; p += align256((size_t)NP * n * sizeof(float));
   w.amb = (int32_t*)p; p += align256((size_t)NP * n * sizeof(int32_t));
+  w.ambc = (uint32_t*)p; p += align256((size_t)NP * n * 2 * sizeof(uint32_t));
+  w.ambn = (uint8_t*)p; p += align256((size_t)NP * n);
   w.amb_cnt = (int32_t*)p; p += align256((size_t)NP * sizeof(int32_t));
   if (transform) {
     w.y = (float*)p; p += align256((size_t)NP * n * kD * sizeof(float));
@@ -694,8 +698,15 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
   __syncthreads();
 
   if (warp == kAccWarps) {
-    // ---- producer: rows of tile k into stage k % kStages once every consumer left it
+    // ---- producer: rows of tile k into stage k % kStages once every consumer left it.  The
+    // tile's assignments are loaded one tile ahead (their latency overlaps the previous tile).
     int last = -1;  // newest tile whose copy was issued
+    int aj_next[kAccT / 32];
+#pragma unroll
+    for (int q = 0; q < kAccT / 32; ++q) {
+      const int64_t i = (int64_t)(k0 * kAccT) + 32 * q + lane;
+      aj_next[q] = i < s.n ? __ldg(a + i) : -1;
+    }
     for (int k = 0; k < nt; ++k) {
       const int st = k % kStages;
       bool ok = true;
@@ -710,8 +721,9 @@ __global__ void __launch_bounds__((kAccWarps + 1) * 32, accum_ctas_per_sm<CPW, E
       int aj[kAccT / 32], pos[kAccT / 32];
 #pragma unroll
       for (int q = 0; q < kAccT / 32; ++q) {
-        const int64_t i = (int64_t)tb + 32 * q + lane;
-        aj[q] = i < s.n ? __ldg(a + i) : -1;
+        aj[q] = aj_next[q];
+        const int64_t i = (int64_t)tb + kAccT + 32 * q + lane;  // the next tile's rows
+        aj_next[q] = (k + 1 < nt && i < s.n) ? __ldg(a + i) : -1;
       }
       for (int i = lane; i < P; i += 32) counts[i] = 0;
       __syncwarp();
@@ -996,6 +1008,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
                                                                       int32_t* __restrict__ assign,
                                                                       float* __restrict__ xsq_cache, int first,
                                                                       int32_t* __restrict__ amb,
+                                                                      uint32_t* __restrict__ ambc,
+                                                                      uint8_t* __restrict__ ambn,
                                                                       int32_t* __restrict__ amb_cnt, int nst,
                                                                       int32_t* __restrict__ status) {
   const int prob = blockIdx.y;
@@ -1206,11 +1220,47 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
       const float nx = sqrtf(xs) * (1.0f + 1e-6f);
       const float Eb = 0x1p-12f * nx * nm_max + 0x1p-20f * (xs + msq_max);
       const float Pe = 0x1p-16f * (msq_max + 2.0f * nx * nm_max);  // largest tag move of e = 2 u
-      if (valid) {
-        if (2.0f * (m2 - m1) > 2.0f * Eb + 2.0f * Pe + 1e-9f * (xs + msq_max))
-          assign[(size_t)prob * s.n + i] = (int32_t)(__float_as_uint(m1) & 127u);
-        else
-          amb[(size_t)prob * s.n + atomicAdd(amb_cnt + prob, 1)] = (int32_t)i;
+      const float dl = 1e-9f * (xs + msq_max);
+      const bool und = valid && !(2.0f * (m2 - m1) > 2.0f * Eb + 2.0f * Pe + dl);
+      if (valid && !und) assign[(size_t)prob * s.n + i] = (int32_t)(__float_as_uint(m1) & 127u);
+      if (__any_sync(kFull, und)) {
+        // undecided: list the patterns that can still be the float64 argmin, those whose tagged
+        // score is within m1 + Eb + Pe + dl (the score error, the tag move and the float64
+        // rounding allowance, each counted on both sides), from a second pass over the columns
+        float thr = m1 + Eb + Pe + dl;
+        thr += fabsf(thr) * 0x1p-20f;  // the roundings of the sum above
+        uint32_t c0w = 0u, c1w = 0u;
+        int cnt = 0;
+        for (int c0 = 0; c0 < Pn; c0 += 8) {
+          tmem_ld8_issue(taddr + c0, hv);
+          tmem_ld8_issue(taddr + Pn + c0, mv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 8; q += 4) {
+            const float4 hq = *reinterpret_cast<const float4*>(hm + c0 + q);
+            float s0, s1, s2, s3, u[4];
+            add2f(hv[q], hv[q + 1], mv[q], mv[q + 1], s0, s1);
+            add2f(hv[q + 2], hv[q + 3], mv[q + 2], mv[q + 3], s2, s3);
+            sub2(hq.x, hq.y, s0, s1, u[0], u[1]);
+            sub2(hq.z, hq.w, s2, s3, u[2], u[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = c0 + q + e;
+              if (und && j < P && tag_score(u[e], j) <= thr) {
+                if (cnt < 4) c0w |= (uint32_t)j << (8 * cnt);
+                else if (cnt < 8) c1w |= (uint32_t)j << (8 * (cnt - 4));
+                ++cnt;
+              }
+            }
+          }
+        }
+        if (und) {
+          const size_t r = (size_t)prob * s.n + atomicAdd(amb_cnt + prob, 1);
+          amb[r] = (int32_t)i;
+          ambc[2 * r] = c0w;
+          ambc[2 * r + 1] = c1w;
+          ambn[r] = (uint8_t)(cnt > 8 ? 255 : cnt);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -1224,115 +1274,64 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tcols) : "memory");
 }
 
-// Tokens the tcgen05 assignment listed as undecided (P <= 128).  A warp takes one token at a
-// time (tokens r = its global warp index, r + all warps, ...), with no block barrier in the
-// loop.  fp32 scores e_j = |m_j|^2 - 2 x.m_j for every pattern (lane l: patterns l + 32 q,
-// an in-order fp32 FMA chain over the channels) are within E_j = 2^-15 |x| |m_j| +
-// 2^-22 (|x|^2 + |m_j|^2) of the exact values (a 128-term fp32 dot product is off by at most
-// 128 2^-24 |x| |m_j|, plus the roundings of |m_j|^2 and of e), so the float64 argmin can
-// only be a pattern with e_j - E_j <= min_k (e_k + E_k) + delta (delta: the float64
-// rounding allowance), and only those candidates (about two) get the float64 squared distance
-// in channel order, as the sequential definition; the lowest index wins among equal
-// distances.  The patterns are staged once per block in shared memory (rows padded to 129
-// floats: lane l reads row l without bank conflicts); their float64 values come from the
-// integer construction of f32_scaled and one exact multiply.
-constexpr int kFixLd = kD + 1;
+// Tokens the tcgen05 assignment left undecided, with the candidate patterns its epilogue
+// listed (P <= 128): a lane per (token, candidate) computes the float64 squared distance exactly
+// as the sequential definition (channels 0..127 in order, no fused multiply-add), and the eight
+// lanes of a token keep the smallest (lowest index among equal distances).  A warp takes four
+// tokens at a time; a token with more than eight candidates has its eight lanes check every
+// pattern instead.  The float64 row of the input is built from its bits (f32_scaled) and one exact
+// multiply, as in the cluster sums.
 constexpr int kFixWarps = 8;
 __global__ void __launch_bounds__(kFixWarps * 32) mine_fixup_kernel(Src s, int P, const float* __restrict__ M,
                                                                     const int32_t* __restrict__ amb,
+                                                                    const uint32_t* __restrict__ ambc,
+                                                                    const uint8_t* __restrict__ ambn,
                                                                     const int32_t* __restrict__ amb_cnt,
                                                                     int32_t* __restrict__ assign) {
-  extern __shared__ float Ms[];  // [P][kFixLd]
-  __shared__ float mn2[128], mnrm[128];
-  __shared__ float xs[kFixWarps][kD];
-  __shared__ double xd[kFixWarps][kD];
   const int prob = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok = lane >> 3, slot = lane & 7;  // token tok of the warp's four, candidate `slot`
   const int count = amb_cnt[prob];
-  if ((int)blockIdx.x * kFixWarps >= count) return;  // uniform across the block
   const float* Mp = M + (size_t)prob * P * kD;
-  // 16-byte loads, eight in flight per thread, stored into the padded rows
-  const float4* M4 = reinterpret_cast<const float4*>(Mp);
-  for (int i0 = threadIdx.x; i0 < P * (kD / 4); i0 += 8 * blockDim.x) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * blockDim.x;
-      v[u] = i < P * (kD / 4) ? __ldg(M4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * blockDim.x;
-      if (i < P * (kD / 4)) {
-        float* dst = Ms + (i / (kD / 4)) * kFixLd + 4 * (i % (kD / 4));
-        dst[0] = v[u].x; dst[1] = v[u].y; dst[2] = v[u].z; dst[3] = v[u].w;
-      }
-    }
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < P; j += blockDim.x) {
-    double acc = 0.0;
-    for (int c = 0; c < kD; ++c) {
-      const double m = Ms[j * kFixLd + c];
-      acc = fma(m, m, acc);
-    }
-    mn2[j] = (float)acc;
-    mnrm[j] = (float)(sqrt(acc) * (1.0 + 1e-6));
-  }
-  __syncthreads();
-  for (int r = blockIdx.x * kFixWarps + warp; r < count; r += gridDim.x * kFixWarps) {
-    const int64_t i = amb[(size_t)prob * s.n + r];
-    float xx = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float v = s.at(prob, i, lane + 32 * k);
-      xs[warp][lane + 32 * k] = v;
-      xd[warp][lane + 32 * k] = (double)v;
-      xx = fmaf(v, v, xx);
-    }
-    xx = warp_sum(xx) * (1.0f + 1e-5f);
-    const float nx = sqrtf(xx) * (1.0f + 1e-5f);
-    __syncwarp();
-    float e[4], E[4];
-    float U = INFINITY;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = lane + 32 * q;
-      e[q] = INFINITY;
-      E[q] = 0.f;
-      if (j < P) {
-        const float* mr = Ms + j * kFixLd;
-        float dot = 0.f;
-#pragma unroll 8
-        for (int c = 0; c < kD; ++c) dot = fmaf(xs[warp][c], mr[c], dot);
-        e[q] = mn2[j] - 2.0f * dot;
-        E[q] = 0x1p-15f * nx * mnrm[j] + 0x1p-22f * (xx + mn2[j]);
-        U = fminf(U, e[q] + E[q]);
-      }
-    }
-    U = warp_min(U);
+  const int set = prob / s.heads, h = prob % s.heads;
+  for (int r0 = (blockIdx.x * kFixWarps + warp) * 4; r0 < count; r0 += gridDim.x * kFixWarps * 4) {
+    const int r = r0 + tok;
+    const bool act = r < count;
+    const size_t ra = (size_t)prob * s.n + (act ? r : 0);
+    const int64_t i = act ? amb[ra] : 0;
+    const int nc = act ? (int)ambn[ra] : 0;
+    const uint32_t cw = act ? ambc[2 * ra + (slot >> 2)] : 0u;
+    const uint16_t* xrow = s.x + set * s.ss + i * s.ts + h * s.hs;
     double bd = INFINITY;
     int bj = 1 << 30;
+    // the candidates of this lane: its slot, or (more than eight) every eighth pattern
+    const int njobs = nc == 255 ? (P - slot + 7) / 8 : (slot < nc ? 1 : 0);
+    for (int q = 0; q < njobs; ++q) {
+      const int j = nc == 255 ? slot + 8 * q : (int)((cw >> (8 * (slot & 3))) & 0xffu);
+      const float* m = Mp + (size_t)j * kD;
+      double acc = 0.0;
+#pragma unroll 4
+      for (int d = 0; d < kD; d += 8) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(xrow + d));
+        const float4 ma = __ldg(reinterpret_cast<const float4*>(m + d));
+        const float4 mb = __ldg(reinterpret_cast<const float4*>(m + d + 4));
+        const uint32_t xw[4] = {u.x, u.y, u.z, u.w};
+        const float mv[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = lane + 32 * q;
-      if (j < P && e[q] - E[q] <= U + 1e-9f * (xx + mn2[j])) {
-        const uint32_t* mrow = reinterpret_cast<const uint32_t*>(Ms + j * kFixLd);
-        double d = 0.0;
-        for (int c = 0; c < kD; ++c) {
-          const double t = __dsub_rn(xd[warp][c], __dmul_rn(f32_scaled(mrow[c]), 0x1p896));
-          d = __dadd_rn(d, __dmul_rn(t, t));
+        for (int e = 0; e < 8; ++e) {
+          const float xv = bits_to_float((uint16_t)((e & 1) ? (xw[e >> 1] >> 16) : (xw[e >> 1] & 0xffffu)), s.dtype);
+          const double t = __dsub_rn((double)xv, (double)mv[e]);
+          acc = __dadd_rn(acc, __dmul_rn(t, t));
         }
-        if (d < bd) { bd = d; bj = j; }  // q ascending: the lowest index of this lane wins ties
       }
+      if (acc < bd || (acc == bd && j < bj)) { bd = acc; bj = j; }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
+    for (int off = 4; off > 0; off >>= 1) {
       const double od = __shfl_xor_sync(kFull, bd, off);
       const int oj = __shfl_xor_sync(kFull, bj, off);
       if (od < bd || (od == bd && oj < bj)) { bd = od; bj = oj; }
     }
-    if (lane == 0) assign[(size_t)prob * s.n + i] = bj;
-    __syncwarp();
+    if (act && slot == 0) assign[(size_t)prob * s.n + i] = bj;
   }
 }
 
@@ -1374,7 +1373,8 @@ size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
   const int NP = sets * heads;
   size_t b = 256 + align256((size_t)NP * P * kD * sizeof(double)) + align256((size_t)NP * P * sizeof(uint32_t)) +
              align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * (size_t)n * sizeof(float)) +
-             align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * sizeof(int32_t));
+             align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * (size_t)n * 8) +
+             align256((size_t)NP * (size_t)n) + align256((size_t)NP * sizeof(int32_t));
   if (transform)
     b += align256((size_t)NP * n * kD * sizeof(float)) + align256((size_t)NP * n * kD * sizeof(double)) +
          align256((size_t)NP * fit_chunks(n) * kD * sizeof(double)) + 4 * align256((size_t)NP * kD * sizeof(double)) +
@@ -1490,19 +1490,16 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
       return e;
     if ((e = make_x_map(a, &xmap, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
-  const size_t fix_smem = (size_t)a.P * kFixLd * sizeof(float);
-  if (use_tc && (e = cudaFuncSetAttribute(mine_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)fix_smem)) != cudaSuccess)
-    return e;
   const unsigned tc_ctas = (unsigned)std::max<int64_t>(
       1, std::min<int64_t>((a.n + kTcM - 1) / kTcM, (int64_t)std::max(1, (a.P <= 64 ? 2 : 1) * sms / NP)));
   for (int it = 0; it < a.iters; ++it) {
     const dim3 ag(mma_ctas, NP);
     if (use_tc) {
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
-          xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.amb_cnt, mine_tc_stages(a.P), w.status);
-      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 4 * sms / NP), NP), kFixWarps * 32, fix_smem, st>>>(
-          s, a.P, a.patterns, w.amb, w.amb_cnt, w.assign);
+          xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.ambc, w.ambn, w.amb_cnt, mine_tc_stages(a.P),
+          w.status);
+      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 2 * sms / NP), NP), kFixWarps * 32, 0, st>>>(
+          s, a.P, a.patterns, w.amb, w.ambc, w.ambn, w.amb_cnt, w.assign);
     } else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
     else if (use_mma && KIND == 1)

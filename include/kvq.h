@@ -159,12 +159,25 @@ typedef struct kvq_cache {
   const int32_t* page_table;  /* [num_seqs][max_pages_per_seq] physical page ids */
   int32_t* seq_len;           /* [num_seqs] tokens held per sequence (updated by append) */
   void* k_tail;               /* [num_seqs][num_kv_heads][32][128] dtype */
-  const float* k_patterns;    /* [num_sets][num_kv_heads][P][128] fp32 */
-  const float* v_patterns;    /* [num_sets][num_kv_heads][P][128] fp32 */
+  const float* k_patterns;    /* [num_sets][num_kv_heads][P][128] fp32 (kvq_decode_step with pattern insertion
+                                 writes rows pattern_counts[..] .. P - 1; nothing else writes them) */
+  const float* v_patterns;    /* [num_sets][num_kv_heads][P][128] fp32 (same) */
   const int32_t* seq_to_set;  /* [num_seqs] pattern set of each sequence, or NULL (all set 0) */
   const float* k_colscale;    /* [num_sets][num_kv_heads][128] fp32; transform only, else NULL */
   const float* v_colscale;    /* [num_sets][num_kv_heads][128] fp32; transform only, else NULL */
   int32_t* status;            /* one int32, device-side error bits (KVQ_DEV_*); caller zeroes it */
+  /* Decode-time pattern insertion ([PKV] Section 3.1 "Decoding Stage", Eq. 5); all optional. */
+  int32_t* pattern_counts;    /* [num_sets][num_kv_heads] patterns in use per set, 1..num_patterns (the rest
+                                 of the P rows are capacity), or NULL: every set uses num_patterns */
+  float* pattern_window;      /* [num_seqs][num_kv_heads][4][128] fp32: running minimum and maximum of the K
+                                 vectors, then of the V vectors, of the current window; the caller sets them to
+                                 +inf / -inf before the first step.  NULL unless pattern_window_len > 0 */
+  int32_t pattern_window_len; /* G_pattern: each time a sequence's length reaches a multiple of it during
+                                 kvq_decode_step, the window's Chebyshev centers fl32(fl32(min + max) * 0.5)
+                                 become the next K and V pattern of the sequence's set (while its count is
+                                 below num_patterns) and the window restarts.  0 = off.  Needs
+                                 pattern_counts, and sequences that do not share a pattern set. */
+  int32_t reserved;           /* must be 0 */
 } kvq_cache;
 
 /* rho*(d, alpha) of [PKV] Eq. 10 rounded to fp32: the root in (0, 1) of
@@ -264,6 +277,29 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, i
 #define KVQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 KVQ_API kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, int32_t num_q_heads,
                                                float sm_scale, float* out, kvq_stream_t stream);
+
+/*
+ * kvq_decode_step -- one step of decoding in a single launch: kvq_quantize_append of one new
+ * token per sequence (n_new = 1) followed by kvq_decode_attention over every token including it
+ * ([PKV] Section 3.4: the fused decode kernels; Section 3.2 / Eq. 6 and Eq. 1 for the append;
+ * Section 3.3 for V).  With cache->pattern_window_len > 0 the step also runs the decode-time
+ * pattern insertion of [PKV] Section 3.1, Eq. 5 (see kvq_cache).
+ *   k_new, v_new  [num_seqs][num_kv_heads][128] dtype: the new token's key and value
+ *   q             [num_seqs][num_q_heads][128] dtype;  out [num_seqs][num_q_heads][128] fp32
+ * Same results (page bytes, K tail, seq_len, out) as the two calls in a row.  The new key and
+ * value are assigned among the patterns in use (a brute-force exact min-max argmin: one token per
+ * sequence and head); when the token completes a page, the page's 32 keys are assigned and
+ * quantized in the same launch.  A sequence whose page table is full, or whose next page id is
+ * invalid, flags KVQ_DEV_OVERFLOW / KVQ_DEV_BAD_PAGE, appends nothing and is decoded as it was.
+ * Workspace: kvq_step_workspace_bytes(), 256-byte aligned, ZERO-FILLED before its first use:
+ * besides the split partials it holds counters that every call leaves at zero again (no memset
+ * per step, so a step can be captured in a CUDA graph as one kernel node).  Two steps in flight
+ * at once on one workspace race.
+ */
+KVQ_API size_t kvq_step_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads);
+KVQ_API kvq_status kvq_decode_step(const kvq_cache* cache, const void* k_new, const void* v_new, const void* q,
+                                   int32_t num_q_heads, float sm_scale, float* out, void* ws, size_t ws_bytes,
+                                   kvq_stream_t stream);
 
 /*
  * kvq_dequantize -- reconstruct tokens [start, start+count) of sequence `seq`
