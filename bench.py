@@ -13,8 +13,10 @@ pre-transform), and the long chain-of-thought loop is timed per decode step (`pe
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME] [--bits 2|4]
 
-Multi-GPU (torchrun): every rank runs its own batch (different seed); there is no data-path
-collective, the step time is the max over ranks, and value counts all ranks' tokens (weak scaling).
+Multi-GPU (torchrun): the batch's samples are sharded over the ranks (contiguous shards of the
+same job); each rank mines, appends and decodes its shard, each step ends with an all-gather of
+the decode outputs (NCCL), the step time is the max over ranks and value counts the whole job's
+tokens (strong scaling: the total work is fixed).
 """
 from __future__ import annotations
 
@@ -194,9 +196,11 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def rank_workload(base, rank: int):
-    """The batch rank `rank` processes: same shape, its own seed (batch-sharded replicas, weak scaling)."""
-    return base.with_(seed=base.seed + 1000 * rank)
+def rank_shard(base, rank: int, world: int):
+    """The sequences [b0, b1) of the job that rank `rank` processes (batch sharding: the samples
+    are independent; total work fixed, strong scaling)."""
+    from bit_kv_cache_26_b200.shard import shard_range
+    return shard_range(base.B, rank, world)
 
 
 def max_over_ranks(values, device=None):
@@ -215,7 +219,9 @@ def workload_config(w, args):
     return {"workload": w.name, "batch": w.B, "context": w.S, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": D,
             "patterns": w.P, "lloyd_iters": w.iters, "bits": w.bits, "group": 32,
             "transform": "hadamard+varnorm" if w.transform else "none",
-            "input_dtype": "bf16" if w.dtype == 1 else "fp16", "parallelism": f"replica x{args.gpus} (batch-sharded)",
+            "input_dtype": "bf16" if w.dtype == 1 else "fp16",
+            "parallelism": "single GPU" if args.gpus == 1 else
+            f"batch-sharded x{args.gpus} (independent samples, per-rank patterns, decode outputs all-gathered)",
             "l2": f"inputs larger than L2 ({w.B * w.S * w.Hkv * D * 4 / 2**30:.1f} GiB of K/V per step, 126 MB L2)",
             "v_threshold_alpha": w.v_alpha}
 
@@ -239,18 +245,23 @@ def launches_per_step(w, full_pages: bool) -> int:
     return 2 * mine + (4 if full_pages else 3) + 1
 
 
-def measure_path(w, args, dev, world: int, rank: int, headline: bool):
+def measure_path(w, args, dev, world: int, rank: int, headline: bool, shard=None):
     """Time `args.steps` steps of the whole path on workload w (mine K and V patterns on the
     pooled prefill, quantize-append the whole context into a reset cache, one decode step).
-    Returns the record (and, for the headline, the end-to-end measurement through host buffers)."""
+    With `shard` = (b0, b1) this rank runs sequences [b0, b1) of w and each step ends with the
+    all-gather of the decode outputs of every rank (NCCL).  Returns the record (and, for the
+    headline, the end-to-end measurement through host buffers)."""
     import numpy as np
     import torch
 
     import bit_kv_cache_26_b200 as kvq
     import synth
 
-    k, v = synth.gen_kv(w)
-    q = synth.gen_q(w)
+    B_total = w.B
+    b0, b1 = shard if shard else (0, w.B)
+    k, v = synth.gen_kv(w, b0=b0, b1=b1)
+    q = synth.gen_q(w, b0=b0, b1=b1)
+    w = w.with_(B=b1 - b0)
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
 
     def pinned(a):
@@ -280,6 +291,9 @@ def measure_path(w, args, dev, world: int, rank: int, headline: bool):
         kvq.kvq_quantize_append(cache.c, kx, vx, w.S, ws_a)
         if ev: ev[2].record()
         kvq.kvq_decode_attention(cache.c, qx, w.Hq, D ** -0.5, out, ws_d)
+        if world > 1:
+            from bit_kv_cache_26_b200.shard import gather_outputs
+            gather_outputs(out, B_total)
         if ev: ev[3].record()
 
     def barrier():
@@ -368,7 +382,7 @@ def measure_path(w, args, dev, world: int, rank: int, headline: bool):
     dom = rooflines[dominant]
     roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],
                 "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dominant, "peak_source": pk["source"]}
-    tokens = n * world
+    tokens = B_total * w.S
     rec = {"workload": w.name, "bits": w.bits, "transform": bool(w.transform), "value": tokens / (ms_per_step * 1e-3),
            "unit": "KV-tokens/s", "ms_per_step": ms_per_step,
            "phases_ms": {"mine_patterns_KV": mine_ms, "quantize_append": append_ms, "decode_attention": decode_ms},
@@ -548,8 +562,9 @@ def main():
     base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
     if args.batch:
         base = base.with_(B=args.batch)
-    w = rank_workload(base, rank)
-    rec, e2e, clk = measure_path(w, args, dev, world, rank, headline=True)
+    w = base
+    shard = rank_shard(base, rank, world) if world > 1 else None
+    rec, e2e, clk = measure_path(w, args, dev, world, rank, headline=True, shard=shard)
 
     per_config = []
     if world == 1 and not args.no_per_config and not args.batch:
@@ -568,7 +583,8 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": rec["value"], "unit": "KV-tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+            "scaling": "strong" if world > 1 else "weak",
             "vs_baseline": None, "dtype": "f32 (fp32 quantization, f64 mining distances, bf16 inputs)",
             "data": "synthetic (seeded Gaussian-mixture K/V with outlier channels and RoPE)",
             "config": workload_config(w, args),
@@ -576,7 +592,7 @@ def main():
             "decode_hbm_gbs": rec["decode_hbm_gbs"], "quant_append_gbs": rec["quant_append_gbs"],
             "v_pattern_utilisation": rec["v_pattern_utilisation"],
             "roofline": rec["roofline"], "rooflines": rec["rooflines"],
-            "e2e": {"value": w.B * w.S * world / (e2e["ms"] / args.steps * 1e-3), "unit": "KV-tokens/s",
+            "e2e": {"value": w.B * w.S / (e2e["ms"] / args.steps * 1e-3), "unit": "KV-tokens/s",
                     "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]},
             "gpu_launches": rec["gpu_launches"],
             "clocks": clk,

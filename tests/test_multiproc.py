@@ -1,5 +1,6 @@
-"""The N > 1 path of bench.py on CPU: two gloo ranks (no GPU).  Each rank gets its own
-batch (distinct seeds, same shape) and the reported time is the maximum over ranks."""
+"""The N > 1 path of bench.py on CPU: two gloo ranks (no GPU).  The batch is sharded over the
+ranks (contiguous shards of the same job's samples), each step's decode outputs are all-gathered,
+and the reported time is the maximum over ranks."""
 import os
 import socket
 
@@ -28,12 +29,21 @@ def _worker(rank, world, port, out):
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
-    base = synth.WORKLOADS["llama3_8b_32k"]
-    w = bench.rank_workload(base, rank)
-    k, _ = synth.gen_kv(w.with_(B=1, S=8), want_v=False)
+    import torch
+
+    from bit_kv_cache_26_b200.shard import gather_outputs
+    base = synth.WORKLOADS["breadth_256x16k"].with_(B=5, S=8)
+    b0, b1 = bench.rank_shard(base, rank, world)
+    k, _ = synth.gen_kv(base, b0=b0, b1=b1, want_v=False)
+    # the shard is exactly those samples of the whole job
+    kall, _ = synth.gen_kv(base, want_v=False)
+    assert (k == kall[b0:b1]).all()
     elapsed = [10.0 * (rank + 1), 3.0 - rank]
     got = bench.max_over_ranks(elapsed)
-    out.put((rank, w.seed, int(k.sum()), w.B, w.S, got))
+    # decode outputs: rank r contributes rows b0..b1 filled with their sequence index
+    local = torch.arange(b0, b1, dtype=torch.float32)[:, None, None].expand(b1 - b0, 2, 4).contiguous()
+    full = gather_outputs(local, base.B)
+    out.put((rank, b0, b1, int(k.sum()), full[:, 0, 0].tolist(), got))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -49,10 +59,21 @@ def test_two_gloo_ranks_shard_and_take_the_max():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, s0, k0, B0, S0, g0), (r1, s1, k1, B1, S1, g1) = res
-    assert s0 != s1 and k0 != k1            # different batches
-    assert (B0, S0) == (B1, S1)              # same per-rank work (weak scaling)
-    assert g0 == g1 == [20.0, 3.0]           # max over ranks, seen identically by both
+    (r0, a0, e0, k0, f0, g0), (r1, a1, e1, k1, f1, g1) = res
+    assert (a0, e0, a1, e1) == (0, 3, 3, 5)           # contiguous shards, sizes differ by at most one
+    assert f0 == f1 == [0.0, 1.0, 2.0, 3.0, 4.0]      # every rank holds the whole batch's output
+    assert g0 == g1 == [20.0, 3.0]                    # max over ranks, seen identically by both
+
+
+def test_shard_ranges_cover_the_batch():
+    from bit_kv_cache_26_b200.shard import shard_range
+    for B in (0, 1, 7, 256):
+        for world in (1, 2, 3, 8):
+            parts = [shard_range(B, r, world) for r in range(world)]
+            assert parts[0][0] == 0 and parts[-1][1] == B
+            assert all(parts[i][1] == parts[i + 1][0] for i in range(world - 1))
+            sizes = [b1 - b0 for b0, b1 in parts]
+            assert max(sizes) - min(sizes) <= 1
 
 
 def test_single_process_max_is_identity():

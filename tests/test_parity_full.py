@@ -1,8 +1,9 @@
 """GPU parity at the workloads' full sizes, on sampled outputs the oracle computes one by
-one: the bench workload (llama3_8b_32k, 2- and 4-bit), the Qwen-shaped 128K workload with
-and without the pre-transform, the breadth workload (per-sample perturbed centers; 32 of its
-256 samples, each at the full 16K context) and the long chain-of-thought decode loop (8K
-prefill, then 4096 one-token appends, each followed by decode attention).
+one: the Llama-shaped workload (llama3_8b_32k, 2- and 4-bit), the Qwen-shaped 128K workload
+with and without the pre-transform, the breadth workload (all 256 samples with per-sample
+perturbed centers, each at the full 16K context: the launched grids are the benchmark's) and
+the long chain-of-thought decode loop (8K prefill, then 4096 decode steps, each one
+kvq_decode_step launch: a one-token append and decode attention).
 
 Per case: mining of one KV head (K and V) against the oracle's Lloyd on the same pooled
 prefill; page bytes, pattern indices and the K tail of sampled (sequence, KV head) units
@@ -71,7 +72,7 @@ FULL = {
     "llama3_8b_32k_4bit": W["llama3_8b_32k"].with_(bits=4),
     "qwen25_7b_128k": W["qwen25_7b_128k"],
     "qwen25_7b_128k_transform": W["qwen25_7b_128k"].with_(transform=1),
-    "breadth_32of256x16k": W["breadth_256x16k"].with_(B=32),
+    "breadth_256x16k": W["breadth_256x16k"],
 }
 
 
@@ -97,8 +98,9 @@ def test_full_size_prefill_and_decode(name):
 
 
 def test_long_cot_decode_loop():
-    """8192-token prefill, patterns mined once and frozen, then 4096 steps of a one-token
-    append per sequence followed by decode attention (queries change every step)."""
+    """8192-token prefill, patterns mined once and frozen, then 4096 decode steps, each one
+    kvq_decode_step launch (a one-token quantize-append per sequence and decode attention with a
+    new query), as the benchmark runs them."""
     import bit_kv_cache_26_b200 as kvq
     w = W["long_cot_8k"]
     total = w.S + w.steps
@@ -109,14 +111,13 @@ def test_long_cot_decode_loop():
     cache.append(kt[:, :w.S].contiguous(), vt[:, :w.S].contiguous())
     MK, MV, cK, cV = _patterns(cache, w)
     _check_mining_head(w, k[:, :w.S], v[:, :w.S], w.Hkv - 1, MK, MV, cK, cV)
-    ws = cache.decode_workspace(w.Hq)
+    ws = cache.step_workspace(w.Hq)
     out = torch.empty(w.B, w.Hq, D, device="cuda")
     check_at = {0, 31, 1000, w.steps - 1}
     units = ((0, 0), (w.B - 1, w.Hkv - 1))
     for t in range(w.steps):
-        cache.append(kt[:, w.S + t:w.S + t + 1].contiguous(), vt[:, w.S + t:w.S + t + 1].contiguous())
         q = synth.gen_q(w, step=t)
-        cache.decode(to_torch(q, w.dtype), out, ws)
+        cache.step(kt[:, w.S + t].contiguous(), vt[:, w.S + t].contiguous(), to_torch(q, w.dtype), out, ws)
         if t in check_at:
             got = out.cpu().numpy()
             for b, h in units:
