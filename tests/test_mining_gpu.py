@@ -30,7 +30,12 @@ def _bf16(a):
     return u.astype(np.uint32).view(np.float32)
 
 
-def planted_ties(n: int, P: int, seed: int):
+def _round16(a, fp16: bool):
+    """float -> nearest value of the 16-bit input type (fp16 or bf16), as float32."""
+    return np.asarray(a, np.float32).astype(np.float16).astype(np.float32) if fp16 else _bf16(a)
+
+
+def planted_ties(n: int, P: int, seed: int, fp16: bool = False):
     """n bf16 rows whose strided-initial patterns (rows floor(j n / P)) come in pairs (2i, 2i+1):
     even pairs are one-channel twins (equal except channel d0, 1.0 vs 1.5), odd pairs differ by
     N(0, 0.3^2) noise.  Other rows: 10 % exact ties between twins (channel d0 at the midpoint
@@ -48,7 +53,7 @@ def planted_ties(n: int, P: int, seed: int):
             pats[j, d0[i]] = 1.5 if j % 2 else 1.0
         elif j % 2:
             pats[j] += rng.standard_normal(D) * 0.3
-    pats = _bf16(pats)
+    pats = _round16(pats, fp16)
     x = np.zeros((n, D), np.float32)
     for r in range(n):
         i = int(rng.integers(0, npair))
@@ -62,7 +67,7 @@ def planted_ties(n: int, P: int, seed: int):
         else:
             t = 0.5 + rng.standard_normal() * 10 ** rng.uniform(-5, -1)
             v = a + t * (b - a) + rng.standard_normal(D) * 0.05
-        x[r] = _bf16(v)
+        x[r] = _round16(v, fp16)
     for j in range(P):
         x[(j * n) // P] = pats[j]
     return x
@@ -82,7 +87,7 @@ def _to_dev(x32: np.ndarray, dtype):
 @pytest.mark.parametrize("iters", [1, 4])
 def test_planted_near_ties_bit_exact(P, n, dtype, iters):
     import bit_kv_cache_26_b200 as kvq
-    x = planted_ties(n, P, seed=P + n)
+    x = planted_ties(n, P, seed=P + n, fp16=dtype == torch.float16)
     xd = _to_dev(x, dtype)
     pats, _, asg = kvq.mine(xd, P, iters, want_assign=True)
     M, a = oracle.mine(x, P, iters)
