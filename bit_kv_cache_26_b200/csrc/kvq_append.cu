@@ -188,10 +188,13 @@ __device__ __forceinline__ unsigned long long dkey(float d, int j) {
 // from a multiply by the correctly rounded reciprocal (error below 2^-19 for quotients below
 // 16), rounded to an integer by adding 1.5 * 2^23 (the integer is then the low mantissa
 // bits); a quotient within 1e-5 of a rounding boundary is recomputed with the correctly
-// rounded division.  R >= z and the quotient stays below maxc + 2^-19, so no clamp is
-// needed; s == 0 gives rinv == 0 and code 0.
+// rounded division.  R >= z and, for a normal scale, the quotient stays below maxc + 2^-19;
+// the division's result is clamped to maxc (a subnormal scale carries less precision); s == 0
+// gives rinv == 0 and code 0.
+template <int BITS>
 __device__ __forceinline__ uint32_t code_pair(float R0, float R1, float z0, float z1, float ri0, float ri1,
                                               const float* s2) {
+  constexpr float kMaxc = (float)((1 << BITS) - 1);
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   float t0, t1, u0, u1, v0, v1, b0, b1, e0, e1;
   sub2(R0, R1, z0, z1, t0, t1);
@@ -199,9 +202,12 @@ __device__ __forceinline__ uint32_t code_pair(float R0, float R1, float z0, floa
   add2f(u0, u1, kShift, kShift, v0, v1);
   sub2(v0, v1, kShift, kShift, b0, b1);
   sub2(u0, u1, b0, b1, e0, e1);  // u - rne(u), exact
-  if (fmaxf(fabsf(e0), fabsf(e1)) > 0.5f - 1e-5f) {
-    if (fabsf(e0) > 0.5f - 1e-5f) v0 = __fadd_rn(rintf(__fdiv_rn(t0, s2[0])), kShift);
-    if (fabsf(e1) > 0.5f - 1e-5f) v1 = __fadd_rn(rintf(__fdiv_rn(t1, s2[1])), kShift);
+  // near a rounding boundary, or not finite (a scale so small that 1/s overflows): the
+  // correctly rounded division; the comparisons are written so that NaN selects it
+  const bool f0 = !(fabsf(e0) <= 0.5f - 1e-5f), f1 = !(fabsf(e1) <= 0.5f - 1e-5f);
+  if (f0 || f1) {
+    if (f0) v0 = __fadd_rn(fminf(rintf(__fdiv_rn(t0, s2[0])), kMaxc), kShift);
+    if (f1) v1 = __fadd_rn(fminf(rintf(__fdiv_rn(t1, s2[1])), kMaxc), kShift);
   }
   return __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410) & 0x00FF00FFu;
 }
@@ -224,7 +230,7 @@ __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const
     const int gi = (ch >> 5) * kG + tok;
     const float2 z = *reinterpret_cast<const float2*>(vz + gi);
     const float2 ri = *reinterpret_cast<const float2*>(vr + gi);
-    const uint32_t c01 = code_pair(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi);
+    const uint32_t c01 = code_pair<BITS>(Rv[tok][ch], Rv[tok + 1][ch], z.x, z.y, ri.x, ri.y, vs + gi);
     const int b0 = BITS * slot, b1 = b0 + 16;
     if constexpr (MASK) {
       const uint32_t c0 = c01 & 0xffu, c1 = c01 >> 16;
@@ -254,7 +260,7 @@ __device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const
     const float2 R = *reinterpret_cast<const float2*>(&Rk[tok][ch]);
     const float2 z = *reinterpret_cast<const float2*>(kz + ch);
     const float2 ri = *reinterpret_cast<const float2*>(kr + ch);
-    word |= code_pair(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch) << (BITS * slot);
+    word |= code_pair<BITS>(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch) << (BITS * slot);
   }
   return word;
 }

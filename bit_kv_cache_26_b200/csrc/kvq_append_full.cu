@@ -3,31 +3,45 @@
 // 4.1 granularity): every page whose 32 tokens all arrive in this call, which is nearly all of
 // them in a prefill.  Pages only partly written by the call go through append_pages_kernel.
 //
-// Persistent CTAs of 4 warps, each walking a contiguous run of (KV head, sequence, page) tasks.
+// Persistent CTAs of 8 warps, each walking a contiguous run of (KV head, sequence, page) tasks.
 // A task's 32 V rows and 32 K rows arrive by TMA (two 64-channel boxes each, 128-byte swizzle)
 // into one of two stage buffers; the copy of the task after next is issued as soon as a stage is
-// free.  Warps 0-1 handle the V rows, warps 2-3 the K rows (16 rows each), with no block-wide
-// barrier inside a task: two lanes per row, lane (r, h) holding channels [64 h, 64 h + 64) of
-// its row in registers and half of the patterns for the bounds.
+// free.  Every phase of a task spreads its work evenly over the 256 threads, with a block barrier
+// between phases:
+//   A  V seeds: the Euclidean nearest pattern on the tensor cores (m16n8k16 scores |m|^2/2 - x.m
+//      against the patterns' 16-bit parts; only a guess), warps 0-1; the other warps gather each
+//      row's values at the probe channels (the channels where the patterns differ most).
+//   B  U = exact min-max distance of each V row to its seed, and the row's own range (adaptive
+//      threshold), 4 threads a row; K lower bounds over 16 probe channels for every pattern
+//      (lane = K row, warp w takes the w-th eighth of the patterns), kept in registers; the
+//      smallest bound names the K seed.
+//   C  U of each K row (4 threads a row); V lower bounds over 8 probe channels for every pattern
+//      (lane = V row, the same split): a pattern whose bound could still beat the seed, or tie
+//      it with a lower index, goes on the warp's own refinement list (a warp prefix sum of the
+//      lanes' candidate counts places them), whose bounds over 32 probe channels the warp then
+//      computes a lane an entry; the survivors go on the warp's exact list.
+//   D  the K patterns of the warp's eighth whose bound does not exceed U join the exact list;
+//      the warp computes the min-max distance of every entry over all 128 channels (4 lanes an
+//      entry) and keeps the minimum (distance, index) per row.  A row whose candidates did not
+//      fit a list is compared with every pattern instead.
+//   F  V rows: residual, scale and zero per 32-channel group, codes (a thread a row and group);
+//      K rows: residuals staged as fp32.
+//   G  K scale and zero per channel over the page's 32 tokens (a thread a channel).
+//   H  K codes (a thread a row and 16 channels).
+//   I  the 16-bit codes, written over the consumed input rows, come back in the page's fragment
+//      order through ldmatrix(.trans); a few shifts pack them into words.
+// The bounds are exact lower bounds: the residual range over a channel subset never exceeds the
+// range over all channels, and a subset's residuals are the same fp32 subtractions.  Ties keep
+// the lowest pattern index (the minimum of (distance bits, index) keys).
 //
-// Exact nearest pattern (same fp32 operations as the definition, lowest index on ties):
-//   V rows: seed = the Euclidean nearest pattern (m16n8k16 tensor-core scores |m|^2/2 - x.m
-//     against the patterns' bf16 / fp16 parts; only a guess), U = its exact d_mm; then a lower
-//     bound for every other pattern from the 8 channels where the patterns differ most (the
-//     residual range over a channel subset never exceeds the range over all channels; same fp32
-//     subtractions), refined to 32 channels for the survivors, and the exact d_mm of the few that
-//     still could beat (or tie below) the seed.
-//   K rows: the 16-channel bound for every pattern first (K's outlier channels make it nearly
-//     exact), seed = its argmin, then the exact d_mm of the patterns whose bound does not exceed it.
-// Quantization: residuals in registers; V scale / zero per (token, 32-channel group) in the lane;
-// K scale / zero per channel from the residuals staged in shared memory.  A code is
-// rne(fl32(fl32(R - z) / s)), produced by one FMA, v = t (1/s) + (1.5 * 2^15 + 0.5): the
-// integer part of (t / s + 1/2) lands in bits 8-15 and its fraction in bits 0-7.  The fraction
-// byte is zero only when t / s lies within 2^-9 of a half-integer; only there could the
-// reciprocal's error move the result across a rounding boundary, and those codes are recomputed
-// with the correctly rounded division.  The 16-bit codes are written over the staged input rows
-// and ldmatrix(.trans) brings them back in the page's fragment order, where a few shifts pack
-// them into words.
+// A code is rne(fl32(fl32(R - z) / s)), produced by one FMA, v = t (1/s) + (1.5 * 2^7 + 1/2)
+// with t = R - z in [0, maxc s]: v stays in [128, 256), so the integer part of (t / s + 1/2) is
+// 192 + code (bits 16-22) and its fraction fills bits 0-15.  v differs from the exact
+// t / s + 1/2 by less than 2^-17 (its own rounding) + 15 * 2^-24 (the reciprocal's), under one
+// fraction step (2^-16); so the integer part can be wrong, or the quotient a tie that rounds to
+// even, only when the fraction is 0x0000 or 0xFFFF.  Those codes (about 2 in 65536), and every
+// code of a scale below 2^-125 whose reciprocal is inexact, are recomputed with the correctly
+// rounded division.
 #include <algorithm>
 #include <cstdint>
 
@@ -38,15 +52,21 @@ namespace kvq {
 
 namespace {
 
-constexpr int kFThreads = 128;
+constexpr int kFThreads = 256;  // 8 warps; two CTAs per SM for up to 64 patterns
 constexpr int kProbeAll = 32;  // probe channels per pattern set in the prep tables
 constexpr int kV1 = 8;         // V: first-level bound channels
+constexpr int kV2 = 32;        // V: refined bound channels
 constexpr int kK1 = 16;        // K: bound channels
+constexpr int kTabLd = 36;     // fp32 row stride of the V probe table and of the rows' probe values
 constexpr int kPhiLd = 136;    // 16-bit row stride of the pattern table for ldmatrix (272 B: conflict-free)
-constexpr int kRkLd = 132;     // fp32 row stride of the staged K residuals
+constexpr int kRkLd = 144;     // fp32 row stride of the staged K residuals (16 mod 32 words)
 constexpr int kStageBytes = 16384;  // V rows (2 x 4 KB halves) then K rows (2 x 4 KB halves)
+constexpr int kMaxSlice = 16;       // patterns per warp in the bound passes (up to 128 patterns)
+constexpr int kW2Cap = 256;         // entries of a warp's refinement list
+constexpr int kWECap = 128;         // entries of a warp's exact list
 constexpr uint32_t kFSpin = 1u << 22;
-constexpr float kCodeMagic = 49152.5f;  // 1.5 * 2^15 + 0.5: 8 fractional bits, +1/2 folded in
+constexpr float kCodeMagic = 192.5f;  // 1.5 * 2^7 + 1/2: 16 fractional bits, +1/2 folded in
+constexpr float kMinScale = 0x1p-125f;  // below this (and nonzero) 1 / s is not within 2^-24 of exact
 
 __device__ __forceinline__ uint32_t s32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -100,6 +120,7 @@ __device__ __forceinline__ void mma_seed(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+
 template <int DT>
 __device__ __forceinline__ float cvt_lo(uint32_t w) {
   if constexpr (DT == KVQ_BF16) return __uint_as_float(w << 16);
@@ -118,26 +139,226 @@ __device__ __forceinline__ uint32_t elem_off(int row, int ch) {
   return (uint32_t)((ch >> 6) * 4096) + swz(row, (ch & 63) >> 3) + (uint32_t)((ch & 7) * 2);
 }
 
+// Channels 32 q .. 32 q + 31 of staged row `row` (16-bit, swizzled) as fp32.
+template <int DT>
+__device__ __forceinline__ void load_x32(const uint8_t* rows, int row, int q, float (&x)[32]) {
+  const uint8_t* hb = rows + (q >> 1) * 4096;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const uint4 u = *reinterpret_cast<const uint4*>(hb + swz(row, 4 * (q & 1) + cc));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * cc + 2 * e] = cvt_lo<DT>(w4[e]);
+      x[8 * cc + 2 * e + 1] = cvt_hi<DT>(w4[e]);
+    }
+  }
+}
+
+// Range of x - m over 32 channels (m: 32 fp32 pattern values in global memory).
+__device__ __forceinline__ void range32(const float (&x)[32], const float* __restrict__ m, float& mx, float& mn) {
+  const float4* m4 = reinterpret_cast<const float4*>(m);
+  float4 mv[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
+  mx = -INFINITY;
+  mn = INFINITY;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float r0, r1, r2, r3;
+    sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, r0, r1);
+    sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, r2, r3);
+    mx = max3(mx, r0, r1);
+    mn = min3(mn, r0, r1);
+    mx = max3(mx, r2, r3);
+    mn = min3(mn, r2, r3);
+  }
+}
+
+// Range of y - t over N probe channels (both in shared memory, 16-byte aligned).
+template <int N>
+__device__ __forceinline__ float probe_range(const float* y, const float* t) {
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 a = reinterpret_cast<const float4*>(y)[q];
+    const float4 m = reinterpret_cast<const float4*>(t)[q];
+    float r0, r1, r2, r3;
+    sub2(a.x, a.y, m.x, m.y, r0, r1);
+    sub2(a.z, a.w, m.z, m.w, r2, r3);
+    mx = max3(mx, r0, r1);
+    mn = min3(mn, r0, r1);
+    mx = max3(mx, r2, r3);
+    mn = min3(mn, r2, r3);
+  }
+  return __fsub_rn(mx, mn);
+}
+
+__device__ __forceinline__ unsigned long long dkey(float d, int j) {
+  return ((unsigned long long)__float_as_uint(d) << 32) | (uint32_t)j;
+}
+
+// Range of y - t over N probe channels (y in registers, t in shared memory, 16-byte aligned).
+template <int N>
+__device__ __forceinline__ float probe_range_reg(const float (&y)[N], const float* t) {
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int q = 0; q < N / 4; ++q) {
+    const float4 m = reinterpret_cast<const float4*>(t)[q];
+    float r0, r1, r2, r3;
+    sub2(y[4 * q], y[4 * q + 1], m.x, m.y, r0, r1);
+    sub2(y[4 * q + 2], y[4 * q + 3], m.z, m.w, r2, r3);
+    mx = max3(mx, r0, r1);
+    mn = min3(mn, r0, r1);
+    mx = max3(mx, r2, r3);
+    mn = min3(mn, r2, r3);
+  }
+  return __fsub_rn(mx, mn);
+}
+
+// A warp's lanes each list the patterns j0 + i (bit i of `mask`) of their row `row`: the
+// entries (row << 8 | pattern) go to list[base ..], placed by a warp prefix sum of the counts.
+// Returns the new (uniform) size, at most cap; an entry past cap flags its row instead.
+__device__ __forceinline__ int warp_compact(uint32_t mask, int lane, int row, int j0, uint16_t* list, int base,
+                                            int cap, int* ovf_row, int* any_ovf) {
+  const int n = __popc(mask);
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(kFull, incl, 31);
+  int pos = base + incl - n;
+  while (mask) {
+    const int i = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    if (pos < cap) list[pos] = (uint16_t)((row << 8) | (j0 + i));
+    else { *ovf_row = 1; *any_ovf = 1; }
+    ++pos;
+  }
+  return min(base + total, cap);
+}
+// Append of one entry per live lane (every lane of the warp calls it); returns the new size.
+__device__ __forceinline__ int warp_append(bool live, uint32_t entry, uint16_t* list, int n, int cap, int* ovf_row,
+                                           int* any_ovf, int lane) {
+  const unsigned m = __ballot_sync(kFull, live);
+  if (live) {
+    const int pos = n + __popc(m & ((1u << lane) - 1u));
+    if (pos < cap) list[pos] = (uint16_t)entry;
+    else { *ovf_row = 1; *any_ovf = 1; }
+  }
+  return min(n + __popc(m), cap);
+}
+
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Codes of N residuals as N / 2 words of two 16-bit halves (the code in bits 8-11 of each
+// half: byte 2 of the FMA result, 0x40 | code); zr(i, z0, z1, r0, r1) gives the zeros and
+// reciprocal scales of values 2i, 2i + 1.  Returns true if no fraction is 0x0000 or 0xFFFF.
+template <int N, class ZR>
+__device__ __forceinline__ bool codes_fma(const float (&x)[N], uint32_t (&p)[N / 2], ZR zr) {
+  uint32_t acc = 0xFFFFFFFFu;  // per half: min over the pairs of (fraction + 1) mod 2^16
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    float z0, z1, r0, r1, t0, t1, v0, v1;
+    zr(i, z0, z1, r0, r1);
+    sub2(x[2 * i], x[2 * i + 1], z0, z1, t0, t1);
+    fma2f(t0, t1, r0, r1, kCodeMagic, kCodeMagic, v0, v1);
+    const uint32_t u0 = __float_as_uint(v0), u1 = __float_as_uint(v1);
+    p[i] = __byte_perm(u0, u1, 0x6420);
+    // a carry out of the low half only happens when that half is flagged anyway
+    acc = vmin_u16x2(acc, __byte_perm(u0, u1, 0x5410) + 0x00010001u);
+  }
+  return (acc & 0x0000FFFEu) != 0u && (acc & 0xFFFE0000u) != 0u;
+}
+
+// 1 / s for the FMA codes: 0 for s == 0 (every code 0, as the definition gives)
+__device__ __forceinline__ float code_rcp(float s) { return s != 0.0f ? __frcp_rn(s) : 0.0f; }
+__device__ __forceinline__ bool tiny_scale(float s) { return s != 0.0f && s < kMinScale; }
+// The definition's code: the correctly rounded quotient, rounded half to even, clamped.
+__device__ __forceinline__ uint32_t exact_code(float t, float s, int maxc) {
+  return s != 0.0f ? (uint32_t)min(max(__float2int_rn(__fdiv_rn(t, s)), 0), maxc) : 0u;
+}
+// fp32 index of (row, channel) in the staged K residuals: 4 floats between the 32-channel
+// quarters and 144 floats between rows, so that the quarters and neighbouring rows fall in
+// different banks
+__device__ __forceinline__ int rk_at(int row, int ch) { return row * kRkLd + ch + 4 * (ch >> 5); }
+
+// The rare paths of codes_fma (a fraction of 0x0000 / 0xFFFF somewhere, or a scale below
+// 2^-125), out of line and reading their inputs from memory, so that no register array of the
+// caller needs an address: every code of the unit recomputed with exact_code.
+// V: channels 32 q .. 32 q + 31 of staged row r (16-bit input, minus the pattern's values m
+// unless null), zero z, scale s; the 16-bit code words replace the input there.
+template <int DT>
+__device__ __noinline__ void v_codes_exact(uint8_t* rows, int r, int q, const float* m, float z, float s, int maxc) {
+  uint8_t* hb = rows + (q >> 1) * 4096;
+  for (int cc = 0; cc < 4; ++cc) {
+    uint4* p = reinterpret_cast<uint4*>(hb + swz(r, 4 * (q & 1) + cc));
+    const uint4 u = *p;
+    uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    for (int e = 0; e < 4; ++e) {
+      const int c = 8 * cc + 2 * e;
+      float x0 = cvt_lo<DT>(w4[e]), x1 = cvt_hi<DT>(w4[e]);
+      if (m) {
+        x0 = __fsub_rn(x0, __ldg(m + c));
+        x1 = __fsub_rn(x1, __ldg(m + c + 1));
+      }
+      w4[e] = (exact_code(__fsub_rn(x0, z), s, maxc) << 8) | (exact_code(__fsub_rn(x1, z), s, maxc) << 24);
+    }
+    *p = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+}
+// K: channels 4 cb + 32 k .. + 3 (k = 0..3) of row r, residuals from Rk, zero / scale per channel.
+__device__ __noinline__ void k_codes_exact(uint8_t* rowsK, const float* Rk, const float2* kzr, const float* kss, int r,
+                                           int cb, int maxc) {
+  for (int k4 = 0; k4 < 4; ++k4) {
+    const int c = 4 * cb + 32 * k4;
+    uint32_t w[2];
+    for (int pr = 0; pr < 2; ++pr) {
+      const int c0 = c + 2 * pr;
+      const uint32_t a = exact_code(__fsub_rn(Rk[rk_at(r, c0)], kzr[c0].x), kss[c0], maxc);
+      const uint32_t b = exact_code(__fsub_rn(Rk[rk_at(r, c0 + 1)], kzr[c0 + 1].x), kss[c0 + 1], maxc);
+      w[pr] = (a << 8) | (b << 24);
+    }
+    *reinterpret_cast<uint2*>(rowsK + elem_off(r, c)) = make_uint2(w[0], w[1]);
+  }
+}
+
 struct FullSmem {
-  int stage, rk, phi, hnorm, tabv, tabk, pcv, pck, lbk, kzr, ks, bars, total;
+  int stage, rk, phi, hnorm, tabv, tabk, pcv, pck, xp, rowu, seed, best, kkey, rraw, ovf, lw2, lwe, ctr, kzr, ks, bars,
+      total;
 };
 __host__ __device__ inline FullSmem full_smem(int P) {
   const int Pp = (P + 7) & ~7;
   FullSmem s;
   int o = 0;
-  s.stage = o; o += 2 * kStageBytes;
-  s.rk = o; o += 32 * kRkLd * 4;
-  s.phi = o; o += Pp * kPhiLd * 2;
-  s.hnorm = o; o += Pp * 4;
-  s.tabv = o; o += P * kProbeAll * 4;
-  s.tabk = o; o += P * kK1 * 4;
-  s.pcv = o; o += kProbeAll * 4;
-  s.pck = o; o += kK1 * 4;
-  s.lbk = o; o += 32 * ((P + 7) & ~7) * 2;
-  o = (o + 15) & ~15;
-  s.kzr = o; o += kD * 8;
-  s.ks = o; o += kD * 4;
-  s.bars = o; o += 2 * 8;
+  auto take = [&](int bytes) { const int r = o; o = (o + bytes + 15) & ~15; return r; };
+  s.stage = take(2 * kStageBytes);
+  s.rk = take(32 * kRkLd * 4);
+  s.phi = take(Pp * kPhiLd * 2);
+  s.hnorm = take(Pp * 4);
+  s.tabv = take(P * kTabLd * 4);
+  s.tabk = take(P * kK1 * 4);
+  s.pcv = take(kProbeAll * 4);
+  s.pck = take(kK1 * 4);
+  s.xp = take(64 * kTabLd * 4);
+  s.rowu = take(64 * 4);
+  s.seed = take(64 * 4);
+  s.best = take(64 * 8);
+  s.kkey = take(32 * 4);
+  s.rraw = take(32 * 4);
+  s.ovf = take(64 * 4);
+  s.lw2 = take(8 * kW2Cap * 2);
+  s.lwe = take(8 * kWECap * 2);
+  s.ctr = take(4 * 4);
+  s.kzr = take(kD * 8);
+  s.ks = take(kD * 4);
+  s.bars = take(2 * 8);
   s.total = o + 1024;  // room to align the stage buffers to 1024 B (128-byte swizzle atoms)
   return s;
 }
@@ -174,76 +395,9 @@ __device__ __forceinline__ Task task_of(const Geom& g, int n_new, int F, int64_t
   return k;
 }
 
-// Range of x - m over this lane's 64 channels (x in registers, m the pattern half in global memory).
-__device__ __forceinline__ void half_range(const float (&x)[64], const float* __restrict__ m, float& mx, float& mn) {
-  const float4* m4 = reinterpret_cast<const float4*>(m);
-  mx = -INFINITY;
-  mn = INFINITY;
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const float4 v = __ldg(m4 + c);
-    float r0, r1, r2, r3;
-    sub2(x[4 * c], x[4 * c + 1], v.x, v.y, r0, r1);
-    sub2(x[4 * c + 2], x[4 * c + 3], v.z, v.w, r2, r3);
-    mx = max3(mx, r0, r1);
-    mn = min3(mn, r0, r1);
-    mx = max3(mx, r2, r3);
-    mn = min3(mn, r2, r3);
-  }
-}
-
-// Exact d_mm of the candidates of both lanes of a row (lane hh's candidates: bit i of its mask =
-// pattern jb(hh) + i, jb(0) = 0, jb(1) = P2), in ascending pattern order; the best (distance,
-// index) so far is (bd, bj).  Both lanes of a row run the same list.
-__device__ __forceinline__ void exact_candidates(const float (&x)[64], const float* __restrict__ M, int hh, int P2,
-                                                 unsigned long long mine, float& bd, int& bj) {
-  const unsigned long long other = __shfl_xor_sync(kFull, mine, 16);
-  unsigned long long ml = hh ? other : mine, mh = hh ? mine : other;
-#pragma unroll 1
-  for (int q = 0; q < 2; ++q) {
-    unsigned long long mq = q ? mh : ml;
-    while (__any_sync(kFull, mq != 0ull)) {
-      const bool act = mq != 0ull;
-      const int j = act ? q * P2 + __ffsll((long long)mq) - 1 : 0;
-      if (act) mq &= mq - 1;
-      float mx = -INFINITY, mn = INFINITY;
-      if (act) half_range(x, M + (size_t)j * kD + 64 * hh, mx, mn);
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-      mn = fminf(mn, __shfl_xor_sync(kFull, mn, 16));
-      const float d = __fsub_rn(mx, mn);
-      if (act && (d < bd || (d == bd && j < bj))) { bd = d; bj = j; }
-    }
-  }
-}
-
-// Codes of this lane's 64 residuals as 32 pairs of 16-bit (code << 8 | fraction) words; zr(i,
-// z0, z1, r0, r1) gives the zero and reciprocal scale of values 2i, 2i + 1.  Returns true if
-// every fraction byte is nonzero (no code within 2^-9 of a rounding boundary).
-template <class ZR>
-__device__ __forceinline__ bool codes64(const float (&x)[64], uint32_t (&p)[32], ZR zr) {
-  uint32_t acc = 0x01000100u;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float z0, z1, r0, r1, t0, t1, v0, v1;
-    zr(i, z0, z1, r0, r1);
-    sub2(x[2 * i], x[2 * i + 1], z0, z1, t0, t1);
-    fma2f(t0, t1, r0, r1, kCodeMagic, kCodeMagic, v0, v1);
-    const uint32_t w = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
-    p[i] = w;
-    acc &= (w & 0x00FF00FFu) + 0x00FF00FFu;
-  }
-  return (acc & 0x01000100u) == 0x01000100u;
-}
-
-// Exact code (the definition: the correctly rounded quotient, round half to even, clamp).
-__device__ __forceinline__ uint32_t exact_code(float R, float z, float s, int maxc) {
-  if (s == 0.0f) return 0u;
-  const float u = __fdiv_rn(__fsub_rn(R, z), s);
-  return (uint32_t)min(max(__float2int_rn(u), 0), maxc);
-}
 
 template <int DT>
-__global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                    const __grid_constant__ CUtensorMap vmap, Geom g,
                                                                    const int32_t* __restrict__ probe,
                                                                    const float* __restrict__ pvals, int n_new,
@@ -253,24 +407,31 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
   const FullSmem sp = full_smem(P);
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage = base + sp.stage;
-  float* Rk = reinterpret_cast<float*>(base + sp.rk);
+  float* Rk = reinterpret_cast<float*>(base + sp.rk);        // K residuals, rk_at(row, channel)
   uint16_t* phi = reinterpret_cast<uint16_t*>(base + sp.phi);
   float* hnorm = reinterpret_cast<float*>(base + sp.hnorm);
-  float* tabv = reinterpret_cast<float*>(base + sp.tabv);
-  float* tabk = reinterpret_cast<float*>(base + sp.tabk);
+  float* tabv = reinterpret_cast<float*>(base + sp.tabv);    // [P][kTabLd]: V patterns at the 32 probe channels
+  float* tabk = reinterpret_cast<float*>(base + sp.tabk);    // [P][16]: K patterns at the 16 probe channels
   int32_t* pcv = reinterpret_cast<int32_t*>(base + sp.pcv);
   int32_t* pck = reinterpret_cast<int32_t*>(base + sp.pck);
-  __half* lbk = reinterpret_cast<__half*>(base + sp.lbk);
-  float2* kzr = reinterpret_cast<float2*>(base + sp.kzr);  // per K channel: z, 1/s
+  float* xp = reinterpret_cast<float*>(base + sp.xp);        // [64 rows][kTabLd]: rows at the probe channels
+  float* rowu = reinterpret_cast<float*>(base + sp.rowu);    // per row: exact distance to the seed
+  int32_t* rseed = reinterpret_cast<int32_t*>(base + sp.seed);
+  unsigned long long* best = reinterpret_cast<unsigned long long*>(base + sp.best);  // (distance, index) keys
+  uint32_t* kkey = reinterpret_cast<uint32_t*>(base + sp.kkey);  // K rows: smallest (bound, index), 7-bit tag
+  float* rraw = reinterpret_cast<float*>(base + sp.rraw);    // V rows: the vector's own range
+  int32_t* ovf = reinterpret_cast<int32_t*>(base + sp.ovf);  // per row: candidates dropped by a full list
+  uint16_t* lw2 = reinterpret_cast<uint16_t*>(base + sp.lw2);  // per warp: refinement list (V rows)
+  uint16_t* lwe = reinterpret_cast<uint16_t*>(base + sp.lwe);  // per warp: exact list (rows 0-31 V, 32-63 K)
+  int32_t* ctr = reinterpret_cast<int32_t*>(base + sp.ctr);  // [0] a tiny K scale, [1] a row overflowed
+  float2* kzr = reinterpret_cast<float2*>(base + sp.kzr);    // per K channel: z, 1/s
   float* kss = reinterpret_cast<float*>(base + sp.ks);       // per K channel: s
   uint64_t* full = reinterpret_cast<uint64_t*>(base + sp.bars);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool isV = warp < 2;
-  const int r = lane & 15, hh = lane >> 4;
-  const int row = 16 * (warp & 1) + r;
-  const int LdP = (P + 7) & ~7;  // row stride of the K bound table (halves)
   const int maxc = (1 << g.bits) - 1;
+  uint16_t* wl2 = lw2 + warp * kW2Cap;
+  uint16_t* wle = lwe + warp * kWECap;
 
   const int64_t T = (int64_t)g.H * g.B * F;
   const int64_t t0 = (int64_t)blockIdx.x * per_cta, t1 = min(T, t0 + per_cta);
@@ -320,8 +481,8 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
     const float* MK = g.kpat + (size_t)sh * P * kD;
     const float* MV = g.vpat + (size_t)sh * P * kD;
     const int Pe = p_eff(g, sh), Pep = (Pe + 7) & ~7;  // patterns in use (P is the capacity)
-    const int P2 = (Pe + 1) >> 1;
-    const int jb = hh * P2, je = min(Pe, jb + P2);  // this lane's pattern half
+    const int S8 = (Pe + 7) >> 3;                        // patterns per warp in the bound passes
+    const int j0w = min(Pe, warp * S8), nsl = min(Pe, j0w + S8) - j0w;
     uint8_t* sub = g.pool + (size_t)g.page_table[(size_t)k.b * g.maxp + k.pg] * g.page_bytes + (size_t)k.h * g.sub_bytes;
 
     // ---- pattern tables of this (set, head), staged when they change
@@ -347,7 +508,8 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
         hnorm[n] = n < Pe ? 0.5f * acc : 1e30f;
       }
       const size_t o = (size_t)sh * 2;
-      for (int q = tid; q < Pe * kProbeAll; q += kFThreads) tabv[q] = __ldg(pvals + (o + 1) * P * kProbeAll + q);
+      for (int q = tid; q < Pe * kProbeAll; q += kFThreads)
+        tabv[(q / kProbeAll) * kTabLd + q % kProbeAll] = __ldg(pvals + (o + 1) * P * kProbeAll + q);
       for (int q = tid; q < Pe * kK1; q += kFThreads)
         tabk[q] = __ldg(pvals + o * P * kProbeAll + (size_t)(q / kK1) * kProbeAll + q % kK1);
       if (tid < kProbeAll) pcv[tid] = __ldg(probe + (o + 1) * kProbeAll + tid);
@@ -360,32 +522,13 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       timed_out = true;
     }
     if (__syncthreads_or(timed_out)) break;
-    uint8_t* rows = stage + buf * kStageBytes + (isV ? 0 : 8192);
-    const uint32_t rows_s = s32(rows);
+    uint8_t* stV = stage + buf * kStageBytes;  // V rows; K rows at + 8192
+    uint8_t* stK = stV + 8192;
 
-    // ---- this lane's 64 channels of its row
-    float x[64];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 u = *reinterpret_cast<const uint4*>(rows + hh * 4096 + swz(row, c));
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[8 * c + 2 * e] = cvt_lo<DT>(w4[e]);
-        x[8 * c + 2 * e + 1] = cvt_hi<DT>(w4[e]);
-      }
-    }
-    auto row_val = [&](int ch) -> float {
-      const uint16_t u = *reinterpret_cast<const uint16_t*>(rows + elem_off(row, ch));
-      return cvt_lo<DT>((uint32_t)u);
-    };
-
-    float bd;
-    int bj;
-    float rraw = 0.f;
-    unsigned long long mask = 0ull;  // this lane's candidates: bit j - jb
-    if (isV) {
-      // ---- seed: Euclidean scores on the tensor cores (rows 16 (warp & 1) .. +15, all patterns)
+    // ---- A: V seeds on the tensor cores; probe values of every row; per-task resets
+    if (warp < 2) {
+      const uint32_t rows_s = s32(stV);
+      const int r = lane & 15;
       const int rb = 16 * (warp & 1);
       uint32_t A[8][4];
 #pragma unroll
@@ -422,214 +565,309 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
       int seed = (int)(__float_as_uint(r < 8 ? s_lo : s_hi) & 127u);
       seed = min(seed, Pe - 1);
 
-      // ---- U = exact d_mm of the seed; the vector's own range (adaptive threshold)
-      float mx, mn;
-      half_range(x, MV + (size_t)seed * kD + 64 * hh, mx, mn);
-      float ymx = -INFINITY, ymn = INFINITY;
+      if (lane < 16) rseed[16 * warp + r] = seed;
+    } else {
+      const int u = tid - 64;  // 0..191
+      if (u < 128) {  // V rows: 32 probe values, 8 per thread
+        const int row = u >> 2, k0 = 8 * (u & 3);
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+        for (int e = 0; e < 8; ++e)
+          xp[row * kTabLd + k0 + e] = cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stV + elem_off(row, pcv[k0 + e])));
+      } else {  // K rows: 16 probe values, 8 per thread
+        const int row = (u - 128) >> 1, k0 = 8 * (u & 1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          xp[(32 + row) * kTabLd + k0 + e] =
+              cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stK + elem_off(row, pck[k0 + e])));
+      }
+      if (u < 64) ovf[u] = 0;
+      else if (u < 96) kkey[u - 64] = 0xFFFFFFFFu;
+      else if (u == 96) ctr[0] = ctr[1] = 0;
+    }
+    __syncthreads();
+
+    // ---- B: V rows: exact distance to the seed and own range (4 threads a row)
+    if (warp < 4) {
+      const int r = tid >> 2, q = tid & 3;
+      float x[32];
+      load_x32<DT>(stV, r, q, x);
+      const int s = rseed[r];
+      float mx, mn, ymx = -INFINITY, ymn = INFINITY;
+      range32(x, MV + (size_t)s * kD + 32 * q, mx, mn);
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
         ymx = max3(ymx, x[c], x[c + 1]);
         ymn = min3(ymn, x[c], x[c + 1]);
       }
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-      mn = fminf(mn, __shfl_xor_sync(kFull, mn, 16));
-      ymx = fmaxf(ymx, __shfl_xor_sync(kFull, ymx, 16));
-      ymn = fminf(ymn, __shfl_xor_sync(kFull, ymn, 16));
-      const float U = __fsub_rn(mx, mn);
-      rraw = __fsub_rn(ymx, ymn);
-      bd = U;
-      bj = seed;
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+        ymx = fmaxf(ymx, __shfl_xor_sync(kFull, ymx, o));
+        ymn = fminf(ymn, __shfl_xor_sync(kFull, ymn, o));
+      }
+      if (q == 0) {
+        const float U = __fsub_rn(mx, mn);
+        rowu[r] = U;
+        best[r] = dkey(U, s);
+        rraw[r] = __fsub_rn(ymx, ymn);
+      }
+    }
+    // K rows: bounds over 16 probe channels for this warp's patterns (lane = K row), kept in
+    // registers until the K candidates are listed; the smallest (tagged with its index in the 7
+    // low bits) names the seed
+    float klb[kMaxSlice];
+    {
+      float y[kK1];
+#pragma unroll
+      for (int q = 0; q < kK1 / 4; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(xp + (32 + lane) * kTabLd)[q];
+        y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
+      }
+      uint32_t kb = 0xFFFFFFFFu;
+#pragma unroll
+      for (int jj = 0; jj < kMaxSlice; ++jj) {
+        klb[jj] = INFINITY;
+        if (jj < nsl) {
+          const int j = j0w + jj;
+          klb[jj] = probe_range_reg<kK1>(y, tabk + (size_t)j * kK1);
+          kb = min(kb, (__float_as_uint(klb[jj]) & ~127u) | (uint32_t)j);
+        }
+      }
+      if (nsl > 0) atomicMin(&kkey[lane], kb);
+    }
+    __syncthreads();
 
-      // ---- bounds: 8 channels for every pattern of this lane's half, 32 for the survivors
-      float pv[kProbeAll];
-#pragma unroll
-      for (int u = 0; u < kProbeAll; ++u) pv[u] = row_val(pcv[u]);
-      for (int j = jb; j < je; ++j) {
-        const float4* t4 = reinterpret_cast<const float4*>(tabv + (size_t)j * kProbeAll);
-        float lmx = -INFINITY, lmn = INFINITY;
-#pragma unroll
-        for (int q = 0; q < kV1 / 4; ++q) {
-          const float4 m = t4[q];
-          float r0, r1, r2, r3;
-          sub2(pv[4 * q], pv[4 * q + 1], m.x, m.y, r0, r1);
-          sub2(pv[4 * q + 2], pv[4 * q + 3], m.z, m.w, r2, r3);
-          lmx = max3(lmx, r0, r1);
-          lmn = min3(lmn, r0, r1);
-          lmx = max3(lmx, r2, r3);
-          lmn = min3(lmn, r2, r3);
-        }
-        float lb = __fsub_rn(lmx, lmn);
-        bool live = j != seed && (lb < U || (lb == U && j < seed));
-        if (live) {
-#pragma unroll
-          for (int q = kV1 / 4; q < kProbeAll / 4; ++q) {
-            const float4 m = t4[q];
-            float r0, r1, r2, r3;
-            sub2(pv[4 * q], pv[4 * q + 1], m.x, m.y, r0, r1);
-            sub2(pv[4 * q + 2], pv[4 * q + 3], m.z, m.w, r2, r3);
-            lmx = max3(lmx, r0, r1);
-            lmn = min3(lmn, r0, r1);
-            lmx = max3(lmx, r2, r3);
-            lmn = min3(lmn, r2, r3);
-          }
-          lb = __fsub_rn(lmx, lmn);
-          live = lb < U || (lb == U && j < seed);
-        }
-        if (live) mask |= 1ull << (j - jb);
-      }
-      exact_candidates(x, MV, hh, P2, mask, bd, bj);
-    } else {
-      // ---- bounds over 16 channels for every pattern of this lane's half; seed = their argmin
-      float pk[kK1];
-#pragma unroll
-      for (int u = 0; u < kK1; ++u) pk[u] = row_val(pck[u]);
-      float lbest = INFINITY;
-      int lj = jb;
-      for (int j = jb; j < je; ++j) {
-        const float4* t4 = reinterpret_cast<const float4*>(tabk + (size_t)j * kK1);
-        float lmx = -INFINITY, lmn = INFINITY;
-#pragma unroll
-        for (int q = 0; q < kK1 / 4; ++q) {
-          const float4 m = t4[q];
-          float r0, r1, r2, r3;
-          sub2(pk[4 * q], pk[4 * q + 1], m.x, m.y, r0, r1);
-          sub2(pk[4 * q + 2], pk[4 * q + 3], m.z, m.w, r2, r3);
-          lmx = max3(lmx, r0, r1);
-          lmn = min3(lmn, r0, r1);
-          lmx = max3(lmx, r2, r3);
-          lmn = min3(lmn, r2, r3);
-        }
-        const float lb = __fsub_rn(lmx, lmn);
-        lbk[row * LdP + j] = __float2half_rz(lb);  // rounded toward zero: still a lower bound
-        if (lb < lbest) { lbest = lb; lj = j; }
-      }
-      const float olb = __shfl_xor_sync(kFull, lbest, 16);
-      const int oj = __shfl_xor_sync(kFull, lj, 16);
-      if (olb < lbest || (olb == lbest && oj < lj)) { lbest = olb; lj = oj; }
-      const int seed = min(max(lj, 0), Pe - 1);
+    // ---- C: K rows: exact distance to the seed (4 threads a row)
+    if (warp >= 4) {
+      const int r = (tid - 128) >> 2, q = tid & 3;
+      const int s = min((int)(kkey[r] & 127u), Pe - 1);
+      float x[32];
+      load_x32<DT>(stK, r, q, x);
       float mx, mn;
-      half_range(x, MK + (size_t)seed * kD + 64 * hh, mx, mn);
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-      mn = fminf(mn, __shfl_xor_sync(kFull, mn, 16));
-      const float U = __fsub_rn(mx, mn);
-      bd = U;
-      bj = seed;
-      __syncwarp();
-      for (int j = jb; j < je; ++j) {
-        const float lb = __half2float(lbk[row * LdP + j]);
-        if (j != seed && lb <= U) mask |= 1ull << (j - jb);
+      range32(x, MK + (size_t)s * kD + 32 * q, mx, mn);
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
       }
-      exact_candidates(x, MK, hh, P2, mask, bd, bj);
+      if (q == 0) {
+        const float U = __fsub_rn(mx, mn);
+        rowu[32 + r] = U;
+        rseed[32 + r] = s;
+        best[32 + r] = dkey(U, s);
+      }
     }
-
-    // ---- index, then residuals (the pattern, or nothing for a V vector the threshold rejects)
-    const bool keep = !isV || v_keep_pattern(g.vrho, bd, rraw);
-    if (hh == 0) sub[(isV ? g.off_vidx : g.off_kidx) + tok_pos(row)] = keep ? (uint8_t)bj : (uint8_t)kRawIndex;
+    // V rows: bounds over 8 probe channels for this warp's patterns (lane = V row); a pattern
+    // that could still beat the seed, or tie it with a lower index, goes on the warp's refinement
+    // list, whose bounds over 32 probe channels pass the survivors to the warp's exact list
+    int nE = 0;  // entries in this warp's exact list (the same in every lane)
     {
-      const float4* m4 = reinterpret_cast<const float4*>((isV ? MV : MK) + (size_t)bj * kD + 64 * hh);
+      float y[kV1];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 m = keep ? __ldg(m4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-        sub2(x[4 * c], x[4 * c + 1], m.x, m.y, x[4 * c], x[4 * c + 1]);
-        sub2(x[4 * c + 2], x[4 * c + 3], m.z, m.w, x[4 * c + 2], x[4 * c + 3]);
+      for (int q = 0; q < kV1 / 4; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(xp + lane * kTabLd)[q];
+        y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
+      }
+      const float U = rowu[lane];
+      const int s = rseed[lane];
+      uint32_t mask = 0u;
+#pragma unroll
+      for (int jj = 0; jj < kMaxSlice; ++jj) {
+        if (jj < nsl) {
+          const int j = j0w + jj;
+          const float lb = probe_range_reg<kV1>(y, tabv + (size_t)j * kTabLd);
+          if (j != s && (lb < U || (lb == U && j < s))) mask |= 1u << jj;
+        }
+      }
+      const int n2 = warp_compact(mask, lane, lane, j0w, wl2, 0, kW2Cap, &ovf[lane], &ctr[1]);
+      __syncwarp();
+      for (int b0 = 0; b0 < n2; b0 += 32) {
+        const int e = b0 + lane;
+        bool live = false;
+        uint32_t ent = 0u;
+        int r = 0;
+        if (e < n2) {
+          ent = wl2[e];
+          r = (int)(ent >> 8);
+          const int j = (int)(ent & 255u);
+          const float lb = probe_range<kV2>(xp + r * kTabLd, tabv + (size_t)j * kTabLd);
+          const float Ur = rowu[r];
+          live = lb < Ur || (lb == Ur && j < rseed[r]);
+        }
+        nE = warp_append(live, ent, wle, nE, kWECap, &ovf[r], &ctr[1], lane);
       }
     }
+    __syncthreads();
 
-    uint32_t pcode[32];
-    if (isV) {
-      // ---- V: scale / zero of this lane's two groups (channels 32 (2 hh + q) ..), codes
-      float gz[2], gr[2], ss[2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float gmx = -INFINITY, gmn = INFINITY;
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          gmx = max3(gmx, x[32 * q + c], x[32 * q + c + 1]);
-          gmn = min3(gmn, x[32 * q + c], x[32 * q + c + 1]);
-        }
-        const float s = __fdiv_rn(__fsub_rn(gmx, gmn), (float)maxc);
-        const float ri = s != 0.0f ? __frcp_rn(s) : 0.0f;
-        ss[q] = s;
-        gz[q] = gmn;
-        gr[q] = ri;
-        const int grp = 2 * hh + q;
-        reinterpret_cast<float*>(sub + g.off_vs)[vsc_pos(row, grp)] = s;
-        reinterpret_cast<float*>(sub + g.off_vz)[vzc_pos(row, grp)] = gmn;
+    // ---- D: the K candidates of this warp's eighth join its exact list; exact distances of the
+    // list (4 lanes an entry), minimum (distance, index) per row
+    const int q4 = lane & 3;
+    auto exact = [&](bool on, int row, int j) {
+      float mx = -INFINITY, mn = INFINITY;
+      if (on) {
+        float x[32];
+        load_x32<DT>(row < 32 ? stV : stK, row & 31, q4, x);
+        range32(x, (row < 32 ? MV : MK) + (size_t)j * kD + 32 * q4, mx, mn);
       }
-      const bool clean = codes64(x, pcode, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
-        z0 = z1 = gz[i2 >> 4];
-        r0 = r1 = gr[i2 >> 4];
-      });
-      if (!clean) {
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-          const uint32_t c0 = exact_code(x[2 * i2], gz[i2 >> 4], ss[i2 >> 4], maxc);
-          const uint32_t c1 = exact_code(x[2 * i2 + 1], gz[i2 >> 4], ss[i2 >> 4], maxc);
-          pcode[i2] = (c0 << 8) | 0x80u | (c1 << 24) | 0x800000u;
+      for (int o = 1; o <= 2; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+      }
+      if (on && q4 == 0) atomicMin(&best[row], dkey(__fsub_rn(mx, mn), j));
+    };
+    {
+      const float U = rowu[32 + lane];
+      const int s = rseed[32 + lane];
+      uint32_t mask = 0u;
+#pragma unroll
+      for (int jj = 0; jj < kMaxSlice; ++jj)
+        if (jj < nsl && j0w + jj != s && klb[jj] <= U) mask |= 1u << jj;
+      nE = warp_compact(mask, lane, 32 + lane, j0w, wle, nE, kWECap, &ovf[32 + lane], &ctr[1]);
+      __syncwarp();
+      for (int b0 = 0; b0 < nE; b0 += 8) {
+        const int e = b0 + (lane >> 2);
+        const uint32_t ent = e < nE ? wle[e] : 0u;
+        exact(e < nE, (int)(ent >> 8), (int)(ent & 255u));
+      }
+    }
+    __syncthreads();
+    if (ctr[1]) {
+      // some row's candidates did not all fit a list: that row against every pattern
+      for (int row = 0; row < 64; ++row) {
+        if (!ovf[row]) continue;
+        for (int jb = 0; jb < Pe; jb += 8) {
+          const int j = jb + (lane >> 2) + 0;
+          if (warp == 0) exact(j < Pe, row, j);  // one warp: the rows are rare
         }
+      }
+      __syncthreads();
+    }
+
+    // ---- F: V rows quantized (a thread a row and 32-channel group); K residuals staged
+    if (warp < 4) {
+      const int r = tid >> 2, q = tid & 3;
+      const unsigned long long bk = best[r];
+      const int j = (int)(bk & 0xffffffffu);
+      const bool keep = v_keep_pattern(g.vrho, __uint_as_float((uint32_t)(bk >> 32)), rraw[r]);
+      float x[32];
+      load_x32<DT>(stV, r, q, x);
+      const float* mrow = MV + (size_t)j * kD + 32 * q;
+      if (keep) {
+        const float4* m4 = reinterpret_cast<const float4*>(mrow);
+        float4 mv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, x[4 * c], x[4 * c + 1]);
+          sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, x[4 * c + 2], x[4 * c + 3]);
+        }
+      }
+      float gmx = -INFINITY, gmn = INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        gmx = max3(gmx, x[c], x[c + 1]);
+        gmn = min3(gmn, x[c], x[c + 1]);
+      }
+      const float s = __fdiv_rn(__fsub_rn(gmx, gmn), (float)maxc);
+      const float ri = code_rcp(s);
+      reinterpret_cast<float*>(sub + g.off_vs)[vsc_pos(r, q)] = s;
+      reinterpret_cast<float*>(sub + g.off_vz)[vzc_pos(r, q)] = gmn;
+      if (q == 0) sub[g.off_vidx + tok_pos(r)] = keep ? (uint8_t)j : (uint8_t)kRawIndex;
+      uint32_t pc[16];
+      const bool clean = codes_fma<32>(x, pc, [&](int, float& z0, float& z1, float& r0, float& r1) {
+        z0 = z1 = gmn;
+        r0 = r1 = ri;
+      });
+      if (clean && !tiny_scale(s)) {
+        uint8_t* hb = stV + (q >> 1) * 4096;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          *reinterpret_cast<uint4*>(hb + swz(r, 4 * (q & 1) + cc)) =
+              make_uint4(pc[4 * cc], pc[4 * cc + 1], pc[4 * cc + 2], pc[4 * cc + 3]);
+      } else {
+        v_codes_exact<DT>(stV, r, q, keep ? mrow : nullptr, gmn, s, maxc);
       }
     } else {
-      // ---- K: residuals to shared memory; scale / zero per channel over the page's 32 tokens
-      float4* dst = reinterpret_cast<float4*>(Rk + row * kRkLd + 64 * hh);
+      const int r = (tid - 128) >> 2, q = tid & 3;
+      const int j = (int)(best[32 + r] & 0xffffffffu);
+      float x[32];
+      load_x32<DT>(stK, r, q, x);
+      const float4* m4 = reinterpret_cast<const float4*>(MK + (size_t)j * kD + 32 * q);
+      float4 mv[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      {
-        const int c2 = 2 * (tid - 64);  // channels c2, c2 + 1
-        float mx0 = -INFINITY, mn0 = INFINITY, mx1 = -INFINITY, mn1 = INFINITY;
-#pragma unroll 8
-        for (int t = 0; t < 32; t += 2) {
-          const float2 a = *reinterpret_cast<const float2*>(Rk + t * kRkLd + c2);
-          const float2 b2 = *reinterpret_cast<const float2*>(Rk + (t + 1) * kRkLd + c2);
-          mx0 = max3(mx0, a.x, b2.x);
-          mn0 = min3(mn0, a.x, b2.x);
-          mx1 = max3(mx1, a.y, b2.y);
-          mn1 = min3(mn1, a.y, b2.y);
-        }
-        const float s0 = __fdiv_rn(__fsub_rn(mx0, mn0), (float)maxc), s1 = __fdiv_rn(__fsub_rn(mx1, mn1), (float)maxc);
-        *reinterpret_cast<float4*>(kzr + c2) =
-            make_float4(mn0, s0 != 0.0f ? __frcp_rn(s0) : 0.0f, mn1, s1 != 0.0f ? __frcp_rn(s1) : 0.0f);
-        *reinterpret_cast<float2*>(kss + c2) = make_float2(s0, s1);
-        float* ksg = reinterpret_cast<float*>(sub + g.off_ks);
-        float* kzg = reinterpret_cast<float*>(sub + g.off_kz);
-        ksg[ksc_pos(c2)] = s0;
-        ksg[ksc_pos(c2 + 1)] = s1;
-        kzg[ksc_pos(c2)] = mn0;
-        kzg[ksc_pos(c2 + 1)] = mn1;
+      for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
+      float4* dst = reinterpret_cast<float4*>(Rk + rk_at(r, 32 * q));
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float4 o;
+        sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, o.x, o.y);
+        sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, o.z, o.w);
+        dst[c] = o;
       }
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      const float4* kz4 = reinterpret_cast<const float4*>(kzr + 64 * hh);  // (z, 1/s) of two channels
-      const bool clean = codes64(x, pcode, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
-        const float4 q = kz4[i2];
-        z0 = q.x; r0 = q.y; z1 = q.z; r1 = q.w;
-      });
-      if (!clean) {
+      if (q == 0) sub[g.off_kidx + tok_pos(r)] = (uint8_t)j;
+    }
+    __syncthreads();
+
+    // ---- G: K scale and zero per channel over the page (a thread a channel)
+    if (tid < kD) {
+      const int c = tid;
+      const float* col = Rk + rk_at(0, c);
+      float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int i2 = 0; i2 < 32; ++i2) {
-          const int c = 64 * hh + 2 * i2;
-          const uint32_t c0 = exact_code(x[2 * i2], kzr[c].x, kss[c], maxc);
-          const uint32_t c1 = exact_code(x[2 * i2 + 1], kzr[c + 1].x, kss[c + 1], maxc);
-          pcode[i2] = (c0 << 8) | 0x80u | (c1 << 24) | 0x800000u;
-        }
+      for (int t = 0; t < kG; t += 2) {
+        const float a = col[t * kRkLd], b2 = col[(t + 1) * kRkLd];
+        mx = max3(mx, a, b2);
+        mn = min3(mn, a, b2);
+      }
+      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)maxc);
+      kzr[c] = make_float2(mn, code_rcp(s));
+      kss[c] = s;
+      reinterpret_cast<float*>(sub + g.off_ks)[ksc_pos(c)] = s;
+      reinterpret_cast<float*>(sub + g.off_kz)[ksc_pos(c)] = mn;
+      if (tiny_scale(s)) ctr[0] = 1;
+    }
+    __syncthreads();
+
+    // ---- H: K codes (a thread a row and 16 channels: 4 x 4 channels, 32 apart)
+    {
+      const int r = tid >> 3, cb = tid & 7;
+      float x[16], zs[16], rs[16];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int c = 4 * cb + 32 * k4;
+        const float4 a = *reinterpret_cast<const float4*>(Rk + rk_at(r, c));
+        x[4 * k4] = a.x; x[4 * k4 + 1] = a.y; x[4 * k4 + 2] = a.z; x[4 * k4 + 3] = a.w;
+        const float4 p0 = *reinterpret_cast<const float4*>(kzr + c);
+        const float4 p1 = *reinterpret_cast<const float4*>(kzr + c + 2);
+        zs[4 * k4] = p0.x; rs[4 * k4] = p0.y; zs[4 * k4 + 1] = p0.z; rs[4 * k4 + 1] = p0.w;
+        zs[4 * k4 + 2] = p1.x; rs[4 * k4 + 2] = p1.y; zs[4 * k4 + 3] = p1.z; rs[4 * k4 + 3] = p1.w;
+      }
+      uint32_t pc[8];
+      const bool clean = codes_fma<16>(x, pc, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
+        z0 = zs[2 * i2]; z1 = zs[2 * i2 + 1];
+        r0 = rs[2 * i2]; r1 = rs[2 * i2 + 1];
+      });
+      if (clean && ctr[0] == 0) {
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)
+          *reinterpret_cast<uint2*>(stK + elem_off(r, 4 * cb + 32 * k4)) = make_uint2(pc[2 * k4], pc[2 * k4 + 1]);
+      } else {
+        k_codes_exact(stK, Rk, kzr, kss, r, cb, maxc);
       }
     }
+    __syncthreads();
 
-    // ---- 16-bit codes over this lane's half of its (already consumed) input row
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<uint4*>(rows + hh * 4096 + swz(row, c)) =
-          make_uint4(pcode[4 * c], pcode[4 * c + 1], pcode[4 * c + 2], pcode[4 * c + 3]);
-    if (isV) asm volatile("bar.sync 1, 64;" ::: "memory");
-    else asm volatile("bar.sync 2, 64;" ::: "memory");
-
-    // ---- words in the page's fragment order: lane = MMA lane, this warp's four words per chunk
+    // ---- I: code words in the page's fragment order (warps 0-3 V, 4-7 K; a 16-byte chunk of
+    // four words per lane and warp)
     {
-      const int q = warp & 1;
-      uint32_t* blk = reinterpret_cast<uint32_t*>(sub + (isV ? g.off_vc : 0));
-      const int mi = lane >> 3, ri8 = lane & 7;
-      const int nchunk = g.bits == 2 ? 1 : 2;  // 16-byte chunks of four words per lane and warp
-      for (int cq = 0; cq < nchunk; ++cq) {
-        const int wq = (g.bits == 2 ? q : 2 * q + cq);  // chunk index: words 4 wq .. 4 wq + 3
+      const bool isV = warp < 4;
+      const int wq = warp & 3;  // chunk index: words 4 wq .. 4 wq + 3 of every lane
+      if (wq < (g.bits == 2 ? 2 : 4)) {
+        uint32_t* blk = reinterpret_cast<uint32_t*>(sub + (isV ? g.off_vc : 0));
+        const int mi = lane >> 3, ri8 = lane & 7;
         uint32_t wd[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -638,9 +876,7 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
 #pragma unroll
           for (int tt = 0; tt < 2; ++tt) {
             if (g.bits == 4 && tt == 1) continue;
-            int tile;
-            if (g.bits == 2) tile = 2 * w + tt;
-            else tile = w;
+            const int tile = g.bits == 2 ? 2 * w + tt : w;
             int rt, ct;  // row tile (16 rows of the code matrix) and column tile
             if (isV) { rt = tile >> 1; ct = tile & 1; }   // V: rows = channels, 2 column tiles of tokens
             else { rt = tile >> 3; ct = tile & 7; }       // K: rows = tokens, 8 column tiles of channels
@@ -648,10 +884,10 @@ __global__ void __launch_bounds__(kFThreads, 1) append_full_kernel(const __grid_
             if (isV) {
               // stored [token][channel]: the transposed load gives rows = channels, columns = tokens
               const int tok = 16 * ct + 8 * (mi >> 1) + ri8, ch = 16 * rt + 8 * (mi & 1);
-              ldsm4t(s32(stage + buf * kStageBytes) + elem_off(tok, ch), a0, a1, a2, a3);
+              ldsm4t(s32(stV) + elem_off(tok, ch), a0, a1, a2, a3);
             } else {
               const int tok = 16 * rt + 8 * (mi & 1) + ri8, ch = 16 * ct + 8 * (mi >> 1);
-              ldsm4(s32(stage + buf * kStageBytes + 8192) + elem_off(tok, ch), a0, a1, a2, a3);
+              ldsm4(s32(stK) + elem_off(tok, ch), a0, a1, a2, a3);
             }
             const uint32_t av[4] = {a0, a1, a2, a3};
 #pragma unroll

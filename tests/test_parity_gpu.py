@@ -199,3 +199,46 @@ def test_identical_patterns_resolve_ties_to_lowest_index():
     e = encode_unit(w, Kf, Vf, 0, 0, MK, MV, None, None)
     assert (e.kidx == 0).all() and (e.vidx == 0).all()
     check_pages(cache, w, e, 0, 0)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_subnormal_scales_bit_exact(bits):
+    # Groups and channels whose residuals differ only by subnormal amounts: the scale
+    # s = (max - min) / maxc is subnormal (or 0), its reciprocal inexact or infinite, and every
+    # code must still be the definition's rne(fl32(t / s)), clamped ("PatternKV", Section 3.2,
+    # Eq. 1).  Two full pages (the full-page kernel) and a 20-token partial page (the general
+    # kernel), the patterns zero where the tiny values sit.
+    w = W["llama3_8b_32k"].with_(B=1, S=84, Hkv=1, Hq=2, P=4, bits=bits, v_alpha=0.0)
+    k, v = synth.gen_kv(w)
+    rng = np.random.default_rng(7)
+    tiny = np.float32(2.0 ** -130)
+
+    def bf16_bits(a):
+        return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+    k, v = k.copy(), v.copy()
+    # V: group 0 (channels 0..31) of every token: zeros and small multiples of 2^-130
+    v[0, :, 0, :32] = bf16_bits(tiny * rng.integers(0, 4, size=(w.S, 32)).astype(np.float32))
+    # V: group 2 of the even tokens: one value 3 * 2^-133 (2^-133: the smallest bf16 subnormal),
+    # the rest 0
+    g2 = np.zeros((w.S, 32), np.float32)
+    g2[::2, 5] = np.float32(3 * 2.0 ** -133)
+    v[0, :, 0, 64:96] = bf16_bits(g2)
+    # K: channels 7 and 100 over every token: tiny values (per-channel scales of the pages)
+    k[0, :, 0, 7] = bf16_bits(tiny * rng.integers(0, 9, size=w.S).astype(np.float32))
+    k[0, :, 0, 100] = bf16_bits(np.where(np.arange(w.S) % 3 == 0, np.float32(2.0 ** -132), np.float32(0)))
+    Kf, Vf = synth.to_float(k, w.dtype), synth.to_float(v, w.dtype)
+    MK, MV, _, _ = oracle_patterns(w, Kf, Vf)
+    MK[:, :, [7, 100]] = 0.0
+    MV[:, :, :32] = 0.0
+    MV[:, :, 64:96] = 0.0
+    cache = make_cache(w, MK, MV, None, None)
+    cache.append(to_torch(k, w.dtype), to_torch(v, w.dtype))
+    torch.cuda.synchronize()
+    assert cache.read_status() == 0
+    e = encode_unit(w, Kf, Vf, 0, 0, MK, MV, None, None)
+    assert np.any(e.vs[:, 0] != 0) and np.all(np.abs(e.vs[:, 0]) < 2.0 ** -126)
+    assert np.any((e.ks != 0) & (np.abs(e.ks) < 2.0 ** -126))
+    assert np.any(e.vs[:, 2] != 0) and np.any(e.ks[:, 100] != 0)
+    check_pages(cache, w, e, 0, 0)
+    check_tail(cache, w, k, 0, 0, w.S)
