@@ -137,16 +137,29 @@ class ClockSampler:
 # CPU baseline: the oracle, as it stands, on a bounded sample of the workload.
 # ---------------------------------------------------------------------------
 
-def cpu_baseline(w, heads: int = 4, seqs: int | None = None):
+def sample_shape(w, target_s: float, unit_s: float):
+    """(KV heads, sequences) of a sample of about target_s seconds, one (sequence, KV head) unit
+    taking about unit_s: heads first (the generator makes every head of a sequence), then
+    sequences."""
+    units = max(1, min(w.B * w.Hkv, int(round(target_s / max(unit_s, 1e-3)))))
+    heads = max(1, min(w.Hkv, units))
+    return heads, max(1, min(w.B, -(-units // heads)))
+
+
+def cpu_baseline(w, heads: int = 1, seqs: int | None = None, target_s: float | None = None):
     """The oracle, as it stands, on a bounded sample of the workload: every sequence (or the
     first `seqs`) of `heads` of the KV heads, the whole path (mining of K and V on the pooled
     prefill, encoding, decode attention of each sequence's query heads), scaled to KV-tokens/s
-    of the whole job (all KV heads)."""
+    of the whole job (all KV heads).  With target_s, one (sequence, KV head) unit is timed first
+    and the sample is sized to about target_s seconds of oracle work."""
     import numpy as np
 
     import oracle
     import synth
 
+    if target_s is not None:
+        _, unit_s = cpu_baseline(w, heads=1, seqs=1)
+        heads, seqs = sample_shape(w, target_s, unit_s)
     B = w.B if seqs is None else min(seqs, w.B)
     heads = max(1, min(heads, w.Hkv))
     sw = w.with_(B=B)
@@ -532,8 +545,10 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--bits", type=int, default=2)
-    ap.add_argument("--ref-heads", type=int, default=1, help="reference arm: KV heads per step (bounded sample)")
-    ap.add_argument("--ref-seqs", type=int, default=2, help="reference arm: sequences per step (bounded sample)")
+    ap.add_argument("--ref-heads", type=int, default=2, help="reference arm: KV heads per step (bounded sample)")
+    ap.add_argument("--ref-seqs", type=int, default=24, help="reference arm: sequences per step (bounded sample)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle work in the headline's cpu_baseline sample (half that per configuration)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="headline workload only")
     ap.add_argument("--batch", type=int, default=0,
@@ -572,7 +587,7 @@ def main():
             wc = synth.WORKLOADS[name].with_(**kw)
             r, _, _ = measure_path(wc, args, dev, 1, 0, headline=False)
             if not args.no_cpu_baseline:
-                r["cpu_baseline"], _ = cpu_baseline(wc, heads=1, seqs=1)
+                r["cpu_baseline"], _ = cpu_baseline(wc, target_s=args.cpu_seconds / 2)
             per_config.append(r)
         wl = synth.WORKLOADS["long_cot_8k"]
         r = measure_decode_loop(wl, args, dev)
@@ -598,7 +613,7 @@ def main():
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"], _ = cpu_baseline(w, heads=1, seqs=2)
+            line["cpu_baseline"], _ = cpu_baseline(w, target_s=args.cpu_seconds)
         if per_config:
             line["per_config"] = per_config
         print(json.dumps(line), flush=True)

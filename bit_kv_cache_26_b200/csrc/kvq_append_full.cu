@@ -364,35 +364,49 @@ __host__ __device__ inline FullSmem full_smem(int P) {
 }
 
 struct Task {
-  int h, b, pg, L, set;
-  bool ok;
+  int h, b, pg, L, set, phys;  // pg < 0: not a page this call fills completely
+};
+// The length and pattern set of the last sequence seen: a CTA's run of tasks covers few sequences.
+struct SeqCache {
+  int b, L, set;
 };
 
-// Task t of this call: (KV head, sequence, f-th page that the call fills completely).
-__device__ __forceinline__ Task task_of(const Geom& g, int n_new, int F, int64_t t, bool flag) {
+// Task t of this call: (KV head, sequence, f-th page that the call fills completely).  The
+// page-table entry is loaded here and checked by task_check, later, so that the load's latency
+// can overlap other work.
+__device__ __forceinline__ Task task_load(const Geom& g, int n_new, int F, int64_t t, SeqCache& sc) {
   Task k;
   k.h = (int)(t / ((int64_t)g.B * F));
   k.b = (int)((t / F) % g.B);
   const int f = (int)(t % F);
-  k.L = g.seq_len[k.b];
-  k.ok = false;
-  k.set = 0;
-  k.pg = 0;
-  if (k.L < 0 || (int64_t)k.L + n_new > (int64_t)g.maxp * kG) return k;  // flagged by the partial-page kernel
-  k.pg = (k.L + kG - 1) / kG + f;
-  if ((k.pg + 1) * kG > k.L + n_new) return k;
-  const int phys = g.page_table[(size_t)k.b * g.maxp + k.pg];
-  if (phys < 0 || phys >= g.npages) {
-    if (flag) set_status(g.status, KVQ_DEV_BAD_PAGE);
-    return k;
+  if (k.b != sc.b) {
+    sc.b = k.b;
+    sc.L = g.seq_len[k.b];
+    sc.set = g.seq_to_set ? g.seq_to_set[k.b] : 0;
   }
-  k.set = g.seq_to_set ? g.seq_to_set[k.b] : 0;
+  k.L = sc.L;
+  k.set = sc.set;
+  k.phys = -1;
+  k.pg = -1;
+  // a length out of range is flagged by the partial-page kernel
+  if (k.L < 0 || (int64_t)k.L + n_new > (int64_t)g.maxp * kG) return k;
+  const int pg = (k.L + kG - 1) / kG + f;
+  if ((pg + 1) * kG > k.L + n_new) return k;
+  k.pg = pg;
+  k.phys = g.page_table[(size_t)k.b * g.maxp + pg];
+  return k;
+}
+__device__ __forceinline__ bool task_check(const Geom& g, const Task& k, bool flag) {
+  if (k.pg < 0) return false;
+  if (k.phys < 0 || k.phys >= g.npages) {
+    if (flag) set_status(g.status, KVQ_DEV_BAD_PAGE);
+    return false;
+  }
   if (k.set < 0 || k.set >= g.S) {
     if (flag) set_status(g.status, KVQ_DEV_BAD_SET);
-    return k;
+    return false;
   }
-  k.ok = true;
-  return k;
+  return true;
 }
 
 
@@ -443,17 +457,19 @@ __global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_
   }
   __syncthreads();
 
-  // next valid task at or after t (t1 if none); the scan visits every task once, so thread 0
-  // flags bad page / set indices here
-  auto next_valid = [&](int64_t t) -> int64_t {
-    for (; t < t1; ++t)
-      if (task_of(g, n_new, F, t, tid == 0).ok) return t;
+  // next valid task at or after t (t1 if none), into `out`; the scan visits every task once, so
+  // thread 0 flags bad page / set indices here
+  SeqCache sc{-1, 0, 0};
+  auto next_valid = [&](int64_t t, Task& out) -> int64_t {
+    for (; t < t1; ++t) {
+      out = task_load(g, n_new, F, t, sc);
+      if (task_check(g, out, tid == 0)) return t;
+    }
     return t1;
   };
   uint32_t n_issued[2] = {0u, 0u};  // thread 0: copies issued into each stage
-  auto issue = [&](int64_t t, int buf) {
+  auto issue = [&](const Task& k, int buf) {
     ++n_issued[buf];
-    const Task k = task_of(g, n_new, F, t, false);
     uint8_t* dst = stage + buf * kStageBytes;
     const int tok = k.b * n_new + (k.pg * kG - k.L);
     fb_expect(&full[buf], kStageBytes);
@@ -463,27 +479,40 @@ __global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_
     tma3(dst + 12288, &kmap, 64, k.h, tok, &full[buf]);
   };
 
-  int64_t cur = next_valid(t0);
+  Task kc, kn;  // the current and the next task
+  int64_t cur = next_valid(t0, kc);
   if (tid == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
-    if (cur < t1) issue(cur, 0);
+    if (cur < t1) issue(kc, 0);
   }
-  int64_t nxt = cur < t1 ? next_valid(cur + 1) : t1;
-  if (tid == 0 && nxt < t1) issue(nxt, 1);
+  int64_t nxt = cur < t1 ? next_valid(cur + 1, kn) : t1;
+  if (tid == 0 && nxt < t1) issue(kn, 1);
+
+  bool timed_out = false;
+  if (cur < t1) {  // the first task's stage (later ones are awaited at the end of the task before)
+    if (!__all_sync(kFull, fb_wait(&full[0], 0u))) {
+      if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
+      timed_out = true;
+    }
+    if (__syncthreads_or(timed_out)) cur = t1;
+  }
 
   int cached_sh = -1;
-  bool timed_out = false;
   for (int i = 0; cur < t1; ++i) {
     const int buf = i & 1;
-    const Task k = task_of(g, n_new, F, cur, false);
+    const Task k = kc;
+    // the task after next: its loads now, its check at the end of this task
+    const int64_t ca = nxt + 1;
+    Task kca = kn;
+    if (nxt < t1 && ca < t1) kca = task_load(g, n_new, F, ca, sc);
     const int sh = k.set * g.H + k.h;
     const float* MK = g.kpat + (size_t)sh * P * kD;
     const float* MV = g.vpat + (size_t)sh * P * kD;
     const int Pe = p_eff(g, sh), Pep = (Pe + 7) & ~7;  // patterns in use (P is the capacity)
     const int S8 = (Pe + 7) >> 3;                        // patterns per warp in the bound passes
     const int j0w = min(Pe, warp * S8), nsl = min(Pe, j0w + S8) - j0w;
-    uint8_t* sub = g.pool + (size_t)g.page_table[(size_t)k.b * g.maxp + k.pg] * g.page_bytes + (size_t)k.h * g.sub_bytes;
+    uint8_t* sub = g.pool + (size_t)k.phys * g.page_bytes + (size_t)k.h * g.sub_bytes;
 
     // ---- pattern tables of this (set, head), staged when they change
     if (sh != cached_sh) {
@@ -517,11 +546,6 @@ __global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_
       __syncthreads();
     }
 
-    if (!__all_sync(kFull, fb_wait(&full[buf], (uint32_t)((i >> 1) & 1)))) {
-      if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
-      timed_out = true;
-    }
-    if (__syncthreads_or(timed_out)) break;
     uint8_t* stV = stage + buf * kStageBytes;  // V rows; K rows at + 8192
     uint8_t* stK = stV + 8192;
 
@@ -908,14 +932,22 @@ __global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_
       }
     }
 
-    // ---- stage free: issue the task after next into it (the generic accesses of this task to the
-    // stage ordered before the tensor copy that overwrites it)
+    // ---- end of the task: the next task's stage awaited (its copy was issued two tasks ago),
+    // then this stage refilled with the task after next (the generic accesses of this task to
+    // the stage ordered before the tensor copy that overwrites it)
+    int64_t after = t1;
+    if (nxt < t1 && ca < t1) after = task_check(g, kca, tid == 0) ? ca : next_valid(ca + 1, kca);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    const int64_t after = nxt < t1 ? next_valid(nxt + 1) : t1;
-    if (tid == 0 && after < t1) issue(after, buf);
+    if (nxt < t1 && !__all_sync(kFull, fb_wait(&full[buf ^ 1], (uint32_t)(((i + 1) >> 1) & 1)))) {
+      if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
+      timed_out = true;
+    }
+    if (__syncthreads_or(timed_out)) break;
+    if (tid == 0 && after < t1) issue(kca, buf);
     cur = nxt;
+    kc = kn;
     nxt = after;
+    kn = kca;
   }
   // drain (after a timeout): the newest copy issued into each stage must land before the CTA
   // exits; phases complete in order, so that covers the older ones
