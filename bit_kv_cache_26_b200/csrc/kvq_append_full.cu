@@ -52,7 +52,6 @@ namespace kvq {
 
 namespace {
 
-constexpr int kFThreads = 256;  // 8 warps; two CTAs per SM for up to 64 patterns
 constexpr int kProbeAll = 32;  // probe channels per pattern set in the prep tables
 constexpr int kV1 = 8;         // V: first-level bound channels
 constexpr int kV2 = 32;        // V: refined bound channels
@@ -329,38 +328,51 @@ __device__ __noinline__ void k_codes_exact(uint8_t* rowsK, const float* Rk, cons
   }
 }
 
-struct FullSmem {
-  int stage, rk, phi, hnorm, tabv, tabk, pcv, pck, xp, rowu, seed, best, kkey, rraw, ovf, lw2, lwe, ctr, kzr, ks, bars,
-      total;
+// Shared memory: the pattern tables of the current (set, head), shared by the CTA's groups, then
+// one block per group (its stage(s), the union of the probe values and candidate lists with the
+// K residuals, per-row state).
+template <int NG, int GW>
+struct FullCfg {
+  static constexpr int kGT = GW * 32;          // threads of a group
+  static constexpr int kNS = NG == 1 ? 2 : 1;  // stages per group
+  static constexpr int kXpBytes = 64 * kTabLd * 4;
+  static constexpr int kListBytes = GW * (kW2Cap + kWECap) * 2;
+  static constexpr int kRkBytes = 32 * kRkLd * 4;
+  static constexpr int kUnion = kRkBytes > kXpBytes + kListBytes ? kRkBytes : kXpBytes + kListBytes;
+  static constexpr int kStage = 0;
+  static constexpr int kU = kNS * kStageBytes;
+  static constexpr int kRowu = kU + kUnion;
+  static constexpr int kSeed = kRowu + 64 * 4;
+  static constexpr int kBest = kSeed + 64 * 4;
+  static constexpr int kKkey = kBest + 64 * 8;
+  static constexpr int kRraw = kKkey + 32 * 4;
+  static constexpr int kOvf = kRraw + 32 * 4;
+  static constexpr int kCtr = kOvf + 64 * 4;
+  static constexpr int kKzr = kCtr + 16;
+  static constexpr int kKs = kKzr + kD * 8;
+  static constexpr int kBars = kKs + kD * 4;
+  static constexpr int kGroupBytes = (kBars + 16 + 1023) & ~1023;  // keeps the stages 1024-byte aligned
 };
-__host__ __device__ inline FullSmem full_smem(int P) {
+struct TabSmem {
+  int phi, hnorm, tabv, tabk, pcv, pck, total;
+};
+__host__ __device__ inline TabSmem tab_smem(int P) {
   const int Pp = (P + 7) & ~7;
-  FullSmem s;
+  TabSmem s;
   int o = 0;
   auto take = [&](int bytes) { const int r = o; o = (o + bytes + 15) & ~15; return r; };
-  s.stage = take(2 * kStageBytes);
-  s.rk = take(32 * kRkLd * 4);
   s.phi = take(Pp * kPhiLd * 2);
   s.hnorm = take(Pp * 4);
   s.tabv = take(P * kTabLd * 4);
   s.tabk = take(P * kK1 * 4);
   s.pcv = take(kProbeAll * 4);
   s.pck = take(kK1 * 4);
-  s.xp = take(64 * kTabLd * 4);
-  s.rowu = take(64 * 4);
-  s.seed = take(64 * 4);
-  s.best = take(64 * 8);
-  s.kkey = take(32 * 4);
-  s.rraw = take(32 * 4);
-  s.ovf = take(64 * 4);
-  s.lw2 = take(8 * kW2Cap * 2);
-  s.lwe = take(8 * kWECap * 2);
-  s.ctr = take(4 * 4);
-  s.kzr = take(kD * 8);
-  s.ks = take(kD * 4);
-  s.bars = take(2 * 8);
-  s.total = o + 1024;  // room to align the stage buffers to 1024 B (128-byte swizzle atoms)
+  s.total = (o + 1023) & ~1023;
   return s;
+}
+template <int NG, int GW>
+inline int full_smem_bytes(int P) {
+  return tab_smem(P).total + NG * FullCfg<NG, GW>::kGroupBytes + 1024;  // + room to align the base
 }
 
 struct Task {
@@ -410,64 +422,105 @@ __device__ __forceinline__ bool task_check(const Geom& g, const Task& k, bool fl
 }
 
 
-template <int DT>
-__global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                   const __grid_constant__ CUtensorMap vmap, Geom g,
-                                                                   const int32_t* __restrict__ probe,
-                                                                   const float* __restrict__ pvals, int n_new,
-                                                                   int F, int64_t per_cta) {
+// The (set, head) whose pattern tables task t uses (the set clamped into range: a task with a bad
+// set index is skipped by task_check, whatever tables are staged).
+__device__ __forceinline__ int task_key(const Geom& g, int F, int64_t t, SeqCache& sc) {
+  const int h = (int)(t / ((int64_t)g.B * F));
+  const int b = (int)((t / F) % g.B);
+  if (b != sc.b) {
+    sc.b = b;
+    sc.L = g.seq_len[b];
+    sc.set = g.seq_to_set ? g.seq_to_set[b] : 0;
+  }
+  return min(max(sc.set, 0), g.S - 1) * g.H + h;
+}
+
+// NG groups of GW warps per CTA.  The CTA walks its run of tasks in segments of one (set, head):
+// all threads stage the segment's tables, then group gi takes the segment's tasks s0 + gi,
+// s0 + gi + NG, ... on its own (named barrier gi + 1, GW * 32 threads), so the groups' phases
+// interleave on the SM; a group's stage refills with its next task when the current one is done
+// (two stages, the copy two tasks ahead, when NG = 1).
+template <int DT, int NG, int GW>
+__global__ void __launch_bounds__(NG * GW * 32, 2) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                      const __grid_constant__ CUtensorMap vmap,
+                                                                      Geom g, const int32_t* __restrict__ probe,
+                                                                      const float* __restrict__ pvals, int n_new,
+                                                                      int F, int64_t per_cta) {
+  using C = FullCfg<NG, GW>;
+  constexpr int GT = C::kGT, CT = NG * GT, NS = C::kNS;
   extern __shared__ uint8_t smraw[];
   const int P = g.P, Pp = (P + 7) & ~7;
-  const FullSmem sp = full_smem(P);
+  const TabSmem ts = tab_smem(P);
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage = base + sp.stage;
-  float* Rk = reinterpret_cast<float*>(base + sp.rk);        // K residuals, rk_at(row, channel)
-  uint16_t* phi = reinterpret_cast<uint16_t*>(base + sp.phi);
-  float* hnorm = reinterpret_cast<float*>(base + sp.hnorm);
-  float* tabv = reinterpret_cast<float*>(base + sp.tabv);    // [P][kTabLd]: V patterns at the 32 probe channels
-  float* tabk = reinterpret_cast<float*>(base + sp.tabk);    // [P][16]: K patterns at the 16 probe channels
-  int32_t* pcv = reinterpret_cast<int32_t*>(base + sp.pcv);
-  int32_t* pck = reinterpret_cast<int32_t*>(base + sp.pck);
-  float* xp = reinterpret_cast<float*>(base + sp.xp);        // [64 rows][kTabLd]: rows at the probe channels
-  float* rowu = reinterpret_cast<float*>(base + sp.rowu);    // per row: exact distance to the seed
-  int32_t* rseed = reinterpret_cast<int32_t*>(base + sp.seed);
-  unsigned long long* best = reinterpret_cast<unsigned long long*>(base + sp.best);  // (distance, index) keys
-  uint32_t* kkey = reinterpret_cast<uint32_t*>(base + sp.kkey);  // K rows: smallest (bound, index), 7-bit tag
-  float* rraw = reinterpret_cast<float*>(base + sp.rraw);    // V rows: the vector's own range
-  int32_t* ovf = reinterpret_cast<int32_t*>(base + sp.ovf);  // per row: candidates dropped by a full list
-  uint16_t* lw2 = reinterpret_cast<uint16_t*>(base + sp.lw2);  // per warp: refinement list (V rows)
-  uint16_t* lwe = reinterpret_cast<uint16_t*>(base + sp.lwe);  // per warp: exact list (rows 0-31 V, 32-63 K)
-  int32_t* ctr = reinterpret_cast<int32_t*>(base + sp.ctr);  // [0] a tiny K scale, [1] a row overflowed
-  float2* kzr = reinterpret_cast<float2*>(base + sp.kzr);    // per K channel: z, 1/s
-  float* kss = reinterpret_cast<float*>(base + sp.ks);       // per K channel: s
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + sp.bars);
+  uint16_t* phi = reinterpret_cast<uint16_t*>(base + ts.phi);
+  float* hnorm = reinterpret_cast<float*>(base + ts.hnorm);
+  float* tabv = reinterpret_cast<float*>(base + ts.tabv);  // [P][kTabLd]: V patterns at the 32 probe channels
+  float* tabk = reinterpret_cast<float*>(base + ts.tabk);  // [P][16]: K patterns at the 16 probe channels
+  int32_t* pcv = reinterpret_cast<int32_t*>(base + ts.pcv);
+  int32_t* pck = reinterpret_cast<int32_t*>(base + ts.pck);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int gi = tid / GT, gtid = tid % GT, gw = gtid >> 5;  // group; thread and warp in the group
+  uint8_t* gb = base + ts.total + gi * C::kGroupBytes;
+  uint8_t* stage = gb + C::kStage;
+  float* Rk = reinterpret_cast<float*>(gb + C::kU);  // K residuals, rk_at(row, channel): phases F-H
+  float* xp = reinterpret_cast<float*>(gb + C::kU);  // [64 rows][kTabLd] probe values: phases A-D
+  uint16_t* wl2 = reinterpret_cast<uint16_t*>(gb + C::kU + C::kXpBytes) + gw * kW2Cap;  // warp's refinement list
+  uint16_t* wle = reinterpret_cast<uint16_t*>(gb + C::kU + C::kXpBytes + GW * kW2Cap * 2) + gw * kWECap;
+  float* rowu = reinterpret_cast<float*>(gb + C::kRowu);  // per row: exact distance to the seed
+  int32_t* rseed = reinterpret_cast<int32_t*>(gb + C::kSeed);
+  unsigned long long* best = reinterpret_cast<unsigned long long*>(gb + C::kBest);  // (distance, index) keys
+  uint32_t* kkey = reinterpret_cast<uint32_t*>(gb + C::kKkey);  // K rows: smallest (bound, index), 7-bit tag
+  float* rraw = reinterpret_cast<float*>(gb + C::kRraw);      // V rows: the vector's own range
+  int32_t* ovf = reinterpret_cast<int32_t*>(gb + C::kOvf);    // per row: candidates dropped by a full list
+  int32_t* ctr = reinterpret_cast<int32_t*>(gb + C::kCtr);    // [0] a tiny K scale, [1] a row overflowed
+  float2* kzr = reinterpret_cast<float2*>(gb + C::kKzr);      // per K channel: z, 1/s
+  float* kss = reinterpret_cast<float*>(gb + C::kKs);         // per K channel: s
+  uint64_t* full = reinterpret_cast<uint64_t*>(gb + C::kBars);
   const int maxc = (1 << g.bits) - 1;
-  uint16_t* wl2 = lw2 + warp * kW2Cap;
-  uint16_t* wle = lwe + warp * kWECap;
+  // group barriers: named barrier 1 (group 0) or 2 (group 1), the group's threads
+  auto gsync = [&]() {
+    if (gi == 0) asm volatile("bar.sync 1, %0;" ::"n"(GT) : "memory");
+    else asm volatile("bar.sync 2, %0;" ::"n"(GT) : "memory");
+  };
+  auto gsync_or = [&](bool v) -> bool {
+    uint32_t r;
+    if (gi == 0)
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+          : "=r"(r)
+          : "r"((uint32_t)v), "n"(GT)
+          : "memory");
+    else
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+          : "=r"(r)
+          : "r"((uint32_t)v), "n"(GT)
+          : "memory");
+    return r != 0u;
+  };
 
   const int64_t T = (int64_t)g.H * g.B * F;
   const int64_t t0 = (int64_t)blockIdx.x * per_cta, t1 = min(T, t0 + per_cta);
 
-  if (tid == 0) {
-    fb_init(&full[0], 1);
-    fb_init(&full[1], 1);
+  if (gtid == 0) {
+    for (int s2 = 0; s2 < NS; ++s2) fb_init(&full[s2], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  // next valid task at or after t (t1 if none), into `out`; the scan visits every task once, so
-  // thread 0 flags bad page / set indices here
-  SeqCache sc{-1, 0, 0};
-  auto next_valid = [&](int64_t t, Task& out) -> int64_t {
-    for (; t < t1; ++t) {
+  SeqCache sc{-1, 0, 0};   // sequence facts for the task walk
+  SeqCache ksc{-1, 0, 0};  // and for the segment keys
+  // next valid task of this group at or after t (stride NG) before e, into `out`; each task of
+  // the group is checked once, so the group's thread 0 flags bad page / set indices here
+  auto next_valid = [&](int64_t t, int64_t e, Task& out) -> int64_t {
+    for (; t < e; t += NG) {
       out = task_load(g, n_new, F, t, sc);
-      if (task_check(g, out, tid == 0)) return t;
+      if (task_check(g, out, gtid == 0)) return t;
     }
-    return t1;
+    return e;
   };
-  uint32_t n_issued[2] = {0u, 0u};  // thread 0: copies issued into each stage
+  uint32_t n_issued[2] = {0u, 0u};  // group thread 0: copies issued into each stage
   auto issue = [&](const Task& k, int buf) {
     ++n_issued[buf];
     uint8_t* dst = stage + buf * kStageBytes;
@@ -478,482 +531,512 @@ __global__ void __launch_bounds__(kFThreads, 2) append_full_kernel(const __grid_
     tma3(dst + 8192, &kmap, 0, k.h, tok, &full[buf]);
     tma3(dst + 12288, &kmap, 64, k.h, tok, &full[buf]);
   };
-
-  Task kc, kn;  // the current and the next task
-  int64_t cur = next_valid(t0, kc);
-  if (tid == 0) {
+  if (gtid == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
-    if (cur < t1) issue(kc, 0);
-  }
-  int64_t nxt = cur < t1 ? next_valid(cur + 1, kn) : t1;
-  if (tid == 0 && nxt < t1) issue(kn, 1);
-
-  bool timed_out = false;
-  if (cur < t1) {  // the first task's stage (later ones are awaited at the end of the task before)
-    if (!__all_sync(kFull, fb_wait(&full[0], 0u))) {
-      if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
-      timed_out = true;
-    }
-    if (__syncthreads_or(timed_out)) cur = t1;
   }
 
-  int cached_sh = -1;
-  for (int i = 0; cur < t1; ++i) {
-    const int buf = i & 1;
-    const Task k = kc;
-    // the task after next: its loads now, its check at the end of this task
-    const int64_t ca = nxt + 1;
-    Task kca = kn;
-    if (nxt < t1 && ca < t1) kca = task_load(g, n_new, F, ca, sc);
-    const int sh = k.set * g.H + k.h;
+  bool dead = false;             // a stage wait of this group expired: it only joins the segment barriers
+  uint32_t waits[2] = {0u, 0u};  // completed waits per stage: the parity of the next one
+  int q_ = 0;                    // this group's tasks so far: the stage of the next one is q_ % NS
+  for (int64_t s0 = t0; s0 < t1;) {
+    // ---- the segment [s0, s1) of one (set, head); every thread computes the same bounds
+    const int sh = task_key(g, F, s0, ksc);
+    int64_t s1 = s0 + 1;
+    while (s1 < t1 && task_key(g, F, s1, ksc) == sh) ++s1;
     const float* MK = g.kpat + (size_t)sh * P * kD;
     const float* MV = g.vpat + (size_t)sh * P * kD;
     const int Pe = p_eff(g, sh), Pep = (Pe + 7) & ~7;  // patterns in use (P is the capacity)
-    const int S8 = (Pe + 7) >> 3;                        // patterns per warp in the bound passes
-    const int j0w = min(Pe, warp * S8), nsl = min(Pe, j0w + S8) - j0w;
-    uint8_t* sub = g.pool + (size_t)k.phys * g.page_bytes + (size_t)k.h * g.sub_bytes;
+    const int Sw = (Pe + GW - 1) / GW;                   // patterns per warp in the bound passes
+    const int j0w = min(Pe, gw * Sw), nsl = min(Pe, j0w + Sw) - j0w;
 
-    // ---- pattern tables of this (set, head), staged when they change
-    if (sh != cached_sh) {
-      cached_sh = sh;
-      for (int i4 = tid; i4 < Pp * (kD / 4); i4 += kFThreads) {
-        const int n = i4 / (kD / 4), c4 = i4 % (kD / 4);
-        float4 m = n < Pe ? __ldg(reinterpret_cast<const float4*>(MV + (size_t)n * kD) + c4) : make_float4(0, 0, 0, 0);
-        uint16_t h4[4];
-        const float mv[4] = {m.x, m.y, m.z, m.w};
+    // this group's first tasks of the segment: their copies go out before the tables are staged
+    Task kc, kn;
+    int64_t cur = dead ? s1 : next_valid(s0 + gi, s1, kc);
+    if (gtid == 0 && cur < s1) issue(kc, q_ % NS);
+    int64_t nxt = s1;
+    if (NS == 2 && cur < s1) {
+      nxt = next_valid(cur + NG, s1, kn);
+      if (gtid == 0 && nxt < s1) issue(kn, (q_ + 1) % NS);
+    }
+
+    // ---- pattern tables of this (set, head), by every thread (the previous segment is done)
+    __syncthreads();
+    for (int i4 = tid; i4 < Pp * (kD / 4); i4 += CT) {
+      const int n = i4 / (kD / 4), c4 = i4 % (kD / 4);
+      float4 m = n < Pe ? __ldg(reinterpret_cast<const float4*>(MV + (size_t)n * kD) + c4) : make_float4(0, 0, 0, 0);
+      uint16_t h4[4];
+      const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float v = -fminf(fmaxf(mv[e], -60000.f), 60000.f);
-          h4[e] = DT == KVQ_BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+      for (int e = 0; e < 4; ++e) {
+        const float v = -fminf(fmaxf(mv[e], -60000.f), 60000.f);
+        h4[e] = DT == KVQ_BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+      }
+      *reinterpret_cast<uint2*>(phi + (size_t)n * kPhiLd + 4 * c4) =
+          make_uint2(h4[0] | ((uint32_t)h4[1] << 16), h4[2] | ((uint32_t)h4[3] << 16));
+    }
+    for (int n = tid; n < Pp; n += CT) {
+      float acc = 0.f;
+      if (n < Pe) {
+        const float4* m4 = reinterpret_cast<const float4*>(MV + (size_t)n * kD);
+        for (int c = 0; c < kD / 4; ++c) {
+          const float4 m = __ldg(m4 + c);
+          acc = fmaf(m.x, m.x, acc);
+          acc = fmaf(m.y, m.y, acc);
+          acc = fmaf(m.z, m.z, acc);
+          acc = fmaf(m.w, m.w, acc);
         }
-        *reinterpret_cast<uint2*>(phi + (size_t)n * kPhiLd + 4 * c4) =
-            make_uint2(h4[0] | ((uint32_t)h4[1] << 16), h4[2] | ((uint32_t)h4[3] << 16));
       }
-      for (int n = tid; n < Pp; n += kFThreads) {
-        float acc = 0.f;
-        if (n < Pe)
-          for (int c = 0; c < kD; ++c) { const float m = __ldg(MV + (size_t)n * kD + c); acc = fmaf(m, m, acc); }
-        hnorm[n] = n < Pe ? 0.5f * acc : 1e30f;
-      }
+      hnorm[n] = n < Pe ? 0.5f * acc : 1e30f;
+    }
+    {
       const size_t o = (size_t)sh * 2;
-      for (int q = tid; q < Pe * kProbeAll; q += kFThreads)
+      for (int q = tid; q < Pe * kProbeAll; q += CT)
         tabv[(q / kProbeAll) * kTabLd + q % kProbeAll] = __ldg(pvals + (o + 1) * P * kProbeAll + q);
-      for (int q = tid; q < Pe * kK1; q += kFThreads)
+      for (int q = tid; q < Pe * kK1; q += CT)
         tabk[q] = __ldg(pvals + o * P * kProbeAll + (size_t)(q / kK1) * kProbeAll + q % kK1);
       if (tid < kProbeAll) pcv[tid] = __ldg(probe + (o + 1) * kProbeAll + tid);
       if (tid < kK1) pck[tid] = __ldg(probe + o * kProbeAll + tid);
-      __syncthreads();
-    }
-
-    uint8_t* stV = stage + buf * kStageBytes;  // V rows; K rows at + 8192
-    uint8_t* stK = stV + 8192;
-
-    // ---- A: V seeds on the tensor cores; probe values of every row; per-task resets
-    if (warp < 2) {
-      const uint32_t rows_s = s32(stV);
-      const int r = lane & 15;
-      const int rb = 16 * (warp & 1);
-      uint32_t A[8][4];
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const int arow = rb + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int ach = 16 * ks + 8 * (lane >> 4);
-        ldsm4(rows_s + elem_off(arow, ach), A[ks][0], A[ks][1], A[ks][2], A[ks][3]);
-      }
-      const int tig = lane & 3;
-      float b0 = INFINITY, b8 = INFINITY;  // tagged scores of rows gq and gq + 8
-      for (int nt = 0; nt < Pep / 8; ++nt) {
-        float acc[4];
-        acc[0] = acc[2] = hnorm[8 * nt + 2 * tig];
-        acc[1] = acc[3] = hnorm[8 * nt + 2 * tig + 1];
-        const uint32_t bbase = s32(phi + (size_t)(8 * nt + (lane & 7)) * kPhiLd + 8 * (lane >> 3));
-#pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          uint32_t q0, q1, q2, q3;
-          ldsm4(bbase + kp * 64, q0, q1, q2, q3);  // k-steps 2kp (q0, q1) and 2kp + 1 (q2, q3)
-          mma_seed<DT>(acc, A[2 * kp][0], A[2 * kp][1], A[2 * kp][2], A[2 * kp][3], q0, q1);
-          mma_seed<DT>(acc, A[2 * kp + 1][0], A[2 * kp + 1][1], A[2 * kp + 1][2], A[2 * kp + 1][3], q2, q3);
-        }
-        const int j0 = 8 * nt + 2 * tig;
-        b0 = fminf(b0, fminf(__uint_as_float((__float_as_uint(acc[0]) & ~127u) | (uint32_t)j0),
-                             __uint_as_float((__float_as_uint(acc[1]) & ~127u) | (uint32_t)(j0 + 1))));
-        b8 = fminf(b8, fminf(__uint_as_float((__float_as_uint(acc[2]) & ~127u) | (uint32_t)j0),
-                             __uint_as_float((__float_as_uint(acc[3]) & ~127u) | (uint32_t)(j0 + 1))));
-      }
-      b0 = fminf(b0, __shfl_xor_sync(kFull, b0, 1));
-      b0 = fminf(b0, __shfl_xor_sync(kFull, b0, 2));
-      b8 = fminf(b8, __shfl_xor_sync(kFull, b8, 1));
-      b8 = fminf(b8, __shfl_xor_sync(kFull, b8, 2));
-      const float s_lo = __shfl_sync(kFull, b0, 4 * (r & 7)), s_hi = __shfl_sync(kFull, b8, 4 * (r & 7));
-      int seed = (int)(__float_as_uint(r < 8 ? s_lo : s_hi) & 127u);
-      seed = min(seed, Pe - 1);
-
-      if (lane < 16) rseed[16 * warp + r] = seed;
-    } else {
-      const int u = tid - 64;  // 0..191
-      if (u < 128) {  // V rows: 32 probe values, 8 per thread
-        const int row = u >> 2, k0 = 8 * (u & 3);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          xp[row * kTabLd + k0 + e] = cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stV + elem_off(row, pcv[k0 + e])));
-      } else {  // K rows: 16 probe values, 8 per thread
-        const int row = (u - 128) >> 1, k0 = 8 * (u & 1);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          xp[(32 + row) * kTabLd + k0 + e] =
-              cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stK + elem_off(row, pck[k0 + e])));
-      }
-      if (u < 64) ovf[u] = 0;
-      else if (u < 96) kkey[u - 64] = 0xFFFFFFFFu;
-      else if (u == 96) ctr[0] = ctr[1] = 0;
     }
     __syncthreads();
 
-    // ---- B: V rows: exact distance to the seed and own range (4 threads a row)
-    if (warp < 4) {
-      const int r = tid >> 2, q = tid & 3;
-      float x[32];
-      load_x32<DT>(stV, r, q, x);
-      const int s = rseed[r];
-      float mx, mn, ymx = -INFINITY, ymn = INFINITY;
-      range32(x, MV + (size_t)s * kD + 32 * q, mx, mn);
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        ymx = max3(ymx, x[c], x[c + 1]);
-        ymn = min3(ymn, x[c], x[c + 1]);
-      }
-#pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
-        ymx = fmaxf(ymx, __shfl_xor_sync(kFull, ymx, o));
-        ymn = fminf(ymn, __shfl_xor_sync(kFull, ymn, o));
-      }
-      if (q == 0) {
-        const float U = __fsub_rn(mx, mn);
-        rowu[r] = U;
-        best[r] = dkey(U, s);
-        rraw[r] = __fsub_rn(ymx, ymn);
-      }
-    }
-    // K rows: bounds over 16 probe channels for this warp's patterns (lane = K row), kept in
-    // registers until the K candidates are listed; the smallest (tagged with its index in the 7
-    // low bits) names the seed
-    float klb[kMaxSlice];
-    {
-      float y[kK1];
-#pragma unroll
-      for (int q = 0; q < kK1 / 4; ++q) {
-        const float4 a = reinterpret_cast<const float4*>(xp + (32 + lane) * kTabLd)[q];
-        y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
-      }
-      uint32_t kb = 0xFFFFFFFFu;
-#pragma unroll
-      for (int jj = 0; jj < kMaxSlice; ++jj) {
-        klb[jj] = INFINITY;
-        if (jj < nsl) {
-          const int j = j0w + jj;
-          klb[jj] = probe_range_reg<kK1>(y, tabk + (size_t)j * kK1);
-          kb = min(kb, (__float_as_uint(klb[jj]) & ~127u) | (uint32_t)j);
-        }
-      }
-      if (nsl > 0) atomicMin(&kkey[lane], kb);
-    }
-    __syncthreads();
+    // ---- this group's tasks of the segment
+    while (cur < s1) {
+      const int buf = q_ % NS;
+      const Task k = kc;
+      // the group's task after the ones in flight: its loads now, its check at the end
+      const int64_t ca = (NS == 2 ? nxt : cur) + NG;
+      Task kca = kc;
+      if (ca < s1 && (NS == 1 || nxt < s1)) kca = task_load(g, n_new, F, ca, sc);
+      uint8_t* sub = g.pool + (size_t)k.phys * g.page_bytes + (size_t)k.h * g.sub_bytes;
 
-    // ---- C: K rows: exact distance to the seed (4 threads a row)
-    if (warp >= 4) {
-      const int r = (tid - 128) >> 2, q = tid & 3;
-      const int s = min((int)(kkey[r] & 127u), Pe - 1);
-      float x[32];
-      load_x32<DT>(stK, r, q, x);
-      float mx, mn;
-      range32(x, MK + (size_t)s * kD + 32 * q, mx, mn);
-#pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+      if (__all_sync(kFull, fb_wait(&full[buf], waits[buf] & 1u))) {
+        ++waits[buf];
+      } else {
+        if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
+        dead = true;
       }
-      if (q == 0) {
-        const float U = __fsub_rn(mx, mn);
-        rowu[32 + r] = U;
-        rseed[32 + r] = s;
-        best[32 + r] = dkey(U, s);
+      if (gsync_or(dead)) {
+        dead = true;
+        break;
       }
-    }
-    // V rows: bounds over 8 probe channels for this warp's patterns (lane = V row); a pattern
-    // that could still beat the seed, or tie it with a lower index, goes on the warp's refinement
-    // list, whose bounds over 32 probe channels pass the survivors to the warp's exact list
-    int nE = 0;  // entries in this warp's exact list (the same in every lane)
-    {
-      float y[kV1];
-#pragma unroll
-      for (int q = 0; q < kV1 / 4; ++q) {
-        const float4 a = reinterpret_cast<const float4*>(xp + lane * kTabLd)[q];
-        y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
-      }
-      const float U = rowu[lane];
-      const int s = rseed[lane];
-      uint32_t mask = 0u;
-#pragma unroll
-      for (int jj = 0; jj < kMaxSlice; ++jj) {
-        if (jj < nsl) {
-          const int j = j0w + jj;
-          const float lb = probe_range_reg<kV1>(y, tabv + (size_t)j * kTabLd);
-          if (j != s && (lb < U || (lb == U && j < s))) mask |= 1u << jj;
-        }
-      }
-      const int n2 = warp_compact(mask, lane, lane, j0w, wl2, 0, kW2Cap, &ovf[lane], &ctr[1]);
-      __syncwarp();
-      for (int b0 = 0; b0 < n2; b0 += 32) {
-        const int e = b0 + lane;
-        bool live = false;
-        uint32_t ent = 0u;
-        int r = 0;
-        if (e < n2) {
-          ent = wl2[e];
-          r = (int)(ent >> 8);
-          const int j = (int)(ent & 255u);
-          const float lb = probe_range<kV2>(xp + r * kTabLd, tabv + (size_t)j * kTabLd);
-          const float Ur = rowu[r];
-          live = lb < Ur || (lb == Ur && j < rseed[r]);
-        }
-        nE = warp_append(live, ent, wle, nE, kWECap, &ovf[r], &ctr[1], lane);
-      }
-    }
-    __syncthreads();
+      uint8_t* stV = stage + buf * kStageBytes;  // V rows; K rows at + 8192
+      uint8_t* stK = stV + 8192;
 
-    // ---- D: the K candidates of this warp's eighth join its exact list; exact distances of the
-    // list (4 lanes an entry), minimum (distance, index) per row
-    const int q4 = lane & 3;
-    auto exact = [&](bool on, int row, int j) {
-      float mx = -INFINITY, mn = INFINITY;
-      if (on) {
+      // ---- A: V seeds on the tensor cores (warps 0-1); probe values of every row; resets
+      if (gw < 2) {
+        const uint32_t rows_s = s32(stV);
+        const int r = lane & 15;
+        const int rb = 16 * (gw & 1);
+        uint32_t A[8][4];
+  #pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int arow = rb + (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int ach = 16 * ks + 8 * (lane >> 4);
+          ldsm4(rows_s + elem_off(arow, ach), A[ks][0], A[ks][1], A[ks][2], A[ks][3]);
+        }
+        const int tig = lane & 3;
+        float b0 = INFINITY, b8 = INFINITY;  // tagged scores of rows gq and gq + 8
+        for (int nt = 0; nt < Pep / 8; ++nt) {
+          float acc[4];
+          acc[0] = acc[2] = hnorm[8 * nt + 2 * tig];
+          acc[1] = acc[3] = hnorm[8 * nt + 2 * tig + 1];
+          const uint32_t bbase = s32(phi + (size_t)(8 * nt + (lane & 7)) * kPhiLd + 8 * (lane >> 3));
+  #pragma unroll
+          for (int kp = 0; kp < 4; ++kp) {
+            uint32_t q0, q1, q2, q3;
+            ldsm4(bbase + kp * 64, q0, q1, q2, q3);  // k-steps 2kp (q0, q1) and 2kp + 1 (q2, q3)
+            mma_seed<DT>(acc, A[2 * kp][0], A[2 * kp][1], A[2 * kp][2], A[2 * kp][3], q0, q1);
+            mma_seed<DT>(acc, A[2 * kp + 1][0], A[2 * kp + 1][1], A[2 * kp + 1][2], A[2 * kp + 1][3], q2, q3);
+          }
+          const int j0 = 8 * nt + 2 * tig;
+          b0 = fminf(b0, fminf(__uint_as_float((__float_as_uint(acc[0]) & ~127u) | (uint32_t)j0),
+                               __uint_as_float((__float_as_uint(acc[1]) & ~127u) | (uint32_t)(j0 + 1))));
+          b8 = fminf(b8, fminf(__uint_as_float((__float_as_uint(acc[2]) & ~127u) | (uint32_t)j0),
+                               __uint_as_float((__float_as_uint(acc[3]) & ~127u) | (uint32_t)(j0 + 1))));
+        }
+        b0 = fminf(b0, __shfl_xor_sync(kFull, b0, 1));
+        b0 = fminf(b0, __shfl_xor_sync(kFull, b0, 2));
+        b8 = fminf(b8, __shfl_xor_sync(kFull, b8, 1));
+        b8 = fminf(b8, __shfl_xor_sync(kFull, b8, 2));
+        const float s_lo = __shfl_sync(kFull, b0, 4 * (r & 7)), s_hi = __shfl_sync(kFull, b8, 4 * (r & 7));
+        int seed = (int)(__float_as_uint(r < 8 ? s_lo : s_hi) & 127u);
+        seed = min(seed, Pe - 1);
+
+        if (lane < 16) rseed[16 * gw + r] = seed;
+      } else {
+        // V rows: 32 probe values, K rows 16; units of 8 values
+        for (int u = gtid - 64; u < 192; u += GT - 64) {
+          if (u < 128) {
+            const int row = u >> 2, k0 = 8 * (u & 3);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              xp[row * kTabLd + k0 + e] =
+                  cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stV + elem_off(row, pcv[k0 + e])));
+          } else {
+            const int row = (u - 128) >> 1, k0 = 8 * (u & 1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              xp[(32 + row) * kTabLd + k0 + e] =
+                  cvt_lo<DT>(*reinterpret_cast<const uint16_t*>(stK + elem_off(row, pck[k0 + e])));
+          }
+        }
+        for (int u = gtid - 64; u < 97; u += GT - 64) {
+          if (u < 64) ovf[u] = 0;
+          else if (u < 96) kkey[u - 64] = 0xFFFFFFFFu;
+          else ctr[0] = ctr[1] = 0;
+        }
+      }
+      gsync();
+
+      // ---- B: V rows: exact distance to the seed and own range (4 threads a row)
+      for (int u = gtid; u < 128; u += GT) {
+        const int r = u >> 2, q = u & 3;
         float x[32];
-        load_x32<DT>(row < 32 ? stV : stK, row & 31, q4, x);
-        range32(x, (row < 32 ? MV : MK) + (size_t)j * kD + 32 * q4, mx, mn);
-      }
+        load_x32<DT>(stV, r, q, x);
+        const int s = rseed[r];
+        float mx, mn, ymx = -INFINITY, ymn = INFINITY;
+        range32(x, MV + (size_t)s * kD + 32 * q, mx, mn);
 #pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
-      }
-      if (on && q4 == 0) atomicMin(&best[row], dkey(__fsub_rn(mx, mn), j));
-    };
-    {
-      const float U = rowu[32 + lane];
-      const int s = rseed[32 + lane];
-      uint32_t mask = 0u;
+        for (int c = 0; c < 32; c += 2) {
+          ymx = max3(ymx, x[c], x[c + 1]);
+          ymn = min3(ymn, x[c], x[c + 1]);
+        }
 #pragma unroll
-      for (int jj = 0; jj < kMaxSlice; ++jj)
-        if (jj < nsl && j0w + jj != s && klb[jj] <= U) mask |= 1u << jj;
-      nE = warp_compact(mask, lane, 32 + lane, j0w, wle, nE, kWECap, &ovf[32 + lane], &ctr[1]);
-      __syncwarp();
-      for (int b0 = 0; b0 < nE; b0 += 8) {
-        const int e = b0 + (lane >> 2);
-        const uint32_t ent = e < nE ? wle[e] : 0u;
-        exact(e < nE, (int)(ent >> 8), (int)(ent & 255u));
-      }
-    }
-    __syncthreads();
-    if (ctr[1]) {
-      // some row's candidates did not all fit a list: that row against every pattern
-      for (int row = 0; row < 64; ++row) {
-        if (!ovf[row]) continue;
-        for (int jb = 0; jb < Pe; jb += 8) {
-          const int j = jb + (lane >> 2) + 0;
-          if (warp == 0) exact(j < Pe, row, j);  // one warp: the rows are rare
+        for (int o = 1; o <= 2; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+          mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+          ymx = fmaxf(ymx, __shfl_xor_sync(kFull, ymx, o));
+          ymn = fminf(ymn, __shfl_xor_sync(kFull, ymn, o));
+        }
+        if (q == 0) {
+          const float U = __fsub_rn(mx, mn);
+          rowu[r] = U;
+          best[r] = dkey(U, s);
+          rraw[r] = __fsub_rn(ymx, ymn);
         }
       }
-      __syncthreads();
-    }
+      // K rows: bounds over 16 probe channels for this warp's patterns (lane = K row), kept in
+      // registers until the K candidates are listed; the smallest (tagged with its index in the 7
+      // low bits) names the seed
+      float klb[kMaxSlice];
+      {
+        float y[kK1];
+#pragma unroll
+        for (int q = 0; q < kK1 / 4; ++q) {
+          const float4 a = reinterpret_cast<const float4*>(xp + (32 + lane) * kTabLd)[q];
+          y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
+        }
+        uint32_t kb = 0xFFFFFFFFu;
+#pragma unroll
+        for (int jj = 0; jj < kMaxSlice; ++jj) {
+          klb[jj] = INFINITY;
+          if (jj < nsl) {
+            const int j = j0w + jj;
+            klb[jj] = probe_range_reg<kK1>(y, tabk + (size_t)j * kK1);
+            kb = min(kb, (__float_as_uint(klb[jj]) & ~127u) | (uint32_t)j);
+          }
+        }
+        if (nsl > 0) atomicMin(&kkey[lane], kb);
+      }
+      gsync();
 
-    // ---- F: V rows quantized (a thread a row and 32-channel group); K residuals staged
-    if (warp < 4) {
-      const int r = tid >> 2, q = tid & 3;
-      const unsigned long long bk = best[r];
-      const int j = (int)(bk & 0xffffffffu);
-      const bool keep = v_keep_pattern(g.vrho, __uint_as_float((uint32_t)(bk >> 32)), rraw[r]);
-      float x[32];
-      load_x32<DT>(stV, r, q, x);
-      const float* mrow = MV + (size_t)j * kD + 32 * q;
-      if (keep) {
-        const float4* m4 = reinterpret_cast<const float4*>(mrow);
-        float4 mv[8];
+      // ---- C: K rows: exact distance to the seed (4 threads a row)
+      for (int u = gtid; u < 128; u += GT) {
+        const int r = u >> 2, q = u & 3;
+        const int s = min((int)(kkey[r] & 127u), Pe - 1);
+        float x[32];
+        load_x32<DT>(stK, r, q, x);
+        float mx, mn;
+        range32(x, MK + (size_t)s * kD + 32 * q, mx, mn);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, x[4 * c], x[4 * c + 1]);
-          sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, x[4 * c + 2], x[4 * c + 3]);
+        for (int o = 1; o <= 2; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+          mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+        }
+        if (q == 0) {
+          const float U = __fsub_rn(mx, mn);
+          rowu[32 + r] = U;
+          rseed[32 + r] = s;
+          best[32 + r] = dkey(U, s);
         }
       }
-      float gmx = -INFINITY, gmn = INFINITY;
+      // V rows: bounds over 8 probe channels for this warp's patterns (lane = V row); a pattern
+      // that could still beat the seed, or tie it with a lower index, goes on the warp's
+      // refinement list, whose bounds over 32 probe channels pass the survivors to its exact list
+      int nE = 0;  // entries in this warp's exact list (the same in every lane)
+      {
+        float y[kV1];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        gmx = max3(gmx, x[c], x[c + 1]);
-        gmn = min3(gmn, x[c], x[c + 1]);
+        for (int q = 0; q < kV1 / 4; ++q) {
+          const float4 a = reinterpret_cast<const float4*>(xp + lane * kTabLd)[q];
+          y[4 * q] = a.x; y[4 * q + 1] = a.y; y[4 * q + 2] = a.z; y[4 * q + 3] = a.w;
+        }
+        const float U = rowu[lane];
+        const int s = rseed[lane];
+        uint32_t mask = 0u;
+#pragma unroll
+        for (int jj = 0; jj < kMaxSlice; ++jj) {
+          if (jj < nsl) {
+            const int j = j0w + jj;
+            const float lb = probe_range_reg<kV1>(y, tabv + (size_t)j * kTabLd);
+            if (j != s && (lb < U || (lb == U && j < s))) mask |= 1u << jj;
+          }
+        }
+        const int n2 = warp_compact(mask, lane, lane, j0w, wl2, 0, kW2Cap, &ovf[lane], &ctr[1]);
+        __syncwarp();
+        for (int b0 = 0; b0 < n2; b0 += 32) {
+          const int e = b0 + lane;
+          bool live = false;
+          uint32_t ent = 0u;
+          int r = 0;
+          if (e < n2) {
+            ent = wl2[e];
+            r = (int)(ent >> 8);
+            const int j = (int)(ent & 255u);
+            const float lb = probe_range<kV2>(xp + r * kTabLd, tabv + (size_t)j * kTabLd);
+            const float Ur = rowu[r];
+            live = lb < Ur || (lb == Ur && j < rseed[r]);
+          }
+          nE = warp_append(live, ent, wle, nE, kWECap, &ovf[r], &ctr[1], lane);
+        }
       }
-      const float s = __fdiv_rn(__fsub_rn(gmx, gmn), (float)maxc);
-      const float ri = code_rcp(s);
-      reinterpret_cast<float*>(sub + g.off_vs)[vsc_pos(r, q)] = s;
-      reinterpret_cast<float*>(sub + g.off_vz)[vzc_pos(r, q)] = gmn;
-      if (q == 0) sub[g.off_vidx + tok_pos(r)] = keep ? (uint8_t)j : (uint8_t)kRawIndex;
-      uint32_t pc[16];
-      const bool clean = codes_fma<32>(x, pc, [&](int, float& z0, float& z1, float& r0, float& r1) {
-        z0 = z1 = gmn;
-        r0 = r1 = ri;
-      });
-      if (clean && !tiny_scale(s)) {
-        uint8_t* hb = stV + (q >> 1) * 4096;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          *reinterpret_cast<uint4*>(hb + swz(r, 4 * (q & 1) + cc)) =
-              make_uint4(pc[4 * cc], pc[4 * cc + 1], pc[4 * cc + 2], pc[4 * cc + 3]);
-      } else {
-        v_codes_exact<DT>(stV, r, q, keep ? mrow : nullptr, gmn, s, maxc);
-      }
-    } else {
-      const int r = (tid - 128) >> 2, q = tid & 3;
-      const int j = (int)(best[32 + r] & 0xffffffffu);
-      float x[32];
-      load_x32<DT>(stK, r, q, x);
-      const float4* m4 = reinterpret_cast<const float4*>(MK + (size_t)j * kD + 32 * q);
-      float4 mv[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
-      float4* dst = reinterpret_cast<float4*>(Rk + rk_at(r, 32 * q));
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float4 o;
-        sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, o.x, o.y);
-        sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, o.z, o.w);
-        dst[c] = o;
-      }
-      if (q == 0) sub[g.off_kidx + tok_pos(r)] = (uint8_t)j;
-    }
-    __syncthreads();
+      gsync();
 
-    // ---- G: K scale and zero per channel over the page (a thread a channel)
-    if (tid < kD) {
-      const int c = tid;
-      const float* col = Rk + rk_at(0, c);
-      float mx = -INFINITY, mn = INFINITY;
+      // ---- D: the K candidates of this warp's patterns join its exact list; exact distances of
+      // the list (4 lanes an entry), minimum (distance, index) per row
+      const int q4 = lane & 3;
+      auto exact = [&](bool on, int row, int j) {
+        float mx = -INFINITY, mn = INFINITY;
+        if (on) {
+          float x[32];
+          load_x32<DT>(row < 32 ? stV : stK, row & 31, q4, x);
+          range32(x, (row < 32 ? MV : MK) + (size_t)j * kD + 32 * q4, mx, mn);
+        }
 #pragma unroll
-      for (int t = 0; t < kG; t += 2) {
-        const float a = col[t * kRkLd], b2 = col[(t + 1) * kRkLd];
-        mx = max3(mx, a, b2);
-        mn = min3(mn, a, b2);
+        for (int o = 1; o <= 2; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+          mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+        }
+        if (on && q4 == 0) atomicMin(&best[row], dkey(__fsub_rn(mx, mn), j));
+      };
+      {
+        const float U = rowu[32 + lane];
+        const int s = rseed[32 + lane];
+        uint32_t mask = 0u;
+#pragma unroll
+        for (int jj = 0; jj < kMaxSlice; ++jj)
+          if (jj < nsl && j0w + jj != s && klb[jj] <= U) mask |= 1u << jj;
+        nE = warp_compact(mask, lane, 32 + lane, j0w, wle, nE, kWECap, &ovf[32 + lane], &ctr[1]);
+        __syncwarp();
+        for (int b0 = 0; b0 < nE; b0 += 8) {
+          const int e = b0 + (lane >> 2);
+          const uint32_t ent = e < nE ? wle[e] : 0u;
+          exact(e < nE, (int)(ent >> 8), (int)(ent & 255u));
+        }
       }
-      const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)maxc);
-      kzr[c] = make_float2(mn, code_rcp(s));
-      kss[c] = s;
-      reinterpret_cast<float*>(sub + g.off_ks)[ksc_pos(c)] = s;
-      reinterpret_cast<float*>(sub + g.off_kz)[ksc_pos(c)] = mn;
-      if (tiny_scale(s)) ctr[0] = 1;
-    }
-    __syncthreads();
+      gsync();
+      if (ctr[1]) {
+        // some row's candidates did not all fit a list: that row against every pattern (warp 0)
+        if (gw == 0)
+          for (int row = 0; row < 64; ++row) {
+            if (!ovf[row]) continue;
+            for (int jb = 0; jb < Pe; jb += 8) exact(jb + (lane >> 2) < Pe, row, jb + (lane >> 2));
+          }
+        gsync();
+      }
 
-    // ---- H: K codes (a thread a row and 16 channels: 4 x 4 channels, 32 apart)
-    {
-      const int r = tid >> 3, cb = tid & 7;
-      float x[16], zs[16], rs[16];
+      // ---- F: V rows quantized (a unit: row and 32-channel group); K residuals staged
+      for (int u = gtid; u < 256; u += GT) {
+        if (u < 128) {
+          const int r = u >> 2, q = u & 3;
+          const unsigned long long bk = best[r];
+          const int j = (int)(bk & 0xffffffffu);
+          const bool keep = v_keep_pattern(g.vrho, __uint_as_float((uint32_t)(bk >> 32)), rraw[r]);
+          float x[32];
+          load_x32<DT>(stV, r, q, x);
+          const float* mrow = MV + (size_t)j * kD + 32 * q;
+          if (keep) {
+            const float4* m4 = reinterpret_cast<const float4*>(mrow);
+            float4 mv[8];
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int c = 4 * cb + 32 * k4;
-        const float4 a = *reinterpret_cast<const float4*>(Rk + rk_at(r, c));
-        x[4 * k4] = a.x; x[4 * k4 + 1] = a.y; x[4 * k4 + 2] = a.z; x[4 * k4 + 3] = a.w;
-        const float4 p0 = *reinterpret_cast<const float4*>(kzr + c);
-        const float4 p1 = *reinterpret_cast<const float4*>(kzr + c + 2);
-        zs[4 * k4] = p0.x; rs[4 * k4] = p0.y; zs[4 * k4 + 1] = p0.z; rs[4 * k4 + 1] = p0.w;
-        zs[4 * k4 + 2] = p1.x; rs[4 * k4 + 2] = p1.y; zs[4 * k4 + 3] = p1.z; rs[4 * k4 + 3] = p1.w;
-      }
-      uint32_t pc[8];
-      const bool clean = codes_fma<16>(x, pc, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
-        z0 = zs[2 * i2]; z1 = zs[2 * i2 + 1];
-        r0 = rs[2 * i2]; r1 = rs[2 * i2 + 1];
-      });
-      if (clean && ctr[0] == 0) {
+            for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4)
-          *reinterpret_cast<uint2*>(stK + elem_off(r, 4 * cb + 32 * k4)) = make_uint2(pc[2 * k4], pc[2 * k4 + 1]);
-      } else {
-        k_codes_exact(stK, Rk, kzr, kss, r, cb, maxc);
-      }
-    }
-    __syncthreads();
-
-    // ---- I: code words in the page's fragment order (warps 0-3 V, 4-7 K; a 16-byte chunk of
-    // four words per lane and warp)
-    {
-      const bool isV = warp < 4;
-      const int wq = warp & 3;  // chunk index: words 4 wq .. 4 wq + 3 of every lane
-      if (wq < (g.bits == 2 ? 2 : 4)) {
-        uint32_t* blk = reinterpret_cast<uint32_t*>(sub + (isV ? g.off_vc : 0));
-        const int mi = lane >> 3, ri8 = lane & 7;
-        uint32_t wd[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int w = 4 * wq + u;
-          // the (up to) two 16 x 16 tiles of word w and their slot offsets
-#pragma unroll
-          for (int tt = 0; tt < 2; ++tt) {
-            if (g.bits == 4 && tt == 1) continue;
-            const int tile = g.bits == 2 ? 2 * w + tt : w;
-            int rt, ct;  // row tile (16 rows of the code matrix) and column tile
-            if (isV) { rt = tile >> 1; ct = tile & 1; }   // V: rows = channels, 2 column tiles of tokens
-            else { rt = tile >> 3; ct = tile & 7; }       // K: rows = tokens, 8 column tiles of channels
-            uint32_t a0, a1, a2, a3;
-            if (isV) {
-              // stored [token][channel]: the transposed load gives rows = channels, columns = tokens
-              const int tok = 16 * ct + 8 * (mi >> 1) + ri8, ch = 16 * rt + 8 * (mi & 1);
-              ldsm4t(s32(stV) + elem_off(tok, ch), a0, a1, a2, a3);
-            } else {
-              const int tok = 16 * rt + 8 * (mi & 1) + ri8, ch = 16 * ct + 8 * (mi >> 1);
-              ldsm4(s32(stK) + elem_off(tok, ch), a0, a1, a2, a3);
+            for (int c = 0; c < 8; ++c) {
+              sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, x[4 * c], x[4 * c + 1]);
+              sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, x[4 * c + 2], x[4 * c + 3]);
             }
-            const uint32_t av[4] = {a0, a1, a2, a3};
+          }
+          float gmx = -INFINITY, gmn = INFINITY;
 #pragma unroll
-            for (int rg = 0; rg < 4; ++rg) {
-              if (g.bits == 2) {
-                const int s = 4 * tt + rg;  // 2-bit slot: codes at bits 2s and 16 + 2s
-                const uint32_t v = av[rg] & 0x03000300u;
-                wd[u] |= s < 4 ? v >> (8 - 2 * s) : v << (2 * s - 8);
+          for (int c = 0; c < 32; c += 2) {
+            gmx = max3(gmx, x[c], x[c + 1]);
+            gmn = min3(gmn, x[c], x[c + 1]);
+          }
+          const float s = __fdiv_rn(__fsub_rn(gmx, gmn), (float)maxc);
+          const float ri = code_rcp(s);
+          reinterpret_cast<float*>(sub + g.off_vs)[vsc_pos(r, q)] = s;
+          reinterpret_cast<float*>(sub + g.off_vz)[vzc_pos(r, q)] = gmn;
+          if (q == 0) sub[g.off_vidx + tok_pos(r)] = keep ? (uint8_t)j : (uint8_t)kRawIndex;
+          uint32_t pc[16];
+          const bool clean = codes_fma<32>(x, pc, [&](int, float& z0, float& z1, float& r0, float& r1) {
+            z0 = z1 = gmn;
+            r0 = r1 = ri;
+          });
+          if (clean && !tiny_scale(s)) {
+            uint8_t* hb = stV + (q >> 1) * 4096;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              *reinterpret_cast<uint4*>(hb + swz(r, 4 * (q & 1) + cc)) =
+                  make_uint4(pc[4 * cc], pc[4 * cc + 1], pc[4 * cc + 2], pc[4 * cc + 3]);
+          } else {
+            v_codes_exact<DT>(stV, r, q, keep ? mrow : nullptr, gmn, s, maxc);
+          }
+        } else {
+          const int r = (u - 128) >> 2, q = u & 3;
+          const int j = (int)(best[32 + r] & 0xffffffffu);
+          float x[32];
+          load_x32<DT>(stK, r, q, x);
+          const float4* m4 = reinterpret_cast<const float4*>(MK + (size_t)j * kD + 32 * q);
+          float4 mv[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mv[c] = __ldg(m4 + c);
+          float4* dst = reinterpret_cast<float4*>(Rk + rk_at(r, 32 * q));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float4 o;
+            sub2(x[4 * c], x[4 * c + 1], mv[c].x, mv[c].y, o.x, o.y);
+            sub2(x[4 * c + 2], x[4 * c + 3], mv[c].z, mv[c].w, o.z, o.w);
+            dst[c] = o;
+          }
+          if (q == 0) sub[g.off_kidx + tok_pos(r)] = (uint8_t)j;
+        }
+      }
+      gsync();
+
+      // ---- G: K scale and zero per channel over the page (a thread a channel)
+      for (int c = gtid; c < kD; c += GT) {
+        const float* col = Rk + rk_at(0, c);
+        float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+        for (int t = 0; t < kG; t += 2) {
+          const float a = col[t * kRkLd], b2 = col[(t + 1) * kRkLd];
+          mx = max3(mx, a, b2);
+          mn = min3(mn, a, b2);
+        }
+        const float s = __fdiv_rn(__fsub_rn(mx, mn), (float)maxc);
+        kzr[c] = make_float2(mn, code_rcp(s));
+        kss[c] = s;
+        reinterpret_cast<float*>(sub + g.off_ks)[ksc_pos(c)] = s;
+        reinterpret_cast<float*>(sub + g.off_kz)[ksc_pos(c)] = mn;
+        if (tiny_scale(s)) ctr[0] = 1;
+      }
+      gsync();
+
+      // ---- H: K codes (a unit: row and 16 channels, 4 x 4 channels 32 apart)
+      for (int u = gtid; u < 256; u += GT) {
+        const int r = u >> 3, cb = u & 7;
+        float x[16], zs[16], rs[16];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int c = 4 * cb + 32 * k4;
+          const float4 a = *reinterpret_cast<const float4*>(Rk + rk_at(r, c));
+          x[4 * k4] = a.x; x[4 * k4 + 1] = a.y; x[4 * k4 + 2] = a.z; x[4 * k4 + 3] = a.w;
+          const float4 p0 = *reinterpret_cast<const float4*>(kzr + c);
+          const float4 p1 = *reinterpret_cast<const float4*>(kzr + c + 2);
+          zs[4 * k4] = p0.x; rs[4 * k4] = p0.y; zs[4 * k4 + 1] = p0.z; rs[4 * k4 + 1] = p0.w;
+          zs[4 * k4 + 2] = p1.x; rs[4 * k4 + 2] = p1.y; zs[4 * k4 + 3] = p1.z; rs[4 * k4 + 3] = p1.w;
+        }
+        uint32_t pc[8];
+        const bool clean = codes_fma<16>(x, pc, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
+          z0 = zs[2 * i2]; z1 = zs[2 * i2 + 1];
+          r0 = rs[2 * i2]; r1 = rs[2 * i2 + 1];
+        });
+        if (clean && ctr[0] == 0) {
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            *reinterpret_cast<uint2*>(stK + elem_off(r, 4 * cb + 32 * k4)) = make_uint2(pc[2 * k4], pc[2 * k4 + 1]);
+        } else {
+          k_codes_exact(stK, Rk, kzr, kss, r, cb, maxc);
+        }
+      }
+      gsync();
+
+      // ---- I: code words in the page's fragment order: 16-byte chunks of four words per lane,
+      // the V block's chunks then the K block's, spread over the group's warps
+      {
+        const int nc = g.bits == 2 ? 2 : 4;  // chunks per block
+        const int mi = lane >> 3, ri8 = lane & 7;
+        for (int ch = gw; ch < 2 * nc; ch += GW) {
+          const bool isV = ch < nc;
+          const int wq = isV ? ch : ch - nc;  // chunk: words 4 wq .. 4 wq + 3 of every lane
+          uint32_t* blk = reinterpret_cast<uint32_t*>(sub + (isV ? g.off_vc : 0));
+          uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int w = 4 * wq + u;
+            // the (up to) two 16 x 16 tiles of word w and their slot offsets
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+              if (g.bits == 4 && tt == 1) continue;
+              const int tile = g.bits == 2 ? 2 * w + tt : w;
+              int rt, ct;  // row tile (16 rows of the code matrix) and column tile
+              if (isV) { rt = tile >> 1; ct = tile & 1; }   // V: rows = channels, 2 column tiles of tokens
+              else { rt = tile >> 3; ct = tile & 7; }       // K: rows = tokens, 8 column tiles of channels
+              uint32_t a0, a1, a2, a3;
+              if (isV) {
+                // stored [token][channel]: the transposed load gives rows = channels, columns = tokens
+                const int tok = 16 * ct + 8 * (mi >> 1) + ri8, chn = 16 * rt + 8 * (mi & 1);
+                ldsm4t(s32(stV) + elem_off(tok, chn), a0, a1, a2, a3);
               } else {
-                const int s = rg;  // 4-bit slot: codes at bits 4s and 16 + 4s
-                const uint32_t v = av[rg] & 0x0F000F00u;
-                wd[u] |= s < 2 ? v >> (8 - 4 * s) : v << (4 * s - 8);
+                const int tok = 16 * rt + 8 * (mi & 1) + ri8, chn = 16 * ct + 8 * (mi >> 1);
+                ldsm4(s32(stK) + elem_off(tok, chn), a0, a1, a2, a3);
+              }
+              const uint32_t av[4] = {a0, a1, a2, a3};
+#pragma unroll
+              for (int rg = 0; rg < 4; ++rg) {
+                if (g.bits == 2) {
+                  const int sl = 4 * tt + rg;  // 2-bit slot: codes at bits 2 sl and 16 + 2 sl
+                  const uint32_t v = av[rg] & 0x03000300u;
+                  wd[u] |= sl < 4 ? v >> (8 - 2 * sl) : v << (2 * sl - 8);
+                } else {
+                  const int sl = rg;  // 4-bit slot: codes at bits 4 sl and 16 + 4 sl
+                  const uint32_t v = av[rg] & 0x0F000F00u;
+                  wd[u] |= sl < 2 ? v >> (8 - 4 * sl) : v << (4 * sl - 8);
+                }
               }
             }
           }
+          *reinterpret_cast<uint4*>(blk + wq * 128 + lane * 4) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
-        *reinterpret_cast<uint4*>(blk + wq * 128 + lane * 4) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      }
+
+      // ---- end of the task: this stage refills with the group's task NS ahead (the generic
+      // accesses of this task to the stage ordered before the tensor copy that overwrites it)
+      int64_t after = s1;
+      if (ca < s1 && (NS == 1 || nxt < s1)) after = task_check(g, kca, gtid == 0) ? ca : next_valid(ca + NG, s1, kca);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      gsync();
+      ++q_;
+      if (gtid == 0 && after < s1) issue(kca, (q_ + NS - 1) % NS);
+      if (NS == 2) {
+        cur = nxt;
+        kc = kn;
+        nxt = after;
+        kn = kca;
+      } else {
+        cur = after;
+        kc = kca;
       }
     }
-
-    // ---- end of the task: the next task's stage awaited (its copy was issued two tasks ago),
-    // then this stage refilled with the task after next (the generic accesses of this task to
-    // the stage ordered before the tensor copy that overwrites it)
-    int64_t after = t1;
-    if (nxt < t1 && ca < t1) after = task_check(g, kca, tid == 0) ? ca : next_valid(ca + 1, kca);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (nxt < t1 && !__all_sync(kFull, fb_wait(&full[buf ^ 1], (uint32_t)(((i + 1) >> 1) & 1)))) {
-      if (lane == 0) set_status(g.status, KVQ_DEV_TIMEOUT);
-      timed_out = true;
-    }
-    if (__syncthreads_or(timed_out)) break;
-    if (tid == 0 && after < t1) issue(kca, buf);
-    cur = nxt;
-    kc = kn;
-    nxt = after;
-    kn = kca;
+    s0 = s1;
   }
-  // drain (after a timeout): the newest copy issued into each stage must land before the CTA
-  // exits; phases complete in order, so that covers the older ones
-  if (tid == 0 && timed_out) {
-    for (int b2 = 0; b2 < 2; ++b2)
-      if (n_issued[b2] > 0 && !fb_wait(&full[b2], (n_issued[b2] - 1u) & 1u)) set_status(g.status, KVQ_DEV_TIMEOUT);
+  // drain: every copy this group issued lands before the CTA exits (phases complete in order,
+  // so the newest of each stage covers the older ones; only a group whose wait expired has
+  // copies that were never awaited)
+  if (gtid == 0 && dead) {
+    for (int b2 = 0; b2 < NS; ++b2)
+      if (n_issued[b2] > waits[b2] && !fb_wait(&full[b2], (n_issued[b2] - 1u) & 1u)) set_status(g.status, KVQ_DEV_TIMEOUT);
   }
 }
 
@@ -963,32 +1046,43 @@ bool append_full_eligible(const Geom& g, int n_new) {
   return !g.tx && g.P <= 128 && n_new >= kG && g.B > 0 && (g.dtype == KVQ_BF16 || g.dtype == KVQ_F16);
 }
 
-cudaError_t launch_append_full(const Geom& g, const void* k_new, const void* v_new, int n_new, const void* probe,
-                               const void* pv, cudaStream_t st) {
-  const int F = n_new / kG + 1;  // most pages a sequence can fill completely in this call
+namespace {
+template <int NG, int GW>
+cudaError_t launch_full_cfg(const Geom& g, const CUtensorMap& kmap, const CUtensorMap& vmap, int n_new, int F,
+                            const void* probe, const void* pv, cudaStream_t st) {
   const int64_t T = (int64_t)g.H * g.B * F;
-  const FullSmem sp = full_smem(g.P);
+  const int smem = full_smem_bytes<NG, GW>(g.P);
   int dev = 0, sms = 148, occ = 1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  auto kern = g.dtype == KVQ_BF16 ? append_full_kernel<KVQ_BF16> : append_full_kernel<KVQ_F16>;
-  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sp.total)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kFThreads, sp.total)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  auto kern = g.dtype == KVQ_BF16 ? append_full_kernel<KVQ_BF16, NG, GW> : append_full_kernel<KVQ_F16, NG, GW>;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NG * GW * 32, smem)) != cudaSuccess) return e;
   const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(T, (int64_t)std::max(occ, 1) * sms));
   const int64_t per = (T + ctas - 1) / ctas;
+  kern<<<(unsigned)((T + per - 1) / per), NG * GW * 32, smem, st>>>(kmap, vmap, g, (const int32_t*)probe,
+                                                                  (const float*)pv, n_new, F, per);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_append_full(const Geom& g, const void* k_new, const void* v_new, int n_new, const void* probe,
+                               const void* pv, cudaStream_t st) {
+  const int F = n_new / kG + 1;  // most pages a sequence can fill completely in this call
   // K / V input as (128 channels, KV heads, tokens of all sequences), boxes of 64 channels x 32 tokens
   CUtensorMap kmap, vmap;
   const CUtensorMapDataType dt = g.dtype == KVQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)g.H, (cuuint64_t)g.B * n_new};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)g.H * kD * 2};
   const cuuint32_t box[3] = {64, 1, 32};
+  cudaError_t e;
   if ((e = encode_tiled_map(&kmap, dt, 3, k_new, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
       (e = encode_tiled_map(&vmap, dt, 3, v_new, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
     return e;
-  kern<<<(unsigned)((T + per - 1) / per), kFThreads, sp.total, st>>>(kmap, vmap, g, (const int32_t*)probe,
-                                                                     (const float*)pv, n_new, F, per);
-  return cudaGetLastError();
+  // up to 64 patterns: two groups of 4 warps per CTA (a group a task); more: one group of 8
+  if (g.P <= 4 * kMaxSlice) return launch_full_cfg<2, 4>(g, kmap, vmap, n_new, F, probe, pv, st);
+  return launch_full_cfg<1, 8>(g, kmap, vmap, n_new, F, probe, pv, st);
 }
 
 }  // namespace kvq
