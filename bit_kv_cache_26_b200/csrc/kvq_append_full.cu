@@ -61,6 +61,7 @@ constexpr int kPhiLd = 136;    // 16-bit row stride of the pattern table for ldm
 constexpr int kRkLd = 144;     // fp32 row stride of the staged K residuals (16 mod 32 words)
 constexpr int kStageBytes = 16384;  // V rows (2 x 4 KB halves) then K rows (2 x 4 KB halves)
 constexpr int kMaxSlice = 16;       // patterns per warp in the bound passes (up to 128 patterns)
+constexpr int kFullGroups = 2;      // 4-warp task groups per CTA (two CTAs per SM) for up to 64 patterns
 constexpr int kW2Cap = 256;         // entries of a warp's refinement list
 constexpr int kWECap = 128;         // entries of a warp's exact list
 constexpr uint32_t kFSpin = 1u << 22;
@@ -441,7 +442,7 @@ __device__ __forceinline__ int task_key(const Geom& g, int F, int64_t t, SeqCach
 // interleave on the SM; a group's stage refills with its next task when the current one is done
 // (two stages, the copy two tasks ahead, when NG = 1).
 template <int DT, int NG, int GW>
-__global__ void __launch_bounds__(NG * GW * 32, 2) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(NG * GW * 32, NG <= 2 ? 2 : 1) append_full_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                       const __grid_constant__ CUtensorMap vmap,
                                                                       Geom g, const int32_t* __restrict__ probe,
                                                                       const float* __restrict__ pvals, int n_new,
@@ -478,25 +479,31 @@ __global__ void __launch_bounds__(NG * GW * 32, 2) append_full_kernel(const __gr
   float* kss = reinterpret_cast<float*>(gb + C::kKs);         // per K channel: s
   uint64_t* full = reinterpret_cast<uint64_t*>(gb + C::kBars);
   const int maxc = (1 << g.bits) - 1;
-  // group barriers: named barrier 1 (group 0) or 2 (group 1), the group's threads
+  // group barriers: named barrier gi + 1 over the group's threads (literal ids, so that the
+  // kernel reserves only the barriers it uses)
   auto gsync = [&]() {
-    if (gi == 0) asm volatile("bar.sync 1, %0;" ::"n"(GT) : "memory");
-    else asm volatile("bar.sync 2, %0;" ::"n"(GT) : "memory");
+    switch (gi) {
+      case 0: asm volatile("bar.sync 1, %0;" ::"n"(GT) : "memory"); break;
+      case 1: asm volatile("bar.sync 2, %0;" ::"n"(GT) : "memory"); break;
+      case 2: asm volatile("bar.sync 3, %0;" ::"n"(GT) : "memory"); break;
+      default: asm volatile("bar.sync 4, %0;" ::"n"(GT) : "memory"); break;
+    }
   };
   auto gsync_or = [&](bool v) -> bool {
     uint32_t r;
-    if (gi == 0)
-      asm volatile(
-          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-          : "=r"(r)
-          : "r"((uint32_t)v), "n"(GT)
-          : "memory");
-    else
-      asm volatile(
-          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-          : "=r"(r)
-          : "r"((uint32_t)v), "n"(GT)
-          : "memory");
+#define KVQ_BAR_OR(ID)                                                                                   \
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, " #ID                   \
+               ", %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"                                                      \
+               : "=r"(r)                                                                                 \
+               : "r"((uint32_t)v), "n"(GT)                                                                \
+               : "memory")
+    switch (gi) {
+      case 0: KVQ_BAR_OR(1); break;
+      case 1: KVQ_BAR_OR(2); break;
+      case 2: KVQ_BAR_OR(3); break;
+      default: KVQ_BAR_OR(4); break;
+    }
+#undef KVQ_BAR_OR
     return r != 0u;
   };
 
@@ -1080,8 +1087,9 @@ cudaError_t launch_append_full(const Geom& g, const void* k_new, const void* v_n
   if ((e = encode_tiled_map(&kmap, dt, 3, k_new, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
       (e = encode_tiled_map(&vmap, dt, 3, v_new, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
     return e;
-  // up to 64 patterns: two groups of 4 warps per CTA (a group a task); more: one group of 8
-  if (g.P <= 4 * kMaxSlice) return launch_full_cfg<2, 4>(g, kmap, vmap, n_new, F, probe, pv, st);
+  // up to 64 patterns: groups of 4 warps (a group a task), all of a CTA on one (set, head); more:
+  // one group of 8
+  if (g.P <= 4 * kMaxSlice) return launch_full_cfg<kFullGroups, 4>(g, kmap, vmap, n_new, F, probe, pv, st);
   return launch_full_cfg<1, 8>(g, kmap, vmap, n_new, F, probe, pv, st);
 }
 
