@@ -249,13 +249,13 @@ PER_CONFIG = [("llama3_8b_32k", {"bits": 2}), ("llama3_8b_32k", {"bits": 4}),
               ("qwen25_7b_128k", {}), ("qwen25_7b_128k", {"transform": 1})]
 
 
-def launches_per_step(w, full_pages: bool) -> int:
+def launches_per_step(w) -> int:
     """Kernels this library launches per step: per mining call init + per Lloyd iteration
     assignment (+ the float64 fix-up after the tcgen05 assignment), cluster sums and update (+16
-    for the pre-transform fit and apply); append: prep, full pages, partial pages, tail; decode: 1."""
+    for the pre-transform fit and apply); append: prep, pages, tail; decode: 1."""
     tc = w.dtype == 1 and not w.transform and w.P <= 128
     mine = 1 + (4 if tc else 3) * w.iters + (16 if w.transform else 0)
-    return 2 * mine + (4 if full_pages else 3) + 1
+    return 2 * mine + 3 + 1
 
 
 def measure_path(w, args, dev, world: int, rank: int, headline: bool, shard=None):
@@ -402,15 +402,10 @@ def measure_path(w, args, dev, world: int, rank: int, headline: bool, shard=None
            "decode_kv_tokens_per_s": tokens / (decode_ms * 1e-3), "decode_hbm_gbs": rooflines["decode_attention"]["achieved"],
            "quant_append_gbs": rooflines["quantize_append"]["achieved"], "v_pattern_utilisation": utilisation,
            "roofline": roofline, "rooflines": rooflines,
-           "gpu_launches": args.steps * launches_per_step(w, kvq_full_pages(w))}
+           "gpu_launches": args.steps * launches_per_step(w)}
     del kd, vd, qd, kh, vh, qh, cache, ws_m, ws_d, ws_a
     torch.cuda.empty_cache()
     return rec, e2e, clk
-
-
-def kvq_full_pages(w) -> bool:
-    """Whether the full-page append kernel serves this workload (16-bit input, no pre-transform, P <= 128)."""
-    return not w.transform and w.P <= 128
 
 
 def measure_decode_loop(w, args, dev, nsteps: int = 512, chunk: int = 64):

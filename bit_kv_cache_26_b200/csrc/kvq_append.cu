@@ -98,10 +98,9 @@ struct PageCtx {
   const float* cV;
 };
 
-// Returns false if the CTA has nothing to do (or an error was flagged).  With `partial_only`
-// (the full-page kernel takes every page the call fills completely) CTA x = 0 takes the first
-// page the call touches and x = 1 the last, each only if the call does not fill it completely.
-__device__ bool page_context(const Geom& g, int n_new, bool partial_only, PageCtx& c) {
+// Returns false if the CTA has nothing to do (or an error was flagged).  CTA x takes the x-th
+// page the call touches.
+__device__ bool page_context(const Geom& g, int n_new, PageCtx& c) {
   const int b = blockIdx.z, h = blockIdx.y;
   c.L = g.seq_len[b];
   c.n = n_new;
@@ -109,17 +108,10 @@ __device__ bool page_context(const Geom& g, int n_new, bool partial_only, PageCt
     if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) set_status(g.status, KVQ_DEV_OVERFLOW);
     return false;
   }
-  if (partial_only) {
-    const int first = c.L / kG, last = (c.L + n_new - 1) / kG;
-    if (blockIdx.x == 1 && last == first) return false;
-    c.pg = blockIdx.x == 0 ? first : last;
-  } else {
-    c.pg = c.L / kG + blockIdx.x;
-  }
+  c.pg = c.L / kG + blockIdx.x;
   c.a = max(c.L, c.pg * kG);
   c.e = min(c.L + n_new, c.pg * kG + kG);
   if (c.a >= c.e) return false;
-  if (partial_only && c.a == c.pg * kG && c.e == c.pg * kG + kG) return false;  // a full page
   const int phys = g.page_table[(size_t)b * g.maxp + c.pg];
   if (phys < 0 || phys >= g.npages) {
     if (threadIdx.x == 0) set_status(g.status, KVQ_DEV_BAD_PAGE);
@@ -310,9 +302,9 @@ __device__ __forceinline__ void group_sz(float mn, float mx, int bits, float& s,
 __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g, AppendWs wsp,
                                                                          const uint16_t* __restrict__ k_new,
                                                                          const uint16_t* __restrict__ v_new,
-                                                                         int n_new, bool partial_only) {
+                                                                         int n_new) {
   PageCtx c;
-  if (!page_context(g, n_new, partial_only, c)) return;
+  if (!page_context(g, n_new, c)) return;
   const int b = blockIdx.z, h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int P = g.P;                          // capacity: the layout of the tables
@@ -664,13 +656,10 @@ cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, i
   if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
       cudaSuccess)
     return e;
-  // pages the call fills completely: the full-page kernel; the rest (at most the first and the
-  // last touched page of each sequence): the general kernel
-  const bool full = append_full_eligible(g, n_new);
-  if (full && (e = launch_append_full(g, k_new, v_new, n_new, w.probe, w.pv, st)) != cudaSuccess) return e;
-  dim3 grid(full ? 2 : n_new / kG + 2, g.H, g.B);
-  append_pages_kernel<<<grid, kAppendThreads, dyn, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new, n_new,
-                                                         full);
+  // one CTA per (page the call touches, KV head, sequence)
+  dim3 grid(n_new / kG + 2, g.H, g.B);
+  append_pages_kernel<<<grid, kAppendThreads, dyn, st>>>(g, w, (const uint16_t*)k_new, (const uint16_t*)v_new,
+                                                         n_new);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   append_tail_kernel<<<g.B, 256, 0, st>>>(g, (const uint16_t*)k_new, n_new);

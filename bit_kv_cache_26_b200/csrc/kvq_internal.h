@@ -56,12 +56,6 @@ cudaError_t encode_tiled_map(CUtensorMap* map, CUtensorMapDataType dt, int rank,
                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                              CUtensorMapSwizzle swz);
 
-// Full-page quantize-append (kvq_append_full.cu): every page whose 32 tokens all arrive in this
-// call, for 16-bit inputs without the pre-transform and P <= 128.  Returns false (launching
-// nothing) when the cache or call is outside that scope.
-bool append_full_eligible(const Geom& g, int n_new);
-cudaError_t launch_append_full(const Geom& g, const void* k_new, const void* v_new, int n_new, const void* probe,
-                               const void* pv, cudaStream_t st);
 cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 
 }  // namespace kvq
