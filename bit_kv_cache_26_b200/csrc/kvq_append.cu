@@ -235,35 +235,134 @@ __device__ __forceinline__ uint32_t v_word(int wd, const float (*Rv)[kLd], const
   return word;
 }
 
-// One 32-bit code word of the K block (rows = tokens, 8 column tiles of 16 channels) from
-// the staged residuals Rk[token][channel] and per-channel s / z / 1/s.
-template <int BITS>
-__device__ __forceinline__ uint32_t k_word(int wd, const float (*Rk)[kLd], const float* ks, const float* kz,
-                                           const float* kr) {
-  constexpr int SPW = 16 / BITS;
-  const int ln = (wd & 127) >> 2, gq = ln >> 2, tig = ln & 3;
-  const int w = (wd >> 7) * 4 + (wd & 3);
-  uint32_t word = 0;
+// Halves per row of the fp16 lower-bound table [64 rows][.]: an odd number of 32-bit words, so
+// that 32 consecutive rows (the bound pass, a lane a row) and 16 rows x 2 pattern halves (the
+// candidate scan) fall in different banks.
+__host__ __device__ inline int lb_ld(int P) { return 2 * (((P + 1) >> 1) | 1); }
+
+// ---- codes of whole pages: one FMA per code, 16-bit codes staged row-major, words by ldmatrix
+// A code is rne(fl32(fl32(R - z) / s)).  v = t (1/s) + (1.5 * 2^7 + 1/2) with t = R - z in
+// [0, maxc s] stays in [128, 256): its bits 16-22 hold 64 + the code and bits 0-15 the fraction.
+// v differs from the exact t / s + 1/2 by less than 2^-17 (its own rounding) + 15 * 2^-24 (the
+// reciprocal's), under one fraction step; so the code can be wrong, or the quotient a tie that
+// rounds to even, only when the fraction is 0x0000 or 0xFFFF (about 2 codes in 65536).  Those
+// units, and every unit with a scale below 2^-125 (whose reciprocal is not within 2^-24 of
+// 1 / s, or overflows), are recomputed with the correctly rounded division.
+constexpr float kCodeMagic = 192.5f;    // 1.5 * 2^7 + 1/2: 16 fraction bits, +1/2 folded in
+constexpr float kMinScale = 0x1p-125f;  // below this (and nonzero) 1 / s is not within 2^-24 of exact
+
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ bool tiny_scale(float s) { return s != 0.0f && s < kMinScale; }
+// Codes of N residuals as N / 2 words of two 16-bit halves (the code in bits 8-11 of each half:
+// byte 2 of the FMA result, 0x40 | code); zr(i, z0, z1, r0, r1) gives the zeros and reciprocal
+// scales of values 2i, 2i + 1.  Returns true if no fraction is 0x0000 or 0xFFFF.
+template <int N, class ZR>
+__device__ __forceinline__ bool codes_fma(const float (&x)[N], uint32_t (&p)[N / 2], ZR zr) {
+  uint32_t acc = 0xFFFFFFFFu;  // per half: min over the pairs of (fraction + 1) mod 2^16
 #pragma unroll
-  for (int slot = 0; slot < SPW; ++slot) {
-    const int tile = (SPW * w + slot) >> 2, r = slot & 3;
-    const int tok = 16 * (tile >> 3) + 8 * (r & 1) + gq;
-    const int ch = 16 * (tile & 7) + 8 * (r >> 1) + 2 * tig;
-    const float2 R = *reinterpret_cast<const float2*>(&Rk[tok][ch]);
-    const float2 z = *reinterpret_cast<const float2*>(kz + ch);
-    const float2 ri = *reinterpret_cast<const float2*>(kr + ch);
-    word |= code_pair<BITS>(R.x, R.y, z.x, z.y, ri.x, ri.y, ks + ch) << (BITS * slot);
+  for (int i = 0; i < N / 2; ++i) {
+    float z0, z1, r0, r1, t0, t1, v0, v1;
+    zr(i, z0, z1, r0, r1);
+    sub2(x[2 * i], x[2 * i + 1], z0, z1, t0, t1);
+    fma2f(t0, t1, r0, r1, kCodeMagic, kCodeMagic, v0, v1);
+    const uint32_t u0 = __float_as_uint(v0), u1 = __float_as_uint(v1);
+    p[i] = __byte_perm(u0, u1, 0x6420);
+    // a carry out of the low half only happens when that half is flagged anyway
+    acc = vmin_u16x2(acc, __byte_perm(u0, u1, 0x5410) + 0x00010001u);
   }
-  return word;
+  return (acc & 0x0000FFFEu) != 0u && (acc & 0xFFFE0000u) != 0u;
+}
+// Byte offset of channel ch (0..127) of row `row` in a 16-bit code buffer of two 64-channel
+// halves of 32 rows x 128 B, 16-byte chunks XOR-swizzled by (row & 7) (conflict-free ldmatrix).
+__device__ __forceinline__ uint32_t cb_off(int row, int ch) {
+  return (uint32_t)((ch >> 6) * 4096 + row * 128 + ((((ch & 63) >> 3) ^ (row & 7)) << 4) + (ch & 7) * 2);
+}
+// The rare paths (a fraction of 0x0000 / 0xFFFF somewhere, or a scale below 2^-125): the
+// unit's codes by the definition (the correctly rounded quotient, round half to even, clamp),
+// written as 16-bit codes; out of line, reading the residuals from shared memory.
+// V: the 32 residuals y of row `row`, channels c0 .., zero z, scale s.
+__device__ __noinline__ void v_codes_exact(const float* y, float z, float s, int maxc, uint8_t* cb, int row, int c0) {
+  for (int i = 0; i < 32; ++i) {
+    uint32_t c = 0u;
+    if (s != 0.0f) c = (uint32_t)min(max(__float2int_rn(__fdiv_rn(__fsub_rn(y[i], z), s)), 0), maxc);
+    *reinterpret_cast<uint16_t*>(cb + cb_off(row, c0 + i)) = (uint16_t)(c << 8);
+  }
+}
+// K: channels 4 cbk + 32 k .. + 3 (k = 0..3) of residual row y, zero kz[c], scale ks[c].
+__device__ __noinline__ void k_codes_exact(const float* y, const float* kz, const float* ks, int cbk, int maxc,
+                                           uint8_t* cb, int row) {
+  for (int i = 0; i < 16; ++i) {
+    const int c = 4 * cbk + 32 * (i >> 2) + (i & 3);
+    const float s = ks[c];
+    uint32_t code = 0u;
+    if (s != 0.0f) code = (uint32_t)min(max(__float2int_rn(__fdiv_rn(__fsub_rn(y[c], kz[c]), s)), 0), maxc);
+    *reinterpret_cast<uint16_t*>(cb + cb_off(row, c)) = (uint16_t)(code << 8);
+  }
+}
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// Words 4 wq .. 4 wq + 3 of every lane of a page's code block from a 16-bit code buffer
+// ([32 tokens][128 channels], cb_off layout): the MMA fragment order of include/kvq.h, the
+// V block (isV) with rows = channels (a transposed ldmatrix), the K block with rows = tokens.
+__device__ __forceinline__ uint4 pack_chunk(const uint8_t* cb, bool isV, int bits, int wq, int lane) {
+  const int mi = lane >> 3, ri8 = lane & 7;
+  uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int w = 4 * wq + u;
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      if (bits == 4 && tt == 1) continue;
+      const int tile = bits == 2 ? 2 * w + tt : w;
+      int rt, ct;  // row tile (16 rows of the code matrix) and column tile
+      if (isV) { rt = tile >> 1; ct = tile & 1; }  // V: rows = channels, 2 column tiles of tokens
+      else { rt = tile >> 3; ct = tile & 7; }      // K: rows = tokens, 8 column tiles of channels
+      uint32_t a0, a1, a2, a3;
+      if (isV) {
+        const int tok = 16 * ct + 8 * (mi >> 1) + ri8, ch = 16 * rt + 8 * (mi & 1);
+        ldsm4t(su32(cb) + cb_off(tok, ch), a0, a1, a2, a3);
+      } else {
+        const int tok = 16 * rt + 8 * (mi & 1) + ri8, ch = 16 * ct + 8 * (mi >> 1);
+        ldsm4(su32(cb) + cb_off(tok, ch), a0, a1, a2, a3);
+      }
+      const uint32_t av[4] = {a0, a1, a2, a3};
+#pragma unroll
+      for (int rg = 0; rg < 4; ++rg) {
+        if (bits == 2) {
+          const int sl = 4 * tt + rg;  // 2-bit slot: codes at bits 2 sl and 16 + 2 sl
+          const uint32_t v = av[rg] & 0x03000300u;
+          wd[u] |= sl < 4 ? v >> (8 - 2 * sl) : v << (2 * sl - 8);
+        } else {
+          const int sl = rg;  // 4-bit slot: codes at bits 4 sl and 16 + 4 sl
+          const uint32_t v = av[rg] & 0x0F000F00u;
+          wd[u] |= sl < 2 ? v >> (8 - 4 * sl) : v << (4 * sl - 8);
+        }
+      }
+    }
+  }
+  return make_uint4(wd[0], wd[1], wd[2], wd[3]);
 }
 
 // Lower bounds over the NPROBE probe channels pc (shared memory) for patterns [j0, j1) of one
 // staged vector y (one lane), from the patterns' values there (shared memory, [P][NPROBE]);
-// written to lbuf[j][row] rounded toward zero to fp16 (still a lower bound); running argmin
+// written to lbuf[row][j] rounded toward zero to fp16 (still a lower bound); running argmin
 // of the fp32 bounds (ties: lowest j) to (blb, bj).
 template <int NPROBE>
 __device__ __forceinline__ void lb_pass(const float* y, const int32_t* pc, const float* pvt, int j0, int j1,
-                                        __half* lbuf, int row, float& blb_out, int& bj_out) {
+                                        __half* lbuf, int ldh, int row, float& blb_out, int& bj_out) {
   float py[NPROBE];
 #pragma unroll
   for (int u = 0; u < NPROBE; ++u) py[u] = y[pc[u]];
@@ -285,7 +384,7 @@ __device__ __forceinline__ void lb_pass(const float* y, const int32_t* pc, const
       mn = min3(mn, r2, r3);
     }
     const float lb = __fsub_rn(mx, mn);
-    lbuf[j * (2 * kG) + row] = __float2half_rz(lb);
+    lbuf[row * ldh + j] = __float2half_rz(lb);
     if (lb < blb) { blb = lb; bj = j; }
   }
   blb_out = blb;
@@ -319,18 +418,22 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __shared__ bool vkeep[kG];      // V rows: the pattern is kept (else quantized raw, index 255)
   __shared__ int seed[2 * kG], hj[2][2 * kG];
   __shared__ int qn;
-  // dynamic: fp16 lower bounds lb[j][row], then the probe tables (V: [P][32], K: [P][16]) and
+  // dynamic: fp16 lower bounds lb[row][j], then the probe tables (V: [P][32], K: [P][16]) and
   // probe channels (32 + 16), whose region holds the work queue once the bounds are done;
-  // after the assignment the s / z / 1/s tables reuse the start of the whole region
+  // after the assignment the s / z / 1/s tables and the 16-bit code buffers reuse the region
   extern __shared__ __align__(16) float dsm[];
-  __half* lbuf = reinterpret_cast<__half*>(dsm);  // [P][64 rows]
-  float* tabV = dsm + 32 * P;
+  const int ldh = lb_ld(P);
+  __half* lbuf = reinterpret_cast<__half*>(dsm);  // [64 rows][ldh]
+  float* tabV = dsm + 32 * ldh;
   float* tabK = tabV + kProbeV * P;
   int32_t* pcV = reinterpret_cast<int32_t*>(tabK + kProbeK * P);
   int32_t* pcK = pcV + kProbeV;
   uint32_t* queue = reinterpret_cast<uint32_t*>(tabV);  // [kQueueCap]
   float* vsz = dsm;            // [3][4][kG]: s, z, 1/s per (group, V slot)
   float* ksz = dsm + 12 * kG;  // [3][kD]:   s, z, 1/s per K channel
+  uint8_t* cbV = reinterpret_cast<uint8_t*>(dsm + 1024);  // 16-bit V codes [32 tokens][128], cb_off layout
+  uint8_t* cbK = cbV + 8192;                              // 16-bit K codes
+  __shared__ int ktiny;  // some K scale of the page is below 2^-125
 
   const int lo = c.a - c.pg * kG, hi = c.e - c.pg * kG;  // new slots [lo, hi)
   const size_t shk = ((size_t)c.set * g.H + h) * 2;       // tables: K at shk, V at shk + 1
@@ -408,8 +511,10 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   {
     const int kind = warp & 1, half = warp >> 1;
     const int r = kind * kG + lane;
-    if (kind == 0) lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? Pe : P0, lbuf, r, hlb[half][r], hj[half][r]);
-    else if (c.seal) lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, r, hlb[half][r], hj[half][r]);
+    if (kind == 0)
+      lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r]);
+    else if (c.seal)
+      lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r]);
     if (kind == 0 || c.seal) {
       // the half's best pattern is the likely seed: its row into L1 ahead of the exact range
       const float* mrow = (kind ? c.MK : c.MV) + (size_t)min(max(hj[half][r], 0), Pe - 1) * kD;
@@ -420,7 +525,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __syncthreads();
 
   // ---- seed = smallest bound; its exact d_mm, two threads per row (channel halves); then the
-  // same two threads queue the patterns (one half each) whose bound does not exclude them
+  // warp's 16 rows queue the patterns whose bound does not exclude them (lane: row 16 w + (lane &
+  // 15), pattern half lane >> 4, the row's seed and distance by shuffle)
   {
     const int r = tid >> 1, hh = tid & 1;
     const bool on = row_on(r);
@@ -454,14 +560,18 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       seed[r] = s;
       best[r] = dkey(ds, s);
     }
-    if (on) {
-      const int j1 = hh ? Pe : P0;
+    const int src = 2 * (lane & 15);
+    const int r2 = 16 * warp + (lane & 15), hh2 = lane >> 4;
+    const float ds2 = __shfl_sync(kFull, ds, src);
+    const int s2 = __shfl_sync(kFull, s, src);
+    if (row_on(r2)) {
+      const int j1 = hh2 ? Pe : P0;
 #pragma unroll 4
-      for (int j = hh ? P0 : 0; j < j1; ++j) {
-        const float lb = __half2float(lbuf[j * (2 * kG) + r]);
-        if (j == s || lb > ds || (lb == ds && j > s)) continue;
+      for (int j = hh2 ? P0 : 0; j < j1; ++j) {
+        const float lb = __half2float(lbuf[r2 * ldh + j]);
+        if (j == s2 || lb > ds2 || (lb == ds2 && j > s2)) continue;
         const int pos = atomicAdd(&qn, 1);
-        if (pos < kQueueCap) queue[pos] = ((uint32_t)r << 16) | (uint32_t)j;
+        if (pos < kQueueCap) queue[pos] = ((uint32_t)r2 << 16) | (uint32_t)j;
       }
     }
   }
@@ -505,7 +615,11 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   __syncthreads();
 
   // ---- residuals in place, R = y - M[k*], one thread per (row, 32-channel group): rows
-  // lane and lane + 32 (V slot, K slot) of group `warp`; the V groups' scale / zero on the way
+  // lane and lane + 32 (V slot, K slot) of group `warp`; the V groups' scale / zero on the way,
+  // and, on a page the call writes whole, the V codes
+  const int maxc = (1 << g.bits) - 1;
+  const bool whole = c.fresh && lo == 0 && hi == kG;  // every token of the page is new
+  if (tid == 0) ktiny = 0;
   {
     const int q = warp;
 #pragma unroll
@@ -523,6 +637,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
 #pragma unroll
         for (int k = 0; k < 8; ++k) mv[k] = keep ? __ldg(m4 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
         float mx = -INFINITY, mn = INFINITY;
+        float x[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float4 a = y4[k];
@@ -530,12 +645,31 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
           sub2(a.x, a.y, mv[k].x, mv[k].y, o.x, o.y);
           sub2(a.z, a.w, mv[k].z, mv[k].w, o.z, o.w);
           y4[k] = o;
+          x[4 * k] = o.x; x[4 * k + 1] = o.y; x[4 * k + 2] = o.z; x[4 * k + 3] = o.w;
           mx = max3(mx, o.x, o.y);
           mn = min3(mn, o.x, o.y);
           mx = max3(mx, o.z, o.w);
           mn = min3(mn, o.z, o.w);
         }
-        if (u == 0) group_sz(mn, mx, g.bits, s, z, ri);
+        if (u == 0) {
+          group_sz(mn, mx, g.bits, s, z, ri);
+          if (whole) {
+            uint32_t pc[16];
+            const float zz = z, rr = ri;
+            const bool clean = codes_fma<32>(x, pc, [&](int, float& z0, float& z1, float& r0, float& r1) {
+              z0 = z1 = zz;
+              r0 = r1 = rr;
+            });
+            if (clean && !tiny_scale(s)) {
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc)
+                *reinterpret_cast<uint4*>(cbV + cb_off(r, 32 * q + 8 * cc)) =
+                    make_uint4(pc[4 * cc], pc[4 * cc + 1], pc[4 * cc + 2], pc[4 * cc + 3]);
+            } else {
+              v_codes_exact(&vec[r][32 * q], z, s, maxc, cbV, r, 32 * q);
+            }
+          }
+        }
       }
       if (u == 0) {  // V: every slot, zeros for tokens not in this call
         vsz[(0 * 4 + q) * kG + lane] = s;
@@ -559,6 +693,7 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       }
       float s, z, ri;
       group_sz(mn, mx, g.bits, s, z, ri);
+      if (tiny_scale(s)) ktiny = 1;
       ksz[0 * kD + d] = s;
       ksz[1 * kD + d] = z;
       ksz[2 * kD + d] = ri;
@@ -568,29 +703,59 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   }
   __syncthreads();
 
-  // ---- code words, one thread per 32-bit word; scales, zeros, indices
+  // ---- K codes of a sealed page (a unit: row and 16 channels, 4 x 4 channels 32 apart)
+  if (c.seal) {
+    for (int u = tid; u < kG * 8; u += blockDim.x) {
+      const int r = u >> 3, cbk = u & 7;
+      float x[16], zs[16], rs[16];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int ch = 4 * cbk + 32 * k4;
+        const float4 a = *reinterpret_cast<const float4*>(&vec[kG + r][ch]);
+        const float4 z4 = *reinterpret_cast<const float4*>(ksz + kD + ch);
+        const float4 r4 = *reinterpret_cast<const float4*>(ksz + 2 * kD + ch);
+        x[4 * k4] = a.x; x[4 * k4 + 1] = a.y; x[4 * k4 + 2] = a.z; x[4 * k4 + 3] = a.w;
+        zs[4 * k4] = z4.x; zs[4 * k4 + 1] = z4.y; zs[4 * k4 + 2] = z4.z; zs[4 * k4 + 3] = z4.w;
+        rs[4 * k4] = r4.x; rs[4 * k4 + 1] = r4.y; rs[4 * k4 + 2] = r4.z; rs[4 * k4 + 3] = r4.w;
+      }
+      uint32_t pc[8];
+      const bool clean = codes_fma<16>(x, pc, [&](int i2, float& z0, float& z1, float& r0, float& r1) {
+        z0 = zs[2 * i2]; z1 = zs[2 * i2 + 1];
+        r0 = rs[2 * i2]; r1 = rs[2 * i2 + 1];
+      });
+      if (clean && ktiny == 0) {
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)
+          *reinterpret_cast<uint2*>(cbK + cb_off(r, 4 * cbk + 32 * k4)) = make_uint2(pc[2 * k4], pc[2 * k4 + 1]);
+      } else {
+        k_codes_exact(vec[kG + r], ksz + kD, ksz, cbk, maxc, cbK, r);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- code words: the whole-page V block and a sealed K block from the 16-bit codes (16-byte
+  // chunks of four words per lane, spread over the warps); a partly written V block one word per
+  // thread, keeping the codes of the tokens already in the page; then scales, zeros, indices
   {
     uint32_t* vdst = reinterpret_cast<uint32_t*>(c.sub + g.off_vc);
-    const int nwords = kG * kD * g.bits / 32;
-    const int keep_lo = c.fresh ? 0 : lo;
-    const float(*Rv)[kLd] = vec;
-    const float(*Rk)[kLd] = vec + kG;
-    const bool whole = keep_lo == 0 && hi == kG;  // every token of the page is new
-    for (int wd = tid; wd < nwords; wd += blockDim.x) {
-      if (whole) {
-        vdst[wd] = g.bits == 2 ? v_word<2, false>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, 0, kG, 0u)
-                               : v_word<4, false>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, 0, kG, 0u);
-      } else {
+    const int nc = g.bits == 2 ? 2 : 4;  // chunks per block
+    const int nch = (whole ? nc : 0) + (c.seal ? nc : 0);
+    for (int ch = warp; ch < nch; ch += nwarps) {
+      const bool isV = whole && ch < nc;
+      const int wq = isV ? ch : ch - (whole ? nc : 0);
+      uint32_t* blk = isV ? vdst : reinterpret_cast<uint32_t*>(c.sub);
+      *reinterpret_cast<uint4*>(blk + wq * 128 + lane * 4) = pack_chunk(isV ? cbV : cbK, isV, g.bits, wq, lane);
+    }
+    if (!whole) {
+      const int nwords = kG * kD * g.bits / 32;
+      const int keep_lo = c.fresh ? 0 : lo;
+      const float(*Rv)[kLd] = vec;
+      for (int wd = tid; wd < nwords; wd += blockDim.x) {
         const uint32_t old = keep_lo > 0 ? vdst[wd] : 0u;  // tokens already in the page keep their codes
         vdst[wd] = g.bits == 2 ? v_word<2, true>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old)
                                : v_word<4, true>(wd, Rv, vsz, vsz + 4 * kG, vsz + 8 * kG, keep_lo, hi, old);
       }
-    }
-    if (c.seal) {
-      uint32_t* kdst = reinterpret_cast<uint32_t*>(c.sub);
-      for (int wd = tid; wd < nwords; wd += blockDim.x)
-        kdst[wd] = g.bits == 2 ? k_word<2>(wd, Rk, ksz, ksz + kD, ksz + 2 * kD)
-                               : k_word<4>(wd, Rk, ksz, ksz + kD, ksz + 2 * kD);
     }
   }
   float* vs_g = reinterpret_cast<float*>(c.sub + g.off_vs);
@@ -652,7 +817,8 @@ cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, i
   // fp16 lower bounds [P][64 rows], probe tables and channels (later the work queue); later the
   // s / z tables (12 kG + 3 kD floats) from the start
   const size_t tabs = std::max<size_t>((size_t)(kProbeV + kProbeK) * g.P + kProbeV + kProbeK, kQueueCap);
-  const size_t dyn = std::max<size_t>((size_t)32 * g.P + tabs, 12 * kG + 3 * kD) * sizeof(float);
+  // (after the assignment: the s / z tables, then two 8 KB code buffers from float 1024 on)
+  const size_t dyn = std::max<size_t>((size_t)32 * lb_ld(g.P) + tabs, 1024 + 4096) * sizeof(float);
   if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
       cudaSuccess)
     return e;
