@@ -1,3 +1,5 @@
+#include <algorithm>
+#include <cmath>
 // Split-K decode attention over the quantized paged cache on tensor cores
 // ("PatternKV", Section 3.4: pattern-index restoration, dequantization and the
 // QK^T / P.V products fused into the attention kernel).
@@ -1105,19 +1107,27 @@ int decode_stages() {
 
 }  // namespace
 
-// Number of splits of the token axis: the CTAs of all (sequence, KV head, split) units run in
-// as few and as full waves as possible, with a small charge per extra split (setup, combine).
+// Number of splits of the token axis.  Model: a CTA costs a fixed setup (the query and the
+// q.M_K table, the combine: about 40 pages' worth, measured) plus its pages; each SM takes
+// ceil(CTAs / SMs) of the CTAs, `occ` at a time, and a round of k concurrent CTAs takes
+// max(k, 3) CTA-times (fewer than 3 CTAs do not saturate an SM).  The page count is the capacity
+// (the lengths are on the device).  Fitted to the measured best split count of four shapes
+// (one B200): 64 groups of 1024 pages -> 9 splits (2-bit) and 13 (4-bit, fewer CTAs per SM),
+// 512 groups of 512 -> 2, 256 groups of ~300 (the decode-step loop) -> 2.
 int decode_mma_splits(const Geom& g, int Hq, int num_sms) {
-  const int occ = dispatch(g, Hq, decode_stages(), [&](auto L) { return decltype(L)::occupancy(g); });
-  const int slots = occ * num_sms;
+  const int occ = std::max(1, dispatch(g, Hq, decode_stages(), [&](auto L) { return decltype(L)::occupancy(g); }));
   const int units = g.B * g.H > 0 ? g.B * g.H : 1;
-  const int maxns = g.maxp > 1 ? (g.maxp < 256 ? g.maxp : 256) : 1;
+  const int pages = g.maxp > 1 ? g.maxp : 1;
+  const int maxns = pages < 256 ? pages : 256;
+  const int sms = num_sms > 0 ? num_sms : 1;
   int best = 1;
-  double best_cost = 1e30;
+  double best_cost = 1e300;
   for (int ns = 1; ns <= maxns; ++ns) {
-    const double waves = (double)((units * ns + slots - 1) / slots);
-    const double cost = waves / ns * (1.0 + 0.01 * ns);
-    if (cost < best_cost - 1e-12) { best_cost = cost; best = ns; }
+    const int64_t per_sm = ((int64_t)units * ns + sms - 1) / sms;  // CTAs of the busiest SM
+    const int64_t full = per_sm / occ, rem = per_sm % occ;
+    const double slots = (double)full * std::max(occ, 3) + (rem ? std::max<int64_t>(rem, 3) : 0);
+    const double cost = slots * (40.0 + std::ceil((double)pages / ns));
+    if (cost < best_cost * (1.0 - 1e-9)) { best_cost = cost; best = ns; }
   }
   return best;
 }
