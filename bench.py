@@ -189,7 +189,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    w = synth.WORKLOADS[args.workload].with_(bits=args.bits, transform=args.transform)
     synth.build()
     import oracle
     oracle.build()
@@ -540,6 +540,8 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--transform", type=int, default=0, choices=[0, 1],
+                    help="the Hadamard + dual-axis pre-transform on the headline workload")
     ap.add_argument("--ref-heads", type=int, default=2, help="reference arm: KV heads per step (bounded sample)")
     ap.add_argument("--ref-seqs", type=int, default=24, help="reference arm: sequences per step (bounded sample)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -569,7 +571,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    base = synth.WORKLOADS[args.workload].with_(bits=args.bits)
+    base = synth.WORKLOADS[args.workload].with_(bits=args.bits, transform=args.transform)
     if args.batch:
         base = base.with_(B=args.batch)
     w = base
