@@ -38,9 +38,10 @@ namespace kvq {
 namespace {
 
 constexpr int kAppendThreads = 128;
-constexpr int kQueueCap = 512;
+constexpr int kQueueCap = 2048;  // candidate (row, pattern) entries of a page; more: every pattern for every row
 constexpr int kProbe = 32;   // probe channels stored per pattern set (by decreasing spread)
-constexpr int kProbeK = 16;  // used for K rows (outlier channels make 16 enough)
+constexpr int kProbeK = 16;  // used for K rows (outlier channels make 16 enough) ...
+constexpr int kProbeKtx = 32;  // ... but not after the Hadamard rotation, which spreads them
 constexpr int kProbeV = 32;  // used for V rows (a tighter bound picks a better seed)
 constexpr int kLd = kD + 4;  // staged row stride (floats): 16-byte aligned, conflict-free columns
 
@@ -425,8 +426,9 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   const int ldh = lb_ld(P);
   __half* lbuf = reinterpret_cast<__half*>(dsm);  // [64 rows][ldh]
   float* tabV = dsm + 32 * ldh;
+  const int nprk = g.tx ? kProbeKtx : kProbeK;  // K probe channels
   float* tabK = tabV + kProbeV * P;
-  int32_t* pcV = reinterpret_cast<int32_t*>(tabK + kProbeK * P);
+  int32_t* pcV = reinterpret_cast<int32_t*>(tabK + nprk * P);
   int32_t* pcK = pcV + kProbeV;
   uint32_t* queue = reinterpret_cast<uint32_t*>(tabV);  // [kQueueCap]
   float* vsz = dsm;            // [3][4][kG]: s, z, 1/s per (group, V slot)
@@ -447,17 +449,18 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
   };
   if (tid == 0) qn = 0;
   {
-    // probe tables of this (set, head): V's 32 probe channels, K's first 16
+    // probe tables of this (set, head): V's 32 probe channels, K's first nprk
     const float4* gV = reinterpret_cast<const float4*>(wsp.pv + (shk + 1) * P * kProbe);
     const float* gK = wsp.pv + shk * P * kProbe;
+    const int nk4 = nprk / 4;
 #pragma unroll 4
     for (int i = tid; i < Pe * (kProbeV / 4); i += kAppendThreads) reinterpret_cast<float4*>(tabV)[i] = __ldg(gV + i);
 #pragma unroll 2
-    for (int i = tid; i < Pe * (kProbeK / 4); i += kAppendThreads)
+    for (int i = tid; i < Pe * nk4; i += kAppendThreads)
       reinterpret_cast<float4*>(tabK)[i] =
-          __ldg(reinterpret_cast<const float4*>(gK + (size_t)(i / (kProbeK / 4)) * kProbe) + i % (kProbeK / 4));
+          __ldg(reinterpret_cast<const float4*>(gK + (size_t)(i / nk4) * kProbe) + i % nk4);
     if (tid < kProbeV) pcV[tid] = __ldg(wsp.probe + (shk + 1) * kProbe + tid);
-    if (tid < kProbeK) pcK[tid] = __ldg(wsp.probe + shk * kProbe + tid);
+    if (tid < nprk) pcK[tid] = __ldg(wsp.probe + shk * kProbe + tid);
   }
 
   // ---- stage (and pre-transform) every vector
@@ -514,7 +517,8 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     if (kind == 0)
       lb_pass<kProbeV>(vec[r], pcV, tabV, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r]);
     else if (c.seal)
-      lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r]);
+      g.tx ? lb_pass<kProbeKtx>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r])
+           : lb_pass<kProbeK>(vec[r], pcK, tabK, half ? P0 : 0, half ? Pe : P0, lbuf, ldh, r, hlb[half][r], hj[half][r]);
     if (kind == 0 || c.seal) {
       // the half's best pattern is the likely seed: its row into L1 ahead of the exact range
       const float* mrow = (kind ? c.MK : c.MV) + (size_t)min(max(hj[half][r], 0), Pe - 1) * kD;
@@ -816,7 +820,8 @@ cudaError_t launch_append(const Geom& g, const void* k_new, const void* v_new, i
   if (e != cudaSuccess) return e;
   // fp16 lower bounds [P][64 rows], probe tables and channels (later the work queue); later the
   // s / z tables (12 kG + 3 kD floats) from the start
-  const size_t tabs = std::max<size_t>((size_t)(kProbeV + kProbeK) * g.P + kProbeV + kProbeK, kQueueCap);
+  const int nprk = g.tx ? kProbeKtx : kProbeK;
+  const size_t tabs = std::max<size_t>((size_t)(kProbeV + nprk) * g.P + kProbeV + nprk, kQueueCap);
   // (after the assignment: the s / z tables, then two 8 KB code buffers from float 1024 on)
   const size_t dyn = std::max<size_t>((size_t)32 * lb_ld(g.P) + tabs, 1024 + 4096) * sizeof(float);
   if ((e = cudaFuncSetAttribute(append_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
