@@ -206,8 +206,8 @@ def test_subnormal_scales_bit_exact(bits):
     # Groups and channels whose residuals differ only by subnormal amounts: the scale
     # s = (max - min) / maxc is subnormal (or 0), its reciprocal inexact or infinite, and every
     # code must still be the definition's rne(fl32(t / s)), clamped ("PatternKV", Section 3.2,
-    # Eq. 1).  Two full pages (the full-page kernel) and a 20-token partial page (the general
-    # kernel), the patterns zero where the tiny values sit.
+    # Eq. 1).  Two whole pages (codes from the one-FMA path, whose tiny-scale exception divides)
+    # and a 20-token partial page (the per-word path), the patterns zero where the tiny values sit.
     w = W["llama3_8b_32k"].with_(B=1, S=84, Hkv=1, Hq=2, P=4, bits=bits, v_alpha=0.0)
     k, v = synth.gen_kv(w)
     rng = np.random.default_rng(7)
@@ -240,5 +240,44 @@ def test_subnormal_scales_bit_exact(bits):
     assert np.any(e.vs[:, 0] != 0) and np.all(np.abs(e.vs[:, 0]) < 2.0 ** -126)
     assert np.any((e.ks != 0) & (np.abs(e.ks) < 2.0 ** -126))
     assert np.any(e.vs[:, 2] != 0) and np.any(e.ks[:, 100] != 0)
+    check_pages(cache, w, e, 0, 0)
+    check_tail(cache, w, k, 0, 0, w.S)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_code_ties_round_half_even(bits):
+    # Residuals placed exactly on rounding boundaries: in V group 1 and K channel 9 the values
+    # are 0, maxc and half-integers in between, so (R - z) / s is a half-integer (exactly) and the
+    # definition rounds it half to even ("PatternKV", Section 3.2, Eq. 1).  Whole pages (the
+    # one-FMA codes, whose boundary exception divides) and a partial page.
+    w = W["llama3_8b_32k"].with_(B=1, S=80, Hkv=1, Hq=2, P=4, bits=bits, v_alpha=0.0)
+    k, v = synth.gen_kv(w)
+    maxc = (1 << bits) - 1
+    rng = np.random.default_rng(11)
+    ladder = np.array([0.0, maxc] + [h + 0.5 for h in range(maxc)], np.float32)  # s = 1 when 0 and maxc occur
+
+    def bf16_bits(a):
+        return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+    k, v = k.copy(), v.copy()
+    g1 = ladder[rng.integers(0, len(ladder), size=(w.S, 32))]
+    g1[:, 0], g1[:, 1] = 0.0, maxc
+    v[0, :, 0, 32:64] = bf16_bits(g1)
+    kc = ladder[rng.integers(0, len(ladder), size=w.S)]
+    kc[::32], kc[1::32] = 0.0, maxc
+    k[0, :, 0, 9] = bf16_bits(kc)
+    Kf, Vf = synth.to_float(k, w.dtype), synth.to_float(v, w.dtype)
+    MK, MV, _, _ = oracle_patterns(w, Kf, Vf)
+    MK[:, :, 9] = 0.0
+    MV[:, :, 32:64] = 0.0
+    cache = make_cache(w, MK, MV, None, None)
+    cache.append(to_torch(k, w.dtype), to_torch(v, w.dtype))
+    torch.cuda.synchronize()
+    assert cache.read_status() == 0
+    e = encode_unit(w, Kf, Vf, 0, 0, MK, MV, None, None)
+    assert np.all(e.vs[:, 1] == 1.0) and np.all(e.ks[:, 9] == 1.0)
+    # the half-integers did round to even codes
+    half = (g1 % 1.0) == 0.5
+    assert half.any() and np.all(e.vcode[:, 32:64][half] % 2 == 0)
     check_pages(cache, w, e, 0, 0)
     check_tail(cache, w, k, 0, 0, w.S)
