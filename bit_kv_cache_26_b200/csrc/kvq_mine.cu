@@ -912,14 +912,17 @@ cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, i
 //     the end read as zeros) into a ring of shared-memory stages: the canonical K-major
 //     layout with 128-byte swizzle, 8-row x 128-byte atoms (SBO = 1024 B), channels 0-63
 //     and 64-127 in two 16 KB halves;
-//   * MMA warp (one thread): 8 tcgen05.mma of M = 128 (tokens) x N = 2 Pn (the bf16 hi parts
-//     of the Pn padded patterns, then their mid parts) x K = 16, fp32 accumulation in one of
-//     two TMEM buffers, so each product term keeps its own chain of 8 MMAs (the error model
-//     of the certification above); commits to the buffer's "full" and the stage's "free"
-//     barriers;
-//   * 8 epilogue warps, two warpgroups: warpgroup g owns TMEM buffer g and takes every other
-//     tile; token t's scores are TMEM lane t, so each warp handles its 32 tokens alone, with
-//     no barrier between warps: u_j = |m_j|^2 / 2 - x.m_j (e_j = 2 u_j) with the pattern index
+//   * MMA warp (one thread): 16 tcgen05.mma of M = 128 (tokens) x N = Pn (padded patterns) x
+//     K = 16, the 8 K steps against the bf16 hi parts of the patterns and then the 8 against
+//     their mid parts, into one fp32 accumulator in one of four TMEM buffers (Pn columns each);
+//     commits to the buffer's "full" and the stage's "free" barriers.  One chain of 16 MMAs:
+//     under the truncation model above it is off by at most 16 * 17 * 2^-22 |x| |m_j| (times
+//     1.008 for the partial sums' bound), which with the 2^-16 |m| below hi + mid gives
+//     |e_hat_j - e_j| <= 2^-12.59 |x| |m_j| plus the fp32 roundings, within E_j;
+//   * 8 epilogue warps, two warpgroups: warpgroup g takes every other tile, in TMEM buffers g
+//     and g + 2 in turn, so the MMAs of its next tile run while it scores this one; token t's
+//     scores are TMEM lane t, so each warp handles its 32 tokens alone, with no barrier
+//     between warps: u_j = |m_j|^2 / 2 - x.m_j (e_j = 2 u_j) with the pattern index
 //     written into the 7 low mantissa bits (a move of at most 2^-16 |u_j|), one running pair
 //     of smallest tagged values per chain, so one min chain yields the candidate, its index
 //     and the gap; the gap test widened by twice the largest move.  A token that fails it
@@ -1015,8 +1018,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
   const int prob = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Pn = (P + 15) & ~15, N = 2 * Pn;
-  const uint32_t tcols = N <= 128 ? 256u : 512u;  // two accumulator buffers
-  const uint32_t buf_cols = tcols / 2;
+  // four accumulator buffers of Pn columns (hi and mid parts of a pattern in one chain), each
+  // starting at a power-of-two column (16 .. 128)
+  const uint32_t buf_cols = Pn <= 16 ? 16u : Pn <= 32 ? 32u : Pn <= 64 ? 64u : 128u;
+  const uint32_t tcols = 4 * buf_cols;
   const uint32_t half_b = (uint32_t)N * 128u;      // B: channels 64-127 start N x 128 B in
   extern __shared__ __align__(16) uint8_t smraw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -1024,12 +1029,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
   uint8_t* At = base + (size_t)N * kD * 2;                              // [nst][2 halves][128 rows][128 B]
   float* hm = reinterpret_cast<float*>(At + (size_t)nst * kTcTileBytes);   // [Pn] |m_j|^2 / 2, padding past P
   float* gmax = hm + Pn;                                                // [4]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);               // full[nst], sfree[nst], tfull[2], tempty[2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gmax + 4);               // full[nst], sfree[nst], tfull[4], tempty[4]
   uint64_t* full = bars;
   uint64_t* sfree = bars + nst;
   uint64_t* tfull = bars + 2 * nst;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + 4;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 4);
   const float* Mp = M + (size_t)prob * P * kD;
   const int set = prob / s.heads, h = prob % s.heads;
 
@@ -1058,11 +1063,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
     gmax[1] = 0.f;
     for (int i = 0; i < nst; ++i) {
       mb_init(&full[i], 1);
-      mb_init(&sfree[i], 1 + kTcEpiWarps / 2);  // the MMA commit and the 4 warps of the tile's warpgroup
+      // the MMA commit, and in the first iteration the 4 warps of the tile's warpgroup (they read
+      // the staged rows for |x|^2)
+      mb_init(&sfree[i], first ? 1 + kTcEpiWarps / 2 : 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mb_init(&tfull[i], 1);
-      mb_init(&tempty[i], kTcEpiWarps / 2);  // buffer i belongs to warpgroup i
+      mb_init(&tempty[i], kTcEpiWarps / 2);  // buffer i belongs to warpgroup i % 2
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1119,52 +1126,59 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
   } else if (warp == 1) {
     // ---- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc(kTcM, N);
+      const uint32_t idesc = umma_idesc(kTcM, Pn);
       const uint32_t b0 = su32(Bt);
       int last = -1;  // newest tile whose MMAs were committed
       for (int k = 0; k < nt; ++k) {
-        const int st = k % nst, buf = k & 1;
+        const int st = k % nst, buf = k & 3;
         if (!tc_wait(&full[st], (uint32_t)((k / nst) & 1)) ||
-            (k >= 2 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 1) - 1) & 1)))) {
+            (k >= 4 && !tc_wait(&tempty[buf], (uint32_t)(((k >> 2) - 1) & 1)))) {
           set_status(status, KVQ_DEV_TIMEOUT);
           break;
         }
         tc_fence_after();
         const uint32_t a0 = su32(At + (size_t)st * kTcTileBytes);
         const uint32_t d = tbase + (uint32_t)buf * buf_cols;
+        // x.hi_j then x.mid_j into the same accumulator: 16 MMAs of N = Pn; the mid rows start
+        // Pn rows (Pn x 128 B, whole 8-row atoms) into each half of B
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks)  // K step ks: half ks / 4, 32 B per step inside the atom
-          umma_bf16(d, umma_desc_sw128(a0 + (ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32),
-                    umma_desc_sw128(b0 + (ks >> 2) * half_b + (ks & 3) * 32), idesc, ks > 0);
+        for (int ks = 0; ks < 2 * (kD / 16); ++ks) {  // K step ks & 7: half (ks & 7) / 4, 32 B per step
+          const int kk = ks & 7;
+          const uint32_t bpart = ks < kD / 16 ? 0u : (uint32_t)Pn * 128u;
+          umma_bf16(d, umma_desc_sw128(a0 + (kk >> 2) * (kTcTileBytes / 2) + (kk & 3) * 32),
+                    umma_desc_sw128(b0 + bpart + (kk >> 2) * half_b + (kk & 3) * 32), idesc, ks > 0);
+        }
         umma_commit(&tfull[buf]);
         umma_commit(&sfree[st]);
         last = k;
       }
       // drain: a commit tracks every tcgen05 operation this thread issued before it, so the
       // newest tile's commit landing means no MMA still writes TMEM or reads shared memory
-      if (last >= 0 && !tc_wait(&tfull[last & 1], (uint32_t)((last >> 1) & 1))) set_status(status, KVQ_DEV_TIMEOUT);
+      if (last >= 0 && !tc_wait(&tfull[last & 3], (uint32_t)((last >> 2) & 1))) set_status(status, KVQ_DEV_TIMEOUT);
     }
   } else {
-    // ---- epilogue warps: warpgroup g takes tiles k with k % 2 == g, i.e. TMEM buffer g, each
-    // warp its 32 rows, with no barrier between warps
+    // ---- epilogue warps: warpgroup g takes tiles k with k % 2 == g, in TMEM buffers g and g + 2
+    // in turn (the next tile's MMAs run while this one is scored), each warp its 32 rows, with no
+    // barrier between warps
     const int ew = warp - 2, wg = ew >> 2, q4 = warp & 3;  // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;
     const float nm_max = gmax[0], msq_max = gmax[1];
-    const uint32_t taddr = tbase + ((uint32_t)(q4 * 32) << 16) + (uint32_t)wg * buf_cols;
+    const uint32_t tlane = tbase + ((uint32_t)(q4 * 32) << 16);
     for (int k = wg; k < nt; k += 2) {
       const int st = k % nst;
       const int64_t i = tile_t0(k) + row;
       const bool valid = i < s.n;
       float xsq = 0.f;
       if (!first && valid) xsq = xsq_cache[(size_t)prob * s.n + i];
-      if (!__all_sync(kFull, tc_wait(&tfull[wg], (uint32_t)((k >> 1) & 1)))) {
+      const int buf = k & 3;
+      const uint32_t taddr = tlane + (uint32_t)buf * buf_cols;
+      if (!__all_sync(kFull, tc_wait(&tfull[buf], (uint32_t)((k >> 2) & 1)))) {
         if (lane == 0) set_status(status, KVQ_DEV_TIMEOUT);
         break;
       }
       tc_fence_after();
-      float hv[8], mv[8], hn[8], mn_[8];
+      float hv[8], hn[8];
       tmem_ld8_issue(taddr, hv);
-      tmem_ld8_issue(taddr + Pn, mv);
       if (first) {
         // |x|^2 of the row from the staged tile (two swizzled halves of 64 channels)
         const uint8_t* stg = At + (size_t)st * kTcTileBytes;
@@ -1183,26 +1197,23 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
         xsq = (a0 + a1) + (b0 + b1);
         if (valid) xsq_cache[(size_t)prob * s.n + i] = xsq;
       }
-      __syncwarp();
-      if (lane == 0) mb_arrive(&sfree[st]);
+      if (first) {
+        __syncwarp();
+        if (lane == 0) mb_arrive(&sfree[st]);
+      }
       tmem_ld_wait();
       // the two smallest tagged scores in two chains (even / odd patterns); blocks of 8
       // columns, the next block's loads in flight while one is scored
       float m1a = INFINITY, m2a = INFINITY, m1b = INFINITY, m2b = INFINITY;
       for (int c0 = 0; c0 < Pn; c0 += 8) {
         const bool more = c0 + 8 < Pn;
-        if (more) {
-          tmem_ld8_issue(taddr + c0 + 8, hn);
-          tmem_ld8_issue(taddr + Pn + c0 + 8, mn_);
-        }
+        if (more) tmem_ld8_issue(taddr + c0 + 8, hn);
 #pragma unroll
         for (int q = 0; q < 8; q += 4) {
           const float4 hq = *reinterpret_cast<const float4*>(hm + c0 + q);
-          float s0, s1, s2, s3, u0, u1, u2, u3;
-          add2f(hv[q], hv[q + 1], mv[q], mv[q + 1], s0, s1);
-          add2f(hv[q + 2], hv[q + 3], mv[q + 2], mv[q + 3], s2, s3);
-          sub2(hq.x, hq.y, s0, s1, u0, u1);
-          sub2(hq.z, hq.w, s2, s3, u2, u3);
+          float u0, u1, u2, u3;
+          sub2(hq.x, hq.y, hv[q], hv[q + 1], u0, u1);
+          sub2(hq.z, hq.w, hv[q + 2], hv[q + 3], u2, u3);
           low2_add(m1a, m2a, tag_score(u0, c0 + q));
           low2_add(m1b, m2b, tag_score(u1, c0 + q + 1));
           low2_add(m1a, m2a, tag_score(u2, c0 + q + 2));
@@ -1211,7 +1222,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
         if (more) {
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { hv[q] = hn[q]; mv[q] = mn_[q]; }
+          for (int q = 0; q < 8; ++q) hv[q] = hn[q];
         }
       }
       const float m1 = fminf(m1a, m1b);
@@ -1233,16 +1244,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
         int cnt = 0;
         for (int c0 = 0; c0 < Pn; c0 += 8) {
           tmem_ld8_issue(taddr + c0, hv);
-          tmem_ld8_issue(taddr + Pn + c0, mv);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 8; q += 4) {
             const float4 hq = *reinterpret_cast<const float4*>(hm + c0 + q);
-            float s0, s1, s2, s3, u[4];
-            add2f(hv[q], hv[q + 1], mv[q], mv[q + 1], s0, s1);
-            add2f(hv[q + 2], hv[q + 3], mv[q + 2], mv[q + 3], s2, s3);
-            sub2(hq.x, hq.y, s0, s1, u[0], u[1]);
-            sub2(hq.z, hq.w, s2, s3, u[2], u[3]);
+            float u[4];
+            sub2(hq.x, hq.y, hv[q], hv[q + 1], u[0], u[1]);
+            sub2(hq.z, hq.w, hv[q + 2], hv[q + 3], u[2], u[3]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = c0 + q + e;
@@ -1264,7 +1272,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) mine_assign_tc_kernel(const __g
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mb_arrive(&tempty[wg]);
+      if (lane == 0) mb_arrive(&tempty[buf]);
     }
   }
   tc_fence_before();
@@ -1338,12 +1346,12 @@ __global__ void __launch_bounds__(kFixWarps * 32) mine_fixup_kernel(Src s, int P
 // ring depth that fits next to the patterns in 227 KB, and the dynamic shared memory it needs
 int mine_tc_stages(int P) {
   const int Pn = (P + 15) & ~15;
-  const int fixed = 2 * Pn * kD * 2 + Pn * 4 + 16 + (2 * kTcMaxStages + 4) * 8 + 16 + 1024;
+  const int fixed = 2 * Pn * kD * 2 + Pn * 4 + 16 + (2 * kTcMaxStages + 8) * 8 + 16 + 1024;
   return std::max(2, std::min(kTcMaxStages, (227 * 1024 - fixed) / kTcTileBytes));
 }
 size_t mine_tc_smem(int P) {
   const int Pn = (P + 15) & ~15, nst = mine_tc_stages(P);
-  return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + Pn * 4 + 16 + (2 * nst + 4) * 8 + 16 + 1024;
+  return (size_t)2 * Pn * kD * 2 + (size_t)nst * kTcTileBytes + Pn * 4 + 16 + (2 * nst + 8) * 8 + 16 + 1024;
 }
 
 // Centroid = fl32(float64 sum / count); an empty cluster keeps its pattern.  With `part` (fp32
