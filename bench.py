@@ -391,6 +391,15 @@ def measure_path(w, args, dev, world: int, rank: int, headline: bool, shard=None
     for name, r in rooflines.items():
         r["traffic"] = traffic.get(name)
         r["frac"] = r["achieved"] / r["peak"]
+    # The exact d_mm argmin by its definition costs 3 lane-ops (subtract, max, min) per channel and
+    # pattern for K and for V; the kernel prunes it with exact bounds, so this is the rate at which
+    # that definitional work gets done, against the fp32 lanes (128 per SM) at the sampled clock.
+    sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+    naive_ops = token_heads * 2 * w.P * D * 3
+    alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * sm_mhz * 1e6
+    rooflines["quantize_append"]["alu_naive_equivalent"] = {
+        "lane_ops_per_token_head": 2 * w.P * D * 3, "achieved_tops": naive_ops / (append_ms * 1e-3) / 1e12,
+        "peak_tops": alu_peak / 1e12, "frac": naive_ops / (append_ms * 1e-3) / alu_peak}
     dominant = max(rooflines, key=lambda kk: rooflines[kk]["ms"])
     dom = rooflines[dominant]
     roofline = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"], "unit": dom["unit"],

@@ -20,7 +20,8 @@ namespace kvq {
 namespace {
 
 constexpr int kFitPasses = 3;
-constexpr int kReduceChunk = 4096;
+constexpr int kFitChunk = 1024;  // tokens per block of a fit pass: the fixed order of the column sums
+constexpr int kFitWarps = 8;
 
 struct MineWs {
   int32_t* status;  // device status word (KVQ_DEV_* bits), at offset 0 of the workspace
@@ -33,12 +34,10 @@ struct MineWs {
   uint8_t* ambn;    // [NP][n] candidates listed (255: more than 8, every pattern is checked)
   int32_t* amb_cnt; // [NP]
   float* y;         // [NP][n][128] (transform only)
-  double* v64;      // [NP][n][128] (transform only)
-  double* colpart;  // [NP][fit chunks][128] per-chunk column partials (transform only)
-  double* colsum;   // [NP][128]
-  double* colsq;    // [NP][128]
+  double* rrow;     // [2][NP][n] reciprocal of each row's running divisor product, one buffer per pass parity
+  double* colpart;  // [NP][fit chunks][2][128] per-chunk shifted column sums and sums of squares
   double* colscale; // [NP][128]  running product of column divisors
-  double* coldiv;   // [NP][128]  this pass's divisor
+  double* cinv;     // [NP][128]  its reciprocal
   double* accpart;  // [NP][sum chunks][P][128] per-CTA cluster sums of the fp32 rows (transform only)
 };
 
@@ -49,7 +48,7 @@ __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_
 // order, so the result is the same on every run.  A fixed CTA budget (two per SM of a 148-SM
 // part) keeps the workspace independent of the device.
 constexpr int kAccF32Ctas = 296;
-inline int64_t fit_chunks(int64_t n) { return (n + kReduceChunk - 1) / kReduceChunk; }
+inline int64_t fit_chunks(int64_t n) { return (n + kFitChunk - 1) / kFitChunk; }
 inline int accum_f32_chunks(int64_t n, int NP, int P) {
   const int slices = P <= 64 ? 1 : (P <= 128 ? 2 : 4);
   const int64_t ntiles = (n + 127) / 128;
@@ -71,12 +70,10 @@ inline MineWs carve(void* ws, int64_t n, int NP, int P, int transform, int32_t* 
   w.amb_cnt = (int32_t*)p; p += align256((size_t)NP * sizeof(int32_t));
   if (transform) {
     w.y = (float*)p; p += align256((size_t)NP * n * kD * sizeof(float));
-    w.v64 = (double*)p; p += align256((size_t)NP * n * kD * sizeof(double));
-    w.colpart = (double*)p; p += align256((size_t)NP * fit_chunks(n) * kD * sizeof(double));
-    w.colsum = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
-    w.colsq = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
+    w.rrow = (double*)p; p += align256((size_t)2 * NP * n * sizeof(double));
+    w.colpart = (double*)p; p += align256((size_t)NP * fit_chunks(n) * 2 * kD * sizeof(double));
     w.colscale = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
-    w.coldiv = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
+    w.cinv = (double*)p; p += align256((size_t)NP * kD * sizeof(double));
     w.accpart = (double*)p; p += align256((size_t)NP * accum_f32_chunks(n, NP, P) * P * kD * sizeof(double));
   }
   return w;
@@ -96,76 +93,177 @@ struct Src {
 };
 
 // ---- pre-transform fit ------------------------------------------------------
+//
+// Three passes of (row normalisation, column std) over v = fwht(x) (KVarN's dual-axis fit), with
+// the rotated rows never stored: pass p recomputes each row as v_p = fwht(x) * (1 / C_p) *
+// (1 / R_{p-1}) (C_p: product of the earlier passes' column divisors, R_{p-1}: of the row's own
+// earlier divisors, kept as its reciprocal), takes its population std r_p (mean first, then
+// squared deviations), and
+// adds w = v_p / r_p, shifted by row 0's w, into per-column sums and sums of squares; the
+// column std is sqrt(S2 / n - (S1 / n)^2) of those shifted values.  float64 throughout; the
+// products and reciprocals stand for the sequential divisions of the definition, a few ulps
+// apart.  Each block takes a fixed chunk of tokens and writes its partial sums, which the
+// finish kernel adds in chunk order, so the fit is the same on every run.
 
-// v64 = fwht(x) (fp32 butterfly) per token; warp per token.
-__global__ void fit_prep_kernel(Src s, double* v64, double* colscale) {
-  const int prob = blockIdx.y, lane = threadIdx.x & 31;
-  const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (blockIdx.x == 0 && threadIdx.x < kD) colscale[prob * kD + threadIdx.x] = 1.0;
-  if (i >= s.n) return;
-  float v[4];
+// warp: R rows' normalised values w (this lane's channels lane + 32 k) and the reciprocals of
+// their std, the rows' steps interleaved (each row's operations as for one row alone).  rin:
+// the rows' running reciprocal divisors of the earlier passes, or null.
+template <int R>
+__device__ __forceinline__ void fit_rows_eval(const Src& s, int prob, const int64_t (&i)[R], const double (&ci)[4],
+                                              const double* rin, int lane, double (&w)[R][4], double (&ri)[R]) {
+  float v[R][4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) v[k] = s.at(prob, i, lane + 32 * k);
-  fwht_warp(v, lane);
-  double* row = v64 + ((size_t)prob * s.n + i) * kD;
+  for (int q = 0; q < R; ++q)
 #pragma unroll
-  for (int k = 0; k < 4; ++k) row[lane + 32 * k] = (double)v[k];
+    for (int k = 0; k < 4; ++k) v[q][k] = s.at(prob, i[q], lane + 32 * k);
+  // the butterfly of fwht_warp, row by row within each stage
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float o = __shfl_xor_sync(kFull, v[q][k], h);
+        v[q][k] = (lane & h) ? __fsub_rn(o, v[q][k]) : __fadd_rn(v[q][k], o);
+      }
+  double u[R][4], m[R], sq[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const float a0 = v[q][0], b0 = v[q][1], a1 = v[q][2], b1 = v[q][3];
+    const float t0 = __fadd_rn(a0, b0), t1 = __fsub_rn(a0, b0), t2 = __fadd_rn(a1, b1), t3 = __fsub_rn(a1, b1);
+    const float f[4] = {__fadd_rn(t0, t2), __fadd_rn(t1, t3), __fsub_rn(t0, t2), __fsub_rn(t1, t3)};
+    const double rr = rin ? rin[i[q]] : 1.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[q][k] = (double)f[k] * ci[k] * rr;
+    m[q] = (u[q][0] + u[q][1]) + (u[q][2] + u[q][3]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q) m[q] += __shfl_xor_sync(kFull, m[q], o);
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const double mean = m[q] / 128.0;
+    sq[q] = 0.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const double t = u[q][k] - mean;
+      sq[q] += t * t;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q) sq[q] += __shfl_xor_sync(kFull, sq[q], o);
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    double r = sqrt(sq[q] / 128.0);
+    if (r == 0.0) r = 1.0;
+    ri[q] = 1.0 / r;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[q][k] = u[q][k] * ri[q];
+  }
 }
 
-// Row pass: divide every row by its population std (1 if zero); warp per row.  Also applies
-// the previous column pass's divisors first when `coldiv` is given.
-__global__ void fit_row_kernel(int64_t n, double* v64, const double* coldiv) {
-  const int prob = blockIdx.y, lane = threadIdx.x & 31;
-  const int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (i >= n) return;
-  double* row = v64 + ((size_t)prob * n + i) * kD;
-  double v[4];
+// One fit pass over the tokens of chunk blockIdx.x of problem blockIdx.y; warp w takes rows
+// i0 + w, i0 + w + kFitWarps, ... (one at a time: interleaving four rows per warp measured
+// slower, its registers halving the warps per SM).  rin: the previous pass's reciprocal row
+// products (null in pass 0); cinv: 1 / C_p (null in pass 0).
+constexpr int kFitRows = 1;
+__global__ void __launch_bounds__(kFitWarps * 32) fit_pass_kernel(Src s, const double* __restrict__ cinv,
+                                                                  const double* __restrict__ rin,
+                                                                  double* __restrict__ rout,
+                                                                  double* __restrict__ colpart) {
+  __shared__ double shift[kD];
+  __shared__ double red[kFitWarps][2][kD];
+  const int prob = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t i0 = (int64_t)blockIdx.x * kFitChunk, i1 = min(s.n, i0 + kFitChunk);
+  double ci[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ci[k] = cinv ? cinv[prob * kD + lane + 32 * k] : 1.0;
+  const double* rp = rin ? rin + (size_t)prob * s.n : nullptr;
+  double* ro = rout + (size_t)prob * s.n;
+  if (warp == 0) {
+    const int64_t z[1] = {0};
+    double w0[1][4], r0[1];
+    fit_rows_eval<1>(s, prob, z, ci, rp, lane, w0, r0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) shift[lane + 32 * k] = w0[0][k];
+  }
+  __syncthreads();
+  double sh[4], s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sh[k] = shift[lane + 32 * k];
+  for (int64_t b = i0 + warp; b < i1; b += kFitRows * kFitWarps) {
+    int64_t ii[kFitRows];
+#pragma unroll
+    for (int q = 0; q < kFitRows; ++q) ii[q] = min(b + (int64_t)q * kFitWarps, i1 - 1);  // past the end: a repeat, unused
+    double w[kFitRows][4], ri[kFitRows];
+    fit_rows_eval<kFitRows>(s, prob, ii, ci, rp, lane, w, ri);
+#pragma unroll
+    for (int q = 0; q < kFitRows; ++q) {
+      if (b + (int64_t)q * kFitWarps >= i1) break;
+      if (lane == 0) ro[ii[q]] = rp ? rp[ii[q]] * ri[q] : ri[q];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const double t = w[q][k] - sh[k];
+        s1[k] += t;
+        s2[k] += t * t;
+      }
+    }
+  }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    v[k] = row[lane + 32 * k];
-    if (coldiv) v[k] = v[k] / coldiv[prob * kD + lane + 32 * k];
+    red[warp][0][lane + 32 * k] = s1[k];
+    red[warp][1][lane + 32 * k] = s2[k];
   }
-  double mean = warp_sum_d(v[0] + v[1] + v[2] + v[3]) / 128.0;
-  double sq = 0.0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) { double t = v[k] - mean; sq += t * t; }
-  double r = sqrt(warp_sum_d(sq) / 128.0);
-  if (r == 0.0) r = 1.0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) row[lane + 32 * k] = v[k] / r;
-}
-
-// Column statistics, per chunk of kReduceChunk tokens: pass 0 sums, pass 1 squared deviations
-// from the mean; 128 threads = channels.  Each chunk writes its own partial, and
-// fit_colreduce_kernel adds the partials in chunk order, so the statistics (and the column
-// factors) are the same on every run.
-__global__ void fit_col_kernel(int64_t n, const double* v64, const double* colsum, double* colpart, int which) {
-  const int prob = blockIdx.y, d = threadIdx.x;
-  const int64_t i0 = (int64_t)blockIdx.x * kReduceChunk, i1 = min(n, i0 + kReduceChunk);
-  const double* base = v64 + (size_t)prob * n * kD;
-  double acc = 0.0;
-  if (which == 0) {
-    for (int64_t i = i0; i < i1; ++i) acc += base[i * kD + d];
-  } else {
-    const double mean = colsum[prob * kD + d] / (double)n;
-    for (int64_t i = i0; i < i1; ++i) { const double t = base[i * kD + d] - mean; acc += t * t; }
+  __syncthreads();
+  if (threadIdx.x < kD) {
+    const int d = threadIdx.x;
+    double a = 0.0, c = 0.0;
+    for (int q = 0; q < kFitWarps; ++q) {
+      a += red[q][0][d];
+      c += red[q][1][d];
+    }
+    double* out = colpart + ((size_t)prob * gridDim.x + blockIdx.x) * 2 * kD;
+    out[d] = a;
+    out[kD + d] = c;
   }
-  colpart[((size_t)prob * gridDim.x + blockIdx.x) * kD + d] = acc;
 }
 
-__global__ void fit_colreduce_kernel(int chunks, const double* colpart, double* out) {
+// Column std of the pass from the chunk partials (added in chunk order); C_{p+1} = C_p * std
+// (1 where the std is 0) and its reciprocal.  One block of 128 threads per problem.
+__global__ void fit_finish_kernel(int64_t n, int chunks, const double* __restrict__ colpart,
+                                  double* __restrict__ colscale, double* __restrict__ cinv, int first) {
   const int prob = blockIdx.x, d = threadIdx.x;
-  double acc = 0.0;
-  for (int c = 0; c < chunks; ++c) acc += colpart[((size_t)prob * chunks + c) * kD + d];
-  out[prob * kD + d] = acc;
-}
-
-__global__ void fit_colfinish_kernel(int64_t n, const double* colsq, double* colscale, double* coldiv) {
-  const int prob = blockIdx.x, d = threadIdx.x;
-  double s = sqrt(colsq[prob * kD + d] / (double)n);
-  if (s == 0.0) s = 1.0;
-  colscale[prob * kD + d] *= s;
-  coldiv[prob * kD + d] = s;
+  double a = 0.0, b = 0.0;
+  const double* q = colpart + (size_t)prob * chunks * 2 * kD + d;
+  int c = 0;
+  for (; c + 8 <= chunks; c += 8) {  // eight chunks' loads in flight, added in order
+    double qa[8], qb[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      qa[e] = q[(size_t)(c + e) * 2 * kD];
+      qb[e] = q[(size_t)(c + e) * 2 * kD + kD];
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      a += qa[e];
+      b += qb[e];
+    }
+  }
+  for (; c < chunks; ++c) {
+    a += q[(size_t)c * 2 * kD];
+    b += q[(size_t)c * 2 * kD + kD];
+  }
+  const double m = a / (double)n;
+  double var = b / (double)n - m * m;
+  if (var < 0.0) var = 0.0;
+  double sd = sqrt(var);
+  if (sd == 0.0) sd = 1.0;
+  const double C = (first ? 1.0 : colscale[prob * kD + d]) * sd;
+  colscale[prob * kD + d] = C;
+  cinv[prob * kD + d] = 1.0 / C;
 }
 
 __global__ void fit_output_kernel(const double* colscale, float* colscale_out) {
@@ -1384,8 +1482,8 @@ size_t mine_workspace(int64_t n, int sets, int heads, int P, int transform) {
              align256((size_t)NP * (size_t)n * sizeof(int32_t)) + align256((size_t)NP * (size_t)n * 8) +
              align256((size_t)NP * (size_t)n) + align256((size_t)NP * sizeof(int32_t));
   if (transform)
-    b += align256((size_t)NP * n * kD * sizeof(float)) + align256((size_t)NP * n * kD * sizeof(double)) +
-         align256((size_t)NP * fit_chunks(n) * kD * sizeof(double)) + 4 * align256((size_t)NP * kD * sizeof(double)) +
+    b += align256((size_t)NP * n * kD * sizeof(float)) + align256((size_t)2 * NP * n * sizeof(double)) +
+         align256((size_t)NP * fit_chunks(n) * 2 * kD * sizeof(double)) + 2 * align256((size_t)NP * kD * sizeof(double)) +
          align256((size_t)NP * accum_f32_chunks(n, NP, P) * P * kD * sizeof(double));
   return b + 256;
 }
@@ -1443,14 +1541,11 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
   if ((e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
 
   if (a.transform) {
-    fit_prep_kernel<<<rows_grid, 256, 0, st>>>(s, w.v64, w.colscale);
     for (int p = 0; p < kFitPasses; ++p) {
-      fit_row_kernel<<<rows_grid, 256, 0, st>>>(a.n, w.v64, p == 0 ? nullptr : w.coldiv);
-      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colpart, 0);
-      fit_colreduce_kernel<<<NP, kD, 0, st>>>((int)chunks, w.colpart, w.colsum);
-      fit_col_kernel<<<dim3(chunks, NP), kD, 0, st>>>(a.n, w.v64, w.colsum, w.colpart, 1);
-      fit_colreduce_kernel<<<NP, kD, 0, st>>>((int)chunks, w.colpart, w.colsq);
-      fit_colfinish_kernel<<<NP, kD, 0, st>>>(a.n, w.colsq, w.colscale, w.coldiv);
+      double* rin = p == 0 ? nullptr : w.rrow + (size_t)((p + 1) & 1) * NP * a.n;
+      double* rout = w.rrow + (size_t)(p & 1) * NP * a.n;
+      fit_pass_kernel<<<dim3(chunks, NP), kFitWarps * 32, 0, st>>>(s, p == 0 ? nullptr : w.cinv, rin, rout, w.colpart);
+      fit_finish_kernel<<<NP, kD, 0, st>>>(a.n, (int)chunks, w.colpart, w.colscale, w.cinv, p == 0);
     }
     fit_output_kernel<<<NP, kD, 0, st>>>(w.colscale, a.colscale);
     apply_kernel<<<rows_grid, 256, 0, st>>>(s, a.colscale, w.y);
