@@ -463,9 +463,9 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     if (tid < nprk) pcK[tid] = __ldg(wsp.probe + shk * kProbe + tid);
   }
 
-  // ---- stage (and pre-transform) every vector
-  if (!g.tx) {
-    // 16 threads per row, 8 channels (one 16-byte load) each; all loads issued first
+  // ---- stage (and pre-transform) every vector: 16 threads per row, 8 channels (one 16-byte
+  // load) each, all loads issued first
+  {
     uint4 raw[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -487,22 +487,29 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
       dst[0] = make_float4(f[0], f[1], f[2], f[3]);
       dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
-  } else {
-    // warp per row: Hadamard rotation and the fitted column / row normalisation
-    for (int r = warp; r < 2 * kG; r += nwarps) {
-      if (!row_on(r)) continue;
-      const bool isv = r < kG;
-      const uint16_t* src = row_src(r);
-      float y[4];
+  }
+  if (g.tx) {
+    // in place, two staged rows per warp at a time: Hadamard rotation and the fitted column / row
+    // normalisation (rows the call does not touch are transformed too and not kept)
+    __syncthreads();
+    for (int r0 = warp; r0 < 2 * kG; r0 += 2 * nwarps) {
+      const int rs[2] = {r0, r0 + nwarps};
+      float y[2][4], rr[2];
+      const float* cq[2] = {rs[0] < kG ? c.cV : c.cK, rs[1] < kG ? c.cV : c.cK};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) y[k] = load_elem(src + lane + 32 * k, g.dtype);
-      float rr = 1.0f;
-      transform_row_warp(y, isv ? c.cV : c.cK, rr, lane);
+      for (int q = 0; q < 2; ++q)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) vec[r][lane + 32 * k] = y[k];
-      if (lane == 0) {
-        if (isv) vrow_s[r] = rr;
-        else krow_s[r - kG] = rr;
+        for (int k = 0; k < 4; ++k) y[q][k] = row_on(rs[q]) ? vec[rs[q]][lane + 32 * k] : 0.f;
+      transform_rows_warp<2>(y, cq, rr, lane);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (!row_on(rs[q])) continue;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) vec[rs[q]][lane + 32 * k] = y[q][k];
+        if (lane == 0) {
+          if (rs[q] < kG) vrow_s[rs[q]] = rr[q];
+          else krow_s[rs[q] - kG] = rr[q];
+        }
       }
     }
   }

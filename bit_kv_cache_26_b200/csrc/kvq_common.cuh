@@ -225,6 +225,63 @@ __device__ __forceinline__ void transform_row_warp(float v[4], const float* c, f
   r_out = r;
 }
 
+// transform_row_warp for R tokens held by a warp at once, their steps interleaved (each token's
+// operations exactly those of transform_row_warp).  c[q]: token q's column factors.
+template <int R>
+__device__ __forceinline__ void transform_rows_warp(float (&v)[R][4], const float* const (&c)[R], float (&r_out)[R],
+                                                    int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float p = __shfl_xor_sync(kFull, v[q][k], h);
+        v[q][k] = (lane & h) ? __fsub_rn(p, v[q][k]) : __fadd_rn(v[q][k], p);
+      }
+  float sm[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const float a0 = v[q][0], b0 = v[q][1], a1 = v[q][2], b1 = v[q][3];
+    const float t0 = __fadd_rn(a0, b0), t1 = __fsub_rn(a0, b0), t2 = __fadd_rn(a1, b1), t3 = __fsub_rn(a1, b1);
+    v[q][0] = __fadd_rn(t0, t2);
+    v[q][1] = __fadd_rn(t1, t3);
+    v[q][2] = __fsub_rn(t0, t2);
+    v[q][3] = __fsub_rn(t1, t3);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[q][k] = __fdiv_rn(v[q][k], __ldg(c[q] + lane + 32 * k));
+    sm[q] = __fadd_rn(__fadd_rn(v[q][0], v[q][2]), __fadd_rn(v[q][1], v[q][3]));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q) sm[q] = __fadd_rn(sm[q], __shfl_xor_sync(kFull, sm[q], o));
+  float sv[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const float mean = __fmul_rn(sm[q], 0.0078125f);
+    float dev[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float t = __fsub_rn(v[q][k], mean);
+      dev[k] = __fmul_rn(t, t);
+    }
+    sv[q] = __fadd_rn(__fadd_rn(dev[0], dev[2]), __fadd_rn(dev[1], dev[3]));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < R; ++q) sv[q] = __fadd_rn(sv[q], __shfl_xor_sync(kFull, sv[q], o));
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    float r = __fsqrt_rn(__fmul_rn(sv[q], 0.0078125f));
+    if (r == 0.0f) r = 1.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[q][k] = __fdiv_rn(v[q][k], r);
+    r_out[q] = r;
+  }
+}
+
 // Nearest pattern under the min-max distance, warp-cooperative, lowest index on ties.
 // y: this lane's 4 channels (lane + 32k).  M: P x 128 fp32 patterns (global or shared).
 __device__ __forceinline__ int assign_warp(const float y[4], const float* M, int P, int lane) {
