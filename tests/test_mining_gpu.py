@@ -83,6 +83,8 @@ def _to_dev(x32: np.ndarray, dtype):
     (64, 8192, torch.bfloat16),    # tcgen05 assignment, 128 score columns, two CTAs per SM
     (100, 8192, torch.bfloat16),   # tcgen05 assignment, 224 score columns, one CTA per SM
     (32, 4096, torch.float16),     # mma.sync assignment (fp16 rows split into hi + lo)
+    (48, 8192, torch.bfloat16),    # tcgen05 assignment, 48 of a 64-column accumulator used
+    (128, 8192, torch.bfloat16),   # tcgen05 assignment, four 128-column accumulators
 ])
 @pytest.mark.parametrize("iters", [1, 4])
 def test_planted_near_ties_bit_exact(P, n, dtype, iters):

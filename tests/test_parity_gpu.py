@@ -31,6 +31,11 @@ CASES = {
     # more than 64 patterns: the tcgen05 assignment with 7-bit tags, 224 score columns and one
     # CTA per SM, the cluster sums with 8 clusters per warp, the fix-up with 128 threads a token
     "gqa4_p100": (W["llama3_8b_32k"].with_(B=2, S=1000, Hkv=2, Hq=8, P=100), [1000]),
+    # pattern counts that pad the tcgen05 tile: 17 (32-column accumulators), 48 (48 of 64
+    # columns used), 128 (the largest tcgen05 tile: four 128-column buffers, all of TMEM)
+    "gqa4_p17": (W["llama3_8b_32k"].with_(B=1, S=500, Hkv=1, Hq=4, P=17), [250, 250]),
+    "gqa4_p48": (W["llama3_8b_32k"].with_(B=2, S=600, Hkv=2, Hq=8, P=48), [600]),
+    "gqa4_p128": (W["llama3_8b_32k"].with_(B=1, S=700, Hkv=1, Hq=4, P=128), [700]),
     # the largest pattern count the u8 indices allow: float64 assignment, 16 clusters per warp
     "p255": (W["llama3_8b_32k"].with_(B=1, S=600, Hkv=1, Hq=4, P=255), [300, 300]),
     # V adaptive threshold: every fourth V vector replaced by one far from every pattern (planted
