@@ -170,7 +170,7 @@ __device__ __forceinline__ void fit_rows_eval(const Src& s, int prob, const int6
 // slower, its registers halving the warps per SM).  rin: the previous pass's reciprocal row
 // products (null in pass 0); cinv: 1 / C_p (null in pass 0).
 constexpr int kFitRows = 1;
-__global__ void __launch_bounds__(kFitWarps * 32) fit_pass_kernel(Src s, const double* __restrict__ cinv,
+__global__ void __launch_bounds__(kFitWarps * 32, 4) fit_pass_kernel(Src s, const double* __restrict__ cinv,
                                                                   const double* __restrict__ rin,
                                                                   double* __restrict__ rout,
                                                                   double* __restrict__ colpart) {

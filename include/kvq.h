@@ -89,7 +89,9 @@
  *   - Pre-transform (KVARN): x' = x H (unnormalised Sylvester Walsh-Hadamard, fp32
  *     butterfly with strides 1..64); u = fl32(x'/c); r = population std of u in fp32
  *     (halving sums); y = fl32(u / r) (r = 1 when the std is 0).  c is fitted per
- *     (set, head) on the prefill by 3 alternating row / column std passes.
+ *     (set, head) on the prefill by 3 alternating row / column std passes in float64 (the
+ *     GPU recomputes each row per pass instead of storing it, a few ulps from the sequential
+ *     divisions, and gives the same c on every run).
  *   - Mining: Lloyd k-means, strided initialisation M_j = x[floor(j*n/P)], float64
  *     squared distances (lowest index on ties), centroid = fl32(float64 mean),
  *     empty clusters keep their pattern.
