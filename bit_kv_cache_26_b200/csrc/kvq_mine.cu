@@ -1415,7 +1415,7 @@ __global__ void __launch_bounds__(kFixWarps * 32) mine_fixup_kernel(Src s, int P
       const int j = nc == 255 ? slot + 8 * q : (int)((cw >> (8 * (slot & 3))) & 0xffu);
       const float* m = Mp + (size_t)j * kD;
       double acc = 0.0;
-#pragma unroll 4
+#pragma unroll 8
       for (int d = 0; d < kD; d += 8) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(xrow + d));
         const float4 ma = __ldg(reinterpret_cast<const float4*>(m + d));
@@ -1601,7 +1601,7 @@ cudaError_t launch_mine(const MineArgs& a, void* ws, size_t ws_bytes, cudaStream
       mine_assign_tc_kernel<<<dim3(tc_ctas, NP), kTcThreads, smem_tc, st>>>(
           xmap, s, a.P, a.patterns, w.assign, w.xsq, it == 0, w.amb, w.ambc, w.ambn, w.amb_cnt, mine_tc_stages(a.P),
           w.status);
-      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 2 * sms / NP), NP), kFixWarps * 32, 0, st>>>(
+      mine_fixup_kernel<<<dim3((unsigned)std::max(1, 4 * sms / NP), NP), kFixWarps * 32, 0, st>>>(
           s, a.P, a.patterns, w.amb, w.ambc, w.ambn, w.amb_cnt, w.assign);
     } else if (use_mma && KIND == 0)
       mine_assign_mma_kernel<0><<<ag, kMmaWarps * 32, smem_mma, st>>>(s, a.P, a.patterns, w.assign);
