@@ -1029,7 +1029,9 @@ cudaError_t launch_accum(const CUtensorMap& amap, const Src& s, int P, int NP, i
 //     iteration and from a per-token cache after that.
 // Every mbarrier wait is bounded.
 constexpr int kTcM = 128;
-constexpr int kTcMaxStages = 2;  // two CTAs per SM share the SM's shared memory and TMEM
+// ring depth: two stages for P <= 64 (two CTAs per SM share the SM's shared memory and TMEM),
+// up to five above (one CTA per SM)
+constexpr int kTcMaxStages = 5;
 constexpr int kTcTileBytes = kTcM * kD * 2;
 constexpr uint32_t kTcSpinLimit = 1u << 22;
 constexpr int kTcEpiWarps = 8;
@@ -1444,6 +1446,7 @@ __global__ void __launch_bounds__(kFixWarps * 32) mine_fixup_kernel(Src s, int P
 // ring depth that fits next to the patterns in 227 KB, and the dynamic shared memory it needs
 int mine_tc_stages(int P) {
   const int Pn = (P + 15) & ~15;
+  if (Pn <= 64) return 2;
   const int fixed = 2 * Pn * kD * 2 + Pn * 4 + 16 + (2 * kTcMaxStages + 8) * 8 + 16 + 1024;
   return std::max(2, std::min(kTcMaxStages, (227 * 1024 - fixed) / kTcTileBytes));
 }
