@@ -251,10 +251,11 @@ PER_CONFIG = [("llama3_8b_32k", {"bits": 2}), ("llama3_8b_32k", {"bits": 4}),
 
 def launches_per_step(w) -> int:
     """Kernels this library launches per step: per mining call init + per Lloyd iteration
-    assignment (+ the float64 fix-up after the tcgen05 assignment), cluster sums and update (+16
-    for the pre-transform fit and apply); append: prep, pages, tail; decode: 1."""
+    assignment (+ the float64 fix-up after the tcgen05 assignment), cluster sums and update (+8
+    for the pre-transform: three fit passes with their finish kernels, the factors' output and
+    apply); append: prep, pages, tail; decode: 1."""
     tc = w.dtype == 1 and not w.transform and w.P <= 128
-    mine = 1 + (4 if tc else 3) * w.iters + (16 if w.transform else 0)
+    mine = 1 + (4 if tc else 3) * w.iters + (8 if w.transform else 0)
     return 2 * mine + 3 + 1
 
 
