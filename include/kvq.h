@@ -252,7 +252,10 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new
  *        keys of the K tail, reconstructed values of all tokens.  A sequence with no
  *        tokens gets zeros.
  * Split-K over the token axis; partial results go to the workspace
- * (kvq_decode_workspace_bytes()).
+ * (kvq_decode_workspace_bytes()).  The environment variable KVQ_DECODE_CFG (read per call,
+ * 0..3) selects the kernel's pipeline form, (ring stages per warp, warps per CTA) =
+ * (3, 4), (2, 4), (2, 8), (3, 8); the default 1 measured fastest on one B200.  The forms
+ * merge their per-warp partials in different orders, so outputs agree to rounding.
  */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t num_q_heads);
 KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, int32_t num_q_heads, float sm_scale,
