@@ -576,14 +576,30 @@ __global__ void __launch_bounds__(kAppendThreads, 4) append_pages_kernel(Geom g,
     const float ds2 = __shfl_sync(kFull, ds, src);
     const int s2 = __shfl_sync(kFull, s, src);
     if (row_on(r2)) {
-      const int j1 = hh2 ? Pe : P0;
-#pragma unroll 4
-      for (int j = hh2 ? P0 : 0; j < j1; ++j) {
-        const float lb = __half2float(lbuf[r2 * ldh + j]);
-        if (j == s2 || lb > ds2 || (lb == ds2 && j > s2)) continue;
+      // a pattern is left out only when its bound (fp16, rounded toward zero) exceeds the seed's
+      // distance rounded up to fp16, so its d_mm is above the seed's; ties and near-ties go to
+      // the exact comparison.  Two bounds (one 4-byte word: the row stride is even) per compare.
+      const __half dsh = __float2half_ru(ds2);
+      const __half2 dsh2 = __half2half2(dsh);
+      const __half* lrow = lbuf + r2 * ldh;
+      auto push = [&](int jj) {
+        if (jj == s2) return;
         const int pos = atomicAdd(&qn, 1);
-        if (pos < kQueueCap) queue[pos] = ((uint32_t)r2 << 16) | (uint32_t)j;
+        if (pos < kQueueCap) queue[pos] = ((uint32_t)r2 << 16) | (uint32_t)jj;
+      };
+      int j = hh2 ? P0 : 0;
+      const int j1 = hh2 ? Pe : P0;
+      if ((j & 1) && j < j1) {
+        if (!__hgt(lrow[j], dsh)) push(j);
+        ++j;
       }
+#pragma unroll 4
+      for (; j + 2 <= j1; j += 2) {
+        const unsigned gt = __hgt2_mask(*reinterpret_cast<const __half2*>(lrow + j), dsh2);
+        if (!(gt & 0xFFFFu)) push(j);
+        if (!(gt >> 16)) push(j + 1);
+      }
+      if (j < j1 && !__hgt(lrow[j], dsh)) push(j);
     }
   }
   __syncthreads();
